@@ -1,0 +1,270 @@
+/*
+ * CPU oracle for the sparse MoE layer forward pass — TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, obviously correct C in fp64.  Only the tests, the smoke check
+ * and the benchmark's CPU-baseline leg load this library; the product path
+ * (the CUDA library) shares no code, header or table with it.
+ *
+ * What it computes, step by step, in the order the pages give the layer
+ * ("Expert Parallelism" guide (infra.bea.ai), section 2 "The Dispatch
+ * Pattern"; "Expert Parallelism" glossary (klaylearn.com), third paragraph):
+ *   1. router logits  l[t,e] = sum_i x[t,i] * Wr[i,e] (+ bias[e]); the router
+ *      is a linear scoring layer with one output per expert
+ *        (inferensys.com glossary, gating-network and router-latency entries)
+ *   2. top-k gating: the k experts with the largest logits, ties to the lower
+ *      expert index; gate weights = softmax over the k selected logits
+ *        (inferensys.com glossary, Top-k Gating; klaylearn.com glossary: the
+ *         router also yields the weights that mix the expert outputs)
+ *   3. capacity C = ceil(cf*k*T/E), dropless (C = T) when cf == 0
+ *        (inferensys.com glossary, capacity-factor entry; "Expert Parallelism
+ *         & All-to-All" (neelmishra), section "Why fixed-size buffers matter
+ *         here")
+ *   4. permutation into per-expert buckets: pairs take bucket slots in token
+ *      order; a pair whose slot is >= C overflows a full bucket and is dropped
+ *        (inferensys.com glossary, Dropped Tokens entry)
+ *   5. per-expert SwiGLU MLP: h = silu(x Wg) * (x Wu), o = h Wd
+ *        (neelmishra, section "Tensor parallelism for experts": gate, up and
+ *         down projections)
+ *   6. combine: y[t] = sum over kept pairs of w * o, in the token's top-k
+ *      order; a token whose every pair was dropped leaves the layer as it came
+ *        (neelmishra, section "All-to-all: the distributed transpose": the
+ *         combine undoes the dispatch permutation and sums the k outputs
+ *         scaled by their gate weights; inferensys.com glossary, Dropped
+ *         Tokens entry: a dropped token goes through the layer untouched)
+ *
+ * bf16 tensors are passed as their raw 16-bit patterns (uint16_t) and are
+ * widened exactly to double.  All accumulation is fp64.  Layouts are
+ * row-major: x[T,d], Wr[d,E], Wg/Wu[E,d,f], Wd[E,f,d].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double bf16_bits_to_f64(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Step 3.  cf == 0 selects the dropless layer: an expert can receive each
+ * token at most once, so C = T never drops.  Evaluated as ((cf*k)*T)/E in
+ * fp64, then rounded up. */
+int64_t oracle_capacity(int64_t T, int64_t E, int64_t k, double cf) {
+    if (cf == 0.0) return T;
+    double c = ((cf * (double)k) * (double)T) / (double)E;
+    return (int64_t)ceil(c);
+}
+
+/* Step 1, fp64 accumulation.  bias may be NULL. */
+void oracle_router_logits(const uint16_t* x, const float* w_router, const float* bias,
+                          int64_t T, int64_t d, int64_t E, double* logits) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < d; ++i)
+                acc += bf16_bits_to_f64(x[t * d + i]) * (double)w_router[i * E + e];
+            if (bias) acc += (double)bias[e];
+            logits[t * E + e] = acc;
+        }
+    }
+}
+
+/* Step 2 on fp32 logits (the precision the routing decision is taken in).
+ * Repeated selection of the largest remaining logit; a strict '>' keeps the
+ * lower expert index on ties.  Output order: descending logit.  Weights:
+ * exp(l_j - l_max) / sum over the k selected, in fp64. */
+void oracle_topk(const float* logits, int64_t T, int64_t E, int64_t k,
+                 int32_t* topk_idx, double* topk_w) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const float* l = logits + t * E;
+        unsigned char* taken = (unsigned char*)calloc((size_t)E, 1);
+        for (int64_t j = 0; j < k; ++j) {
+            int64_t best = -1;
+            for (int64_t e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || l[e] > l[best]) best = e;
+            }
+            taken[best] = 1;
+            topk_idx[t * k + j] = (int32_t)best;
+        }
+        free(taken);
+        double lmax = (double)l[topk_idx[t * k]];
+        double sum = 0.0;
+        for (int64_t j = 0; j < k; ++j) {
+            double v = exp((double)l[topk_idx[t * k + j]] - lmax);
+            topk_w[t * k + j] = v;
+            sum += v;
+        }
+        for (int64_t j = 0; j < k; ++j) topk_w[t * k + j] /= sum;
+    }
+}
+
+/* Step 4.  Walk tokens in index order; each (token, expert) pair takes the
+ * next free slot of its expert's bucket; slot >= C means dropped (slot = -1).
+ * counts[e] = pairs kept by e, offsets = exclusive prefix sum of counts
+ * (offsets[E] = N kept pairs), row_src[offsets[e] + slot] = t for kept pairs.
+ * Returns the number of dropped pairs. */
+int64_t oracle_permute(const int32_t* topk_idx, int64_t T, int64_t E, int64_t k, int64_t C,
+                       int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_src) {
+    int64_t* demand = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t j = 0; j < k; ++j) {
+            int64_t e = topk_idx[t * k + j];
+            int64_t s = demand[e]++;
+            slot[t * k + j] = (s < C) ? (int32_t)s : -1;
+        }
+    }
+    int64_t n_drop = 0, run = 0;
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t kept = demand[e] < C ? demand[e] : C;
+        counts[e] = (int32_t)kept;
+        offsets[e] = (int32_t)run;
+        run += kept;
+        n_drop += demand[e] - kept;
+    }
+    offsets[E] = (int32_t)run;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < k; ++j) {
+            int32_t s = slot[t * k + j];
+            if (s >= 0) row_src[offsets[topk_idx[t * k + j]] + s] = (int32_t)t;
+        }
+    free(demand);
+    return n_drop;
+}
+
+/* The gather half of step 4: row r of the permuted buffer is token row_src[r]. */
+void oracle_dispatch(const uint16_t* x, const int32_t* row_src, int64_t N, int64_t d,
+                     uint16_t* x_perm) {
+    for (int64_t r = 0; r < N; ++r)
+        memcpy(x_perm + r * d, x + (int64_t)row_src[r] * d, (size_t)d * sizeof(uint16_t));
+}
+
+/* Step 5 for n rows that all go to one expert whose weights are wg/wu [d,f]
+ * and wd [f,d].  h [n,f] (may be NULL) and o [n,d] in fp64, no intermediate
+ * rounding.  silu(z) = z * sigmoid(z) = z / (1 + exp(-z)). */
+void oracle_swiglu_rows(const uint16_t* x_rows, int64_t n, int64_t d, int64_t f,
+                        const uint16_t* wg, const uint16_t* wu, const uint16_t* wd,
+                        double* h_out, double* o_out) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+        double* g = (double*)calloc((size_t)f, sizeof(double));
+        double* u = (double*)calloc((size_t)f, sizeof(double));
+        const uint16_t* xr = x_rows + r * d;
+        for (int64_t i = 0; i < d; ++i) {
+            double xi = bf16_bits_to_f64(xr[i]);
+            const uint16_t* wgi = wg + i * f;
+            const uint16_t* wui = wu + i * f;
+            for (int64_t j = 0; j < f; ++j) {
+                g[j] += xi * bf16_bits_to_f64(wgi[j]);
+                u[j] += xi * bf16_bits_to_f64(wui[j]);
+            }
+        }
+        double* o = o_out + r * d;
+        for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+        for (int64_t j = 0; j < f; ++j) {
+            double hj = g[j] / (1.0 + exp(-g[j])) * u[j];
+            if (h_out) h_out[r * f + j] = hj;
+            const uint16_t* wdj = wd + j * d;
+            for (int64_t c = 0; c < d; ++c) o[c] += hj * bf16_bits_to_f64(wdj[c]);
+        }
+        free(g);
+        free(u);
+    }
+}
+
+/* Step 5 over every bucket: rows offsets[e] .. offsets[e+1]-1 use expert e. */
+void oracle_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, int64_t E, int64_t d,
+                       int64_t f, const uint16_t* w_gate, const uint16_t* w_up,
+                       const uint16_t* w_down, double* h, double* y_perm) {
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t r0 = offsets[e], n = offsets[e + 1] - offsets[e];
+        if (n == 0) continue;
+        oracle_swiglu_rows(x_perm + r0 * d, n, d, f, w_gate + e * d * f, w_up + e * d * f,
+                           w_down + e * f * d, h ? h + r0 * f : NULL, y_perm + r0 * d);
+    }
+}
+
+/* Step 6.  Sum in the token's top-k order; a token with no kept pair returns
+ * its input row. */
+void oracle_combine(const double* y_perm, const uint16_t* x, const int32_t* topk_idx,
+                    const double* topk_w, const int32_t* slot, const int32_t* offsets,
+                    int64_t T, int64_t d, int64_t k, double* y) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double* yt = y + t * d;
+        int kept = 0;
+        for (int64_t c = 0; c < d; ++c) yt[c] = 0.0;
+        for (int64_t j = 0; j < k; ++j) {
+            int32_t s = slot[t * k + j];
+            if (s < 0) continue;
+            kept = 1;
+            const double* o = y_perm + ((int64_t)offsets[topk_idx[t * k + j]] + s) * d;
+            double w = topk_w[t * k + j];
+            for (int64_t c = 0; c < d; ++c) yt[c] += w * o[c];
+        }
+        if (!kept)
+            for (int64_t c = 0; c < d; ++c) yt[c] = bf16_bits_to_f64(x[t * d + c]);
+    }
+}
+
+/* Steps 1-6 end to end.  decision_logits (fp32 [T,E]) may be given, in which
+ * case the routing decision is taken on those values; when NULL the oracle's
+ * own fp64 logits, rounded to fp32, are used.  Optional outputs (NULL to skip):
+ * logits64 [T,E], topk_idx [T,k], topk_w [T,k], slot [T,k], counts [E],
+ * offsets [E+1].  Returns the number of dropped pairs. */
+int64_t oracle_moe_forward(const uint16_t* x, const float* w_router, const float* bias,
+                           const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
+                           int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf,
+                           const float* decision_logits, double* y, double* logits64_out,
+                           int32_t* topk_idx_out, double* topk_w_out, int32_t* slot_out,
+                           int32_t* counts_out, int32_t* offsets_out) {
+    double* l64 = (double*)malloc((size_t)(T * E) * sizeof(double));
+    float* l32 = (float*)malloc((size_t)(T * E) * sizeof(float));
+    int32_t* idx = (int32_t*)malloc((size_t)(T * k) * sizeof(int32_t));
+    double* w = (double*)malloc((size_t)(T * k) * sizeof(double));
+    int32_t* slot = (int32_t*)malloc((size_t)(T * k) * sizeof(int32_t));
+    int32_t* counts = (int32_t*)malloc((size_t)E * sizeof(int32_t));
+    int32_t* offsets = (int32_t*)malloc((size_t)(E + 1) * sizeof(int32_t));
+    int32_t* row_src = (int32_t*)malloc((size_t)(T * k) * sizeof(int32_t));
+
+    oracle_router_logits(x, w_router, bias, T, d, E, l64);
+    if (decision_logits) {
+        memcpy(l32, decision_logits, (size_t)(T * E) * sizeof(float));
+    } else {
+        for (int64_t i = 0; i < T * E; ++i) l32[i] = (float)l64[i];
+    }
+    oracle_topk(l32, T, E, k, idx, w);
+    int64_t C = oracle_capacity(T, E, k, cf);
+    int64_t n_drop = oracle_permute(idx, T, E, k, C, counts, offsets, slot, row_src);
+    int64_t N = offsets[E];
+    uint16_t* x_perm = (uint16_t*)malloc((size_t)(N * d + 1) * sizeof(uint16_t));
+    double* y_perm = (double*)malloc((size_t)(N * d + 1) * sizeof(double));
+    oracle_dispatch(x, row_src, N, d, x_perm);
+    oracle_expert_mlp(x_perm, offsets, E, d, f, w_gate, w_up, w_down, NULL, y_perm);
+    oracle_combine(y_perm, x, idx, w, slot, offsets, T, d, k, y);
+
+    if (logits64_out) memcpy(logits64_out, l64, (size_t)(T * E) * sizeof(double));
+    if (topk_idx_out) memcpy(topk_idx_out, idx, (size_t)(T * k) * sizeof(int32_t));
+    if (topk_w_out) memcpy(topk_w_out, w, (size_t)(T * k) * sizeof(double));
+    if (slot_out) memcpy(slot_out, slot, (size_t)(T * k) * sizeof(int32_t));
+    if (counts_out) memcpy(counts_out, counts, (size_t)E * sizeof(int32_t));
+    if (offsets_out) memcpy(offsets_out, offsets, (size_t)(E + 1) * sizeof(int32_t));
+    free(l64); free(l32); free(idx); free(w); free(slot); free(counts); free(offsets);
+    free(row_src); free(x_perm); free(y_perm);
+    return n_drop;
+}

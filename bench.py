@@ -1,0 +1,420 @@
+"""Benchmark of the MoE layer forward pass on B200: tokens/s of the whole layer,
+with the dominant kernel's roofline fraction and the CPU oracle beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one pass of the whole layer (router + top-k, permute, grouped
+gate/up GEMM with SwiGLU, grouped down GEMM, combine) over one batch of T
+seeded synthetic tokens, inputs and weights resident in HBM.  Multi-GPU runs
+(torchrun, one process per GPU) are independent replicas: every rank runs the
+same layer on its own token batch; there is no data-path collective, only a
+barrier around the timed region and a max-over-ranks of the device time.
+
+Prints one JSON line on rank 0.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
+
+METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 7     # router 1, permute 3, gate/up GEMM 1, down GEMM 1, combine 1
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return json.load(fh), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def describe(cfg):
+    cf = "dropless" if cfg.cf == 0 else f"cf={cfg.cf}"
+    extra = f", zipf bias s={cfg.zipf_s}" if cfg.zipf_s else ""
+    return (f"{cfg.name}: T={cfg.T} d={cfg.d} E={cfg.E} k={cfg.k} SwiGLU f={cfg.f} {cf}{extra}, "
+            f"seed {cfg.seed}")
+
+
+# ----------------------------------------------------------------- clocks sampling
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        props = torch.cuda.get_device_properties(device)
+        uuid = str(getattr(props, "uuid", "") or "")
+        self.gpu = ("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or "0")
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r)
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- the GPU arm
+
+class Layer:
+    """Inputs, weights and buffers of one workload, resident on the device,
+    and the step as five C-ABI calls on one stream."""
+
+    def __init__(self, cfg, device, token_seed):
+        import mixture_experts_layer_36_b200 as moe
+        self.moe = moe
+        self.cfg = cfg
+        self.dev = device
+        w = synth.make_weights(cfg, device)
+        self.w = w
+        self.x = synth.make_tokens(cfg, device, seed=token_seed)
+        T, d, E, k, f = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f
+        self.rows = moe.moe_max_rows(T, E, k, cfg.cf)
+        z = lambda *s, dt: torch.empty(*s, dtype=dt, device=device)  # noqa: E731
+        self.logits = z(T, E, dt=torch.float32)
+        self.idx = z(T, k, dt=torch.int32)
+        self.tw = z(T, k, dt=torch.float32)
+        self.perm = {"counts": z(E, dt=torch.int32), "offsets": z(E + 1, dt=torch.int32),
+                     "slot": z(T, k, dt=torch.int32), "row_src": z(self.rows, dt=torch.int32),
+                     "x_perm": z(self.rows, d, dt=torch.bfloat16),
+                     "n_dropped": z(1, dt=torch.int32)}
+        self.pws = z(max(moe.moe_permute_workspace_size(T, E, k), 16), dt=torch.uint8)
+        self.h = z(self.rows, f, dt=torch.bfloat16)
+        self.y_perm = z(self.rows, d, dt=torch.bfloat16)
+        self.y = z(T, d, dt=torch.bfloat16)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ws = z(moe.moe_workspace_size(T, d, E, k, f, cfg.cf), dt=torch.uint8)
+
+    def step(self, ev=None):
+        """One layer pass; ev = list of 6 events recorded between the stages."""
+        m, w, c = self.moe, self.w, self.cfg
+        if ev:
+            ev[0].record()
+        m.moe_route(self.x, w["w_router"], w["bias"], c.k, self.logits, self.idx, self.tw)
+        if ev:
+            ev[1].record()
+        m.moe_permute(self.x, self.idx, c.E, c.cf, out=self.perm, ws=self.pws)
+        if ev:
+            ev[2].record()
+        m.moe_expert_gate_up(self.perm["x_perm"], self.perm["offsets"], w["w_gate"], w["w_up"],
+                             h=self.h, dev_status=self.status)
+        if ev:
+            ev[3].record()
+        m.moe_expert_down(self.h, self.perm["offsets"], w["w_down"], y_perm=self.y_perm,
+                          dev_status=self.status)
+        if ev:
+            ev[4].record()
+        m.moe_combine(self.y_perm, self.x, self.idx, self.tw, self.perm["slot"],
+                      self.perm["offsets"], y=self.y)
+        if ev:
+            ev[5].record()
+
+    def layer_forward(self, x, y):
+        w, c = self.w, self.cfg
+        self.moe.moe_layer_forward(x, w["w_router"], w["bias"], w["w_gate"], w["w_up"],
+                                   w["w_down"], c.k, c.cf, y=y, ws=self.ws)
+
+
+def gpu_arm(args, cfg, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = world > 1
+    if dist:
+        import torch.distributed as td
+    layer = Layer(cfg, dev, token_seed=cfg.seed * 1000 + rank)
+    stream = torch.cuda.current_stream()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the clock sampler starts before the warm-up so that it is running
+    # (nvidia-smi takes a moment to start) when the timed region begins
+    with ClockSampler(dev) as clk:
+        for _ in range(args.warmup):
+            layer.step()
+        torch.cuda.synchronize()
+        if dist:
+            td.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(K):
+            layer.step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        td.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if dist:
+        td.all_reduce(t, op=td.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+
+    names = ["route", "permute", "gate_up", "down", "combine"]
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+                for j, n in enumerate(names)}
+    status = int(layer.status.item())
+    N = int(layer.perm["offsets"][cfg.E].item())
+    n_drop = int(layer.perm["n_dropped"].item())
+
+    # end to end through the one-shot public call, host buffers in and out
+    x_host = layer.x.cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(layer.x)
+    y_dev = torch.empty_like(layer.x)
+    for _ in range(max(1, args.warmup)):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.layer_forward(x_dev, y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        td.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.layer_forward(x_dev, y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if dist:
+        td.all_reduce(t, op=td.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+    return {"elapsed_ms": elapsed_ms, "stage_ms": stage_ms, "status": status, "N": N,
+            "n_dropped": n_drop, "clocks": clk.summary(), "e2e_ms": e2e_ms,
+            "h2d": x_host.numel() * 2, "d2h": y_host.numel() * 2, "layer": layer}
+
+
+def traffic_from_profile(kernel_tag, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        prof = json.load(fh)
+    src = os.path.join(ROOT, prof.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return prof.get("dram_bytes_per_launch") if h == prof.get("source_sha256") else None
+
+
+# ----------------------------------------------------------------- the CPU oracle
+
+def oracle_sample(cfg, weights_host, x_host_bits, n_tokens):
+    """Time the oracle (as it stands) on the first n_tokens tokens of the batch,
+    whole layer (capacity recomputed for the sample size).  Returns seconds."""
+    import numpy as np
+    import oracle
+    bias = None if weights_host["bias"] is None else weights_host["bias"]
+    t0 = time.perf_counter()
+    oracle.moe_forward(x_host_bits[:n_tokens], weights_host["w_router"], bias,
+                       weights_host["w_gate"], weights_host["w_up"], weights_host["w_down"],
+                       cfg.k, cfg.cf)
+    return time.perf_counter() - t0, oracle.num_threads()
+
+
+def host_weights(w):
+    import oracle
+    return {"w_router": w["w_router"].cpu().numpy(),
+            "bias": None if w["bias"] is None else w["bias"].cpu().numpy(),
+            "w_gate": oracle.bf16_bits(w["w_gate"]), "w_up": oracle.bf16_bits(w["w_up"]),
+            "w_down": oracle.bf16_bits(w["w_down"])}
+
+
+def sample_tokens(cfg):
+    """Tokens per oracle sample: about 10-30 s of CPU work on a few cores."""
+    per_token_flop = 6.0 * cfg.k * cfg.d * cfg.f + 2.0 * cfg.d * cfg.E
+    return int(max(2, min(cfg.T, round(2.0e10 / per_token_flop))))
+
+
+# ----------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="mixtral")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    cfg = configs.by_name(args.config)
+
+    if args.impl == "reference":
+        return reference_arm(args, cfg, rank, world)
+
+    if world > 1:
+        import datetime
+        import torch.distributed as td
+        torch.cuda.set_device(local_rank)
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                              device_id=torch.device("cuda", local_rank))
+    r = gpu_arm(args, cfg, rank, world, local_rank)
+    pk, pk_kind = peaks()
+    K = args.steps
+    tokens = cfg.T * world * K
+    value = tokens / (r["elapsed_ms"] / 1e3)
+    gemm1_flop = 4.0 * r["N"] * cfg.d * cfg.f
+    gemm2_flop = 2.0 * r["N"] * cfg.d * cfg.f
+    t_g1 = r["stage_ms"]["gate_up"] / 1e3
+    t_g2 = r["stage_ms"]["down"] / 1e3
+    peak_tf = pk["bf16_tflops"]
+    achieved = gemm1_flop / t_g1 / 1e12
+    bytes_perm = cfg.T * cfg.d * 2 + r["N"] * cfg.d * 2
+    bytes_comb = r["N"] * cfg.d * 2 + cfg.T * cfg.d * 2
+    out = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(r["elapsed_ms"] / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights of the named shape)",
+        "config": {"workload": describe(cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "f": cfg.f, "cf": cfg.cf, "kept_pairs": r["N"], "dropped_pairs": r["n_dropped"],
+                   "parallelism": f"replicas x{world} (token batches, no collective)",
+                   "l2": "inputs larger than L2 (expert weights "
+                         f"{3 * cfg.E * cfg.d * cfg.f * 2 / 1e9:.1f} GB); no flush"},
+        "roofline": {"kernel": "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)",
+                     "bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                     "peak_source": f"{pk_kind} bf16 burst",
+                     "traffic": traffic_from_profile("gemm_gate_up", cfg.name)},
+        "stages_ms": {k_: round(v, 4) for k_, v in r["stage_ms"].items()},
+        "stage_rooflines": {
+            "down_gemm": {"bound": "tensor", "achieved": round(gemm2_flop / t_g2 / 1e12, 1),
+                          "unit": "TFLOP/s", "frac": round(gemm2_flop / t_g2 / 1e12 / peak_tf, 4)},
+            "permute": {"bound": "hbm", "unit": "GB/s",
+                        "achieved": round(bytes_perm / (r["stage_ms"]["permute"] / 1e3) / 1e9, 1),
+                        "frac": round(bytes_perm / (r["stage_ms"]["permute"] / 1e3) / 1e9
+                                      / pk["hbm_gbs"], 4)},
+            "combine": {"bound": "hbm", "unit": "GB/s",
+                        "achieved": round(bytes_comb / (r["stage_ms"]["combine"] / 1e3) / 1e9, 1),
+                        "frac": round(bytes_comb / (r["stage_ms"]["combine"] / 1e3) / 1e9
+                                      / pk["hbm_gbs"], 4)},
+        },
+        "device_status": r["status"],
+        "clocks": {k_: r["clocks"][k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "e2e": {"value": round(cfg.T * world * K / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "api": "moe_layer_forward (one-shot C-ABI call), pinned host x in, y out"},
+        "gpu_launches": KERNELS_PER_STEP * K,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = sample_tokens(cfg)
+        wh = host_weights(r["layer"].w)
+        import oracle
+        secs, cores = oracle_sample(cfg, wh, oracle.bf16_bits(r["layer"].x), n)
+        out["cpu_baseline"] = {"value": round(n / secs, 3), "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle",
+                               "sample": f"first {n} tokens of the batch through the whole "
+                                         f"layer (fp64 C oracle, OpenMP), {secs:.1f} s"}
+    if world > 1:
+        import torch.distributed as td
+        td.barrier()
+        td.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def reference_arm(args, cfg, rank, world):
+    """The oracle timed as it stands on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    n = max(2, sample_tokens(cfg) // 8)
+    # weights drawn on the CPU with the same recipe (one step is a bounded sample)
+    w = synth.make_weights(cfg, "cpu")
+    x = synth.make_tokens(cfg, "cpu")
+    wh = host_weights(w)
+    xb = oracle.bf16_bits(x)
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(cfg, wh, xb, n)
+    t = 0.0
+    for _ in range(args.steps):
+        s, cores = oracle_sample(cfg, wh, xb, n)
+        t += s
+    value = n * args.steps / t
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; random-init weights of the named shape)",
+        "config": {"workload": describe(cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "f": cfg.f, "cf": cfg.cf},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"each step: first {n} tokens of the batch through the whole "
+                                   f"layer (fp64 C oracle, OpenMP)"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+/*
+ * libmoe — forward pass of a sparse Mixture-of-Experts layer on one B200
+ * (sm_100a).  C ABI: plain pointers and sizes, no framework types.
+ *
+ * The layer (the local part of the expert-parallel pipeline that all the
+ * source pages describe: "Expert Parallelism" guide (infra.bea.ai), section 2
+ * "The Dispatch Pattern"; "Expert Parallelism" glossary (klaylearn.com), third
+ * paragraph):
+ *   route    l = x Wr (+ bias); top-k experts per token; gate weights =
+ *            softmax renormalised over the k selected logits
+ *   permute  pairs (token, expert) into per-expert buckets of capacity
+ *            C = ceil(cf*k*T/E) (dropless when cf == 0), slots in token order,
+ *            overflow dropped
+ *   experts  per expert e: h = silu(x_perm Wg[e]) * (x_perm Wu[e]),
+ *            y_perm = h Wd[e]  (SwiGLU)
+ *   combine  y[t] = sum over kept pairs j of w[t,j] * y_perm[row(t,j)], in
+ *            top-k order; a token whose k pairs were all dropped gets x[t]
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *     library never allocates or frees device memory and keeps no state
+ *     beyond a per-device cache of attributes.  Outputs must not alias inputs.
+ *   - Tensors are dense row-major.  bf16 = IEEE bfloat16 (__nv_bfloat16),
+ *     passed as void*.  Base pointers must be 16-byte aligned.
+ *   - Work is enqueued asynchronously on `stream` (cudaStream_t passed as
+ *     void*; NULL = legacy default stream).  No entry point synchronises.
+ *   - Return codes report host-side validation and launch errors only.  A
+ *     kernel that detects a problem on the device (a bounded wait that gave
+ *     up, inconsistent bucket offsets) ORs a bit into the caller's int32
+ *     device status word `dev_status` (nullable: then nothing is reported);
+ *     read it after synchronising.  Bits: 1 = wait timeout, 2 = bad offsets.
+ *   - Limits: 1 <= E <= 256, 1 <= k <= min(E, 8), T*k < 2^31, d and f
+ *     multiples of 128 (else MOE_ERR_UNSUPPORTED).  T == 0 is a no-op.
+ */
+#ifndef LIBMOE_MOE_H_
+#define LIBMOE_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer  */
+  MOE_ERR_WORKSPACE = 2,     /* workspace smaller than the size query says  */
+  MOE_ERR_CUDA = 3,          /* a CUDA runtime / driver call failed          */
+  MOE_ERR_UNSUPPORTED = 4,   /* shape outside the kernels' tiling limits     */
+  MOE_ERR_DEVICE_CHECK = 5   /* reserved: device status word was non-zero    */
+} moe_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+int moe_version(void);
+
+/* Expert capacity, step "capacity" above: ceil(((cf*k)*T)/E) evaluated in
+ * fp64; cf == 0 selects the dropless layer and returns T.  Source: the
+ * capacity-factor entry of the inferensys.com glossary and section "Why
+ * fixed-size buffers matter here" of "Expert Parallelism & All-to-All"
+ * (neelmishra.github.io); the infra.bea.ai guide's section 4 states the same
+ * rule without k, read here as the k = 1 case.  Returns -1 on bad args. */
+int64_t moe_capacity(int64_t T, int64_t E, int64_t k, double cf);
+
+/* Rows of the permuted buffers: min(T*k, E*C), the most pairs that can be
+ * kept.  Returns -1 on bad args. */
+int64_t moe_max_rows(int64_t T, int64_t E, int64_t k, double cf);
+
+/* Device scratch bytes moe_permute needs (per-chunk bucket histograms). */
+size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k);
+
+/* Device workspace bytes moe_layer_forward needs: every intermediate
+ * (status word, logits, routing, slots, buckets, x_perm, h, y_perm). */
+size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf);
+
+/* Fields of the moe_layer_forward workspace, for callers that want to read
+ * an intermediate after the call. */
+typedef enum {
+  MOE_WS_STATUS = 0,     /* int32[1]  device status word (zeroed by the call) */
+  MOE_WS_LOGITS = 1,     /* f32 [T,E] */
+  MOE_WS_TOPK_IDX = 2,   /* i32 [T,k] */
+  MOE_WS_TOPK_W = 3,     /* f32 [T,k] */
+  MOE_WS_SLOT = 4,       /* i32 [T,k] */
+  MOE_WS_COUNTS = 5,     /* i32 [E]   */
+  MOE_WS_OFFSETS = 6,    /* i32 [E+1] */
+  MOE_WS_N_DROPPED = 7,  /* i32 [1]   */
+  MOE_WS_ROW_SRC = 8,    /* i32 [max_rows] */
+  MOE_WS_PERMUTE = 9,    /* moe_permute scratch */
+  MOE_WS_X_PERM = 10,    /* bf16 [max_rows, d] */
+  MOE_WS_H = 11,         /* bf16 [max_rows, f] */
+  MOE_WS_Y_PERM = 12,    /* bf16 [max_rows, d] */
+  MOE_WS_NUM_FIELDS = 13
+} moe_ws_field;
+
+/* Byte offset of a field inside the moe_layer_forward workspace (each field
+ * 256-byte aligned); -1 on bad args. */
+int64_t moe_workspace_field_offset(int field, int64_t T, int64_t d, int64_t E, int64_t k,
+                                   int64_t f, double cf);
+
+/* Router and top-k gating.  The router is a linear layer giving one score per
+ * expert (inferensys.com glossary, gating-network and router-latency entries);
+ * top-k gating keeps the k highest (same glossary, Top-k Gating); the router
+ * also supplies the weights that mix the chosen experts' outputs
+ * (klaylearn.com glossary, third paragraph).
+ *   x        bf16 [T,d]     tokens
+ *   w_router f32  [d,E]     router weight
+ *   bias     f32  [E]       nullable; added to every token's logits
+ *   logits   f32  [T,E]     out: sum_i x[t,i]*w_router[i,e] + bias[e], fp32
+ *   topk_idx i32  [T,k]     out: the k largest logits, descending; equal
+ *                           logits rank the lower expert index first
+ *   topk_w   f32  [T,k]     out: exp(l_j - l_max) / sum over the k selected
+ * The selection is taken on the fp32 values written to `logits`. */
+int moe_route(const void* x, const float* w_router, const float* bias, int64_t T, int64_t d,
+              int64_t E, int64_t k, float* logits, int32_t* topk_idx, float* topk_w,
+              void* stream);
+
+/* Capacity-limited permutation into per-expert buckets (pairs are bucketed by
+ * expert, overflow beyond the capacity is dropped: inferensys.com glossary,
+ * Expert Capacity and Dropped Tokens entries; the tokens are permuted before
+ * the experts run: klaylearn.com glossary, third paragraph).
+ *   x         bf16 [T,d]        tokens
+ *   topk_idx  i32  [T,k]        experts per token (distinct within a token)
+ *   cf                          capacity factor, C = moe_capacity(T,E,k,cf)
+ *   counts    i32  [E]          out: pairs kept by each expert (<= C)
+ *   offsets   i32  [E+1]        out: exclusive prefix sum of counts
+ *   slot      i32  [T,k]        out: bucket slot of pair (t,j) = number of
+ *                               tokens t' < t that chose the same expert;
+ *                               -1 when that slot is >= C (dropped)
+ *   row_src   i32  [max_rows]   out: token of permuted row r (rows < offsets[E])
+ *   x_perm    bf16 [max_rows,d] out: row offsets[e]+slot holds x[t]
+ *   n_dropped i32  [1]          out: number of dropped pairs
+ *   ws, ws_bytes                device scratch, >= moe_permute_workspace_size
+ * Rows at and beyond offsets[E] of row_src / x_perm are left untouched. */
+int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
+                int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
+                int32_t* row_src, void* x_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
+                void* stream);
+
+/* Grouped expert GEMM 1 with the SwiGLU fused into its epilogue: for every
+ * expert e and every row r of its bucket (offsets[e] <= r < offsets[e+1]),
+ *   h[r,:] = silu(x_perm[r,:] Wg[e]) * (x_perm[r,:] Wu[e]),  silu(z) = z*sigmoid(z)
+ * (experts are gate/up/down MLPs: neelmishra.github.io, section "Tensor
+ * parallelism for experts"; grouped GEMMs over the buckets: klaylearn.com
+ * glossary, fourth paragraph).  bf16 operands, fp32 accumulation, bf16 h.
+ *   x_perm bf16 [max_rows,d], offsets i32 [E+1] (device), w_gate / w_up bf16
+ *   [E,d,f], h bf16 [max_rows,f] out (rows of no bucket are left untouched). */
+int moe_expert_gate_up(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d,
+                       int64_t f, int64_t max_rows, const void* w_gate, const void* w_up,
+                       void* h, int32_t* dev_status, void* stream);
+
+/* Grouped expert GEMM 2 (down projection): y_perm[r,:] = h[r,:] Wd[e] for the
+ * rows of bucket e.  h bf16 [max_rows,f], w_down bf16 [E,f,d], y_perm bf16
+ * [max_rows,d] out.  Same source passages as moe_expert_gate_up. */
+int moe_expert_down(const void* h, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
+                    int64_t max_rows, const void* w_down, void* y_perm, int32_t* dev_status,
+                    void* stream);
+
+/* Both expert GEMMs: moe_expert_gate_up then moe_expert_down, with h as the
+ * caller's buffer in between. */
+int moe_expert_mlp(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
+                   int64_t max_rows, const void* w_gate, const void* w_up, const void* w_down,
+                   void* h, void* y_perm, int32_t* dev_status, void* stream);
+
+/* Inverse permutation and gate-weighted sum (the combine undoes the dispatch
+ * permutation and adds each token's k expert outputs scaled by their gate
+ * weights: neelmishra.github.io, section "All-to-all: the distributed
+ * transpose"; the weighted sum closes the infra.bea.ai guide's section 2
+ * diagram; a dropped token goes through the layer untouched: inferensys.com
+ * glossary, Dropped Tokens entry).
+ *   y[t,:] = sum_{j: slot[t,j] >= 0} topk_w[t,j] * y_perm[offsets[topk_idx[t,j]] + slot[t,j], :]
+ * summed in fp32 in j order and rounded once to bf16; if no pair of t was
+ * kept, y[t,:] = x[t,:] exactly.  y bf16 [T,d] out. */
+int moe_combine(const void* y_perm, const void* x, const int32_t* topk_idx, const float* topk_w,
+                const int32_t* slot, const int32_t* offsets, int64_t T, int64_t d, int64_t k,
+                void* y, void* stream);
+
+/* The whole layer: moe_route, moe_permute, moe_expert_mlp, moe_combine on
+ * one stream, every intermediate in `ws` (>= moe_workspace_size bytes; field
+ * layout from moe_workspace_field_offset).  No host synchronisation: bucket
+ * sizes stay on the device.  y bf16 [T,d] out. */
+int moe_layer_forward(const void* x, const float* w_router, const float* bias, const void* w_gate,
+                      const void* w_up, const void* w_down, int64_t T, int64_t d, int64_t E,
+                      int64_t k, int64_t f, double cf, void* y, void* ws, size_t ws_bytes,
+                      void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBMOE_MOE_H_ */

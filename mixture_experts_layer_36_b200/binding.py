@@ -1,0 +1,298 @@
+"""Python binding of libmoe (sparse MoE layer forward on one B200).
+
+Thin ctypes marshalling over the C ABI declared in ``include/moe.h``: the
+functions below carry the same names, check dtypes / devices / shapes, pass
+raw device pointers and torch's current CUDA stream, and raise on any non-OK
+status.  Every step of the layer runs in the library's CUDA kernels; nothing
+here computes.  If ``libmoe.so`` is missing the import fails loudly — there is
+no fallback path.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_WORKSPACE", 3: "MOE_ERR_CUDA",
+                4: "MOE_ERR_UNSUPPORTED", 5: "MOE_ERR_DEVICE_CHECK"}
+DEV_ERR_WAIT_TIMEOUT = 1
+DEV_ERR_BAD_OFFSETS = 2
+
+# workspace fields of moe_layer_forward (enum moe_ws_field)
+WS_FIELDS = ["status", "logits", "topk_idx", "topk_w", "slot", "counts", "offsets", "n_dropped",
+             "row_src", "permute", "x_perm", "h", "y_perm"]
+
+EXPORTED = ["moe_status_string", "moe_version", "moe_capacity", "moe_max_rows",
+            "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
+            "moe_route", "moe_permute", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
+            "moe_combine", "moe_layer_forward"]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmoe.so not built at {LIB_PATH}; run "
+                          "`python -m mixture_experts_layer_36_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, dbl, p, sz = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p, ctypes.c_size_t
+    sig = {
+        "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "moe_version": (ctypes.c_int, []),
+        "moe_capacity": (i64, [i64, i64, i64, dbl]),
+        "moe_max_rows": (i64, [i64, i64, i64, dbl]),
+        "moe_permute_workspace_size": (sz, [i64, i64, i64]),
+        "moe_workspace_size": (sz, [i64, i64, i64, i64, i64, dbl]),
+        "moe_workspace_field_offset": (i64, [ctypes.c_int, i64, i64, i64, i64, i64, dbl]),
+        "moe_route": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p]),
+        "moe_permute": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p, sz, p]),
+        "moe_expert_gate_up": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p]),
+        "moe_expert_down": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p]),
+        "moe_expert_mlp": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p, p, p]),
+        "moe_combine": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, p, p]),
+        "moe_layer_forward": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl, p, p,
+                                             sz, p]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(name, st):
+    if st != MOE_OK:
+        raise MoEError(name, st)
+
+
+def _want(t, name, dtype, shape=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+# ----------------------------------------------------------------- size queries
+
+def moe_capacity(T, E, k, cf):
+    return int(_lib.moe_capacity(T, E, k, float(cf)))
+
+
+def moe_max_rows(T, E, k, cf):
+    return int(_lib.moe_max_rows(T, E, k, float(cf)))
+
+
+def moe_permute_workspace_size(T, E, k):
+    return int(_lib.moe_permute_workspace_size(T, E, k))
+
+
+def moe_workspace_size(T, d, E, k, f, cf):
+    return int(_lib.moe_workspace_size(T, d, E, k, f, float(cf)))
+
+
+def moe_workspace_field_offset(field, T, d, E, k, f, cf):
+    if isinstance(field, str):
+        field = WS_FIELDS.index(field)
+    return int(_lib.moe_workspace_field_offset(field, T, d, E, k, f, float(cf)))
+
+
+def moe_version():
+    return int(_lib.moe_version())
+
+
+def moe_status_string(status):
+    return _lib.moe_status_string(status).decode()
+
+
+# ----------------------------------------------------------------- stages
+
+def moe_route(x, w_router, bias, k, logits=None, topk_idx=None, topk_w=None, stream=None):
+    """Router + top-k gating.  Returns (logits f32 [T,E], topk_idx i32 [T,k], topk_w f32 [T,k])."""
+    T, d = x.shape
+    E = w_router.shape[1]
+    _want(x, "x", torch.bfloat16)
+    _want(w_router, "w_router", torch.float32, (d, E))
+    if bias is not None:
+        _want(bias, "bias", torch.float32, (E,))
+    dev = x.device
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev) if logits is None else logits
+    topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev) if topk_idx is None else topk_idx
+    topk_w = torch.empty(T, k, dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    _want(logits, "logits", torch.float32, (T, E))
+    _want(topk_idx, "topk_idx", torch.int32, (T, k))
+    _want(topk_w, "topk_w", torch.float32, (T, k))
+    _check("moe_route", _lib.moe_route(_ptr(x), _ptr(w_router), _ptr(bias), T, d, E, k,
+                                       _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
+                                       _stream(stream)))
+    return logits, topk_idx, topk_w
+
+
+def moe_permute(x, topk_idx, E, cf, out=None, ws=None, stream=None):
+    """Capacity-limited permutation.  Returns a dict with counts, offsets, slot,
+    row_src, x_perm (max_rows rows; rows >= offsets[E] untouched), n_dropped."""
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    _want(x, "x", torch.bfloat16)
+    _want(topk_idx, "topk_idx", torch.int32, (T, k))
+    rows = moe_max_rows(T, E, k, cf)
+    dev = x.device
+    if out is None:
+        out = {
+            "counts": torch.empty(E, dtype=torch.int32, device=dev),
+            "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+            "slot": torch.empty(T, k, dtype=torch.int32, device=dev),
+            "row_src": torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+            "x_perm": torch.empty(max(rows, 1), d, dtype=torch.bfloat16, device=dev),
+            "n_dropped": torch.empty(1, dtype=torch.int32, device=dev),
+        }
+    nbytes = moe_permute_workspace_size(T, E, k)
+    if ws is None:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    _want(ws, "ws", torch.uint8)
+    _check("moe_permute", _lib.moe_permute(
+        _ptr(x), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]),
+        _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["x_perm"]),
+        _ptr(out["n_dropped"]), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def moe_expert_gate_up(x_perm, offsets, w_gate, w_up, h=None, dev_status=None, stream=None):
+    rows, d = x_perm.shape
+    E, _, f = w_gate.shape
+    _want(x_perm, "x_perm", torch.bfloat16)
+    _want(offsets, "offsets", torch.int32, (E + 1,))
+    _want(w_gate, "w_gate", torch.bfloat16, (E, d, f))
+    _want(w_up, "w_up", torch.bfloat16, (E, d, f))
+    h = torch.empty(rows, f, dtype=torch.bfloat16, device=x_perm.device) if h is None else h
+    _want(h, "h", torch.bfloat16, (rows, f))
+    _check("moe_expert_gate_up", _lib.moe_expert_gate_up(
+        _ptr(x_perm), _ptr(offsets), E, d, f, rows, _ptr(w_gate), _ptr(w_up), _ptr(h),
+        _ptr(dev_status), _stream(stream)))
+    return h
+
+
+def moe_expert_down(h, offsets, w_down, y_perm=None, dev_status=None, stream=None):
+    rows, f = h.shape
+    E, _, d = w_down.shape
+    _want(h, "h", torch.bfloat16)
+    _want(offsets, "offsets", torch.int32, (E + 1,))
+    _want(w_down, "w_down", torch.bfloat16, (E, f, d))
+    y_perm = torch.empty(rows, d, dtype=torch.bfloat16, device=h.device) if y_perm is None \
+        else y_perm
+    _want(y_perm, "y_perm", torch.bfloat16, (rows, d))
+    _check("moe_expert_down", _lib.moe_expert_down(
+        _ptr(h), _ptr(offsets), E, d, f, rows, _ptr(w_down), _ptr(y_perm), _ptr(dev_status),
+        _stream(stream)))
+    return y_perm
+
+
+def moe_expert_mlp(x_perm, offsets, w_gate, w_up, w_down, h=None, y_perm=None, dev_status=None,
+                   stream=None):
+    rows, d = x_perm.shape
+    E, _, f = w_gate.shape
+    _want(x_perm, "x_perm", torch.bfloat16)
+    _want(offsets, "offsets", torch.int32, (E + 1,))
+    _want(w_gate, "w_gate", torch.bfloat16, (E, d, f))
+    _want(w_up, "w_up", torch.bfloat16, (E, d, f))
+    _want(w_down, "w_down", torch.bfloat16, (E, f, d))
+    dev = x_perm.device
+    h = torch.empty(rows, f, dtype=torch.bfloat16, device=dev) if h is None else h
+    y_perm = torch.empty(rows, d, dtype=torch.bfloat16, device=dev) if y_perm is None else y_perm
+    _want(h, "h", torch.bfloat16, (rows, f))
+    _want(y_perm, "y_perm", torch.bfloat16, (rows, d))
+    _check("moe_expert_mlp", _lib.moe_expert_mlp(
+        _ptr(x_perm), _ptr(offsets), E, d, f, rows, _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(h), _ptr(y_perm), _ptr(dev_status), _stream(stream)))
+    return h, y_perm
+
+
+def moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, y=None, stream=None):
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    _want(y_perm, "y_perm", torch.bfloat16)
+    _want(x, "x", torch.bfloat16)
+    _want(topk_idx, "topk_idx", torch.int32, (T, k))
+    _want(topk_w, "topk_w", torch.float32, (T, k))
+    _want(slot, "slot", torch.int32, (T, k))
+    _want(offsets, "offsets", torch.int32)
+    y = torch.empty_like(x) if y is None else y
+    _want(y, "y", torch.bfloat16, (T, d))
+    _check("moe_combine", _lib.moe_combine(
+        _ptr(y_perm), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(slot), _ptr(offsets), T, d, k,
+        _ptr(y), _stream(stream)))
+    return y
+
+
+def moe_layer_forward(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws=None,
+                      stream=None):
+    """The whole layer in one call.  Returns (y bf16 [T,d], ws uint8 workspace)."""
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    _want(x, "x", torch.bfloat16)
+    _want(w_router, "w_router", torch.float32, (d, E))
+    if bias is not None:
+        _want(bias, "bias", torch.float32, (E,))
+    _want(w_gate, "w_gate", torch.bfloat16, (E, d, f))
+    _want(w_up, "w_up", torch.bfloat16, (E, d, f))
+    _want(w_down, "w_down", torch.bfloat16, (E, f, d))
+    nbytes = moe_workspace_size(T, d, E, k, f, cf)
+    if ws is None:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _want(ws, "ws", torch.uint8)
+    y = torch.empty_like(x) if y is None else y
+    _want(y, "y", torch.bfloat16, (T, d))
+    _check("moe_layer_forward", _lib.moe_layer_forward(
+        _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k,
+        f, float(cf), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+    return y, ws
+
+
+def workspace_view(ws, field, T, d, E, k, f, cf):
+    """A typed view of one intermediate inside a moe_layer_forward workspace."""
+    rows = moe_max_rows(T, E, k, cf)
+    spec = {
+        "status": (torch.int32, (1,)), "logits": (torch.float32, (T, E)),
+        "topk_idx": (torch.int32, (T, k)), "topk_w": (torch.float32, (T, k)),
+        "slot": (torch.int32, (T, k)), "counts": (torch.int32, (E,)),
+        "offsets": (torch.int32, (E + 1,)), "n_dropped": (torch.int32, (1,)),
+        "row_src": (torch.int32, (rows,)), "x_perm": (torch.bfloat16, (rows, d)),
+        "h": (torch.bfloat16, (rows, f)), "y_perm": (torch.bfloat16, (rows, d)),
+    }[field]
+    dtype, shape = spec
+    off = moe_workspace_field_offset(field, T, d, E, k, f, cf)
+    n = 1
+    for s in shape:
+        n *= s
+    nbytes = n * torch.tensor([], dtype=dtype).element_size()
+    return ws[off:off + nbytes].view(dtype).view(shape)

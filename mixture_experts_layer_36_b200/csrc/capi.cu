@@ -1,0 +1,294 @@
+// libmoe C ABI: argument validation, capacity and workspace arithmetic, and
+// the stage launches.  Every compute step runs in the kernels of router.cu,
+// permute.cu, grouped_gemm.cu and combine.cu.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace moe {
+cudaError_t launch_route(const __nv_bfloat16* x, const float* wr, const float* bias, int T,
+                         int d, int E, int k, float* logits, int32_t* idx, float* w,
+                         cudaStream_t s);
+size_t permute_scratch_bytes(int64_t T, int64_t E);
+cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d, int E,
+                           int k, int64_t C, int32_t* counts, int32_t* offsets, int32_t* slot,
+                           int32_t* row_src, __nv_bfloat16* x_perm, int32_t* n_dropped,
+                           int32_t* chunk_hist, cudaStream_t s);
+cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
+                           int f, int max_rows, const __nv_bfloat16* w_gate,
+                           const __nv_bfloat16* w_up, __nv_bfloat16* h, int32_t* status,
+                           cudaStream_t s, bool* map_failed);
+cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
+                        int max_rows, const __nv_bfloat16* w_down, __nv_bfloat16* y_perm,
+                        int32_t* status, cudaStream_t s, bool* map_failed);
+cudaError_t launch_combine(const __nv_bfloat16* y_perm, const __nv_bfloat16* x,
+                           const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
+                           const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
+                           cudaStream_t s);
+}  // namespace moe
+
+using moe::launch_combine;
+using moe::launch_down;
+using moe::launch_gate_up;
+using moe::launch_permute;
+using moe::launch_route;
+
+namespace {
+
+constexpr int64_t kMaxE = 256;
+constexpr int64_t kMaxK = 8;
+constexpr int64_t kTileMultiple = 128;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Shape checks common to every entry point.  Returns MOE_OK or an error.
+int check_routing_shape(int64_t T, int64_t E, int64_t k) {
+  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E) return MOE_ERR_INVALID_ARG;
+  if (T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int check_width(int64_t w) {
+  if (w < 1) return MOE_ERR_INVALID_ARG;
+  if (w % kTileMultiple != 0 || w > (int64_t(1) << 20)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Byte sizes of the moe_layer_forward workspace fields, in field order.
+bool field_sizes(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf,
+                 size_t out[MOE_WS_NUM_FIELDS]) {
+  const int64_t rows = moe_max_rows(T, E, k, cf);
+  if (rows < 0 || d < 1 || f < 1) return false;
+  out[MOE_WS_STATUS] = sizeof(int32_t);
+  out[MOE_WS_LOGITS] = size_t(T * E) * sizeof(float);
+  out[MOE_WS_TOPK_IDX] = size_t(T * k) * sizeof(int32_t);
+  out[MOE_WS_TOPK_W] = size_t(T * k) * sizeof(float);
+  out[MOE_WS_SLOT] = size_t(T * k) * sizeof(int32_t);
+  out[MOE_WS_COUNTS] = size_t(E) * sizeof(int32_t);
+  out[MOE_WS_OFFSETS] = size_t(E + 1) * sizeof(int32_t);
+  out[MOE_WS_N_DROPPED] = sizeof(int32_t);
+  out[MOE_WS_ROW_SRC] = size_t(rows) * sizeof(int32_t);
+  out[MOE_WS_PERMUTE] = moe_permute_workspace_size(T, E, k);
+  out[MOE_WS_X_PERM] = size_t(rows * d) * 2;
+  out[MOE_WS_H] = size_t(rows * f) * 2;
+  out[MOE_WS_Y_PERM] = size_t(rows * d) * 2;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+int moe_version(void) { return (1 << 16) | 0; }
+
+int64_t moe_capacity(int64_t T, int64_t E, int64_t k, double cf) {
+  if (T < 0 || E < 1 || k < 1 || !(cf >= 0.0) || isinf(cf)) return -1;
+  if (cf == 0.0) return T;
+  const double c = ceil(((cf * (double)k) * (double)T) / (double)E);
+  if (c > 9.0e15) return -1;
+  return (int64_t)c;
+}
+
+int64_t moe_max_rows(int64_t T, int64_t E, int64_t k, double cf) {
+  const int64_t C = moe_capacity(T, E, k, cf);
+  if (C < 0) return -1;
+  const int64_t pairs = T * k;
+  // E * C may exceed int64 only for absurd cf; the min keeps it bounded
+  if (C >= pairs) return pairs;
+  const int64_t cap_rows = E * C;
+  return cap_rows < pairs ? cap_rows : pairs;
+}
+
+size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k) {
+  (void)k;
+  if (T < 0 || E < 1) return 0;
+  return moe::permute_scratch_bytes(T, E);
+}
+
+int64_t moe_workspace_field_offset(int field, int64_t T, int64_t d, int64_t E, int64_t k,
+                                   int64_t f, double cf) {
+  size_t sz[MOE_WS_NUM_FIELDS];
+  if (field < 0 || field >= MOE_WS_NUM_FIELDS) return -1;
+  if (!field_sizes(T, d, E, k, f, cf, sz)) return -1;
+  size_t off = 0;
+  for (int i = 0; i < field; ++i) off += align256(sz[i]);
+  return (int64_t)off;
+}
+
+size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf) {
+  size_t sz[MOE_WS_NUM_FIELDS];
+  if (!field_sizes(T, d, E, k, f, cf, sz)) return 0;
+  size_t off = 0;
+  for (int i = 0; i < MOE_WS_NUM_FIELDS; ++i) off += align256(sz[i]);
+  return off;
+}
+
+int moe_route(const void* x, const float* w_router, const float* bias, int64_t T, int64_t d,
+              int64_t E, int64_t k, float* logits, int32_t* topk_idx, float* topk_w,
+              void* stream) {
+  int st = check_routing_shape(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_width(d)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_route(static_cast<const __nv_bfloat16*>(x), w_router, bias, (int)T,
+                                  (int)d, (int)E, (int)k, logits, topk_idx, topk_w,
+                                  as_stream(stream)));
+}
+
+int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
+                int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
+                int32_t* row_src, void* x_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
+                void* stream) {
+  int st = check_routing_shape(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_width(d)) != MOE_OK) return st;
+  const int64_t C = moe_capacity(T, E, k, cf);
+  if (C < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !topk_idx || !counts || !offsets || !slot || !row_src || !x_perm || !n_dropped ||
+      !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_permute_workspace_size(T, E, k)) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_permute(static_cast<const __nv_bfloat16*>(x), topk_idx, (int)T,
+                                    (int)d, (int)E, (int)k, C, counts, offsets, slot, row_src,
+                                    static_cast<__nv_bfloat16*>(x_perm), n_dropped,
+                                    static_cast<int32_t*>(ws), as_stream(stream)));
+}
+
+static int check_gemm_args(int64_t E, int64_t d, int64_t f, int64_t max_rows) {
+  if (E < 1 || E > kMaxE || max_rows < 0 || max_rows >= (int64_t(1) << 31))
+    return MOE_ERR_INVALID_ARG;
+  int st = check_width(d);
+  if (st != MOE_OK) return st;
+  return check_width(f);
+}
+
+int moe_expert_gate_up(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d,
+                       int64_t f, int64_t max_rows, const void* w_gate, const void* w_up,
+                       void* h, int32_t* dev_status, void* stream) {
+  int st = check_gemm_args(E, d, f, max_rows);
+  if (st != MOE_OK) return st;
+  if (max_rows == 0) return MOE_OK;
+  if (!x_perm || !offsets || !w_gate || !w_up || !h) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(h))
+    return MOE_ERR_INVALID_ARG;
+  bool map_failed = false;
+  cudaError_t err = launch_gate_up(
+      static_cast<const __nv_bfloat16*>(x_perm), offsets, (int)E, (int)d, (int)f, (int)max_rows,
+      static_cast<const __nv_bfloat16*>(w_gate), static_cast<const __nv_bfloat16*>(w_up),
+      static_cast<__nv_bfloat16*>(h), dev_status, as_stream(stream), &map_failed);
+  if (map_failed) return MOE_ERR_CUDA;
+  return cuda_status(err);
+}
+
+int moe_expert_down(const void* h, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
+                    int64_t max_rows, const void* w_down, void* y_perm, int32_t* dev_status,
+                    void* stream) {
+  int st = check_gemm_args(E, d, f, max_rows);
+  if (st != MOE_OK) return st;
+  if (max_rows == 0) return MOE_OK;
+  if (!h || !offsets || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_down) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  bool map_failed = false;
+  cudaError_t err = launch_down(static_cast<const __nv_bfloat16*>(h), offsets, (int)E, (int)d,
+                                (int)f, (int)max_rows, static_cast<const __nv_bfloat16*>(w_down),
+                                static_cast<__nv_bfloat16*>(y_perm), dev_status,
+                                as_stream(stream), &map_failed);
+  if (map_failed) return MOE_ERR_CUDA;
+  return cuda_status(err);
+}
+
+int moe_expert_mlp(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
+                   int64_t max_rows, const void* w_gate, const void* w_up, const void* w_down,
+                   void* h, void* y_perm, int32_t* dev_status, void* stream) {
+  int st = moe_expert_gate_up(x_perm, offsets, E, d, f, max_rows, w_gate, w_up, h, dev_status,
+                              stream);
+  if (st != MOE_OK) return st;
+  return moe_expert_down(h, offsets, E, d, f, max_rows, w_down, y_perm, dev_status, stream);
+}
+
+int moe_combine(const void* y_perm, const void* x, const int32_t* topk_idx, const float* topk_w,
+                const int32_t* slot, const int32_t* offsets, int64_t T, int64_t d, int64_t k,
+                void* y, void* stream) {
+  if (T < 0 || k < 1 || k > kMaxK || T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  int st = check_width(d);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!y_perm || !x || !topk_idx || !topk_w || !slot || !offsets || !y)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_combine(static_cast<const __nv_bfloat16*>(y_perm),
+                                    static_cast<const __nv_bfloat16*>(x), topk_idx, topk_w, slot,
+                                    offsets, (int)T, (int)d, (int)k,
+                                    static_cast<__nv_bfloat16*>(y), as_stream(stream)));
+}
+
+int moe_layer_forward(const void* x, const float* w_router, const float* bias, const void* w_gate,
+                      const void* w_up, const void* w_down, int64_t T, int64_t d, int64_t E,
+                      int64_t k, int64_t f, double cf, void* y, void* ws, size_t ws_bytes,
+                      void* stream) {
+  int st = check_routing_shape(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_width(d)) != MOE_OK) return st;
+  if ((st = check_width(f)) != MOE_OK) return st;
+  if (moe_capacity(T, E, k, cf) < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !w_gate || !w_up || !w_down || !y || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_workspace_size(T, d, E, k, f, cf)) return MOE_ERR_WORKSPACE;
+
+  char* base = static_cast<char*>(ws);
+  auto field = [&](int id) {
+    return base + moe_workspace_field_offset(id, T, d, E, k, f, cf);
+  };
+  int32_t* status = reinterpret_cast<int32_t*>(field(MOE_WS_STATUS));
+  float* logits = reinterpret_cast<float*>(field(MOE_WS_LOGITS));
+  int32_t* topk_idx = reinterpret_cast<int32_t*>(field(MOE_WS_TOPK_IDX));
+  float* topk_w = reinterpret_cast<float*>(field(MOE_WS_TOPK_W));
+  int32_t* slot = reinterpret_cast<int32_t*>(field(MOE_WS_SLOT));
+  int32_t* counts = reinterpret_cast<int32_t*>(field(MOE_WS_COUNTS));
+  int32_t* offsets = reinterpret_cast<int32_t*>(field(MOE_WS_OFFSETS));
+  int32_t* n_dropped = reinterpret_cast<int32_t*>(field(MOE_WS_N_DROPPED));
+  int32_t* row_src = reinterpret_cast<int32_t*>(field(MOE_WS_ROW_SRC));
+  void* pscratch = field(MOE_WS_PERMUTE);
+  void* x_perm = field(MOE_WS_X_PERM);
+  void* h = field(MOE_WS_H);
+  void* y_perm = field(MOE_WS_Y_PERM);
+  const int64_t max_rows = moe_max_rows(T, E, k, cf);
+  cudaStream_t s = as_stream(stream);
+
+  if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, stream)) != MOE_OK)
+    return st;
+  if ((st = moe_permute(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src, x_perm,
+                        n_dropped, pscratch, moe_permute_workspace_size(T, E, k), stream)) !=
+      MOE_OK)
+    return st;
+  if ((st = moe_expert_mlp(x_perm, offsets, E, d, f, max_rows, w_gate, w_up, w_down, h, y_perm,
+                           status, stream)) != MOE_OK)
+    return st;
+  return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// Combine: inverse permutation plus gate-weighted sum.
+//
+// The combine undoes the dispatch permutation and sums each token's k expert
+// outputs scaled by their gate weights ("Expert Parallelism & All-to-All"
+// (neelmishra.github.io), section "All-to-all: the distributed transpose";
+// last step of the infra.bea.ai guide's section 2 diagram).  A token whose
+// pairs were all dropped leaves the layer unchanged (inferensys.com glossary,
+// Dropped Tokens entry).
+//
+// One warp per token: lanes 0..k-1 resolve the k source rows and weights,
+// broadcast them, then the warp streams the d-wide rows in 16-byte vectors,
+// accumulating in fp32 in top-k order and rounding once to bf16.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kCombThreads = 256;
+
+__global__ void __launch_bounds__(kCombThreads)
+    combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const __nv_bfloat16* __restrict__ x,
+                   const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
+                   const int32_t* __restrict__ slot, const int32_t* __restrict__ offsets, int T,
+                   int d, int k, __nv_bfloat16* __restrict__ y) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x * (kCombThreads / 32) + warp;
+  if (t >= T) return;
+  int my_row = -1;
+  float my_w = 0.f;
+  if (lane < k) {
+    const size_t p = (size_t)t * k + lane;
+    const int s = slot[p];
+    if (s >= 0) {
+      my_row = offsets[topk_idx[p]] + s;
+      my_w = topk_w[p];
+    }
+  }
+  int rows[8];
+  float w[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+    w[j] = __shfl_sync(0xffffffffu, my_w, j);
+  }
+  const bool any_kept = __any_sync(0xffffffffu, my_row >= 0);
+  const int nvec = d / 8;
+  uint4* dst = reinterpret_cast<uint4*>(y + (size_t)t * d);
+  if (!any_kept) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    return;
+  }
+  for (int v0 = lane; v0 < nvec; v0 += 64) {
+    float acc[2][8];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      if (rows[j] < 0) continue;
+      const uint4* src = reinterpret_cast<const uint4*>(y_perm + (size_t)rows[j] * d);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int v = v0 + u * 32;
+        if (v >= nvec) continue;
+        const uint4 raw = __ldg(src + v);
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f2 = __bfloat1622float2(b[q]);
+          acc[u][2 * q] = fmaf(w[j], f2.x, acc[u][2 * q]);
+          acc[u][2 * q + 1] = fmaf(w[j], f2.y, acc[u][2 * q + 1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = v0 + u * 32;
+      if (v >= nvec) continue;
+      uint4 o;
+      o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+      o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+      o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+      o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+      dst[v] = o;
+    }
+  }
+}
+
+cudaError_t launch_combine(const __nv_bfloat16* y_perm, const __nv_bfloat16* x,
+                           const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
+                           const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
+                           cudaStream_t s) {
+  const int per_cta = kCombThreads / 32;
+  combine_kernel<<<(T + per_cta - 1) / per_cta, kCombThreads, 0, s>>>(
+      y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

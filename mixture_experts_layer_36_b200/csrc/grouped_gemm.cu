@@ -1,0 +1,446 @@
+// Grouped expert GEMMs over ragged per-expert buckets on the sm_100a tensor
+// cores (tcgen05.mma, accumulators in TMEM, operands staged by TMA).
+//
+// Experts are gate/up/down MLPs ("Expert Parallelism & All-to-All"
+// (neelmishra.github.io), section "Tensor parallelism for experts"); the
+// per-expert matmuls over the token buckets are grouped GEMMs (klaylearn.com
+// "Expert Parallelism" glossary, fourth paragraph).
+//
+//   GEMM 1 (SWIGLU = true):  h[r, :]      = silu(x_perm[r] Wg[e]) * (x_perm[r] Wu[e])
+//   GEMM 2 (SWIGLU = false): y_perm[r, :] = h[r] Wd[e]
+// for every row r of bucket e (offsets[e] <= r < offsets[e+1]).
+//
+// Tiling.  A tile is 128 bucket rows x BN accumulator columns.  GEMM 1 puts the
+// gate and the up projection of the same 128 h-columns side by side in one
+// N = 256 MMA (accumulator columns [0,128) = gate, [128,256) = up), so the
+// SwiGLU is an epilogue over one TMEM tile.  A (rows, K-contiguous) is loaded
+// K-major; B is the weight [K, N] with N contiguous, loaded and consumed
+// MN-major, so the weights are used in the layout they are given.
+//
+// Schedule.  Persistent CTAs (one per SM) walk a tile list built on the device
+// from `offsets` (no host sync): per-expert tile counts ceil(n_e/128) x
+// n_tiles are prefix-summed in shared memory and tile i is decoded by binary
+// search.  Inside an expert the row tile varies fastest, so CTAs running at
+// the same time share each weight tile through L2.
+//
+// Roles (192 threads): warp 0 lane 0 issues TMA into a ring of smem stages,
+// warp 1 lane 0 issues tcgen05.mma into one of two TMEM accumulators, warps
+// 2..5 drain the other accumulator (tcgen05.ld -> SwiGLU -> bf16 stores), so
+// the epilogue of tile i overlaps the main loop of tile i+1.
+//
+// Every mbarrier wait is time-limited: a role that gives up sets the CTA's
+// abort flag and the caller's status bit, the others notice and stop, the
+// producer waits for its copies in flight, the MMA issuer waits for its MMAs,
+// and TMEM is freed before the CTA exits.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;                 // one 128-byte swizzle atom of bf16 along K
+constexpr int kGemmThreads = 192;
+constexpr int kUmmaK = 16;
+constexpr int kChunkBytes = 64 * kBK * 2;   // one B chunk: 64 N x 64 K bf16 = 8 KB
+
+template <int BN, bool SWIGLU>
+struct GemmCfg {
+  static constexpr int kOutCols = SWIGLU ? BN / 2 : BN;  // output columns per tile
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
+};
+
+struct GemmShared {
+  uint64_t full_bar[8];
+  uint64_t empty_bar[8];
+  uint64_t tfull_bar[2];
+  uint64_t tempty_bar[2];
+  uint64_t drain_bar;
+  uint32_t tmem_base;
+  int abort_flag;
+  int never;                       // stays 0: wait with a time limit only
+  int tile_prefix[257];
+  int row_off[256];
+  int row_cnt[256];
+};
+
+__device__ __forceinline__ void decode_tile(const GemmShared& sh, int tile, int E, int n_tiles,
+                                            int& e, int& m, int& n) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sh.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int local = tile - sh.tile_prefix[e];
+  const int mt = (sh.tile_prefix[e + 1] - sh.tile_prefix[e]) / n_tiles;
+  n = local / mt;
+  m = local - n * mt;
+}
+
+template <int BN, bool SWIGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1,
+                        const int32_t* __restrict__ offsets, int E, int K, int n_out,
+                        int max_rows, __nv_bfloat16* __restrict__ out, int32_t* status) {
+  using Cfg = GemmCfg<BN, SWIGLU>;
+  extern __shared__ uint8_t dsmem_raw[];
+  __shared__ GemmShared sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_tiles = n_out / Cfg::kOutCols;
+  const int nkb = K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&sh.full_bar[s], 1);
+      mbar_init(&sh.empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sh.tfull_bar[a], 1);
+      mbar_init(&sh.tempty_bar[a], 4);
+    }
+    mbar_init(&sh.drain_bar, 1);
+    sh.abort_flag = 0;
+    sh.never = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 1 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB0);
+    if (SWIGLU) prefetch_tensormap(&tmB1);
+  }
+  if (warp == 2) {
+    // per-expert tile counts -> exclusive prefix; row offsets to smem
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int tiles = 0;
+      if (e < E) {
+        const int o0 = offsets[e], o1 = offsets[e + 1];
+        int cnt = o1 - o0;
+        if (o0 < 0 || cnt < 0 || o1 > max_rows) {
+          report(status, kDevErrBadOffsets);
+          cnt = 0;
+        }
+        sh.row_off[e] = o0;
+        sh.row_cnt[e] = cnt;
+        tiles = cnt > 0 ? ((cnt + kBM - 1) / kBM) * n_tiles : 0;
+      }
+      int incl = tiles;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (e < E) sh.tile_prefix[e] = carry + incl - tiles;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) sh.tile_prefix[E] = carry;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = sh.tmem_base;
+  const int total_tiles = sh.tile_prefix[E];
+  volatile int* abort_flag = &sh.abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int it = 0;
+      int last_it[8];
+      for (int s = 0; s < Cfg::kStages; ++s) last_it[s] = -1;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        int e, m, n;
+        decode_tile(sh, tile, E, n_tiles, e, m, n);
+        const int row0 = sh.row_off[e] + m * kBM;
+        const int col0 = n * Cfg::kOutCols;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % Cfg::kStages;
+          const uint32_t ph = (it / Cfg::kStages) & 1;
+          if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t* sa = smem + s * Cfg::kStageBytes;
+          uint8_t* sb = sa + Cfg::kABytes;
+          mbar_arrive_expect_tx(&sh.full_bar[s], Cfg::kStageBytes);
+          tma_load_2d(sa, &tmA, &sh.full_bar[s], kb * kBK, row0);
+          if (SWIGLU) {
+#pragma unroll
+            for (int c = 0; c < BN / 128; ++c)
+              tma_load_3d(sb + c * kChunkBytes, &tmB0, &sh.full_bar[s], col0 + c * 64, kb * kBK, e);
+#pragma unroll
+            for (int c = 0; c < BN / 128; ++c)
+              tma_load_3d(sb + (BN / 128 + c) * kChunkBytes, &tmB1, &sh.full_bar[s],
+                          col0 + c * 64, kb * kBK, e);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_3d(sb + c * kChunkBytes, &tmB0, &sh.full_bar[s], col0 + c * 64, kb * kBK, e);
+          }
+          last_it[s] = it;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(status, kDevErrWaitTimeout);
+      }
+      // never leave with copies in flight: every stage's last fill must land
+      for (int s = 0; s < Cfg::kStages; ++s)
+        if (last_it[s] >= 0)
+          mbar_wait(&sh.full_bar[s], (last_it[s] / Cfg::kStages) & 1, &sh.never);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++lt) {
+        const int a = lt & 1;
+        const uint32_t aph = (lt >> 1) & 1;
+        if (!mbar_wait(&sh.tempty_bar[a], aph ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BN);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % Cfg::kStages;
+          const uint32_t ph = (it / Cfg::kStages) & 1;
+          if (!mbar_wait(&sh.full_bar[s], ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * Cfg::kStageBytes);
+          const uint32_t b_addr = a_addr + Cfg::kABytes;
+#pragma unroll
+          for (int ks = 0; ks < kBK / kUmmaK; ++ks) {
+            // A: K-major rows of 128 B, 8-row atoms 1024 B apart; +32 B per K step
+            const uint64_t adesc = smem_desc_sw128(a_addr + ks * 32, 16, 1024);
+            // B: MN-major; 64-wide N chunks 8 KB apart (LBO), 8-row K groups
+            // 1024 B apart (SBO); +16 K rows = +2048 B per K step
+            const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, kChunkBytes, 1024);
+            umma_bf16(d_tmem, adesc, bdesc, Cfg::kIdesc, (kb | ks) != 0 ? 1u : 0u);
+          }
+          umma_commit(&sh.empty_bar[s]);
+        }
+        if (!ok) break;
+        umma_commit(&sh.tfull_bar[a]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(status, kDevErrWaitTimeout);
+      }
+      // wait until every MMA issued by this thread has finished
+      umma_commit(&sh.drain_bar);
+      mbar_wait(&sh.drain_bar, 0, &sh.never);
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;                 // TMEM lane quarter this warp may read
+    const int row_in_tile = q * 32 + lane;
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
+      int e, m, n;
+      decode_tile(sh, tile, E, n_tiles, e, m, n);
+      const int a = lt & 1;
+      const uint32_t aph = (lt >> 1) & 1;
+      if (!mbar_wait(&sh.tfull_bar[a], aph, abort_flag)) {
+        *abort_flag = 1;
+        report(status, kDevErrWaitTimeout);
+        break;
+      }
+      tc_fence_after();
+      const int local_row = m * kBM + row_in_tile;
+      const bool valid = local_row < sh.row_cnt[e];
+      __nv_bfloat16* orow = out + (size_t)(sh.row_off[e] + local_row) * n_out +
+                            (size_t)n * Cfg::kOutCols;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * BN);
+      if (SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2 / 32; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, g);
+          tmem_ld_32x32b_x32(tbase + BN / 2 + c * 32, u);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+              pk[i] = pack_bf16x2(silu(g0) * u0, silu(g1) * u1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.tempty_bar[a]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 [outer, inner] row-major, box (64 inner, box_outer), 128-B swizzle.
+static bool map_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                     uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// 3-D bf16 weights [E, K, N] (N contiguous), box (64 N, 64 K, 1), 128-B swizzle.
+static bool map_weights(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {N, K, E};
+  cuuint64_t strides[2] = {N * 2, K * N * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kBK, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool attr_set[4] = {false, false, false, false};
+};
+static DeviceInfo g_dev[64];
+
+static cudaError_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  DeviceInfo& di = g_dev[dev];
+  if (di.sms == 0) {
+    err = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+  }
+  *out = &di;
+  return cudaSuccess;
+}
+
+template <int BN, bool SWIGLU>
+static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& b0,
+                               const CUtensorMap& b1, const int32_t* offsets, int E, int K,
+                               int n_out, int max_rows, __nv_bfloat16* out, int32_t* status,
+                               cudaStream_t s) {
+  using Cfg = GemmCfg<BN, SWIGLU>;
+  DeviceInfo* di = nullptr;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  auto kern = grouped_gemm_kernel<BN, SWIGLU>;
+  if (!di->attr_set[slot]) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    di->attr_set[slot] = true;
+  }
+  const int n_tiles = n_out / Cfg::kOutCols;
+  const long long row_tiles = (long long)max_rows / kBM + (E < max_rows ? E : max_rows);
+  long long ub = row_tiles * n_tiles;
+  int grid = (int)(ub < di->sms ? ub : di->sms);
+  if (grid < 1) grid = 1;
+  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, b0, b1, offsets, E, K, n_out, max_rows,
+                                                     out, status);
+  return cudaGetLastError();
+}
+
+// GEMM 1: h = silu(x_perm Wg) * (x_perm Wu)
+cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
+                           int f, int max_rows, const __nv_bfloat16* w_gate,
+                           const __nv_bfloat16* w_up, __nv_bfloat16* h, int32_t* status,
+                           cudaStream_t s, bool* map_failed) {
+  CUtensorMap ta, tg, tu;
+  *map_failed = !(map_rows(&ta, x_perm, d, max_rows, kBM) && map_weights(&tg, w_gate, E, d, f) &&
+                  map_weights(&tu, w_up, E, d, f));
+  if (*map_failed) return cudaSuccess;
+  return launch_gemm<256, true>(0, ta, tg, tu, offsets, E, d, f, max_rows, h, status, s);
+}
+
+// GEMM 2: y_perm = h Wd
+cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
+                        int max_rows, const __nv_bfloat16* w_down, __nv_bfloat16* y_perm,
+                        int32_t* status, cudaStream_t s, bool* map_failed) {
+  CUtensorMap ta, td;
+  *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_weights(&td, w_down, E, f, d));
+  if (*map_failed) return cudaSuccess;
+  if (d % 256 == 0)
+    return launch_gemm<256, false>(1, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);
+  return launch_gemm<128, false>(2, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);
+}
+
+int device_sm_count() {
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != cudaSuccess) return 0;
+  return di->sms;
+}
+
+}  // namespace moe

@@ -19,3 +19,10 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_sessionstart(session):
+    # nvcc cross-compiles sm_100a without a GPU, so the C-ABI library can be
+    # (re)built here when the sources are newer than the .so
+    from mixture_experts_layer_36_b200 import build
+    build.build()

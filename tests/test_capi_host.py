@@ -1,0 +1,112 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/moe.h declares, and its host-side arithmetic and validation behave as
+documented (no kernel is launched by any call here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import mixture_experts_layer_36_b200 as moe
+from mixture_experts_layer_36_b200 import binding, configs
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "moe.h")
+
+OK, INVALID, WORKSPACE, CUDA, UNSUPPORTED = 0, 1, 2, 3, 4
+FAKE = ctypes.c_void_p(1 << 20)   # aligned non-null pointer; never dereferenced on these paths
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 14
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(binding.EXPORTED) == names
+
+
+def test_version_and_status_strings():
+    assert moe.lib().moe_version() >> 16 == 1
+    assert moe.moe_status_string(0) == "MOE_OK"
+    assert moe.moe_status_string(4) == "MOE_ERR_UNSUPPORTED"
+    assert moe.moe_status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("T,E,k,cf", [(64, 8, 2, 1.25), (8192, 256, 8, 1.25), (16384, 64, 6, 1.0),
+                                      (4096, 8, 2, 0.0), (10, 3, 1, 1.0), (7, 5, 2, 3.3),
+                                      (0, 4, 2, 1.0)])
+def test_capacity_agrees_with_oracle(T, E, k, cf):
+    assert moe.moe_capacity(T, E, k, cf) == oracle.capacity(T, E, k, cf)
+    C = oracle.capacity(T, E, k, cf)
+    assert moe.moe_max_rows(T, E, k, cf) == min(T * k, E * C)
+
+
+def test_capacity_rejects_bad_args():
+    assert moe.moe_capacity(10, 0, 1, 1.0) == -1
+    assert moe.moe_capacity(10, 4, 0, 1.0) == -1
+    assert moe.moe_capacity(10, 4, 1, -1.0) == -1
+    assert moe.moe_capacity(10, 4, 1, float("nan")) == -1
+
+
+@pytest.mark.parametrize("cfg", list(configs.ALL.values()), ids=list(configs.ALL))
+def test_workspace_layout(cfg):
+    T, d, E, k, f, cf = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.cf
+    total = moe.moe_workspace_size(T, d, E, k, f, cf)
+    offs = [moe.moe_workspace_field_offset(i, T, d, E, k, f, cf) for i in range(13)]
+    assert offs[0] == 0 and all(o % 256 == 0 for o in offs)
+    assert offs == sorted(offs)
+    rows = moe.moe_max_rows(T, E, k, cf)
+    assert total - offs[12] >= rows * d * 2          # y_perm is last
+    assert offs[12] - offs[11] >= rows * f * 2       # h
+    assert offs[11] - offs[10] >= rows * d * 2       # x_perm
+    assert moe.moe_workspace_field_offset(13, T, d, E, k, f, cf) == -1
+
+
+def test_validation_codes_without_launch():
+    L = moe.lib()
+    s = ctypes.c_void_p(0)
+    # route: bad E, bad k, k > E, unsupported width, empty batch
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 0, 1, FAKE, FAKE, FAKE, s) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 300, 2, FAKE, FAKE, FAKE, s) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 8, 9, FAKE, FAKE, FAKE, s) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 2, 3, FAKE, FAKE, FAKE, s) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 4, 100, 8, 2, FAKE, FAKE, FAKE, s) == UNSUPPORTED
+    assert L.moe_route(None, FAKE, None, 4, 128, 8, 2, FAKE, FAKE, FAKE, s) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 0, 128, 8, 2, FAKE, FAKE, FAKE, s) == OK
+    misaligned = ctypes.c_void_p((1 << 20) + 2)
+    assert L.moe_route(misaligned, FAKE, None, 4, 128, 8, 2, FAKE, FAKE, FAKE, s) == INVALID
+    # permute: workspace too small
+    need = moe.moe_permute_workspace_size(100, 8, 2)
+    assert need > 0
+    args = [FAKE, FAKE, 100, 128, 8, 2, 1.25, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE]
+    assert L.moe_permute(*args, need - 1, s) == WORKSPACE
+    assert L.moe_permute(*args[:6], -1.0, *args[7:], need, s) == INVALID
+    # experts: widths must be multiples of 128
+    assert L.moe_expert_gate_up(FAKE, FAKE, 8, 192, 256, 100, FAKE, FAKE, FAKE, None, s) \
+        == UNSUPPORTED
+    assert L.moe_expert_down(FAKE, FAKE, 8, 256, 200, 100, FAKE, FAKE, None, s) == UNSUPPORTED
+    assert L.moe_expert_mlp(FAKE, FAKE, 8, 256, 256, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None, s) \
+        == OK
+    # combine / layer
+    assert L.moe_combine(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10, 128, 9, FAKE, s) == INVALID
+    ws_need = moe.moe_workspace_size(64, 128, 8, 2, 256, 1.25)
+    assert L.moe_layer_forward(FAKE, FAKE, None, FAKE, FAKE, FAKE, 64, 128, 8, 2, 256, 1.25, FAKE,
+                               FAKE, ws_need - 1, s) == WORKSPACE
+    assert L.moe_layer_forward(FAKE, FAKE, None, FAKE, FAKE, FAKE, 64, 128, 8, 2, 250, 1.25, FAKE,
+                               FAKE, ws_need, s) == UNSUPPORTED
+    assert L.moe_layer_forward(FAKE, FAKE, None, FAKE, FAKE, FAKE, 0, 128, 8, 2, 256, 1.25, FAKE,
+                               FAKE, 0, s) == OK
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        moe.moe_route(x, torch.zeros(128, 8), None, 2)

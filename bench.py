@@ -128,7 +128,7 @@ class Layer:
                      "n_dropped": z(1, dt=torch.int32)}
         self.pws = z(max(moe.moe_permute_workspace_size(T, E, k), 16), dt=torch.uint8)
         self.h = z(self.rows, f, dt=torch.bfloat16)
-        self.y_perm = z(self.rows, d, dt=torch.bfloat16)
+        self.y_perm = z(self.rows, d, dt=torch.float32)
         self.y = z(T, d, dt=torch.bfloat16)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.ws = z(moe.moe_workspace_size(T, d, E, k, f, cfg.cf), dt=torch.uint8)
@@ -319,7 +319,7 @@ def main():
     peak_tf = pk["bf16_tflops"]
     achieved = gemm1_flop / t_g1 / 1e12
     bytes_perm = cfg.T * cfg.d * 2 + r["N"] * cfg.d * 2
-    bytes_comb = r["N"] * cfg.d * 2 + cfg.T * cfg.d * 2
+    bytes_comb = r["N"] * cfg.d * 4 + cfg.T * cfg.d * 2
     out = {
         "metric": METRIC,
         "value": round(value, 1),

@@ -12,7 +12,8 @@
  *            C = ceil(cf*k*T/E) (dropless when cf == 0), slots in token order,
  *            overflow dropped
  *   experts  per expert e: h = silu(x_perm Wg[e]) * (x_perm Wu[e]),
- *            y_perm = h Wd[e]  (SwiGLU)
+ *            y_perm = h Wd[e]  (SwiGLU; h stored bf16, y_perm kept fp32 so the
+ *            layer output is rounded to bf16 only once, in the combine)
  *   combine  y[t] = sum over kept pairs j of w[t,j] * y_perm[row(t,j)], in
  *            top-k order; a token whose k pairs were all dropped gets x[t]
  *
@@ -91,7 +92,7 @@ typedef enum {
   MOE_WS_PERMUTE = 9,    /* moe_permute scratch */
   MOE_WS_X_PERM = 10,    /* bf16 [max_rows, d] */
   MOE_WS_H = 11,         /* bf16 [max_rows, f] */
-  MOE_WS_Y_PERM = 12,    /* bf16 [max_rows, d] */
+  MOE_WS_Y_PERM = 12,    /* f32  [max_rows, d] */
   MOE_WS_NUM_FIELDS = 13
 } moe_ws_field;
 
@@ -152,17 +153,18 @@ int moe_expert_gate_up(const void* x_perm, const int32_t* offsets, int64_t E, in
                        void* h, int32_t* dev_status, void* stream);
 
 /* Grouped expert GEMM 2 (down projection): y_perm[r,:] = h[r,:] Wd[e] for the
- * rows of bucket e.  h bf16 [max_rows,f], w_down bf16 [E,f,d], y_perm bf16
- * [max_rows,d] out.  Same source passages as moe_expert_gate_up. */
+ * rows of bucket e.  h bf16 [max_rows,f], w_down bf16 [E,f,d], y_perm f32
+ * [max_rows,d] out (fp32 accumulation, stored unrounded; rows of no bucket
+ * are left untouched).  Same source passages as moe_expert_gate_up. */
 int moe_expert_down(const void* h, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
-                    int64_t max_rows, const void* w_down, void* y_perm, int32_t* dev_status,
+                    int64_t max_rows, const void* w_down, float* y_perm, int32_t* dev_status,
                     void* stream);
 
 /* Both expert GEMMs: moe_expert_gate_up then moe_expert_down, with h as the
  * caller's buffer in between. */
 int moe_expert_mlp(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
                    int64_t max_rows, const void* w_gate, const void* w_up, const void* w_down,
-                   void* h, void* y_perm, int32_t* dev_status, void* stream);
+                   void* h, float* y_perm, int32_t* dev_status, void* stream);
 
 /* Inverse permutation and gate-weighted sum (the combine undoes the dispatch
  * permutation and adds each token's k expert outputs scaled by their gate
@@ -172,8 +174,9 @@ int moe_expert_mlp(const void* x_perm, const int32_t* offsets, int64_t E, int64_
  * glossary, Dropped Tokens entry).
  *   y[t,:] = sum_{j: slot[t,j] >= 0} topk_w[t,j] * y_perm[offsets[topk_idx[t,j]] + slot[t,j], :]
  * summed in fp32 in j order and rounded once to bf16; if no pair of t was
- * kept, y[t,:] = x[t,:] exactly.  y bf16 [T,d] out. */
-int moe_combine(const void* y_perm, const void* x, const int32_t* topk_idx, const float* topk_w,
+ * kept, y[t,:] = x[t,:] exactly.  y_perm f32 [>= offsets[E], d], x bf16
+ * [T,d], y bf16 [T,d] out. */
+int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, const float* topk_w,
                 const int32_t* slot, const int32_t* offsets, int64_t T, int64_t d, int64_t k,
                 void* y, void* stream);
 

@@ -208,9 +208,9 @@ def moe_expert_down(h, offsets, w_down, y_perm=None, dev_status=None, stream=Non
     _want(h, "h", torch.bfloat16)
     _want(offsets, "offsets", torch.int32, (E + 1,))
     _want(w_down, "w_down", torch.bfloat16, (E, f, d))
-    y_perm = torch.empty(rows, d, dtype=torch.bfloat16, device=h.device) if y_perm is None \
+    y_perm = torch.empty(rows, d, dtype=torch.float32, device=h.device) if y_perm is None \
         else y_perm
-    _want(y_perm, "y_perm", torch.bfloat16, (rows, d))
+    _want(y_perm, "y_perm", torch.float32, (rows, d))
     _check("moe_expert_down", _lib.moe_expert_down(
         _ptr(h), _ptr(offsets), E, d, f, rows, _ptr(w_down), _ptr(y_perm), _ptr(dev_status),
         _stream(stream)))
@@ -228,9 +228,9 @@ def moe_expert_mlp(x_perm, offsets, w_gate, w_up, w_down, h=None, y_perm=None, d
     _want(w_down, "w_down", torch.bfloat16, (E, f, d))
     dev = x_perm.device
     h = torch.empty(rows, f, dtype=torch.bfloat16, device=dev) if h is None else h
-    y_perm = torch.empty(rows, d, dtype=torch.bfloat16, device=dev) if y_perm is None else y_perm
+    y_perm = torch.empty(rows, d, dtype=torch.float32, device=dev) if y_perm is None else y_perm
     _want(h, "h", torch.bfloat16, (rows, f))
-    _want(y_perm, "y_perm", torch.bfloat16, (rows, d))
+    _want(y_perm, "y_perm", torch.float32, (rows, d))
     _check("moe_expert_mlp", _lib.moe_expert_mlp(
         _ptr(x_perm), _ptr(offsets), E, d, f, rows, _ptr(w_gate), _ptr(w_up), _ptr(w_down),
         _ptr(h), _ptr(y_perm), _ptr(dev_status), _stream(stream)))
@@ -240,7 +240,7 @@ def moe_expert_mlp(x_perm, offsets, w_gate, w_up, w_down, h=None, y_perm=None, d
 def moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, y=None, stream=None):
     T, d = x.shape
     k = topk_idx.shape[1]
-    _want(y_perm, "y_perm", torch.bfloat16)
+    _want(y_perm, "y_perm", torch.float32)
     _want(x, "x", torch.bfloat16)
     _want(topk_idx, "topk_idx", torch.int32, (T, k))
     _want(topk_w, "topk_w", torch.float32, (T, k))
@@ -287,7 +287,7 @@ def workspace_view(ws, field, T, d, E, k, f, cf):
         "slot": (torch.int32, (T, k)), "counts": (torch.int32, (E,)),
         "offsets": (torch.int32, (E + 1,)), "n_dropped": (torch.int32, (1,)),
         "row_src": (torch.int32, (rows,)), "x_perm": (torch.bfloat16, (rows, d)),
-        "h": (torch.bfloat16, (rows, f)), "y_perm": (torch.bfloat16, (rows, d)),
+        "h": (torch.bfloat16, (rows, f)), "y_perm": (torch.float32, (rows, d)),
     }[field]
     dtype, shape = spec
     off = moe_workspace_field_offset(field, T, d, E, k, f, cf)

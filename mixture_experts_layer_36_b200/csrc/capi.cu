@@ -19,9 +19,9 @@ cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, 
                            const __nv_bfloat16* w_up, __nv_bfloat16* h, int32_t* status,
                            cudaStream_t s, bool* map_failed);
 cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
-                        int max_rows, const __nv_bfloat16* w_down, __nv_bfloat16* y_perm,
+                        int max_rows, const __nv_bfloat16* w_down, float* y_perm,
                         int32_t* status, cudaStream_t s, bool* map_failed);
-cudaError_t launch_combine(const __nv_bfloat16* y_perm, const __nv_bfloat16* x,
+cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t s);
@@ -77,7 +77,7 @@ bool field_sizes(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double c
   out[MOE_WS_PERMUTE] = moe_permute_workspace_size(T, E, k);
   out[MOE_WS_X_PERM] = size_t(rows * d) * 2;
   out[MOE_WS_H] = size_t(rows * f) * 2;
-  out[MOE_WS_Y_PERM] = size_t(rows * d) * 2;
+  out[MOE_WS_Y_PERM] = size_t(rows * d) * sizeof(float);
   return true;
 }
 
@@ -203,7 +203,7 @@ int moe_expert_gate_up(const void* x_perm, const int32_t* offsets, int64_t E, in
 }
 
 int moe_expert_down(const void* h, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
-                    int64_t max_rows, const void* w_down, void* y_perm, int32_t* dev_status,
+                    int64_t max_rows, const void* w_down, float* y_perm, int32_t* dev_status,
                     void* stream) {
   int st = check_gemm_args(E, d, f, max_rows);
   if (st != MOE_OK) return st;
@@ -213,7 +213,7 @@ int moe_expert_down(const void* h, const int32_t* offsets, int64_t E, int64_t d,
   bool map_failed = false;
   cudaError_t err = launch_down(static_cast<const __nv_bfloat16*>(h), offsets, (int)E, (int)d,
                                 (int)f, (int)max_rows, static_cast<const __nv_bfloat16*>(w_down),
-                                static_cast<__nv_bfloat16*>(y_perm), dev_status,
+                                y_perm, dev_status,
                                 as_stream(stream), &map_failed);
   if (map_failed) return MOE_ERR_CUDA;
   return cuda_status(err);
@@ -221,14 +221,14 @@ int moe_expert_down(const void* h, const int32_t* offsets, int64_t E, int64_t d,
 
 int moe_expert_mlp(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
                    int64_t max_rows, const void* w_gate, const void* w_up, const void* w_down,
-                   void* h, void* y_perm, int32_t* dev_status, void* stream) {
+                   void* h, float* y_perm, int32_t* dev_status, void* stream) {
   int st = moe_expert_gate_up(x_perm, offsets, E, d, f, max_rows, w_gate, w_up, h, dev_status,
                               stream);
   if (st != MOE_OK) return st;
   return moe_expert_down(h, offsets, E, d, f, max_rows, w_down, y_perm, dev_status, stream);
 }
 
-int moe_combine(const void* y_perm, const void* x, const int32_t* topk_idx, const float* topk_w,
+int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, const float* topk_w,
                 const int32_t* slot, const int32_t* offsets, int64_t T, int64_t d, int64_t k,
                 void* y, void* stream) {
   if (T < 0 || k < 1 || k > kMaxK || T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
@@ -238,8 +238,8 @@ int moe_combine(const void* y_perm, const void* x, const int32_t* topk_idx, cons
   if (!y_perm || !x || !topk_idx || !topk_w || !slot || !offsets || !y)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(y_perm) || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_combine(static_cast<const __nv_bfloat16*>(y_perm),
-                                    static_cast<const __nv_bfloat16*>(x), topk_idx, topk_w, slot,
+  return cuda_status(launch_combine(y_perm, static_cast<const __nv_bfloat16*>(x), topk_idx,
+                                    topk_w, slot,
                                     offsets, (int)T, (int)d, (int)k,
                                     static_cast<__nv_bfloat16*>(y), as_stream(stream)));
 }
@@ -274,7 +274,7 @@ int moe_layer_forward(const void* x, const float* w_router, const float* bias, c
   void* pscratch = field(MOE_WS_PERMUTE);
   void* x_perm = field(MOE_WS_X_PERM);
   void* h = field(MOE_WS_H);
-  void* y_perm = field(MOE_WS_Y_PERM);
+  float* y_perm = reinterpret_cast<float*>(field(MOE_WS_Y_PERM));
   const int64_t max_rows = moe_max_rows(T, E, k, cf);
   cudaStream_t s = as_stream(stream);
 

@@ -8,8 +8,8 @@
 // Dropped Tokens entry).
 //
 // One warp per token: lanes 0..k-1 resolve the k source rows and weights,
-// broadcast them, then the warp streams the d-wide rows in 16-byte vectors,
-// accumulating in fp32 in top-k order and rounding once to bf16.
+// broadcast them, then the warp streams the d-wide fp32 rows in 16-byte
+// vectors, accumulating in fp32 in top-k order and rounding once to bf16.
 #include "common.cuh"
 
 namespace moe {
@@ -17,7 +17,7 @@ namespace moe {
 constexpr int kCombThreads = 256;
 
 __global__ void __launch_bounds__(kCombThreads)
-    combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const __nv_bfloat16* __restrict__ x,
+    combine_kernel(const float* __restrict__ y_perm, const __nv_bfloat16* __restrict__ x,
                    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ slot, const int32_t* __restrict__ offsets, int T,
                    int d, int k, __nv_bfloat16* __restrict__ y) {
@@ -59,19 +59,21 @@ __global__ void __launch_bounds__(kCombThreads)
     for (int j = 0; j < 8; ++j) {
       if (j >= k) break;
       if (rows[j] < 0) continue;
-      const uint4* src = reinterpret_cast<const uint4*>(y_perm + (size_t)rows[j] * d);
+      const float4* src = reinterpret_cast<const float4*>(y_perm + (size_t)rows[j] * d);
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int v = v0 + u * 32;
         if (v >= nvec) continue;
-        const uint4 raw = __ldg(src + v);
-        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f2 = __bfloat1622float2(b[q]);
-          acc[u][2 * q] = fmaf(w[j], f2.x, acc[u][2 * q]);
-          acc[u][2 * q + 1] = fmaf(w[j], f2.y, acc[u][2 * q + 1]);
-        }
+        const float4 a = __ldg(src + 2 * v);
+        const float4 b = __ldg(src + 2 * v + 1);
+        acc[u][0] = fmaf(w[j], a.x, acc[u][0]);
+        acc[u][1] = fmaf(w[j], a.y, acc[u][1]);
+        acc[u][2] = fmaf(w[j], a.z, acc[u][2]);
+        acc[u][3] = fmaf(w[j], a.w, acc[u][3]);
+        acc[u][4] = fmaf(w[j], b.x, acc[u][4]);
+        acc[u][5] = fmaf(w[j], b.y, acc[u][5]);
+        acc[u][6] = fmaf(w[j], b.z, acc[u][6]);
+        acc[u][7] = fmaf(w[j], b.w, acc[u][7]);
       }
     }
 #pragma unroll
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(kCombThreads)
   }
 }
 
-cudaError_t launch_combine(const __nv_bfloat16* y_perm, const __nv_bfloat16* x,
+cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t s) {

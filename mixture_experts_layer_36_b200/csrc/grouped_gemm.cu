@@ -7,7 +7,7 @@
 // "Expert Parallelism" glossary, fourth paragraph).
 //
 //   GEMM 1 (SWIGLU = true):  h[r, :]      = silu(x_perm[r] Wg[e]) * (x_perm[r] Wu[e])
-//   GEMM 2 (SWIGLU = false): y_perm[r, :] = h[r] Wd[e]
+//   GEMM 2 (SWIGLU = false): y_perm[r, :] = h[r] Wd[e]      (stored fp32)
 // for every row r of bucket e (offsets[e] <= r < offsets[e+1]).
 //
 // Tiling.  A tile is 128 bucket rows x BN accumulator columns.  GEMM 1 puts the
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1,
                         const int32_t* __restrict__ offsets, int E, int K, int n_out,
-                        int max_rows, __nv_bfloat16* __restrict__ out, int32_t* status) {
+                        int max_rows, void* __restrict__ out_raw, int32_t* status) {
   using Cfg = GemmCfg<BN, SWIGLU>;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ GemmShared sh;
@@ -261,8 +261,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int local_row = m * kBM + row_in_tile;
       const bool valid = local_row < sh.row_cnt[e];
-      __nv_bfloat16* orow = out + (size_t)(sh.row_off[e] + local_row) * n_out +
-                            (size_t)n * Cfg::kOutCols;
+      const size_t out_off =
+          (size_t)(sh.row_off[e] + local_row) * n_out + (size_t)n * Cfg::kOutCols;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * BN);
       if (SWIGLU) {
@@ -280,7 +280,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
               pk[i] = pack_bf16x2(silu(g0) * u0, silu(g1) * u1);
             }
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(
+                static_cast<__nv_bfloat16*>(out_raw) + out_off + c * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
               dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
@@ -293,14 +294,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld_32x32b_x32(tbase + c * 32, v);
           tmem_ld_wait();
           if (valid) {
-            uint32_t pk[16];
+            // fp32 rows: the combine rounds to bf16 once, after the weighted sum
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(out_raw) + out_off + c * 32);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         }
       }
@@ -390,7 +388,7 @@ static cudaError_t device_info(DeviceInfo** out) {
 template <int BN, bool SWIGLU>
 static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& b0,
                                const CUtensorMap& b1, const int32_t* offsets, int E, int K,
-                               int n_out, int max_rows, __nv_bfloat16* out, int32_t* status,
+                               int n_out, int max_rows, void* out, int32_t* status,
                                cudaStream_t s) {
   using Cfg = GemmCfg<BN, SWIGLU>;
   DeviceInfo* di = nullptr;
@@ -427,7 +425,7 @@ cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, 
 
 // GEMM 2: y_perm = h Wd
 cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
-                        int max_rows, const __nv_bfloat16* w_down, __nv_bfloat16* y_perm,
+                        int max_rows, const __nv_bfloat16* w_down, float* y_perm,
                         int32_t* status, cudaStream_t s, bool* map_failed) {
   CUtensorMap ta, td;
   *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_weights(&td, w_down, E, f, d));

@@ -41,6 +41,8 @@ def lib():
         _lib.oracle_num_threads.restype = ctypes.c_int
         _lib.oracle_permute.restype = _i64
         _lib.oracle_moe_forward.restype = _i64
+        _lib.oracle_round_bf16.restype = _dbl
+        _lib.oracle_round_bf16.argtypes = [_dbl]
     return _lib
 
 
@@ -104,9 +106,15 @@ def dispatch(x_bits, row_src):
     return out
 
 
-def swiglu_rows(x_rows_bits, wg_bits, wu_bits, wd_bits, want_h=False):
+def round_bf16(v):
+    """Nearest bf16 value (ties to even) of a double, as the oracle rounds h."""
+    return lib().oracle_round_bf16(float(v))
+
+
+def swiglu_rows(x_rows_bits, wg_bits, wu_bits, wd_bits, want_h=False, h_bf16=True):
     """One expert: x_rows [n,d], wg/wu [d,f], wd [f,d] (bf16 bits).  Returns
-    (h [n,f] or None, o [n,d]) in fp64."""
+    (h [n,f] or None, o [n,d]) in fp64.  h_bf16: round h to bf16 before the
+    down projection (the expert GEMMs take bf16 operands)."""
     x_rows_bits = _c(x_rows_bits, np.uint16)
     wg_bits, wu_bits, wd_bits = (_c(a, np.uint16) for a in (wg_bits, wu_bits, wd_bits))
     n, d = x_rows_bits.shape
@@ -114,11 +122,13 @@ def swiglu_rows(x_rows_bits, wg_bits, wu_bits, wd_bits, want_h=False):
     h = np.empty((n, f), np.float64) if want_h else None
     o = np.empty((n, d), np.float64)
     lib().oracle_swiglu_rows(_ptr(x_rows_bits), _i64(n), _i64(d), _i64(f), _ptr(wg_bits),
-                             _ptr(wu_bits), _ptr(wd_bits), _ptr(h), _ptr(o))
+                             _ptr(wu_bits), _ptr(wd_bits), ctypes.c_int(int(h_bf16)), _ptr(h),
+                             _ptr(o))
     return h, o
 
 
-def expert_mlp(x_perm_bits, offsets, w_gate_bits, w_up_bits, w_down_bits, want_h=False):
+def expert_mlp(x_perm_bits, offsets, w_gate_bits, w_up_bits, w_down_bits, want_h=False,
+               h_bf16=True):
     x_perm_bits = _c(x_perm_bits, np.uint16)
     offsets = _c(offsets, np.int32)
     wg, wu, wd = (_c(a, np.uint16) for a in (w_gate_bits, w_up_bits, w_down_bits))
@@ -127,7 +137,8 @@ def expert_mlp(x_perm_bits, offsets, w_gate_bits, w_up_bits, w_down_bits, want_h
     h = np.empty((N, f), np.float64) if want_h else None
     y = np.empty((N, d), np.float64)
     lib().oracle_expert_mlp(_ptr(x_perm_bits), _ptr(offsets), _i64(E), _i64(d), _i64(f),
-                            _ptr(wg), _ptr(wu), _ptr(wd), _ptr(h), _ptr(y))
+                            _ptr(wg), _ptr(wu), _ptr(wd), ctypes.c_int(int(h_bf16)), _ptr(h),
+                            _ptr(y))
     return h, y
 
 
@@ -147,9 +158,11 @@ def combine(y_perm, x_bits, topk_idx, topk_w, slot, offsets):
 
 
 def moe_forward(x_bits, w_router, bias, w_gate_bits, w_up_bits, w_down_bits, k, cf,
-                decision_logits=None):
+                decision_logits=None, h_bf16=True):
     """The whole layer.  Returns a dict with y [T,d] fp64 and the routing
-    intermediates (logits64, topk_idx, topk_w, slot, counts, offsets, n_dropped)."""
+    intermediates (logits64, topk_idx, topk_w, slot, counts, offsets, n_dropped).
+    h_bf16: round h to bf16 before the down projection (default: the expert
+    GEMMs take bf16 operands); False keeps the MLP entirely in fp64."""
     x_bits = _c(x_bits, np.uint16)
     w_router = _c(w_router, np.float32)
     bias = _c(bias, np.float32)
@@ -168,7 +181,8 @@ def moe_forward(x_bits, w_router, bias, w_gate_bits, w_up_bits, w_down_bits, k, 
     }
     n_drop = lib().oracle_moe_forward(
         _ptr(x_bits), _ptr(w_router), _ptr(bias), _ptr(wg), _ptr(wu), _ptr(wd), _i64(T), _i64(d),
-        _i64(E), _i64(k), _i64(f), _dbl(cf), _ptr(decision_logits), _ptr(out["y"]),
+        _i64(E), _i64(k), _i64(f), _dbl(cf), ctypes.c_int(int(h_bf16)), _ptr(decision_logits),
+        _ptr(out["y"]),
         _ptr(out["logits64"]), _ptr(out["topk_idx"]), _ptr(out["topk_w"]), _ptr(out["slot"]),
         _ptr(out["counts"]), _ptr(out["offsets"]))
     out["n_dropped"] = int(n_drop)

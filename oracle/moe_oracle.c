@@ -24,7 +24,10 @@
  *        (inferensys.com glossary, Dropped Tokens entry)
  *   5. per-expert SwiGLU MLP: h = silu(x Wg) * (x Wu), o = h Wd
  *        (neelmishra, section "Tensor parallelism for experts": gate, up and
- *         down projections)
+ *         down projections).  The expert GEMMs take bf16 operands, so h, the
+ *        down projection's input, is rounded to bf16 (nearest, ties to even)
+ *        before o = h Wd when round_h is set; with round_h clear the whole
+ *        MLP stays in fp64.
  *   6. combine: y[t] = sum over kept pairs of w * o, in the token's top-k
  *      order; a token whose every pair was dropped leaves the layer as it came
  *        (neelmishra, section "All-to-all: the distributed transpose": the
@@ -154,12 +157,24 @@ void oracle_dispatch(const uint16_t* x, const int32_t* row_src, int64_t N, int64
         memcpy(x_perm + r * d, x + (int64_t)row_src[r] * d, (size_t)d * sizeof(uint16_t));
 }
 
+/* Round a finite double in the normal bf16 range to the nearest bf16 value
+ * (8 significant bits), ties to even: scale the mantissa to [128, 256) and
+ * round it to an integer in the default round-half-even mode. */
+double oracle_round_bf16(double v) {
+    if (v == 0.0 || !isfinite(v)) return v;
+    int ex;
+    double m = frexp(v, &ex);            /* v = m * 2^ex, 0.5 <= |m| < 1 */
+    double r = nearbyint(ldexp(m, 8));
+    return ldexp(r, ex - 8);
+}
+
 /* Step 5 for n rows that all go to one expert whose weights are wg/wu [d,f]
- * and wd [f,d].  h [n,f] (may be NULL) and o [n,d] in fp64, no intermediate
- * rounding.  silu(z) = z * sigmoid(z) = z / (1 + exp(-z)). */
+ * and wd [f,d].  h [n,f] (may be NULL) and o [n,d] in fp64; h is rounded to
+ * bf16 before the down projection when round_h != 0.
+ * silu(z) = z * sigmoid(z) = z / (1 + exp(-z)). */
 void oracle_swiglu_rows(const uint16_t* x_rows, int64_t n, int64_t d, int64_t f,
                         const uint16_t* wg, const uint16_t* wu, const uint16_t* wd,
-                        double* h_out, double* o_out) {
+                        int round_h, double* h_out, double* o_out) {
     #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < n; ++r) {
         double* g = (double*)calloc((size_t)f, sizeof(double));
@@ -178,6 +193,7 @@ void oracle_swiglu_rows(const uint16_t* x_rows, int64_t n, int64_t d, int64_t f,
         for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
         for (int64_t j = 0; j < f; ++j) {
             double hj = g[j] / (1.0 + exp(-g[j])) * u[j];
+            if (round_h) hj = oracle_round_bf16(hj);
             if (h_out) h_out[r * f + j] = hj;
             const uint16_t* wdj = wd + j * d;
             for (int64_t c = 0; c < d; ++c) o[c] += hj * bf16_bits_to_f64(wdj[c]);
@@ -190,12 +206,12 @@ void oracle_swiglu_rows(const uint16_t* x_rows, int64_t n, int64_t d, int64_t f,
 /* Step 5 over every bucket: rows offsets[e] .. offsets[e+1]-1 use expert e. */
 void oracle_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, int64_t E, int64_t d,
                        int64_t f, const uint16_t* w_gate, const uint16_t* w_up,
-                       const uint16_t* w_down, double* h, double* y_perm) {
+                       const uint16_t* w_down, int round_h, double* h, double* y_perm) {
     for (int64_t e = 0; e < E; ++e) {
         int64_t r0 = offsets[e], n = offsets[e + 1] - offsets[e];
         if (n == 0) continue;
         oracle_swiglu_rows(x_perm + r0 * d, n, d, f, w_gate + e * d * f, w_up + e * d * f,
-                           w_down + e * f * d, h ? h + r0 * f : NULL, y_perm + r0 * d);
+                           w_down + e * f * d, round_h, h ? h + r0 * f : NULL, y_perm + r0 * d);
     }
 }
 
@@ -222,7 +238,7 @@ void oracle_combine(const double* y_perm, const uint16_t* x, const int32_t* topk
     }
 }
 
-/* Steps 1-6 end to end.  decision_logits (fp32 [T,E]) may be given, in which
+/* Steps 1-6 end to end (round_h as in step 5).  decision_logits (fp32 [T,E]) may be given, in which
  * case the routing decision is taken on those values; when NULL the oracle's
  * own fp64 logits, rounded to fp32, are used.  Optional outputs (NULL to skip):
  * logits64 [T,E], topk_idx [T,k], topk_w [T,k], slot [T,k], counts [E],
@@ -230,7 +246,8 @@ void oracle_combine(const double* y_perm, const uint16_t* x, const int32_t* topk
 int64_t oracle_moe_forward(const uint16_t* x, const float* w_router, const float* bias,
                            const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
                            int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf,
-                           const float* decision_logits, double* y, double* logits64_out,
+                           int round_h, const float* decision_logits, double* y,
+                           double* logits64_out,
                            int32_t* topk_idx_out, double* topk_w_out, int32_t* slot_out,
                            int32_t* counts_out, int32_t* offsets_out) {
     double* l64 = (double*)malloc((size_t)(T * E) * sizeof(double));
@@ -255,7 +272,7 @@ int64_t oracle_moe_forward(const uint16_t* x, const float* w_router, const float
     uint16_t* x_perm = (uint16_t*)malloc((size_t)(N * d + 1) * sizeof(uint16_t));
     double* y_perm = (double*)malloc((size_t)(N * d + 1) * sizeof(double));
     oracle_dispatch(x, row_src, N, d, x_perm);
-    oracle_expert_mlp(x_perm, offsets, E, d, f, w_gate, w_up, w_down, NULL, y_perm);
+    oracle_expert_mlp(x_perm, offsets, E, d, f, w_gate, w_up, w_down, round_h, NULL, y_perm);
     oracle_combine(y_perm, x, idx, w, slot, offsets, T, d, k, y);
 
     if (logits64_out) memcpy(logits64_out, l64, (size_t)(T * E) * sizeof(double));

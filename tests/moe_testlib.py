@@ -6,7 +6,14 @@ Tolerances (written once, used everywhere):
     row_src, n_dropped) and pure copies (x_perm, passthrough rows): bit-exact;
   * fp32 logits: |gpu - ref| <= 1e-4 * max(|ref|, rms(ref)) elementwise;
   * fp32 gate weights: |gpu - ref| <= 1e-6 absolute;
-  * bf16 outputs (h, y_perm, y): max |gpu - ref| <= 2e-2 * rms(ref).
+  * the layer output y (bf16) and the down GEMM's fp32 rows y_perm:
+    max |gpu - ref| <= 2e-2 * rms(ref);
+  * the bf16 intermediate h = silu(g) * u: elementwise
+    |gpu - ref| <= 2^-8 * |ref| + 1e-3 * rms(ref).  h is heavy-tailed (a
+    product of two near-Gaussian values), so one bf16 rounding of its largest
+    elements alone exceeds 2e-2 * rms; the bound is one rounding to bf16
+    (at most 2^-9 relative, doubled for margin) plus an absolute term for the
+    fp32 accumulation order and the exponential in silu.
 """
 import numpy as np
 import torch
@@ -49,6 +56,24 @@ def assert_bf16_close(gpu, ref64, what):
     rms = np.sqrt(np.mean(ref ** 2))
     err = np.max(np.abs(g - ref))
     assert err <= BF16_RMS_TOL * rms, f"{what}: max|err| {err:.4e} > {BF16_RMS_TOL} * rms {rms:.4e}"
+
+
+H_REL_TOL = 2.0 ** -8
+H_ABS_RMS_TOL = 1e-3
+
+
+def assert_bf16_rounding_close(gpu, ref64, what):
+    ref = np.asarray(ref64, np.float64)
+    g = np.asarray(gpu, np.float64)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    if ref.size == 0:
+        return
+    rms = np.sqrt(np.mean(ref ** 2))
+    bound = H_REL_TOL * np.abs(ref) + H_ABS_RMS_TOL * rms
+    excess = np.abs(g - ref) - bound
+    i = np.unravel_index(np.argmax(excess), excess.shape)
+    assert excess[i] <= 0, (f"{what}: at {i} gpu {g[i]:.6g} ref {ref[i]:.6g} "
+                            f"exceeds the bf16-rounding bound by {excess[i]:.3e}")
 
 
 def small(name, T, d, E, k, f, cf, seed, zipf_s=None):

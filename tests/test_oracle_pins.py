@@ -257,31 +257,68 @@ def test_swiglu_closed_form_unit_rows():
     wu = bf16_round(r.standard_normal((d, f)))
     wd = bf16_round(np.eye(f))
     x = bf16_round(np.eye(d))
-    h, o = oracle.swiglu_rows(x, wg, wu, wd, want_h=True)
+    h, o = oracle.swiglu_rows(x, wg, wu, wd, want_h=True, h_bf16=False)
     g, u = oracle.bits_to_f64(wg), oracle.bits_to_f64(wu)
     ref = g * expit(g) * u
     np.testing.assert_allclose(h, ref, rtol=1e-14, atol=1e-300)
     np.testing.assert_allclose(o, ref, rtol=1e-14, atol=1e-300)
+    # with bf16 h (the GEMM operand precision) both outputs are the rounded value
+    hr, orr = oracle.swiglu_rows(x, wg, wu, wd, want_h=True, h_bf16=True)
+    np.testing.assert_array_equal(hr, np_round_bf16(h))
+    np.testing.assert_array_equal(orr, np_round_bf16(h))
 
 
-def np_swiglu(x64, wg64, wu64, wd64):
+def np_round_bf16(a):
+    """Nearest bf16 of fp64 values by bit manipulation (keep 7 of the 52
+    stored mantissa bits, ties to even) — a different method from the
+    oracle's frexp / nearbyint rounding."""
+    a = np.ascontiguousarray(a, np.float64)
+    b = a.view(np.uint64)
+    drop = np.uint64(45)
+    lsb = (b >> drop) & np.uint64(1)
+    b = (b + (np.uint64(1) << np.uint64(44)) - np.uint64(1) + lsb) & ~((np.uint64(1) << drop)
+                                                                     - np.uint64(1))
+    return b.view(np.float64)
+
+
+def np_swiglu(x64, wg64, wu64, wd64, h_bf16=False):
     g = x64 @ wg64
     u = x64 @ wu64
-    return (g * expit(g) * u) @ wd64
+    h = g * expit(g) * u
+    if h_bf16:
+        h = np_round_bf16(h)
+    return h @ wd64
+
+
+def test_round_bf16_matches_library_conversion():
+    import torch
+    r = np.random.default_rng(31)
+    v = (r.standard_normal(4000) * np.exp(r.uniform(-20, 20, 4000))).astype(np.float32)
+    # exact ties: bf16 values plus half an ulp
+    base = torch.from_numpy(v[:500]).to(torch.bfloat16).float().numpy()
+    half_ulp = np.ldexp(np.ones_like(base), np.frexp(base)[1] - 9)
+    ties = (base + np.sign(base) * half_ulp).astype(np.float32)
+    v = np.concatenate([v, ties, -ties, np.float32([1.0, -1.0, 3.0, 1e-3])])
+    want = torch.from_numpy(v).to(torch.bfloat16).double().numpy()
+    got = np.array([oracle.round_bf16(float(a)) for a in v])
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal(np_round_bf16(v.astype(np.float64)), want)
 
 
 def test_single_expert_is_dense_swiglu_mlp():
     # E = 1, k = 1, dropless: the layer is one dense SwiGLU MLP (gate weight 1)
     T, d, f = 12, 32, 48
     x, wr, b, wg, wu, wd = rand_layer(T, d, 1, f, seed=12)
-    out = oracle.moe_forward(x, wr, b, wg, wu, wd, k=1, cf=0.0)
-    ref = np_swiglu(oracle.bits_to_f64(x), *(oracle.bits_to_f64(a[0]) for a in (wg, wu, wd)))
-    np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+    for h_bf16 in (False, True):
+        out = oracle.moe_forward(x, wr, b, wg, wu, wd, k=1, cf=0.0, h_bf16=h_bf16)
+        ref = np_swiglu(oracle.bits_to_f64(x), *(oracle.bits_to_f64(a[0]) for a in (wg, wu, wd)),
+                        h_bf16=h_bf16)
+        np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
     assert out["topk_idx"].ravel().tolist() == [0] * T
     np.testing.assert_array_equal(out["topk_w"], 1.0)
 
 
-def dense_bruteforce(x, wr, b, wg, wu, wd, k, cf):
+def dense_bruteforce(x, wr, b, wg, wu, wd, k, cf, h_bf16):
     """Every token through every expert, then masked to its kept top-k pairs.
     Routing by full sort, slots by the O(T^2) count."""
     T = x.shape[0]
@@ -294,8 +331,8 @@ def dense_bruteforce(x, wr, b, wg, wu, wd, k, cf):
     w = softmax(sel, axis=1)
     C = T if cf == 0 else math.ceil(cf * k * T / E)
     slot, _, _, _ = brute_permute(idx, E, C)
-    all_out = np.stack([np_swiglu(x64, *(oracle.bits_to_f64(a[e]) for a in (wg, wu, wd)))
-                        for e in range(E)])  # [E, T, d]
+    all_out = np.stack([np_swiglu(x64, *(oracle.bits_to_f64(a[e]) for a in (wg, wu, wd)),
+                                  h_bf16=h_bf16) for e in range(E)])  # [E, T, d]
     y = np.zeros_like(x64)
     for t in range(T):
         kept = [j for j in range(k) if slot[t, j] >= 0]
@@ -306,16 +343,17 @@ def dense_bruteforce(x, wr, b, wg, wu, wd, k, cf):
     return y, idx, w, slot
 
 
+@pytest.mark.parametrize("h_bf16", [False, True])
 @pytest.mark.parametrize("T,d,E,k,f,cf,bias", [
     (64, 32, 8, 2, 48, 1.25, False),
     (48, 16, 6, 3, 32, 0.5, True),     # heavy dropping, some tokens fully dropped
     (30, 24, 4, 2, 16, 0.0, False),    # dropless
     (20, 16, 5, 5, 8, 0.0, True),      # k = E
 ])
-def test_layer_matches_dense_bruteforce(T, d, E, k, f, cf, bias):
+def test_layer_matches_dense_bruteforce(T, d, E, k, f, cf, bias, h_bf16):
     x, wr, b, wg, wu, wd = rand_layer(T, d, E, f, seed=T * d + E, bias=bias)
-    out = oracle.moe_forward(x, wr, b, wg, wu, wd, k=k, cf=cf)
-    y, idx, w, slot = dense_bruteforce(x, wr, b, wg, wu, wd, k, cf)
+    out = oracle.moe_forward(x, wr, b, wg, wu, wd, k=k, cf=cf, h_bf16=h_bf16)
+    y, idx, w, slot = dense_bruteforce(x, wr, b, wg, wu, wd, k, cf, h_bf16)
     np.testing.assert_array_equal(out["topk_idx"], idx)
     np.testing.assert_array_equal(out["slot"], slot)
     np.testing.assert_allclose(out["topk_w"], w, rtol=1e-13, atol=1e-15)
@@ -326,7 +364,7 @@ def test_layer_matches_dense_bruteforce(T, d, E, k, f, cf, bias):
 def test_k_equals_E_dropless_is_softmax_mixture():
     T, d, E, f = 10, 16, 4, 24
     x, wr, b, wg, wu, wd = rand_layer(T, d, E, f, seed=99, bias=True)
-    out = oracle.moe_forward(x, wr, b, wg, wu, wd, k=E, cf=0.0)
+    out = oracle.moe_forward(x, wr, b, wg, wu, wd, k=E, cf=0.0, h_bf16=False)
     x64 = oracle.bits_to_f64(x)
     l = (x64 @ wr.astype(np.float64) + b).astype(np.float32).astype(np.float64)
     p = softmax(l, axis=1)

@@ -8,12 +8,13 @@ Tolerances (written once, used everywhere):
   * fp32 gate weights: |gpu - ref| <= 1e-6 absolute;
   * the layer output y (bf16) and the down GEMM's fp32 rows y_perm:
     max |gpu - ref| <= 2e-2 * rms(ref);
-  * the bf16 intermediate h = silu(g) * u: elementwise
-    |gpu - ref| <= 2^-8 * |ref| + 1e-3 * rms(ref).  h is heavy-tailed (a
-    product of two near-Gaussian values), so one bf16 rounding of its largest
-    elements alone exceeds 2e-2 * rms; the bound is one rounding to bf16
-    (at most 2^-9 relative, doubled for margin) plus an absolute term for the
-    fp32 accumulation order and the exponential in silu.
+  * the bf16 intermediate h = silu(g) * u, against the oracle's h rounded to
+    bf16 as well: elementwise |gpu - ref| <= 2^-7 * |ref| + 1e-3 * rms(ref).
+    Both sides round a value to bf16; when the fp32 (GPU) and fp64 (oracle)
+    values straddle a rounding boundary the results differ by one bf16 ulp,
+    which is at most 2^-7 of the value; the absolute term covers the fp32
+    accumulation order and the exponential in silu near zero.  (h is
+    heavy-tailed, so a max-relative-to-rms bound would not describe it.)
 """
 import numpy as np
 import torch
@@ -58,7 +59,7 @@ def assert_bf16_close(gpu, ref64, what):
     assert err <= BF16_RMS_TOL * rms, f"{what}: max|err| {err:.4e} > {BF16_RMS_TOL} * rms {rms:.4e}"
 
 
-H_REL_TOL = 2.0 ** -8
+H_REL_TOL = 2.0 ** -7
 H_ABS_RMS_TOL = 1e-3
 
 

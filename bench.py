@@ -15,7 +15,6 @@ Prints one JSON line on rank 0.
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -102,6 +101,22 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ----------------------------------------------------------------- replicas
+
+def rank_token_seed(cfg, rank):
+    """Each replica draws its own token batch; weights share the workload seed."""
+    return cfg.seed * 1000 + rank
+
+
+def max_over_ranks(value, device, dist):
+    """The slowest rank's time (every rank takes the same collective step)."""
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist:
+        import torch.distributed as td
+        td.all_reduce(t, op=td.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------- the GPU arm
 
 class Layer:
@@ -169,7 +184,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     dist = world > 1
     if dist:
         import torch.distributed as td
-    layer = Layer(cfg, dev, token_seed=cfg.seed * 1000 + rank)
+    layer = Layer(cfg, dev, token_seed=rank_token_seed(cfg, rank))
     stream = torch.cuda.current_stream()
 
     K = args.steps
@@ -191,11 +206,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
         torch.cuda.synchronize()
     if dist:
         td.barrier()
-    elapsed_ms = start.elapsed_time(stop)
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if dist:
-        td.all_reduce(t, op=td.ReduceOp.MAX)
-    elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), dev, dist)
 
     names = ["route", "permute", "gate_up", "down", "combine"]
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
@@ -225,11 +236,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
         y_host.copy_(y_dev, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if dist:
-        td.all_reduce(t, op=td.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, dist)
     return {"elapsed_ms": elapsed_ms, "stage_ms": stage_ms, "status": status, "N": N,
             "n_dropped": n_drop, "clocks": clk.summary(), "e2e_ms": e2e_ms,
             "h2d": x_host.numel() * 2, "d2h": y_host.numel() * 2, "layer": layer}
@@ -273,10 +280,11 @@ def host_weights(w):
             "w_down": oracle.bf16_bits(w["w_down"])}
 
 
-def sample_tokens(cfg):
-    """Tokens per oracle sample: about 10-30 s of CPU work on a few cores."""
-    per_token_flop = 6.0 * cfg.k * cfg.d * cfg.f + 2.0 * cfg.d * cfg.E
-    return int(max(2, min(cfg.T, round(2.0e10 / per_token_flop))))
+def calibrated_tokens(cfg, wh, xb, seconds):
+    """Tokens whose oracle pass takes about `seconds` on this host: time a
+    2-token pass, scale, clamp to [2, T]."""
+    t2, _ = oracle_sample(cfg, wh, xb, 2)
+    return int(max(2, min(cfg.T, round(2 * seconds / max(t2, 1e-6)))))
 
 
 # ----------------------------------------------------------------- main
@@ -289,6 +297,9 @@ def main():
     ap.add_argument("--config", default="mixtral")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run W + K layer steps only (no timing, e2e or oracle): a short, "
+                         "fixed launch sequence for ncu")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -300,6 +311,15 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args, cfg, rank, world)
+    if args.profile:
+        layer = Layer(cfg, torch.device("cuda", local_rank), token_seed=rank_token_seed(cfg, 0))
+        for _ in range(args.warmup + args.steps):
+            layer.step()
+        torch.cuda.synchronize()
+        assert int(layer.status.item()) == 0
+        print(json.dumps({"profile_run": cfg.name, "launches": KERNELS_PER_STEP *
+                          (args.warmup + args.steps)}))
+        return
 
     if world > 1:
         import datetime
@@ -364,10 +384,11 @@ def main():
         "gpu_launches": KERNELS_PER_STEP * K,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n = sample_tokens(cfg)
         wh = host_weights(r["layer"].w)
         import oracle
-        secs, cores = oracle_sample(cfg, wh, oracle.bf16_bits(r["layer"].x), n)
+        xb = oracle.bf16_bits(r["layer"].x)
+        n = calibrated_tokens(cfg, wh, xb, seconds=15.0)
+        secs, cores = oracle_sample(cfg, wh, xb, n)
         out["cpu_baseline"] = {"value": round(n / secs, 3), "unit": "tokens/s", "cores": cores,
                                "kind": "oracle",
                                "sample": f"first {n} tokens of the batch through the whole "
@@ -385,14 +406,15 @@ def reference_arm(args, cfg, rank, world):
     if rank != 0:
         return
     import oracle
-    n = max(2, sample_tokens(cfg) // 8)
     # weights drawn on the CPU with the same recipe (one step is a bounded sample)
     w = synth.make_weights(cfg, "cpu")
     x = synth.make_tokens(cfg, "cpu")
     wh = host_weights(w)
     xb = oracle.bf16_bits(x)
-    for _ in range(min(args.warmup, 1)):
-        oracle_sample(cfg, wh, xb, n)
+    # each step is a sample sized so that warm-up + steps take about 90 s
+    per_step = min(2.0, 90.0 / (args.steps + 1))
+    n = calibrated_tokens(cfg, wh, xb, per_step)
+    oracle_sample(cfg, wh, xb, n)     # one untimed warm-up pass
     t = 0.0
     for _ in range(args.steps):
         s, cores = oracle_sample(cfg, wh, xb, n)

@@ -36,7 +36,14 @@ SKEWED = MoEConfig("skewed", T=16384, d=2048, E=64, k=6, f=1408, cf=1.0, seed=3,
 DECODE = MoEConfig("decode", T=256, d=7168, E=256, k=8, f=2048, cf=0.0, seed=4)
 DECODE_T = (16, 64, 256)
 
-ALL = {c.name: c for c in (TINY, MIXTRAL, FINE, SKEWED, DECODE)}
+# Profiling slice of the Mixtral-shaped layer: 2 of its experts with the same
+# rows per expert (T*k/E = 1024), so a full ncu capture of the expert GEMMs
+# holds under 1 GB on the device while the per-expert GEMM shape is unchanged.
+MIXTRAL_SLICE = MoEConfig("mixtral_slice", T=1024, d=4096, E=2, k=2, f=14336, cf=0.0, seed=1)
+# Same idea for the fine-grained layer: 16 of its 256 experts, 320 rows each.
+FINE_SLICE = MoEConfig("fine_slice", T=512, d=7168, E=16, k=8, f=2048, cf=1.25, seed=2)
+
+ALL = {c.name: c for c in (TINY, MIXTRAL, FINE, SKEWED, DECODE, MIXTRAL_SLICE, FINE_SLICE)}
 
 
 def by_name(name: str) -> MoEConfig:

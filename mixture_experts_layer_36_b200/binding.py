@@ -27,7 +27,7 @@ WS_FIELDS = ["status", "logits", "topk_idx", "topk_w", "slot", "counts", "offset
 
 EXPORTED = ["moe_status_string", "moe_version", "moe_capacity", "moe_max_rows",
             "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
-            "moe_route", "moe_permute", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
+            "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
             "moe_combine", "moe_layer_forward"]
 
 
@@ -53,6 +53,7 @@ def _load():
         "moe_workspace_field_offset": (i64, [ctypes.c_int, i64, i64, i64, i64, i64, dbl]),
         "moe_route": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p]),
         "moe_permute": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p, sz, p]),
+        "moe_permute_noalloc": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p]),
         "moe_expert_gate_up": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p]),
         "moe_expert_down": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p]),
         "moe_expert_mlp": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p, p, p]),
@@ -184,6 +185,21 @@ def moe_permute(x, topk_idx, E, cf, out=None, ws=None, stream=None):
         _ptr(x), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]),
         _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["x_perm"]),
         _ptr(out["n_dropped"]), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def moe_permute_noalloc(x, topk_idx, E, cf, out, stream=None):
+    """moe_permute for callers that cannot provide scratch memory: the library
+    uses a fixed array of its own (shared by every call; see include/moe.h).
+    `out` holds the caller's output tensors, as returned by moe_permute."""
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    _want(x, "x", torch.bfloat16)
+    _want(topk_idx, "topk_idx", torch.int32, (T, k))
+    _check("moe_permute_noalloc", _lib.moe_permute_noalloc(
+        _ptr(x), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]),
+        _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["x_perm"]),
+        _ptr(out["n_dropped"]), _stream(stream)))
     return out
 
 

@@ -30,7 +30,7 @@ from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
 
 METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 7     # router 1, permute 3, gate/up GEMM 1, down GEMM 1, combine 1
+KERNELS_PER_STEP = 9     # router 3, permute 3, gate/up GEMM 1, down GEMM 1, combine 1
 
 
 def peaks():
@@ -142,6 +142,7 @@ class Layer:
                      "x_perm": z(self.rows, d, dt=torch.bfloat16),
                      "n_dropped": z(1, dt=torch.int32)}
         self.pws = z(max(moe.moe_permute_workspace_size(T, E, k), 16), dt=torch.uint8)
+        self.rws = z(max(moe.moe_route_workspace_size(T, d, E, k), 16), dt=torch.uint8)
         self.h = z(self.rows, f, dt=torch.bfloat16)
         self.y_perm = z(self.rows, d, dt=torch.float32)
         self.y = z(T, d, dt=torch.bfloat16)
@@ -153,7 +154,8 @@ class Layer:
         m, w, c = self.moe, self.w, self.cfg
         if ev:
             ev[0].record()
-        m.moe_route(self.x, w["w_router"], w["bias"], c.k, self.logits, self.idx, self.tw)
+        m.moe_route(self.x, w["w_router"], w["bias"], c.k, self.logits, self.idx, self.tw,
+                    ws=self.rws, dev_status=self.status)
         if ev:
             ev[1].record()
         m.moe_permute(self.x, self.idx, c.E, c.cf, out=self.perm, ws=self.pws)

@@ -70,6 +70,10 @@ int64_t moe_capacity(int64_t T, int64_t E, int64_t k, double cf);
  * kept.  Returns -1 on bad args. */
 int64_t moe_max_rows(int64_t T, int64_t E, int64_t k, double cf);
 
+/* Device scratch bytes moe_route needs: the two-term bf16 split of the router
+ * weight (2*d*round_up(E,64) bf16) and the split-K partial logits. */
+size_t moe_route_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k);
+
 /* Device scratch bytes moe_permute needs (per-chunk bucket histograms). */
 size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k);
 
@@ -93,7 +97,8 @@ typedef enum {
   MOE_WS_X_PERM = 10,    /* bf16 [max_rows, d] */
   MOE_WS_H = 11,         /* bf16 [max_rows, f] */
   MOE_WS_Y_PERM = 12,    /* f32  [max_rows, d] */
-  MOE_WS_NUM_FIELDS = 13
+  MOE_WS_ROUTE = 13,     /* moe_route scratch */
+  MOE_WS_NUM_FIELDS = 14
 } moe_ws_field;
 
 /* Byte offset of a field inside the moe_layer_forward workspace (each field
@@ -113,10 +118,15 @@ int64_t moe_workspace_field_offset(int field, int64_t T, int64_t d, int64_t E, i
  *   topk_idx i32  [T,k]     out: the k largest logits, descending; equal
  *                           logits rank the lower expert index first
  *   topk_w   f32  [T,k]     out: exp(l_j - l_max) / sum over the k selected
- * The selection is taken on the fp32 values written to `logits`. */
+ *   ws, ws_bytes            device scratch, >= moe_route_workspace_size
+ *   dev_status              nullable device status word (see conventions)
+ * The selection is taken on the fp32 values written to `logits`.  The logits
+ * are computed on the tensor cores from a two-term bf16 split of w_router
+ * (hi = bf16(w), lo = bf16(w - hi); x is bf16 already), with fp32
+ * accumulation; the split's residual is below 2^-18 |w| per weight. */
 int moe_route(const void* x, const float* w_router, const float* bias, int64_t T, int64_t d,
-              int64_t E, int64_t k, float* logits, int32_t* topk_idx, float* topk_w,
-              void* stream);
+              int64_t E, int64_t k, float* logits, int32_t* topk_idx, float* topk_w, void* ws,
+              size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* Capacity-limited permutation into per-expert buckets (pairs are bucketed by
  * expert, overflow beyond the capacity is dropped: inferensys.com glossary,

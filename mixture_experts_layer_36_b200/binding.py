@@ -23,10 +23,10 @@ DEV_ERR_BAD_OFFSETS = 2
 
 # workspace fields of moe_layer_forward (enum moe_ws_field)
 WS_FIELDS = ["status", "logits", "topk_idx", "topk_w", "slot", "counts", "offsets", "n_dropped",
-             "row_src", "permute", "x_perm", "h", "y_perm"]
+             "row_src", "permute", "x_perm", "h", "y_perm", "route"]
 
 EXPORTED = ["moe_status_string", "moe_version", "moe_capacity", "moe_max_rows",
-            "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
+            "moe_route_workspace_size", "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
             "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
             "moe_combine", "moe_layer_forward"]
 
@@ -48,10 +48,11 @@ def _load():
         "moe_version": (ctypes.c_int, []),
         "moe_capacity": (i64, [i64, i64, i64, dbl]),
         "moe_max_rows": (i64, [i64, i64, i64, dbl]),
+        "moe_route_workspace_size": (sz, [i64, i64, i64, i64]),
         "moe_permute_workspace_size": (sz, [i64, i64, i64]),
         "moe_workspace_size": (sz, [i64, i64, i64, i64, i64, dbl]),
         "moe_workspace_field_offset": (i64, [ctypes.c_int, i64, i64, i64, i64, i64, dbl]),
-        "moe_route": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p]),
+        "moe_route": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, sz, p, p]),
         "moe_permute": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p, sz, p]),
         "moe_permute_noalloc": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p]),
         "moe_expert_gate_up": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p]),
@@ -114,6 +115,10 @@ def moe_max_rows(T, E, k, cf):
     return int(_lib.moe_max_rows(T, E, k, float(cf)))
 
 
+def moe_route_workspace_size(T, d, E, k):
+    return int(_lib.moe_route_workspace_size(T, d, E, k))
+
+
 def moe_permute_workspace_size(T, E, k):
     return int(_lib.moe_permute_workspace_size(T, E, k))
 
@@ -138,7 +143,8 @@ def moe_status_string(status):
 
 # ----------------------------------------------------------------- stages
 
-def moe_route(x, w_router, bias, k, logits=None, topk_idx=None, topk_w=None, stream=None):
+def moe_route(x, w_router, bias, k, logits=None, topk_idx=None, topk_w=None, ws=None,
+              dev_status=None, stream=None):
     """Router + top-k gating.  Returns (logits f32 [T,E], topk_idx i32 [T,k], topk_w f32 [T,k])."""
     T, d = x.shape
     E = w_router.shape[1]
@@ -153,9 +159,13 @@ def moe_route(x, w_router, bias, k, logits=None, topk_idx=None, topk_w=None, str
     _want(logits, "logits", torch.float32, (T, E))
     _want(topk_idx, "topk_idx", torch.int32, (T, k))
     _want(topk_w, "topk_w", torch.float32, (T, k))
+    if ws is None:
+        ws = torch.empty(max(moe_route_workspace_size(T, d, E, k), 16), dtype=torch.uint8,
+                         device=dev)
+    _want(ws, "ws", torch.uint8)
     _check("moe_route", _lib.moe_route(_ptr(x), _ptr(w_router), _ptr(bias), T, d, E, k,
-                                       _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
-                                       _stream(stream)))
+                                       _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
+                                       ws.numel(), _ptr(dev_status), _stream(stream)))
     return logits, topk_idx, topk_w
 
 

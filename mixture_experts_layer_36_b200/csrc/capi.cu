@@ -8,7 +8,8 @@
 namespace moe {
 cudaError_t launch_route(const __nv_bfloat16* x, const float* wr, const float* bias, int T,
                          int d, int E, int k, float* logits, int32_t* idx, float* w,
-                         cudaStream_t s);
+                         void* scratch, int32_t* status, cudaStream_t s, bool* map_failed);
+size_t route_scratch_bytes(int64_t T, int64_t d, int64_t E);
 size_t permute_scratch_bytes(int64_t T, int64_t E);
 cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d, int E,
                            int k, int64_t C, int32_t* counts, int32_t* offsets, int32_t* slot,
@@ -78,6 +79,7 @@ bool field_sizes(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double c
   out[MOE_WS_X_PERM] = size_t(rows * d) * 2;
   out[MOE_WS_H] = size_t(rows * f) * 2;
   out[MOE_WS_Y_PERM] = size_t(rows * d) * sizeof(float);
+  out[MOE_WS_ROUTE] = moe_route_workspace_size(T, d, E, k);
   return true;
 }
 
@@ -117,6 +119,13 @@ int64_t moe_max_rows(int64_t T, int64_t E, int64_t k, double cf) {
   return cap_rows < pairs ? cap_rows : pairs;
 }
 
+size_t moe_route_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k) {
+  (void)k;
+  if (T < 0 || d < 1 || E < 1 || E > kMaxE) return 0;
+  if (T == 0) return 0;
+  return moe::route_scratch_bytes(T, d, E);
+}
+
 size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k) {
   (void)k;
   if (T < 0 || E < 1) return 0;
@@ -142,17 +151,21 @@ size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
 }
 
 int moe_route(const void* x, const float* w_router, const float* bias, int64_t T, int64_t d,
-              int64_t E, int64_t k, float* logits, int32_t* topk_idx, float* topk_w,
-              void* stream) {
+              int64_t E, int64_t k, float* logits, int32_t* topk_idx, float* topk_w, void* ws,
+              size_t ws_bytes, int32_t* dev_status, void* stream) {
   int st = check_routing_shape(T, E, k);
   if (st != MOE_OK) return st;
   if ((st = check_width(d)) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
-  if (!x || !w_router || !logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_route(static_cast<const __nv_bfloat16*>(x), w_router, bias, (int)T,
-                                  (int)d, (int)E, (int)k, logits, topk_idx, topk_w,
-                                  as_stream(stream)));
+  if (!x || !w_router || !logits || !topk_idx || !topk_w || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_route_workspace_size(T, d, E, k)) return MOE_ERR_WORKSPACE;
+  bool map_failed = false;
+  cudaError_t err = launch_route(static_cast<const __nv_bfloat16*>(x), w_router, bias, (int)T,
+                                 (int)d, (int)E, (int)k, logits, topk_idx, topk_w, ws,
+                                 dev_status, as_stream(stream), &map_failed);
+  if (map_failed) return MOE_ERR_CUDA;
+  return cuda_status(err);
 }
 
 int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
@@ -275,11 +288,13 @@ int moe_layer_forward(const void* x, const float* w_router, const float* bias, c
   void* x_perm = field(MOE_WS_X_PERM);
   void* h = field(MOE_WS_H);
   float* y_perm = reinterpret_cast<float*>(field(MOE_WS_Y_PERM));
+  void* rscratch = field(MOE_WS_ROUTE);
   const int64_t max_rows = moe_max_rows(T, E, k, cf);
   cudaStream_t s = as_stream(stream);
 
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, stream)) != MOE_OK)
+  if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, rscratch,
+                      moe_route_workspace_size(T, d, E, k), status, stream)) != MOE_OK)
     return st;
   if ((st = moe_permute(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src, x_perm,
                         n_dropped, pscratch, moe_permute_workspace_size(T, E, k), stream)) !=

@@ -33,6 +33,7 @@
 // producer waits for its copies in flight, the MMA issuer waits for its MMAs,
 // and TMEM is freed before the CTA exits.
 #include "common.cuh"
+#include "host_util.cuh"
 
 namespace moe {
 
@@ -317,73 +318,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 2-D bf16 [outer, inner] row-major, box (64 inner, box_outer), 128-B swizzle.
-static bool map_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                     uint32_t box_outer) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-// 3-D bf16 weights [E, K, N] (N contiguous), box (64 N, 64 K, 1), 128-B swizzle.
-static bool map_weights(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {N, K, E};
-  cuuint64_t strides[2] = {N * 2, K * N * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)kBK, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-struct DeviceInfo {
-  int sms = 0;
-  bool attr_set[4] = {false, false, false, false};
-};
-static DeviceInfo g_dev[64];
-
-static cudaError_t device_info(DeviceInfo** out) {
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  DeviceInfo& di = g_dev[dev];
-  if (di.sms == 0) {
-    err = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
-    if (err != cudaSuccess) return err;
-  }
-  *out = &di;
-  return cudaSuccess;
-}
 
 template <int BN, bool SWIGLU>
 static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& b0,

@@ -1,185 +1,429 @@
-// Router logits and top-k softmax gating in one kernel.
+// Router logits and top-k softmax gating.
 //
 // The router is a linear layer with one output score per expert; top-k gating
 // keeps the k best-scoring experts and their scores become the mixing weights
 // (inferensys.com "Expert Parallelism" glossary, gating-network and Top-k
 // Gating entries; klaylearn.com glossary, third paragraph).
 //
-// logits = x (bf16, widened exactly) @ Wr (fp32) + bias, fp32 FMA on the CUDA
-// cores.  A CTA owns BT tokens and all (padded) EP experts; K is walked in
-// chunks of KC with the x chunk (transposed) and the Wr chunk staged in shared
-// memory; each thread keeps a TPT x EPT register tile.  The logits tile is then
-// parked in shared memory and one warp per token runs k rounds of a warp-wide
-// arg-max (value descending, expert index ascending on equal values).
+// logits = x Wr + bias is a dense contraction (T x d by d x E), so it runs on
+// the tensor cores.  x is bf16 already; the fp32 router weight is split into
+// two bf16 terms, Wr = hi + lo + r with hi = bf16(Wr), lo = bf16(Wr - hi) and
+// |r| <= 2^-18 |Wr|, so x Wr = x hi + x lo up to that residual, with exact
+// bf16 products and fp32 accumulation.  Three launches:
+//   1. split:  Wr (fp32 [d,E]) -> W2 (bf16 [2d, Ep]), 64-row blocks of hi and
+//              lo interleaved (hi block j at rows 128j.., lo block j at
+//              rows 128j+64..), so the two k-blocks that share an x tile run
+//              back to back; Ep = E rounded up to 64, padding zero;
+//   2. GEMM:   persistent tcgen05 kernel over (row tile of 128 tokens, K split
+//              s); each tile accumulates its k-blocks of x W2 in TMEM and
+//              writes fp32 partial logits [S][T][E] (K is split so that small
+//              batches still occupy every SM);
+//   3. top-k:  per token, the S partials are summed in a fixed order, the bias
+//              added, the fp32 logits written, and one warp runs k rounds of
+//              a warp-wide arg-max (value descending, lower expert index on
+//              equal values) on exactly those values; weights are the softmax
+//              over the k selected logits.
 #include "common.cuh"
+#include "host_util.cuh"
 
 namespace moe {
 
-constexpr int kRouterThreads = 256;
-constexpr int kRouterKC = 32;
+constexpr int kRBM = 128;
+constexpr int kRBK = 64;
+constexpr int kRThreads = 192;
+constexpr int kRMaxSplitSMs = 256;     // upper bound on SMs, sizes the partials buffer
 
-template <int EP, int EPT, int TPT>
-struct RouterShape {
-  static constexpr int TX = EP / EPT;                  // threads along experts
-  static constexpr int TY = kRouterThreads / TX;       // threads along tokens
-  static constexpr int BT = TY * TPT;                  // tokens per CTA
-  static constexpr int kStageFloats = kRouterKC * EP + kRouterKC * BT;
-  static constexpr int kLogitFloats = BT * EP;
-  static constexpr int kSmemFloats = kStageFloats > kLogitFloats ? kStageFloats : kLogitFloats;
+// ---------------------------------------------------------------- 1. split
+__global__ void __launch_bounds__(256)
+    router_split_kernel(const float* __restrict__ wr, int d, int E, int Ep,
+                        __nv_bfloat16* __restrict__ w2) {
+  const size_t n = (size_t)d * Ep;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / Ep), e = (int)(idx % Ep);
+    const float w = e < E ? wr[(size_t)i * E + e] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+    const int blk = i / kRBK, r = i % kRBK;
+    w2[(size_t)(blk * 2 * kRBK + r) * Ep + e] = hi;
+    w2[(size_t)(blk * 2 * kRBK + kRBK + r) * Ep + e] = lo;
+  }
+}
+
+// ---------------------------------------------------------------- 2. GEMM
+template <int NCH>
+struct RouterCfg {
+  static constexpr int N = 64 * NCH;                      // MMA N = Ep
+  static constexpr int kABytes = kRBM * kRBK * 2;
+  static constexpr int kBBytes = N * kRBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStagesFit = (192 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kTmemCols = (2 * N <= 128) ? 128 : (2 * N <= 256 ? 256 : 512);
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(kRBM, N, /*b_mn_major=*/true);
 };
 
-template <int EP, int EPT, int TPT>
-__global__ void __launch_bounds__(kRouterThreads)
-    router_topk_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
-                       const float* __restrict__ bias, int T, int d, int E, int k,
-                       float* __restrict__ logits, int32_t* __restrict__ topk_idx,
-                       float* __restrict__ topk_w) {
-  using S = RouterShape<EP, EPT, TPT>;
-  __shared__ __align__(16) float smem[S::kSmemFloats];
-  float* ws = smem;                          // [KC][EP]
-  float* xs = smem + kRouterKC * EP;         // [KC][BT]
+struct RouterShared {
+  uint64_t full_bar[8];
+  uint64_t empty_bar[8];
+  uint64_t tfull_bar[2];
+  uint64_t tempty_bar[2];
+  uint64_t drain_bar;
+  uint32_t tmem_base;
+  int abort_flag;
+  int never;
+};
 
-  const int tid = threadIdx.x;
-  const int tx = tid % S::TX, ty = tid / S::TX;
-  const int t0 = blockIdx.x * S::BT;
+template <int NCH>
+__global__ void __launch_bounds__(kRThreads, 1)
+    router_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmW, int T, int E, int S,
+                       int kb_total, float* __restrict__ partial, int32_t* status) {
+  using Cfg = RouterCfg<NCH>;
+  extern __shared__ uint8_t dsmem_raw[];
+  __shared__ RouterShared sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int m_tiles = (T + kRBM - 1) / kRBM;
+  const int total_tiles = m_tiles * S;
 
-  float acc[TPT][EPT];
-#pragma unroll
-  for (int i = 0; i < TPT; ++i)
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) acc[i][j] = 0.f;
-
-  for (int k0 = 0; k0 < d; k0 += kRouterKC) {
-    // x chunk: BT tokens x KC values, 8 bf16 (16 B) per load, stored transposed
-    for (int v = tid; v < S::BT * (kRouterKC / 8); v += kRouterThreads) {
-      const int tt = v / (kRouterKC / 8), part = v % (kRouterKC / 8);
-      const int t = t0 + tt;
-      uint4 raw = make_uint4(0, 0, 0, 0);
-      if (t < T) raw = *reinterpret_cast<const uint4*>(x + (size_t)t * d + k0 + part * 8);
-      const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) xs[(part * 8 + q) * S::BT + tt] = __bfloat162float(b[q]);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&sh.full_bar[s], 1);
+      mbar_init(&sh.empty_bar[s], 1);
     }
-    // Wr chunk: KC rows x EP experts (experts >= E read as zero)
-    for (int v = tid; v < kRouterKC * EP; v += kRouterThreads) {
-      const int kk = v / EP, e = v % EP;
-      ws[v] = (e < E) ? wr[(size_t)(k0 + kk) * E + e] : 0.f;
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sh.tfull_bar[a], 1);
+      mbar_init(&sh.tempty_bar[a], 4);
     }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kRouterKC; ++kk) {
-      float xv[TPT], wv[EPT];
-#pragma unroll
-      for (int i = 0; i < TPT; ++i) xv[i] = xs[kk * S::BT + ty * TPT + i];
-#pragma unroll
-      for (int j = 0; j < EPT; ++j) wv[j] = ws[kk * EP + tx * EPT + j];
-#pragma unroll
-      for (int i = 0; i < TPT; ++i)
-#pragma unroll
-        for (int j = 0; j < EPT; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
-    }
-    __syncthreads();
+    mbar_init(&sh.drain_bar, 1);
+    sh.abort_flag = 0;
+    sh.never = 0;
+    fence_barrier_init();
   }
-
-  // logits (+bias) to global memory and to the shared tile [BT][EP]
-  float* ls = smem;
-#pragma unroll
-  for (int i = 0; i < TPT; ++i) {
-    const int tt = ty * TPT + i, t = t0 + tt;
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-      const int e = tx * EPT + j;
-      float v = acc[i][j];
-      if (e < E) {
-        if (bias) v += bias[e];
-        if (t < T) logits[(size_t)t * E + e] = v;
-      }
-      ls[tt * EP + e] = v;
-    }
+  if (warp == 0) {
+    tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
+    tmem_relinquish();
   }
+  if (warp == 1 && lane == 0) {
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmW);
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sh.tmem_base;
+  volatile int* abort_flag = &sh.abort_flag;
 
-  // top-k: one warp per token
-  constexpr int kPerLane = EP >= 32 ? EP / 32 : 1;
-  const int warp = tid / 32, lane = tid % 32;
-  for (int tt = warp; tt < S::BT; tt += kRouterThreads / 32) {
-    const int t = t0 + tt;
-    if (t >= T) break;
-    float val[kPerLane];
-    bool live[kPerLane];
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int it = 0;
+      int last_it[8];
+      for (int s = 0; s < Cfg::kStages; ++s) last_it[s] = -1;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        const int sp = tile / m_tiles, m = tile - sp * m_tiles;
+        const int kb0 = (int)((long long)sp * kb_total / S);
+        const int kb1 = (int)((long long)(sp + 1) * kb_total / S);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % Cfg::kStages;
+          const uint32_t ph = (it / Cfg::kStages) & 1;
+          if (!mbar_wait(&sh.empty_bar[st], ph ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t* sa = smem + st * Cfg::kStageBytes;
+          uint8_t* sb = sa + Cfg::kABytes;
+          mbar_arrive_expect_tx(&sh.full_bar[st], Cfg::kStageBytes);
+          tma_load_2d(sa, &tmX, &sh.full_bar[st], (kb >> 1) * kRBK, m * kRBM);
 #pragma unroll
-    for (int c = 0; c < kPerLane; ++c) {
-      const int e = lane + 32 * c;
-      live[c] = e < E;
-      val[c] = live[c] ? ls[tt * EP + e] : 0.f;
+          for (int c = 0; c < NCH; ++c)
+            tma_load_2d(sb + c * 8192, &tmW, &sh.full_bar[st], c * 64, kb * kRBK);
+          last_it[st] = it;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(status, kDevErrWaitTimeout);
+      }
+      for (int st = 0; st < Cfg::kStages; ++st)
+        if (last_it[st] >= 0)
+          mbar_wait(&sh.full_bar[st], (last_it[st] / Cfg::kStages) & 1, &sh.never);
     }
-    float sel_v[8];
-    int sel_e[8];
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++lt) {
+        const int sp = tile / m_tiles;
+        const int kb0 = (int)((long long)sp * kb_total / S);
+        const int kb1 = (int)((long long)(sp + 1) * kb_total / S);
+        const int a = lt & 1;
+        const uint32_t aph = (lt >> 1) & 1;
+        if (!mbar_wait(&sh.tempty_bar[a], aph ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * Cfg::N);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % Cfg::kStages;
+          const uint32_t ph = (it / Cfg::kStages) & 1;
+          if (!mbar_wait(&sh.full_bar[st], ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + st * Cfg::kStageBytes);
+          const uint32_t b_addr = a_addr + Cfg::kABytes;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j >= k) break;
-      // best live candidate of this lane
-      float bv = 0.f;
-      int be = INT32_MAX;
+          for (int ks = 0; ks < kRBK / 16; ++ks) {
+            const uint64_t adesc = smem_desc_sw128(a_addr + ks * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, 8192, 1024);
+            umma_bf16(d_tmem, adesc, bdesc, Cfg::kIdesc, (kb != kb0 || ks != 0) ? 1u : 0u);
+          }
+          umma_commit(&sh.empty_bar[st]);
+        }
+        if (!ok) break;
+        umma_commit(&sh.tfull_bar[a]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(status, kDevErrWaitTimeout);
+      }
+      umma_commit(&sh.drain_bar);
+      mbar_wait(&sh.drain_bar, 0, &sh.never);
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
+      const int sp = tile / m_tiles, m = tile - sp * m_tiles;
+      const int a = lt & 1;
+      const uint32_t aph = (lt >> 1) & 1;
+      if (!mbar_wait(&sh.tfull_bar[a], aph, abort_flag)) {
+        *abort_flag = 1;
+        report(status, kDevErrWaitTimeout);
+        break;
+      }
+      tc_fence_after();
+      const int row = m * kRBM + q * 32 + lane;
+      const bool valid = row < T;
+      float* prow = partial + ((size_t)sp * T + row) * E;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * Cfg::N);
+#pragma unroll 1
+      for (int c = 0; c < Cfg::N / 32; ++c) {
+        if (c * 32 >= E) break;                     // warp-uniform
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + c * 32, v);
+        tmem_ld_wait();
+        if (valid) {
+          if ((E & 31) == 0) {
+            uint4* dst = reinterpret_cast<uint4*>(prow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i < E) prow[c * 32 + i] = __uint_as_float(v[i]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.tempty_bar[a]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- 3. top-k
+// 256 threads.  tpc tokens per CTA (8 when S < 8: one warp per token; 1 when
+// S >= 8: the 8 warps split the partial sums of one token, combined in warp
+// order through shared memory).
+template <int EP>
+__global__ void __launch_bounds__(256)
+    router_topk_kernel(const float* __restrict__ partial, int S, const float* __restrict__ bias,
+                       int T, int E, int k, int tpc, float* __restrict__ logits,
+                       int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  constexpr int kPerLane = EP / 32;
+  __shared__ float red[8][EP];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int wpt = 8 / tpc;
+  const int tok = warp / wpt, part = warp % wpt;
+  const int t = blockIdx.x * tpc + tok;
+  float v[kPerLane];
+#pragma unroll
+  for (int c = 0; c < kPerLane; ++c) v[c] = 0.f;
+  if (t < T) {
+    for (int s = part; s < S; s += wpt) {
+      const float* p = partial + ((size_t)s * T + t) * E;
 #pragma unroll
       for (int c = 0; c < kPerLane; ++c) {
         const int e = lane + 32 * c;
-        if (live[c] && (be == INT32_MAX || val[c] > bv)) { bv = val[c]; be = e; }
+        if (e < E) v[c] += p[e];
       }
-      // warp arg-max: larger value wins, equal values go to the lower index
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        const bool take = (oe != INT32_MAX) &&
-                          (be == INT32_MAX || ov > bv || (ov == bv && oe < be));
-        if (take) { bv = ov; be = oe; }
-      }
-      sel_v[j] = bv;
-      sel_e[j] = be;
-#pragma unroll
-      for (int c = 0; c < kPerLane; ++c)
-        if (lane + 32 * c == be) live[c] = false;
     }
-    if (lane == 0) {
-      const float m = sel_v[0];
-      float p[8], s = 0.f;
+  }
+  if (wpt > 1) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j >= k) break;
-        p[j] = expf(sel_v[j] - m);
-        s += p[j];
-      }
+    for (int c = 0; c < kPerLane; ++c) red[warp][lane + 32 * c] = v[c];
+    __syncthreads();
+    if (part == 0) {
+      for (int w = 1; w < wpt; ++w)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j >= k) break;
-        topk_idx[(size_t)t * k + j] = sel_e[j];
-        topk_w[(size_t)t * k + j] = p[j] / s;
-      }
+        for (int c = 0; c < kPerLane; ++c) v[c] += red[warp + w][lane + 32 * c];
+    }
+  }
+  if (part != 0 || t >= T) return;
+
+  bool live[kPerLane];
+#pragma unroll
+  for (int c = 0; c < kPerLane; ++c) {
+    const int e = lane + 32 * c;
+    live[c] = e < E;
+    if (live[c]) {
+      if (bias) v[c] += bias[e];
+      logits[(size_t)t * E + e] = v[c];
+    }
+  }
+  float sel_v[8];
+  int sel_e[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    float bv = 0.f;
+    int be = INT32_MAX;
+#pragma unroll
+    for (int c = 0; c < kPerLane; ++c) {
+      const int e = lane + 32 * c;
+      if (live[c] && (be == INT32_MAX || v[c] > bv)) { bv = v[c]; be = e; }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      const bool take = (oe != INT32_MAX) &&
+                        (be == INT32_MAX || ov > bv || (ov == bv && oe < be));
+      if (take) { bv = ov; be = oe; }
+    }
+    sel_v[j] = bv;
+    sel_e[j] = be;
+#pragma unroll
+    for (int c = 0; c < kPerLane; ++c)
+      if (lane + 32 * c == be) live[c] = false;
+  }
+  if (lane == 0) {
+    const float mx = sel_v[0];
+    float p[8], sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      p[j] = expf(sel_v[j] - mx);
+      sum += p[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      topk_idx[(size_t)t * k + j] = sel_e[j];
+      topk_w[(size_t)t * k + j] = p[j] / sum;
     }
   }
 }
 
-template <int EP, int EPT, int TPT>
-static cudaError_t launch_router(const __nv_bfloat16* x, const float* wr, const float* bias,
-                                 int T, int d, int E, int k, float* logits, int32_t* idx,
-                                 float* w, cudaStream_t s) {
-  using S = RouterShape<EP, EPT, TPT>;
-  const int grid = (T + S::BT - 1) / S::BT;
-  router_topk_kernel<EP, EPT, TPT><<<grid, kRouterThreads, 0, s>>>(x, wr, bias, T, d, E, k,
-                                                                    logits, idx, w);
+// ---------------------------------------------------------------- host side
+
+static int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// K splits for a batch: enough (row tile, split) tiles to occupy `sms` SMs,
+// at most one split per k-block.
+static int route_splits(int T, int d, int sms) {
+  const int m_tiles = (T + kRBM - 1) / kRBM;
+  const int kb_total = 2 * d / kRBK;
+  int S = sms / m_tiles;
+  if (S < 1) S = 1;
+  if (S > kb_total) S = kb_total;
+  return S;
+}
+
+size_t route_scratch_bytes(int64_t T, int64_t d, int64_t E) {
+  const int Ep = round_up((int)E, 64);
+  const size_t w2 = align256((size_t)2 * d * Ep * 2);
+  const int S = route_splits((int)T, (int)d, kRMaxSplitSMs);
+  return w2 + align256((size_t)S * T * E * sizeof(float));
+}
+
+template <int NCH>
+static cudaError_t launch_router_gemm(DeviceInfo* di, const CUtensorMap& tx,
+                                      const CUtensorMap& tw, int T, int E, int S, int kb_total,
+                                      float* partial, int32_t* status, cudaStream_t s) {
+  using Cfg = RouterCfg<NCH>;
+  auto kern = router_gemm_kernel<NCH>;
+  const int slot = 2 + NCH;                      // attribute slots 3..6
+  if (!di->attr_set[slot]) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           Cfg::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    di->attr_set[slot] = true;
+  }
+  const int tiles = ((T + kRBM - 1) / kRBM) * S;
+  const int grid = tiles < di->sms ? tiles : di->sms;
+  kern<<<grid, kRThreads, Cfg::kSmemBytes, s>>>(tx, tw, T, E, S, kb_total, partial, status);
+  return cudaGetLastError();
+}
+
+template <int EP>
+static cudaError_t launch_topk(const float* partial, int S, const float* bias, int T, int E,
+                               int k, float* logits, int32_t* idx, float* w, cudaStream_t s) {
+  const int tpc = S >= 8 ? 1 : 8;
+  router_topk_kernel<EP><<<(T + tpc - 1) / tpc, 256, 0, s>>>(partial, S, bias, T, E, k, tpc,
+                                                              logits, idx, w);
   return cudaGetLastError();
 }
 
 cudaError_t launch_route(const __nv_bfloat16* x, const float* wr, const float* bias, int T,
                          int d, int E, int k, float* logits, int32_t* idx, float* w,
-                         cudaStream_t s) {
-  if (E <= 8) return launch_router<8, 2, 1>(x, wr, bias, T, d, E, k, logits, idx, w, s);
-  if (E <= 16) return launch_router<16, 2, 2>(x, wr, bias, T, d, E, k, logits, idx, w, s);
-  if (E <= 32) return launch_router<32, 4, 2>(x, wr, bias, T, d, E, k, logits, idx, w, s);
-  if (E <= 64) return launch_router<64, 8, 2>(x, wr, bias, T, d, E, k, logits, idx, w, s);
-  if (E <= 128) return launch_router<128, 8, 4>(x, wr, bias, T, d, E, k, logits, idx, w, s);
-  return launch_router<256, 8, 4>(x, wr, bias, T, d, E, k, logits, idx, w, s);
+                         void* scratch, int32_t* status, cudaStream_t s, bool* map_failed) {
+  *map_failed = false;
+  DeviceInfo* di = nullptr;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  const int Ep = round_up(E, 64);
+  const int NCH = Ep / 64;
+  __nv_bfloat16* w2 = static_cast<__nv_bfloat16*>(scratch);
+  float* partial = reinterpret_cast<float*>(static_cast<char*>(scratch) +
+                                            align256((size_t)2 * d * Ep * 2));
+  int S = route_splits(T, d, di->sms < kRMaxSplitSMs ? di->sms : kRMaxSplitSMs);
+  const int kb_total = 2 * d / kRBK;
+
+  const size_t n = (size_t)d * Ep;
+  int blocks = (int)((n + 255) / 256);
+  if (blocks > 8 * di->sms) blocks = 8 * di->sms;
+  router_split_kernel<<<blocks, 256, 0, s>>>(wr, d, E, Ep, w2);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+
+  CUtensorMap tx, tw;
+  if (!map_rows(&tx, x, d, T, kRBM) || !map_rows(&tw, w2, Ep, 2 * (uint64_t)d, kRBK)) {
+    *map_failed = true;
+    return cudaSuccess;
+  }
+  switch (NCH) {
+    case 1: err = launch_router_gemm<1>(di, tx, tw, T, E, S, kb_total, partial, status, s); break;
+    case 2: err = launch_router_gemm<2>(di, tx, tw, T, E, S, kb_total, partial, status, s); break;
+    case 3: err = launch_router_gemm<3>(di, tx, tw, T, E, S, kb_total, partial, status, s); break;
+    default: err = launch_router_gemm<4>(di, tx, tw, T, E, S, kb_total, partial, status, s); break;
+  }
+  if (err != cudaSuccess) return err;
+  if (E <= 32) return launch_topk<32>(partial, S, bias, T, E, k, logits, idx, w, s);
+  if (E <= 64) return launch_topk<64>(partial, S, bias, T, E, k, logits, idx, w, s);
+  if (E <= 128) return launch_topk<128>(partial, S, bias, T, E, k, logits, idx, w, s);
+  return launch_topk<256>(partial, S, bias, T, E, k, logits, idx, w, s);
 }
 
 }  // namespace moe

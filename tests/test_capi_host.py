@@ -59,29 +59,37 @@ def test_capacity_rejects_bad_args():
 def test_workspace_layout(cfg):
     T, d, E, k, f, cf = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.cf
     total = moe.moe_workspace_size(T, d, E, k, f, cf)
-    offs = [moe.moe_workspace_field_offset(i, T, d, E, k, f, cf) for i in range(13)]
+    offs = [moe.moe_workspace_field_offset(i, T, d, E, k, f, cf) for i in range(14)]
     assert offs[0] == 0 and all(o % 256 == 0 for o in offs)
     assert offs == sorted(offs)
     rows = moe.moe_max_rows(T, E, k, cf)
-    assert total - offs[12] >= rows * d * 2          # y_perm is last
-    assert offs[12] - offs[11] >= rows * f * 2       # h
-    assert offs[11] - offs[10] >= rows * d * 2       # x_perm
-    assert moe.moe_workspace_field_offset(13, T, d, E, k, f, cf) == -1
+    ends = offs[1:] + [total]
+    need = {1: T * E * 4, 2: T * k * 4, 3: T * k * 4, 4: T * k * 4, 5: E * 4, 6: (E + 1) * 4,
+            8: rows * 4, 9: moe.moe_permute_workspace_size(T, E, k), 10: rows * d * 2,
+            11: rows * f * 2, 12: rows * d * 4, 13: moe.moe_route_workspace_size(T, d, E, k)}
+    for i, n in need.items():
+        assert ends[i] - offs[i] >= n, binding.WS_FIELDS[i]
+    assert moe.moe_route_workspace_size(T, d, E, k) >= 2 * d * ((E + 63) // 64 * 64) * 2
+    assert moe.moe_workspace_field_offset(14, T, d, E, k, f, cf) == -1
 
 
 def test_validation_codes_without_launch():
     L = moe.lib()
     s = ctypes.c_void_p(0)
-    # route: bad E, bad k, k > E, unsupported width, empty batch
-    assert L.moe_route(FAKE, FAKE, None, 4, 128, 0, 1, FAKE, FAKE, FAKE, s) == INVALID
-    assert L.moe_route(FAKE, FAKE, None, 4, 128, 300, 2, FAKE, FAKE, FAKE, s) == INVALID
-    assert L.moe_route(FAKE, FAKE, None, 4, 128, 8, 9, FAKE, FAKE, FAKE, s) == INVALID
-    assert L.moe_route(FAKE, FAKE, None, 4, 128, 2, 3, FAKE, FAKE, FAKE, s) == INVALID
-    assert L.moe_route(FAKE, FAKE, None, 4, 100, 8, 2, FAKE, FAKE, FAKE, s) == UNSUPPORTED
-    assert L.moe_route(None, FAKE, None, 4, 128, 8, 2, FAKE, FAKE, FAKE, s) == INVALID
-    assert L.moe_route(FAKE, FAKE, None, 0, 128, 8, 2, FAKE, FAKE, FAKE, s) == OK
+    # route: bad E, bad k, k > E, unsupported width, empty batch, small workspace
+    R = moe.moe_route_workspace_size(4, 128, 8, 2)
+    W = [FAKE, R, None, s]
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 0, 1, FAKE, FAKE, FAKE, *W) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 300, 2, FAKE, FAKE, FAKE, *W) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 8, 9, FAKE, FAKE, FAKE, *W) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 2, 3, FAKE, FAKE, FAKE, *W) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 4, 100, 8, 2, FAKE, FAKE, FAKE, *W) == UNSUPPORTED
+    assert L.moe_route(None, FAKE, None, 4, 128, 8, 2, FAKE, FAKE, FAKE, *W) == INVALID
+    assert L.moe_route(FAKE, FAKE, None, 0, 128, 8, 2, FAKE, FAKE, FAKE, *W) == OK
+    assert L.moe_route(FAKE, FAKE, None, 4, 128, 8, 2, FAKE, FAKE, FAKE, FAKE, R - 1, None, s) \
+        == WORKSPACE
     misaligned = ctypes.c_void_p((1 << 20) + 2)
-    assert L.moe_route(misaligned, FAKE, None, 4, 128, 8, 2, FAKE, FAKE, FAKE, s) == INVALID
+    assert L.moe_route(misaligned, FAKE, None, 4, 128, 8, 2, FAKE, FAKE, FAKE, *W) == INVALID
     # permute: workspace too small
     need = moe.moe_permute_workspace_size(100, 8, 2)
     assert need > 0

@@ -62,6 +62,9 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        import threading
+        self.lines = []
+        self.first = threading.Event()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
@@ -69,17 +72,26 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+
+        def reader():
+            for line in self.proc.stdout:
+                self.lines.append(line)
+                self.first.set()
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        self.first.wait(timeout=10)      # sampling has started before timing begins
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+            self.thread.join(timeout=5)
+        self.out = "".join(self.lines)
         return False
 
     def summary(self):
@@ -215,6 +227,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
                 for j, n in enumerate(names)}
     status = int(layer.status.item())
     N = int(layer.perm["offsets"][cfg.E].item())
+    active = int((layer.perm["counts"] > 0).sum().item())
     n_drop = int(layer.perm["n_dropped"].item())
 
     # end to end through the one-shot public call, host buffers in and out
@@ -240,6 +253,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, dist)
     return {"elapsed_ms": elapsed_ms, "stage_ms": stage_ms, "status": status, "N": N,
+            "active_experts": active,
             "n_dropped": n_drop, "clocks": clk.summary(), "e2e_ms": e2e_ms,
             "h2d": x_host.numel() * 2, "d2h": y_host.numel() * 2, "layer": layer}
 
@@ -340,6 +354,13 @@ def main():
     t_g2 = r["stage_ms"]["down"] / 1e3
     peak_tf = pk["bf16_tflops"]
     achieved = gemm1_flop / t_g1 / 1e12
+    # bytes the gate/up GEMM must move: weights of the experts that got rows,
+    # x_perm rows in, h rows out
+    A = r["active_experts"]
+    g1_bytes = A * 2.0 * cfg.d * cfg.f * 2 + r["N"] * cfg.d * 2 + r["N"] * cfg.f * 2
+    g2_bytes = A * 1.0 * cfg.d * cfg.f * 2 + r["N"] * cfg.f * 2 + r["N"] * cfg.d * 4
+    ridge = peak_tf * 1e12 / (pk["hbm_gbs"] * 1e9)
+    hbm_bound = gemm1_flop / g1_bytes < ridge
     bytes_perm = cfg.T * cfg.d * 2 + r["N"] * cfg.d * 2
     bytes_comb = r["N"] * cfg.d * 4 + cfg.T * cfg.d * 2
     out = {
@@ -360,15 +381,28 @@ def main():
                    "parallelism": f"replicas x{world} (token batches, no collective)",
                    "l2": "inputs larger than L2 (expert weights "
                          f"{3 * cfg.E * cfg.d * cfg.f * 2 / 1e9:.1f} GB); no flush"},
-        "roofline": {"kernel": "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)",
-                     "bound": "tensor", "achieved": round(achieved, 1),
-                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
-                     "peak_source": f"{pk_kind} bf16 burst",
-                     "traffic": traffic_from_profile("gemm_gate_up", cfg.name)},
+        "roofline": ({"kernel": "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)",
+                      "bound": "tensor", "achieved": round(achieved, 1),
+                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                      "peak_source": f"{pk_kind} bf16 burst",
+                      "traffic": traffic_from_profile("gemm_gate_up", cfg.name)}
+                     if not hbm_bound else
+                     {"kernel": "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)",
+                      "bound": "hbm", "achieved": round(g1_bytes / t_g1 / 1e9, 1),
+                      "peak": pk["hbm_gbs"], "unit": "GB/s",
+                      "frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
+                      "peak_source": f"{pk_kind} HBM copy",
+                      "algorithmic_bytes": g1_bytes, "active_experts": A,
+                      "traffic": traffic_from_profile("gemm_gate_up", cfg.name)}),
         "stages_ms": {k_: round(v, 4) for k_, v in r["stage_ms"].items()},
         "stage_rooflines": {
             "down_gemm": {"bound": "tensor", "achieved": round(gemm2_flop / t_g2 / 1e12, 1),
-                          "unit": "TFLOP/s", "frac": round(gemm2_flop / t_g2 / 1e12 / peak_tf, 4)},
+                          "unit": "TFLOP/s", "frac": round(gemm2_flop / t_g2 / 1e12 / peak_tf, 4),
+                          "hbm_GBps": round(g2_bytes / t_g2 / 1e9, 1),
+                          "hbm_frac": round(g2_bytes / t_g2 / 1e9 / pk["hbm_gbs"], 4)},
+            "gate_up_gemm_hbm": {"GBps": round(g1_bytes / t_g1 / 1e9, 1),
+                                 "frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
+                                 "active_experts": A},
             "permute": {"bound": "hbm", "unit": "GB/s",
                         "achieved": round(bytes_perm / (r["stage_ms"]["permute"] / 1e3) / 1e9, 1),
                         "frac": round(bytes_perm / (r["stage_ms"]["permute"] / 1e3) / 1e9

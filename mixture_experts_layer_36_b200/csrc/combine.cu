@@ -7,23 +7,28 @@
 // pairs were all dropped leaves the layer unchanged (inferensys.com glossary,
 // Dropped Tokens entry).
 //
-// One warp per token: lanes 0..k-1 resolve the k source rows and weights,
-// broadcast them, then the warp streams the d-wide fp32 rows in 16-byte
-// vectors, accumulating in fp32 in top-k order and rounding once to bf16.
+// One warp per (token, 512-column segment): lanes 0..k-1 resolve the k source
+// rows and weights, broadcast them, then the warp streams its segment of the
+// fp32 rows in 16-byte vectors, accumulating in fp32 in top-k order and
+// rounding once to bf16.
 #include "common.cuh"
 
 namespace moe {
 
 constexpr int kCombThreads = 256;
+constexpr int kSegVec = 64;        // 16-byte output vectors per warp work unit (512 elements)
 
+// One warp per (token, 512-column segment), so that a handful of tokens still
+// spreads over many SMs.
 __global__ void __launch_bounds__(kCombThreads)
     combine_kernel(const float* __restrict__ y_perm, const __nv_bfloat16* __restrict__ x,
                    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ slot, const int32_t* __restrict__ offsets, int T,
-                   int d, int k, __nv_bfloat16* __restrict__ y) {
+                   int d, int k, int nseg, __nv_bfloat16* __restrict__ y) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int t = blockIdx.x * (kCombThreads / 32) + warp;
-  if (t >= T) return;
+  const long long unit = (long long)blockIdx.x * (kCombThreads / 32) + warp;
+  if (unit >= (long long)T * nseg) return;
+  const int t = (int)(unit / nseg), seg = (int)(unit % nseg);
   int my_row = -1;
   float my_w = 0.f;
   if (lane < k) {
@@ -43,50 +48,50 @@ __global__ void __launch_bounds__(kCombThreads)
   }
   const bool any_kept = __any_sync(0xffffffffu, my_row >= 0);
   const int nvec = d / 8;
+  const int v_begin = seg * kSegVec;
+  const int v_end = min(nvec, v_begin + kSegVec);
   uint4* dst = reinterpret_cast<uint4*>(y + (size_t)t * d);
   if (!any_kept) {
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-    for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    for (int v = v_begin + lane; v < v_end; v += 32) dst[v] = __ldg(src + v);
     return;
   }
-  for (int v0 = lane; v0 < nvec; v0 += 64) {
-    float acc[2][8];
+  float acc[2][8];
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+  for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
+    for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j >= k) break;
-      if (rows[j] < 0) continue;
-      const float4* src = reinterpret_cast<const float4*>(y_perm + (size_t)rows[j] * d);
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int v = v0 + u * 32;
-        if (v >= nvec) continue;
-        const float4 a = __ldg(src + 2 * v);
-        const float4 b = __ldg(src + 2 * v + 1);
-        acc[u][0] = fmaf(w[j], a.x, acc[u][0]);
-        acc[u][1] = fmaf(w[j], a.y, acc[u][1]);
-        acc[u][2] = fmaf(w[j], a.z, acc[u][2]);
-        acc[u][3] = fmaf(w[j], a.w, acc[u][3]);
-        acc[u][4] = fmaf(w[j], b.x, acc[u][4]);
-        acc[u][5] = fmaf(w[j], b.y, acc[u][5]);
-        acc[u][6] = fmaf(w[j], b.z, acc[u][6]);
-        acc[u][7] = fmaf(w[j], b.w, acc[u][7]);
-      }
-    }
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    if (rows[j] < 0) continue;
+    const float4* src = reinterpret_cast<const float4*>(y_perm + (size_t)rows[j] * d);
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int v = v0 + u * 32;
-      if (v >= nvec) continue;
-      uint4 o;
-      o.x = pack_bf16x2(acc[u][0], acc[u][1]);
-      o.y = pack_bf16x2(acc[u][2], acc[u][3]);
-      o.z = pack_bf16x2(acc[u][4], acc[u][5]);
-      o.w = pack_bf16x2(acc[u][6], acc[u][7]);
-      dst[v] = o;
+      const int v = v_begin + lane + u * 32;
+      if (v >= v_end) continue;
+      const float4 a = __ldg(src + 2 * v);
+      const float4 b = __ldg(src + 2 * v + 1);
+      acc[u][0] = fmaf(w[j], a.x, acc[u][0]);
+      acc[u][1] = fmaf(w[j], a.y, acc[u][1]);
+      acc[u][2] = fmaf(w[j], a.z, acc[u][2]);
+      acc[u][3] = fmaf(w[j], a.w, acc[u][3]);
+      acc[u][4] = fmaf(w[j], b.x, acc[u][4]);
+      acc[u][5] = fmaf(w[j], b.y, acc[u][5]);
+      acc[u][6] = fmaf(w[j], b.z, acc[u][6]);
+      acc[u][7] = fmaf(w[j], b.w, acc[u][7]);
     }
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int v = v_begin + lane + u * 32;
+    if (v >= v_end) continue;
+    uint4 o;
+    o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+    o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+    o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+    o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+    dst[v] = o;
   }
 }
 
@@ -94,9 +99,11 @@ cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t s) {
+  const int nseg = (d / 8 + kSegVec - 1) / kSegVec;
+  const long long units = (long long)T * nseg;
   const int per_cta = kCombThreads / 32;
-  combine_kernel<<<(T + per_cta - 1) / per_cta, kCombThreads, 0, s>>>(
-      y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y);
+  combine_kernel<<<(unsigned)((units + per_cta - 1) / per_cta), kCombThreads, 0, s>>>(
+      y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, nseg, y);
   return cudaGetLastError();
 }
 

@@ -317,6 +317,329 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA-pair variant
+// Two CTAs of a cluster share one tcgen05.mma.cta_group::2 of M = 256, N = 256:
+// each CTA stages its own 128 bucket rows of A and half of the B columns
+// (GEMM 1: CTA 0 the gate columns, CTA 1 the up columns of the same 128
+// h-columns; GEMM 2: 128 of the 256 output columns each), so each SM receives
+// 32 KB of operands per 64-deep k-block instead of 48 KB.  Both CTAs' TMA
+// loads complete on the leader CTA's stage barrier (armed by the leader for
+// the bytes of both); the leader issues the MMAs and multicasts "stage free"
+// and "accumulator ready" to both CTAs; both epilogues (each on its own 128
+// accumulator rows, all 256 columns) report back to the leader.  Used when
+// buckets are large (the pair tile is 256 rows).
+//
+// Half tiles.  When the last tile of an expert has at most 128 rows, the pair
+// runs the M = 128 form of the MMA instead (64 rows per CTA).  Its accumulator
+// puts columns [0,128) in TMEM lanes 0-63 and [128,256) in lanes 64-127, so
+// epilogue warps 0-1 and 2-3 take the two column halves of the same 64 rows.
+// For GEMM 1 each CTA then stages 64 gate + 64 up columns (CTA r: h-columns
+// [64r, 64r+64) of the tile), so every thread still holds g and u of the same
+// h-column.  This halves the rows computed in vain at each expert's tail.
+// Epilogue pieces: 32 accumulator columns of this thread's row.
+__device__ __forceinline__ void swiglu_chunk_store(uint32_t tg, uint32_t tu, bool valid,
+                                                   __nv_bfloat16* dst_row) {
+  uint32_t g[32], u[32];
+  tmem_ld_32x32b_x32(tg, g);
+  tmem_ld_32x32b_x32(tu, u);
+  tmem_ld_wait();
+  if (!valid) return;
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+    const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+    pk[i] = pack_bf16x2(silu(g0) * u0, silu(g1) * u1);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+}
+
+__device__ __forceinline__ void f32_chunk_store(uint32_t t, bool valid, float* dst_row) {
+  uint32_t v[32];
+  tmem_ld_32x32b_x32(t, v);
+  tmem_ld_wait();
+  if (!valid) return;
+  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+constexpr int kPairStages = 6;
+constexpr int kPairStageBytes = 2 * kBM * kBK * 2;      // A 16 KB + half of B 16 KB
+
+struct PairShared {
+  uint64_t full_bar[kPairStages];
+  uint64_t empty_bar[kPairStages];
+  uint64_t tfull_bar[2];
+  uint64_t tempty_bar[2];
+  uint64_t drain_bar;
+  uint32_t tmem_base;
+  int abort_flag;
+  int never;
+  int tile_prefix[257];
+  int row_off[256];
+  int row_cnt[256];
+};
+
+__device__ __forceinline__ void decode_pair_tile(const PairShared& sh, int tile, int E,
+                                                 int n_tiles, int& e, int& m, int& n) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sh.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int local = tile - sh.tile_prefix[e];
+  const int mt = (sh.tile_prefix[e + 1] - sh.tile_prefix[e]) / n_tiles;
+  n = local / mt;
+  m = local - n * mt;
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB0,
+                             const __grid_constant__ CUtensorMap tmB1,
+                             const int32_t* __restrict__ offsets, int E, int K, int n_out,
+                             int max_rows, void* __restrict__ out_raw, int32_t* status) {
+  constexpr int kOutCols = SWIGLU ? 128 : 256;        // output columns per pair tile
+  constexpr int kPairM = 2 * kBM;
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kPairM, 256, /*b_mn_major=*/true);
+  constexpr uint32_t kIdescHalf = idesc_bf16_f32(kBM, 256, /*b_mn_major=*/true);
+  constexpr int kTmemCols = 512;
+  extern __shared__ uint8_t dsmem_raw[];
+  __shared__ PairShared sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int n_tiles = n_out / kOutCols;
+  const int nkb = K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&sh.full_bar[s], 1);
+      mbar_init(&sh.empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sh.tfull_bar[a], 1);
+      mbar_init(&sh.tempty_bar[a], 8);       // 4 epilogue warps in each CTA
+    }
+    mbar_init(&sh.drain_bar, 1);
+    sh.abort_flag = 0;
+    sh.never = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(&sh.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == 1 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB0);
+    if (SWIGLU) prefetch_tensormap(&tmB1);
+  }
+  if (warp == 2) {
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int tiles = 0;
+      if (e < E) {
+        const int o0 = offsets[e], o1 = offsets[e + 1];
+        int cnt = o1 - o0;
+        if (o0 < 0 || cnt < 0 || o1 > max_rows) {
+          report(status, kDevErrBadOffsets);
+          cnt = 0;
+        }
+        sh.row_off[e] = o0;
+        sh.row_cnt[e] = cnt;
+        tiles = cnt > 0 ? ((cnt + kPairM - 1) / kPairM) * n_tiles : 0;
+      }
+      int incl = tiles;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (e < E) sh.tile_prefix[e] = carry + incl - tiles;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) sh.tile_prefix[E] = carry;
+  }
+  tc_fence_before();
+  cluster_sync();            // both CTAs' barriers initialised, TMEM allocated
+  tc_fence_after();
+
+  const uint32_t tmem_base = sh.tmem_base;
+  const int total_tiles = sh.tile_prefix[E];
+  volatile int* abort_flag = &sh.abort_flag;
+  const uint32_t peer_abort = mapa_shared(&sh.abort_flag, rank ^ 1u);
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    st_shared_cluster_u32(peer_abort, 1u);
+    report(status, kDevErrWaitTimeout);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      int it = 0;
+      int last_it[kPairStages];
+      for (int s = 0; s < kPairStages; ++s) last_it[s] = -1;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+        int e, m, n;
+        decode_pair_tile(sh, tile, E, n_tiles, e, m, n);
+        const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
+        const int row0 = sh.row_off[e] + m * kPairM + (int)rank * (half ? kBM / 2 : kBM);
+        const int col0 = n * kOutCols;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kPairStages;
+          const uint32_t ph = (it / kPairStages) & 1;
+          if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t* sa = smem + s * kPairStageBytes;
+          uint8_t* sb = sa + kBM * kBK * 2;
+          const uint32_t full_lead = mapa_shared(&sh.full_bar[s], 0);
+          if (leader) mbar_arrive_expect_tx(&sh.full_bar[s], 2 * kPairStageBytes);
+          tma_load_2d_pair(sa, &tmA, full_lead, kb * kBK, row0);
+          if (SWIGLU && half) {
+            tma_load_3d_pair(sb, &tmB0, full_lead, col0 + (int)rank * 64, kb * kBK, e);
+            tma_load_3d_pair(sb + kChunkBytes, &tmB1, full_lead, col0 + (int)rank * 64, kb * kBK,
+                             e);
+          } else if (SWIGLU) {
+            const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d_pair(sb + c * kChunkBytes, mb, full_lead, col0 + c * 64, kb * kBK, e);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d_pair(sb + c * kChunkBytes, &tmB0, full_lead,
+                               col0 + (int)rank * 128 + c * 64, kb * kBK, e);
+          }
+          last_it[s] = it;
+        }
+      }
+      if (!ok) give_up();
+      if (leader) {
+        // both CTAs' copies of every issued phase count on the leader's barriers
+        for (int s = 0; s < kPairStages; ++s)
+          if (last_it[s] >= 0)
+            mbar_wait(&sh.full_bar[s], (last_it[s] / kPairStages) & 1, &sh.never);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (leader CTA)
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs, ++lt) {
+        int e, m, n;
+        decode_pair_tile(sh, tile, E, n_tiles, e, m, n);
+        const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
+        const uint32_t idesc = half ? kIdescHalf : kIdesc;
+        const int a = lt & 1;
+        const uint32_t aph = (lt >> 1) & 1;
+        if (!mbar_wait(&sh.tempty_bar[a], aph ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * 256);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kPairStages;
+          const uint32_t ph = (it / kPairStages) & 1;
+          if (!mbar_wait(&sh.full_bar[s], ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * kPairStageBytes);
+          const uint32_t b_addr = a_addr + kBM * kBK * 2;
+#pragma unroll
+          for (int ks = 0; ks < kBK / kUmmaK; ++ks) {
+            const uint64_t adesc = smem_desc_sw128(a_addr + ks * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, kChunkBytes, 1024);
+            umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair_mc(&sh.empty_bar[s], 0x3);
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(&sh.tfull_bar[a], 0x3);
+      }
+      if (!ok) give_up();
+      umma_commit_pair_mc(&sh.drain_bar, 0x1);
+      mbar_wait(&sh.drain_bar, 0, &sh.never);
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..5, both CTAs)
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    int lt = 0;
+    for (int tile = pair; tile < total_tiles; tile += npairs, ++lt) {
+      int e, m, n;
+      decode_pair_tile(sh, tile, E, n_tiles, e, m, n);
+      const int a = lt & 1;
+      const uint32_t aph = (lt >> 1) & 1;
+      if (!mbar_wait(&sh.tfull_bar[a], aph, abort_flag)) {
+        give_up();
+        break;
+      }
+      tc_fence_after();
+      const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
+      if (!half) {
+        const int local_row = m * kPairM + (int)rank * kBM + row_in_tile;
+        const bool valid = local_row < sh.row_cnt[e];
+        const size_t out_off =
+            (size_t)(sh.row_off[e] + local_row) * n_out + (size_t)n * kOutCols;
+        if (SWIGLU) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c)
+            swiglu_chunk_store(tbase + c * 32, tbase + 128 + c * 32, valid,
+                               static_cast<__nv_bfloat16*>(out_raw) + out_off + c * 32);
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c)
+            f32_chunk_store(tbase + c * 32, valid, static_cast<float*>(out_raw) + out_off + c * 32);
+        }
+      } else {
+        // lanes 0-63: accumulator columns [0,128); lanes 64-127: [128,256)
+        const int hh = q >> 1;
+        const int local_row = m * kPairM + (int)rank * (kBM / 2) + (q & 1) * 32 + lane;
+        const bool valid = local_row < sh.row_cnt[e];
+        const size_t row_off = (size_t)(sh.row_off[e] + local_row) * n_out;
+        if (SWIGLU) {
+          // this CTA's h-columns [64*rank ... ) of the tile: gate in TMEM
+          // columns [0,64), up in [64,128); lanes 64-127 hold the next 64
+          // columns of the tile (staged by the other half of B)
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row_off +
+                             (size_t)n * kOutCols + hh * 64;
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c)
+            swiglu_chunk_store(tbase + c * 32, tbase + 64 + c * 32, valid, o + c * 32);
+        } else {
+          float* o = static_cast<float*>(out_raw) + row_off + (size_t)n * kOutCols + hh * 128;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) f32_chunk_store(tbase + c * 32, valid, o + c * 32);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(&sh.tempty_bar[a], 0));
+    }
+  }
+
+  if (*abort_flag) spin_ns(200000);      // let copies still in flight land
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 template <int BN, bool SWIGLU>
@@ -345,6 +668,48 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
   return cudaGetLastError();
 }
 
+template <bool SWIGLU>
+static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtensorMap& b0,
+                                    const CUtensorMap& b1, const int32_t* offsets, int E, int K,
+                                    int n_out, int max_rows, void* out, int32_t* status,
+                                    cudaStream_t s) {
+  // + 16 KB slack past the last stage, so the pair kernel's smem window also
+  // covers a full-width B read from the last stage
+  constexpr int kSmem = kPairStages * kPairStageBytes + 1024 + 16384;
+  DeviceInfo* di = nullptr;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  auto kern = grouped_gemm_pair_kernel<SWIGLU>;
+  if (!di->attr_set[slot]) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (err != cudaSuccess) return err;
+    di->attr_set[slot] = true;
+  }
+  const int n_tiles = n_out / (SWIGLU ? 128 : 256);
+  const long long pair_rows = (long long)max_rows / (2 * kBM) + (E < max_rows ? E : max_rows);
+  long long pairs = pair_rows * n_tiles;
+  const int max_pairs = di->sms / 2;
+  if (pairs > max_pairs) pairs = max_pairs;
+  if (pairs < 1) pairs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, offsets, E, K, n_out, max_rows, out, status);
+}
+
+// Pair tiles (256 rows) pay off when buckets are large; the buffer's rows
+// per expert bound the average bucket from above.
+static bool use_pair_tiles(int E, int max_rows) { return max_rows >= 512LL * E; }
+
 // GEMM 1: h = silu(x_perm Wg) * (x_perm Wu)
 cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
                            int f, int max_rows, const __nv_bfloat16* w_gate,
@@ -354,6 +719,8 @@ cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, 
   *map_failed = !(map_rows(&ta, x_perm, d, max_rows, kBM) && map_weights(&tg, w_gate, E, d, f) &&
                   map_weights(&tu, w_up, E, d, f));
   if (*map_failed) return cudaSuccess;
+  if (use_pair_tiles(E, max_rows))
+    return launch_gemm_pair<true>(7, ta, tg, tu, offsets, E, d, f, max_rows, h, status, s);
   return launch_gemm<256, true>(0, ta, tg, tu, offsets, E, d, f, max_rows, h, status, s);
 }
 
@@ -364,6 +731,8 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
   CUtensorMap ta, td;
   *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_weights(&td, w_down, E, f, d));
   if (*map_failed) return cudaSuccess;
+  if (d % 256 == 0 && use_pair_tiles(E, max_rows))
+    return launch_gemm_pair<false>(8, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);
   if (d % 256 == 0)
     return launch_gemm<256, false>(1, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);
   return launch_gemm<128, false>(2, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);

@@ -35,6 +35,9 @@ SMALL = [
     small("single_expert", T=200, d=128, E=1, k=1, f=256, cf=0.0, seed=16),
     small("k_equals_E", T=100, d=128, E=4, k=4, f=128, cf=0.0, seed=17),
     small("one_token", T=1, d=128, E=8, k=2, f=128, cf=1.25, seed=18),
+    # buffers of >= 512 rows per expert select the CTA-pair GEMM tiles
+    small("pair_tiles", T=2048, d=256, E=4, k=2, f=256, cf=0.0, seed=19),
+    small("pair_tiles_drops", T=3000, d=512, E=4, k=3, f=384, cf=0.8, seed=20),
 ]
 IDS = [c.name for c in SMALL]
 
@@ -128,22 +131,26 @@ def test_permute_matches_oracle(T, d, E, k, cf):
 # ----------------------------------------------------------------------------- stage: experts
 
 MLP_CASES = [
-    # (d, f, bucket sizes): ragged tails, empty buckets, one-row buckets,
-    # exact tile multiples, several row tiles
-    (256, 384, [300, 0, 1, 129, 128, 257]),
-    (128, 256, [5, 140, 0, 0, 64, 128]),
-    (384, 128, [1, 1, 1, 400]),
-    (512, 640, [129] * 3),
-    (256, 256, [0, 0, 0]),
+    # (d, f, bucket sizes, pair): ragged tails, empty buckets, one-row buckets,
+    # exact tile multiples, several row tiles; pair=True gives the buffer >= 512
+    # rows per expert, which selects the CTA-pair tiles (256 rows)
+    (256, 384, [300, 0, 1, 129, 128, 257], False),
+    (128, 256, [5, 140, 0, 0, 64, 128], False),
+    (384, 128, [1, 1, 1, 400], False),
+    (512, 640, [129] * 3, False),
+    (256, 256, [0, 0, 0], False),
+    (256, 384, [300, 0, 1, 129, 128, 257, 700], True),
+    (512, 256, [1, 256, 511, 513, 1024], True),
+    (384, 256, [255, 257, 0], True),      # down GEMM: d % 256 != 0 keeps single-CTA tiles
 ]
 
 
-@pytest.mark.parametrize("d,f,sizes", MLP_CASES)
-def test_expert_mlp_matches_oracle(d, f, sizes):
+@pytest.mark.parametrize("d,f,sizes,pair", MLP_CASES)
+def test_expert_mlp_matches_oracle(d, f, sizes, pair):
     E = len(sizes)
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     N = int(offsets[-1])
-    max_rows = N + 37
+    max_rows = max(N + 37, 512 * E + 5) if pair else N + 37
     g = torch.Generator().manual_seed(d + f + E)
     x_perm = torch.randn(max_rows, d, generator=g).to(torch.bfloat16)
     wg = (torch.randn(E, d, f, generator=g) / d ** 0.5).to(torch.bfloat16)

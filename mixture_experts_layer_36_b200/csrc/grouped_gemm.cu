@@ -43,6 +43,50 @@ constexpr int kGemmThreads = 192;
 constexpr int kUmmaK = 16;
 constexpr int kChunkBytes = 64 * kBK * 2;   // one B chunk: 64 N x 64 K bf16 = 8 KB
 
+// ---------------------------------------------------------------- epilogue stores
+// Each epilogue thread owns one accumulator row; a warp owns 32 rows.  fp32
+// rows are written through a padded 32 x 32 staging tile in shared memory (one
+// per warp) so that each store instruction covers a whole 128-byte row segment
+// instead of 16 B in each of 32 rows.
+constexpr int kStageWords = 32 * 33;     // per warp, 32-bit words
+
+// fp32: row `lane` holds v[0..31]; rows [0, nvalid) of the warp are stored
+// to out_row0 + r * ld (columns [0, 32)).
+__device__ __forceinline__ void store_chunk_f32(const uint32_t (&v)[32], uint32_t* stage,
+                                                float* out_row0, size_t ld, int nvalid,
+                                                int lane) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) stage[lane * 33 + j] = v[j];
+  __syncwarp();
+  for (int r = 0; r < nvalid; ++r) out_row0[(size_t)r * ld + lane] = __uint_as_float(stage[r * 33 + lane]);
+  __syncwarp();
+}
+
+// bf16: row `lane` holds pk[0..15] (32 bf16), stored directly as four
+// 16-byte vectors (the SwiGLU tile is a quarter of the fp32 one's bytes and
+// measured faster without staging).
+__device__ __forceinline__ void store_chunk_bf16(const uint32_t (&pk)[16],
+                                                 __nv_bfloat16* out_row0, size_t ld, int nvalid,
+                                                 int lane) {
+  if (lane >= nvalid) return;
+  uint4* dst = reinterpret_cast<uint4*>(out_row0 + (size_t)lane * ld);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+}
+
+__device__ __forceinline__ void swiglu_pack(const uint32_t (&g)[32], const uint32_t (&u)[32],
+                                            uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+    const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+    pk[i] = pack_bf16x2(silu(g0) * u0, silu(g1) * u1);
+  }
+}
+
+__device__ __forceinline__ int clamp_rows(int v) { return v < 0 ? 0 : (v > 32 ? 32 : v); }
+
 template <int BN, bool SWIGLU>
 struct GemmCfg {
   static constexpr int kOutCols = SWIGLU ? BN / 2 : BN;  // output columns per tile
@@ -51,7 +95,8 @@ struct GemmCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (BN == 256) ? 4 : 6;
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  static constexpr int kStagingOff = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kStagingOff + 4 * kStageWords * 4 + 1024;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
 };
 
@@ -247,7 +292,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // -------------------------------------------------- epilogue (warps 2..5)
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
-    const int row_in_tile = q * 32 + lane;
     int lt = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
       int e, m, n;
@@ -260,47 +304,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int local_row = m * kBM + row_in_tile;
-      const bool valid = local_row < sh.row_cnt[e];
-      const size_t out_off =
-          (size_t)(sh.row_off[e] + local_row) * n_out + (size_t)n * Cfg::kOutCols;
+      const int nvalid = clamp_rows(sh.row_cnt[e] - (m * kBM + q * 32));
+      const size_t row0 = (size_t)sh.row_off[e] + m * kBM + q * 32;
+      uint32_t* stage = reinterpret_cast<uint32_t*>(smem + Cfg::kStagingOff) + q * kStageWords;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * BN);
       if (SWIGLU) {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out +
+                           (size_t)n * Cfg::kOutCols;
 #pragma unroll 1
         for (int c = 0; c < BN / 2 / 32; ++c) {
-          uint32_t g[32], u[32];
+          uint32_t g[32], u[32], pk[16];
           tmem_ld_32x32b_x32(tbase + c * 32, g);
           tmem_ld_32x32b_x32(tbase + BN / 2 + c * 32, u);
           tmem_ld_wait();
-          if (valid) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-              pk[i] = pack_bf16x2(silu(g0) * u0, silu(g1) * u1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(
-                static_cast<__nv_bfloat16*>(out_raw) + out_off + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
+          swiglu_pack(g, u, pk);
+          store_chunk_bf16(pk, o + c * 32, n_out, nvalid, lane);
         }
       } else {
+        float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * Cfg::kOutCols;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tbase + c * 32, v);
           tmem_ld_wait();
-          if (valid) {
-            // fp32 rows: the combine rounds to bf16 once, after the weighted sum
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(out_raw) + out_off + c * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          }
+          store_chunk_f32(v, stage, o + c * 32, n_out, nvalid, lane);
         }
       }
       tc_fence_before();
@@ -336,39 +364,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // For GEMM 1 each CTA then stages 64 gate + 64 up columns (CTA r: h-columns
 // [64r, 64r+64) of the tile), so every thread still holds g and u of the same
 // h-column.  This halves the rows computed in vain at each expert's tail.
-// Epilogue pieces: 32 accumulator columns of this thread's row.
-__device__ __forceinline__ void swiglu_chunk_store(uint32_t tg, uint32_t tu, bool valid,
-                                                   __nv_bfloat16* dst_row) {
-  uint32_t g[32], u[32];
+// Epilogue pieces of the pair kernel: 32 accumulator columns of 32 rows.
+__device__ __forceinline__ void swiglu_chunk_store(uint32_t tg, uint32_t tu,
+                                                   __nv_bfloat16* out_row0, size_t ld, int nvalid,
+                                                   int lane) {
+  uint32_t g[32], u[32], pk[16];
   tmem_ld_32x32b_x32(tg, g);
   tmem_ld_32x32b_x32(tu, u);
   tmem_ld_wait();
-  if (!valid) return;
-  uint32_t pk[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-    const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-    pk[i] = pack_bf16x2(silu(g0) * u0, silu(g1) * u1);
-  }
-  uint4* dst = reinterpret_cast<uint4*>(dst_row);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+  swiglu_pack(g, u, pk);
+  store_chunk_bf16(pk, out_row0, ld, nvalid, lane);
 }
 
-__device__ __forceinline__ void f32_chunk_store(uint32_t t, bool valid, float* dst_row) {
+__device__ __forceinline__ void f32_chunk_store(uint32_t t, uint32_t* stage, float* out_row0,
+                                                size_t ld, int nvalid, int lane) {
   uint32_t v[32];
   tmem_ld_32x32b_x32(t, v);
   tmem_ld_wait();
-  if (!valid) return;
-  uint4* dst = reinterpret_cast<uint4*>(dst_row);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  store_chunk_f32(v, stage, out_row0, ld, nvalid, lane);
 }
 
 constexpr int kPairStages = 6;
 constexpr int kPairStageBytes = 2 * kBM * kBK * 2;      // A 16 KB + half of B 16 KB
+constexpr int kPairStagingOff = kPairStages * kPairStageBytes;
 
 struct PairShared {
   uint64_t full_bar[kPairStages];
@@ -574,7 +592,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // -------------------------------------------------- epilogue (warps 2..5, both CTAs)
     const int q = warp & 3;
-    const int row_in_tile = q * 32 + lane;
     int lt = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++lt) {
       int e, m, n;
@@ -589,40 +606,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
+      uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kPairStagingOff) + q * kStageWords;
       if (!half) {
-        const int local_row = m * kPairM + (int)rank * kBM + row_in_tile;
-        const bool valid = local_row < sh.row_cnt[e];
-        const size_t out_off =
-            (size_t)(sh.row_off[e] + local_row) * n_out + (size_t)n * kOutCols;
+        const int first = m * kPairM + (int)rank * kBM + q * 32;   // first row of this warp
+        const int nvalid = clamp_rows(sh.row_cnt[e] - first);
+        const size_t row0 = (size_t)(sh.row_off[e] + first);
         if (SWIGLU) {
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out +
+                             (size_t)n * kOutCols;
 #pragma unroll 1
           for (int c = 0; c < 4; ++c)
-            swiglu_chunk_store(tbase + c * 32, tbase + 128 + c * 32, valid,
-                               static_cast<__nv_bfloat16*>(out_raw) + out_off + c * 32);
+            swiglu_chunk_store(tbase + c * 32, tbase + 128 + c * 32, o + c * 32, n_out, nvalid,
+                               lane);
         } else {
+          float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * kOutCols;
 #pragma unroll 1
           for (int c = 0; c < 8; ++c)
-            f32_chunk_store(tbase + c * 32, valid, static_cast<float*>(out_raw) + out_off + c * 32);
+            f32_chunk_store(tbase + c * 32, stage, o + c * 32, n_out, nvalid, lane);
         }
       } else {
         // lanes 0-63: accumulator columns [0,128); lanes 64-127: [128,256)
         const int hh = q >> 1;
-        const int local_row = m * kPairM + (int)rank * (kBM / 2) + (q & 1) * 32 + lane;
-        const bool valid = local_row < sh.row_cnt[e];
-        const size_t row_off = (size_t)(sh.row_off[e] + local_row) * n_out;
+        const int first = m * kPairM + (int)rank * (kBM / 2) + (q & 1) * 32;
+        const int nvalid = clamp_rows(sh.row_cnt[e] - first);
+        const size_t row0 = (size_t)(sh.row_off[e] + first);
         if (SWIGLU) {
           // this CTA's h-columns [64*rank ... ) of the tile: gate in TMEM
           // columns [0,64), up in [64,128); lanes 64-127 hold the next 64
           // columns of the tile (staged by the other half of B)
-          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row_off +
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out +
                              (size_t)n * kOutCols + hh * 64;
 #pragma unroll 1
           for (int c = 0; c < 2; ++c)
-            swiglu_chunk_store(tbase + c * 32, tbase + 64 + c * 32, valid, o + c * 32);
+            swiglu_chunk_store(tbase + c * 32, tbase + 64 + c * 32, o + c * 32, n_out, nvalid,
+                               lane);
         } else {
-          float* o = static_cast<float*>(out_raw) + row_off + (size_t)n * kOutCols + hh * 128;
+          float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * kOutCols + hh * 128;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) f32_chunk_store(tbase + c * 32, valid, o + c * 32);
+          for (int c = 0; c < 4; ++c)
+            f32_chunk_store(tbase + c * 32, stage, o + c * 32, n_out, nvalid, lane);
         }
       }
       tc_fence_before();
@@ -673,9 +695,7 @@ static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtens
                                     const CUtensorMap& b1, const int32_t* offsets, int E, int K,
                                     int n_out, int max_rows, void* out, int32_t* status,
                                     cudaStream_t s) {
-  // + 16 KB slack past the last stage, so the pair kernel's smem window also
-  // covers a full-width B read from the last stage
-  constexpr int kSmem = kPairStages * kPairStageBytes + 1024 + 16384;
+  constexpr int kSmem = kPairStagingOff + 4 * kStageWords * 4 + 1024;
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;

@@ -38,6 +38,7 @@ SMALL = [
     # buffers of >= 512 rows per expert select the CTA-pair GEMM tiles
     small("pair_tiles", T=2048, d=256, E=4, k=2, f=256, cf=0.0, seed=19),
     small("pair_tiles_drops", T=3000, d=512, E=4, k=3, f=384, cf=0.8, seed=20),
+    small("medium_buckets", T=1024, d=256, E=16, k=4, f=384, cf=1.25, seed=22),
 ]
 IDS = [c.name for c in SMALL]
 
@@ -133,7 +134,8 @@ def test_permute_matches_oracle(T, d, E, k, cf):
 MLP_CASES = [
     # (d, f, bucket sizes, pair): ragged tails, empty buckets, one-row buckets,
     # exact tile multiples, several row tiles; pair=True gives the buffer >= 512
-    # rows per expert, which selects the CTA-pair tiles (256 rows)
+    # rows per expert, which selects the CTA-pair tiles (256 rows); smaller
+    # buffers select the single-CTA 128-row tiles
     (256, 384, [300, 0, 1, 129, 128, 257], False),
     (128, 256, [5, 140, 0, 0, 64, 128], False),
     (384, 128, [1, 1, 1, 400], False),
@@ -142,6 +144,8 @@ MLP_CASES = [
     (256, 384, [300, 0, 1, 129, 128, 257, 700], True),
     (512, 256, [1, 256, 511, 513, 1024], True),
     (384, 256, [255, 257, 0], True),      # down GEMM: d % 256 != 0 keeps single-CTA tiles
+    (256, 256, [170, 0, 128, 129, 233, 256, 250, 131], False),
+    (384, 128, [300, 301, 15, 16], False),
 ]
 
 

@@ -419,6 +419,7 @@ __device__ __forceinline__ void decode_pair_tile(const PairShared& sh, int tile,
 template <bool SWIGLU>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
                              const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1,
                              const int32_t* __restrict__ offsets, int E, int K, int n_out,
@@ -460,6 +461,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   if (warp == 1 && lane == 0) {
     prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmA64);
     prefetch_tensormap(&tmB0);
     if (SWIGLU) prefetch_tensormap(&tmB1);
   }
@@ -524,8 +526,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = smem + s * kPairStageBytes;
           uint8_t* sb = sa + kBM * kBK * 2;
           const uint32_t full_lead = mapa_shared(&sh.full_bar[s], 0);
-          if (leader) mbar_arrive_expect_tx(&sh.full_bar[s], 2 * kPairStageBytes);
-          tma_load_2d_pair(sa, &tmA, full_lead, kb * kBK, row0);
+          // a half tile reads 64 rows of A per CTA (8 KB instead of 16 KB)
+          if (leader)
+            mbar_arrive_expect_tx(&sh.full_bar[s],
+                                  half ? 2 * (kPairStageBytes - kBM * kBK) : 2 * kPairStageBytes);
+          if (half)
+            tma_load_2d_pair(sa, &tmA64, full_lead, kb * kBK, row0);
+          else
+            tma_load_2d_pair(sa, &tmA, full_lead, kb * kBK, row0);
           if (SWIGLU && half) {
             tma_load_3d_pair(sb, &tmB0, full_lead, col0 + (int)rank * 64, kb * kBK, e);
             tma_load_3d_pair(sb + kChunkBytes, &tmB1, full_lead, col0 + (int)rank * 64, kb * kBK,
@@ -691,10 +699,10 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
 }
 
 template <bool SWIGLU>
-static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtensorMap& b0,
-                                    const CUtensorMap& b1, const int32_t* offsets, int E, int K,
-                                    int n_out, int max_rows, void* out, int32_t* status,
-                                    cudaStream_t s) {
+static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+                                    const CUtensorMap& b0, const CUtensorMap& b1,
+                                    const int32_t* offsets, int E, int K, int n_out, int max_rows,
+                                    void* out, int32_t* status, cudaStream_t s) {
   constexpr int kSmem = kPairStagingOff + 4 * kStageWords * 4 + 1024;
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
@@ -723,7 +731,8 @@ static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtens
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, offsets, E, K, n_out, max_rows, out, status);
+  return cudaLaunchKernelEx(&cfg, kern, a, a64, b0, b1, offsets, E, K, n_out, max_rows, out,
+                            status);
 }
 
 // Pair tiles (256 rows) pay off when buckets are large; the buffer's rows
@@ -739,8 +748,14 @@ cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, 
   *map_failed = !(map_rows(&ta, x_perm, d, max_rows, kBM) && map_weights(&tg, w_gate, E, d, f) &&
                   map_weights(&tu, w_up, E, d, f));
   if (*map_failed) return cudaSuccess;
-  if (use_pair_tiles(E, max_rows))
-    return launch_gemm_pair<true>(7, ta, tg, tu, offsets, E, d, f, max_rows, h, status, s);
+  if (use_pair_tiles(E, max_rows)) {
+    CUtensorMap ta64;
+    if (!map_rows(&ta64, x_perm, d, max_rows, kBM / 2)) {
+      *map_failed = true;
+      return cudaSuccess;
+    }
+    return launch_gemm_pair<true>(7, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s);
+  }
   return launch_gemm<256, true>(0, ta, tg, tu, offsets, E, d, f, max_rows, h, status, s);
 }
 
@@ -751,8 +766,15 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
   CUtensorMap ta, td;
   *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_weights(&td, w_down, E, f, d));
   if (*map_failed) return cudaSuccess;
-  if (d % 256 == 0 && use_pair_tiles(E, max_rows))
-    return launch_gemm_pair<false>(8, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);
+  if (d % 256 == 0 && use_pair_tiles(E, max_rows)) {
+    CUtensorMap ta64;
+    if (!map_rows(&ta64, h, f, max_rows, kBM / 2)) {
+      *map_failed = true;
+      return cudaSuccess;
+    }
+    return launch_gemm_pair<false>(8, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
+                                   s);
+  }
   if (d % 256 == 0)
     return launch_gemm<256, false>(1, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);
   return launch_gemm<128, false>(2, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);

@@ -15,6 +15,7 @@ Prints one JSON line on rank 0.
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -31,6 +32,12 @@ from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
 METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 9     # router 3, permute 3, gate/up GEMM 1, down GEMM 1, combine 1
+
+
+def moe_max_rows_host(cfg):
+    """min(T*k, E*C): the rows of the permuted buffers (decides the GEMM tiles)."""
+    C = cfg.T if cfg.cf == 0 else math.ceil(((cfg.cf * cfg.k) * cfg.T) / cfg.E)
+    return min(cfg.T * cfg.k, cfg.E * C)
 
 
 def peaks():
@@ -320,9 +327,15 @@ def host_weights(w):
 
 def calibrated_tokens(cfg, wh, xb, seconds):
     """Tokens whose oracle pass takes about `seconds` on this host: time a
-    2-token pass, scale, clamp to [2, T]."""
-    t2, _ = oracle_sample(cfg, wh, xb, 2)
-    return int(max(2, min(cfg.T, round(2 * seconds / max(t2, 1e-6)))))
+    small pass, scale, re-time once if far off; clamp to [2, T]."""
+    n = 8 if cfg.T >= 8 else cfg.T
+    for _ in range(3):
+        t, _ = oracle_sample(cfg, wh, xb, n)
+        want = int(max(2, min(cfg.T, round(n * seconds / max(t, 1e-6)))))
+        if t > 0.3 * seconds or want == n or n == cfg.T:
+            return want
+        n = min(want, max(n * 4, 2))
+    return n
 
 
 # ----------------------------------------------------------------- main
@@ -374,7 +387,15 @@ def main():
     gemm2_flop = 2.0 * r["N"] * cfg.d * cfg.f
     t_g1 = r["stage_ms"]["gate_up"] / 1e3
     t_g2 = r["stage_ms"]["down"] / 1e3
-    peak_tf = pk["bf16_tflops"]
+    # a kernel timed inside a long run under the power cap is compared with
+    # the sustained peak, otherwise with the burst peak
+    capped = "sw_power_cap" in (r["clocks"].get("reasons") or [])
+    peak_tf = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
+    peak_src = f"{pk_kind} bf16 {'sustained (power cap active)' if capped else 'burst'}"
+    pair = moe_max_rows_host(cfg) >= 512 * cfg.E
+    kname = ("grouped_gemm_pair_kernel<true> (gate/up + SwiGLU, CTA pairs)" if pair else
+             "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")
+    ktag = "gemm_pair_gate_up" if pair else "gemm_gate_up"
     achieved = gemm1_flop / t_g1 / 1e12
     # bytes the gate/up GEMM must move: weights of the experts that got rows,
     # x_perm rows in, h rows out
@@ -403,19 +424,20 @@ def main():
                    "parallelism": f"replicas x{world} (token batches, no collective)",
                    "l2": "inputs larger than L2 (expert weights "
                          f"{3 * cfg.E * cfg.d * cfg.f * 2 / 1e9:.1f} GB); no flush"},
-        "roofline": ({"kernel": "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)",
+        "roofline": ({"kernel": kname,
                       "bound": "tensor", "achieved": round(achieved, 1),
                       "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
-                      "peak_source": f"{pk_kind} bf16 burst",
-                      "traffic": traffic_from_profile("gemm_gate_up", cfg.name)}
+                      "peak_source": peak_src,
+                      "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4),
+                      "traffic": traffic_from_profile(ktag, cfg.name)}
                      if not hbm_bound else
-                     {"kernel": "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)",
+                     {"kernel": kname,
                       "bound": "hbm", "achieved": round(g1_bytes / t_g1 / 1e9, 1),
                       "peak": pk["hbm_gbs"], "unit": "GB/s",
                       "frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
                       "peak_source": f"{pk_kind} HBM copy",
                       "algorithmic_bytes": g1_bytes, "active_experts": A,
-                      "traffic": traffic_from_profile("gemm_gate_up", cfg.name)}),
+                      "traffic": traffic_from_profile(ktag, cfg.name)}),
         "stages_ms": {k_: round(v, 4) for k_, v in r["stage_ms"].items()},
         "stage_rooflines": {
             "down_gemm": {"bound": "tensor", "achieved": round(gemm2_flop / t_g2 / 1e12, 1),

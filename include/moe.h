@@ -58,6 +58,14 @@ const char* moe_status_string(int status);
 /* Library ABI version, (major << 16) | minor. */
 int moe_version(void);
 
+/* Self-test of the kernels' time-limited waits (no counterpart on the pages):
+ * launches one CTA that waits, with the same bounded mbarrier wait the GEMM
+ * kernels use, on a barrier nothing arrives at, for at most limit_ns
+ * (0 .. 10 s), then ORs the wait-timeout bit (1) into *dev_status (device
+ * int32).  A caller can check that a wait that cannot complete ends with a
+ * status word instead of a hang, and that the context stays usable. */
+int moe_selftest_bounded_wait(int32_t* dev_status, int64_t limit_ns, void* stream);
+
 /* Expert capacity, step "capacity" above: ceil(((cf*k)*T)/E) evaluated in
  * fp64; cf == 0 selects the dropless layer and returns T.  Source: the
  * capacity-factor entry of the inferensys.com glossary and section "Why

@@ -25,7 +25,8 @@ DEV_ERR_BAD_OFFSETS = 2
 WS_FIELDS = ["status", "logits", "topk_idx", "topk_w", "slot", "counts", "offsets", "n_dropped",
              "row_src", "permute", "x_perm", "h", "y_perm", "route"]
 
-EXPORTED = ["moe_status_string", "moe_version", "moe_capacity", "moe_max_rows",
+EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "moe_capacity",
+            "moe_max_rows",
             "moe_route_workspace_size", "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
             "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
             "moe_combine", "moe_layer_forward"]
@@ -46,6 +47,7 @@ def _load():
     sig = {
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_version": (ctypes.c_int, []),
+        "moe_selftest_bounded_wait": (ctypes.c_int, [p, i64, p]),
         "moe_capacity": (i64, [i64, i64, i64, dbl]),
         "moe_max_rows": (i64, [i64, i64, i64, dbl]),
         "moe_route_workspace_size": (sz, [i64, i64, i64, i64]),
@@ -135,6 +137,13 @@ def moe_workspace_field_offset(field, T, d, E, k, f, cf):
 
 def moe_version():
     return int(_lib.moe_version())
+
+
+def moe_selftest_bounded_wait(dev_status, limit_ns, stream=None):
+    """Run the bounded-wait self-test kernel (see include/moe.h)."""
+    _want(dev_status, "dev_status", torch.int32, (1,))
+    _check("moe_selftest_bounded_wait",
+           _lib.moe_selftest_bounded_wait(_ptr(dev_status), int(limit_ns), _stream(stream)))
 
 
 def moe_status_string(status):

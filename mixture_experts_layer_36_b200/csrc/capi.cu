@@ -28,6 +28,23 @@ cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            cudaStream_t s);
 }  // namespace moe
 
+namespace moe {
+// One CTA waits, with the kernels' time-limited wait, on an mbarrier that
+// nothing arrives at; on expiry it reports like the GEMM kernels do.
+__global__ void selftest_wait_kernel(int32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, limit_ns))
+    report(status, kDevErrWaitTimeout);
+}
+}  // namespace moe
+
 using moe::launch_combine;
 using moe::launch_down;
 using moe::launch_gate_up;
@@ -100,6 +117,12 @@ const char* moe_status_string(int status) {
 }
 
 int moe_version(void) { return (1 << 16) | 0; }
+
+int moe_selftest_bounded_wait(int32_t* dev_status, int64_t limit_ns, void* stream) {
+  if (!dev_status || limit_ns < 0 || limit_ns > 10000000000LL) return MOE_ERR_INVALID_ARG;
+  moe::selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(dev_status, (uint64_t)limit_ns);
+  return cuda_status(cudaGetLastError());
+}
 
 int64_t moe_capacity(int64_t T, int64_t E, int64_t k, double cf) {
   if (T < 0 || E < 1 || k < 1 || !(cf >= 0.0) || isinf(cf)) return -1;

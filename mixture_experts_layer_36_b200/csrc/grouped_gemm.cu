@@ -98,6 +98,7 @@ struct GemmCfg {
   static constexpr int kStagingOff = kStages * kStageBytes;
   static constexpr int kSmemBytes = kStagingOff + 4 * kStageWords * 4 + 1024;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
+  static constexpr uint32_t kIdesc64 = idesc_bf16_f32(kBM / 2, BN, /*b_mn_major=*/true);
 };
 
 struct GemmShared {
@@ -131,6 +132,7 @@ __device__ __forceinline__ void decode_tile(const GemmShared& sh, int tile, int 
 template <int BN, bool SWIGLU>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1,
                         const int32_t* __restrict__ offsets, int E, int K, int n_out,
@@ -165,6 +167,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   if (warp == 1 && lane == 0) {
     prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmA64);
     prefetch_tensormap(&tmB0);
     if (SWIGLU) prefetch_tensormap(&tmB1);
   }
@@ -216,14 +219,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         decode_tile(sh, tile, E, n_tiles, e, m, n);
         const int row0 = sh.row_off[e] + m * kBM;
         const int col0 = n * Cfg::kOutCols;
+        const bool small = sh.row_cnt[e] - m * kBM <= kBM / 2;   // M = 64 tile
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % Cfg::kStages;
           const uint32_t ph = (it / Cfg::kStages) & 1;
           if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
           uint8_t* sa = smem + s * Cfg::kStageBytes;
           uint8_t* sb = sa + Cfg::kABytes;
-          mbar_arrive_expect_tx(&sh.full_bar[s], Cfg::kStageBytes);
-          tma_load_2d(sa, &tmA, &sh.full_bar[s], kb * kBK, row0);
+          mbar_arrive_expect_tx(&sh.full_bar[s],
+                                small ? Cfg::kStageBytes - Cfg::kABytes / 2 : Cfg::kStageBytes);
+          if (small)
+            tma_load_2d(sa, &tmA64, &sh.full_bar[s], kb * kBK, row0);
+          else
+            tma_load_2d(sa, &tmA, &sh.full_bar[s], kb * kBK, row0);
           if (SWIGLU) {
 #pragma unroll
             for (int c = 0; c < BN / 128; ++c)
@@ -255,6 +263,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0, lt = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++lt) {
+        int e, m, n;
+        decode_tile(sh, tile, E, n_tiles, e, m, n);
+        const uint32_t idesc = (sh.row_cnt[e] - m * kBM <= kBM / 2) ? Cfg::kIdesc64 : Cfg::kIdesc;
         const int a = lt & 1;
         const uint32_t aph = (lt >> 1) & 1;
         if (!mbar_wait(&sh.tempty_bar[a], aph ^ 1, abort_flag)) { ok = false; break; }
@@ -274,7 +285,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // B: MN-major; 64-wide N chunks 8 KB apart (LBO), 8-row K groups
             // 1024 B apart (SBO); +16 K rows = +2048 B per K step
             const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, kChunkBytes, 1024);
-            umma_bf16(d_tmem, adesc, bdesc, Cfg::kIdesc, (kb | ks) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
           }
           umma_commit(&sh.empty_bar[s]);
         }
@@ -304,8 +315,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int nvalid = clamp_rows(sh.row_cnt[e] - (m * kBM + q * 32));
-      const size_t row0 = (size_t)sh.row_off[e] + m * kBM + q * 32;
+      // M = 64 tiles put rows 16q..16q+15 in TMEM lanes 32q..32q+15
+      const bool small = sh.row_cnt[e] - m * kBM <= kBM / 2;
+      const int rows_per_warp = small ? 16 : 32;
+      const int first = m * kBM + q * rows_per_warp;
+      int nvalid = clamp_rows(sh.row_cnt[e] - first);
+      if (nvalid > rows_per_warp) nvalid = rows_per_warp;
+      const size_t row0 = (size_t)sh.row_off[e] + first;
       uint32_t* stage = reinterpret_cast<uint32_t*>(smem + Cfg::kStagingOff) + q * kStageWords;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * BN);
@@ -673,8 +689,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ---------------------------------------------------------------- host side
 
 template <int BN, bool SWIGLU>
-static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& b0,
-                               const CUtensorMap& b1, const int32_t* offsets, int E, int K,
+static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+                               const CUtensorMap& b0, const CUtensorMap& b1,
+                               const int32_t* offsets, int E, int K,
                                int n_out, int max_rows, void* out, int32_t* status,
                                cudaStream_t s) {
   using Cfg = GemmCfg<BN, SWIGLU>;
@@ -693,8 +710,8 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
   long long ub = row_tiles * n_tiles;
   int grid = (int)(ub < di->sms ? ub : di->sms);
   if (grid < 1) grid = 1;
-  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, b0, b1, offsets, E, K, n_out, max_rows,
-                                                     out, status);
+  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, offsets, E, K, n_out,
+                                                     max_rows, out, status);
   return cudaGetLastError();
 }
 
@@ -744,40 +761,32 @@ cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, 
                            int f, int max_rows, const __nv_bfloat16* w_gate,
                            const __nv_bfloat16* w_up, __nv_bfloat16* h, int32_t* status,
                            cudaStream_t s, bool* map_failed) {
-  CUtensorMap ta, tg, tu;
-  *map_failed = !(map_rows(&ta, x_perm, d, max_rows, kBM) && map_weights(&tg, w_gate, E, d, f) &&
-                  map_weights(&tu, w_up, E, d, f));
+  CUtensorMap ta, ta64, tg, tu;
+  *map_failed = !(map_rows(&ta, x_perm, d, max_rows, kBM) &&
+                  map_rows(&ta64, x_perm, d, max_rows, kBM / 2) &&
+                  map_weights(&tg, w_gate, E, d, f) && map_weights(&tu, w_up, E, d, f));
   if (*map_failed) return cudaSuccess;
-  if (use_pair_tiles(E, max_rows)) {
-    CUtensorMap ta64;
-    if (!map_rows(&ta64, x_perm, d, max_rows, kBM / 2)) {
-      *map_failed = true;
-      return cudaSuccess;
-    }
+  if (use_pair_tiles(E, max_rows))
     return launch_gemm_pair<true>(7, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s);
-  }
-  return launch_gemm<256, true>(0, ta, tg, tu, offsets, E, d, f, max_rows, h, status, s);
+  return launch_gemm<256, true>(0, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s);
 }
 
 // GEMM 2: y_perm = h Wd
 cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
                         int max_rows, const __nv_bfloat16* w_down, float* y_perm,
                         int32_t* status, cudaStream_t s, bool* map_failed) {
-  CUtensorMap ta, td;
-  *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_weights(&td, w_down, E, f, d));
+  CUtensorMap ta, ta64, td;
+  *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_rows(&ta64, h, f, max_rows, kBM / 2) &&
+                  map_weights(&td, w_down, E, f, d));
   if (*map_failed) return cudaSuccess;
-  if (d % 256 == 0 && use_pair_tiles(E, max_rows)) {
-    CUtensorMap ta64;
-    if (!map_rows(&ta64, h, f, max_rows, kBM / 2)) {
-      *map_failed = true;
-      return cudaSuccess;
-    }
+  if (d % 256 == 0 && use_pair_tiles(E, max_rows))
     return launch_gemm_pair<false>(8, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
                                    s);
-  }
   if (d % 256 == 0)
-    return launch_gemm<256, false>(1, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);
-  return launch_gemm<128, false>(2, ta, td, td, offsets, E, f, d, max_rows, y_perm, status, s);
+    return launch_gemm<256, false>(1, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
+                                   s);
+  return launch_gemm<128, false>(2, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
+                                 s);
 }
 
 int device_sm_count() {

@@ -31,7 +31,7 @@ from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
 
 METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 9     # router 3, permute 3, gate/up GEMM 1, down GEMM 1, combine 1
+KERNELS_PER_STEP = 8     # router 3, permute 2, gate/up GEMM 1, down GEMM 1, combine 1
 
 
 def moe_max_rows_host(cfg):

@@ -8,38 +8,50 @@
 //
 // slot(t, j) = number of tokens t' < t that also chose expert e = topk_idx[t,j]
 // (each expert appears at most once per token).  This is a stable counting
-// sort keyed by expert, done in three launches:
+// sort keyed by expert, done in two launches:
 //   1. rank:    per chunk of 256 tokens, the rank of each pair among the
 //               chunk's pairs of the same expert (token order), plus the
 //               chunk's per-expert histogram;
-//   2. scan:    per expert, exclusive prefix of the histograms over chunks
-//               (chunk bases), demand, kept = min(demand, C), offsets,
-//               dropped-pair count;
-//   3. scatter: slot = chunk base + rank; kept pairs copy their token row into
-//               x_perm[offsets[e] + slot] with 16-byte vector loads/stores.
+//   2. scan + scatter: each CTA sums the histograms into per-expert demand,
+//               kept = min(demand, C), offsets (exclusive scan over experts)
+//               and its chunk's base (prefix over earlier chunks); then
+//               slot = chunk base + rank, and kept pairs copy their token row
+//               into x_perm[offsets[e] + slot] with 16-byte vector loads and
+//               stores.
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kChunk = 256;          // tokens per rank/histogram chunk
-constexpr int kPermThreads = 256;    // 8 warps, 32 tokens each
+constexpr int kChunk = 256;            // tokens per rank/histogram chunk
+constexpr int kRankThreads = 1024;     // 32 warps x 8 tokens per chunk
+constexpr int kRankWarps = kRankThreads / 32;
+constexpr int kTokPerWarp = kChunk / kRankWarps;
+constexpr int kScatThreads = 256;      // 8 warps
+// tokens per scatter CTA (a divisor of kChunk): 8 (one per warp) keeps small
+// batches spread over many SMs; 32 (four per warp) when every CTA's pass over
+// the chunk histograms (nchunks x E counters) would be long
+constexpr int kScatTokensSmall = 8;
+constexpr int kScatTokensLarge = 32;
 
-__global__ void __launch_bounds__(kPermThreads)
+// 1. rank: per chunk, the rank of each pair among the chunk's pairs of the
+//    same expert (token order), and the chunk's per-expert histogram.
+__global__ void __launch_bounds__(kRankThreads)
     permute_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
                         int32_t* __restrict__ rank, int32_t* __restrict__ chunk_hist) {
-  __shared__ int32_t cnt[kPermThreads / 32][256];
+  __shared__ int32_t cnt[kRankWarps][256];
   __shared__ int32_t pairs[kChunk * 8];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int chunk_t0 = blockIdx.x * kChunk;
   const int nt = min(kChunk, T - chunk_t0);
 
-  for (int i = tid; i < (kPermThreads / 32) * 256; i += kPermThreads) (&cnt[0][0])[i] = 0;
-  for (int i = tid; i < nt * k; i += kPermThreads) pairs[i] = topk_idx[(size_t)chunk_t0 * k + i];
+  for (int i = tid; i < kRankWarps * 256; i += kRankThreads) (&cnt[0][0])[i] = 0;
+  for (int i = tid; i < nt * k; i += kRankThreads) pairs[i] = topk_idx[(size_t)chunk_t0 * k + i];
   __syncthreads();
 
-  // each warp walks its 32 tokens in order; lane j handles pair j
-  const int w_t0 = warp * 32;
-  for (int i = 0; i < 32; ++i) {
+  // each warp walks its 8 tokens in order; lane j handles pair j
+  const int w_t0 = warp * kTokPerWarp;
+#pragma unroll
+  for (int i = 0; i < kTokPerWarp; ++i) {
     const int tt = w_t0 + i;
     if (tt < nt && lane < k) {
       const int e = pairs[tt * k + lane];
@@ -52,10 +64,10 @@ __global__ void __launch_bounds__(kPermThreads)
   __syncthreads();
 
   // per expert: exclusive prefix over the warps, chunk total to global
-  for (int e = tid; e < E; e += kPermThreads) {
+  for (int e = tid; e < E; e += kRankThreads) {
     int run = 0;
-#pragma unroll
-    for (int w = 0; w < kPermThreads / 32; ++w) {
+#pragma unroll 8
+    for (int w = 0; w < kRankWarps; ++w) {
       const int c = cnt[w][e];
       cnt[w][e] = run;
       run += c;
@@ -64,34 +76,47 @@ __global__ void __launch_bounds__(kPermThreads)
   }
   __syncthreads();
 
-  // shift each pair's in-warp rank by its warp's base
-  for (int i = tid; i < nt * k; i += kPermThreads) {
+  for (int i = tid; i < nt * k; i += kRankThreads) {
     const int tt = i / k;
-    const int e = pairs[i];
-    rank[(size_t)chunk_t0 * k + i] += cnt[tt / 32][e];
+    rank[(size_t)chunk_t0 * k + i] += cnt[tt / kTokPerWarp][pairs[i]];
   }
 }
 
-// One CTA of 256 threads, thread e owns expert e.
-__global__ void __launch_bounds__(256)
-    permute_scan_kernel(int32_t* __restrict__ chunk_hist, int nchunks, int E, int64_t C,
-                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                        int32_t* __restrict__ n_dropped) {
+// 2. scan + scatter: every CTA derives, from all chunk histograms, the
+//    per-expert kept counts and offsets (exclusive scan over experts) and its
+//    own chunk's per-expert base (exclusive prefix over earlier chunks); CTA 0
+//    also writes counts / offsets / n_dropped.  Then one warp per token turns
+//    ranks into slots, drops pairs at slot >= C, and copies the token row to
+//    its kept rows with 16-byte vectors.
+__global__ void __launch_bounds__(kScatThreads)
+    permute_scatter_kernel(const __nv_bfloat16* __restrict__ x,
+                           const int32_t* __restrict__ topk_idx, int32_t* __restrict__ slot,
+                           const int32_t* __restrict__ chunk_hist, int nchunks, int T, int d,
+                           int E, int k, int64_t C, int tokens_per_cta,
+                           int32_t* __restrict__ counts,
+                           int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped,
+                           int32_t* __restrict__ row_src, __nv_bfloat16* __restrict__ x_perm) {
+  __shared__ int32_t s_off[256];
+  __shared__ int32_t s_base[256];
   __shared__ int32_t warp_sum[8];
   __shared__ int32_t warp_drop[8];
-  const int e = threadIdx.x, lane = e % 32, warp = e / 32;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int t0 = blockIdx.x * tokens_per_cta;
+  const int my_chunk = t0 / kChunk;
+
+  // ---- per-expert totals, kept, chunk base (thread e owns expert e)
   int kept = 0, drop = 0;
-  if (e < E) {
-    int run = 0;
+  if (tid < E) {
+    int total = 0, base = 0;
     for (int c = 0; c < nchunks; ++c) {
-      const int v = chunk_hist[(size_t)c * E + e];
-      chunk_hist[(size_t)c * E + e] = run;
-      run += v;
+      const int v = chunk_hist[(size_t)c * E + tid];
+      if (c < my_chunk) base += v;
+      total += v;
     }
-    kept = (int64_t)run < C ? run : (int)C;
-    drop = run - kept;
+    kept = (int64_t)total < C ? total : (int)C;
+    drop = total - kept;
+    s_base[tid] = base;
   }
-  // block exclusive scan of kept, block sum of drop
   int incl = kept;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -104,68 +129,65 @@ __global__ void __launch_bounds__(256)
   if (lane == 31) warp_sum[warp] = incl;
   if (lane == 0) warp_drop[warp] = dsum;
   __syncthreads();
-  int base = 0, total = 0, dtotal = 0;
+  int wbase = 0, total_rows = 0, dtotal = 0;
 #pragma unroll
   for (int w = 0; w < 8; ++w) {
-    if (w < warp) base += warp_sum[w];
-    total += warp_sum[w];
+    if (w < warp) wbase += warp_sum[w];
+    total_rows += warp_sum[w];
     dtotal += warp_drop[w];
   }
-  if (e < E) {
-    counts[e] = kept;
-    offsets[e] = base + incl - kept;
-  }
-  if (e == 0) {
-    offsets[E] = total;
-    *n_dropped = dtotal;
-  }
-}
-
-// One warp per token.
-__global__ void __launch_bounds__(kPermThreads)
-    permute_scatter_kernel(const __nv_bfloat16* __restrict__ x,
-                           const int32_t* __restrict__ topk_idx, int32_t* __restrict__ slot,
-                           const int32_t* __restrict__ chunk_base,
-                           const int32_t* __restrict__ offsets, int T, int d, int E, int k,
-                           int64_t C, int32_t* __restrict__ row_src,
-                           __nv_bfloat16* __restrict__ x_perm) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int t = blockIdx.x * (kPermThreads / 32) + warp;
-  if (t >= T) return;
-  int my_row = -1;
-  if (lane < k) {
-    const size_t p = (size_t)t * k + lane;
-    const int e = topk_idx[p];
-    const int s = chunk_base[(size_t)(t / kChunk) * E + e] + slot[p];   // slot holds the rank
-    const bool keep = (int64_t)s < C;
-    slot[p] = keep ? s : -1;
-    if (keep) {
-      my_row = offsets[e] + s;
-      row_src[my_row] = t;
+  if (tid < E) s_off[tid] = wbase + incl - kept;
+  if (blockIdx.x == 0) {
+    if (tid < E) {
+      counts[tid] = kept;
+      offsets[tid] = wbase + incl - kept;
+    }
+    if (tid == 0) {
+      offsets[E] = total_rows;
+      *n_dropped = dtotal;
     }
   }
-  int rows[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+  __syncthreads();
 
+  // ---- one warp per token
   const int nvec = d / 8;
-  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-  for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
-    uint4 val[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int v = v0 + u * 32;
-      if (v < nvec) val[u] = __ldg(src + v);
+  for (int tt = warp; tt < tokens_per_cta; tt += kScatThreads / 32) {
+    const int t = t0 + tt;
+    if (t >= T) break;
+    int my_row = -1;
+    if (lane < k) {
+      const size_t p = (size_t)t * k + lane;
+      const int e = topk_idx[p];
+      const int sl = s_base[e] + slot[p];          // slot holds the in-chunk rank
+      const bool keep = (int64_t)sl < C;
+      slot[p] = keep ? sl : -1;
+      if (keep) {
+        my_row = s_off[e] + sl;
+        row_src[my_row] = t;
+      }
     }
+    int rows[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j >= k) break;
-      if (rows[j] < 0) continue;
-      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)rows[j] * d);
+    for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
+      uint4 val[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int v = v0 + u * 32;
-        if (v < nvec) dst[v] = val[u];
+        if (v < nvec) val[u] = __ldg(src + v);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j >= k) break;
+        if (rows[j] < 0) continue;
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)rows[j] * d);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + u * 32;
+          if (v < nvec) dst[v] = val[u];
+        }
       }
     }
   }
@@ -181,11 +203,11 @@ cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int 
                            int32_t* row_src, __nv_bfloat16* x_perm, int32_t* n_dropped,
                            int32_t* chunk_hist, cudaStream_t s) {
   const int nchunks = (T + kChunk - 1) / kChunk;
-  permute_rank_kernel<<<nchunks, kPermThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist);
-  permute_scan_kernel<<<1, 256, 0, s>>>(chunk_hist, nchunks, E, C, counts, offsets, n_dropped);
-  const int tokens_per_cta = kPermThreads / 32;
-  permute_scatter_kernel<<<(T + tokens_per_cta - 1) / tokens_per_cta, kPermThreads, 0, s>>>(
-      x, topk_idx, slot, chunk_hist, offsets, T, d, E, k, C, row_src, x_perm);
+  permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist);
+  const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
+  permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
+      x, topk_idx, slot, chunk_hist, nchunks, T, d, E, k, C, tpc, counts, offsets, n_dropped,
+      row_src, x_perm);
   return cudaGetLastError();
 }
 

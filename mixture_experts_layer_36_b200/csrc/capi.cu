@@ -217,7 +217,12 @@ static int check_gemm_args(int64_t E, int64_t d, int64_t f, int64_t max_rows) {
     return MOE_ERR_INVALID_ARG;
   int st = check_width(d);
   if (st != MOE_OK) return st;
-  return check_width(f);
+  if ((st = check_width(f)) != MOE_OK) return st;
+  // the kernels count tiles in 32-bit integers: (row tiles) x (column tiles)
+  const int64_t row_tiles = max_rows / 64 + E;
+  const int64_t col_tiles = (d > f ? d : f) / 64;
+  if (row_tiles * col_tiles >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
 }
 
 int moe_expert_gate_up(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d,

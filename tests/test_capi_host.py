@@ -102,6 +102,9 @@ def test_validation_codes_without_launch():
     assert L.moe_expert_down(FAKE, FAKE, 8, 256, 200, 100, FAKE, FAKE, None, s) == UNSUPPORTED
     assert L.moe_expert_mlp(FAKE, FAKE, 8, 256, 256, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None, s) \
         == OK
+    # tile counts that would overflow the kernels' 32-bit tile indices
+    assert L.moe_expert_gate_up(FAKE, FAKE, 8, 1 << 20, 1 << 20, (1 << 31) - 1, FAKE, FAKE, FAKE,
+                                None, s) == UNSUPPORTED
     # combine / layer
     assert L.moe_combine(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10, 128, 9, FAKE, s) == INVALID
     ws_need = moe.moe_workspace_size(64, 128, 8, 2, 256, 1.25)

@@ -142,13 +142,19 @@ class Layer:
     """Inputs, weights and buffers of one workload, resident on the device,
     and the step as five C-ABI calls on one stream."""
 
-    def __init__(self, cfg, device, token_seed):
+    def __init__(self, cfg, device, token_seed, fp8=False):
         import mixture_experts_layer_36_b200 as moe
         self.moe = moe
         self.cfg = cfg
         self.dev = device
         w = synth.make_weights(cfg, device)
         self.w = w
+        self.fp8 = fp8
+        if fp8:
+            # one-time preprocessing, outside any timed region: e4m3 codes and
+            # per-column scales of the expert weights
+            self.q = {n: moe.moe_quantize_weights_fp8(w[n]) for n in ("w_gate", "w_up", "w_down")}
+            torch.cuda.synchronize(device)
         self.x = synth.make_tokens(cfg, device, seed=token_seed)
         T, d, E, k, f = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f
         self.rows = moe.moe_max_rows(T, E, k, cfg.cf)
@@ -180,12 +186,20 @@ class Layer:
         m.moe_permute(self.x, self.idx, c.E, c.cf, out=self.perm, ws=self.pws)
         if ev:
             ev[2].record()
-        m.moe_expert_gate_up(self.perm["x_perm"], self.perm["offsets"], w["w_gate"], w["w_up"],
-                             h=self.h, dev_status=self.status)
+        if self.fp8:
+            m.moe_expert_gate_up_fp8(self.perm["x_perm"], self.perm["offsets"], *self.q["w_gate"],
+                                     *self.q["w_up"], h=self.h, dev_status=self.status)
+        else:
+            m.moe_expert_gate_up(self.perm["x_perm"], self.perm["offsets"], w["w_gate"],
+                                 w["w_up"], h=self.h, dev_status=self.status)
         if ev:
             ev[3].record()
-        m.moe_expert_down(self.h, self.perm["offsets"], w["w_down"], y_perm=self.y_perm,
-                          dev_status=self.status)
+        if self.fp8:
+            m.moe_expert_down_fp8(self.h, self.perm["offsets"], *self.q["w_down"],
+                                  y_perm=self.y_perm, dev_status=self.status)
+        else:
+            m.moe_expert_down(self.h, self.perm["offsets"], w["w_down"], y_perm=self.y_perm,
+                              dev_status=self.status)
         if ev:
             ev[4].record()
         m.moe_combine(self.y_perm, self.x, self.idx, self.tw, self.perm["slot"],
@@ -195,6 +209,11 @@ class Layer:
 
     def layer_forward(self, x, y):
         w, c = self.w, self.cfg
+        if self.fp8:
+            q = self.q
+            self.moe.moe_layer_forward_fp8(x, w["w_router"], w["bias"], *q["w_gate"], *q["w_up"],
+                                           *q["w_down"], c.k, c.cf, y=y, ws=self.ws)
+            return
         self.moe.moe_layer_forward(x, w["w_router"], w["bias"], w["w_gate"], w["w_up"],
                                    w["w_down"], c.k, c.cf, y=y, ws=self.ws)
 
@@ -205,7 +224,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     dist = world > 1
     if dist:
         import torch.distributed as td
-    layer = Layer(cfg, dev, token_seed=rank_token_seed(cfg, rank))
+    layer = Layer(cfg, dev, token_seed=rank_token_seed(cfg, rank), fp8=args.fp8)
     stream = torch.cuda.current_stream()
 
     K = args.steps
@@ -348,6 +367,9 @@ def main():
     ap.add_argument("--config", default="mixtral")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="expert weights as e4m3 codes + fp32 column scales (quantized once "
+                         "before timing); activations and accumulation as in the bf16 path")
     ap.add_argument("--profile", action="store_true",
                     help="run W + K layer steps only (no timing, e2e or oracle): a short, "
                          "fixed launch sequence for ncu")
@@ -363,7 +385,8 @@ def main():
     if args.impl == "reference":
         return reference_arm(args, cfg, rank, world)
     if args.profile:
-        layer = Layer(cfg, torch.device("cuda", local_rank), token_seed=rank_token_seed(cfg, 0))
+        layer = Layer(cfg, torch.device("cuda", local_rank), token_seed=rank_token_seed(cfg, 0),
+                      fp8=args.fp8)
         for _ in range(args.warmup + args.steps):
             layer.step()
         torch.cuda.synchronize()
@@ -392,16 +415,22 @@ def main():
     capped = "sw_power_cap" in (r["clocks"].get("reasons") or [])
     peak_tf = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
     peak_src = f"{pk_kind} bf16 {'sustained (power cap active)' if capped else 'burst'}"
-    pair = moe_max_rows_host(cfg) >= 512 * cfg.E
+    pair = moe_max_rows_host(cfg) >= 512 * cfg.E and not args.fp8
     kname = ("grouped_gemm_pair_kernel<true> (gate/up + SwiGLU, CTA pairs)" if pair else
-             "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")
-    ktag = "gemm_pair_gate_up" if pair else "gemm_gate_up"
+             "grouped_gemm_kernel<256,true,true> (gate/up + SwiGLU, e4m3 weights)" if args.fp8
+             else "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")
+    ktag = "gemm_pair_gate_up" if pair else "gemm_fp8_gate_up" if args.fp8 else "gemm_gate_up"
     achieved = gemm1_flop / t_g1 / 1e12
     # bytes the gate/up GEMM must move: weights of the experts that got rows,
     # x_perm rows in, h rows out
     A = r["active_experts"]
-    g1_bytes = A * 2.0 * cfg.d * cfg.f * 2 + r["N"] * cfg.d * 2 + r["N"] * cfg.f * 2
-    g2_bytes = A * 1.0 * cfg.d * cfg.f * 2 + r["N"] * cfg.f * 2 + r["N"] * cfg.d * 4
+    # weight bytes per element: bf16 2; e4m3 1 plus a 4-byte scale per column
+    wb = 1 if args.fp8 else 2
+    g1_bytes = A * 2.0 * cfg.d * cfg.f * wb + r["N"] * cfg.d * 2 + r["N"] * cfg.f * 2
+    g2_bytes = A * 1.0 * cfg.d * cfg.f * wb + r["N"] * cfg.f * 2 + r["N"] * cfg.d * 4
+    if args.fp8:
+        g1_bytes += A * 2.0 * cfg.f * 4
+        g2_bytes += A * 1.0 * cfg.d * 4
     ridge = peak_tf * 1e12 / (pk["hbm_gbs"] * 1e9)
     hbm_bound = gemm1_flop / g1_bytes < ridge
     bytes_perm = cfg.T * cfg.d * 2 + r["N"] * cfg.d * 2
@@ -417,13 +446,14 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16 (e4m3 expert weights)" if args.fp8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the named shape)",
         "config": {"workload": describe(cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
                    "f": cfg.f, "cf": cfg.cf, "kept_pairs": r["N"], "dropped_pairs": r["n_dropped"],
                    "parallelism": f"replicas x{world} (token batches, no collective)",
+                   "expert_weights": "e4m3 + fp32 column scales" if args.fp8 else "bf16",
                    "l2": "inputs larger than L2 (expert weights "
-                         f"{3 * cfg.E * cfg.d * cfg.f * 2 / 1e9:.1f} GB); no flush"},
+                         f"{3 * cfg.E * cfg.d * cfg.f * wb / 1e9:.1f} GB); no flush"},
         "roofline": ({"kernel": kname,
                       "bound": "tensor", "achieved": round(achieved, 1),
                       "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
@@ -460,8 +490,9 @@ def main():
         "clocks": {k_: r["clocks"][k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},
         "e2e": {"value": round(cfg.T * world * K / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-                "api": "moe_layer_forward (one-shot C-ABI call); every step copies x from pinned "
-                       "host memory and y back, on copy streams overlapping adjacent steps' compute"},
+                "api": ("moe_layer_forward_fp8" if args.fp8 else "moe_layer_forward") +
+                       " (one-shot C-ABI call); every step copies x from pinned host memory and "
+                       "y back, on copy streams overlapping adjacent steps' compute"},
         "gpu_launches": KERNELS_PER_STEP * K,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -219,6 +219,40 @@ int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, con
                 const int32_t* slot, const int32_t* offsets, int64_t T, int64_t d, int64_t k,
                 void* y, void* stream);
 
+/* ---- FP8 expert weights (weight-only e4m3; an optional variant) ----
+ * Post-training FP8 quantization of the experts (inferensys.com glossary,
+ * quantization entry) halves the weight bytes the layer streams, which is
+ * what bounds decode-sized batches.  Activations, accumulation, h, y_perm and
+ * y stay as in the bf16 path; each weight is q * s with q an e4m3 code and s
+ * an fp32 scale per (expert, output column). */
+
+/* Quantize bf16 weights w [E,K,N] (N contiguous; gate/up: K=d, N=f; down:
+ * K=f, N=d): scale[e,n] = max_k |w[e,k,n]| / 448 in fp32 (1 for an all-zero
+ * column); w_q[e,k,n] = e4m3 code of w[e,k,n] / scale[e,n], rounded to
+ * nearest even, saturating at +-448.  w_q u8 [E,K,N] out, scale f32 [E,N]
+ * out. */
+int moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t N, uint8_t* w_q,
+                             float* scale, void* stream);
+
+/* moe_expert_gate_up / moe_expert_down with e4m3 weights and their scales
+ * (single-CTA tiles; the weights are widened exactly to bf16 in shared
+ * memory, the column scales applied to the fp32 accumulators).  Arguments as
+ * the bf16 entry points, all buffers 16-byte aligned. */
+int moe_expert_gate_up_fp8(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d,
+                           int64_t f, int64_t max_rows, const uint8_t* wq_gate,
+                           const float* s_gate, const uint8_t* wq_up, const float* s_up, void* h,
+                           int32_t* dev_status, void* stream);
+int moe_expert_down_fp8(const void* h, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
+                        int64_t max_rows, const uint8_t* wq_down, const float* s_down,
+                        float* y_perm, int32_t* dev_status, void* stream);
+
+/* moe_layer_forward with e4m3 expert weights (same workspace layout). */
+int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bias,
+                          const uint8_t* wq_gate, const float* s_gate, const uint8_t* wq_up,
+                          const float* s_up, const uint8_t* wq_down, const float* s_down,
+                          int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf,
+                          void* y, void* ws, size_t ws_bytes, void* stream);
+
 /* The whole layer: moe_route, moe_permute, moe_expert_mlp, moe_combine on
  * one stream, every intermediate in `ws` (>= moe_workspace_size bytes; field
  * layout from moe_workspace_field_offset).  No host synchronisation: bucket

@@ -29,7 +29,8 @@ EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "mo
             "moe_max_rows",
             "moe_route_workspace_size", "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
             "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
-            "moe_combine", "moe_layer_forward"]
+            "moe_combine", "moe_layer_forward", "moe_quantize_weights_fp8",
+            "moe_expert_gate_up_fp8", "moe_expert_down_fp8", "moe_layer_forward_fp8"]
 
 
 class MoEError(RuntimeError):
@@ -63,6 +64,11 @@ def _load():
         "moe_combine": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, p, p]),
         "moe_layer_forward": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl, p, p,
                                              sz, p]),
+        "moe_quantize_weights_fp8": (ctypes.c_int, [p, i64, i64, i64, p, p, p]),
+        "moe_expert_gate_up_fp8": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p, p, p]),
+        "moe_expert_down_fp8": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p]),
+        "moe_layer_forward_fp8": (ctypes.c_int, [p, p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64,
+                                                 dbl, p, p, sz, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -310,6 +316,81 @@ def moe_layer_forward(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws
     _check("moe_layer_forward", _lib.moe_layer_forward(
         _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k,
         f, float(cf), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+    return y, ws
+
+
+# ----------------------------------------------------------------- FP8 expert weights
+
+def moe_quantize_weights_fp8(w, stream=None):
+    """bf16 weights [E,K,N] -> (e4m3 codes uint8 [E,K,N], fp32 scales [E,N])."""
+    E, K, N = w.shape
+    _want(w, "w", torch.bfloat16)
+    q = torch.empty(E, K, N, dtype=torch.uint8, device=w.device)
+    sc = torch.empty(E, N, dtype=torch.float32, device=w.device)
+    _check("moe_quantize_weights_fp8",
+           _lib.moe_quantize_weights_fp8(_ptr(w), E, K, N, _ptr(q), _ptr(sc), _stream(stream)))
+    return q, sc
+
+
+def moe_expert_gate_up_fp8(x_perm, offsets, wq_gate, s_gate, wq_up, s_up, h=None, dev_status=None,
+                           stream=None):
+    rows, d = x_perm.shape
+    E, _, f = wq_gate.shape
+    _want(x_perm, "x_perm", torch.bfloat16)
+    _want(offsets, "offsets", torch.int32, (E + 1,))
+    _want(wq_gate, "wq_gate", torch.uint8, (E, d, f))
+    _want(wq_up, "wq_up", torch.uint8, (E, d, f))
+    _want(s_gate, "s_gate", torch.float32, (E, f))
+    _want(s_up, "s_up", torch.float32, (E, f))
+    h = torch.empty(rows, f, dtype=torch.bfloat16, device=x_perm.device) if h is None else h
+    _want(h, "h", torch.bfloat16, (rows, f))
+    _check("moe_expert_gate_up_fp8", _lib.moe_expert_gate_up_fp8(
+        _ptr(x_perm), _ptr(offsets), E, d, f, rows, _ptr(wq_gate), _ptr(s_gate), _ptr(wq_up),
+        _ptr(s_up), _ptr(h), _ptr(dev_status), _stream(stream)))
+    return h
+
+
+def moe_expert_down_fp8(h, offsets, wq_down, s_down, y_perm=None, dev_status=None, stream=None):
+    rows, f = h.shape
+    E, _, d = wq_down.shape
+    _want(h, "h", torch.bfloat16)
+    _want(offsets, "offsets", torch.int32, (E + 1,))
+    _want(wq_down, "wq_down", torch.uint8, (E, f, d))
+    _want(s_down, "s_down", torch.float32, (E, d))
+    y_perm = torch.empty(rows, d, dtype=torch.float32, device=h.device) if y_perm is None \
+        else y_perm
+    _want(y_perm, "y_perm", torch.float32, (rows, d))
+    _check("moe_expert_down_fp8", _lib.moe_expert_down_fp8(
+        _ptr(h), _ptr(offsets), E, d, f, rows, _ptr(wq_down), _ptr(s_down), _ptr(y_perm),
+        _ptr(dev_status), _stream(stream)))
+    return y_perm
+
+
+def moe_layer_forward_fp8(x, w_router, bias, wq_gate, s_gate, wq_up, s_up, wq_down, s_down, k, cf,
+                          y=None, ws=None, stream=None):
+    """The whole layer with e4m3 expert weights.  Returns (y, ws)."""
+    T, d = x.shape
+    E, _, f = wq_gate.shape
+    _want(x, "x", torch.bfloat16)
+    _want(w_router, "w_router", torch.float32, (d, E))
+    if bias is not None:
+        _want(bias, "bias", torch.float32, (E,))
+    for name, t, shape in (("wq_gate", wq_gate, (E, d, f)), ("wq_up", wq_up, (E, d, f)),
+                           ("wq_down", wq_down, (E, f, d))):
+        _want(t, name, torch.uint8, shape)
+    for name, t, shape in (("s_gate", s_gate, (E, f)), ("s_up", s_up, (E, f)),
+                           ("s_down", s_down, (E, d))):
+        _want(t, name, torch.float32, shape)
+    nbytes = moe_workspace_size(T, d, E, k, f, cf)
+    if ws is None:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _want(ws, "ws", torch.uint8)
+    y = torch.empty_like(x) if y is None else y
+    _want(y, "y", torch.bfloat16, (T, d))
+    _check("moe_layer_forward_fp8", _lib.moe_layer_forward_fp8(
+        _ptr(x), _ptr(w_router), _ptr(bias), _ptr(wq_gate), _ptr(s_gate), _ptr(wq_up), _ptr(s_up),
+        _ptr(wq_down), _ptr(s_down), T, d, E, k, f, float(cf), _ptr(y), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return y, ws
 
 

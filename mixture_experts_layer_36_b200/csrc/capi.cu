@@ -26,6 +26,15 @@ cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t s);
+cudaError_t launch_quantize_fp8(const __nv_bfloat16* w, int E, int K, int N, uint8_t* q,
+                                float* scale, cudaStream_t s);
+cudaError_t launch_gate_up_fp8(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
+                               int f, int max_rows, const uint8_t* wq_gate, const float* s_gate,
+                               const uint8_t* wq_up, const float* s_up, __nv_bfloat16* h,
+                               int32_t* status, cudaStream_t s, bool* map_failed);
+cudaError_t launch_down_fp8(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
+                            int max_rows, const uint8_t* wq_down, const float* s_down,
+                            float* y_perm, int32_t* status, cudaStream_t s, bool* map_failed);
 }  // namespace moe
 
 namespace moe {
@@ -283,6 +292,102 @@ int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, con
                                     topk_w, slot,
                                     offsets, (int)T, (int)d, (int)k,
                                     static_cast<__nv_bfloat16*>(y), as_stream(stream)));
+}
+
+int moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t N, uint8_t* w_q,
+                             float* scale, void* stream) {
+  if (E < 1 || K < 1 || N < 1 || E > 65535 || E * K * N >= (int64_t(1) << 40))
+    return MOE_ERR_INVALID_ARG;
+  if (!w || !w_q || !scale) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_quantize_fp8(static_cast<const __nv_bfloat16*>(w), (int)E,
+                                              (int)K, (int)N, w_q, scale, as_stream(stream)));
+}
+
+int moe_expert_gate_up_fp8(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d,
+                           int64_t f, int64_t max_rows, const uint8_t* wq_gate,
+                           const float* s_gate, const uint8_t* wq_up, const float* s_up, void* h,
+                           int32_t* dev_status, void* stream) {
+  int st = check_gemm_args(E, d, f, max_rows);
+  if (st != MOE_OK) return st;
+  if (max_rows == 0) return MOE_OK;
+  if (!x_perm || !offsets || !wq_gate || !s_gate || !wq_up || !s_up || !h)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(wq_gate) || !aligned16(wq_up) || !aligned16(s_gate) ||
+      !aligned16(s_up) || !aligned16(h))
+    return MOE_ERR_INVALID_ARG;
+  bool map_failed = false;
+  cudaError_t err = moe::launch_gate_up_fp8(
+      static_cast<const __nv_bfloat16*>(x_perm), offsets, (int)E, (int)d, (int)f, (int)max_rows,
+      wq_gate, s_gate, wq_up, s_up, static_cast<__nv_bfloat16*>(h), dev_status,
+      as_stream(stream), &map_failed);
+  if (map_failed) return MOE_ERR_CUDA;
+  return cuda_status(err);
+}
+
+int moe_expert_down_fp8(const void* h, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
+                        int64_t max_rows, const uint8_t* wq_down, const float* s_down,
+                        float* y_perm, int32_t* dev_status, void* stream) {
+  int st = check_gemm_args(E, d, f, max_rows);
+  if (st != MOE_OK) return st;
+  if (max_rows == 0) return MOE_OK;
+  if (!h || !offsets || !wq_down || !s_down || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(wq_down) || !aligned16(s_down) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  bool map_failed = false;
+  cudaError_t err = moe::launch_down_fp8(static_cast<const __nv_bfloat16*>(h), offsets, (int)E,
+                                         (int)d, (int)f, (int)max_rows, wq_down, s_down, y_perm,
+                                         dev_status, as_stream(stream), &map_failed);
+  if (map_failed) return MOE_ERR_CUDA;
+  return cuda_status(err);
+}
+
+int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bias,
+                          const uint8_t* wq_gate, const float* s_gate, const uint8_t* wq_up,
+                          const float* s_up, const uint8_t* wq_down, const float* s_down,
+                          int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf,
+                          void* y, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_routing_shape(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_width(d)) != MOE_OK) return st;
+  if ((st = check_width(f)) != MOE_OK) return st;
+  if (moe_capacity(T, E, k, cf) < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !wq_gate || !s_gate || !wq_up || !s_up || !wq_down || !s_down || !y ||
+      !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_workspace_size(T, d, E, k, f, cf)) return MOE_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  auto field = [&](int id) { return base + moe_workspace_field_offset(id, T, d, E, k, f, cf); };
+  int32_t* status = reinterpret_cast<int32_t*>(field(MOE_WS_STATUS));
+  float* logits = reinterpret_cast<float*>(field(MOE_WS_LOGITS));
+  int32_t* topk_idx = reinterpret_cast<int32_t*>(field(MOE_WS_TOPK_IDX));
+  float* topk_w = reinterpret_cast<float*>(field(MOE_WS_TOPK_W));
+  int32_t* slot = reinterpret_cast<int32_t*>(field(MOE_WS_SLOT));
+  int32_t* counts = reinterpret_cast<int32_t*>(field(MOE_WS_COUNTS));
+  int32_t* offsets = reinterpret_cast<int32_t*>(field(MOE_WS_OFFSETS));
+  int32_t* n_dropped = reinterpret_cast<int32_t*>(field(MOE_WS_N_DROPPED));
+  int32_t* row_src = reinterpret_cast<int32_t*>(field(MOE_WS_ROW_SRC));
+  void* x_perm = field(MOE_WS_X_PERM);
+  void* h = field(MOE_WS_H);
+  float* y_perm = reinterpret_cast<float*>(field(MOE_WS_Y_PERM));
+  const int64_t max_rows = moe_max_rows(T, E, k, cf);
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, field(MOE_WS_ROUTE),
+                      moe_route_workspace_size(T, d, E, k), status, stream)) != MOE_OK)
+    return st;
+  if ((st = moe_permute(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src, x_perm,
+                        n_dropped, field(MOE_WS_PERMUTE), moe_permute_workspace_size(T, E, k),
+                        stream)) != MOE_OK)
+    return st;
+  if ((st = moe_expert_gate_up_fp8(x_perm, offsets, E, d, f, max_rows, wq_gate, s_gate, wq_up,
+                                   s_up, h, status, stream)) != MOE_OK)
+    return st;
+  if ((st = moe_expert_down_fp8(h, offsets, E, d, f, max_rows, wq_down, s_down, y_perm, status,
+                                stream)) != MOE_OK)
+    return st;
+  return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
 }
 
 int moe_layer_forward(const void* x, const float* w_router, const float* bias, const void* w_gate,

@@ -270,6 +270,34 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
   }
 }
 
+// ---------------------------------------------------------------- FP8 weights
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tensor-core operand reads) before signalling them on an mbarrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Four e4m3 bytes -> four bf16 (two 32-bit words), exactly.  The hardware
+// converts pairs of e4m3 to f16 (every e4m3 value is zero or a normal f16);
+// f16 -> bf16 then only re-biases the exponent (+112) and drops the three
+// mantissa bits that are zero here.
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2_exact(uint32_t h) {
+  const uint32_t sign = h & 0x80008000u;
+  const uint32_t mag = h & 0x7FFF7FFFu;
+  uint32_t t = (mag >> 3) & 0x0FFF0FFFu;
+  if (mag & 0x00007FFFu) t += 112u << 7;
+  if (mag & 0x7FFF0000u) t += 112u << 23;
+  return t | sign;
+}
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  uint32_t h01, h23;
+  const uint16_t b01 = static_cast<uint16_t>(w & 0xFFFFu), b23 = static_cast<uint16_t>(w >> 16);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"(b01));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"(b23));
+  lo = f16x2_to_bf16x2_exact(h01);
+  hi = f16x2_to_bf16x2_exact(h23);
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -87,6 +87,19 @@ __device__ __forceinline__ void swiglu_pack(const uint32_t (&g)[32], const uint3
 
 __device__ __forceinline__ int clamp_rows(int v) { return v < 0 ? 0 : (v > 32 ? 32 : v); }
 
+// v[i] *= scale[i] for the 32 accumulator columns of a chunk (fp32 bits)
+__device__ __forceinline__ void apply_col_scales(uint32_t (&v)[32], const float* __restrict__ scale) {
+  const float4* s4 = reinterpret_cast<const float4*>(scale);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 sc = __ldg(s4 + i);
+    v[4 * i + 0] = __float_as_uint(__uint_as_float(v[4 * i + 0]) * sc.x);
+    v[4 * i + 1] = __float_as_uint(__uint_as_float(v[4 * i + 1]) * sc.y);
+    v[4 * i + 2] = __float_as_uint(__uint_as_float(v[4 * i + 2]) * sc.z);
+    v[4 * i + 3] = __float_as_uint(__uint_as_float(v[4 * i + 3]) * sc.w);
+  }
+}
+
 template <int BN, bool SWIGLU>
 struct GemmCfg {
   static constexpr int kOutCols = SWIGLU ? BN / 2 : BN;  // output columns per tile
@@ -129,12 +142,22 @@ __device__ __forceinline__ void decode_tile(const GemmShared& sh, int tile, int 
   m = local - n * mt;
 }
 
-template <int BN, bool SWIGLU>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// FP8W: the weights arrive as e4m3 codes [E, K, n_out] with fp32 column
+// scales [E, n_out] (tmB0/tmB1 unused).  Four more warps (6..9) each take
+// every fourth k-block: they load its fp8 weight tile with 16-byte loads,
+// widen it exactly to bf16 into the stage's swizzled B buffer, fence it to the
+// async proxy and arrive on the stage barrier (armed by the producer for the
+// A bytes only).  The epilogue multiplies each column by its scale.
+constexpr int kConvWarps = 4;
+
+template <int BN, bool SWIGLU, bool FP8W = false>
+__global__ void __launch_bounds__(FP8W ? kGemmThreads + 32 * kConvWarps : kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1,
+                        const uint8_t* __restrict__ wq0, const uint8_t* __restrict__ wq1,
+                        const float* __restrict__ wscale0, const float* __restrict__ wscale1,
                         const int32_t* __restrict__ offsets, int E, int K, int n_out,
                         int max_rows, void* __restrict__ out_raw, int32_t* status) {
   using Cfg = GemmCfg<BN, SWIGLU>;
@@ -149,7 +172,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::kStages; ++s) {
-      mbar_init(&sh.full_bar[s], 1);
+      mbar_init(&sh.full_bar[s], FP8W ? 2 : 1);     // + the converting warp
       mbar_init(&sh.empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -168,8 +191,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmA64);
-    prefetch_tensormap(&tmB0);
-    if (SWIGLU) prefetch_tensormap(&tmB1);
+    if (!FP8W) prefetch_tensormap(&tmB0);
+    if (SWIGLU && !FP8W) prefetch_tensormap(&tmB1);
   }
   if (warp == 2) {
     // per-expert tile counts -> exclusive prefix; row offsets to smem
@@ -226,13 +249,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
           uint8_t* sa = smem + s * Cfg::kStageBytes;
           uint8_t* sb = sa + Cfg::kABytes;
-          mbar_arrive_expect_tx(&sh.full_bar[s],
-                                small ? Cfg::kStageBytes - Cfg::kABytes / 2 : Cfg::kStageBytes);
+          const uint32_t a_bytes = small ? Cfg::kABytes / 2 : Cfg::kABytes;
+          mbar_arrive_expect_tx(&sh.full_bar[s], FP8W ? a_bytes : a_bytes + Cfg::kBBytes);
           if (small)
             tma_load_2d(sa, &tmA64, &sh.full_bar[s], kb * kBK, row0);
           else
             tma_load_2d(sa, &tmA, &sh.full_bar[s], kb * kBK, row0);
-          if (SWIGLU) {
+          if (FP8W) {
+            // B is written by the converting warps
+          } else if (SWIGLU) {
 #pragma unroll
             for (int c = 0; c < BN / 128; ++c)
               tma_load_3d(sb + c * kChunkBytes, &tmB0, &sh.full_bar[s], col0 + c * 64, kb * kBK, e);
@@ -300,7 +325,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       umma_commit(&sh.drain_bar);
       mbar_wait(&sh.drain_bar, 0, &sh.never);
     }
-  } else {
+  } else if (warp < 6) {
     // -------------------------------------------------- epilogue (warps 2..5)
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     int lt = 0;
@@ -334,6 +359,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld_32x32b_x32(tbase + c * 32, g);
           tmem_ld_32x32b_x32(tbase + BN / 2 + c * 32, u);
           tmem_ld_wait();
+          if (FP8W) {
+            const size_t sc = (size_t)e * n_out + (size_t)n * Cfg::kOutCols + c * 32;
+            apply_col_scales(g, wscale0 + sc);
+            apply_col_scales(u, wscale1 + sc);
+          }
           swiglu_pack(g, u, pk);
           store_chunk_bf16(pk, o + c * 32, n_out, nvalid, lane);
         }
@@ -344,12 +374,61 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t v[32];
           tmem_ld_32x32b_x32(tbase + c * 32, v);
           tmem_ld_wait();
+          if (FP8W)
+            apply_col_scales(v, wscale0 + (size_t)e * n_out + (size_t)n * Cfg::kOutCols + c * 32);
           store_chunk_f32(v, stage, o + c * 32, n_out, nvalid, lane);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.tempty_bar[a]);
+    }
+  } else if (FP8W) {
+    // -------------------------------------------------- fp8 -> bf16 weights (warps 6..9)
+    const int cw = warp - 6;
+    constexpr int kVecPerRow = FP8W && SWIGLU ? BN / 2 / 16 : BN / 16;   // 16-B vectors per K row
+    constexpr int kVecPerOp = kBK * kVecPerRow;
+    constexpr int kVecs = SWIGLU ? 2 * kVecPerOp : kVecPerOp;            // per k-block
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int e, m, n;
+      decode_tile(sh, tile, E, n_tiles, e, m, n);
+      const int col0 = n * Cfg::kOutCols;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        if (it % kConvWarps != cw) continue;
+        const int s = it % Cfg::kStages;
+        const uint32_t ph = (it / Cfg::kStages) & 1;
+        if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
+        uint8_t* sb = smem + s * Cfg::kStageBytes + Cfg::kABytes;
+#pragma unroll 4
+        for (int v = lane; v < kVecs; v += 32) {
+          const int op = SWIGLU ? v / kVecPerOp : 0;
+          const int rem = v - op * kVecPerOp;
+          const int k = rem / kVecPerRow, c16 = rem % kVecPerRow;
+          const uint8_t* src = (op ? wq1 : wq0) +
+                               ((size_t)e * K + (size_t)kb * kBK + k) * n_out + col0 + c16 * 16;
+          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
+          uint4 lo, hi;
+          e4m3x4_to_bf16x4(raw.x, lo.x, lo.y);
+          e4m3x4_to_bf16x4(raw.y, lo.z, lo.w);
+          e4m3x4_to_bf16x4(raw.z, hi.x, hi.y);
+          e4m3x4_to_bf16x4(raw.w, hi.z, hi.w);
+          // 64-column chunk and 16-byte unit inside the 128-byte swizzled row
+          const int chunk = (SWIGLU ? op * (BN / 128) : 0) + (c16 >> 2);
+          const int unit = (c16 & 3) * 2;
+          uint8_t* row = sb + chunk * kChunkBytes + k * 128;
+          *reinterpret_cast<uint4*>(row + ((unit ^ (k & 7)) << 4)) = lo;
+          *reinterpret_cast<uint4*>(row + (((unit + 1) ^ (k & 7)) << 4)) = hi;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.full_bar[s]);
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      report(status, kDevErrWaitTimeout);
     }
   }
 
@@ -688,17 +767,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-template <int BN, bool SWIGLU>
+template <int BN, bool SWIGLU, bool FP8W = false>
 static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& a64,
                                const CUtensorMap& b0, const CUtensorMap& b1,
                                const int32_t* offsets, int E, int K,
                                int n_out, int max_rows, void* out, int32_t* status,
-                               cudaStream_t s) {
+                               cudaStream_t s, const uint8_t* wq0 = nullptr,
+                               const uint8_t* wq1 = nullptr, const float* ws0 = nullptr,
+                               const float* ws1 = nullptr) {
   using Cfg = GemmCfg<BN, SWIGLU>;
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  auto kern = grouped_gemm_kernel<BN, SWIGLU>;
+  auto kern = grouped_gemm_kernel<BN, SWIGLU, FP8W>;
   if (!di->attr_set[slot]) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg::kSmemBytes);
@@ -710,8 +791,9 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
   long long ub = row_tiles * n_tiles;
   int grid = (int)(ub < di->sms ? ub : di->sms);
   if (grid < 1) grid = 1;
-  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, offsets, E, K, n_out,
-                                                     max_rows, out, status);
+  const int threads = FP8W ? kGemmThreads + 32 * kConvWarps : kGemmThreads;
+  kern<<<grid, threads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, wq0, wq1, ws0, ws1, offsets, E, K,
+                                              n_out, max_rows, out, status);
   return cudaGetLastError();
 }
 
@@ -787,6 +869,32 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
                                    s);
   return launch_gemm<128, false>(2, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
                                  s);
+}
+
+// GEMM 1 / GEMM 2 with e4m3 weights and fp32 column scales (single-CTA tiles)
+cudaError_t launch_gate_up_fp8(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
+                               int f, int max_rows, const uint8_t* wq_gate, const float* s_gate,
+                               const uint8_t* wq_up, const float* s_up, __nv_bfloat16* h,
+                               int32_t* status, cudaStream_t s, bool* map_failed) {
+  CUtensorMap ta, ta64;
+  *map_failed = !(map_rows(&ta, x_perm, d, max_rows, kBM) &&
+                  map_rows(&ta64, x_perm, d, max_rows, kBM / 2));
+  if (*map_failed) return cudaSuccess;
+  return launch_gemm<256, true, true>(11, ta, ta64, ta, ta, offsets, E, d, f, max_rows, h, status,
+                                      s, wq_gate, wq_up, s_gate, s_up);
+}
+
+cudaError_t launch_down_fp8(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
+                            int max_rows, const uint8_t* wq_down, const float* s_down,
+                            float* y_perm, int32_t* status, cudaStream_t s, bool* map_failed) {
+  CUtensorMap ta, ta64;
+  *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_rows(&ta64, h, f, max_rows, kBM / 2));
+  if (*map_failed) return cudaSuccess;
+  if (d % 256 == 0)
+    return launch_gemm<256, false, true>(12, ta, ta64, ta, ta, offsets, E, f, d, max_rows, y_perm,
+                                         status, s, wq_down, nullptr, s_down, nullptr);
+  return launch_gemm<128, false, true>(13, ta, ta64, ta, ta, offsets, E, f, d, max_rows, y_perm,
+                                       status, s, wq_down, nullptr, s_down, nullptr);
 }
 
 int device_sm_count() {

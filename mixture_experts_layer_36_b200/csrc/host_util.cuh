@@ -55,7 +55,8 @@ inline bool map_weights(CUtensorMap* m, const void* base, uint64_t E, uint64_t K
          CUDA_SUCCESS;
 }
 
-// attr_set slots: 0-2 grouped GEMM (1 CTA), 3-6 router GEMM, 7-8 grouped GEMM (CTA pair)
+// attr_set slots: 0-2 grouped GEMM (1 CTA), 3-6 router GEMM, 7-8 grouped GEMM (CTA pair),
+// 11-13 grouped GEMM with fp8 weights, 14 fp8 quantizer
 struct DeviceInfo {
   int sms = 0;
   bool attr_set[16] = {};

@@ -43,6 +43,10 @@ def lib():
         _lib.oracle_moe_forward.restype = _i64
         _lib.oracle_round_bf16.restype = _dbl
         _lib.oracle_round_bf16.argtypes = [_dbl]
+        _lib.oracle_e4m3_encode.restype = ctypes.c_ubyte
+        _lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        _lib.oracle_e4m3_decode.restype = _dbl
+        _lib.oracle_e4m3_decode.argtypes = [ctypes.c_ubyte]
     return _lib
 
 
@@ -187,6 +191,48 @@ def moe_forward(x_bits, w_router, bias, w_gate_bits, w_up_bits, w_down_bits, k, 
         _ptr(out["counts"]), _ptr(out["offsets"]))
     out["n_dropped"] = int(n_drop)
     return out
+
+
+def e4m3_encode(v):
+    """Nearest e4m3 code (ties to even, saturating at +-448) of a float."""
+    return int(lib().oracle_e4m3_encode(float(v)))
+
+
+def e4m3_decode(q):
+    return float(lib().oracle_e4m3_decode(int(q)))
+
+
+def quantize_fp8(w_bits):
+    """bf16 weights [E,K,N] (bits) -> (e4m3 codes uint8 [E,K,N], fp32 scales [E,N])."""
+    w_bits = _c(w_bits, np.uint16)
+    E, K, N = w_bits.shape
+    q = np.empty((E, K, N), np.uint8)
+    s = np.empty((E, N), np.float32)
+    lib().oracle_quantize_fp8(_ptr(w_bits), _i64(E), _i64(K), _i64(N), _ptr(q), _ptr(s))
+    return q, s
+
+
+def dequant_fp8(q, scale):
+    q = _c(q, np.uint8)
+    scale = _c(scale, np.float32)
+    E, K, N = q.shape
+    out = np.empty((E, K, N), np.float64)
+    lib().oracle_dequant_fp8(_ptr(q), _ptr(scale), _i64(E), _i64(K), _i64(N), _ptr(out))
+    return out
+
+
+def swiglu_rows_f64w(x_rows_bits, wg, wu, wd, want_h=False, h_bf16=True):
+    """One expert with fp64 weights (e.g. dequantized FP8): x_rows [n,d] bf16
+    bits, wg/wu [d,f], wd [f,d] fp64.  Returns (h or None, o) in fp64."""
+    x_rows_bits = _c(x_rows_bits, np.uint16)
+    wg, wu, wd = (_c(a, np.float64) for a in (wg, wu, wd))
+    n, d = x_rows_bits.shape
+    f = wg.shape[1]
+    h = np.empty((n, f), np.float64) if want_h else None
+    o = np.empty((n, d), np.float64)
+    lib().oracle_swiglu_rows_f64w(_ptr(x_rows_bits), _i64(n), _i64(d), _i64(f), _ptr(wg), _ptr(wu),
+                                  _ptr(wd), ctypes.c_int(int(h_bf16)), _ptr(h), _ptr(o))
+    return h, o
 
 
 def bf16_bits(t):

@@ -203,6 +203,99 @@ void oracle_swiglu_rows(const uint16_t* x_rows, int64_t n, int64_t d, int64_t f,
     }
 }
 
+/* ---- FP8 (e4m3) expert weights: one variant of step 5's operands ----
+ * Weight-only quantization with one scale per (expert, output column):
+ *   s[e,n] = max_k |w[e,k,n]| / 448   (fp32, as the quantizer computes it)
+ *   q[e,k,n] = e4m3(w[e,k,n] / s[e,n]) (the fp32 quotient rounded to the
+ *             nearest e4m3 value, ties to even; 448 is the largest finite)
+ * and the dequantized weight q * s used in place of w.  e4m3: 1 sign bit,
+ * 4 exponent bits (bias 7), 3 mantissa bits; normal values 2^-6 .. 448,
+ * subnormals k * 2^-9. */
+
+/* nearest e4m3 code (ties to even) of a finite float, saturating to +-448 */
+unsigned char oracle_e4m3_encode(float v) {
+    unsigned char sign = (v < 0.0f || (v == 0.0f && signbit(v))) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0) return sign | 0x7E;                 /* 1.75 * 2^8 */
+    if (a < ldexp(1.0, -6)) {                            /* subnormal range: k * 2^-9 */
+        double k = nearbyint(a * 512.0);                 /* ties to even */
+        if (k >= 8.0) return sign | 0x08;                /* rounds up to 2^-6 */
+        return sign | (unsigned char)k;
+    }
+    int ex;
+    double m = frexp(a, &ex);                            /* a = m * 2^ex, 0.5 <= m < 1 */
+    double r = nearbyint(ldexp(m, 4));                   /* 4 significant bits: 8..16 */
+    if (r >= 16.0) { r = 8.0; ex += 1; }
+    int e = ex - 1 + 7;                                  /* biased exponent of r/8 * 2^(ex-1) */
+    if (e > 15 || (e == 15 && r > 14.0)) return sign | 0x7E;
+    return sign | (unsigned char)((e << 3) | ((int)r - 8));
+}
+
+double oracle_e4m3_decode(unsigned char q) {
+    int e = (q >> 3) & 0xF, m = q & 7;
+    double v = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (q & 0x80) ? -v : v;
+}
+
+/* Quantize bf16 weights [E,K,N] to e4m3 codes + fp32 column scales [E,N]. */
+void oracle_quantize_fp8(const uint16_t* w, int64_t E, int64_t K, int64_t N, unsigned char* q,
+                         float* scale) {
+    for (int64_t e = 0; e < E; ++e)
+        for (int64_t n = 0; n < N; ++n) {
+            float mx = 0.0f;
+            for (int64_t k = 0; k < K; ++k) {
+                float a = fabsf((float)bf16_bits_to_f64(w[(e * K + k) * N + n]));
+                if (a > mx) mx = a;
+            }
+            float s = mx > 0.0f ? mx / 448.0f : 1.0f;
+            scale[e * N + n] = s;
+            for (int64_t k = 0; k < K; ++k) {
+                float v = (float)bf16_bits_to_f64(w[(e * K + k) * N + n]) / s;
+                q[(e * K + k) * N + n] = oracle_e4m3_encode(v);
+            }
+        }
+}
+
+/* Dequantized weights q * s as fp64 [E,K,N]. */
+void oracle_dequant_fp8(const unsigned char* q, const float* scale, int64_t E, int64_t K,
+                        int64_t N, double* out) {
+    for (int64_t e = 0; e < E; ++e)
+        for (int64_t k = 0; k < K; ++k)
+            for (int64_t n = 0; n < N; ++n)
+                out[(e * K + k) * N + n] =
+                    oracle_e4m3_decode(q[(e * K + k) * N + n]) * (double)scale[e * N + n];
+}
+
+/* Step 5 for n rows of one expert with fp64 weights wg/wu [d,f], wd [f,d]
+ * (e.g. dequantized FP8); otherwise as oracle_swiglu_rows. */
+void oracle_swiglu_rows_f64w(const uint16_t* x_rows, int64_t n, int64_t d, int64_t f,
+                             const double* wg, const double* wu, const double* wd, int round_h,
+                             double* h_out, double* o_out) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+        double* g = (double*)calloc((size_t)f, sizeof(double));
+        double* u = (double*)calloc((size_t)f, sizeof(double));
+        const uint16_t* xr = x_rows + r * d;
+        for (int64_t i = 0; i < d; ++i) {
+            double xi = bf16_bits_to_f64(xr[i]);
+            for (int64_t j = 0; j < f; ++j) {
+                g[j] += xi * wg[i * f + j];
+                u[j] += xi * wu[i * f + j];
+            }
+        }
+        double* o = o_out + r * d;
+        for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+        for (int64_t j = 0; j < f; ++j) {
+            double hj = g[j] / (1.0 + exp(-g[j])) * u[j];
+            if (round_h) hj = oracle_round_bf16(hj);
+            if (h_out) h_out[r * f + j] = hj;
+            for (int64_t c = 0; c < d; ++c) o[c] += hj * wd[j * d + c];
+        }
+        free(g);
+        free(u);
+    }
+}
+
 /* Step 5 over every bucket: rows offsets[e] .. offsets[e+1]-1 use expert e. */
 void oracle_expert_mlp(const uint16_t* x_perm, const int32_t* offsets, int64_t E, int64_t d,
                        int64_t f, const uint16_t* w_gate, const uint16_t* w_up,

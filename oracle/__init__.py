@@ -235,6 +235,46 @@ def swiglu_rows_f64w(x_rows_bits, wg, wu, wd, want_h=False, h_bf16=True):
     return h, o
 
 
+def quantize_rows_fp8(x_bits):
+    """bf16 rows [R,K] (bits) -> (e4m3 codes uint8 [R,K], fp32 row scales [R])."""
+    x_bits = _c(x_bits, np.uint16)
+    R, K = x_bits.shape
+    q = np.empty((R, K), np.uint8)
+    s = np.empty(R, np.float32)
+    lib().oracle_quantize_rows_fp8(_ptr(x_bits), _i64(R), _i64(K), _ptr(q), _ptr(s))
+    return q, s
+
+
+def dequant_rows_fp8(q, scale):
+    q = _c(q, np.uint8)
+    scale = _c(scale, np.float32)
+    R, K = q.shape
+    out = np.empty((R, K), np.float64)
+    lib().oracle_dequant_rows_fp8(_ptr(q), _ptr(scale), _i64(R), _i64(K), _ptr(out))
+    return out
+
+
+def gate_up_f64(a, wg, wu, h_bf16=True):
+    """h = silu(a wg) * (a wu) in fp64 for a [n,d], wg/wu [d,f]; rounded to
+    bf16 when h_bf16."""
+    a, wg, wu = (_c(t, np.float64) for t in (a, wg, wu))
+    n, d = a.shape
+    f = wg.shape[1]
+    h = np.empty((n, f), np.float64)
+    lib().oracle_gate_up_f64(_ptr(a), _i64(n), _i64(d), _i64(f), _ptr(wg), _ptr(wu),
+                             ctypes.c_int(int(h_bf16)), _ptr(h))
+    return h
+
+
+def matmul_f64(a, w):
+    a, w = _c(a, np.float64), _c(w, np.float64)
+    n, K = a.shape
+    N = w.shape[1]
+    out = np.empty((n, N), np.float64)
+    lib().oracle_matmul_f64(_ptr(a), _i64(n), _i64(K), _ptr(w), _i64(N), _ptr(out))
+    return out
+
+
 def bf16_bits(t):
     """torch bf16 tensor -> numpy uint16 bit patterns (no arithmetic)."""
     import torch

@@ -35,6 +35,10 @@
  *         scaled by their gate weights; inferensys.com glossary, Dropped
  *         Tokens entry: a dropped token goes through the layer untouched)
  *
+ * The FP8 variant of step 5 (e4m3 weights with one fp32 scale per expert
+ * column, e4m3 activations with one fp32 scale per row; inferensys.com
+ * glossary, quantization entry) is defined further down with its own rule.
+ *
  * bf16 tensors are passed as their raw 16-bit patterns (uint16_t) and are
  * widened exactly to double.  All accumulation is fp64.  Layouts are
  * row-major: x[T,d], Wr[d,E], Wg/Wu[E,d,f], Wd[E,f,d].
@@ -293,6 +297,74 @@ void oracle_swiglu_rows_f64w(const uint16_t* x_rows, int64_t n, int64_t d, int64
         }
         free(g);
         free(u);
+    }
+}
+
+/* ---- FP8 weights and activations (the W8A8 variant of step 5) ----
+ * Activations are quantized per row with the same rule as the weight
+ * columns above: s[r] = max_k |x[r,k]| / 448 (fp32; 1 for an all-zero row),
+ * q[r,k] = e4m3(x[r,k] / s[r]).  A product of a row scale and a column scale
+ * is constant along the contraction, so the quantized GEMM is
+ *   out[r,n] = sum_k (q_a[r,k] s_a[r]) (q_w[k,n] s_w[n])
+ * evaluated here on the dequantized operands in fp64. */
+void oracle_quantize_rows_fp8(const uint16_t* x, int64_t R, int64_t K, unsigned char* q,
+                              float* scale) {
+    for (int64_t r = 0; r < R; ++r) {
+        float mx = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf((float)bf16_bits_to_f64(x[r * K + k]));
+            if (a > mx) mx = a;
+        }
+        float s = mx > 0.0f ? mx / 448.0f : 1.0f;
+        scale[r] = s;
+        for (int64_t k = 0; k < K; ++k)
+            q[r * K + k] = oracle_e4m3_encode((float)bf16_bits_to_f64(x[r * K + k]) / s);
+    }
+}
+
+/* Dequantized rows q * s as fp64 [R,K]. */
+void oracle_dequant_rows_fp8(const unsigned char* q, const float* scale, int64_t R, int64_t K,
+                             double* out) {
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = oracle_e4m3_decode(q[r * K + k]) * (double)scale[r];
+}
+
+/* Gate/up of one expert on fp64 operands: h = silu(a wg) * (a wu) for a [n,d],
+ * wg/wu [d,f]; h rounded to bf16 when round_h is set. */
+void oracle_gate_up_f64(const double* a, int64_t n, int64_t d, int64_t f, const double* wg,
+                        const double* wu, int round_h, double* h_out) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+        double* g = (double*)calloc((size_t)f, sizeof(double));
+        double* u = (double*)calloc((size_t)f, sizeof(double));
+        for (int64_t i = 0; i < d; ++i) {
+            double ai = a[r * d + i];
+            for (int64_t j = 0; j < f; ++j) {
+                g[j] += ai * wg[i * f + j];
+                u[j] += ai * wu[i * f + j];
+            }
+        }
+        for (int64_t j = 0; j < f; ++j) {
+            double hj = g[j] / (1.0 + exp(-g[j])) * u[j];
+            h_out[r * f + j] = round_h ? oracle_round_bf16(hj) : hj;
+        }
+        free(g);
+        free(u);
+    }
+}
+
+/* out[n,N] = a[n,K] w[K,N] in fp64. */
+void oracle_matmul_f64(const double* a, int64_t n, int64_t K, const double* w, int64_t N,
+                       double* out) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+        double* o = out + r * N;
+        for (int64_t c = 0; c < N; ++c) o[c] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double ak = a[r * K + k];
+            for (int64_t c = 0; c < N; ++c) o[c] += ak * w[k * N + c];
+        }
     }
 }
 

@@ -9,7 +9,10 @@ than the oracle itself:
     maximum mapping to the code of 448, and the dequantized weight within half
     an e4m3 step of the original;
   * the fp64-weight SwiGLU expert equal to the bf16-weight expert on weights
-    that are exactly bf16, and to a numpy brute force on a tiny case.
+    that are exactly bf16, and to a numpy brute force on a tiny case;
+  * row quantization of activations: scales from numpy's fp32 arithmetic and
+    codes from PyTorch's conversion, as for the weight columns; the fp64
+    gate/up and matmul steps against numpy / scipy on small cases.
 """
 import numpy as np
 import pytest
@@ -147,3 +150,52 @@ def test_swiglu_f64w_bruteforce():
         for c in range(d):
             assert o[i, c] == pytest.approx(sum(h[i, j] * wd[j, c] for j in range(f)),
                                             rel=1e-12, abs=1e-12)
+
+
+def test_quantize_rows_scales_and_codes():
+    g = torch.Generator().manual_seed(11)
+    x = (torch.randn(37, 96, generator=g) * 3).to(torch.bfloat16)
+    x[4] = 0                                        # all-zero row: scale 1, codes 0
+    x[9, :] = 0
+    x[9, 50] = 1e-30                                # tiny row: subnormal fp32 scale
+    x[20, 3] = -2e5                                 # one large value: the rest small codes
+    q, s = oracle.quantize_rows_fp8(oracle.bf16_bits(x))
+    xf = x.float().numpy()
+    mx = np.abs(xf).max(axis=1)
+    want_s = np.where(mx > 0, mx / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    np.testing.assert_array_equal(s, want_s)
+    np.testing.assert_array_equal(q, torch_e4m3_codes((xf / s[:, None]).astype(np.float32)))
+    assert np.all(q[4] == 0) and q[20, 3] == 0xFE
+    deq = oracle.dequant_rows_fp8(q, s)
+    np.testing.assert_array_equal(
+        deq, np.vectorize(oracle.e4m3_decode)(q) * s[:, None].astype(np.float64))
+    bound = 2.0 ** -4 * np.abs(xf) * (1 + 2.0 ** -20) + 2.0 ** -10 * s[:, None]
+    assert np.all(np.abs(deq - xf) <= bound)
+
+
+def test_gate_up_f64_and_matmul_bruteforce():
+    r = np.random.default_rng(13)
+    n, d, f = 4, 12, 10
+    a, wg, wu = r.standard_normal((n, d)), r.standard_normal((d, f)), r.standard_normal((d, f))
+    h = oracle.gate_up_f64(a, wg, wu, h_bf16=False)
+    g, u = a @ wg, a @ wu
+    np.testing.assert_allclose(h, g * expit(g) * u, rtol=1e-12, atol=1e-12)
+    hb = oracle.gate_up_f64(a, wg, wu, h_bf16=True)
+    np.testing.assert_array_equal(hb, np.vectorize(oracle.round_bf16)(h))
+    w = r.standard_normal((f, 7))
+    np.testing.assert_allclose(oracle.matmul_f64(h, w), h @ w, rtol=1e-12, atol=1e-12)
+
+
+def test_gate_up_f64_equals_bf16_expert():
+    g = torch.Generator().manual_seed(17)
+    n, d, f = 5, 32, 24
+    x = torch.randn(n, d, generator=g).to(torch.bfloat16)
+    wg, wu = ((torch.randn(d, f, generator=g) / d ** 0.5).to(torch.bfloat16) for _ in range(2))
+    wd = (torch.randn(f, d, generator=g) / f ** 0.5).to(torch.bfloat16)
+    b = oracle.bf16_bits
+    h_ref, o_ref = oracle.swiglu_rows(b(x), b(wg), b(wu), b(wd), want_h=True)
+    h = oracle.gate_up_f64(oracle.bits_to_f64(b(x)), oracle.bits_to_f64(b(wg)),
+                           oracle.bits_to_f64(b(wu)))
+    np.testing.assert_allclose(h, h_ref, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(oracle.matmul_f64(h, oracle.bits_to_f64(b(wd))), o_ref,
+                               rtol=1e-12, atol=1e-14)

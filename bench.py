@@ -32,6 +32,8 @@ from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
 METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 8     # router 3, permute 2, gate/up GEMM 1, down GEMM 1, combine 1
+KERNELS_PER_STEP_FP8 = 10   # + the row quantizer on x_perm and on h
+FP8_OVER_BF16 = 2.0      # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
 def moe_max_rows_host(cfg):
@@ -172,40 +174,54 @@ class Layer:
         self.y_perm = z(self.rows, d, dt=torch.float32)
         self.y = z(T, d, dt=torch.bfloat16)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
-        self.ws = z(moe.moe_workspace_size(T, d, E, k, f, cfg.cf), dt=torch.uint8)
+        if fp8:
+            self.xq, self.sx = z(self.rows, d, dt=torch.uint8), z(self.rows, dt=torch.float32)
+            self.hq, self.sh = z(self.rows, f, dt=torch.uint8), z(self.rows, dt=torch.float32)
+            self.ws = z(moe.moe_workspace_size_fp8(T, d, E, k, f, cfg.cf), dt=torch.uint8)
+        else:
+            self.ws = z(moe.moe_workspace_size(T, d, E, k, f, cfg.cf), dt=torch.uint8)
+        self.steps = self.stages()
+        self.stage_names = [n for n, _ in self.steps]
+
+    def stages(self):
+        """The step as (name, call) pairs, in launch order."""
+        m, w, c = self.moe, self.w, self.cfg
+        p = self.perm
+        st = [("route", lambda: m.moe_route(self.x, w["w_router"], w["bias"], c.k, self.logits,
+                                            self.idx, self.tw, ws=self.rws,
+                                            dev_status=self.status)),
+              ("permute", lambda: m.moe_permute(self.x, self.idx, c.E, c.cf, out=p, ws=self.pws))]
+        if self.fp8:
+            q, n_rows = self.q, p["offsets"][c.E:]
+            st += [("quant_x", lambda: m.moe_quantize_rows_fp8(p["x_perm"], n_rows=n_rows,
+                                                               q=self.xq, scale=self.sx)),
+                   ("gate_up", lambda: m.moe_expert_gate_up_fp8(
+                       self.xq, self.sx, p["offsets"], *q["w_gate"], *q["w_up"], h=self.h,
+                       dev_status=self.status)),
+                   ("quant_h", lambda: m.moe_quantize_rows_fp8(self.h, n_rows=n_rows, q=self.hq,
+                                                               scale=self.sh)),
+                   ("down", lambda: m.moe_expert_down_fp8(self.hq, self.sh, p["offsets"],
+                                                          *q["w_down"], y_perm=self.y_perm,
+                                                          dev_status=self.status))]
+        else:
+            st += [("gate_up", lambda: m.moe_expert_gate_up(p["x_perm"], p["offsets"], w["w_gate"],
+                                                            w["w_up"], h=self.h,
+                                                            dev_status=self.status)),
+                   ("down", lambda: m.moe_expert_down(self.h, p["offsets"], w["w_down"],
+                                                      y_perm=self.y_perm,
+                                                      dev_status=self.status))]
+        st.append(("combine", lambda: m.moe_combine(self.y_perm, self.x, self.idx, self.tw,
+                                                    p["slot"], p["offsets"], y=self.y)))
+        return st
 
     def step(self, ev=None):
-        """One layer pass; ev = list of 6 events recorded between the stages."""
-        m, w, c = self.moe, self.w, self.cfg
+        """One layer pass; ev = events recorded around every stage."""
+        for i, (_, call) in enumerate(self.steps):
+            if ev:
+                ev[i].record()
+            call()
         if ev:
-            ev[0].record()
-        m.moe_route(self.x, w["w_router"], w["bias"], c.k, self.logits, self.idx, self.tw,
-                    ws=self.rws, dev_status=self.status)
-        if ev:
-            ev[1].record()
-        m.moe_permute(self.x, self.idx, c.E, c.cf, out=self.perm, ws=self.pws)
-        if ev:
-            ev[2].record()
-        if self.fp8:
-            m.moe_expert_gate_up_fp8(self.perm["x_perm"], self.perm["offsets"], *self.q["w_gate"],
-                                     *self.q["w_up"], h=self.h, dev_status=self.status)
-        else:
-            m.moe_expert_gate_up(self.perm["x_perm"], self.perm["offsets"], w["w_gate"],
-                                 w["w_up"], h=self.h, dev_status=self.status)
-        if ev:
-            ev[3].record()
-        if self.fp8:
-            m.moe_expert_down_fp8(self.h, self.perm["offsets"], *self.q["w_down"],
-                                  y_perm=self.y_perm, dev_status=self.status)
-        else:
-            m.moe_expert_down(self.h, self.perm["offsets"], w["w_down"], y_perm=self.y_perm,
-                              dev_status=self.status)
-        if ev:
-            ev[4].record()
-        m.moe_combine(self.y_perm, self.x, self.idx, self.tw, self.perm["slot"],
-                      self.perm["offsets"], y=self.y)
-        if ev:
-            ev[5].record()
+            ev[len(self.steps)].record()
 
     def layer_forward(self, x, y):
         w, c = self.w, self.cfg
@@ -228,7 +244,8 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    nst = len(layer.stage_names)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # the clock sampler starts before the warm-up so that it is running
     # (nvidia-smi takes a moment to start) when the timed region begins
@@ -248,7 +265,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
         td.barrier()
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), dev, dist)
 
-    names = ["route", "permute", "gate_up", "down", "combine"]
+    names = layer.stage_names
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                 for j, n in enumerate(names)}
     status = int(layer.status.item())
@@ -391,8 +408,8 @@ def main():
             layer.step()
         torch.cuda.synchronize()
         assert int(layer.status.item()) == 0
-        print(json.dumps({"profile_run": cfg.name, "launches": KERNELS_PER_STEP *
-                          (args.warmup + args.steps)}))
+        kps = KERNELS_PER_STEP_FP8 if args.fp8 else KERNELS_PER_STEP
+        print(json.dumps({"profile_run": cfg.name, "launches": kps * (args.warmup + args.steps)}))
         return
 
     if world > 1:
@@ -415,22 +432,26 @@ def main():
     capped = "sw_power_cap" in (r["clocks"].get("reasons") or [])
     peak_tf = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
     peak_src = f"{pk_kind} bf16 {'sustained (power cap active)' if capped else 'burst'}"
+    if args.fp8:
+        # e4m3 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (2)
+        peak_tf *= FP8_OVER_BF16
+        peak_src += f" x {FP8_OVER_BF16:g} (nominal e4m3 / bf16 dense ratio)"
     pair = moe_max_rows_host(cfg) >= 512 * cfg.E and not args.fp8
     kname = ("grouped_gemm_pair_kernel<true> (gate/up + SwiGLU, CTA pairs)" if pair else
-             "grouped_gemm_kernel<256,true,true> (gate/up + SwiGLU, e4m3 weights)" if args.fp8
+             "grouped_gemm_e4m3_kernel<256,true> (gate/up + SwiGLU, e4m3 operands)" if args.fp8
              else "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")
-    ktag = "gemm_pair_gate_up" if pair else "gemm_fp8_gate_up" if args.fp8 else "gemm_gate_up"
+    ktag = "gemm_pair_gate_up" if pair else "gemm_e4m3_gate_up" if args.fp8 else "gemm_gate_up"
     achieved = gemm1_flop / t_g1 / 1e12
     # bytes the gate/up GEMM must move: weights of the experts that got rows,
     # x_perm rows in, h rows out
     A = r["active_experts"]
-    # weight bytes per element: bf16 2; e4m3 1 plus a 4-byte scale per column
+    # operand bytes per element: bf16 2; e4m3 1 (plus 4-byte row / column scales)
     wb = 1 if args.fp8 else 2
-    g1_bytes = A * 2.0 * cfg.d * cfg.f * wb + r["N"] * cfg.d * 2 + r["N"] * cfg.f * 2
-    g2_bytes = A * 1.0 * cfg.d * cfg.f * wb + r["N"] * cfg.f * 2 + r["N"] * cfg.d * 4
+    g1_bytes = A * 2.0 * cfg.d * cfg.f * wb + r["N"] * cfg.d * wb + r["N"] * cfg.f * 2
+    g2_bytes = A * 1.0 * cfg.d * cfg.f * wb + r["N"] * cfg.f * wb + r["N"] * cfg.d * 4
     if args.fp8:
-        g1_bytes += A * 2.0 * cfg.f * 4
-        g2_bytes += A * 1.0 * cfg.d * 4
+        g1_bytes += A * 2.0 * cfg.f * 4 + r["N"] * 4
+        g2_bytes += A * 1.0 * cfg.d * 4 + r["N"] * 4
     ridge = peak_tf * 1e12 / (pk["hbm_gbs"] * 1e9)
     hbm_bound = gemm1_flop / g1_bytes < ridge
     bytes_perm = cfg.T * cfg.d * 2 + r["N"] * cfg.d * 2
@@ -446,12 +467,13 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 (e4m3 expert weights)" if args.fp8 else "bf16",
+        "dtype": "e4m3 (expert GEMM operands; fp32 accumulation)" if args.fp8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the named shape)",
         "config": {"workload": describe(cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
                    "f": cfg.f, "cf": cfg.cf, "kept_pairs": r["N"], "dropped_pairs": r["n_dropped"],
                    "parallelism": f"replicas x{world} (token batches, no collective)",
-                   "expert_weights": "e4m3 + fp32 column scales" if args.fp8 else "bf16",
+                   "experts": ("e4m3 weights (fp32 column scales) x e4m3 activations (fp32 row "
+                               "scales)") if args.fp8 else "bf16",
                    "l2": "inputs larger than L2 (expert weights "
                          f"{3 * cfg.E * cfg.d * cfg.f * wb / 1e9:.1f} GB); no flush"},
         "roofline": ({"kernel": kname,
@@ -493,7 +515,7 @@ def main():
                 "api": ("moe_layer_forward_fp8" if args.fp8 else "moe_layer_forward") +
                        " (one-shot C-ABI call); every step copies x from pinned host memory and "
                        "y back, on copy streams overlapping adjacent steps' compute"},
-        "gpu_launches": KERNELS_PER_STEP * K,
+        "gpu_launches": (KERNELS_PER_STEP_FP8 if args.fp8 else KERNELS_PER_STEP) * K,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wh = host_weights(r["layer"].w)

@@ -106,11 +106,18 @@ typedef enum {
   MOE_WS_H = 11,         /* bf16 [max_rows, f] */
   MOE_WS_Y_PERM = 12,    /* f32  [max_rows, d] */
   MOE_WS_ROUTE = 13,     /* moe_route scratch */
-  MOE_WS_NUM_FIELDS = 14
+  MOE_WS_NUM_FIELDS = 14,
+  /* moe_layer_forward_fp8 only (after the fields above) */
+  MOE_WS_XQ = 14,        /* u8  [max_rows, d] e4m3 codes of x_perm */
+  MOE_WS_SX = 15,        /* f32 [max_rows]    their row scales */
+  MOE_WS_HQ = 16,        /* u8  [max_rows, f] e4m3 codes of h */
+  MOE_WS_SH = 17,        /* f32 [max_rows]    their row scales */
+  MOE_WS_FP8_NUM_FIELDS = 18
 } moe_ws_field;
 
 /* Byte offset of a field inside the moe_layer_forward workspace (each field
- * 256-byte aligned); -1 on bad args. */
+ * 256-byte aligned; fields MOE_WS_XQ .. MOE_WS_SH exist only in a
+ * moe_layer_forward_fp8 workspace); -1 on bad args. */
 int64_t moe_workspace_field_offset(int field, int64_t T, int64_t d, int64_t E, int64_t k,
                                    int64_t f, double cf);
 
@@ -219,34 +226,55 @@ int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, con
                 const int32_t* slot, const int32_t* offsets, int64_t T, int64_t d, int64_t k,
                 void* y, void* stream);
 
-/* ---- FP8 expert weights (weight-only e4m3; an optional variant) ----
- * Post-training FP8 quantization of the experts (inferensys.com glossary,
- * quantization entry) halves the weight bytes the layer streams, which is
- * what bounds decode-sized batches.  Activations, accumulation, h, y_perm and
- * y stay as in the bf16 path; each weight is q * s with q an e4m3 code and s
- * an fp32 scale per (expert, output column). */
+/* ---- FP8 experts (e4m3 activations and weights; an optional variant) ----
+ * Post-training FP8 quantization of the experts (inferensys.com "Expert
+ * Parallelism" glossary, quantization entry).  One rule for every group of
+ * values that shares a scale (a weight column over K, an activation row over
+ * K): s = max |v| / 448 in fp32 (1 for an all-zero group), code = e4m3 of
+ * v / s rounded to nearest even, saturating at +-448.  A row scale times a
+ * column scale is constant along the contraction, so the expert GEMMs run on
+ * the codes (tcgen05.mma.kind::f8f6f4, fp32 accumulation) and multiply each
+ * accumulator by its row and column scales.  Routing, the permutation, h as
+ * stored (bf16), y_perm (f32) and the combine are those of the bf16 path. */
 
 /* Quantize bf16 weights w [E,K,N] (N contiguous; gate/up: K=d, N=f; down:
- * K=f, N=d): scale[e,n] = max_k |w[e,k,n]| / 448 in fp32 (1 for an all-zero
- * column); w_q[e,k,n] = e4m3 code of w[e,k,n] / scale[e,n], rounded to
- * nearest even, saturating at +-448.  w_q u8 [E,K,N] out, scale f32 [E,N]
- * out. */
+ * K=f, N=d) per (expert, column n): scale [E,N] f32 out, codes w_q out
+ * stored K-major as u8 [E,N,K] (the transpose of w's layout).  Any K, N >= 1,
+ * E <= 65535.  A one-time preprocessing step. */
 int moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t N, uint8_t* w_q,
                              float* scale, void* stream);
 
-/* moe_expert_gate_up / moe_expert_down with e4m3 weights and their scales
- * (single-CTA tiles; the weights are widened exactly to bf16 in shared
- * memory, the column scales applied to the fp32 accumulators).  Arguments as
- * the bf16 entry points, all buffers 16-byte aligned. */
-int moe_expert_gate_up_fp8(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d,
-                           int64_t f, int64_t max_rows, const uint8_t* wq_gate,
+/* Quantize bf16 rows x [R,K] per row: codes q u8 [R,K], scale [R] f32.  Rows
+ * r >= *n_rows are skipped when n_rows (a device int32, e.g. offsets[E] of a
+ * permutation) is non-null.  K a multiple of 16; x and q 16-byte aligned. */
+int moe_quantize_rows_fp8(const void* x, int64_t R, int64_t K, const int32_t* n_rows, uint8_t* q,
+                          float* scale, void* stream);
+
+/* GEMM 1 + SwiGLU on e4m3 operands: h[r,:] = silu(g) * u with
+ * g[r,n] = sx[r] * s_gate[e,n] * sum_k xq[r,k] wq_gate[e,n,k] (u likewise) for
+ * rows r of bucket e.  xq u8 [max_rows,d], sx f32 [max_rows], wq_* u8 [E,f,d]
+ * (from moe_quantize_weights_fp8), s_* f32 [E,f]; h bf16 [max_rows,f] out.
+ * Shapes and errors as moe_expert_gate_up. */
+int moe_expert_gate_up_fp8(const uint8_t* xq, const float* sx, const int32_t* offsets, int64_t E,
+                           int64_t d, int64_t f, int64_t max_rows, const uint8_t* wq_gate,
                            const float* s_gate, const uint8_t* wq_up, const float* s_up, void* h,
                            int32_t* dev_status, void* stream);
-int moe_expert_down_fp8(const void* h, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
-                        int64_t max_rows, const uint8_t* wq_down, const float* s_down,
-                        float* y_perm, int32_t* dev_status, void* stream);
 
-/* moe_layer_forward with e4m3 expert weights (same workspace layout). */
+/* GEMM 2 on e4m3 operands: y_perm[r,n] = sh[r] * s_down[e,n] * sum_k
+ * hq[r,k] wq_down[e,n,k].  hq u8 [max_rows,f], sh f32 [max_rows], wq_down u8
+ * [E,d,f], s_down f32 [E,d]; y_perm f32 [max_rows,d] out. */
+int moe_expert_down_fp8(const uint8_t* hq, const float* sh, const int32_t* offsets, int64_t E,
+                        int64_t d, int64_t f, int64_t max_rows, const uint8_t* wq_down,
+                        const float* s_down, float* y_perm, int32_t* dev_status, void* stream);
+
+/* Workspace of moe_layer_forward_fp8: the moe_layer_forward fields followed by
+ * MOE_WS_XQ .. MOE_WS_SH (0 on invalid shapes). */
+size_t moe_workspace_size_fp8(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf);
+
+/* The layer with FP8 experts: moe_route, moe_permute, moe_quantize_rows_fp8
+ * (x_perm), moe_expert_gate_up_fp8, moe_quantize_rows_fp8 (h),
+ * moe_expert_down_fp8, moe_combine on `stream`.  Weights and scales from
+ * moe_quantize_weights_fp8; other arguments as moe_layer_forward. */
 int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bias,
                           const uint8_t* wq_gate, const float* s_gate, const uint8_t* wq_up,
                           const float* s_up, const uint8_t* wq_down, const float* s_down,

@@ -23,14 +23,15 @@ DEV_ERR_BAD_OFFSETS = 2
 
 # workspace fields of moe_layer_forward (enum moe_ws_field)
 WS_FIELDS = ["status", "logits", "topk_idx", "topk_w", "slot", "counts", "offsets", "n_dropped",
-             "row_src", "permute", "x_perm", "h", "y_perm", "route"]
+             "row_src", "permute", "x_perm", "h", "y_perm", "route", "xq", "sx", "hq", "sh"]
 
 EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "moe_capacity",
             "moe_max_rows",
             "moe_route_workspace_size", "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
             "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
             "moe_combine", "moe_layer_forward", "moe_quantize_weights_fp8",
-            "moe_expert_gate_up_fp8", "moe_expert_down_fp8", "moe_layer_forward_fp8"]
+            "moe_quantize_rows_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8",
+            "moe_workspace_size_fp8", "moe_layer_forward_fp8"]
 
 
 class MoEError(RuntimeError):
@@ -65,8 +66,11 @@ def _load():
         "moe_layer_forward": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl, p, p,
                                              sz, p]),
         "moe_quantize_weights_fp8": (ctypes.c_int, [p, i64, i64, i64, p, p, p]),
-        "moe_expert_gate_up_fp8": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p, p, p]),
-        "moe_expert_down_fp8": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p]),
+        "moe_quantize_rows_fp8": (ctypes.c_int, [p, i64, i64, p, p, p, p]),
+        "moe_expert_gate_up_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p, p,
+                                                  p]),
+        "moe_expert_down_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p]),
+        "moe_workspace_size_fp8": (sz, [i64, i64, i64, i64, i64, dbl]),
         "moe_layer_forward_fp8": (ctypes.c_int, [p, p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64,
                                                  dbl, p, p, sz, p]),
     }
@@ -319,69 +323,91 @@ def moe_layer_forward(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws
     return y, ws
 
 
-# ----------------------------------------------------------------- FP8 expert weights
+# ----------------------------------------------------------------- FP8 experts
 
 def moe_quantize_weights_fp8(w, stream=None):
-    """bf16 weights [E,K,N] -> (e4m3 codes uint8 [E,K,N], fp32 scales [E,N])."""
+    """bf16 weights [E,K,N] -> (e4m3 codes uint8 [E,N,K] (K-major), fp32 scales [E,N])."""
     E, K, N = w.shape
     _want(w, "w", torch.bfloat16)
-    q = torch.empty(E, K, N, dtype=torch.uint8, device=w.device)
+    q = torch.empty(E, N, K, dtype=torch.uint8, device=w.device)
     sc = torch.empty(E, N, dtype=torch.float32, device=w.device)
     _check("moe_quantize_weights_fp8",
            _lib.moe_quantize_weights_fp8(_ptr(w), E, K, N, _ptr(q), _ptr(sc), _stream(stream)))
     return q, sc
 
 
-def moe_expert_gate_up_fp8(x_perm, offsets, wq_gate, s_gate, wq_up, s_up, h=None, dev_status=None,
-                           stream=None):
-    rows, d = x_perm.shape
-    E, _, f = wq_gate.shape
-    _want(x_perm, "x_perm", torch.bfloat16)
+def moe_quantize_rows_fp8(x, n_rows=None, q=None, scale=None, stream=None):
+    """bf16 rows [R,K] -> (e4m3 codes uint8 [R,K], fp32 row scales [R])."""
+    R, K = x.shape
+    _want(x, "x", torch.bfloat16)
+    q = torch.empty(R, K, dtype=torch.uint8, device=x.device) if q is None else q
+    scale = torch.empty(R, dtype=torch.float32, device=x.device) if scale is None else scale
+    _want(q, "q", torch.uint8, (R, K))
+    _want(scale, "scale", torch.float32, (R,))
+    if n_rows is not None:
+        _want(n_rows, "n_rows", torch.int32)
+    _check("moe_quantize_rows_fp8", _lib.moe_quantize_rows_fp8(
+        _ptr(x), R, K, _ptr(n_rows), _ptr(q), _ptr(scale), _stream(stream)))
+    return q, scale
+
+
+def moe_expert_gate_up_fp8(xq, sx, offsets, wq_gate, s_gate, wq_up, s_up, h=None,
+                           dev_status=None, stream=None):
+    rows, d = xq.shape
+    E, f, _ = wq_gate.shape
+    _want(xq, "xq", torch.uint8)
+    _want(sx, "sx", torch.float32, (rows,))
     _want(offsets, "offsets", torch.int32, (E + 1,))
-    _want(wq_gate, "wq_gate", torch.uint8, (E, d, f))
-    _want(wq_up, "wq_up", torch.uint8, (E, d, f))
+    _want(wq_gate, "wq_gate", torch.uint8, (E, f, d))
+    _want(wq_up, "wq_up", torch.uint8, (E, f, d))
     _want(s_gate, "s_gate", torch.float32, (E, f))
     _want(s_up, "s_up", torch.float32, (E, f))
-    h = torch.empty(rows, f, dtype=torch.bfloat16, device=x_perm.device) if h is None else h
+    h = torch.empty(rows, f, dtype=torch.bfloat16, device=xq.device) if h is None else h
     _want(h, "h", torch.bfloat16, (rows, f))
     _check("moe_expert_gate_up_fp8", _lib.moe_expert_gate_up_fp8(
-        _ptr(x_perm), _ptr(offsets), E, d, f, rows, _ptr(wq_gate), _ptr(s_gate), _ptr(wq_up),
-        _ptr(s_up), _ptr(h), _ptr(dev_status), _stream(stream)))
+        _ptr(xq), _ptr(sx), _ptr(offsets), E, d, f, rows, _ptr(wq_gate), _ptr(s_gate),
+        _ptr(wq_up), _ptr(s_up), _ptr(h), _ptr(dev_status), _stream(stream)))
     return h
 
 
-def moe_expert_down_fp8(h, offsets, wq_down, s_down, y_perm=None, dev_status=None, stream=None):
-    rows, f = h.shape
-    E, _, d = wq_down.shape
-    _want(h, "h", torch.bfloat16)
+def moe_expert_down_fp8(hq, sh, offsets, wq_down, s_down, y_perm=None, dev_status=None,
+                        stream=None):
+    rows, f = hq.shape
+    E, d, _ = wq_down.shape
+    _want(hq, "hq", torch.uint8)
+    _want(sh, "sh", torch.float32, (rows,))
     _want(offsets, "offsets", torch.int32, (E + 1,))
-    _want(wq_down, "wq_down", torch.uint8, (E, f, d))
+    _want(wq_down, "wq_down", torch.uint8, (E, d, f))
     _want(s_down, "s_down", torch.float32, (E, d))
-    y_perm = torch.empty(rows, d, dtype=torch.float32, device=h.device) if y_perm is None \
+    y_perm = torch.empty(rows, d, dtype=torch.float32, device=hq.device) if y_perm is None \
         else y_perm
     _want(y_perm, "y_perm", torch.float32, (rows, d))
     _check("moe_expert_down_fp8", _lib.moe_expert_down_fp8(
-        _ptr(h), _ptr(offsets), E, d, f, rows, _ptr(wq_down), _ptr(s_down), _ptr(y_perm),
-        _ptr(dev_status), _stream(stream)))
+        _ptr(hq), _ptr(sh), _ptr(offsets), E, d, f, rows, _ptr(wq_down), _ptr(s_down),
+        _ptr(y_perm), _ptr(dev_status), _stream(stream)))
     return y_perm
+
+
+def moe_workspace_size_fp8(T, d, E, k, f, cf):
+    return int(_lib.moe_workspace_size_fp8(T, d, E, k, f, float(cf)))
 
 
 def moe_layer_forward_fp8(x, w_router, bias, wq_gate, s_gate, wq_up, s_up, wq_down, s_down, k, cf,
                           y=None, ws=None, stream=None):
-    """The whole layer with e4m3 expert weights.  Returns (y, ws)."""
+    """The whole layer with FP8 experts.  Returns (y, ws)."""
     T, d = x.shape
-    E, _, f = wq_gate.shape
+    E, f, _ = wq_gate.shape
     _want(x, "x", torch.bfloat16)
     _want(w_router, "w_router", torch.float32, (d, E))
     if bias is not None:
         _want(bias, "bias", torch.float32, (E,))
-    for name, t, shape in (("wq_gate", wq_gate, (E, d, f)), ("wq_up", wq_up, (E, d, f)),
-                           ("wq_down", wq_down, (E, f, d))):
+    for name, t, shape in (("wq_gate", wq_gate, (E, f, d)), ("wq_up", wq_up, (E, f, d)),
+                           ("wq_down", wq_down, (E, d, f))):
         _want(t, name, torch.uint8, shape)
     for name, t, shape in (("s_gate", s_gate, (E, f)), ("s_up", s_up, (E, f)),
                            ("s_down", s_down, (E, d))):
         _want(t, name, torch.float32, shape)
-    nbytes = moe_workspace_size(T, d, E, k, f, cf)
+    nbytes = moe_workspace_size_fp8(T, d, E, k, f, cf)
     if ws is None:
         ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
     _want(ws, "ws", torch.uint8)
@@ -404,6 +430,8 @@ def workspace_view(ws, field, T, d, E, k, f, cf):
         "offsets": (torch.int32, (E + 1,)), "n_dropped": (torch.int32, (1,)),
         "row_src": (torch.int32, (rows,)), "x_perm": (torch.bfloat16, (rows, d)),
         "h": (torch.bfloat16, (rows, f)), "y_perm": (torch.float32, (rows, d)),
+        "xq": (torch.uint8, (rows, d)), "sx": (torch.float32, (rows,)),
+        "hq": (torch.uint8, (rows, f)), "sh": (torch.float32, (rows,)),
     }[field]
     dtype, shape = spec
     off = moe_workspace_field_offset(field, T, d, E, k, f, cf)

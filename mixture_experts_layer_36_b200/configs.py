@@ -43,7 +43,12 @@ MIXTRAL_SLICE = MoEConfig("mixtral_slice", T=1024, d=4096, E=2, k=2, f=14336, cf
 # Same idea for the fine-grained layer: 16 of its 256 experts, 320 rows each.
 FINE_SLICE = MoEConfig("fine_slice", T=512, d=7168, E=16, k=8, f=2048, cf=1.25, seed=2)
 
-ALL = {c.name: c for c in (TINY, MIXTRAL, FINE, SKEWED, DECODE, MIXTRAL_SLICE, FINE_SLICE)}
+# And for the decode layer: 32 of its 256 experts with 8 rows each (as at
+# T = 256), about 4 GB of bf16 + e4m3 expert weights on the device.
+DECODE_SLICE = MoEConfig("decode_slice", T=32, d=7168, E=32, k=8, f=2048, cf=0.0, seed=4)
+
+ALL = {c.name: c for c in (TINY, MIXTRAL, FINE, SKEWED, DECODE, MIXTRAL_SLICE, FINE_SLICE,
+                           DECODE_SLICE)}
 
 
 def by_name(name: str) -> MoEConfig:

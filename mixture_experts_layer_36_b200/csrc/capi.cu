@@ -26,15 +26,19 @@ cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t s);
-cudaError_t launch_quantize_fp8(const __nv_bfloat16* w, int E, int K, int N, uint8_t* q,
-                                float* scale, cudaStream_t s);
-cudaError_t launch_gate_up_fp8(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
-                               int f, int max_rows, const uint8_t* wq_gate, const float* s_gate,
-                               const uint8_t* wq_up, const float* s_up, __nv_bfloat16* h,
-                               int32_t* status, cudaStream_t s, bool* map_failed);
-cudaError_t launch_down_fp8(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
-                            int max_rows, const uint8_t* wq_down, const float* s_down,
-                            float* y_perm, int32_t* status, cudaStream_t s, bool* map_failed);
+cudaError_t launch_quantize_weights(const __nv_bfloat16* w, int E, int K, int N, uint8_t* q,
+                                    float* scale, cudaStream_t s);
+cudaError_t launch_quantize_rows(const __nv_bfloat16* x, int R, int K, const int32_t* n_rows,
+                                 uint8_t* q, float* scale, cudaStream_t s);
+cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_t* offsets,
+                                int E, int d, int f, int max_rows, const uint8_t* wq_gate,
+                                const float* s_gate, const uint8_t* wq_up, const float* s_up,
+                                __nv_bfloat16* h, int32_t* status, cudaStream_t s,
+                                bool* map_failed);
+cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int32_t* offsets,
+                             int E, int d, int f, int max_rows, const uint8_t* wq_down,
+                             const float* s_down, float* y_perm, int32_t* status, cudaStream_t s,
+                             bool* map_failed);
 }  // namespace moe
 
 namespace moe {
@@ -109,6 +113,18 @@ bool field_sizes(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double c
   return true;
 }
 
+// Byte sizes of the FP8 layer's extra fields (after the standard ones).
+bool fp8_field_sizes(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf,
+                     size_t out[MOE_WS_FP8_NUM_FIELDS - MOE_WS_NUM_FIELDS]) {
+  const int64_t rows = moe_max_rows(T, E, k, cf);
+  if (rows < 0 || d < 1 || f < 1) return false;
+  out[MOE_WS_XQ - MOE_WS_NUM_FIELDS] = size_t(rows * d);
+  out[MOE_WS_SX - MOE_WS_NUM_FIELDS] = size_t(rows) * sizeof(float);
+  out[MOE_WS_HQ - MOE_WS_NUM_FIELDS] = size_t(rows * f);
+  out[MOE_WS_SH - MOE_WS_NUM_FIELDS] = size_t(rows) * sizeof(float);
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -167,10 +183,12 @@ size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k) {
 int64_t moe_workspace_field_offset(int field, int64_t T, int64_t d, int64_t E, int64_t k,
                                    int64_t f, double cf) {
   size_t sz[MOE_WS_NUM_FIELDS];
-  if (field < 0 || field >= MOE_WS_NUM_FIELDS) return -1;
-  if (!field_sizes(T, d, E, k, f, cf, sz)) return -1;
+  size_t sz8[MOE_WS_FP8_NUM_FIELDS - MOE_WS_NUM_FIELDS];
+  if (field < 0 || field >= MOE_WS_FP8_NUM_FIELDS) return -1;
+  if (!field_sizes(T, d, E, k, f, cf, sz) || !fp8_field_sizes(T, d, E, k, f, cf, sz8)) return -1;
   size_t off = 0;
-  for (int i = 0; i < field; ++i) off += align256(sz[i]);
+  for (int i = 0; i < field; ++i)
+    off += align256(i < MOE_WS_NUM_FIELDS ? sz[i] : sz8[i - MOE_WS_NUM_FIELDS]);
   return (int64_t)off;
 }
 
@@ -179,6 +197,15 @@ size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
   if (!field_sizes(T, d, E, k, f, cf, sz)) return 0;
   size_t off = 0;
   for (int i = 0; i < MOE_WS_NUM_FIELDS; ++i) off += align256(sz[i]);
+  return off;
+}
+
+size_t moe_workspace_size_fp8(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf) {
+  const size_t base = moe_workspace_size(T, d, E, k, f, cf);
+  size_t sz8[MOE_WS_FP8_NUM_FIELDS - MOE_WS_NUM_FIELDS];
+  if (base == 0 || !fp8_field_sizes(T, d, E, k, f, cf, sz8)) return 0;
+  size_t off = base;
+  for (int i = 0; i < MOE_WS_FP8_NUM_FIELDS - MOE_WS_NUM_FIELDS; ++i) off += align256(sz8[i]);
   return off;
 }
 
@@ -296,47 +323,58 @@ int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, con
 
 int moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t N, uint8_t* w_q,
                              float* scale, void* stream) {
-  if (E < 1 || K < 1 || N < 1 || E > 65535 || E * K * N >= (int64_t(1) << 40))
+  if (E < 1 || K < 1 || N < 1 || E > 65535 || K > (1 << 30) || N > (1 << 30) ||
+      E * K * N >= (int64_t(1) << 40))
     return MOE_ERR_INVALID_ARG;
   if (!w || !w_q || !scale) return MOE_ERR_INVALID_ARG;
-  return cuda_status(moe::launch_quantize_fp8(static_cast<const __nv_bfloat16*>(w), (int)E,
-                                              (int)K, (int)N, w_q, scale, as_stream(stream)));
+  return cuda_status(moe::launch_quantize_weights(static_cast<const __nv_bfloat16*>(w), (int)E,
+                                                  (int)K, (int)N, w_q, scale, as_stream(stream)));
 }
 
-int moe_expert_gate_up_fp8(const void* x_perm, const int32_t* offsets, int64_t E, int64_t d,
-                           int64_t f, int64_t max_rows, const uint8_t* wq_gate,
+int moe_quantize_rows_fp8(const void* x, int64_t R, int64_t K, const int32_t* n_rows, uint8_t* q,
+                          float* scale, void* stream) {
+  if (R < 0 || K < 16 || K % 16 != 0 || R >= (int64_t(1) << 31) || K > (1 << 30))
+    return MOE_ERR_INVALID_ARG;
+  if (R == 0) return MOE_OK;
+  if (!x || !q || !scale) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_quantize_rows(static_cast<const __nv_bfloat16*>(x), (int)R,
+                                               (int)K, n_rows, q, scale, as_stream(stream)));
+}
+
+int moe_expert_gate_up_fp8(const uint8_t* xq, const float* sx, const int32_t* offsets, int64_t E,
+                           int64_t d, int64_t f, int64_t max_rows, const uint8_t* wq_gate,
                            const float* s_gate, const uint8_t* wq_up, const float* s_up, void* h,
                            int32_t* dev_status, void* stream) {
   int st = check_gemm_args(E, d, f, max_rows);
   if (st != MOE_OK) return st;
   if (max_rows == 0) return MOE_OK;
-  if (!x_perm || !offsets || !wq_gate || !s_gate || !wq_up || !s_up || !h)
+  if (!xq || !sx || !offsets || !wq_gate || !s_gate || !wq_up || !s_up || !h)
     return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x_perm) || !aligned16(wq_gate) || !aligned16(wq_up) || !aligned16(s_gate) ||
+  if (!aligned16(xq) || !aligned16(wq_gate) || !aligned16(wq_up) || !aligned16(s_gate) ||
       !aligned16(s_up) || !aligned16(h))
     return MOE_ERR_INVALID_ARG;
   bool map_failed = false;
-  cudaError_t err = moe::launch_gate_up_fp8(
-      static_cast<const __nv_bfloat16*>(x_perm), offsets, (int)E, (int)d, (int)f, (int)max_rows,
-      wq_gate, s_gate, wq_up, s_up, static_cast<__nv_bfloat16*>(h), dev_status,
-      as_stream(stream), &map_failed);
+  cudaError_t err = moe::launch_gate_up_e4m3(
+      xq, sx, offsets, (int)E, (int)d, (int)f, (int)max_rows, wq_gate, s_gate, wq_up, s_up,
+      static_cast<__nv_bfloat16*>(h), dev_status, as_stream(stream), &map_failed);
   if (map_failed) return MOE_ERR_CUDA;
   return cuda_status(err);
 }
 
-int moe_expert_down_fp8(const void* h, const int32_t* offsets, int64_t E, int64_t d, int64_t f,
-                        int64_t max_rows, const uint8_t* wq_down, const float* s_down,
-                        float* y_perm, int32_t* dev_status, void* stream) {
+int moe_expert_down_fp8(const uint8_t* hq, const float* sh, const int32_t* offsets, int64_t E,
+                        int64_t d, int64_t f, int64_t max_rows, const uint8_t* wq_down,
+                        const float* s_down, float* y_perm, int32_t* dev_status, void* stream) {
   int st = check_gemm_args(E, d, f, max_rows);
   if (st != MOE_OK) return st;
   if (max_rows == 0) return MOE_OK;
-  if (!h || !offsets || !wq_down || !s_down || !y_perm) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(h) || !aligned16(wq_down) || !aligned16(s_down) || !aligned16(y_perm))
+  if (!hq || !sh || !offsets || !wq_down || !s_down || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hq) || !aligned16(wq_down) || !aligned16(s_down) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
   bool map_failed = false;
-  cudaError_t err = moe::launch_down_fp8(static_cast<const __nv_bfloat16*>(h), offsets, (int)E,
-                                         (int)d, (int)f, (int)max_rows, wq_down, s_down, y_perm,
-                                         dev_status, as_stream(stream), &map_failed);
+  cudaError_t err = moe::launch_down_e4m3(hq, sh, offsets, (int)E, (int)d, (int)f, (int)max_rows,
+                                          wq_down, s_down, y_perm, dev_status, as_stream(stream),
+                                          &map_failed);
   if (map_failed) return MOE_ERR_CUDA;
   return cuda_status(err);
 }
@@ -356,7 +394,7 @@ int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bia
       !ws)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
-  if (ws_bytes < moe_workspace_size(T, d, E, k, f, cf)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_workspace_size_fp8(T, d, E, k, f, cf)) return MOE_ERR_WORKSPACE;
   char* base = static_cast<char*>(ws);
   auto field = [&](int id) { return base + moe_workspace_field_offset(id, T, d, E, k, f, cf); };
   int32_t* status = reinterpret_cast<int32_t*>(field(MOE_WS_STATUS));
@@ -371,7 +409,12 @@ int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bia
   void* x_perm = field(MOE_WS_X_PERM);
   void* h = field(MOE_WS_H);
   float* y_perm = reinterpret_cast<float*>(field(MOE_WS_Y_PERM));
+  uint8_t* xq = reinterpret_cast<uint8_t*>(field(MOE_WS_XQ));
+  float* sx = reinterpret_cast<float*>(field(MOE_WS_SX));
+  uint8_t* hq = reinterpret_cast<uint8_t*>(field(MOE_WS_HQ));
+  float* shr = reinterpret_cast<float*>(field(MOE_WS_SH));
   const int64_t max_rows = moe_max_rows(T, E, k, cf);
+  const int32_t* n_rows = offsets + E;          // kept rows, written by the permutation
   cudaStream_t s = as_stream(stream);
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, field(MOE_WS_ROUTE),
@@ -381,11 +424,14 @@ int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bia
                         n_dropped, field(MOE_WS_PERMUTE), moe_permute_workspace_size(T, E, k),
                         stream)) != MOE_OK)
     return st;
-  if ((st = moe_expert_gate_up_fp8(x_perm, offsets, E, d, f, max_rows, wq_gate, s_gate, wq_up,
+  if ((st = moe_quantize_rows_fp8(x_perm, max_rows, d, n_rows, xq, sx, stream)) != MOE_OK)
+    return st;
+  if ((st = moe_expert_gate_up_fp8(xq, sx, offsets, E, d, f, max_rows, wq_gate, s_gate, wq_up,
                                    s_up, h, status, stream)) != MOE_OK)
     return st;
-  if ((st = moe_expert_down_fp8(h, offsets, E, d, f, max_rows, wq_down, s_down, y_perm, status,
-                                stream)) != MOE_OK)
+  if ((st = moe_quantize_rows_fp8(h, max_rows, f, n_rows, hq, shr, stream)) != MOE_OK) return st;
+  if ((st = moe_expert_down_fp8(hq, shr, offsets, E, d, f, max_rows, wq_down, s_down, y_perm,
+                                status, stream)) != MOE_OK)
     return st;
   return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
 }

@@ -135,6 +135,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D (+)= A * B with e4m3 A and B (K = 32 per instruction), fp32 accumulators
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on an mbarrier once every tcgen05.mma issued so far by this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -186,6 +197,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          | (1u << 10)                    // B format: bf16
          | (0u << 15)                    // A: K-major
          | ((b_mn_major ? 1u : 0u) << 16)
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// kind::f8f6f4 with e4m3 A and B (format code 0), both K-major, fp32 D
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                       // D format: f32
+         | (0u << 7) | (0u << 10)        // A, B format: e4m3
          | (static_cast<uint32_t>(N >> 3) << 17)
          | (static_cast<uint32_t>(M >> 4) << 24);
 }
@@ -268,34 +287,6 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
   const uint64_t t0 = global_timer_ns();
   while (global_timer_ns() - t0 < ns) {
   }
-}
-
-// ---------------------------------------------------------------- FP8 weights
-// Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (tensor-core operand reads) before signalling them on an mbarrier.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Four e4m3 bytes -> four bf16 (two 32-bit words), exactly.  The hardware
-// converts pairs of e4m3 to f16 (every e4m3 value is zero or a normal f16);
-// f16 -> bf16 then only re-biases the exponent (+112) and drops the three
-// mantissa bits that are zero here.
-__device__ __forceinline__ uint32_t f16x2_to_bf16x2_exact(uint32_t h) {
-  const uint32_t sign = h & 0x80008000u;
-  const uint32_t mag = h & 0x7FFF7FFFu;
-  uint32_t t = (mag >> 3) & 0x0FFF0FFFu;
-  if (mag & 0x00007FFFu) t += 112u << 7;
-  if (mag & 0x7FFF0000u) t += 112u << 23;
-  return t | sign;
-}
-__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  uint32_t h01, h23;
-  const uint16_t b01 = static_cast<uint16_t>(w & 0xFFFFu), b23 = static_cast<uint16_t>(w >> 16);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"(b01));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"(b23));
-  lo = f16x2_to_bf16x2_exact(h01);
-  hi = f16x2_to_bf16x2_exact(h23);
 }
 
 // ---------------------------------------------------------------- misc

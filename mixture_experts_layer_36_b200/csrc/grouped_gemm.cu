@@ -28,6 +28,10 @@
 // 2..5 drain the other accumulator (tcgen05.ld -> SwiGLU -> bf16 stores), so
 // the epilogue of tile i overlaps the main loop of tile i+1.
 //
+// FP8 experts (grouped_gemm_e4m3_kernel): the same tiles and roles on e4m3
+// activations and weights (tcgen05.mma.kind::f8f6f4), the per-row and
+// per-column fp32 quantization scales applied to the accumulators.
+//
 // Every mbarrier wait is time-limited: a role that gives up sets the CTA's
 // abort flag and the caller's status bit, the others notice and stop, the
 // producer waits for its copies in flight, the MMA issuer waits for its MMAs,
@@ -87,16 +91,18 @@ __device__ __forceinline__ void swiglu_pack(const uint32_t (&g)[32], const uint3
 
 __device__ __forceinline__ int clamp_rows(int v) { return v < 0 ? 0 : (v > 32 ? 32 : v); }
 
-// v[i] *= scale[i] for the 32 accumulator columns of a chunk (fp32 bits)
-__device__ __forceinline__ void apply_col_scales(uint32_t (&v)[32], const float* __restrict__ scale) {
-  const float4* s4 = reinterpret_cast<const float4*>(scale);
+// v[i] *= row_scale * col_scale[i] for the 32 accumulator columns of a chunk
+// (fp32 bits): the e4m3 GEMMs' per-row and per-column quantization scales
+__device__ __forceinline__ void apply_scales(uint32_t (&v)[32], const float* __restrict__ col_scale,
+                                             float row_scale) {
+  const float4* s4 = reinterpret_cast<const float4*>(col_scale);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 sc = __ldg(s4 + i);
-    v[4 * i + 0] = __float_as_uint(__uint_as_float(v[4 * i + 0]) * sc.x);
-    v[4 * i + 1] = __float_as_uint(__uint_as_float(v[4 * i + 1]) * sc.y);
-    v[4 * i + 2] = __float_as_uint(__uint_as_float(v[4 * i + 2]) * sc.z);
-    v[4 * i + 3] = __float_as_uint(__uint_as_float(v[4 * i + 3]) * sc.w);
+    v[4 * i + 0] = __float_as_uint(__uint_as_float(v[4 * i + 0]) * row_scale * sc.x);
+    v[4 * i + 1] = __float_as_uint(__uint_as_float(v[4 * i + 1]) * row_scale * sc.y);
+    v[4 * i + 2] = __float_as_uint(__uint_as_float(v[4 * i + 2]) * row_scale * sc.z);
+    v[4 * i + 3] = __float_as_uint(__uint_as_float(v[4 * i + 3]) * row_scale * sc.w);
   }
 }
 
@@ -142,37 +148,18 @@ __device__ __forceinline__ void decode_tile(const GemmShared& sh, int tile, int 
   m = local - n * mt;
 }
 
-// FP8W: the weights arrive as e4m3 codes [E, K, n_out] with fp32 column
-// scales [E, n_out] (tmB0/tmB1 unused).  Four more warps (6..9) each take
-// every fourth k-block: they load its fp8 weight tile with 16-byte loads,
-// widen it exactly to bf16 into the stage's swizzled B buffer, fence it to the
-// async proxy and arrive on the stage barrier (armed by the producer for the
-// A bytes only).  The epilogue multiplies each column by its scale.
-constexpr int kConvWarps = 4;
+// ---------------------------------------------------------------- roles
+// The pieces below are shared by the bf16 kernel and the e4m3-weight kernel.
 
-template <int BN, bool SWIGLU, bool FP8W = false>
-__global__ void __launch_bounds__(FP8W ? kGemmThreads + 32 * kConvWarps : kGemmThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
-                        const __grid_constant__ CUtensorMap tmB0,
-                        const __grid_constant__ CUtensorMap tmB1,
-                        const uint8_t* __restrict__ wq0, const uint8_t* __restrict__ wq1,
-                        const float* __restrict__ wscale0, const float* __restrict__ wscale1,
-                        const int32_t* __restrict__ offsets, int E, int K, int n_out,
-                        int max_rows, void* __restrict__ out_raw, int32_t* status) {
-  using Cfg = GemmCfg<BN, SWIGLU>;
-  extern __shared__ uint8_t dsmem_raw[];
-  __shared__ GemmShared sh;
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int n_tiles = n_out / Cfg::kOutCols;
-  const int nkb = K / kBK;
-
+// Barriers, TMEM, and the device-side tile list (warp 2: per-expert tile
+// counts -> exclusive prefix, bucket offsets to smem).
+__device__ __forceinline__ void gemm_setup(GemmShared& sh, int stages, int full_count,
+                                           int tmem_cols, const int32_t* offsets, int E,
+                                           int n_tiles, int max_rows, int32_t* status, int warp,
+                                           int lane) {
   if (threadIdx.x == 0) {
-    for (int s = 0; s < Cfg::kStages; ++s) {
-      mbar_init(&sh.full_bar[s], FP8W ? 2 : 1);     // + the converting warp
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&sh.full_bar[s], full_count);
       mbar_init(&sh.empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -185,17 +172,10 @@ __global__ void __launch_bounds__(FP8W ? kGemmThreads + 32 * kConvWarps : kGemmT
     fence_barrier_init();
   }
   if (warp == 0) {
-    tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
+    tmem_alloc(&sh.tmem_base, tmem_cols);
     tmem_relinquish();
   }
-  if (warp == 1 && lane == 0) {
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmA64);
-    if (!FP8W) prefetch_tensormap(&tmB0);
-    if (SWIGLU && !FP8W) prefetch_tensormap(&tmB1);
-  }
   if (warp == 2) {
-    // per-expert tile counts -> exclusive prefix; row offsets to smem
     int carry = 0;
     for (int base = 0; base < E; base += 32) {
       const int e = base + lane;
@@ -222,221 +202,334 @@ __global__ void __launch_bounds__(FP8W ? kGemmThreads + 32 * kConvWarps : kGemmT
     }
     if (lane == 0) sh.tile_prefix[E] = carry;
   }
+}
+
+// TMA producer (one thread): per k-block the A tile (128 or, for a bucket's
+// last <= 64 rows, 64 rows) and, through load_b(stage B buffer, bar, e, n,
+// kb), the weight tile.
+template <int STAGES, int STAGE_BYTES, int A_BYTES, int B_BYTES, class LoadB>
+__device__ __forceinline__ void producer_role(GemmShared& sh, uint8_t* smem,
+                                              const CUtensorMap* tmA, const CUtensorMap* tmA64,
+                                              int E, int n_tiles, int nkb, int32_t* status,
+                                              LoadB load_b, int kb_elems = kBK) {
+  volatile int* abort_flag = &sh.abort_flag;
+  const int total_tiles = sh.tile_prefix[E];
+  int it = 0;
+  int last_it[8];
+  for (int s = 0; s < STAGES; ++s) last_it[s] = -1;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+    int e, m, n;
+    decode_tile(sh, tile, E, n_tiles, e, m, n);
+    const int row0 = sh.row_off[e] + m * kBM;
+    const bool small = sh.row_cnt[e] - m * kBM <= kBM / 2;   // M = 64 tile
+    for (int kb = 0; kb < nkb; ++kb, ++it) {
+      const int s = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
+      uint8_t* sa = smem + s * STAGE_BYTES;
+      const uint32_t a_bytes = small ? A_BYTES / 2 : A_BYTES;
+      mbar_arrive_expect_tx(&sh.full_bar[s], a_bytes + B_BYTES);
+      if (small)
+        tma_load_2d(sa, tmA64, &sh.full_bar[s], kb * kb_elems, row0);
+      else
+        tma_load_2d(sa, tmA, &sh.full_bar[s], kb * kb_elems, row0);
+      load_b(sa + A_BYTES, &sh.full_bar[s], e, n, kb);
+      last_it[s] = it;
+    }
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    report(status, kDevErrWaitTimeout);
+  }
+  // never leave with copies in flight: every stage's last fill must land
+  for (int s = 0; s < STAGES; ++s)
+    if (last_it[s] >= 0) mbar_wait(&sh.full_bar[s], (last_it[s] / STAGES) & 1, &sh.never);
+}
+
+// MMA issuer (one thread): per k-block, four K = 16 MMAs from the stage into
+// accumulator buffer lt & 1; commits free the stage / hand the tile over.
+template <int BN, int STAGES, int STAGE_BYTES, int A_BYTES, bool E4M3 = false>
+__device__ __forceinline__ void mma_role(GemmShared& sh, uint8_t* smem, int E, int n_tiles,
+                                         int nkb, uint32_t idesc, uint32_t idesc64,
+                                         int32_t* status) {
+  volatile int* abort_flag = &sh.abort_flag;
+  const int total_tiles = sh.tile_prefix[E];
+  const uint32_t tmem_base = sh.tmem_base;
+  int it = 0, lt = 0;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++lt) {
+    int e, m, n;
+    decode_tile(sh, tile, E, n_tiles, e, m, n);
+    const uint32_t id = (sh.row_cnt[e] - m * kBM <= kBM / 2) ? idesc64 : idesc;
+    const int a = lt & 1;
+    const uint32_t aph = (lt >> 1) & 1;
+    if (!mbar_wait(&sh.tempty_bar[a], aph ^ 1, abort_flag)) { ok = false; break; }
+    tc_fence_after();
+    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BN);
+    for (int kb = 0; kb < nkb; ++kb, ++it) {
+      const int s = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      if (!mbar_wait(&sh.full_bar[s], ph, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+      const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        // A: K-major rows of 128 B, 8-row atoms 1024 B apart; +32 B per K step
+        // (16 bf16 or 32 e4m3 values)
+        const uint64_t adesc = smem_desc_sw128(a_addr + ks * 32, 16, 1024);
+        if (E4M3) {
+          // B: K-major like A (e4m3 weights are stored [E, N, K])
+          const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 32, 16, 1024);
+          umma_e4m3(d_tmem, adesc, bdesc, id, (kb | ks) != 0 ? 1u : 0u);
+        } else {
+          // B: MN-major; 64-wide N chunks 8 KB apart (LBO), 8-row K groups
+          // 1024 B apart (SBO); +16 K rows = +2048 B per K step
+          const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, kChunkBytes, 1024);
+          umma_bf16(d_tmem, adesc, bdesc, id, (kb | ks) != 0 ? 1u : 0u);
+        }
+      }
+      umma_commit(&sh.empty_bar[s]);
+    }
+    if (!ok) break;
+    umma_commit(&sh.tfull_bar[a]);
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    report(status, kDevErrWaitTimeout);
+  }
+  // wait until every MMA issued by this thread has finished
+  umma_commit(&sh.drain_bar);
+  mbar_wait(&sh.drain_bar, 0, &sh.never);
+}
+
+// Epilogue (warps 2..5): drain accumulator buffer lt & 1 of each tile
+// (tcgen05.ld -> [column scales] -> SwiGLU + bf16 stores, or fp32 stores).
+template <int BN, bool SWIGLU, bool SCALED>
+__device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, int warp,
+                                              int lane, int E, int n_tiles, int n_out,
+                                              void* out_raw, const float* row_scale,
+                                              const float* sc0, const float* sc1,
+                                              int32_t* status) {
+  constexpr int kOutCols = SWIGLU ? BN / 2 : BN;
+  volatile int* abort_flag = &sh.abort_flag;
+  const int total_tiles = sh.tile_prefix[E];
+  const uint32_t tmem_base = sh.tmem_base;
+  const int q = warp & 3;                 // TMEM lane quarter this warp may read
+  int lt = 0;
+  for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
+    int e, m, n;
+    decode_tile(sh, tile, E, n_tiles, e, m, n);
+    const int a = lt & 1;
+    const uint32_t aph = (lt >> 1) & 1;
+    if (!mbar_wait(&sh.tfull_bar[a], aph, abort_flag)) {
+      *abort_flag = 1;
+      report(status, kDevErrWaitTimeout);
+      break;
+    }
+    tc_fence_after();
+    // M = 64 tiles put rows 16q..16q+15 in TMEM lanes 32q..32q+15
+    const bool small = sh.row_cnt[e] - m * kBM <= kBM / 2;
+    const int rows_per_warp = small ? 16 : 32;
+    const int first = m * kBM + q * rows_per_warp;
+    int nvalid = clamp_rows(sh.row_cnt[e] - first);
+    if (nvalid > rows_per_warp) nvalid = rows_per_warp;
+    const size_t row0 = (size_t)sh.row_off[e] + first;
+    const size_t sc_off = (size_t)e * n_out + (size_t)n * kOutCols;
+    const float sr = (SCALED && lane < nvalid) ? row_scale[row0 + lane] : 0.f;
+    uint32_t* stage = reinterpret_cast<uint32_t*>(staging) + q * kStageWords;
+    const uint32_t tbase =
+        tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * BN);
+    if (SWIGLU) {
+      __nv_bfloat16* o =
+          static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out + (size_t)n * kOutCols;
+#pragma unroll 1
+      for (int c = 0; c < BN / 2 / 32; ++c) {
+        uint32_t g[32], u[32], pk[16];
+        tmem_ld_32x32b_x32(tbase + c * 32, g);
+        tmem_ld_32x32b_x32(tbase + BN / 2 + c * 32, u);
+        tmem_ld_wait();
+        if (SCALED) {
+          apply_scales(g, sc0 + sc_off + c * 32, sr);
+          apply_scales(u, sc1 + sc_off + c * 32, sr);
+        }
+        swiglu_pack(g, u, pk);
+        store_chunk_bf16(pk, o + c * 32, n_out, nvalid, lane);
+      }
+    } else {
+      float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * kOutCols;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + c * 32, v);
+        tmem_ld_wait();
+        if (SCALED) apply_scales(v, sc0 + sc_off + c * 32, sr);
+        store_chunk_f32(v, stage, o + c * 32, n_out, nvalid, lane);
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.tempty_bar[a]);
+  }
+}
+
+// ---------------------------------------------------------------- bf16 weights
+template <int BN, bool SWIGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1,
+                        const int32_t* __restrict__ offsets, int E, int K, int n_out,
+                        int max_rows, void* __restrict__ out_raw, int32_t* status) {
+  using Cfg = GemmCfg<BN, SWIGLU>;
+  extern __shared__ uint8_t dsmem_raw[];
+  __shared__ GemmShared sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_tiles = n_out / Cfg::kOutCols;
+  const int nkb = K / kBK;
+
+  gemm_setup(sh, Cfg::kStages, 1, Cfg::kTmemCols, offsets, E, n_tiles, max_rows, status, warp,
+             lane);
+  if (warp == 1 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmA64);
+    prefetch_tensormap(&tmB0);
+    if (SWIGLU) prefetch_tensormap(&tmB1);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
-  const uint32_t tmem_base = sh.tmem_base;
-  const int total_tiles = sh.tile_prefix[E];
-  volatile int* abort_flag = &sh.abort_flag;
-
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
-      int it = 0;
-      int last_it[8];
-      for (int s = 0; s < Cfg::kStages; ++s) last_it[s] = -1;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        int e, m, n;
-        decode_tile(sh, tile, E, n_tiles, e, m, n);
-        const int row0 = sh.row_off[e] + m * kBM;
+      auto load_b = [&](uint8_t* sb, uint64_t* bar, int e, int n, int kb) {
         const int col0 = n * Cfg::kOutCols;
-        const bool small = sh.row_cnt[e] - m * kBM <= kBM / 2;   // M = 64 tile
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % Cfg::kStages;
-          const uint32_t ph = (it / Cfg::kStages) & 1;
-          if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
-          uint8_t* sa = smem + s * Cfg::kStageBytes;
-          uint8_t* sb = sa + Cfg::kABytes;
-          const uint32_t a_bytes = small ? Cfg::kABytes / 2 : Cfg::kABytes;
-          mbar_arrive_expect_tx(&sh.full_bar[s], FP8W ? a_bytes : a_bytes + Cfg::kBBytes);
-          if (small)
-            tma_load_2d(sa, &tmA64, &sh.full_bar[s], kb * kBK, row0);
-          else
-            tma_load_2d(sa, &tmA, &sh.full_bar[s], kb * kBK, row0);
-          if (FP8W) {
-            // B is written by the converting warps
-          } else if (SWIGLU) {
+        if (SWIGLU) {
 #pragma unroll
-            for (int c = 0; c < BN / 128; ++c)
-              tma_load_3d(sb + c * kChunkBytes, &tmB0, &sh.full_bar[s], col0 + c * 64, kb * kBK, e);
+          for (int c = 0; c < BN / 128; ++c)
+            tma_load_3d(sb + c * kChunkBytes, &tmB0, bar, col0 + c * 64, kb * kBK, e);
 #pragma unroll
-            for (int c = 0; c < BN / 128; ++c)
-              tma_load_3d(sb + (BN / 128 + c) * kChunkBytes, &tmB1, &sh.full_bar[s],
-                          col0 + c * 64, kb * kBK, e);
-          } else {
+          for (int c = 0; c < BN / 128; ++c)
+            tma_load_3d(sb + (BN / 128 + c) * kChunkBytes, &tmB1, bar, col0 + c * 64, kb * kBK,
+                        e);
+        } else {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_3d(sb + c * kChunkBytes, &tmB0, &sh.full_bar[s], col0 + c * 64, kb * kBK, e);
-          }
-          last_it[s] = it;
+          for (int c = 0; c < BN / 64; ++c)
+            tma_load_3d(sb + c * kChunkBytes, &tmB0, bar, col0 + c * 64, kb * kBK, e);
         }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        report(status, kDevErrWaitTimeout);
-      }
-      // never leave with copies in flight: every stage's last fill must land
-      for (int s = 0; s < Cfg::kStages; ++s)
-        if (last_it[s] >= 0)
-          mbar_wait(&sh.full_bar[s], (last_it[s] / Cfg::kStages) & 1, &sh.never);
+      };
+      producer_role<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
+          sh, smem, &tmA, &tmA64, E, n_tiles, nkb, status, load_b);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------ MMA issuer
-      int it = 0, lt = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++lt) {
-        int e, m, n;
-        decode_tile(sh, tile, E, n_tiles, e, m, n);
-        const uint32_t idesc = (sh.row_cnt[e] - m * kBM <= kBM / 2) ? Cfg::kIdesc64 : Cfg::kIdesc;
-        const int a = lt & 1;
-        const uint32_t aph = (lt >> 1) & 1;
-        if (!mbar_wait(&sh.tempty_bar[a], aph ^ 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * BN);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % Cfg::kStages;
-          const uint32_t ph = (it / Cfg::kStages) & 1;
-          if (!mbar_wait(&sh.full_bar[s], ph, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * Cfg::kStageBytes);
-          const uint32_t b_addr = a_addr + Cfg::kABytes;
-#pragma unroll
-          for (int ks = 0; ks < kBK / kUmmaK; ++ks) {
-            // A: K-major rows of 128 B, 8-row atoms 1024 B apart; +32 B per K step
-            const uint64_t adesc = smem_desc_sw128(a_addr + ks * 32, 16, 1024);
-            // B: MN-major; 64-wide N chunks 8 KB apart (LBO), 8-row K groups
-            // 1024 B apart (SBO); +16 K rows = +2048 B per K step
-            const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, kChunkBytes, 1024);
-            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
-          }
-          umma_commit(&sh.empty_bar[s]);
-        }
-        if (!ok) break;
-        umma_commit(&sh.tfull_bar[a]);
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        report(status, kDevErrWaitTimeout);
-      }
-      // wait until every MMA issued by this thread has finished
-      umma_commit(&sh.drain_bar);
-      mbar_wait(&sh.drain_bar, 0, &sh.never);
-    }
-  } else if (warp < 6) {
-    // -------------------------------------------------- epilogue (warps 2..5)
-    const int q = warp & 3;                 // TMEM lane quarter this warp may read
-    int lt = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
-      int e, m, n;
-      decode_tile(sh, tile, E, n_tiles, e, m, n);
-      const int a = lt & 1;
-      const uint32_t aph = (lt >> 1) & 1;
-      if (!mbar_wait(&sh.tfull_bar[a], aph, abort_flag)) {
-        *abort_flag = 1;
-        report(status, kDevErrWaitTimeout);
-        break;
-      }
-      tc_fence_after();
-      // M = 64 tiles put rows 16q..16q+15 in TMEM lanes 32q..32q+15
-      const bool small = sh.row_cnt[e] - m * kBM <= kBM / 2;
-      const int rows_per_warp = small ? 16 : 32;
-      const int first = m * kBM + q * rows_per_warp;
-      int nvalid = clamp_rows(sh.row_cnt[e] - first);
-      if (nvalid > rows_per_warp) nvalid = rows_per_warp;
-      const size_t row0 = (size_t)sh.row_off[e] + first;
-      uint32_t* stage = reinterpret_cast<uint32_t*>(smem + Cfg::kStagingOff) + q * kStageWords;
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * BN);
-      if (SWIGLU) {
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out +
-                           (size_t)n * Cfg::kOutCols;
-#pragma unroll 1
-        for (int c = 0; c < BN / 2 / 32; ++c) {
-          uint32_t g[32], u[32], pk[16];
-          tmem_ld_32x32b_x32(tbase + c * 32, g);
-          tmem_ld_32x32b_x32(tbase + BN / 2 + c * 32, u);
-          tmem_ld_wait();
-          if (FP8W) {
-            const size_t sc = (size_t)e * n_out + (size_t)n * Cfg::kOutCols + c * 32;
-            apply_col_scales(g, wscale0 + sc);
-            apply_col_scales(u, wscale1 + sc);
-          }
-          swiglu_pack(g, u, pk);
-          store_chunk_bf16(pk, o + c * 32, n_out, nvalid, lane);
-        }
-      } else {
-        float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * Cfg::kOutCols;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tbase + c * 32, v);
-          tmem_ld_wait();
-          if (FP8W)
-            apply_col_scales(v, wscale0 + (size_t)e * n_out + (size_t)n * Cfg::kOutCols + c * 32);
-          store_chunk_f32(v, stage, o + c * 32, n_out, nvalid, lane);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.tempty_bar[a]);
-    }
-  } else if (FP8W) {
-    // -------------------------------------------------- fp8 -> bf16 weights (warps 6..9)
-    const int cw = warp - 6;
-    constexpr int kVecPerRow = FP8W && SWIGLU ? BN / 2 / 16 : BN / 16;   // 16-B vectors per K row
-    constexpr int kVecPerOp = kBK * kVecPerRow;
-    constexpr int kVecs = SWIGLU ? 2 * kVecPerOp : kVecPerOp;            // per k-block
-    int it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-      int e, m, n;
-      decode_tile(sh, tile, E, n_tiles, e, m, n);
-      const int col0 = n * Cfg::kOutCols;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        if (it % kConvWarps != cw) continue;
-        const int s = it % Cfg::kStages;
-        const uint32_t ph = (it / Cfg::kStages) & 1;
-        if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
-        uint8_t* sb = smem + s * Cfg::kStageBytes + Cfg::kABytes;
-#pragma unroll 4
-        for (int v = lane; v < kVecs; v += 32) {
-          const int op = SWIGLU ? v / kVecPerOp : 0;
-          const int rem = v - op * kVecPerOp;
-          const int k = rem / kVecPerRow, c16 = rem % kVecPerRow;
-          const uint8_t* src = (op ? wq1 : wq0) +
-                               ((size_t)e * K + (size_t)kb * kBK + k) * n_out + col0 + c16 * 16;
-          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
-          uint4 lo, hi;
-          e4m3x4_to_bf16x4(raw.x, lo.x, lo.y);
-          e4m3x4_to_bf16x4(raw.y, lo.z, lo.w);
-          e4m3x4_to_bf16x4(raw.z, hi.x, hi.y);
-          e4m3x4_to_bf16x4(raw.w, hi.z, hi.w);
-          // 64-column chunk and 16-byte unit inside the 128-byte swizzled row
-          const int chunk = (SWIGLU ? op * (BN / 128) : 0) + (c16 >> 2);
-          const int unit = (c16 & 3) * 2;
-          uint8_t* row = sb + chunk * kChunkBytes + k * 128;
-          *reinterpret_cast<uint4*>(row + ((unit ^ (k & 7)) << 4)) = lo;
-          *reinterpret_cast<uint4*>(row + (((unit + 1) ^ (k & 7)) << 4)) = hi;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.full_bar[s]);
-      }
-    }
-    if (!ok) {
-      *abort_flag = 1;
-      report(status, kDevErrWaitTimeout);
-    }
+    if (lane == 0)
+      mma_role<BN, Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes>(sh, smem, E, n_tiles, nkb,
+                                                                 Cfg::kIdesc, Cfg::kIdesc64,
+                                                                 status);
+  } else {
+    epilogue_role<BN, SWIGLU, false>(sh, smem + Cfg::kStagingOff, warp, lane, E, n_tiles, n_out,
+                                     out_raw, nullptr, nullptr, nullptr, status);
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    tmem_dealloc(sh.tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- e4m3 operands
+// FP8 experts: activations and weights both e4m3, the activations with one
+// fp32 scale per row, the weights with one per (expert, output column); both
+// operands K-major (weights stored [E, N, K]).  The same tiles and roles as
+// the bf16 kernel, a 128-deep K block per stage (one 128-byte swizzle row of
+// e4m3) and tcgen05.mma.kind::f8f6f4 (K = 32 per instruction); the epilogue
+// multiplies each accumulator by its row and column scales.
+template <int BN, bool SWIGLU>
+struct E4m3Cfg {
+  static constexpr int kBKe = 128;                    // e4m3 values per k-block
+  static constexpr int kOutCols = SWIGLU ? BN / 2 : BN;
+  static constexpr int kABytes = kBM * kBKe;
+  static constexpr int kBBytes = BN * kBKe;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kStagingOff = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kStagingOff + 4 * kStageWords * 4 + 1024;
+  static constexpr uint32_t kIdesc = idesc_e4m3_f32(kBM, BN);
+  static constexpr uint32_t kIdesc64 = idesc_e4m3_f32(kBM / 2, BN);
+};
+
+template <int BN, bool SWIGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,     // codes [rows, K]
+                             const __grid_constant__ CUtensorMap tmA64,
+                             const __grid_constant__ CUtensorMap tmB0,    // codes [E, N, K]
+                             const __grid_constant__ CUtensorMap tmB1,    // (SwiGLU: up)
+                             const float* __restrict__ row_scale,
+                             const float* __restrict__ col_scale0,
+                             const float* __restrict__ col_scale1,
+                             const int32_t* __restrict__ offsets, int E, int K, int n_out,
+                             int max_rows, void* __restrict__ out_raw, int32_t* status) {
+  using Cfg = E4m3Cfg<BN, SWIGLU>;
+  extern __shared__ uint8_t dsmem_raw[];
+  __shared__ GemmShared sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_tiles = n_out / Cfg::kOutCols;
+  const int nkb = K / Cfg::kBKe;
+
+  gemm_setup(sh, Cfg::kStages, 1, Cfg::kTmemCols, offsets, E, n_tiles, max_rows, status, warp,
+             lane);
+  if (warp == 1 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmA64);
+    prefetch_tensormap(&tmB0);
+    if (SWIGLU) prefetch_tensormap(&tmB1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // B: 128 weight rows (output columns) x 128 K per copy
+      auto load_b = [&](uint8_t* sb, uint64_t* bar, int e, int n, int kb) {
+        const int col0 = n * Cfg::kOutCols;
+        if (SWIGLU) {
+          tma_load_3d(sb, &tmB0, bar, kb * Cfg::kBKe, col0, e);
+          tma_load_3d(sb + 128 * Cfg::kBKe, &tmB1, bar, kb * Cfg::kBKe, col0, e);
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN / 128; ++c)
+            tma_load_3d(sb + c * 128 * Cfg::kBKe, &tmB0, bar, kb * Cfg::kBKe, col0 + c * 128, e);
+        }
+      };
+      producer_role<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
+          sh, smem, &tmA, &tmA64, E, n_tiles, nkb, status, load_b, Cfg::kBKe);
+    }
+  } else if (warp == 1) {
+    if (lane == 0)
+      mma_role<BN, Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, true>(
+          sh, smem, E, n_tiles, nkb, Cfg::kIdesc, Cfg::kIdesc64, status);
+  } else {
+    epilogue_role<BN, SWIGLU, true>(sh, smem + Cfg::kStagingOff, warp, lane, E, n_tiles, n_out,
+                                    out_raw, row_scale, col_scale0, col_scale1, status);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(sh.tmem_base, Cfg::kTmemCols);
   }
 }
 
@@ -767,19 +860,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-template <int BN, bool SWIGLU, bool FP8W = false>
+template <int BN, bool SWIGLU>
 static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& a64,
                                const CUtensorMap& b0, const CUtensorMap& b1,
                                const int32_t* offsets, int E, int K,
                                int n_out, int max_rows, void* out, int32_t* status,
-                               cudaStream_t s, const uint8_t* wq0 = nullptr,
-                               const uint8_t* wq1 = nullptr, const float* ws0 = nullptr,
-                               const float* ws1 = nullptr) {
+                               cudaStream_t s) {
   using Cfg = GemmCfg<BN, SWIGLU>;
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  auto kern = grouped_gemm_kernel<BN, SWIGLU, FP8W>;
+  auto kern = grouped_gemm_kernel<BN, SWIGLU>;
   if (!di->attr_set[slot]) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg::kSmemBytes);
@@ -791,9 +882,8 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
   long long ub = row_tiles * n_tiles;
   int grid = (int)(ub < di->sms ? ub : di->sms);
   if (grid < 1) grid = 1;
-  const int threads = FP8W ? kGemmThreads + 32 * kConvWarps : kGemmThreads;
-  kern<<<grid, threads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, wq0, wq1, ws0, ws1, offsets, E, K,
-                                              n_out, max_rows, out, status);
+  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, offsets, E, K, n_out,
+                                                     max_rows, out, status);
   return cudaGetLastError();
 }
 
@@ -871,30 +961,63 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
                                  s);
 }
 
-// GEMM 1 / GEMM 2 with e4m3 weights and fp32 column scales (single-CTA tiles)
-cudaError_t launch_gate_up_fp8(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
-                               int f, int max_rows, const uint8_t* wq_gate, const float* s_gate,
-                               const uint8_t* wq_up, const float* s_up, __nv_bfloat16* h,
-                               int32_t* status, cudaStream_t s, bool* map_failed) {
-  CUtensorMap ta, ta64;
-  *map_failed = !(map_rows(&ta, x_perm, d, max_rows, kBM) &&
-                  map_rows(&ta64, x_perm, d, max_rows, kBM / 2));
-  if (*map_failed) return cudaSuccess;
-  return launch_gemm<256, true, true>(11, ta, ta64, ta, ta, offsets, E, d, f, max_rows, h, status,
-                                      s, wq_gate, wq_up, s_gate, s_up);
+template <int BN, bool SWIGLU>
+static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+                                    const CUtensorMap& b0, const CUtensorMap& b1,
+                                    const float* row_scale, const float* s0, const float* s1,
+                                    const int32_t* offsets, int E, int K, int n_out, int max_rows,
+                                    void* out, int32_t* status, cudaStream_t s) {
+  using Cfg = E4m3Cfg<BN, SWIGLU>;
+  DeviceInfo* di = nullptr;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  auto kern = grouped_gemm_e4m3_kernel<BN, SWIGLU>;
+  if (!di->attr_set[slot]) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    di->attr_set[slot] = true;
+  }
+  const int n_tiles = n_out / Cfg::kOutCols;
+  const long long row_tiles = (long long)max_rows / kBM + (E < max_rows ? E : max_rows);
+  long long ub = row_tiles * n_tiles;
+  int grid = (int)(ub < di->sms ? ub : di->sms);
+  if (grid < 1) grid = 1;
+  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, row_scale, s0, s1, offsets, E,
+                                                   K, n_out, max_rows, out, status);
+  return cudaGetLastError();
 }
 
-cudaError_t launch_down_fp8(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
-                            int max_rows, const uint8_t* wq_down, const float* s_down,
-                            float* y_perm, int32_t* status, cudaStream_t s, bool* map_failed) {
-  CUtensorMap ta, ta64;
-  *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_rows(&ta64, h, f, max_rows, kBM / 2));
+// GEMM 1 / GEMM 2 on e4m3 rows (per-row scales) and e4m3 weights stored
+// [E, N, K] (per-column scales); single-CTA tiles
+cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_t* offsets,
+                                int E, int d, int f, int max_rows, const uint8_t* wq_gate,
+                                const float* s_gate, const uint8_t* wq_up, const float* s_up,
+                                __nv_bfloat16* h, int32_t* status, cudaStream_t s,
+                                bool* map_failed) {
+  CUtensorMap ta, ta64, tg, tu;
+  *map_failed = !(map_rows_e4m3(&ta, xq, d, max_rows, kBM) &&
+                  map_rows_e4m3(&ta64, xq, d, max_rows, kBM / 2) &&
+                  map_weights_e4m3(&tg, wq_gate, E, f, d) && map_weights_e4m3(&tu, wq_up, E, f, d));
+  if (*map_failed) return cudaSuccess;
+  return launch_gemm_e4m3<256, true>(11, ta, ta64, tg, tu, sx, s_gate, s_up, offsets, E, d, f,
+                                     max_rows, h, status, s);
+}
+
+cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int32_t* offsets,
+                             int E, int d, int f, int max_rows, const uint8_t* wq_down,
+                             const float* s_down, float* y_perm, int32_t* status, cudaStream_t s,
+                             bool* map_failed) {
+  CUtensorMap ta, ta64, td;
+  *map_failed = !(map_rows_e4m3(&ta, hq, f, max_rows, kBM) &&
+                  map_rows_e4m3(&ta64, hq, f, max_rows, kBM / 2) &&
+                  map_weights_e4m3(&td, wq_down, E, d, f));
   if (*map_failed) return cudaSuccess;
   if (d % 256 == 0)
-    return launch_gemm<256, false, true>(12, ta, ta64, ta, ta, offsets, E, f, d, max_rows, y_perm,
-                                         status, s, wq_down, nullptr, s_down, nullptr);
-  return launch_gemm<128, false, true>(13, ta, ta64, ta, ta, offsets, E, f, d, max_rows, y_perm,
-                                       status, s, wq_down, nullptr, s_down, nullptr);
+    return launch_gemm_e4m3<256, false>(12, ta, ta64, td, td, sh_rows, s_down, nullptr, offsets,
+                                        E, f, d, max_rows, y_perm, status, s);
+  return launch_gemm_e4m3<128, false>(13, ta, ta64, td, td, sh_rows, s_down, nullptr, offsets, E,
+                                      f, d, max_rows, y_perm, status, s);
 }
 
 int device_sm_count() {

@@ -70,7 +70,15 @@ def test_workspace_layout(cfg):
     for i, n in need.items():
         assert ends[i] - offs[i] >= n, binding.WS_FIELDS[i]
     assert moe.moe_route_workspace_size(T, d, E, k) >= 2 * d * ((E + 63) // 64 * 64) * 2
-    assert moe.moe_workspace_field_offset(14, T, d, E, k, f, cf) == -1
+    # the FP8 layer's extra fields follow the standard ones
+    total8 = moe.moe_workspace_size_fp8(T, d, E, k, f, cf)
+    offs8 = [moe.moe_workspace_field_offset(i, T, d, E, k, f, cf) for i in range(14, 18)]
+    assert offs8[0] == total and all(o % 256 == 0 for o in offs8) and offs8 == sorted(offs8)
+    ends8 = offs8[1:] + [total8]
+    for i, n in enumerate((rows * d, rows * 4, rows * f, rows * 4)):
+        assert ends8[i] - offs8[i] >= n, binding.WS_FIELDS[14 + i]
+    assert moe.moe_workspace_field_offset(18, T, d, E, k, f, cf) == -1
+    assert moe.moe_workspace_field_offset(-1, T, d, E, k, f, cf) == -1
 
 
 def test_validation_codes_without_launch():

@@ -1,13 +1,14 @@
-"""GPU parity for the FP8 (e4m3) expert-weight variant, through the C ABI,
-against the CPU oracle:
-  * the weight quantizer: codes and scales bit-exact;
-  * the grouped gate/up and down GEMMs on e4m3 weights against the oracle's
-    expert evaluated on its own dequantized weights (same tolerances as the
-    bf16 path: h within one bf16 rounding, y_perm within 2e-2 rms);
-  * the whole layer with e4m3 experts, small workloads element by element and
-    the decode-sized workloads on sampled tokens.
-The oracle's quantization (codes and scales) is what the GPU GEMMs are fed, so
-every expected value comes from the oracle alone.
+"""GPU parity for the FP8 expert variant (e4m3 activations and weights, fp32
+row and column scales), through the C ABI, against the CPU oracle:
+  * the weight quantizer and the row quantizer: codes and scales bit-exact
+    (the weights come back K-major, the transpose of the oracle's layout);
+  * the grouped gate/up and down GEMMs on e4m3 operands against the oracle's
+    expert on the dequantized operands: h within one bf16 rounding, y_perm
+    within 2e-2 rms (the bf16 path's tolerances);
+  * the whole layer, small workloads element by element and the decode-sized
+    workloads on sampled tokens.
+Where floating point decides a code (the quantization of h), the oracle
+quantizes the GPU's own h, after that h has been checked against the oracle's.
 """
 import numpy as np
 import pytest
@@ -42,23 +43,101 @@ def edge_weights(E, K, N, seed, std):
     return w
 
 
-def quantize_oracle(w):
+def quantize_w(w):
+    """Oracle quantization of bf16 weights [E,K,N]: codes [E,K,N], scales [E,N]."""
     q, s = oracle.quantize_fp8(bits(w))
-    return torch.from_numpy(q), torch.from_numpy(s)
+    return q, s
 
 
-def dequant(q, s):
-    return oracle.dequant_fp8(q.numpy(), s.numpy())
+def kmajor(q):
+    """Oracle codes [E,K,N] -> the GPU's K-major layout [E,N,K] on the device."""
+    return torch.from_numpy(np.ascontiguousarray(q.transpose(0, 2, 1))).cuda()
 
 
 @pytest.mark.parametrize("E,K,N", [(3, 64, 40), (8, 256, 384), (2, 1000, 129)])
-def test_quantizer_bit_exact(E, K, N):
+def test_weight_quantizer_bit_exact(E, K, N):
     w = edge_weights(E, K, N, E + K + N, 0.05)
     q, s = moe.moe_quantize_weights_fp8(w.cuda())
     torch.cuda.synchronize()
-    q_ref, s_ref = quantize_oracle(w)
-    assert torch.equal(s.cpu(), s_ref)       # fp32 bit patterns (no NaN is possible)
-    assert torch.equal(q.cpu(), q_ref)
+    q_ref, s_ref = quantize_w(w)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy().transpose(0, 2, 1), q_ref)
+
+
+@pytest.mark.parametrize("R,K,n_rows", [(37, 96, None), (300, 256, 211), (9, 7168, None)])
+def test_row_quantizer_bit_exact(R, K, n_rows):
+    g = torch.Generator().manual_seed(R + K)
+    x = (torch.randn(R, K, generator=g) * 3).to(torch.bfloat16)
+    x[1] = 0                                         # all-zero row
+    x[2, :] = 0
+    x[2, 5] = 1e-30                                  # fp32-subnormal scale
+    x[3, 7] = -2e5                                   # the rest of the row: small codes
+    x[4, :] = 460.0                                  # saturating quotients
+    q = torch.full((R, K), 0x55, dtype=torch.uint8, device="cuda")
+    s = torch.full((R,), -1.0, dtype=torch.float32, device="cuda")
+    nr = None if n_rows is None else torch.tensor([n_rows], dtype=torch.int32, device="cuda")
+    moe.moe_quantize_rows_fp8(x.cuda(), n_rows=nr, q=q, scale=s)
+    torch.cuda.synchronize()
+    n = R if n_rows is None else n_rows
+    q_ref, s_ref = oracle.quantize_rows_fp8(bits(x[:n]))
+    np.testing.assert_array_equal(s[:n].cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q[:n].cpu().numpy(), q_ref)
+    assert torch.all(q[n:] == 0x55) and torch.all(s[n:] == -1.0)   # rows past n_rows untouched
+
+
+def deq_rows(q, s):
+    return oracle.dequant_rows_fp8(q, s)
+
+
+def run_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, max_rows, d, f):
+    """GPU: gate/up on (xq, sx), the row quantizer on h, down.  Inputs numpy
+    (weights in the oracle's [E,K,N] layout).  Returns (h, hq, sh, y) on the host."""
+    N = int(offsets[-1])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    off = torch.from_numpy(offsets).cuda()
+    xq_d = torch.zeros(max_rows, d, dtype=torch.uint8, device="cuda")
+    sx_d = torch.zeros(max_rows, dtype=torch.float32, device="cuda")
+    xq_d[:N] = torch.from_numpy(xq).cuda()
+    sx_d[:N] = torch.from_numpy(sx).cuda()
+    sentinel = -7.0
+    h = torch.full((max_rows, f), sentinel, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((max_rows, d), sentinel, dtype=torch.float32, device="cuda")
+    moe.moe_expert_gate_up_fp8(xq_d, sx_d, off, kmajor(qg), torch.from_numpy(sg).cuda(),
+                               kmajor(qu), torch.from_numpy(su).cuda(), h=h, dev_status=status)
+    hq, sh = moe.moe_quantize_rows_fp8(h, n_rows=off[-1:])
+    moe.moe_expert_down_fp8(hq, sh, off, kmajor(qd), torch.from_numpy(sd).cuda(), y_perm=y,
+                            dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.all(h[N:] == sentinel) and torch.all(y[N:] == sentinel)
+    return h[:N], hq[:N].cpu().numpy(), sh[:N].cpu().numpy(), y[:N]
+
+
+def check_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, h, hq, sh, y):
+    """Oracle check of one GPU expert-MLP pass (see run_mlp)."""
+    N, f = h.shape
+    d = y.shape[1]
+    E = len(offsets) - 1
+    a = deq_rows(xq, sx)
+    g64, u64, d64 = oracle.dequant_fp8(qg, sg), oracle.dequant_fp8(qu, su), \
+        oracle.dequant_fp8(qd, sd)
+    o_h = np.zeros((N, f))
+    for e in range(E):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            o_h[lo:hi] = oracle.gate_up_f64(a[lo:hi], g64[e], u64[e])
+    assert_bf16_rounding_close(f64(h), o_h, "h")
+    # the codes of h: the oracle's quantizer on the GPU's h, bit for bit
+    hq_ref, sh_ref = oracle.quantize_rows_fp8(bits(h))
+    np.testing.assert_array_equal(sh.view(np.uint32), sh_ref.view(np.uint32))
+    np.testing.assert_array_equal(hq, hq_ref)
+    b = deq_rows(hq_ref, sh_ref)
+    o_y = np.zeros((N, d))
+    for e in range(E):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            o_y[lo:hi] = oracle.matmul_f64(b[lo:hi], d64[e])
+    assert_bf16_close(f64(y), o_y, "y_perm")
 
 
 MLP_CASES = [
@@ -78,57 +157,38 @@ def test_expert_mlp_fp8_matches_oracle(d, f, sizes):
     E = len(sizes)
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     N = int(offsets[-1])
-    max_rows = N + 37
     g = torch.Generator().manual_seed(3 * d + f + E)
-    x_perm = torch.randn(max_rows, d, generator=g).to(torch.bfloat16)
-    wg = edge_weights(E, d, f, d + 1, d ** -0.5)
-    wu = edge_weights(E, d, f, d + 2, d ** -0.5)
-    wd = edge_weights(E, f, d, d + 3, f ** -0.5)
-    (qg, sg), (qu, su), (qd, sd) = (quantize_oracle(w) for w in (wg, wu, wd))
-    sentinel = -7.0
-    h = torch.full((max_rows, f), sentinel, dtype=torch.bfloat16, device="cuda")
-    y = torch.full((max_rows, d), sentinel, dtype=torch.float32, device="cuda")
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    off = torch.from_numpy(offsets).cuda()
-    moe.moe_expert_gate_up_fp8(x_perm.cuda(), off, qg.cuda(), sg.cuda(), qu.cuda(), su.cuda(),
-                               h=h, dev_status=status)
-    moe.moe_expert_down_fp8(h, off, qd.cuda(), sd.cuda(), y_perm=y, dev_status=status)
-    torch.cuda.synchronize()
-    assert status.item() == 0
-    g64, u64, d64 = dequant(qg, sg), dequant(qu, su), dequant(qd, sd)
-    xb = bits(x_perm[:N])
-    o_h, o_y = np.zeros((N, f)), np.zeros((N, d))
-    for e in range(E):
-        a, b = offsets[e], offsets[e + 1]
-        if b > a:
-            o_h[a:b], o_y[a:b] = oracle.swiglu_rows_f64w(xb[a:b], g64[e], u64[e], d64[e],
-                                                         want_h=True)
-    assert_bf16_rounding_close(f64(h[:N]), o_h, "h")
-    assert_bf16_close(f64(y[:N]), o_y, "y_perm")
-    assert torch.all(h[N:] == sentinel) and torch.all(y[N:] == sentinel)
+    x_perm = torch.randn(N, d, generator=g).to(torch.bfloat16)
+    xq, sx = oracle.quantize_rows_fp8(bits(x_perm))
+    qg, sg = quantize_w(edge_weights(E, d, f, d + 1, d ** -0.5))
+    qu, su = quantize_w(edge_weights(E, d, f, d + 2, d ** -0.5))
+    qd, sd = quantize_w(edge_weights(E, f, d, d + 3, f ** -0.5))
+    out = run_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, N + 37, d, f)
+    check_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, *out)
 
 
-def oracle_layer_fp8(cpu, k, cf, gl, q):
-    """The layer on the oracle's dequantized experts, routed on the GPU's fp32
-    logits (the arg-max decision is taken in the kernel's precision)."""
-    x_bits = bits(cpu["x"])
-    T, d = x_bits.shape
-    E = cpu["w_gate"].shape[0]
-    o_idx, o_w = oracle.topk(gl, k)
-    C = oracle.capacity(T, E, k, cf)
-    counts, offsets, slot, row_src, n_drop = oracle.permute(o_idx, E, C)
-    x_perm = oracle.dispatch(x_bits, row_src)
-    f = cpu["w_gate"].shape[2]
-    y_perm = np.zeros((int(offsets[-1]), d))
-    for e in range(E):
-        a, b = offsets[e], offsets[e + 1]
-        if b > a:
-            wg, wu, wd = (oracle.dequant_fp8(q[n][0][e:e + 1].numpy(), q[n][1][e:e + 1].numpy())[0]
-                          for n in ("w_gate", "w_up", "w_down"))
-            _, y_perm[a:b] = oracle.swiglu_rows_f64w(x_perm[a:b], wg, wu, wd)
-    y = oracle.combine(y_perm, x_bits, o_idx, o_w, slot, offsets)
-    return dict(topk_idx=o_idx, topk_w=o_w, slot=slot, counts=counts, offsets=offsets,
-                n_dropped=n_drop, y=y, f=f)
+def random_codes(shape, rng):
+    """Every finite e4m3 code, drawn uniformly (zero and subnormals included)."""
+    q = rng.integers(0, 256, size=shape, dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] -= 1                       # no NaN codes
+    return q
+
+
+def test_expert_mlp_fp8_every_code():
+    d, f, sizes = 256, 384, [70, 0, 129, 1]
+    E = len(sizes)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    N = int(offsets[-1])
+    rng = np.random.default_rng(31)
+    xq = random_codes((N, d), rng)
+    sx = rng.uniform(0.5, 2, N).astype(np.float32) / 64
+    qg, qu, qd = random_codes((E, d, f), rng), random_codes((E, d, f), rng), \
+        random_codes((E, f, d), rng)
+    sg, su = (rng.uniform(0.5, 2, (E, f)).astype(np.float32) / (64 * d ** 0.5) for _ in range(2))
+    sd = rng.uniform(0.5, 2, (E, d)).astype(np.float32) / (64 * f ** 0.5)
+    assert ((qg & 0x78) == 0).any() and (qg == 0).any() and ((xq & 0x78) == 0).any()
+    out = run_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, N + 5, d, f)
+    check_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, *out)
 
 
 SMALL = [
@@ -144,29 +204,58 @@ def _ws(ws, name, cfg):
     return moe.workspace_view(ws, name, cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.cf)
 
 
+def gpu_quantized_weights(w, names=("w_gate", "w_up", "w_down")):
+    return {n: moe.moe_quantize_weights_fp8(w[n]) for n in names}
+
+
 @pytest.mark.parametrize("cfg", SMALL, ids=[c.name for c in SMALL])
 def test_layer_forward_fp8_matches_oracle(cfg):
     inp, cpu = cuda_inputs(cfg)
-    q = {n: quantize_oracle(cpu[n]) for n in ("w_gate", "w_up", "w_down")}
-    qd = {n: (a.cuda(), b.cuda()) for n, (a, b) in q.items()}
-    y, ws = moe.moe_layer_forward_fp8(inp["x"], inp["w_router"], inp["bias"], *qd["w_gate"],
-                                      *qd["w_up"], *qd["w_down"], cfg.k, cfg.cf)
+    qw = gpu_quantized_weights(inp)
+    y, ws = moe.moe_layer_forward_fp8(inp["x"], inp["w_router"], inp["bias"], *qw["w_gate"],
+                                      *qw["w_up"], *qw["w_down"], cfg.k, cfg.cf)
     torch.cuda.synchronize()
     assert _ws(ws, "status", cfg).item() == 0
     gl = _ws(ws, "logits", cfg).cpu().numpy()
     bias = None if cpu["bias"] is None else cpu["bias"].numpy()
-    assert_logits_close(gl, oracle.router_logits(bits(cpu["x"]), cpu["w_router"].numpy(), bias))
-    ref = oracle_layer_fp8(cpu, cfg.k, cfg.cf, gl, q)
-    np.testing.assert_array_equal(_ws(ws, "topk_idx", cfg).cpu().numpy(), ref["topk_idx"])
-    assert np.max(np.abs(_ws(ws, "topk_w", cfg).cpu().double().numpy() - ref["topk_w"])) \
-        <= WEIGHT_ATOL
-    np.testing.assert_array_equal(_ws(ws, "slot", cfg).cpu().numpy(), ref["slot"])
-    np.testing.assert_array_equal(_ws(ws, "offsets", cfg).cpu().numpy(), ref["offsets"])
-    assert _ws(ws, "n_dropped", cfg).item() == ref["n_dropped"]
-    assert_bf16_close(f64(y), ref["y"], "y")
-    dropped = (ref["slot"] < 0).all(axis=1)
+    x_bits = bits(cpu["x"])
+    assert_logits_close(gl, oracle.router_logits(x_bits, cpu["w_router"].numpy(), bias))
+    o_idx, o_w = oracle.topk(gl, cfg.k)
+    C = oracle.capacity(cfg.T, cfg.E, cfg.k, cfg.cf)
+    counts, offsets, slot, row_src, n_drop = oracle.permute(o_idx, cfg.E, C)
+    np.testing.assert_array_equal(_ws(ws, "topk_idx", cfg).cpu().numpy(), o_idx)
+    assert np.max(np.abs(_ws(ws, "topk_w", cfg).cpu().double().numpy() - o_w)) <= WEIGHT_ATOL
+    np.testing.assert_array_equal(_ws(ws, "slot", cfg).cpu().numpy(), slot)
+    np.testing.assert_array_equal(_ws(ws, "offsets", cfg).cpu().numpy(), offsets)
+    assert _ws(ws, "n_dropped", cfg).item() == n_drop
+    N = int(offsets[-1])
+    # the weights' and x_perm's codes
+    q = {n: quantize_w(cpu[n]) for n in ("w_gate", "w_up", "w_down")}
+    for n in q:
+        np.testing.assert_array_equal(qw[n][0].cpu().numpy().transpose(0, 2, 1), q[n][0])
+    xq, sx = oracle.quantize_rows_fp8(oracle.dispatch(x_bits, row_src))
+    np.testing.assert_array_equal(_ws(ws, "xq", cfg)[:N].cpu().numpy(), xq)
+    np.testing.assert_array_equal(_ws(ws, "sx", cfg)[:N].cpu().numpy(), sx)
+    h = _ws(ws, "h", cfg)[:N]
+    hq = _ws(ws, "hq", cfg)[:N].cpu().numpy()
+    sh = _ws(ws, "sh", cfg)[:N].cpu().numpy()
+    y_perm = _ws(ws, "y_perm", cfg)[:N]
+    (qg, sg), (qu, su), (qd, sd) = q["w_gate"], q["w_up"], q["w_down"]
+    check_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, h, hq, sh, y_perm)
+    # the combine on the oracle's y_perm (from the GPU's h codes)
+    hq_ref, sh_ref = oracle.quantize_rows_fp8(bits(h))
+    b = deq_rows(hq_ref, sh_ref)
+    d64 = oracle.dequant_fp8(qd, sd)
+    o_y = np.zeros((N, cfg.d))
+    for e in range(cfg.E):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            o_y[lo:hi] = oracle.matmul_f64(b[lo:hi], d64[e])
+    y_ref = oracle.combine(o_y, x_bits, o_idx, o_w, slot, offsets)
+    assert_bf16_close(f64(y), y_ref, "y")
+    dropped = (slot < 0).all(axis=1)
     if dropped.any():
-        np.testing.assert_array_equal(bits(y)[dropped], bits(cpu["x"])[dropped])
+        np.testing.assert_array_equal(bits(y)[dropped], x_bits[dropped])
 
 
 DECODE = [configs.DECODE.with_tokens(t) for t in configs.DECODE_T]
@@ -174,14 +263,13 @@ DECODE = [configs.DECODE.with_tokens(t) for t in configs.DECODE_T]
 
 @pytest.mark.parametrize("cfg", DECODE, ids=[c.name for c in DECODE])
 def test_decode_fp8_full_size_sampled(cfg):
-    """Decode-sized layer with e4m3 experts quantized on the GPU: the
-    quantizer bit-exact on the experts the sampled tokens use, routing exact
-    for every token, outputs on sampled tokens from the oracle's own
-    quantization of those experts."""
+    """Decode-sized layer with FP8 experts quantized on the GPU: routing exact
+    for every token; the weight codes of the experts that two sampled tokens
+    use bit-exact; those tokens' outputs from the oracle."""
     torch.cuda.empty_cache()
     w = synth.make_weights(cfg, "cuda")
     x = synth.make_tokens(cfg, "cuda")
-    qw = {n: moe.moe_quantize_weights_fp8(w[n]) for n in ("w_gate", "w_up", "w_down")}
+    qw = gpu_quantized_weights(w)
     y, ws = moe.moe_layer_forward_fp8(x, w["w_router"], w["bias"], *qw["w_gate"], *qw["w_up"],
                                       *qw["w_down"], cfg.k, cfg.cf)
     torch.cuda.synchronize()
@@ -196,18 +284,25 @@ def test_decode_fp8_full_size_sampled(cfg):
     rng = np.random.default_rng(cfg.seed + 1)
     toks = np.sort(rng.choice(cfg.T, size=2, replace=False))
     x_bits = bits(x)
+    h_gpu = _ws(ws, "h", cfg)
     y_ref = np.zeros((len(toks), cfg.d))
     for i, t in enumerate(toks):
+        xq, sx = oracle.quantize_rows_fp8(x_bits[t:t + 1])
+        a = deq_rows(xq, sx)
         for j in range(cfg.k):
             e = int(o_idx[t, j])
             mats = []
             for n in ("w_gate", "w_up", "w_down"):
-                q_ref, s_ref = quantize_oracle(w[n][e:e + 1].cpu())
-                assert torch.equal(qw[n][0][e:e + 1].cpu(), q_ref), (n, e)
-                assert torch.equal(qw[n][1][e:e + 1].cpu(), s_ref), (n, e)
-                mats.append(dequant(q_ref, s_ref)[0])
-            _, o = oracle.swiglu_rows_f64w(x_bits[t:t + 1], *mats)
-            y_ref[i] += o_w[t, j] * o[0]
+                q_ref, s_ref = quantize_w(w[n][e:e + 1].cpu())
+                assert np.array_equal(qw[n][0][e].cpu().numpy().T, q_ref[0]), (n, e)
+                assert np.array_equal(qw[n][1][e].cpu().numpy(), s_ref[0]), (n, e)
+                mats.append(oracle.dequant_fp8(q_ref, s_ref)[0])
+            h_ref = oracle.gate_up_f64(a, mats[0], mats[1])
+            row = int(offsets[e] + slot[t, j])
+            h_row = h_gpu[row:row + 1]
+            assert_bf16_rounding_close(f64(h_row), h_ref, "h (sampled)")
+            hq, sh = oracle.quantize_rows_fp8(bits(h_row))
+            y_ref[i] += o_w[t, j] * oracle.matmul_f64(deq_rows(hq, sh), mats[2])[0]
     assert_bf16_close(f64(y[torch.from_numpy(toks).cuda().long()]), y_ref, "y (sampled)")
     del w, x, y, ws, qw
     torch.cuda.empty_cache()

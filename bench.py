@@ -32,7 +32,7 @@ from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
 METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 8     # router 3, permute 2, gate/up GEMM 1, down GEMM 1, combine 1
-KERNELS_PER_STEP_FP8 = 10   # + the row quantizer on x_perm and on h
+KERNELS_PER_STEP_FP8 = 10   # + the row quantizer on x and on h
 FP8_OVER_BF16 = 2.0      # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
@@ -142,7 +142,7 @@ def max_over_ranks(value, device, dist):
 
 class Layer:
     """Inputs, weights and buffers of one workload, resident on the device,
-    and the step as five C-ABI calls on one stream."""
+    and the step as C-ABI calls on one stream (five; seven with FP8 experts)."""
 
     def __init__(self, cfg, device, token_seed, fp8=False):
         import mixture_experts_layer_36_b200 as moe
@@ -166,8 +166,13 @@ class Layer:
         self.tw = z(T, k, dt=torch.float32)
         self.perm = {"counts": z(E, dt=torch.int32), "offsets": z(E + 1, dt=torch.int32),
                      "slot": z(T, k, dt=torch.int32), "row_src": z(self.rows, dt=torch.int32),
-                     "x_perm": z(self.rows, d, dt=torch.bfloat16),
                      "n_dropped": z(1, dt=torch.int32)}
+        if fp8:
+            # the FP8 layer quantizes each token once and permutes codes + scales
+            self.perm.update(xq=z(self.rows, d, dt=torch.uint8), sx=z(self.rows, dt=torch.float32))
+            self.xq_tok, self.sx_tok = z(T, d, dt=torch.uint8), z(T, dt=torch.float32)
+        else:
+            self.perm["x_perm"] = z(self.rows, d, dt=torch.bfloat16)
         self.pws = z(max(moe.moe_permute_workspace_size(T, E, k), 16), dt=torch.uint8)
         self.rws = z(max(moe.moe_route_workspace_size(T, d, E, k), 16), dt=torch.uint8)
         self.h = z(self.rows, f, dt=torch.bfloat16)
@@ -189,14 +194,15 @@ class Layer:
         p = self.perm
         st = [("route", lambda: m.moe_route(self.x, w["w_router"], w["bias"], c.k, self.logits,
                                             self.idx, self.tw, ws=self.rws,
-                                            dev_status=self.status)),
-              ("permute", lambda: m.moe_permute(self.x, self.idx, c.E, c.cf, out=p, ws=self.pws))]
+                                            dev_status=self.status))]
         if self.fp8:
             q, n_rows = self.q, p["offsets"][c.E:]
-            st += [("quant_x", lambda: m.moe_quantize_rows_fp8(p["x_perm"], n_rows=n_rows,
-                                                               q=self.xq, scale=self.sx)),
+            st += [("quant_x", lambda: m.moe_quantize_rows_fp8(self.x, q=self.xq_tok,
+                                                               scale=self.sx_tok)),
+                   ("permute", lambda: m.moe_permute_fp8(self.xq_tok, self.sx_tok, self.idx, c.E,
+                                                         c.cf, out=p, ws=self.pws)),
                    ("gate_up", lambda: m.moe_expert_gate_up_fp8(
-                       self.xq, self.sx, p["offsets"], *q["w_gate"], *q["w_up"], h=self.h,
+                       p["xq"], p["sx"], p["offsets"], *q["w_gate"], *q["w_up"], h=self.h,
                        dev_status=self.status)),
                    ("quant_h", lambda: m.moe_quantize_rows_fp8(self.h, n_rows=n_rows, q=self.hq,
                                                                scale=self.sh)),
@@ -204,7 +210,9 @@ class Layer:
                                                           *q["w_down"], y_perm=self.y_perm,
                                                           dev_status=self.status))]
         else:
-            st += [("gate_up", lambda: m.moe_expert_gate_up(p["x_perm"], p["offsets"], w["w_gate"],
+            st += [("permute", lambda: m.moe_permute(self.x, self.idx, c.E, c.cf, out=p,
+                                                     ws=self.pws)),
+                   ("gate_up", lambda: m.moe_expert_gate_up(p["x_perm"], p["offsets"], w["w_gate"],
                                                             w["w_up"], h=self.h,
                                                             dev_status=self.status)),
                    ("down", lambda: m.moe_expert_down(self.h, p["offsets"], w["w_down"],
@@ -454,8 +462,18 @@ def main():
         g2_bytes += A * 1.0 * cfg.d * 4 + r["N"] * 4
     ridge = peak_tf * 1e12 / (pk["hbm_gbs"] * 1e9)
     hbm_bound = gemm1_flop / g1_bytes < ridge
-    bytes_perm = cfg.T * cfg.d * 2 + r["N"] * cfg.d * 2
+    bytes_perm = cfg.T * cfg.d * wb + r["N"] * cfg.d * wb
     bytes_comb = r["N"] * cfg.d * 4 + cfg.T * cfg.d * 2
+    quant_rooflines = {}
+    if args.fp8:
+        # the row quantizers: bf16 rows read once (the second pass hits cache),
+        # codes + fp32 scales written
+        for name, rows, width in (("quant_x", cfg.T, cfg.d), ("quant_h", r["N"], cfg.f)):
+            nbytes = rows * width * 3 + rows * 4
+            t = r["stage_ms"][name] / 1e3
+            quant_rooflines[name] = {"bound": "hbm", "unit": "GB/s",
+                                     "achieved": round(nbytes / t / 1e9, 1),
+                                     "frac": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4)}
     out = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -507,6 +525,7 @@ def main():
                         "achieved": round(bytes_comb / (r["stage_ms"]["combine"] / 1e3) / 1e9, 1),
                         "frac": round(bytes_comb / (r["stage_ms"]["combine"] / 1e3) / 1e9
                                       / pk["hbm_gbs"], 4)},
+            **quant_rooflines,
         },
         "device_status": r["status"],
         "clocks": {k_: r["clocks"][k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},

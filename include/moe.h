@@ -112,11 +112,13 @@ typedef enum {
   MOE_WS_SX = 15,        /* f32 [max_rows]    their row scales */
   MOE_WS_HQ = 16,        /* u8  [max_rows, f] e4m3 codes of h */
   MOE_WS_SH = 17,        /* f32 [max_rows]    their row scales */
-  MOE_WS_FP8_NUM_FIELDS = 18
+  MOE_WS_XQ_TOK = 18,    /* u8  [T, d]        e4m3 codes of x (before the permutation) */
+  MOE_WS_SX_TOK = 19,    /* f32 [T]           their row scales */
+  MOE_WS_FP8_NUM_FIELDS = 20
 } moe_ws_field;
 
 /* Byte offset of a field inside the moe_layer_forward workspace (each field
- * 256-byte aligned; fields MOE_WS_XQ .. MOE_WS_SH exist only in a
+ * 256-byte aligned; fields MOE_WS_XQ .. MOE_WS_SX_TOK exist only in a
  * moe_layer_forward_fp8 workspace); -1 on bad args. */
 int64_t moe_workspace_field_offset(int field, int64_t T, int64_t d, int64_t E, int64_t k,
                                    int64_t f, double cf);
@@ -250,6 +252,17 @@ int moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t N, uin
 int moe_quantize_rows_fp8(const void* x, int64_t R, int64_t K, const int32_t* n_rows, uint8_t* q,
                           float* scale, void* stream);
 
+/* moe_permute on e4m3 token rows: the same counts, offsets, slots, row_src
+ * and n_dropped, with the codes xq u8 [T,d] and row scales sx f32 [T] (from
+ * moe_quantize_rows_fp8 on x) moved to xq_perm u8 [max_rows,d] and sx_perm
+ * f32 [max_rows].  Per-row quantization commutes with the row copy, so this
+ * equals quantizing moe_permute's x_perm. */
+int moe_permute_fp8(const uint8_t* xq, const float* sx, const int32_t* topk_idx, int64_t T,
+                    int64_t d, int64_t E, int64_t k, double cf, int32_t* counts,
+                    int32_t* offsets, int32_t* slot, int32_t* row_src, uint8_t* xq_perm,
+                    float* sx_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
+                    void* stream);
+
 /* GEMM 1 + SwiGLU on e4m3 operands: h[r,:] = silu(g) * u with
  * g[r,n] = sx[r] * s_gate[e,n] * sum_k xq[r,k] wq_gate[e,n,k] (u likewise) for
  * rows r of bucket e.  xq u8 [max_rows,d], sx f32 [max_rows], wq_* u8 [E,f,d]
@@ -268,12 +281,13 @@ int moe_expert_down_fp8(const uint8_t* hq, const float* sh, const int32_t* offse
                         const float* s_down, float* y_perm, int32_t* dev_status, void* stream);
 
 /* Workspace of moe_layer_forward_fp8: the moe_layer_forward fields followed by
- * MOE_WS_XQ .. MOE_WS_SH (0 on invalid shapes). */
+ * MOE_WS_XQ .. MOE_WS_SX_TOK (0 on invalid shapes). */
 size_t moe_workspace_size_fp8(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, double cf);
 
-/* The layer with FP8 experts: moe_route, moe_permute, moe_quantize_rows_fp8
- * (x_perm), moe_expert_gate_up_fp8, moe_quantize_rows_fp8 (h),
- * moe_expert_down_fp8, moe_combine on `stream`.  Weights and scales from
+/* The layer with FP8 experts: moe_route, moe_quantize_rows_fp8 (x),
+ * moe_permute_fp8, moe_expert_gate_up_fp8, moe_quantize_rows_fp8 (h),
+ * moe_expert_down_fp8, moe_combine on `stream` (the bf16 x_perm field of the
+ * workspace is not used).  Weights and scales from
  * moe_quantize_weights_fp8; other arguments as moe_layer_forward. */
 int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bias,
                           const uint8_t* wq_gate, const float* s_gate, const uint8_t* wq_up,

@@ -23,14 +23,15 @@ DEV_ERR_BAD_OFFSETS = 2
 
 # workspace fields of moe_layer_forward (enum moe_ws_field)
 WS_FIELDS = ["status", "logits", "topk_idx", "topk_w", "slot", "counts", "offsets", "n_dropped",
-             "row_src", "permute", "x_perm", "h", "y_perm", "route", "xq", "sx", "hq", "sh"]
+             "row_src", "permute", "x_perm", "h", "y_perm", "route", "xq", "sx", "hq", "sh",
+             "xq_tok", "sx_tok"]
 
 EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "moe_capacity",
             "moe_max_rows",
             "moe_route_workspace_size", "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
             "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
             "moe_combine", "moe_layer_forward", "moe_quantize_weights_fp8",
-            "moe_quantize_rows_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8",
+            "moe_quantize_rows_fp8", "moe_permute_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8",
             "moe_workspace_size_fp8", "moe_layer_forward_fp8"]
 
 
@@ -67,6 +68,8 @@ def _load():
                                              sz, p]),
         "moe_quantize_weights_fp8": (ctypes.c_int, [p, i64, i64, i64, p, p, p]),
         "moe_quantize_rows_fp8": (ctypes.c_int, [p, i64, i64, p, p, p, p]),
+        "moe_permute_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
+                                           p, sz, p]),
         "moe_expert_gate_up_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p, p,
                                                   p]),
         "moe_expert_down_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p]),
@@ -351,6 +354,34 @@ def moe_quantize_rows_fp8(x, n_rows=None, q=None, scale=None, stream=None):
     return q, scale
 
 
+def moe_permute_fp8(xq, sx, topk_idx, E, cf, out=None, ws=None, stream=None):
+    """moe_permute on e4m3 token rows (codes + row scales).  Returns a dict
+    like moe_permute's, with "xq" / "sx" in place of "x_perm"."""
+    T, d = xq.shape
+    k = topk_idx.shape[1]
+    _want(xq, "xq", torch.uint8)
+    _want(sx, "sx", torch.float32, (T,))
+    _want(topk_idx, "topk_idx", torch.int32, (T, k))
+    rows = moe_max_rows(T, E, k, cf)
+    dev = xq.device
+    if out is None:
+        out = {"counts": torch.empty(E, dtype=torch.int32, device=dev),
+               "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+               "slot": torch.empty(T, k, dtype=torch.int32, device=dev),
+               "row_src": torch.empty(rows, dtype=torch.int32, device=dev),
+               "xq": torch.empty(rows, d, dtype=torch.uint8, device=dev),
+               "sx": torch.empty(rows, dtype=torch.float32, device=dev),
+               "n_dropped": torch.empty(1, dtype=torch.int32, device=dev)}
+    if ws is None:
+        ws = torch.empty(max(moe_permute_workspace_size(T, E, k), 16), dtype=torch.uint8,
+                         device=dev)
+    _check("moe_permute_fp8", _lib.moe_permute_fp8(
+        _ptr(xq), _ptr(sx), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]),
+        _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["xq"]),
+        _ptr(out["sx"]), _ptr(out["n_dropped"]), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
 def moe_expert_gate_up_fp8(xq, sx, offsets, wq_gate, s_gate, wq_up, s_up, h=None,
                            dev_status=None, stream=None):
     rows, d = xq.shape
@@ -432,6 +463,7 @@ def workspace_view(ws, field, T, d, E, k, f, cf):
         "h": (torch.bfloat16, (rows, f)), "y_perm": (torch.float32, (rows, d)),
         "xq": (torch.uint8, (rows, d)), "sx": (torch.float32, (rows,)),
         "hq": (torch.uint8, (rows, f)), "sh": (torch.float32, (rows,)),
+        "xq_tok": (torch.uint8, (T, d)), "sx_tok": (torch.float32, (T,)),
     }[field]
     dtype, shape = spec
     off = moe_workspace_field_offset(field, T, d, E, k, f, cf)

@@ -26,6 +26,11 @@ cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t s);
+cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_scale,
+                                const int32_t* topk_idx, int T, int E, int k, int64_t C,
+                                int32_t* counts, int32_t* offsets, int32_t* slot,
+                                int32_t* row_src, uint8_t* x_perm, float* perm_scale,
+                                int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s);
 cudaError_t launch_quantize_weights(const __nv_bfloat16* w, int E, int K, int N, uint8_t* q,
                                     float* scale, cudaStream_t s);
 cudaError_t launch_quantize_rows(const __nv_bfloat16* x, int R, int K, const int32_t* n_rows,
@@ -122,6 +127,8 @@ bool fp8_field_sizes(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, doub
   out[MOE_WS_SX - MOE_WS_NUM_FIELDS] = size_t(rows) * sizeof(float);
   out[MOE_WS_HQ - MOE_WS_NUM_FIELDS] = size_t(rows * f);
   out[MOE_WS_SH - MOE_WS_NUM_FIELDS] = size_t(rows) * sizeof(float);
+  out[MOE_WS_XQ_TOK - MOE_WS_NUM_FIELDS] = size_t(T * d);
+  out[MOE_WS_SX_TOK - MOE_WS_NUM_FIELDS] = size_t(T) * sizeof(float);
   return true;
 }
 
@@ -342,6 +349,28 @@ int moe_quantize_rows_fp8(const void* x, int64_t R, int64_t K, const int32_t* n_
                                                (int)K, n_rows, q, scale, as_stream(stream)));
 }
 
+int moe_permute_fp8(const uint8_t* xq, const float* sx, const int32_t* topk_idx, int64_t T,
+                    int64_t d, int64_t E, int64_t k, double cf, int32_t* counts,
+                    int32_t* offsets, int32_t* slot, int32_t* row_src, uint8_t* xq_perm,
+                    float* sx_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
+                    void* stream) {
+  int st = check_routing_shape(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_width(d)) != MOE_OK) return st;
+  const int64_t C = moe_capacity(T, E, k, cf);
+  if (C < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!xq || !sx || !topk_idx || !counts || !offsets || !slot || !row_src || !xq_perm ||
+      !sx_perm || !n_dropped || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(xq_perm) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_permute_workspace_size(T, E, k)) return MOE_ERR_WORKSPACE;
+  return cuda_status(moe::launch_permute_rows(xq, (int)d, sx, topk_idx, (int)T, (int)E, (int)k, C,
+                                              counts, offsets, slot, row_src, xq_perm, sx_perm,
+                                              n_dropped, static_cast<int32_t*>(ws),
+                                              as_stream(stream)));
+}
+
 int moe_expert_gate_up_fp8(const uint8_t* xq, const float* sx, const int32_t* offsets, int64_t E,
                            int64_t d, int64_t f, int64_t max_rows, const uint8_t* wq_gate,
                            const float* s_gate, const uint8_t* wq_up, const float* s_up, void* h,
@@ -406,7 +435,6 @@ int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bia
   int32_t* offsets = reinterpret_cast<int32_t*>(field(MOE_WS_OFFSETS));
   int32_t* n_dropped = reinterpret_cast<int32_t*>(field(MOE_WS_N_DROPPED));
   int32_t* row_src = reinterpret_cast<int32_t*>(field(MOE_WS_ROW_SRC));
-  void* x_perm = field(MOE_WS_X_PERM);
   void* h = field(MOE_WS_H);
   float* y_perm = reinterpret_cast<float*>(field(MOE_WS_Y_PERM));
   uint8_t* xq = reinterpret_cast<uint8_t*>(field(MOE_WS_XQ));
@@ -420,11 +448,13 @@ int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bia
   if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, field(MOE_WS_ROUTE),
                       moe_route_workspace_size(T, d, E, k), status, stream)) != MOE_OK)
     return st;
-  if ((st = moe_permute(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src, x_perm,
-                        n_dropped, field(MOE_WS_PERMUTE), moe_permute_workspace_size(T, E, k),
-                        stream)) != MOE_OK)
-    return st;
-  if ((st = moe_quantize_rows_fp8(x_perm, max_rows, d, n_rows, xq, sx, stream)) != MOE_OK)
+  // each token is quantized once; the permutation moves its codes and scale
+  uint8_t* xq_tok = reinterpret_cast<uint8_t*>(field(MOE_WS_XQ_TOK));
+  float* sx_tok = reinterpret_cast<float*>(field(MOE_WS_SX_TOK));
+  if ((st = moe_quantize_rows_fp8(x, T, d, nullptr, xq_tok, sx_tok, stream)) != MOE_OK) return st;
+  if ((st = moe_permute_fp8(xq_tok, sx_tok, topk_idx, T, d, E, k, cf, counts, offsets, slot,
+                            row_src, xq, sx, n_dropped, field(MOE_WS_PERMUTE),
+                            moe_permute_workspace_size(T, E, k), stream)) != MOE_OK)
     return st;
   if ((st = moe_expert_gate_up_fp8(xq, sx, offsets, E, d, f, max_rows, wq_gate, s_gate, wq_up,
                                    s_up, h, status, stream)) != MOE_OK)

@@ -553,22 +553,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // [64r, 64r+64) of the tile), so every thread still holds g and u of the same
 // h-column.  This halves the rows computed in vain at each expert's tail.
 // Epilogue pieces of the pair kernel: 32 accumulator columns of 32 rows.
+// SCALED (e4m3 operands): the accumulators are multiplied by the row's scale
+// sr and the 32 columns' scales first.
+template <bool SCALED>
 __device__ __forceinline__ void swiglu_chunk_store(uint32_t tg, uint32_t tu,
                                                    __nv_bfloat16* out_row0, size_t ld, int nvalid,
-                                                   int lane) {
+                                                   int lane, const float* sg, const float* su,
+                                                   float sr) {
   uint32_t g[32], u[32], pk[16];
   tmem_ld_32x32b_x32(tg, g);
   tmem_ld_32x32b_x32(tu, u);
   tmem_ld_wait();
+  if (SCALED) {
+    apply_scales(g, sg, sr);
+    apply_scales(u, su, sr);
+  }
   swiglu_pack(g, u, pk);
   store_chunk_bf16(pk, out_row0, ld, nvalid, lane);
 }
 
+template <bool SCALED>
 __device__ __forceinline__ void f32_chunk_store(uint32_t t, uint32_t* stage, float* out_row0,
-                                                size_t ld, int nvalid, int lane) {
+                                                size_t ld, int nvalid, int lane,
+                                                const float* sc, float sr) {
   uint32_t v[32];
   tmem_ld_32x32b_x32(t, v);
   tmem_ld_wait();
+  if (SCALED) apply_scales(v, sc, sr);
   store_chunk_f32(v, stage, out_row0, ld, nvalid, lane);
 }
 
@@ -604,18 +615,29 @@ __device__ __forceinline__ void decode_pair_tile(const PairShared& sh, int tile,
   m = local - n * mt;
 }
 
-template <bool SWIGLU>
+// E4M3: e4m3 operands, both K-major (weights [E, N, K]), 128-deep k-blocks,
+// kind::f8f6f4; tmB0h / tmB1h are 64-row weight boxes for the half tiles'
+// 64 + 64 column split; the epilogue applies the row and column scales.
+template <bool SWIGLU, bool E4M3>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
                              const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1,
+                             const __grid_constant__ CUtensorMap tmB0h,
+                             const __grid_constant__ CUtensorMap tmB1h,
+                             const float* __restrict__ row_scale,
+                             const float* __restrict__ col_scale0,
+                             const float* __restrict__ col_scale1,
                              const int32_t* __restrict__ offsets, int E, int K, int n_out,
                              int max_rows, void* __restrict__ out_raw, int32_t* status) {
   constexpr int kOutCols = SWIGLU ? 128 : 256;        // output columns per pair tile
   constexpr int kPairM = 2 * kBM;
-  constexpr uint32_t kIdesc = idesc_bf16_f32(kPairM, 256, /*b_mn_major=*/true);
-  constexpr uint32_t kIdescHalf = idesc_bf16_f32(kBM, 256, /*b_mn_major=*/true);
+  constexpr int kKb = E4M3 ? 128 : kBK;               // K values per k-block (128 bytes)
+  constexpr uint32_t kIdesc = E4M3 ? idesc_e4m3_f32(kPairM, 256)
+                                   : idesc_bf16_f32(kPairM, 256, /*b_mn_major=*/true);
+  constexpr uint32_t kIdescHalf = E4M3 ? idesc_e4m3_f32(kBM, 256)
+                                       : idesc_bf16_f32(kBM, 256, /*b_mn_major=*/true);
   constexpr int kTmemCols = 512;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ PairShared sh;
@@ -627,7 +649,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int n_tiles = n_out / kOutCols;
-  const int nkb = K / kBK;
+  const int nkb = K / kKb;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
@@ -652,6 +674,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     prefetch_tensormap(&tmA64);
     prefetch_tensormap(&tmB0);
     if (SWIGLU) prefetch_tensormap(&tmB1);
+    if (E4M3) prefetch_tensormap(&tmB0h);
+    if (E4M3 && SWIGLU) prefetch_tensormap(&tmB1h);
   }
   if (warp == 2) {
     int carry = 0;
@@ -719,10 +743,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_arrive_expect_tx(&sh.full_bar[s],
                                   half ? 2 * (kPairStageBytes - kBM * kBK) : 2 * kPairStageBytes);
           if (half)
-            tma_load_2d_pair(sa, &tmA64, full_lead, kb * kBK, row0);
+            tma_load_2d_pair(sa, &tmA64, full_lead, kb * kKb, row0);
           else
-            tma_load_2d_pair(sa, &tmA, full_lead, kb * kBK, row0);
-          if (SWIGLU && half) {
+            tma_load_2d_pair(sa, &tmA, full_lead, kb * kKb, row0);
+          if (E4M3) {
+            // K-major weights: 128 rows (output columns) of 128 K bytes per CTA
+            const int k0 = kb * kKb;
+            if (SWIGLU && half) {
+              tma_load_3d_pair(sb, &tmB0h, full_lead, k0, col0 + (int)rank * 64, e);
+              tma_load_3d_pair(sb + 64 * 128, &tmB1h, full_lead, k0, col0 + (int)rank * 64, e);
+            } else if (SWIGLU) {
+              tma_load_3d_pair(sb, leader ? &tmB0 : &tmB1, full_lead, k0, col0, e);
+            } else {
+              tma_load_3d_pair(sb, &tmB0, full_lead, k0, col0 + (int)rank * 128, e);
+            }
+          } else if (SWIGLU && half) {
             tma_load_3d_pair(sb, &tmB0, full_lead, col0 + (int)rank * 64, kb * kBK, e);
             tma_load_3d_pair(sb + kChunkBytes, &tmB1, full_lead, col0 + (int)rank * 64, kb * kBK,
                              e);
@@ -771,10 +806,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_addr = smem_u32(smem + s * kPairStageBytes);
           const uint32_t b_addr = a_addr + kBM * kBK * 2;
 #pragma unroll
-          for (int ks = 0; ks < kBK / kUmmaK; ++ks) {
+          for (int ks = 0; ks < 4; ++ks) {
             const uint64_t adesc = smem_desc_sw128(a_addr + ks * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, kChunkBytes, 1024);
-            umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
+            if (E4M3) {
+              const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 32, 16, 1024);
+              umma_e4m3_pair(d_tmem, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
+            } else {
+              const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, kChunkBytes, 1024);
+              umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
+            }
           }
           umma_commit_pair_mc(&sh.empty_bar[s], 0x3);
         }
@@ -803,22 +843,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
       uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kPairStagingOff) + q * kStageWords;
+      // E4M3: column scales from (e, column), the row's scale per thread
+      const float* cs0 = E4M3 ? col_scale0 + (size_t)e * n_out : nullptr;
+      const float* cs1 = (E4M3 && SWIGLU) ? col_scale1 + (size_t)e * n_out : nullptr;
       if (!half) {
         const int first = m * kPairM + (int)rank * kBM + q * 32;   // first row of this warp
         const int nvalid = clamp_rows(sh.row_cnt[e] - first);
         const size_t row0 = (size_t)(sh.row_off[e] + first);
+        const float sr = (E4M3 && lane < nvalid) ? row_scale[row0 + lane] : 0.f;
         if (SWIGLU) {
-          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out +
-                             (size_t)n * kOutCols;
+          const int c0 = n * kOutCols;
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out + c0;
 #pragma unroll 1
           for (int c = 0; c < 4; ++c)
-            swiglu_chunk_store(tbase + c * 32, tbase + 128 + c * 32, o + c * 32, n_out, nvalid,
-                               lane);
+            swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 128 + c * 32, o + c * 32, n_out,
+                                     nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
         } else {
-          float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * kOutCols;
+          const int c0 = n * kOutCols;
+          float* o = static_cast<float*>(out_raw) + row0 * n_out + c0;
 #pragma unroll 1
           for (int c = 0; c < 8; ++c)
-            f32_chunk_store(tbase + c * 32, stage, o + c * 32, n_out, nvalid, lane);
+            f32_chunk_store<E4M3>(tbase + c * 32, stage, o + c * 32, n_out, nvalid, lane,
+                                  cs0 + c0 + c * 32, sr);
         }
       } else {
         // lanes 0-63: accumulator columns [0,128); lanes 64-127: [128,256)
@@ -826,21 +872,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int first = m * kPairM + (int)rank * (kBM / 2) + (q & 1) * 32;
         const int nvalid = clamp_rows(sh.row_cnt[e] - first);
         const size_t row0 = (size_t)(sh.row_off[e] + first);
+        const float sr = (E4M3 && lane < nvalid) ? row_scale[row0 + lane] : 0.f;
         if (SWIGLU) {
           // this CTA's h-columns [64*rank ... ) of the tile: gate in TMEM
           // columns [0,64), up in [64,128); lanes 64-127 hold the next 64
           // columns of the tile (staged by the other half of B)
-          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out +
-                             (size_t)n * kOutCols + hh * 64;
+          const int c0 = n * kOutCols + hh * 64;
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out + c0;
 #pragma unroll 1
           for (int c = 0; c < 2; ++c)
-            swiglu_chunk_store(tbase + c * 32, tbase + 64 + c * 32, o + c * 32, n_out, nvalid,
-                               lane);
+            swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 64 + c * 32, o + c * 32, n_out,
+                                     nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
         } else {
-          float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * kOutCols + hh * 128;
+          const int c0 = n * kOutCols + hh * 128;
+          float* o = static_cast<float*>(out_raw) + row0 * n_out + c0;
 #pragma unroll 1
           for (int c = 0; c < 4; ++c)
-            f32_chunk_store(tbase + c * 32, stage, o + c * 32, n_out, nvalid, lane);
+            f32_chunk_store<E4M3>(tbase + c * 32, stage, o + c * 32, n_out, nvalid, lane,
+                                  cs0 + c0 + c * 32, sr);
         }
       }
       tc_fence_before();
@@ -887,16 +936,20 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
   return cudaGetLastError();
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool E4M3 = false>
 static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtensorMap& a64,
                                     const CUtensorMap& b0, const CUtensorMap& b1,
                                     const int32_t* offsets, int E, int K, int n_out, int max_rows,
-                                    void* out, int32_t* status, cudaStream_t s) {
+                                    void* out, int32_t* status, cudaStream_t s,
+                                    const CUtensorMap* b0h = nullptr,
+                                    const CUtensorMap* b1h = nullptr,
+                                    const float* row_scale = nullptr,
+                                    const float* cs0 = nullptr, const float* cs1 = nullptr) {
   constexpr int kSmem = kPairStagingOff + 4 * kStageWords * 4 + 1024;
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  auto kern = grouped_gemm_pair_kernel<SWIGLU>;
+  auto kern = grouped_gemm_pair_kernel<SWIGLU, E4M3>;
   if (!di->attr_set[slot]) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (err != cudaSuccess) return err;
@@ -920,8 +973,8 @@ static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtens
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, a64, b0, b1, offsets, E, K, n_out, max_rows, out,
-                            status);
+  return cudaLaunchKernelEx(&cfg, kern, a, a64, b0, b1, b0h ? *b0h : b0, b1h ? *b1h : b1,
+                            row_scale, cs0, cs1, offsets, E, K, n_out, max_rows, out, status);
 }
 
 // Pair tiles (256 rows) pay off when buckets are large; the buffer's rows
@@ -1000,6 +1053,14 @@ cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_
                   map_rows_e4m3(&ta64, xq, d, max_rows, kBM / 2) &&
                   map_weights_e4m3(&tg, wq_gate, E, f, d) && map_weights_e4m3(&tu, wq_up, E, f, d));
   if (*map_failed) return cudaSuccess;
+  if (use_pair_tiles(E, max_rows)) {
+    CUtensorMap tgh, tuh;
+    *map_failed = !(map_weights_e4m3(&tgh, wq_gate, E, f, d, 64) &&
+                    map_weights_e4m3(&tuh, wq_up, E, f, d, 64));
+    if (*map_failed) return cudaSuccess;
+    return launch_gemm_pair<true, true>(9, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h,
+                                        status, s, &tgh, &tuh, sx, s_gate, s_up);
+  }
   return launch_gemm_e4m3<256, true>(11, ta, ta64, tg, tu, sx, s_gate, s_up, offsets, E, d, f,
                                      max_rows, h, status, s);
 }
@@ -1013,6 +1074,9 @@ cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int3
                   map_rows_e4m3(&ta64, hq, f, max_rows, kBM / 2) &&
                   map_weights_e4m3(&td, wq_down, E, d, f));
   if (*map_failed) return cudaSuccess;
+  if (d % 256 == 0 && use_pair_tiles(E, max_rows))
+    return launch_gemm_pair<false, true>(10, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,
+                                         status, s, &td, &td, sh_rows, s_down, nullptr);
   if (d % 256 == 0)
     return launch_gemm_e4m3<256, false>(12, ta, ta64, td, td, sh_rows, s_down, nullptr, offsets,
                                         E, f, d, max_rows, y_perm, status, s);

@@ -71,14 +71,14 @@ inline bool map_rows_e4m3(CUtensorMap* m, const void* base, uint64_t inner, uint
 }
 
 // 3-D e4m3 weights stored K-major, codes [E, N, K] (K contiguous), box
-// (128 K, 128 N, 1), 128-B swizzle: a 128 x 128 tile lands as 128 rows of 128 B.
+// (128 K, box_rows N, 1), 128-B swizzle: a tile lands as box_rows rows of 128 B.
 inline bool map_weights_e4m3(CUtensorMap* m, const void* base, uint64_t E, uint64_t N,
-                             uint64_t K) {
+                             uint64_t K, uint32_t box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {K, N, E};
   cuuint64_t strides[2] = {K, N * K};
-  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t box[3] = {128, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -87,7 +87,7 @@ inline bool map_weights_e4m3(CUtensorMap* m, const void* base, uint64_t E, uint6
 }
 
 // attr_set slots: 0-2 grouped GEMM (1 CTA), 3-6 router GEMM, 7-8 grouped GEMM (CTA pair),
-// 11-13 grouped GEMM on e4m3 operands
+// 9-10 CTA-pair GEMM on e4m3 operands, 11-13 grouped GEMM on e4m3 operands
 struct DeviceInfo {
   int sms = 0;
   bool attr_set[16] = {};

@@ -18,6 +18,8 @@
 //               slot = chunk base + rank, and kept pairs copy their token row
 //               into x_perm[offsets[e] + slot] with 16-byte vector loads and
 //               stores.
+// Rows are moved as bytes: bf16 rows, or e4m3 rows with their fp32 scale
+// (the FP8 layer quantizes each token once, before the permutation).
 #include "common.cuh"
 
 namespace moe {
@@ -89,13 +91,15 @@ __global__ void __launch_bounds__(kRankThreads)
 //    ranks into slots, drops pairs at slot >= C, and copies the token row to
 //    its kept rows with 16-byte vectors.
 __global__ void __launch_bounds__(kScatThreads)
-    permute_scatter_kernel(const __nv_bfloat16* __restrict__ x,
+    permute_scatter_kernel(const uint8_t* __restrict__ x, int row_bytes,
+                           const float* __restrict__ x_scale,
                            const int32_t* __restrict__ topk_idx, int32_t* __restrict__ slot,
-                           const int32_t* __restrict__ chunk_hist, int nchunks, int T, int d,
+                           const int32_t* __restrict__ chunk_hist, int nchunks, int T,
                            int E, int k, int64_t C, int tokens_per_cta,
                            int32_t* __restrict__ counts,
                            int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped,
-                           int32_t* __restrict__ row_src, __nv_bfloat16* __restrict__ x_perm) {
+                           int32_t* __restrict__ row_src, uint8_t* __restrict__ x_perm,
+                           float* __restrict__ perm_scale) {
   __shared__ int32_t s_off[256];
   __shared__ int32_t s_base[256];
   __shared__ int32_t warp_sum[8];
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(kScatThreads)
   __syncthreads();
 
   // ---- one warp per token
-  const int nvec = d / 8;
+  const int nvec = row_bytes / 16;
   for (int tt = warp; tt < tokens_per_cta; tt += kScatThreads / 32) {
     const int t = t0 + tt;
     if (t >= T) break;
@@ -164,13 +168,14 @@ __global__ void __launch_bounds__(kScatThreads)
       if (keep) {
         my_row = s_off[e] + sl;
         row_src[my_row] = t;
+        if (x_scale) perm_scale[my_row] = x_scale[t];
       }
     }
     int rows[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
 
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
     for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
       uint4 val[4];
 #pragma unroll
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(kScatThreads)
       for (int j = 0; j < 8; ++j) {
         if (j >= k) break;
         if (rows[j] < 0) continue;
-        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)rows[j] * d);
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)rows[j] * row_bytes);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int v = v0 + u * 32;
@@ -198,17 +203,30 @@ size_t permute_scratch_bytes(int64_t T, int64_t E) {
   return (size_t)(nchunks * E * (int64_t)sizeof(int32_t));
 }
 
-cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d, int E,
-                           int k, int64_t C, int32_t* counts, int32_t* offsets, int32_t* slot,
-                           int32_t* row_src, __nv_bfloat16* x_perm, int32_t* n_dropped,
-                           int32_t* chunk_hist, cudaStream_t s) {
+// Rows of row_bytes bytes (a multiple of 16); x_scale / perm_scale (one fp32
+// per row, moved with it) may be null.
+cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_scale,
+                                const int32_t* topk_idx, int T, int E, int k, int64_t C,
+                                int32_t* counts, int32_t* offsets, int32_t* slot,
+                                int32_t* row_src, uint8_t* x_perm, float* perm_scale,
+                                int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s) {
   const int nchunks = (T + kChunk - 1) / kChunk;
   permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist);
   const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
   permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
-      x, topk_idx, slot, chunk_hist, nchunks, T, d, E, k, C, tpc, counts, offsets, n_dropped,
-      row_src, x_perm);
+      x, row_bytes, x_scale, topk_idx, slot, chunk_hist, nchunks, T, E, k, C, tpc, counts,
+      offsets, n_dropped, row_src, x_perm, perm_scale);
   return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d, int E,
+                           int k, int64_t C, int32_t* counts, int32_t* offsets, int32_t* slot,
+                           int32_t* row_src, __nv_bfloat16* x_perm, int32_t* n_dropped,
+                           int32_t* chunk_hist, cudaStream_t s) {
+  return launch_permute_rows(reinterpret_cast<const uint8_t*>(x), d * 2, nullptr, topk_idx, T, E,
+                             k, C, counts, offsets, slot, row_src,
+                             reinterpret_cast<uint8_t*>(x_perm), nullptr, n_dropped, chunk_hist,
+                             s);
 }
 
 }  // namespace moe

@@ -91,8 +91,8 @@ cudaError_t launch_quantize_weights(const __nv_bfloat16* w, int E, int K, int N,
 }
 
 // ---------------------------------------------------------------- activation rows
-// One warp per row: the row's max magnitude (16-byte loads), then its codes
-// (the row is read again, now from cache).  Rows at or beyond *n_rows (a
+// Long rows (K > 16384): one warp per row, the row's max magnitude (16-byte
+// loads), then its codes (the row is read again, now from cache).  Rows at or beyond *n_rows (a
 // device count, e.g. offsets[E] of the permutation) are skipped.
 constexpr int kRowWarps = 8;
 __global__ void __launch_bounds__(32 * kRowWarps)
@@ -132,11 +132,123 @@ __global__ void __launch_bounds__(32 * kRowWarps)
   }
 }
 
+// Short rows (K <= 2048): one warp per row holds the whole row in registers
+// (at most 8 16-byte vectors per lane), so each value is read once.
+constexpr int kShortVecs = 8;
+__global__ void __launch_bounds__(32 * kRowWarps)
+    quantize_rows_short_kernel(const __nv_bfloat16* __restrict__ x, int R, int K,
+                               const int32_t* __restrict__ n_rows, uint8_t* __restrict__ q,
+                               float* __restrict__ scale) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int r = blockIdx.x * kRowWarps + warp;
+  int limit = R;
+  if (n_rows) limit = min(limit, *n_rows);
+  if (r >= limit) return;
+  const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)r * K);
+  const int nvec = K / 8;
+  uint4 v[kShortVecs];
+#pragma unroll
+  for (int j = 0; j < kShortVecs; ++j) {
+    const int i = lane + 32 * j;
+    v[j] = i < nvec ? __ldg(row + i) : make_uint4(0, 0, 0, 0);
+  }
+  float mx = 0.f;
+#pragma unroll
+  for (int j = 0; j < kShortVecs; ++j) {
+    const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mx = fmaxf(mx, fabsf(__uint_as_float(w[i] << 16)));
+      mx = fmaxf(mx, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  const float s = scale_of(mx);
+  if (lane == 0) scale[r] = s;
+  uint2* out = reinterpret_cast<uint2*>(q + (size_t)r * K);
+#pragma unroll
+  for (int j = 0; j < kShortVecs; ++j) {
+    const int i = lane + 32 * j;
+    if (i < nvec) {
+      const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      uint32_t p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        p[e] = e4m3_pair(__uint_as_float(w[e] << 16) / s, __uint_as_float(w[e] & 0xFFFF0000u) / s);
+      out[i] = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+    }
+  }
+}
+
+// Wide rows (2048 < K <= 16384): one CTA of THREADS threads per row holds the whole row
+// in registers (at most kWideVecs 16-byte vectors per thread), so each value
+// is read from memory once; the max magnitude is reduced across the CTA.
+constexpr int kWideVecs = 8;             // K <= THREADS * 8 * 8
+template <int kWideThreads>
+__global__ void __launch_bounds__(kWideThreads)
+    quantize_rows_wide_kernel(const __nv_bfloat16* __restrict__ x, int R, int K,
+                              const int32_t* __restrict__ n_rows, uint8_t* __restrict__ q,
+                              float* __restrict__ scale) {
+  __shared__ float warp_max[kWideThreads / 32];
+  const int r = blockIdx.x;
+  int limit = R;
+  if (n_rows) limit = min(limit, *n_rows);
+  if (r >= limit) return;
+  const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)r * K);
+  const int nvec = K / 8;
+  uint4 v[kWideVecs];
+  float mx = 0.f;
+#pragma unroll
+  for (int j = 0; j < kWideVecs; ++j) {
+    const int i = threadIdx.x + j * kWideThreads;
+    v[j] = i < nvec ? __ldg(row + i) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int j = 0; j < kWideVecs; ++j) {
+    const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mx = fmaxf(mx, fabsf(__uint_as_float(w[i] << 16)));
+      mx = fmaxf(mx, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (threadIdx.x % 32 == 0) warp_max[threadIdx.x / 32] = mx;
+  __syncthreads();
+  mx = warp_max[0];
+#pragma unroll
+  for (int w = 1; w < kWideThreads / 32; ++w) mx = fmaxf(mx, warp_max[w]);
+  const float s = scale_of(mx);
+  if (threadIdx.x == 0) scale[r] = s;
+  uint2* out = reinterpret_cast<uint2*>(q + (size_t)r * K);
+#pragma unroll
+  for (int j = 0; j < kWideVecs; ++j) {
+    const int i = threadIdx.x + j * kWideThreads;
+    if (i < nvec) {
+      const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      uint32_t p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        p[e] = e4m3_pair(__uint_as_float(w[e] << 16) / s, __uint_as_float(w[e] & 0xFFFF0000u) / s);
+      out[i] = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+    }
+  }
+}
+
 cudaError_t launch_quantize_rows(const __nv_bfloat16* x, int R, int K, const int32_t* n_rows,
                                  uint8_t* q, float* scale, cudaStream_t s) {
   if (R == 0) return cudaSuccess;
-  quantize_rows_kernel<<<(R + kRowWarps - 1) / kRowWarps, 32 * kRowWarps, 0, s>>>(x, R, K, n_rows,
-                                                                                 q, scale);
+  const int rows_ctas = (R + kRowWarps - 1) / kRowWarps;
+  if (K <= 32 * kShortVecs * 8)
+    quantize_rows_short_kernel<<<rows_ctas, 32 * kRowWarps, 0, s>>>(x, R, K, n_rows, q, scale);
+  else if (K <= 128 * kWideVecs * 8)
+    quantize_rows_wide_kernel<128><<<R, 128, 0, s>>>(x, R, K, n_rows, q, scale);
+  else if (K <= 256 * kWideVecs * 8)
+    quantize_rows_wide_kernel<256><<<R, 256, 0, s>>>(x, R, K, n_rows, q, scale);
+  else
+    quantize_rows_kernel<<<rows_ctas, 32 * kRowWarps, 0, s>>>(x, R, K, n_rows, q, scale);
   return cudaGetLastError();
 }
 

@@ -72,12 +72,12 @@ def test_workspace_layout(cfg):
     assert moe.moe_route_workspace_size(T, d, E, k) >= 2 * d * ((E + 63) // 64 * 64) * 2
     # the FP8 layer's extra fields follow the standard ones
     total8 = moe.moe_workspace_size_fp8(T, d, E, k, f, cf)
-    offs8 = [moe.moe_workspace_field_offset(i, T, d, E, k, f, cf) for i in range(14, 18)]
+    offs8 = [moe.moe_workspace_field_offset(i, T, d, E, k, f, cf) for i in range(14, 20)]
     assert offs8[0] == total and all(o % 256 == 0 for o in offs8) and offs8 == sorted(offs8)
     ends8 = offs8[1:] + [total8]
-    for i, n in enumerate((rows * d, rows * 4, rows * f, rows * 4)):
+    for i, n in enumerate((rows * d, rows * 4, rows * f, rows * 4, T * d, T * 4)):
         assert ends8[i] - offs8[i] >= n, binding.WS_FIELDS[14 + i]
-    assert moe.moe_workspace_field_offset(18, T, d, E, k, f, cf) == -1
+    assert moe.moe_workspace_field_offset(20, T, d, E, k, f, cf) == -1
     assert moe.moe_workspace_field_offset(-1, T, d, E, k, f, cf) == -1
 
 

@@ -64,7 +64,9 @@ def test_weight_quantizer_bit_exact(E, K, N):
     np.testing.assert_array_equal(q.cpu().numpy().transpose(0, 2, 1), q_ref)
 
 
-@pytest.mark.parametrize("R,K,n_rows", [(37, 96, None), (300, 256, 211), (9, 7168, None)])
+@pytest.mark.parametrize("R,K,n_rows", [(37, 96, None), (300, 256, 211), (9, 7168, None),
+                                         (6, 2048, 5), (5, 16384, None), (5, 16400, None),
+                                         (7, 2064, None), (7, 8192, 6), (7, 8208, None)])
 def test_row_quantizer_bit_exact(R, K, n_rows):
     g = torch.Generator().manual_seed(R + K)
     x = (torch.randn(R, K, generator=g) * 3).to(torch.bfloat16)
@@ -83,6 +85,31 @@ def test_row_quantizer_bit_exact(R, K, n_rows):
     np.testing.assert_array_equal(s[:n].cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     np.testing.assert_array_equal(q[:n].cpu().numpy(), q_ref)
     assert torch.all(q[n:] == 0x55) and torch.all(s[n:] == -1.0)   # rows past n_rows untouched
+
+
+@pytest.mark.parametrize("T,d,E,k,cf", [(333, 384, 6, 3, 0.5), (512, 256, 256, 8, 1.25),
+                                        (64, 128, 8, 2, 0.0)])
+def test_permute_fp8_matches_oracle(T, d, E, k, cf):
+    """Codes and scales of each token, moved by the permutation: equal to the
+    oracle's row quantization of its dispatched rows, bit for bit."""
+    from moe_testlib import random_routing
+    g = torch.Generator().manual_seed(T + E)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    idx = random_routing(T, E, k, seed=T + d)
+    xq_tok, sx_tok = moe.moe_quantize_rows_fp8(x.cuda())
+    out = moe.moe_permute_fp8(xq_tok, sx_tok, torch.from_numpy(idx).cuda(), E, cf)
+    torch.cuda.synchronize()
+    C = oracle.capacity(T, E, k, cf)
+    counts, offsets, slot, row_src, n_drop = oracle.permute(idx, E, C)
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), counts)
+    np.testing.assert_array_equal(out["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(out["slot"].cpu().numpy(), slot)
+    assert out["n_dropped"].item() == n_drop
+    N = int(offsets[-1])
+    np.testing.assert_array_equal(out["row_src"][:N].cpu().numpy(), row_src)
+    xq, sx = oracle.quantize_rows_fp8(oracle.dispatch(bits(x), row_src))
+    np.testing.assert_array_equal(out["xq"][:N].cpu().numpy(), xq)
+    np.testing.assert_array_equal(out["sx"][:N].cpu().numpy().view(np.uint32), sx.view(np.uint32))
 
 
 def deq_rows(q, s):
@@ -141,19 +168,24 @@ def check_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, h, hq, sh, y):
 
 
 MLP_CASES = [
-    # (d, f, bucket sizes): ragged tails, M=64 tail tiles, empty and one-row
-    # buckets, several row tiles, both down-GEMM tile widths (d % 256)
-    (256, 384, [300, 0, 1, 129, 128, 257]),
-    (128, 256, [5, 140, 0, 0, 64, 128]),
-    (384, 128, [1, 1, 1, 400]),
-    (512, 640, [129] * 3),
-    (256, 256, [0, 0, 0]),
-    (256, 256, [170, 0, 128, 129, 233, 256, 250, 131]),
+    # (d, f, bucket sizes, pair): ragged tails, M=64 tail tiles, empty and
+    # one-row buckets, several row tiles, both down-GEMM tile widths (d % 256);
+    # pair=True gives a buffer of >= 512 rows per expert, which selects the
+    # CTA-pair tiles (256 rows, half tiles of 128 at the tails)
+    (256, 384, [300, 0, 1, 129, 128, 257], False),
+    (128, 256, [5, 140, 0, 0, 64, 128], False),
+    (384, 128, [1, 1, 1, 400], False),
+    (512, 640, [129] * 3, False),
+    (256, 256, [0, 0, 0], False),
+    (256, 256, [170, 0, 128, 129, 233, 256, 250, 131], False),
+    (256, 384, [300, 0, 1, 129, 128, 257, 700], True),
+    (512, 256, [1, 256, 511, 513, 1024], True),
+    (384, 256, [255, 257, 0], True),      # down GEMM: d % 256 != 0 keeps single-CTA tiles
 ]
 
 
-@pytest.mark.parametrize("d,f,sizes", MLP_CASES)
-def test_expert_mlp_fp8_matches_oracle(d, f, sizes):
+@pytest.mark.parametrize("d,f,sizes,pair", MLP_CASES)
+def test_expert_mlp_fp8_matches_oracle(d, f, sizes, pair):
     E = len(sizes)
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     N = int(offsets[-1])
@@ -163,7 +195,8 @@ def test_expert_mlp_fp8_matches_oracle(d, f, sizes):
     qg, sg = quantize_w(edge_weights(E, d, f, d + 1, d ** -0.5))
     qu, su = quantize_w(edge_weights(E, d, f, d + 2, d ** -0.5))
     qd, sd = quantize_w(edge_weights(E, f, d, d + 3, f ** -0.5))
-    out = run_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, N + 37, d, f)
+    max_rows = max(N + 37, 512 * E + 5) if pair else N + 37
+    out = run_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, max_rows, d, f)
     check_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, *out)
 
 
@@ -197,6 +230,8 @@ SMALL = [
     small("fine_small", T=512, d=256, E=256, k=8, f=256, cf=1.25, seed=12),
     small("decode_small", T=16, d=256, E=256, k=8, f=256, cf=0.0, seed=14),
     small("ragged_T", T=333, d=384, E=6, k=3, f=128, cf=0.5, seed=15),
+    small("pair_tiles", T=2048, d=256, E=4, k=2, f=256, cf=0.0, seed=19),
+    small("pair_tiles_drops", T=3000, d=512, E=4, k=3, f=384, cf=0.8, seed=20),
 ]
 
 

@@ -110,6 +110,19 @@ def dispatch(x_bits, row_src):
     return out
 
 
+def dispatch_padded(x_bits, topk_idx, slot, E, C):
+    """The padded [E*C, d] buffer and its row_src (-1 on padding rows)."""
+    x_bits = _c(x_bits, np.uint16)
+    topk_idx, slot = _c(topk_idx, np.int32), _c(slot, np.int32)
+    T, d = x_bits.shape
+    k = topk_idx.shape[1]
+    out = np.empty((E * C, d), np.uint16)
+    row_src = np.empty(E * C, np.int32)
+    lib().oracle_dispatch_padded(_ptr(x_bits), _ptr(topk_idx), _ptr(slot), _i64(T), _i64(d),
+                                 _i64(k), _i64(E), _i64(C), _ptr(out), _ptr(row_src))
+    return out, row_src
+
+
 def round_bf16(v):
     """Nearest bf16 value (ties to even) of a double, as the oracle rounds h."""
     return lib().oracle_round_bf16(float(v))

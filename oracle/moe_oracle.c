@@ -207,6 +207,27 @@ void oracle_swiglu_rows(const uint16_t* x_rows, int64_t n, int64_t d, int64_t f,
     }
 }
 
+/* ---- The padded [E, C, d] layout (a variant of step 4's buffer) ----
+ * Fixed-size expert buffers ("Expert Parallelism & All-to-All" (neelmishra),
+ * section "Why fixed-size buffers matter here"): bucket e occupies rows
+ * e*C .. e*C + C - 1; a kept pair (t, j) of expert e with slot s puts x[t] at
+ * row e*C + s; rows past a bucket's count stay zero.  row_src gives each
+ * row's token, -1 on padding rows. */
+void oracle_dispatch_padded(const uint16_t* x, const int32_t* topk_idx, const int32_t* slot,
+                            int64_t T, int64_t d, int64_t k, int64_t E, int64_t C, uint16_t* out,
+                            int32_t* row_src) {
+    memset(out, 0, (size_t)(E * C * d) * sizeof(uint16_t));
+    for (int64_t r = 0; r < E * C; ++r) row_src[r] = -1;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < k; ++j) {
+            const int64_t s = slot[t * k + j];
+            if (s < 0) continue;
+            const int64_t row = (int64_t)topk_idx[t * k + j] * C + s;
+            memcpy(out + row * d, x + t * d, (size_t)d * sizeof(uint16_t));
+            row_src[row] = (int32_t)t;
+        }
+}
+
 /* ---- FP8 (e4m3) expert weights: one variant of step 5's operands ----
  * Weight-only quantization with one scale per (expert, output column):
  *   s[e,n] = max_k |w[e,k,n]| / 448   (fp32, as the quantizer computes it)

@@ -405,3 +405,31 @@ def test_combine_inverts_dispatch_with_identity_expert():
             np.testing.assert_allclose(y, x64, rtol=1e-14, atol=1e-14)
         else:
             assert n_drop > 0 and none_kept.any() and (~none_kept).any()
+
+
+@pytest.mark.parametrize("T,E,k,cf", [(40, 4, 2, 0.75), (64, 8, 2, 1.25), (10, 3, 3, 0.0)])
+def test_dispatch_padded_bruteforce(T, E, k, cf):
+    """The padded buffer from its definition: bucket e at rows e*C.., token
+    rows at their slots, zero elsewhere; the kept rows are the ragged rows."""
+    r = np.random.default_rng(T + E)
+    x = r.integers(0, 1 << 16, size=(T, 6), dtype=np.uint16)
+    idx = np.argsort(r.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    C = oracle.capacity(T, E, k, cf)
+    counts, offsets, slot, row_src, _ = oracle.permute(idx, E, C)
+    pad, src = oracle.dispatch_padded(x, idx, slot, E, C)
+    want = np.zeros((E * C, 6), np.uint16)
+    want_src = np.full(E * C, -1, np.int32)
+    for e in range(E):
+        n = 0
+        for t in range(T):
+            if e in idx[t]:
+                if n < C:
+                    want[e * C + n] = x[t]
+                    want_src[e * C + n] = t
+                n += 1
+    np.testing.assert_array_equal(pad, want)
+    np.testing.assert_array_equal(src, want_src)
+    ragged = oracle.dispatch(x, row_src)
+    for e in range(E):
+        np.testing.assert_array_equal(pad[e * C:e * C + counts[e]],
+                                      ragged[offsets[e]:offsets[e + 1]])

@@ -144,7 +144,7 @@ class Layer:
     """Inputs, weights and buffers of one workload, resident on the device,
     and the step as C-ABI calls on one stream (five; seven with FP8 experts)."""
 
-    def __init__(self, cfg, device, token_seed, fp8=False):
+    def __init__(self, cfg, device, token_seed, fp8=False, padded=False):
         import mixture_experts_layer_36_b200 as moe
         self.moe = moe
         self.cfg = cfg
@@ -159,7 +159,10 @@ class Layer:
             torch.cuda.synchronize(device)
         self.x = synth.make_tokens(cfg, device, seed=token_seed)
         T, d, E, k, f = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f
-        self.rows = moe.moe_max_rows(T, E, k, cfg.cf)
+        self.padded = padded
+        # padded [E, C, d] layout: every bucket is C rows, all of them computed
+        self.rows = moe.moe_padded_rows(T, E, k, cfg.cf) if padded else \
+            moe.moe_max_rows(T, E, k, cfg.cf)
         z = lambda *s, dt: torch.empty(*s, dtype=dt, device=device)  # noqa: E731
         self.logits = z(T, E, dt=torch.float32)
         self.idx = z(T, k, dt=torch.int32)
@@ -171,6 +174,8 @@ class Layer:
             # the FP8 layer quantizes each token once and permutes codes + scales
             self.perm.update(xq=z(self.rows, d, dt=torch.uint8), sx=z(self.rows, dt=torch.float32))
             self.xq_tok, self.sx_tok = z(T, d, dt=torch.uint8), z(T, dt=torch.float32)
+        elif padded:
+            self.perm["x_pad"] = z(self.rows, d, dt=torch.bfloat16)
         else:
             self.perm["x_perm"] = z(self.rows, d, dt=torch.bfloat16)
         self.pws = z(max(moe.moe_permute_workspace_size(T, E, k), 16), dt=torch.uint8)
@@ -210,9 +215,14 @@ class Layer:
                                                           *q["w_down"], y_perm=self.y_perm,
                                                           dev_status=self.status))]
         else:
-            st += [("permute", lambda: m.moe_permute(self.x, self.idx, c.E, c.cf, out=p,
-                                                     ws=self.pws)),
-                   ("gate_up", lambda: m.moe_expert_gate_up(p["x_perm"], p["offsets"], w["w_gate"],
+            if self.padded:
+                st.append(("permute", lambda: m.moe_permute_padded(self.x, self.idx, c.E, c.cf,
+                                                                   out=p, ws=self.pws)))
+            else:
+                st.append(("permute", lambda: m.moe_permute(self.x, self.idx, c.E, c.cf, out=p,
+                                                            ws=self.pws)))
+            xin = p["x_pad"] if self.padded else p["x_perm"]
+            st += [("gate_up", lambda: m.moe_expert_gate_up(xin, p["offsets"], w["w_gate"],
                                                             w["w_up"], h=self.h,
                                                             dev_status=self.status)),
                    ("down", lambda: m.moe_expert_down(self.h, p["offsets"], w["w_down"],
@@ -233,6 +243,14 @@ class Layer:
 
     def layer_forward(self, x, y):
         w, c = self.w, self.cfg
+        if self.padded:
+            # no one-shot call for this layout: the stage entry points on x, y
+            x0, y0 = self.x, self.y
+            self.x, self.y = x, y
+            for _, call in self.steps:
+                call()
+            self.x, self.y = x0, y0
+            return
         if self.fp8:
             q = self.q
             self.moe.moe_layer_forward_fp8(x, w["w_router"], w["bias"], *q["w_gate"], *q["w_up"],
@@ -248,7 +266,8 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     dist = world > 1
     if dist:
         import torch.distributed as td
-    layer = Layer(cfg, dev, token_seed=rank_token_seed(cfg, rank), fp8=args.fp8)
+    layer = Layer(cfg, dev, token_seed=rank_token_seed(cfg, rank), fp8=args.fp8,
+                  padded=args.layout == "padded")
     stream = torch.cuda.current_stream()
 
     K = args.steps
@@ -277,7 +296,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                 for j, n in enumerate(names)}
     status = int(layer.status.item())
-    N = int(layer.perm["offsets"][cfg.E].item())
+    N = int(layer.perm["counts"].sum().item())          # kept pairs (either layout)
     active = int((layer.perm["counts"] > 0).sum().item())
     n_drop = int(layer.perm["n_dropped"].item())
 
@@ -392,6 +411,9 @@ def main():
     ap.add_argument("--config", default="mixtral")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layout", choices=["ragged", "padded"], default="ragged",
+                    help="padded: the static [E, C, d] expert buffers (every bucket C rows, all "
+                         "computed) in place of the ragged buckets")
     ap.add_argument("--fp8", action="store_true",
                     help="expert weights as e4m3 codes + fp32 column scales (quantized once "
                          "before timing); activations and accumulation as in the bf16 path")
@@ -411,7 +433,7 @@ def main():
         return reference_arm(args, cfg, rank, world)
     if args.profile:
         layer = Layer(cfg, torch.device("cuda", local_rank), token_seed=rank_token_seed(cfg, 0),
-                      fp8=args.fp8)
+                      fp8=args.fp8, padded=args.layout == "padded")
         for _ in range(args.warmup + args.steps):
             layer.step()
         torch.cuda.synchronize()
@@ -490,6 +512,8 @@ def main():
         "config": {"workload": describe(cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
                    "f": cfg.f, "cf": cfg.cf, "kept_pairs": r["N"], "dropped_pairs": r["n_dropped"],
                    "parallelism": f"replicas x{world} (token batches, no collective)",
+                   "layout": args.layout,
+                   "gemm_rows_computed": (r["layer"].rows if args.layout == "padded" else r["N"]),
                    "experts": ("e4m3 weights (fp32 column scales) x e4m3 activations (fp32 row "
                                "scales)") if args.fp8 else "bf16",
                    "l2": "inputs larger than L2 (expert weights "
@@ -531,9 +555,13 @@ def main():
         "clocks": {k_: r["clocks"][k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},
         "e2e": {"value": round(cfg.T * world * K / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-                "api": ("moe_layer_forward_fp8" if args.fp8 else "moe_layer_forward") +
-                       " (one-shot C-ABI call); every step copies x from pinned host memory and "
-                       "y back, on copy streams overlapping adjacent steps' compute"},
+                "api": ("the stage entry points (moe_route, moe_permute_padded, "
+                        "moe_expert_gate_up, moe_expert_down, moe_combine)"
+                        if args.layout == "padded" else
+                        ("moe_layer_forward_fp8" if args.fp8 else "moe_layer_forward") +
+                        " (one-shot C-ABI call)") +
+                       "; every step copies x from pinned host memory and y back, on copy "
+                       "streams overlapping adjacent steps' compute"},
         "gpu_launches": (KERNELS_PER_STEP_FP8 if args.fp8 else KERNELS_PER_STEP) * K,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -228,6 +228,26 @@ int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, con
                 const int32_t* slot, const int32_t* offsets, int64_t T, int64_t d, int64_t k,
                 void* y, void* stream);
 
+/* ---- Padded-capacity layout (an optional variant of moe_permute) ----
+ * The static [E, C, d] buffer the neelmishra page contrasts with ragged
+ * buckets ("Expert Parallelism & All-to-All", section "Why fixed-size buffers
+ * matter here": fixed-shape buffers cost padded compute when an expert is
+ * under-filled).  Bucket e occupies rows e*C .. e*C + C - 1 whatever its
+ * count. */
+
+/* E*C rows of the padded buffer; -1 on bad args or E*C >= 2^31. */
+int64_t moe_padded_rows(int64_t T, int64_t E, int64_t k, double cf);
+
+/* moe_permute into the padded layout: counts, slot and n_dropped as
+ * moe_permute; offsets[e] = e*C (offsets[E] = E*C), so the grouped GEMM and
+ * combine entry points run on it unchanged and compute every row of every
+ * bucket; x_pad bf16 [E*C, d] holds bucket e's kept rows at e*C + slot and
+ * zeros after them; row_src i32 [E*C] the source token, -1 on padding rows. */
+int moe_permute_padded(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
+                       int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
+                       int32_t* row_src, void* x_pad, int32_t* n_dropped, void* ws,
+                       size_t ws_bytes, void* stream);
+
 /* ---- FP8 experts (e4m3 activations and weights; an optional variant) ----
  * Post-training FP8 quantization of the experts (inferensys.com "Expert
  * Parallelism" glossary, quantization entry).  One rule for every group of

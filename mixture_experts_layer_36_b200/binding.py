@@ -32,7 +32,8 @@ EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "mo
             "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
             "moe_combine", "moe_layer_forward", "moe_quantize_weights_fp8",
             "moe_quantize_rows_fp8", "moe_permute_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8",
-            "moe_workspace_size_fp8", "moe_layer_forward_fp8"]
+            "moe_workspace_size_fp8", "moe_layer_forward_fp8", "moe_padded_rows",
+            "moe_permute_padded"]
 
 
 class MoEError(RuntimeError):
@@ -74,6 +75,9 @@ def _load():
                                                   p]),
         "moe_expert_down_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p]),
         "moe_workspace_size_fp8": (sz, [i64, i64, i64, i64, i64, dbl]),
+        "moe_padded_rows": (i64, [i64, i64, i64, dbl]),
+        "moe_permute_padded": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
+                                              sz, p]),
         "moe_layer_forward_fp8": (ctypes.c_int, [p, p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64,
                                                  dbl, p, p, sz, p]),
     }
@@ -324,6 +328,40 @@ def moe_layer_forward(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws
         _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k,
         f, float(cf), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
     return y, ws
+
+
+# ----------------------------------------------------------------- padded layout
+
+def moe_padded_rows(T, E, k, cf):
+    return int(_lib.moe_padded_rows(T, E, k, float(cf)))
+
+
+def moe_permute_padded(x, topk_idx, E, cf, out=None, ws=None, stream=None):
+    """moe_permute into the padded [E*C, d] layout.  Returns a dict like
+    moe_permute's with "x_pad" in place of "x_perm" (offsets[e] = e*C)."""
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    _want(x, "x", torch.bfloat16)
+    _want(topk_idx, "topk_idx", torch.int32, (T, k))
+    rows = moe_padded_rows(T, E, k, cf)
+    if rows < 0:
+        raise ValueError("padded layout too large")
+    dev = x.device
+    if out is None:
+        out = {"counts": torch.empty(E, dtype=torch.int32, device=dev),
+               "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+               "slot": torch.empty(T, k, dtype=torch.int32, device=dev),
+               "row_src": torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+               "x_pad": torch.empty(max(rows, 1), d, dtype=torch.bfloat16, device=dev),
+               "n_dropped": torch.empty(1, dtype=torch.int32, device=dev)}
+    if ws is None:
+        ws = torch.empty(max(moe_permute_workspace_size(T, E, k), 16), dtype=torch.uint8,
+                         device=dev)
+    _check("moe_permute_padded", _lib.moe_permute_padded(
+        _ptr(x), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]), _ptr(out["offsets"]),
+        _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["x_pad"]), _ptr(out["n_dropped"]),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out
 
 
 # ----------------------------------------------------------------- FP8 experts

@@ -31,6 +31,10 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
                                 int32_t* counts, int32_t* offsets, int32_t* slot,
                                 int32_t* row_src, uint8_t* x_perm, float* perm_scale,
                                 int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s);
+cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d,
+                                  int E, int k, int64_t C, int32_t* counts, int32_t* offsets,
+                                  int32_t* slot, int32_t* row_src, __nv_bfloat16* x_pad,
+                                  int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s);
 cudaError_t launch_quantize_weights(const __nv_bfloat16* w, int E, int K, int N, uint8_t* q,
                                     float* scale, cudaStream_t s);
 cudaError_t launch_quantize_rows(const __nv_bfloat16* x, int R, int K, const int32_t* n_rows,
@@ -326,6 +330,33 @@ int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, con
                                     topk_w, slot,
                                     offsets, (int)T, (int)d, (int)k,
                                     static_cast<__nv_bfloat16*>(y), as_stream(stream)));
+}
+
+int64_t moe_padded_rows(int64_t T, int64_t E, int64_t k, double cf) {
+  const int64_t C = moe_capacity(T, E, k, cf);
+  if (C < 0) return -1;
+  const int64_t rows = E * C;
+  return rows >= (int64_t(1) << 31) ? -1 : rows;
+}
+
+int moe_permute_padded(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
+                       int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
+                       int32_t* row_src, void* x_pad, int32_t* n_dropped, void* ws,
+                       size_t ws_bytes, void* stream) {
+  int st = check_routing_shape(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_width(d)) != MOE_OK) return st;
+  const int64_t C = moe_capacity(T, E, k, cf);
+  if (C < 0 || moe_padded_rows(T, E, k, cf) < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !topk_idx || !counts || !offsets || !slot || !row_src || !x_pad || !n_dropped || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_pad) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_permute_workspace_size(T, E, k)) return MOE_ERR_WORKSPACE;
+  return cuda_status(moe::launch_permute_padded(
+      static_cast<const __nv_bfloat16*>(x), topk_idx, (int)T, (int)d, (int)E, (int)k, C, counts,
+      offsets, slot, row_src, static_cast<__nv_bfloat16*>(x_pad), n_dropped,
+      static_cast<int32_t*>(ws), as_stream(stream)));
 }
 
 int moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t N, uint8_t* w_q,

@@ -44,7 +44,6 @@ namespace moe {
 constexpr int kBM = 128;
 constexpr int kBK = 64;                 // one 128-byte swizzle atom of bf16 along K
 constexpr int kGemmThreads = 192;
-constexpr int kUmmaK = 16;
 constexpr int kChunkBytes = 64 * kBK * 2;   // one B chunk: 64 N x 64 K bf16 = 8 KB
 
 // ---------------------------------------------------------------- epilogue stores

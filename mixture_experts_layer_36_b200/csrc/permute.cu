@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kScatThreads)
                            int32_t* __restrict__ counts,
                            int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped,
                            int32_t* __restrict__ row_src, uint8_t* __restrict__ x_perm,
-                           float* __restrict__ perm_scale) {
+                           float* __restrict__ perm_scale, bool padded) {
   __shared__ int32_t s_off[256];
   __shared__ int32_t s_base[256];
   __shared__ int32_t warp_sum[8];
@@ -140,14 +140,16 @@ __global__ void __launch_bounds__(kScatThreads)
     total_rows += warp_sum[w];
     dtotal += warp_drop[w];
   }
-  if (tid < E) s_off[tid] = wbase + incl - kept;
+  // ragged: buckets packed back to back; padded: bucket e starts at row e*C
+  const int my_off = padded ? (int)((int64_t)tid * C) : wbase + incl - kept;
+  if (tid < E) s_off[tid] = my_off;
   if (blockIdx.x == 0) {
     if (tid < E) {
       counts[tid] = kept;
-      offsets[tid] = wbase + incl - kept;
+      offsets[tid] = my_off;
     }
     if (tid == 0) {
-      offsets[E] = total_rows;
+      offsets[E] = padded ? (int)((int64_t)E * C) : total_rows;
       *n_dropped = dtotal;
     }
   }
@@ -203,6 +205,21 @@ size_t permute_scratch_bytes(int64_t T, int64_t E) {
   return (size_t)(nchunks * E * (int64_t)sizeof(int32_t));
 }
 
+// 3. padded layout only: rows of each bucket past its kept count are zeroed
+//    (row_src = -1), one warp per padded row.
+__global__ void __launch_bounds__(256)
+    permute_pad_fill_kernel(const int32_t* __restrict__ counts, int E, int64_t C, int row_bytes,
+                            int32_t* __restrict__ row_src, uint8_t* __restrict__ x_pad) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t r = (int64_t)blockIdx.x * 8 + warp;
+  if (r >= (int64_t)E * C) return;
+  const int e = (int)(r / C);
+  if (r - (int64_t)e * C < counts[e]) return;
+  if (lane == 0) row_src[r] = -1;
+  uint4* dst = reinterpret_cast<uint4*>(x_pad + r * row_bytes);
+  for (int v = lane; v < row_bytes / 16; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+}
+
 // Rows of row_bytes bytes (a multiple of 16); x_scale / perm_scale (one fp32
 // per row, moved with it) may be null.
 cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_scale,
@@ -215,7 +232,26 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
   const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
   permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
       x, row_bytes, x_scale, topk_idx, slot, chunk_hist, nchunks, T, E, k, C, tpc, counts,
-      offsets, n_dropped, row_src, x_perm, perm_scale);
+      offsets, n_dropped, row_src, x_perm, perm_scale, false);
+  return cudaGetLastError();
+}
+
+// The padded [E, C, d] layout: bucket e holds rows e*C .. e*C + C - 1, its
+// kept pairs first (in slot order), the rest zero.
+cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d,
+                                  int E, int k, int64_t C, int32_t* counts, int32_t* offsets,
+                                  int32_t* slot, int32_t* row_src, __nv_bfloat16* x_pad,
+                                  int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s) {
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist);
+  const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
+  uint8_t* xp = reinterpret_cast<uint8_t*>(x_pad);
+  permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
+      reinterpret_cast<const uint8_t*>(x), d * 2, nullptr, topk_idx, slot, chunk_hist, nchunks, T,
+      E, k, C, tpc, counts, offsets, n_dropped, row_src, xp, nullptr, true);
+  const int64_t rows = (int64_t)E * C;
+  permute_pad_fill_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(counts, E, C, d * 2, row_src,
+                                                                     xp);
   return cudaGetLastError();
 }
 

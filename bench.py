@@ -144,7 +144,7 @@ class Layer:
     """Inputs, weights and buffers of one workload, resident on the device,
     and the step as C-ABI calls on one stream (five; seven with FP8 experts)."""
 
-    def __init__(self, cfg, device, token_seed, fp8=False, padded=False):
+    def __init__(self, cfg, device, token_seed, fp8=False, padded=False, fused=False):
         import mixture_experts_layer_36_b200 as moe
         self.moe = moe
         self.cfg = cfg
@@ -160,6 +160,7 @@ class Layer:
         self.x = synth.make_tokens(cfg, device, seed=token_seed)
         T, d, E, k, f = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f
         self.padded = padded
+        self.fused = fused
         # padded [E, C, d] layout: every bucket is C rows, all of them computed
         self.rows = moe.moe_padded_rows(T, E, k, cfg.cf) if padded else \
             moe.moe_max_rows(T, E, k, cfg.cf)
@@ -176,6 +177,11 @@ class Layer:
             self.xq_tok, self.sx_tok = z(T, d, dt=torch.uint8), z(T, dt=torch.float32)
         elif padded:
             self.perm["x_pad"] = z(self.rows, d, dt=torch.bfloat16)
+        elif fused:
+            # no permuted copies: row_pair for the scatter, an fp32 token accumulator
+            self.perm.update(row_pair=z(self.rows, dt=torch.int32),
+                             y32=z(T, d, dt=torch.float32),
+                             x_perm=z(self.rows, d, dt=torch.bfloat16))
         else:
             self.perm["x_perm"] = z(self.rows, d, dt=torch.bfloat16)
         self.pws = z(max(moe.moe_permute_workspace_size(T, E, k), 16), dt=torch.uint8)
@@ -185,9 +191,10 @@ class Layer:
         self.y = z(T, d, dt=torch.bfloat16)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         if fp8:
-            self.xq, self.sx = z(self.rows, d, dt=torch.uint8), z(self.rows, dt=torch.float32)
             self.hq, self.sh = z(self.rows, f, dt=torch.uint8), z(self.rows, dt=torch.float32)
             self.ws = z(moe.moe_workspace_size_fp8(T, d, E, k, f, cfg.cf), dt=torch.uint8)
+        elif fused:
+            self.ws = z(moe.moe_workspace_size_fused(T, d, E, k, f, cfg.cf), dt=torch.uint8)
         else:
             self.ws = z(moe.moe_workspace_size(T, d, E, k, f, cfg.cf), dt=torch.uint8)
         self.steps = self.stages()
@@ -214,6 +221,18 @@ class Layer:
                    ("down", lambda: m.moe_expert_down_fp8(self.hq, self.sh, p["offsets"],
                                                           *q["w_down"], y_perm=self.y_perm,
                                                           dev_status=self.status))]
+        elif self.fused:
+            st += [("permute", lambda: m.moe_permute_fused(self.x, self.idx, c.E, c.cf, out=p,
+                                                           ws=self.pws)),
+                   ("gate_up", lambda: m.moe_expert_gate_up(p["x_perm"], p["offsets"],
+                                                            w["w_gate"], w["w_up"], h=self.h,
+                                                            dev_status=self.status)),
+                   ("down", lambda: m.moe_expert_down_scatter(
+                       self.h, p["offsets"], w["w_down"], p["row_pair"], self.tw, p["y32"],
+                       dev_status=self.status)),
+                   ("combine", lambda: m.moe_combine_finalize(p["y32"], self.x, p["slot"],
+                                                              y=self.y))]
+            return st
         else:
             if self.padded:
                 st.append(("permute", lambda: m.moe_permute_padded(self.x, self.idx, c.E, c.cf,
@@ -251,6 +270,10 @@ class Layer:
                 call()
             self.x, self.y = x0, y0
             return
+        if self.fused:
+            self.moe.moe_layer_forward_fused(x, w["w_router"], w["bias"], w["w_gate"], w["w_up"],
+                                             w["w_down"], c.k, c.cf, y=y, ws=self.ws)
+            return
         if self.fp8:
             q = self.q
             self.moe.moe_layer_forward_fp8(x, w["w_router"], w["bias"], *q["w_gate"], *q["w_up"],
@@ -267,7 +290,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     if dist:
         import torch.distributed as td
     layer = Layer(cfg, dev, token_seed=rank_token_seed(cfg, rank), fp8=args.fp8,
-                  padded=args.layout == "padded")
+                  padded=args.layout == "padded", fused=args.fused)
     stream = torch.cuda.current_stream()
 
     K = args.steps
@@ -414,6 +437,9 @@ def main():
     ap.add_argument("--layout", choices=["ragged", "padded"], default="ragged",
                     help="padded: the static [E, C, d] expert buffers (every bucket C rows, all "
                          "computed) in place of the ragged buckets")
+    ap.add_argument("--fused", action="store_true",
+                    help="the fused path: the down GEMM adds gate-weighted rows into an fp32 "
+                         "token accumulator (no y_perm, no separate combine)")
     ap.add_argument("--fp8", action="store_true",
                     help="expert weights as e4m3 codes + fp32 column scales (quantized once "
                          "before timing); activations and accumulation as in the bf16 path")
@@ -421,6 +447,10 @@ def main():
                     help="run W + K layer steps only (no timing, e2e or oracle): a short, "
                          "fixed launch sequence for ncu")
     args = ap.parse_args()
+    if args.fused and (args.fp8 or args.layout != "ragged"):
+        ap.error("--fused runs the bf16 experts on ragged buckets")
+    if args.fp8 and args.layout != "ragged":
+        ap.error("--fp8 runs on ragged buckets")
     if args.warmup < 3:
         args.warmup = 3
 
@@ -433,7 +463,7 @@ def main():
         return reference_arm(args, cfg, rank, world)
     if args.profile:
         layer = Layer(cfg, torch.device("cuda", local_rank), token_seed=rank_token_seed(cfg, 0),
-                      fp8=args.fp8, padded=args.layout == "padded")
+                      fp8=args.fp8, padded=args.layout == "padded", fused=args.fused)
         for _ in range(args.warmup + args.steps):
             layer.step()
         torch.cuda.synchronize()
@@ -486,6 +516,11 @@ def main():
     hbm_bound = gemm1_flop / g1_bytes < ridge
     bytes_perm = cfg.T * cfg.d * wb + r["N"] * cfg.d * wb
     bytes_comb = r["N"] * cfg.d * 4 + cfg.T * cfg.d * 2
+    if args.fused:
+        # the permutation also zeroes the fp32 accumulator; the finishing pass
+        # reads it and writes y
+        bytes_perm += cfg.T * cfg.d * 4
+        bytes_comb = cfg.T * cfg.d * 4 + cfg.T * cfg.d * 2
     quant_rooflines = {}
     if args.fp8:
         # the row quantizers: bf16 rows read once (the second pass hits cache),
@@ -513,6 +548,7 @@ def main():
                    "f": cfg.f, "cf": cfg.cf, "kept_pairs": r["N"], "dropped_pairs": r["n_dropped"],
                    "parallelism": f"replicas x{world} (token batches, no collective)",
                    "layout": args.layout,
+                   "path": "fused (down GEMM + weighted scatter)" if args.fused else "staged",
                    "gemm_rows_computed": (r["layer"].rows if args.layout == "padded" else r["N"]),
                    "experts": ("e4m3 weights (fp32 column scales) x e4m3 activations (fp32 row "
                                "scales)") if args.fp8 else "bf16",
@@ -558,7 +594,8 @@ def main():
                 "api": ("the stage entry points (moe_route, moe_permute_padded, "
                         "moe_expert_gate_up, moe_expert_down, moe_combine)"
                         if args.layout == "padded" else
-                        ("moe_layer_forward_fp8" if args.fp8 else "moe_layer_forward") +
+                        ("moe_layer_forward_fused" if args.fused else
+                         "moe_layer_forward_fp8" if args.fp8 else "moe_layer_forward") +
                         " (one-shot C-ABI call)") +
                        "; every step copies x from pinned host memory and y back, on copy "
                        "streams overlapping adjacent steps' compute"},

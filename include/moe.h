@@ -114,12 +114,16 @@ typedef enum {
   MOE_WS_SH = 17,        /* f32 [max_rows]    their row scales */
   MOE_WS_XQ_TOK = 18,    /* u8  [T, d]        e4m3 codes of x (before the permutation) */
   MOE_WS_SX_TOK = 19,    /* f32 [T]           their row scales */
-  MOE_WS_FP8_NUM_FIELDS = 20
+  MOE_WS_FP8_NUM_FIELDS = 20,
+  /* moe_layer_forward_fused only (right after the first MOE_WS_NUM_FIELDS) */
+  MOE_WS_ROW_PAIR = 20,  /* i32 [max_rows]    t*k + j of each kept row */
+  MOE_WS_Y32 = 21        /* f32 [T, d]        gate-weighted sum of the expert outputs */
 } moe_ws_field;
 
 /* Byte offset of a field inside the moe_layer_forward workspace (each field
  * 256-byte aligned; fields MOE_WS_XQ .. MOE_WS_SX_TOK exist only in a
- * moe_layer_forward_fp8 workspace); -1 on bad args. */
+ * moe_layer_forward_fp8 workspace, MOE_WS_ROW_PAIR and MOE_WS_Y32 only in a
+ * moe_layer_forward_fused one); -1 on bad args. */
 int64_t moe_workspace_field_offset(int field, int64_t T, int64_t d, int64_t E, int64_t k,
                                    int64_t f, double cf);
 
@@ -247,6 +251,61 @@ int moe_permute_padded(const void* x, const int32_t* topk_idx, int64_t T, int64_
                        int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
                        int32_t* row_src, void* x_pad, int32_t* n_dropped, void* ws,
                        size_t ws_bytes, void* stream);
+
+/* ---- Fused path (an optional variant) ----
+ * The combine folded into the down GEMM ("Expert Parallelism" guide
+ * (infra.bea.ai), section 5: fuse the gather into the expert GEMM and the
+ * weighted scatter into its epilogue): GEMM 2 adds each gate-weighted output
+ * row into an fp32 token accumulator y32 (red.add) instead of storing y_perm,
+ * and a last pass rounds y32 to bf16.  The summation order of a token's k
+ * terms then follows the GEMM tiles' completion, not j: results agree with
+ * moe_layer_forward to fp32 rounding but are not bit-reproducible run to run.
+ * The gather side (GEMM 1 reading x by row_src with TMA tile::gather4, no
+ * x_perm) is available as moe_expert_gate_up_gather; it saves the x_perm
+ * buffer but costs one 4-row copy per 512 bytes of A, which on B200 made the
+ * gate/up GEMM ~3x slower than the permuted copy plus a tile load, so the
+ * fused layer keeps the copy. */
+
+/* The permutation for the fused path: moe_permute (counts, offsets, slot,
+ * row_src, n_dropped; x_perm when x and x_perm are non-null, else no row
+ * copy) plus row_pair i32 [max_rows] (t*k + j of each kept row) and, when
+ * y32 is non-null, y32 f32 [T,d] zeroed. */
+int moe_permute_fused(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
+                      int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
+                      int32_t* row_src, int32_t* row_pair, void* x_perm, int32_t* n_dropped,
+                      float* y32, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_expert_gate_up with A row r of bucket storage = x[row_src[r]] (x bf16
+ * [T,d], row_src from the permutation; no x_perm). */
+int moe_expert_gate_up_gather(const void* x, int64_t T, const int32_t* row_src,
+                              const int32_t* offsets, int64_t E, int64_t d, int64_t f,
+                              int64_t max_rows, const void* w_gate, const void* w_up, void* h,
+                              int32_t* dev_status, void* stream);
+
+/* moe_expert_down with the combine's weighted sum in its epilogue:
+ * y32[t, :] += topk_w[p] * (h[r] Wd[e]) for each kept row r, p = row_pair[r],
+ * t = p / k.  y32 f32 [T,d] must hold zeros (or a sum to add to). */
+int moe_expert_down_scatter(const void* h, const int32_t* offsets, int64_t E, int64_t d,
+                            int64_t f, int64_t max_rows, const void* w_down,
+                            const int32_t* row_pair, const float* topk_w, int64_t k, float* y32,
+                            int32_t* dev_status, void* stream);
+
+/* y[t] = bf16(y32[t]), or x[t] when every pair of t was dropped (slot < 0). */
+int moe_combine_finalize(const float* y32, const void* x, const int32_t* slot, int64_t T,
+                         int64_t d, int64_t k, void* y, void* stream);
+
+/* Workspace of moe_layer_forward_fused: the moe_layer_forward fields followed
+ * by MOE_WS_ROW_PAIR and MOE_WS_Y32 (0 on invalid shapes). */
+size_t moe_workspace_size_fused(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                                double cf);
+
+/* The layer on the fused path: moe_route, moe_permute_fused (with x_perm),
+ * moe_expert_gate_up, moe_expert_down_scatter, moe_combine_finalize.
+ * Arguments as moe_layer_forward. */
+int moe_layer_forward_fused(const void* x, const float* w_router, const float* bias,
+                            const void* w_gate, const void* w_up, const void* w_down, int64_t T,
+                            int64_t d, int64_t E, int64_t k, int64_t f, double cf, void* y,
+                            void* ws, size_t ws_bytes, void* stream);
 
 /* ---- FP8 experts (e4m3 activations and weights; an optional variant) ----
  * Post-training FP8 quantization of the experts (inferensys.com "Expert

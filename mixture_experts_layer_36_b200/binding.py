@@ -24,7 +24,7 @@ DEV_ERR_BAD_OFFSETS = 2
 # workspace fields of moe_layer_forward (enum moe_ws_field)
 WS_FIELDS = ["status", "logits", "topk_idx", "topk_w", "slot", "counts", "offsets", "n_dropped",
              "row_src", "permute", "x_perm", "h", "y_perm", "route", "xq", "sx", "hq", "sh",
-             "xq_tok", "sx_tok"]
+             "xq_tok", "sx_tok", "row_pair", "y32"]
 
 EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "moe_capacity",
             "moe_max_rows",
@@ -33,7 +33,9 @@ EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "mo
             "moe_combine", "moe_layer_forward", "moe_quantize_weights_fp8",
             "moe_quantize_rows_fp8", "moe_permute_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8",
             "moe_workspace_size_fp8", "moe_layer_forward_fp8", "moe_padded_rows",
-            "moe_permute_padded"]
+            "moe_permute_padded", "moe_permute_fused", "moe_expert_gate_up_gather",
+            "moe_expert_down_scatter", "moe_combine_finalize", "moe_workspace_size_fused",
+            "moe_layer_forward_fused"]
 
 
 class MoEError(RuntimeError):
@@ -76,6 +78,16 @@ def _load():
         "moe_expert_down_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p]),
         "moe_workspace_size_fp8": (sz, [i64, i64, i64, i64, i64, dbl]),
         "moe_padded_rows": (i64, [i64, i64, i64, dbl]),
+        "moe_permute_fused": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
+                                             p, p, sz, p]),
+        "moe_expert_gate_up_gather": (ctypes.c_int, [p, i64, p, p, i64, i64, i64, i64, p, p, p, p,
+                                                     p]),
+        "moe_expert_down_scatter": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, i64, p, p,
+                                                   p]),
+        "moe_combine_finalize": (ctypes.c_int, [p, p, p, i64, i64, i64, p, p]),
+        "moe_workspace_size_fused": (sz, [i64, i64, i64, i64, i64, dbl]),
+        "moe_layer_forward_fused": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl,
+                                                   p, p, sz, p]),
         "moe_permute_padded": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
                                               sz, p]),
         "moe_layer_forward_fp8": (ctypes.c_int, [p, p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64,
@@ -330,6 +342,115 @@ def moe_layer_forward(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws
     return y, ws
 
 
+# ----------------------------------------------------------------- fused path
+
+def moe_permute_fused(x, topk_idx, E, cf, copy_rows=True, out=None, ws=None, stream=None):
+    """The permutation for the fused path.  Returns a dict with counts, offsets,
+    slot, row_src, row_pair, n_dropped, a zeroed fp32 token accumulator "y32"
+    [T, d] and, with copy_rows, "x_perm"."""
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    _want(x, "x", torch.bfloat16)
+    _want(topk_idx, "topk_idx", torch.int32, (T, k))
+    rows = moe_max_rows(T, E, k, cf)
+    dev = x.device
+    if out is None:
+        out = {"counts": torch.empty(E, dtype=torch.int32, device=dev),
+               "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+               "slot": torch.empty(T, k, dtype=torch.int32, device=dev),
+               "row_src": torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+               "row_pair": torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+               "n_dropped": torch.empty(1, dtype=torch.int32, device=dev),
+               "y32": torch.empty(T, d, dtype=torch.float32, device=dev)}
+        if copy_rows:
+            out["x_perm"] = torch.empty(max(rows, 1), d, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = torch.empty(max(moe_permute_workspace_size(T, E, k), 16), dtype=torch.uint8,
+                         device=dev)
+    xp = out.get("x_perm") if copy_rows else None
+    _check("moe_permute_fused", _lib.moe_permute_fused(
+        _ptr(x) if copy_rows else None, _ptr(topk_idx), T, d, E, k, float(cf),
+        _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]),
+        _ptr(out["row_pair"]), _ptr(xp), _ptr(out["n_dropped"]), _ptr(out.get("y32")), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return out
+
+
+def moe_expert_gate_up_gather(x, row_src, offsets, w_gate, w_up, max_rows, h=None,
+                              dev_status=None, stream=None):
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    _want(x, "x", torch.bfloat16)
+    _want(row_src, "row_src", torch.int32)
+    _want(offsets, "offsets", torch.int32, (E + 1,))
+    _want(w_gate, "w_gate", torch.bfloat16, (E, d, f))
+    _want(w_up, "w_up", torch.bfloat16, (E, d, f))
+    h = torch.empty(max_rows, f, dtype=torch.bfloat16, device=x.device) if h is None else h
+    _want(h, "h", torch.bfloat16, (max_rows, f))
+    _check("moe_expert_gate_up_gather", _lib.moe_expert_gate_up_gather(
+        _ptr(x), T, _ptr(row_src), _ptr(offsets), E, d, f, max_rows, _ptr(w_gate), _ptr(w_up),
+        _ptr(h), _ptr(dev_status), _stream(stream)))
+    return h
+
+
+def moe_expert_down_scatter(h, offsets, w_down, row_pair, topk_w, y32, dev_status=None,
+                            stream=None):
+    rows, f = h.shape
+    E, _, d = w_down.shape
+    k = topk_w.shape[1]
+    _want(h, "h", torch.bfloat16)
+    _want(offsets, "offsets", torch.int32, (E + 1,))
+    _want(w_down, "w_down", torch.bfloat16, (E, f, d))
+    _want(row_pair, "row_pair", torch.int32)
+    _want(topk_w, "topk_w", torch.float32)
+    _want(y32, "y32", torch.float32, (topk_w.shape[0], d))
+    _check("moe_expert_down_scatter", _lib.moe_expert_down_scatter(
+        _ptr(h), _ptr(offsets), E, d, f, rows, _ptr(w_down), _ptr(row_pair), _ptr(topk_w), k,
+        _ptr(y32), _ptr(dev_status), _stream(stream)))
+    return y32
+
+
+def moe_combine_finalize(y32, x, slot, y=None, stream=None):
+    T, d = x.shape
+    k = slot.shape[1]
+    _want(y32, "y32", torch.float32, (T, d))
+    _want(x, "x", torch.bfloat16)
+    _want(slot, "slot", torch.int32, (T, k))
+    y = torch.empty_like(x) if y is None else y
+    _want(y, "y", torch.bfloat16, (T, d))
+    _check("moe_combine_finalize", _lib.moe_combine_finalize(
+        _ptr(y32), _ptr(x), _ptr(slot), T, d, k, _ptr(y), _stream(stream)))
+    return y
+
+
+def moe_workspace_size_fused(T, d, E, k, f, cf):
+    return int(_lib.moe_workspace_size_fused(T, d, E, k, f, float(cf)))
+
+
+def moe_layer_forward_fused(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws=None,
+                            stream=None):
+    """The whole layer on the fused path.  Returns (y, ws)."""
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    _want(x, "x", torch.bfloat16)
+    _want(w_router, "w_router", torch.float32, (d, E))
+    if bias is not None:
+        _want(bias, "bias", torch.float32, (E,))
+    _want(w_gate, "w_gate", torch.bfloat16, (E, d, f))
+    _want(w_up, "w_up", torch.bfloat16, (E, d, f))
+    _want(w_down, "w_down", torch.bfloat16, (E, f, d))
+    nbytes = moe_workspace_size_fused(T, d, E, k, f, cf)
+    if ws is None:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _want(ws, "ws", torch.uint8)
+    y = torch.empty_like(x) if y is None else y
+    _want(y, "y", torch.bfloat16, (T, d))
+    _check("moe_layer_forward_fused", _lib.moe_layer_forward_fused(
+        _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k,
+        f, float(cf), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+    return y, ws
+
+
 # ----------------------------------------------------------------- padded layout
 
 def moe_padded_rows(T, E, k, cf):
@@ -502,6 +623,7 @@ def workspace_view(ws, field, T, d, E, k, f, cf):
         "xq": (torch.uint8, (rows, d)), "sx": (torch.float32, (rows,)),
         "hq": (torch.uint8, (rows, f)), "sh": (torch.float32, (rows,)),
         "xq_tok": (torch.uint8, (T, d)), "sx_tok": (torch.float32, (T,)),
+        "row_pair": (torch.int32, (rows,)), "y32": (torch.float32, (T, d)),
     }[field]
     dtype, shape = spec
     off = moe_workspace_field_offset(field, T, d, E, k, f, cf)

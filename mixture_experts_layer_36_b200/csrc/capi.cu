@@ -15,13 +15,15 @@ cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int 
                            int k, int64_t C, int32_t* counts, int32_t* offsets, int32_t* slot,
                            int32_t* row_src, __nv_bfloat16* x_perm, int32_t* n_dropped,
                            int32_t* chunk_hist, cudaStream_t s);
-cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
+cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, int E, int d,
                            int f, int max_rows, const __nv_bfloat16* w_gate,
                            const __nv_bfloat16* w_up, __nv_bfloat16* h, int32_t* status,
-                           cudaStream_t s, bool* map_failed);
+                           cudaStream_t s, bool* map_failed, const FuseArgs& fz);
 cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
                         int max_rows, const __nv_bfloat16* w_down, float* y_perm,
-                        int32_t* status, cudaStream_t s, bool* map_failed);
+                        int32_t* status, cudaStream_t s, bool* map_failed, const FuseArgs& fz);
+cudaError_t launch_finalize(const float* y32, const __nv_bfloat16* x, const int32_t* slot, int T,
+                            int d, int k, __nv_bfloat16* y, cudaStream_t s);
 cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
@@ -30,7 +32,8 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
                                 const int32_t* topk_idx, int T, int E, int k, int64_t C,
                                 int32_t* counts, int32_t* offsets, int32_t* slot,
                                 int32_t* row_src, uint8_t* x_perm, float* perm_scale,
-                                int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s);
+                                int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
+                                int32_t* row_pair, float* zero_rows, int zero_cols);
 cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d,
                                   int E, int k, int64_t C, int32_t* counts, int32_t* offsets,
                                   int32_t* slot, int32_t* row_src, __nv_bfloat16* x_pad,
@@ -43,11 +46,11 @@ cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_
                                 int E, int d, int f, int max_rows, const uint8_t* wq_gate,
                                 const float* s_gate, const uint8_t* wq_up, const float* s_up,
                                 __nv_bfloat16* h, int32_t* status, cudaStream_t s,
-                                bool* map_failed);
+                                bool* map_failed, const FuseArgs& fz);
 cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int32_t* offsets,
                              int E, int d, int f, int max_rows, const uint8_t* wq_down,
                              const float* s_down, float* y_perm, int32_t* status, cudaStream_t s,
-                             bool* map_failed);
+                             bool* map_failed, const FuseArgs& fz);
 }  // namespace moe
 
 namespace moe {
@@ -72,6 +75,7 @@ using moe::launch_down;
 using moe::launch_gate_up;
 using moe::launch_permute;
 using moe::launch_route;
+using moe::FuseArgs;
 
 namespace {
 
@@ -195,6 +199,15 @@ int64_t moe_workspace_field_offset(int field, int64_t T, int64_t d, int64_t E, i
                                    int64_t f, double cf) {
   size_t sz[MOE_WS_NUM_FIELDS];
   size_t sz8[MOE_WS_FP8_NUM_FIELDS - MOE_WS_NUM_FIELDS];
+  if (field == MOE_WS_ROW_PAIR || field == MOE_WS_Y32) {
+    // the fused layer's extra fields follow the standard ones
+    const size_t base = moe_workspace_size(T, d, E, k, f, cf);
+    const int64_t rows = moe_max_rows(T, E, k, cf);
+    if (base == 0 || rows < 0) return -1;
+    return (int64_t)(field == MOE_WS_ROW_PAIR
+                         ? base
+                         : base + align256(size_t(rows) * sizeof(int32_t)));
+  }
   if (field < 0 || field >= MOE_WS_FP8_NUM_FIELDS) return -1;
   if (!field_sizes(T, d, E, k, f, cf, sz) || !fp8_field_sizes(T, d, E, k, f, cf, sz8)) return -1;
   size_t off = 0;
@@ -285,7 +298,7 @@ int moe_expert_gate_up(const void* x_perm, const int32_t* offsets, int64_t E, in
   cudaError_t err = launch_gate_up(
       static_cast<const __nv_bfloat16*>(x_perm), offsets, (int)E, (int)d, (int)f, (int)max_rows,
       static_cast<const __nv_bfloat16*>(w_gate), static_cast<const __nv_bfloat16*>(w_up),
-      static_cast<__nv_bfloat16*>(h), dev_status, as_stream(stream), &map_failed);
+      static_cast<__nv_bfloat16*>(h), dev_status, as_stream(stream), &map_failed, FuseArgs{});
   if (map_failed) return MOE_ERR_CUDA;
   return cuda_status(err);
 }
@@ -301,8 +314,7 @@ int moe_expert_down(const void* h, const int32_t* offsets, int64_t E, int64_t d,
   bool map_failed = false;
   cudaError_t err = launch_down(static_cast<const __nv_bfloat16*>(h), offsets, (int)E, (int)d,
                                 (int)f, (int)max_rows, static_cast<const __nv_bfloat16*>(w_down),
-                                y_perm, dev_status,
-                                as_stream(stream), &map_failed);
+                                y_perm, dev_status, as_stream(stream), &map_failed, FuseArgs{});
   if (map_failed) return MOE_ERR_CUDA;
   return cuda_status(err);
 }
@@ -399,7 +411,7 @@ int moe_permute_fp8(const uint8_t* xq, const float* sx, const int32_t* topk_idx,
   return cuda_status(moe::launch_permute_rows(xq, (int)d, sx, topk_idx, (int)T, (int)E, (int)k, C,
                                               counts, offsets, slot, row_src, xq_perm, sx_perm,
                                               n_dropped, static_cast<int32_t*>(ws),
-                                              as_stream(stream)));
+                                              as_stream(stream), nullptr, nullptr, 0));
 }
 
 int moe_expert_gate_up_fp8(const uint8_t* xq, const float* sx, const int32_t* offsets, int64_t E,
@@ -417,7 +429,7 @@ int moe_expert_gate_up_fp8(const uint8_t* xq, const float* sx, const int32_t* of
   bool map_failed = false;
   cudaError_t err = moe::launch_gate_up_e4m3(
       xq, sx, offsets, (int)E, (int)d, (int)f, (int)max_rows, wq_gate, s_gate, wq_up, s_up,
-      static_cast<__nv_bfloat16*>(h), dev_status, as_stream(stream), &map_failed);
+      static_cast<__nv_bfloat16*>(h), dev_status, as_stream(stream), &map_failed, FuseArgs{});
   if (map_failed) return MOE_ERR_CUDA;
   return cuda_status(err);
 }
@@ -434,7 +446,7 @@ int moe_expert_down_fp8(const uint8_t* hq, const float* sh, const int32_t* offse
   bool map_failed = false;
   cudaError_t err = moe::launch_down_e4m3(hq, sh, offsets, (int)E, (int)d, (int)f, (int)max_rows,
                                           wq_down, s_down, y_perm, dev_status, as_stream(stream),
-                                          &map_failed);
+                                          &map_failed, FuseArgs{});
   if (map_failed) return MOE_ERR_CUDA;
   return cuda_status(err);
 }
@@ -495,6 +507,143 @@ int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bia
                                 status, stream)) != MOE_OK)
     return st;
   return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
+}
+
+// ---------------------------------------------------------------- fused path
+int moe_permute_fused(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
+                      int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
+                      int32_t* row_src, int32_t* row_pair, void* x_perm, int32_t* n_dropped,
+                      float* y32, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_routing_shape(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_width(d)) != MOE_OK) return st;
+  const int64_t C = moe_capacity(T, E, k, cf);
+  if (C < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!topk_idx || !counts || !offsets || !slot || !row_src || !row_pair || !n_dropped || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws) || (y32 && !aligned16(y32)) || (x && (!aligned16(x) || !aligned16(x_perm))))
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_permute_workspace_size(T, E, k)) return MOE_ERR_WORKSPACE;
+  return cuda_status(moe::launch_permute_rows(
+      static_cast<const uint8_t*>(x), (int)d * 2, nullptr, topk_idx, (int)T, (int)E, (int)k, C,
+      counts, offsets, slot, row_src, static_cast<uint8_t*>(x_perm), nullptr, n_dropped,
+      static_cast<int32_t*>(ws), as_stream(stream), row_pair, y32, y32 ? (int)d : 0));
+}
+
+int moe_expert_gate_up_gather(const void* x, int64_t T, const int32_t* row_src,
+                              const int32_t* offsets, int64_t E, int64_t d, int64_t f,
+                              int64_t max_rows, const void* w_gate, const void* w_up, void* h,
+                              int32_t* dev_status, void* stream) {
+  int st = check_gemm_args(E, d, f, max_rows);
+  if (st != MOE_OK) return st;
+  if (T < 1 || T >= (int64_t(1) << 31) - 1) return MOE_ERR_INVALID_ARG;
+  if (max_rows == 0) return MOE_OK;
+  if (!x || !row_src || !offsets || !w_gate || !w_up || !h) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(h))
+    return MOE_ERR_INVALID_ARG;
+  FuseArgs fz{};
+  fz.row_src = row_src;
+  fz.n_tok = (int)T;
+  bool map_failed = false;
+  cudaError_t err = launch_gate_up(
+      static_cast<const __nv_bfloat16*>(x), offsets, (int)E, (int)d, (int)f, (int)max_rows,
+      static_cast<const __nv_bfloat16*>(w_gate), static_cast<const __nv_bfloat16*>(w_up),
+      static_cast<__nv_bfloat16*>(h), dev_status, as_stream(stream), &map_failed, fz);
+  if (map_failed) return MOE_ERR_CUDA;
+  return cuda_status(err);
+}
+
+int moe_expert_down_scatter(const void* h, const int32_t* offsets, int64_t E, int64_t d,
+                            int64_t f, int64_t max_rows, const void* w_down,
+                            const int32_t* row_pair, const float* topk_w, int64_t k, float* y32,
+                            int32_t* dev_status, void* stream) {
+  int st = check_gemm_args(E, d, f, max_rows);
+  if (st != MOE_OK) return st;
+  if (k < 1 || k > kMaxK) return MOE_ERR_INVALID_ARG;
+  if (max_rows == 0) return MOE_OK;
+  if (!h || !offsets || !w_down || !row_pair || !topk_w || !y32) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_down) || !aligned16(y32)) return MOE_ERR_INVALID_ARG;
+  FuseArgs fz{};
+  fz.row_pair = row_pair;
+  fz.topk_w = topk_w;
+  fz.k = (int)k;
+  fz.y32 = y32;
+  bool map_failed = false;
+  cudaError_t err = launch_down(static_cast<const __nv_bfloat16*>(h), offsets, (int)E, (int)d,
+                                (int)f, (int)max_rows, static_cast<const __nv_bfloat16*>(w_down),
+                                nullptr, dev_status, as_stream(stream), &map_failed, fz);
+  if (map_failed) return MOE_ERR_CUDA;
+  return cuda_status(err);
+}
+
+int moe_combine_finalize(const float* y32, const void* x, const int32_t* slot, int64_t T,
+                         int64_t d, int64_t k, void* y, void* stream) {
+  if (T < 0 || k < 1 || k > kMaxK || T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  int st = check_width(d);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!y32 || !x || !slot || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y32) || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_finalize(y32, static_cast<const __nv_bfloat16*>(x), slot,
+                                          (int)T, (int)d, (int)k,
+                                          static_cast<__nv_bfloat16*>(y), as_stream(stream)));
+}
+
+size_t moe_workspace_size_fused(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                                double cf) {
+  const size_t base = moe_workspace_size(T, d, E, k, f, cf);
+  const int64_t rows = moe_max_rows(T, E, k, cf);
+  if (base == 0 || rows < 0) return 0;
+  return base + align256(size_t(rows) * sizeof(int32_t)) + align256(size_t(T * d) * sizeof(float));
+}
+
+int moe_layer_forward_fused(const void* x, const float* w_router, const float* bias,
+                            const void* w_gate, const void* w_up, const void* w_down, int64_t T,
+                            int64_t d, int64_t E, int64_t k, int64_t f, double cf, void* y,
+                            void* ws, size_t ws_bytes, void* stream) {
+  int st = check_routing_shape(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_width(d)) != MOE_OK) return st;
+  if ((st = check_width(f)) != MOE_OK) return st;
+  if (moe_capacity(T, E, k, cf) < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !w_gate || !w_up || !w_down || !y || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_workspace_size_fused(T, d, E, k, f, cf)) return MOE_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  auto field = [&](int id) { return base + moe_workspace_field_offset(id, T, d, E, k, f, cf); };
+  int32_t* status = reinterpret_cast<int32_t*>(field(MOE_WS_STATUS));
+  float* logits = reinterpret_cast<float*>(field(MOE_WS_LOGITS));
+  int32_t* topk_idx = reinterpret_cast<int32_t*>(field(MOE_WS_TOPK_IDX));
+  float* topk_w = reinterpret_cast<float*>(field(MOE_WS_TOPK_W));
+  int32_t* slot = reinterpret_cast<int32_t*>(field(MOE_WS_SLOT));
+  int32_t* counts = reinterpret_cast<int32_t*>(field(MOE_WS_COUNTS));
+  int32_t* offsets = reinterpret_cast<int32_t*>(field(MOE_WS_OFFSETS));
+  int32_t* n_dropped = reinterpret_cast<int32_t*>(field(MOE_WS_N_DROPPED));
+  int32_t* row_src = reinterpret_cast<int32_t*>(field(MOE_WS_ROW_SRC));
+  void* x_perm = field(MOE_WS_X_PERM);
+  void* h = field(MOE_WS_H);
+  int32_t* row_pair = reinterpret_cast<int32_t*>(field(MOE_WS_ROW_PAIR));
+  float* y32 = reinterpret_cast<float*>(field(MOE_WS_Y32));
+  const int64_t max_rows = moe_max_rows(T, E, k, cf);
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, field(MOE_WS_ROUTE),
+                      moe_route_workspace_size(T, d, E, k), status, stream)) != MOE_OK)
+    return st;
+  if ((st = moe_permute_fused(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src,
+                              row_pair, x_perm, n_dropped, y32, field(MOE_WS_PERMUTE),
+                              moe_permute_workspace_size(T, E, k), stream)) != MOE_OK)
+    return st;
+  if ((st = moe_expert_gate_up(x_perm, offsets, E, d, f, max_rows, w_gate, w_up, h, status,
+                               stream)) != MOE_OK)
+    return st;
+  if ((st = moe_expert_down_scatter(h, offsets, E, d, f, max_rows, w_down, row_pair, topk_w, k,
+                                    y32, status, stream)) != MOE_OK)
+    return st;
+  return moe_combine_finalize(y32, x, slot, T, d, k, y, stream);
 }
 
 int moe_layer_forward(const void* x, const float* w_router, const float* bias, const void* w_gate,

@@ -107,4 +107,36 @@ cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
   return cudaGetLastError();
 }
 
+// Fused-combine finish: the down GEMM has added w * (expert output) of every
+// kept pair into y32[t] (fp32); y[t] = bf16(y32[t]), or x[t] when all of the
+// token's pairs were dropped.  One warp per token, 16-byte vectors.
+__global__ void __launch_bounds__(256)
+    finalize_kernel(const float* __restrict__ y32, const __nv_bfloat16* __restrict__ x,
+                    const int32_t* __restrict__ slot, int T, int d, int k,
+                    __nv_bfloat16* __restrict__ y) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  const int kept = __any_sync(0xffffffffu, lane < k && slot[(size_t)t * k + lane] >= 0);
+  uint4* dst = reinterpret_cast<uint4*>(y + (size_t)t * d);
+  const int nvec = d / 8;
+  if (!kept) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    return;
+  }
+  const float4* src = reinterpret_cast<const float4*>(y32 + (size_t)t * d);
+  for (int v = lane; v < nvec; v += 32) {
+    const float4 a = __ldg(src + 2 * v), b = __ldg(src + 2 * v + 1);
+    dst[v] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                        pack_bf16x2(b.z, b.w));
+  }
+}
+
+cudaError_t launch_finalize(const float* y32, const __nv_bfloat16* x, const int32_t* slot, int T,
+                            int d, int k, __nv_bfloat16* y, cudaStream_t s) {
+  finalize_kernel<<<(T + 7) / 8, 256, 0, s>>>(y32, x, slot, T, d, k, y);
+  return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -101,6 +101,20 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Four rows r0..r3 (any rows, any order) of a 2-D tensor, from inner
+// coordinate c0 on, into four consecutive box rows at dst (tile::gather4; the
+// tensor map's box is one row high).  Rows outside the tensor read zeros.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t r0, int32_t r1, int32_t r2,
+                                            int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -252,6 +266,17 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// tile::gather4 for a CTA pair: completes on the leader CTA's barrier.
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int32_t c0, int32_t r0,
+                                                 int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst_smem)),
@@ -297,6 +322,22 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
   while (global_timer_ns() - t0 < ns) {
   }
 }
+
+// Fusions with the neighbouring steps (all pointers null: plain GEMMs).
+//  * gather (GEMM 1): A rows come straight from the token rows, row r of
+//    bucket storage being token row_src[r] (tile::gather4, 4 rows per copy),
+//    so the permutation writes no copy of the rows;
+//  * scatter (GEMM 2): instead of storing y_perm row r, the epilogue adds
+//    w * row into y32[t] (fp32, red.global.add), where row_pair[r] = t*k + j
+//    and w = topk_w[t*k + j], so the combine reads no y_perm.
+struct FuseArgs {
+  const int32_t* row_src;
+  int n_tok;                  // token rows (an index >= n_tok reads a zero row)
+  const int32_t* row_pair;
+  const float* topk_w;
+  int k;
+  float* y32;
+};
 
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -65,6 +65,32 @@ __device__ __forceinline__ void store_chunk_f32(const uint32_t (&v)[32], uint32_
   __syncwarp();
 }
 
+// fp32 scatter-add (the fused combine): row `lane` holds v[0..31] of a
+// permuted row whose token is my_t and gate weight my_w; for the warp's valid
+// rows, y32_col0[t * ld + c] += w * v[c].  Staged through the padded tile so
+// that each instruction covers four rows with one 16-byte vector add per lane
+// (8 lanes per row, 32 consecutive columns).
+__device__ __forceinline__ void scatter_chunk_f32(const uint32_t (&v)[32], uint32_t* stage,
+                                                  float* y32_col0, size_t ld, int my_t,
+                                                  float my_w, int nvalid, int lane) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) stage[lane * 33 + j] = v[j];
+  __syncwarp();
+  const int c = (lane % 8) * 4;
+  for (int r0 = 0; r0 < nvalid; r0 += 4) {
+    const int r = r0 + lane / 8;
+    const int t = __shfl_sync(0xffffffffu, my_t, r);
+    const float w = __shfl_sync(0xffffffffu, my_w, r);
+    if (r < nvalid) {
+      const uint32_t* src = stage + r * 33 + c;
+      const float4 add = make_float4(w * __uint_as_float(src[0]), w * __uint_as_float(src[1]),
+                                     w * __uint_as_float(src[2]), w * __uint_as_float(src[3]));
+      atomicAdd(reinterpret_cast<float4*>(y32_col0 + (size_t)t * ld + c), add);
+    }
+  }
+  __syncwarp();
+}
+
 // bf16: row `lane` holds pk[0..15] (32 bf16), stored directly as four
 // 16-byte vectors (the SwiGLU tile is a quarter of the fp32 one's bytes and
 // measured faster without staging).
@@ -203,6 +229,61 @@ __device__ __forceinline__ void gemm_setup(GemmShared& sh, int stages, int full_
   }
 }
 
+// Gathering TMA producer (all 32 lanes of warp 0): lane L copies rows
+// 4L .. 4L+3 of each A tile from the token rows with one tile::gather4 per
+// k-block; rows past the bucket read the zero row n_tok.  Lane 0 waits, arms
+// the stage barrier and loads B.
+template <int STAGES, int STAGE_BYTES, int A_BYTES, int B_BYTES, class LoadB>
+__device__ __forceinline__ void producer_role_gather(GemmShared& sh, uint8_t* smem,
+                                                     const CUtensorMap* tmX, const FuseArgs& fz,
+                                                     int E, int n_tiles, int nkb, int32_t* status,
+                                                     LoadB load_b, int kb_elems, int lane) {
+  volatile int* abort_flag = &sh.abort_flag;
+  const int total_tiles = sh.tile_prefix[E];
+  int it = 0;
+  int last_it[8];
+  for (int s = 0; s < STAGES; ++s) last_it[s] = -1;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+    int e, m, n;
+    decode_tile(sh, tile, E, n_tiles, e, m, n);
+    const int left = sh.row_cnt[e] - m * kBM;
+    const bool small = left <= kBM / 2;   // M = 64 tile
+    const int nrows = small ? kBM / 2 : kBM;
+    int idx[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rr = 4 * lane + i;
+      idx[i] = (rr < nrows && rr < left) ? fz.row_src[sh.row_off[e] + m * kBM + rr] : fz.n_tok;
+    }
+    for (int kb = 0; kb < nkb; ++kb, ++it) {
+      const int s = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      bool good = true;
+      if (lane == 0) good = mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag);
+      if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
+      uint8_t* sa = smem + s * STAGE_BYTES;
+      const uint32_t a_bytes = small ? A_BYTES / 2 : A_BYTES;
+      if (lane == 0) mbar_arrive_expect_tx(&sh.full_bar[s], a_bytes + B_BYTES);
+      __syncwarp();
+      if (4 * lane < nrows)
+        tma_gather4(sa + 4 * lane * 128, tmX, &sh.full_bar[s], kb * kb_elems, idx[0], idx[1],
+                    idx[2], idx[3]);
+      if (lane == 0) load_b(sa + A_BYTES, &sh.full_bar[s], e, n, kb);
+      last_it[s] = it;
+    }
+  }
+  if (lane == 0) {
+    if (!ok) {
+      *abort_flag = 1;
+      report(status, kDevErrWaitTimeout);
+    }
+    // never leave with copies in flight: every stage's last fill must land
+    for (int s = 0; s < STAGES; ++s)
+      if (last_it[s] >= 0) mbar_wait(&sh.full_bar[s], (last_it[s] / STAGES) & 1, &sh.never);
+  }
+}
+
 // TMA producer (one thread): per k-block the A tile (128 or, for a bucket's
 // last <= 64 rows, 64 rows) and, through load_b(stage B buffer, bar, e, n,
 // kb), the weight tile.
@@ -310,7 +391,7 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
                                               int lane, int E, int n_tiles, int n_out,
                                               void* out_raw, const float* row_scale,
                                               const float* sc0, const float* sc1,
-                                              int32_t* status) {
+                                              const FuseArgs& fz, int32_t* status) {
   constexpr int kOutCols = SWIGLU ? BN / 2 : BN;
   volatile int* abort_flag = &sh.abort_flag;
   const int total_tiles = sh.tile_prefix[E];
@@ -356,6 +437,24 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
         swiglu_pack(g, u, pk);
         store_chunk_bf16(pk, o + c * 32, n_out, nvalid, lane);
       }
+    } else if (fz.y32) {
+      // fused combine: weighted rows added into the token accumulator
+      int my_t = 0;
+      float my_w = 0.f;
+      if (lane < nvalid) {
+        const int p = fz.row_pair[row0 + lane];
+        my_t = p / fz.k;
+        my_w = fz.topk_w[p];
+      }
+      float* o = fz.y32 + (size_t)n * kOutCols;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + c * 32, v);
+        tmem_ld_wait();
+        if (SCALED) apply_scales(v, sc0 + sc_off + c * 32, sr);
+        scatter_chunk_f32(v, stage, o + c * 32, n_out, my_t, my_w, nvalid, lane);
+      }
     } else {
       float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * kOutCols;
 #pragma unroll 1
@@ -381,7 +480,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1,
                         const int32_t* __restrict__ offsets, int E, int K, int n_out,
-                        int max_rows, void* __restrict__ out_raw, int32_t* status) {
+                        int max_rows, void* __restrict__ out_raw, int32_t* status,
+                        const FuseArgs fz) {
   using Cfg = GemmCfg<BN, SWIGLU>;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ GemmShared sh;
@@ -405,26 +505,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
 
   if (warp == 0) {
-    if (lane == 0) {
-      auto load_b = [&](uint8_t* sb, uint64_t* bar, int e, int n, int kb) {
-        const int col0 = n * Cfg::kOutCols;
-        if (SWIGLU) {
+    auto load_b = [&](uint8_t* sb, uint64_t* bar, int e, int n, int kb) {
+      const int col0 = n * Cfg::kOutCols;
+      if (SWIGLU) {
 #pragma unroll
-          for (int c = 0; c < BN / 128; ++c)
-            tma_load_3d(sb + c * kChunkBytes, &tmB0, bar, col0 + c * 64, kb * kBK, e);
+        for (int c = 0; c < BN / 128; ++c)
+          tma_load_3d(sb + c * kChunkBytes, &tmB0, bar, col0 + c * 64, kb * kBK, e);
 #pragma unroll
-          for (int c = 0; c < BN / 128; ++c)
-            tma_load_3d(sb + (BN / 128 + c) * kChunkBytes, &tmB1, bar, col0 + c * 64, kb * kBK,
-                        e);
-        } else {
+        for (int c = 0; c < BN / 128; ++c)
+          tma_load_3d(sb + (BN / 128 + c) * kChunkBytes, &tmB1, bar, col0 + c * 64, kb * kBK, e);
+      } else {
 #pragma unroll
-          for (int c = 0; c < BN / 64; ++c)
-            tma_load_3d(sb + c * kChunkBytes, &tmB0, bar, col0 + c * 64, kb * kBK, e);
-        }
-      };
+        for (int c = 0; c < BN / 64; ++c)
+          tma_load_3d(sb + c * kChunkBytes, &tmB0, bar, col0 + c * 64, kb * kBK, e);
+      }
+    };
+    if (fz.row_src)      // A rows gathered from the token rows (tmA maps those)
+      producer_role_gather<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
+          sh, smem, &tmA, fz, E, n_tiles, nkb, status, load_b, kBK, lane);
+    else if (lane == 0)
       producer_role<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
           sh, smem, &tmA, &tmA64, E, n_tiles, nkb, status, load_b);
-    }
   } else if (warp == 1) {
     if (lane == 0)
       mma_role<BN, Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes>(sh, smem, E, n_tiles, nkb,
@@ -432,7 +533,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                                  status);
   } else {
     epilogue_role<BN, SWIGLU, false>(sh, smem + Cfg::kStagingOff, warp, lane, E, n_tiles, n_out,
-                                     out_raw, nullptr, nullptr, nullptr, status);
+                                     out_raw, nullptr, nullptr, nullptr, fz, status);
   }
 
   tc_fence_before();
@@ -475,7 +576,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              const float* __restrict__ col_scale0,
                              const float* __restrict__ col_scale1,
                              const int32_t* __restrict__ offsets, int E, int K, int n_out,
-                             int max_rows, void* __restrict__ out_raw, int32_t* status) {
+                             int max_rows, void* __restrict__ out_raw, int32_t* status,
+                             const FuseArgs fz) {
   using Cfg = E4m3Cfg<BN, SWIGLU>;
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ GemmShared sh;
@@ -499,29 +601,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
 
   if (warp == 0) {
-    if (lane == 0) {
-      // B: 128 weight rows (output columns) x 128 K per copy
-      auto load_b = [&](uint8_t* sb, uint64_t* bar, int e, int n, int kb) {
-        const int col0 = n * Cfg::kOutCols;
-        if (SWIGLU) {
-          tma_load_3d(sb, &tmB0, bar, kb * Cfg::kBKe, col0, e);
-          tma_load_3d(sb + 128 * Cfg::kBKe, &tmB1, bar, kb * Cfg::kBKe, col0, e);
-        } else {
+    // B: 128 weight rows (output columns) x 128 K per copy
+    auto load_b = [&](uint8_t* sb, uint64_t* bar, int e, int n, int kb) {
+      const int col0 = n * Cfg::kOutCols;
+      if (SWIGLU) {
+        tma_load_3d(sb, &tmB0, bar, kb * Cfg::kBKe, col0, e);
+        tma_load_3d(sb + 128 * Cfg::kBKe, &tmB1, bar, kb * Cfg::kBKe, col0, e);
+      } else {
 #pragma unroll
-          for (int c = 0; c < BN / 128; ++c)
-            tma_load_3d(sb + c * 128 * Cfg::kBKe, &tmB0, bar, kb * Cfg::kBKe, col0 + c * 128, e);
-        }
-      };
+        for (int c = 0; c < BN / 128; ++c)
+          tma_load_3d(sb + c * 128 * Cfg::kBKe, &tmB0, bar, kb * Cfg::kBKe, col0 + c * 128, e);
+      }
+    };
+    if (fz.row_src)
+      producer_role_gather<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
+          sh, smem, &tmA, fz, E, n_tiles, nkb, status, load_b, Cfg::kBKe, lane);
+    else if (lane == 0)
       producer_role<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
           sh, smem, &tmA, &tmA64, E, n_tiles, nkb, status, load_b, Cfg::kBKe);
-    }
   } else if (warp == 1) {
     if (lane == 0)
       mma_role<BN, Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, true>(
           sh, smem, E, n_tiles, nkb, Cfg::kIdesc, Cfg::kIdesc64, status);
   } else {
     epilogue_role<BN, SWIGLU, true>(sh, smem + Cfg::kStagingOff, warp, lane, E, n_tiles, n_out,
-                                    out_raw, row_scale, col_scale0, col_scale1, status);
+                                    out_raw, row_scale, col_scale0, col_scale1, fz, status);
   }
 
   tc_fence_before();
@@ -582,6 +686,18 @@ __device__ __forceinline__ void f32_chunk_store(uint32_t t, uint32_t* stage, flo
   store_chunk_f32(v, stage, out_row0, ld, nvalid, lane);
 }
 
+template <bool SCALED>
+__device__ __forceinline__ void f32_chunk_scatter(uint32_t t, uint32_t* stage, float* y32_col0,
+                                                  size_t ld, int nvalid, int lane,
+                                                  const float* sc, float sr, int my_t,
+                                                  float my_w) {
+  uint32_t v[32];
+  tmem_ld_32x32b_x32(t, v);
+  tmem_ld_wait();
+  if (SCALED) apply_scales(v, sc, sr);
+  scatter_chunk_f32(v, stage, y32_col0, ld, my_t, my_w, nvalid, lane);
+}
+
 constexpr int kPairStages = 6;
 constexpr int kPairStageBytes = 2 * kBM * kBK * 2;      // A 16 KB + half of B 16 KB
 constexpr int kPairStagingOff = kPairStages * kPairStageBytes;
@@ -629,7 +745,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              const float* __restrict__ col_scale0,
                              const float* __restrict__ col_scale1,
                              const int32_t* __restrict__ offsets, int E, int K, int n_out,
-                             int max_rows, void* __restrict__ out_raw, int32_t* status) {
+                             int max_rows, void* __restrict__ out_raw, int32_t* status,
+                             const FuseArgs fz) {
   constexpr int kOutCols = SWIGLU ? 128 : 256;        // output columns per pair tile
   constexpr int kPairM = 2 * kBM;
   constexpr int kKb = E4M3 ? 128 : kBK;               // K values per k-block (128 bytes)
@@ -718,7 +835,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   };
 
   if (warp == 0) {
-    if (lane == 0) {
+    // A rows gathered from the token rows (all 32 lanes issue tile::gather4),
+    // else one thread loads the permuted rows' tile
+    const bool gather = fz.row_src != nullptr;
+    if (gather || lane == 0) {
       // ------------------------------------------------ TMA producer (both CTAs)
       int it = 0;
       int last_it[kPairStages];
@@ -728,58 +848,81 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int e, m, n;
         decode_pair_tile(sh, tile, E, n_tiles, e, m, n);
         const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
-        const int row0 = sh.row_off[e] + m * kPairM + (int)rank * (half ? kBM / 2 : kBM);
+        const int mrow = m * kPairM + (int)rank * (half ? kBM / 2 : kBM);  // in the bucket
+        const int row0 = sh.row_off[e] + mrow;
         const int col0 = n * kOutCols;
+        const int nrows = half ? kBM / 2 : kBM;
+        int idx[4] = {0, 0, 0, 0};
+        if (gather) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int rr = 4 * lane + i;
+            idx[i] = (rr < nrows && mrow + rr < sh.row_cnt[e]) ? fz.row_src[row0 + rr] : fz.n_tok;
+          }
+        }
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kPairStages;
           const uint32_t ph = (it / kPairStages) & 1;
-          if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
+          bool good = true;
+          if (lane == 0) good = mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag);
+          if (gather) good = __shfl_sync(0xffffffffu, good, 0);
+          if (!good) { ok = false; break; }
           uint8_t* sa = smem + s * kPairStageBytes;
           uint8_t* sb = sa + kBM * kBK * 2;
           const uint32_t full_lead = mapa_shared(&sh.full_bar[s], 0);
           // a half tile reads 64 rows of A per CTA (8 KB instead of 16 KB)
-          if (leader)
+          if (leader && lane == 0)
             mbar_arrive_expect_tx(&sh.full_bar[s],
                                   half ? 2 * (kPairStageBytes - kBM * kBK) : 2 * kPairStageBytes);
-          if (half)
+          if (gather) {
+            __syncwarp();
+            if (4 * lane < nrows)
+              tma_gather4_pair(sa + 4 * lane * 128, &tmA, full_lead, kb * kKb, idx[0], idx[1],
+                               idx[2], idx[3]);
+          } else if (half) {
             tma_load_2d_pair(sa, &tmA64, full_lead, kb * kKb, row0);
-          else
-            tma_load_2d_pair(sa, &tmA, full_lead, kb * kKb, row0);
-          if (E4M3) {
-            // K-major weights: 128 rows (output columns) of 128 K bytes per CTA
-            const int k0 = kb * kKb;
-            if (SWIGLU && half) {
-              tma_load_3d_pair(sb, &tmB0h, full_lead, k0, col0 + (int)rank * 64, e);
-              tma_load_3d_pair(sb + 64 * 128, &tmB1h, full_lead, k0, col0 + (int)rank * 64, e);
-            } else if (SWIGLU) {
-              tma_load_3d_pair(sb, leader ? &tmB0 : &tmB1, full_lead, k0, col0, e);
-            } else {
-              tma_load_3d_pair(sb, &tmB0, full_lead, k0, col0 + (int)rank * 128, e);
-            }
-          } else if (SWIGLU && half) {
-            tma_load_3d_pair(sb, &tmB0, full_lead, col0 + (int)rank * 64, kb * kBK, e);
-            tma_load_3d_pair(sb + kChunkBytes, &tmB1, full_lead, col0 + (int)rank * 64, kb * kBK,
-                             e);
-          } else if (SWIGLU) {
-            const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-              tma_load_3d_pair(sb + c * kChunkBytes, mb, full_lead, col0 + c * 64, kb * kBK, e);
           } else {
+            tma_load_2d_pair(sa, &tmA, full_lead, kb * kKb, row0);
+          }
+          if (lane == 0) {
+            if (E4M3) {
+              // K-major weights: 128 rows (output columns) of 128 K bytes per CTA
+              const int k0 = kb * kKb;
+              if (SWIGLU && half) {
+                tma_load_3d_pair(sb, &tmB0h, full_lead, k0, col0 + (int)rank * 64, e);
+                tma_load_3d_pair(sb + 64 * 128, &tmB1h, full_lead, k0, col0 + (int)rank * 64, e);
+              } else if (SWIGLU) {
+                tma_load_3d_pair(sb, leader ? &tmB0 : &tmB1, full_lead, k0, col0, e);
+              } else {
+                tma_load_3d_pair(sb, &tmB0, full_lead, k0, col0 + (int)rank * 128, e);
+              }
+            } else if (SWIGLU && half) {
+              tma_load_3d_pair(sb, &tmB0, full_lead, col0 + (int)rank * 64, kb * kBK, e);
+              tma_load_3d_pair(sb + kChunkBytes, &tmB1, full_lead, col0 + (int)rank * 64,
+                               kb * kBK, e);
+            } else if (SWIGLU) {
+              const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-              tma_load_3d_pair(sb + c * kChunkBytes, &tmB0, full_lead,
-                               col0 + (int)rank * 128 + c * 64, kb * kBK, e);
+              for (int c = 0; c < 2; ++c)
+                tma_load_3d_pair(sb + c * kChunkBytes, mb, full_lead, col0 + c * 64, kb * kBK, e);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 2; ++c)
+                tma_load_3d_pair(sb + c * kChunkBytes, &tmB0, full_lead,
+                                 col0 + (int)rank * 128 + c * 64, kb * kBK, e);
+            }
           }
           last_it[s] = it;
         }
       }
-      if (!ok) give_up();
-      if (leader) {
-        // both CTAs' copies of every issued phase count on the leader's barriers
-        for (int s = 0; s < kPairStages; ++s)
-          if (last_it[s] >= 0)
-            mbar_wait(&sh.full_bar[s], (last_it[s] / kPairStages) & 1, &sh.never);
+      if (lane == 0) {
+        if (!ok) give_up();
+        if (leader) {
+          // both CTAs' copies of every issued phase count on the leader's barriers
+          for (int s = 0; s < kPairStages; ++s)
+            if (last_it[s] >= 0)
+              mbar_wait(&sh.full_bar[s], (last_it[s] / kPairStages) & 1, &sh.never);
+        }
       }
     }
   } else if (warp == 1) {
@@ -857,6 +1000,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int c = 0; c < 4; ++c)
             swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 128 + c * 32, o + c * 32, n_out,
                                      nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
+        } else if (fz.y32) {
+          const int c0 = n * kOutCols;
+          int my_t = 0;
+          float my_w = 0.f;
+          if (lane < nvalid) {
+            const int p = fz.row_pair[row0 + lane];
+            my_t = p / fz.k;
+            my_w = fz.topk_w[p];
+          }
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c)
+            f32_chunk_scatter<E4M3>(tbase + c * 32, stage, fz.y32 + c0 + c * 32, n_out, nvalid,
+                                    lane, cs0 + c0 + c * 32, sr, my_t, my_w);
         } else {
           const int c0 = n * kOutCols;
           float* o = static_cast<float*>(out_raw) + row0 * n_out + c0;
@@ -882,6 +1038,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int c = 0; c < 2; ++c)
             swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 64 + c * 32, o + c * 32, n_out,
                                      nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
+        } else if (fz.y32) {
+          const int c0 = n * kOutCols + hh * 128;
+          int my_t = 0;
+          float my_w = 0.f;
+          if (lane < nvalid) {
+            const int p = fz.row_pair[row0 + lane];
+            my_t = p / fz.k;
+            my_w = fz.topk_w[p];
+          }
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c)
+            f32_chunk_scatter<E4M3>(tbase + c * 32, stage, fz.y32 + c0 + c * 32, n_out, nvalid,
+                                    lane, cs0 + c0 + c * 32, sr, my_t, my_w);
         } else {
           const int c0 = n * kOutCols + hh * 128;
           float* o = static_cast<float*>(out_raw) + row0 * n_out + c0;
@@ -913,7 +1082,7 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
                                const CUtensorMap& b0, const CUtensorMap& b1,
                                const int32_t* offsets, int E, int K,
                                int n_out, int max_rows, void* out, int32_t* status,
-                               cudaStream_t s) {
+                               cudaStream_t s, const FuseArgs& fz) {
   using Cfg = GemmCfg<BN, SWIGLU>;
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
@@ -931,7 +1100,7 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
   int grid = (int)(ub < di->sms ? ub : di->sms);
   if (grid < 1) grid = 1;
   kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, offsets, E, K, n_out,
-                                                     max_rows, out, status);
+                                                     max_rows, out, status, fz);
   return cudaGetLastError();
 }
 
@@ -940,7 +1109,7 @@ static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtens
                                     const CUtensorMap& b0, const CUtensorMap& b1,
                                     const int32_t* offsets, int E, int K, int n_out, int max_rows,
                                     void* out, int32_t* status, cudaStream_t s,
-                                    const CUtensorMap* b0h = nullptr,
+                                    const FuseArgs& fz, const CUtensorMap* b0h = nullptr,
                                     const CUtensorMap* b1h = nullptr,
                                     const float* row_scale = nullptr,
                                     const float* cs0 = nullptr, const float* cs1 = nullptr) {
@@ -973,44 +1142,58 @@ static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtens
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a, a64, b0, b1, b0h ? *b0h : b0, b1h ? *b1h : b1,
-                            row_scale, cs0, cs1, offsets, E, K, n_out, max_rows, out, status);
+                            row_scale, cs0, cs1, offsets, E, K, n_out, max_rows, out, status, fz);
 }
 
 // Pair tiles (256 rows) pay off when buckets are large; the buffer's rows
 // per expert bound the average bucket from above.
 static bool use_pair_tiles(int E, int max_rows) { return max_rows >= 512LL * E; }
 
-// GEMM 1: h = silu(x_perm Wg) * (x_perm Wu)
-cudaError_t launch_gate_up(const __nv_bfloat16* x_perm, const int32_t* offsets, int E, int d,
+// The A operand: the permuted rows [max_rows, K] (128- and 64-row boxes), or,
+// when gathering, the token rows [fz.n_tok, K] (one-row boxes for gather4).
+static bool map_a(CUtensorMap* a, CUtensorMap* a64, const void* rows, int K, int max_rows,
+                  bool e4m3, const FuseArgs& fz) {
+  if (fz.row_src) {
+    *a64 = {};
+    return map_rows_gather(a, rows, K, fz.n_tok, e4m3);
+  }
+  if (e4m3)
+    return map_rows_e4m3(a, rows, K, max_rows, kBM) && map_rows_e4m3(a64, rows, K, max_rows, kBM / 2);
+  return map_rows(a, rows, K, max_rows, kBM) && map_rows(a64, rows, K, max_rows, kBM / 2);
+}
+
+// GEMM 1: h = silu(A Wg) * (A Wu), A = x_perm or (gathering) the token rows
+cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, int E, int d,
                            int f, int max_rows, const __nv_bfloat16* w_gate,
                            const __nv_bfloat16* w_up, __nv_bfloat16* h, int32_t* status,
-                           cudaStream_t s, bool* map_failed) {
+                           cudaStream_t s, bool* map_failed, const FuseArgs& fz) {
   CUtensorMap ta, ta64, tg, tu;
-  *map_failed = !(map_rows(&ta, x_perm, d, max_rows, kBM) &&
-                  map_rows(&ta64, x_perm, d, max_rows, kBM / 2) &&
+  *map_failed = !(map_a(&ta, &ta64, a_rows, d, max_rows, false, fz) &&
                   map_weights(&tg, w_gate, E, d, f) && map_weights(&tu, w_up, E, d, f));
   if (*map_failed) return cudaSuccess;
   if (use_pair_tiles(E, max_rows))
-    return launch_gemm_pair<true>(7, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s);
-  return launch_gemm<256, true>(0, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s);
+    return launch_gemm_pair<true>(7, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s,
+                                  fz);
+  return launch_gemm<256, true>(0, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s,
+                                fz);
 }
 
-// GEMM 2: y_perm = h Wd
+// GEMM 2: y_perm = h Wd, or (scattering) y32[t] += w * (h Wd)
 cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
                         int max_rows, const __nv_bfloat16* w_down, float* y_perm,
-                        int32_t* status, cudaStream_t s, bool* map_failed) {
+                        int32_t* status, cudaStream_t s, bool* map_failed, const FuseArgs& fz) {
   CUtensorMap ta, ta64, td;
   *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_rows(&ta64, h, f, max_rows, kBM / 2) &&
                   map_weights(&td, w_down, E, f, d));
   if (*map_failed) return cudaSuccess;
   if (d % 256 == 0 && use_pair_tiles(E, max_rows))
     return launch_gemm_pair<false>(8, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
-                                   s);
+                                   s, fz);
   if (d % 256 == 0)
     return launch_gemm<256, false>(1, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
-                                   s);
+                                   s, fz);
   return launch_gemm<128, false>(2, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
-                                 s);
+                                 s, fz);
 }
 
 template <int BN, bool SWIGLU>
@@ -1018,7 +1201,8 @@ static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtens
                                     const CUtensorMap& b0, const CUtensorMap& b1,
                                     const float* row_scale, const float* s0, const float* s1,
                                     const int32_t* offsets, int E, int K, int n_out, int max_rows,
-                                    void* out, int32_t* status, cudaStream_t s) {
+                                    void* out, int32_t* status, cudaStream_t s,
+                                    const FuseArgs& fz) {
   using Cfg = E4m3Cfg<BN, SWIGLU>;
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
@@ -1036,20 +1220,19 @@ static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtens
   int grid = (int)(ub < di->sms ? ub : di->sms);
   if (grid < 1) grid = 1;
   kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, row_scale, s0, s1, offsets, E,
-                                                   K, n_out, max_rows, out, status);
+                                                   K, n_out, max_rows, out, status, fz);
   return cudaGetLastError();
 }
 
-// GEMM 1 / GEMM 2 on e4m3 rows (per-row scales) and e4m3 weights stored
-// [E, N, K] (per-column scales); single-CTA tiles
+// GEMM 1 / GEMM 2 on e4m3 rows (per-row scales, indexed by permuted row) and
+// e4m3 weights stored [E, N, K] (per-column scales)
 cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_t* offsets,
                                 int E, int d, int f, int max_rows, const uint8_t* wq_gate,
                                 const float* s_gate, const uint8_t* wq_up, const float* s_up,
                                 __nv_bfloat16* h, int32_t* status, cudaStream_t s,
-                                bool* map_failed) {
+                                bool* map_failed, const FuseArgs& fz) {
   CUtensorMap ta, ta64, tg, tu;
-  *map_failed = !(map_rows_e4m3(&ta, xq, d, max_rows, kBM) &&
-                  map_rows_e4m3(&ta64, xq, d, max_rows, kBM / 2) &&
+  *map_failed = !(map_a(&ta, &ta64, xq, d, max_rows, true, fz) &&
                   map_weights_e4m3(&tg, wq_gate, E, f, d) && map_weights_e4m3(&tu, wq_up, E, f, d));
   if (*map_failed) return cudaSuccess;
   if (use_pair_tiles(E, max_rows)) {
@@ -1058,16 +1241,16 @@ cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_
                     map_weights_e4m3(&tuh, wq_up, E, f, d, 64));
     if (*map_failed) return cudaSuccess;
     return launch_gemm_pair<true, true>(9, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h,
-                                        status, s, &tgh, &tuh, sx, s_gate, s_up);
+                                        status, s, fz, &tgh, &tuh, sx, s_gate, s_up);
   }
   return launch_gemm_e4m3<256, true>(11, ta, ta64, tg, tu, sx, s_gate, s_up, offsets, E, d, f,
-                                     max_rows, h, status, s);
+                                     max_rows, h, status, s, fz);
 }
 
 cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int32_t* offsets,
                              int E, int d, int f, int max_rows, const uint8_t* wq_down,
                              const float* s_down, float* y_perm, int32_t* status, cudaStream_t s,
-                             bool* map_failed) {
+                             bool* map_failed, const FuseArgs& fz) {
   CUtensorMap ta, ta64, td;
   *map_failed = !(map_rows_e4m3(&ta, hq, f, max_rows, kBM) &&
                   map_rows_e4m3(&ta64, hq, f, max_rows, kBM / 2) &&
@@ -1075,12 +1258,12 @@ cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int3
   if (*map_failed) return cudaSuccess;
   if (d % 256 == 0 && use_pair_tiles(E, max_rows))
     return launch_gemm_pair<false, true>(10, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,
-                                         status, s, &td, &td, sh_rows, s_down, nullptr);
+                                         status, s, fz, &td, &td, sh_rows, s_down, nullptr);
   if (d % 256 == 0)
     return launch_gemm_e4m3<256, false>(12, ta, ta64, td, td, sh_rows, s_down, nullptr, offsets,
-                                        E, f, d, max_rows, y_perm, status, s);
+                                        E, f, d, max_rows, y_perm, status, s, fz);
   return launch_gemm_e4m3<128, false>(13, ta, ta64, td, td, sh_rows, s_down, nullptr, offsets, E,
-                                      f, d, max_rows, y_perm, status, s);
+                                      f, d, max_rows, y_perm, status, s, fz);
 }
 
 int device_sm_count() {

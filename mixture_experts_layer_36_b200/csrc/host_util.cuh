@@ -55,6 +55,23 @@ inline bool map_weights(CUtensorMap* m, const void* base, uint64_t E, uint64_t K
          CUDA_SUCCESS;
 }
 
+// 2-D rows [outer, inner] for tile::gather4: box (128 bytes of inner, 1 row),
+// 128-B swizzle (4 gathered rows land as 4 rows of a swizzled K-major tile).
+inline bool map_rows_gather(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                            bool e4m3) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t elem = e4m3 ? 1 : 2;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * elem};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), 1};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D e4m3 codes [outer, inner] row-major, box (128 inner, box_outer), 128-B swizzle.
 inline bool map_rows_e4m3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                           uint32_t box_outer) {

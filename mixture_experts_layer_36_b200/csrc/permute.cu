@@ -99,7 +99,9 @@ __global__ void __launch_bounds__(kScatThreads)
                            int32_t* __restrict__ counts,
                            int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped,
                            int32_t* __restrict__ row_src, uint8_t* __restrict__ x_perm,
-                           float* __restrict__ perm_scale, bool padded) {
+                           float* __restrict__ perm_scale, bool padded,
+                           int32_t* __restrict__ row_pair, float* __restrict__ zero_rows,
+                           int zero_cols) {
   __shared__ int32_t s_off[256];
   __shared__ int32_t s_base[256];
   __shared__ int32_t warp_sum[8];
@@ -170,9 +172,15 @@ __global__ void __launch_bounds__(kScatThreads)
       if (keep) {
         my_row = s_off[e] + sl;
         row_src[my_row] = t;
+        if (row_pair) row_pair[my_row] = t * k + lane;
         if (x_scale) perm_scale[my_row] = x_scale[t];
       }
     }
+    if (zero_rows) {          // the fused combine's fp32 accumulator row of t
+      float4* z = reinterpret_cast<float4*>(zero_rows + (size_t)t * zero_cols);
+      for (int v = lane; v < zero_cols / 4; v += 32) z[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (!x) continue;         // index-only: the GEMM gathers the rows itself
     int rows[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
@@ -221,18 +229,21 @@ __global__ void __launch_bounds__(256)
 }
 
 // Rows of row_bytes bytes (a multiple of 16); x_scale / perm_scale (one fp32
-// per row, moved with it) may be null.
+// per row, moved with it) may be null; x null: no row copy (index-only), with
+// row_pair (t*k + j of each kept row) and zeroed fp32 rows zero_rows[T,
+// zero_cols] for the fused combine when those are non-null.
 cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_scale,
                                 const int32_t* topk_idx, int T, int E, int k, int64_t C,
                                 int32_t* counts, int32_t* offsets, int32_t* slot,
                                 int32_t* row_src, uint8_t* x_perm, float* perm_scale,
-                                int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s) {
+                                int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
+                                int32_t* row_pair, float* zero_rows, int zero_cols) {
   const int nchunks = (T + kChunk - 1) / kChunk;
   permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist);
   const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
   permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
       x, row_bytes, x_scale, topk_idx, slot, chunk_hist, nchunks, T, E, k, C, tpc, counts,
-      offsets, n_dropped, row_src, x_perm, perm_scale, false);
+      offsets, n_dropped, row_src, x_perm, perm_scale, false, row_pair, zero_rows, zero_cols);
   return cudaGetLastError();
 }
 
@@ -248,7 +259,7 @@ cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_id
   uint8_t* xp = reinterpret_cast<uint8_t*>(x_pad);
   permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
       reinterpret_cast<const uint8_t*>(x), d * 2, nullptr, topk_idx, slot, chunk_hist, nchunks, T,
-      E, k, C, tpc, counts, offsets, n_dropped, row_src, xp, nullptr, true);
+      E, k, C, tpc, counts, offsets, n_dropped, row_src, xp, nullptr, true, nullptr, nullptr, 0);
   const int64_t rows = (int64_t)E * C;
   permute_pad_fill_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(counts, E, C, d * 2, row_src,
                                                                      xp);
@@ -262,7 +273,7 @@ cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int 
   return launch_permute_rows(reinterpret_cast<const uint8_t*>(x), d * 2, nullptr, topk_idx, T, E,
                              k, C, counts, offsets, slot, row_src,
                              reinterpret_cast<uint8_t*>(x_perm), nullptr, n_dropped, chunk_hist,
-                             s);
+                             s, nullptr, nullptr, 0);
 }
 
 }  // namespace moe

@@ -77,7 +77,12 @@ def test_workspace_layout(cfg):
     ends8 = offs8[1:] + [total8]
     for i, n in enumerate((rows * d, rows * 4, rows * f, rows * 4, T * d, T * 4)):
         assert ends8[i] - offs8[i] >= n, binding.WS_FIELDS[14 + i]
-    assert moe.moe_workspace_field_offset(20, T, d, E, k, f, cf) == -1
+    # and so do the fused layer's (independently of the FP8 ones)
+    o_pair = moe.moe_workspace_field_offset(20, T, d, E, k, f, cf)
+    o_y32 = moe.moe_workspace_field_offset(21, T, d, E, k, f, cf)
+    assert o_pair == total and o_y32 >= o_pair + rows * 4 and o_y32 % 256 == 0
+    assert moe.moe_workspace_size_fused(T, d, E, k, f, cf) >= o_y32 + T * d * 4
+    assert moe.moe_workspace_field_offset(22, T, d, E, k, f, cf) == -1
     assert moe.moe_workspace_field_offset(-1, T, d, E, k, f, cf) == -1
 
 

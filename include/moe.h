@@ -252,6 +252,23 @@ int moe_permute_padded(const void* x, const int32_t* topk_idx, int64_t T, int64_
                        int32_t* row_src, void* x_pad, int32_t* n_dropped, void* ws,
                        size_t ws_bytes, void* stream);
 
+/* ---- Buckets that are not experts (expert parallelism) ----
+ * With the experts spread over P ranks ("Expert Parallelism & All-to-All"
+ * (neelmishra), sections on dispatch and combine; "Expert Parallelism" guide
+ * (infra.bea.ai), section 2), a rank receives from every source rank q a
+ * fixed-size slot per local expert; bucket b = q * E_w + e holds the rows q
+ * sent to local expert e, of which only the first bucket_rows[b] are real. */
+
+/* moe_expert_mlp over B buckets: bucket b = rows offsets[b] .. offsets[b+1]-1
+ * of x_rows (only the first bucket_rows[b] of them when bucket_rows is
+ * non-null) through expert b % E_w of w_gate/w_up [E_w,d,f], w_down [E_w,f,d];
+ * h bf16 [max_rows,f] and y_rows f32 [max_rows,d] out (rows past
+ * bucket_rows[b] are not written).  B <= 256, B a multiple of E_w. */
+int moe_expert_mlp_buckets(const void* x_rows, const int32_t* offsets, const int32_t* bucket_rows,
+                           int64_t B, int64_t E_w, int64_t d, int64_t f, int64_t max_rows,
+                           const void* w_gate, const void* w_up, const void* w_down, void* h,
+                           float* y_rows, int32_t* dev_status, void* stream);
+
 /* ---- Fused path (an optional variant) ----
  * The combine folded into the down GEMM ("Expert Parallelism" guide
  * (infra.bea.ai), section 5: fuse the gather into the expert GEMM and the

@@ -35,7 +35,7 @@ EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "mo
             "moe_workspace_size_fp8", "moe_layer_forward_fp8", "moe_padded_rows",
             "moe_permute_padded", "moe_permute_fused", "moe_expert_gate_up_gather",
             "moe_expert_down_scatter", "moe_combine_finalize", "moe_workspace_size_fused",
-            "moe_layer_forward_fused"]
+            "moe_layer_forward_fused", "moe_expert_mlp_buckets"]
 
 
 class MoEError(RuntimeError):
@@ -78,6 +78,8 @@ def _load():
         "moe_expert_down_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p]),
         "moe_workspace_size_fp8": (sz, [i64, i64, i64, i64, i64, dbl]),
         "moe_padded_rows": (i64, [i64, i64, i64, dbl]),
+        "moe_expert_mlp_buckets": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, i64, p, p, p, p, p,
+                                                  p, p]),
         "moe_permute_fused": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
                                              p, p, sz, p]),
         "moe_expert_gate_up_gather": (ctypes.c_int, [p, i64, p, p, i64, i64, i64, i64, p, p, p, p,
@@ -340,6 +342,31 @@ def moe_layer_forward(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws
         _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k,
         f, float(cf), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
     return y, ws
+
+
+# ----------------------------------------------------------------- buckets
+
+def moe_expert_mlp_buckets(x_rows, offsets, bucket_rows, w_gate, w_up, w_down, h=None,
+                           y_rows=None, dev_status=None, stream=None):
+    """Grouped SwiGLU MLP over B buckets, bucket b through expert b % E_w,
+    only its first bucket_rows[b] rows.  Returns (h, y_rows)."""
+    rows, d = x_rows.shape
+    B = offsets.shape[0] - 1
+    E_w, _, f = w_gate.shape
+    _want(x_rows, "x_rows", torch.bfloat16)
+    _want(offsets, "offsets", torch.int32, (B + 1,))
+    if bucket_rows is not None:
+        _want(bucket_rows, "bucket_rows", torch.int32, (B,))
+    _want(w_gate, "w_gate", torch.bfloat16, (E_w, d, f))
+    _want(w_up, "w_up", torch.bfloat16, (E_w, d, f))
+    _want(w_down, "w_down", torch.bfloat16, (E_w, f, d))
+    dev = x_rows.device
+    h = torch.empty(rows, f, dtype=torch.bfloat16, device=dev) if h is None else h
+    y_rows = torch.empty(rows, d, dtype=torch.float32, device=dev) if y_rows is None else y_rows
+    _check("moe_expert_mlp_buckets", _lib.moe_expert_mlp_buckets(
+        _ptr(x_rows), _ptr(offsets), _ptr(bucket_rows), B, E_w, d, f, rows, _ptr(w_gate),
+        _ptr(w_up), _ptr(w_down), _ptr(h), _ptr(y_rows), _ptr(dev_status), _stream(stream)))
+    return h, y_rows
 
 
 # ----------------------------------------------------------------- fused path

@@ -509,6 +509,37 @@ int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bia
   return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
 }
 
+// ---------------------------------------------------------------- buckets (expert parallelism)
+int moe_expert_mlp_buckets(const void* x_rows, const int32_t* offsets, const int32_t* bucket_rows,
+                           int64_t B, int64_t E_w, int64_t d, int64_t f, int64_t max_rows,
+                           const void* w_gate, const void* w_up, const void* w_down, void* h,
+                           float* y_rows, int32_t* dev_status, void* stream) {
+  if (E_w < 1 || B % E_w != 0) return MOE_ERR_INVALID_ARG;
+  int st = check_gemm_args(B, d, f, max_rows);
+  if (st != MOE_OK) return st;
+  if (max_rows == 0) return MOE_OK;
+  if (!x_rows || !offsets || !w_gate || !w_up || !w_down || !h || !y_rows)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_rows) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+      !aligned16(h) || !aligned16(y_rows))
+    return MOE_ERR_INVALID_ARG;
+  FuseArgs fz{};
+  fz.bucket_rows = bucket_rows;
+  fz.n_weights = (int)E_w;
+  bool map_failed = false;
+  cudaError_t err = launch_gate_up(
+      static_cast<const __nv_bfloat16*>(x_rows), offsets, (int)B, (int)d, (int)f, (int)max_rows,
+      static_cast<const __nv_bfloat16*>(w_gate), static_cast<const __nv_bfloat16*>(w_up),
+      static_cast<__nv_bfloat16*>(h), dev_status, as_stream(stream), &map_failed, fz);
+  if (map_failed) return MOE_ERR_CUDA;
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  err = launch_down(static_cast<const __nv_bfloat16*>(h), offsets, (int)B, (int)d, (int)f,
+                    (int)max_rows, static_cast<const __nv_bfloat16*>(w_down), y_rows, dev_status,
+                    as_stream(stream), &map_failed, fz);
+  if (map_failed) return MOE_ERR_CUDA;
+  return cuda_status(err);
+}
+
 // ---------------------------------------------------------------- fused path
 int moe_permute_fused(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
                       int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,

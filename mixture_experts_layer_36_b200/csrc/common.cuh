@@ -337,7 +337,16 @@ struct FuseArgs {
   const float* topk_w;
   int k;
   float* y32;
+  // buckets that are not experts (expert parallelism: bucket b holds the rows
+  // one source rank sent to local expert b % n_weights, in a fixed-size slot
+  // of which only the first bucket_rows[b] rows are real)
+  const int32_t* bucket_rows;
+  int n_weights;              // 0: bucket b uses expert b
 };
+
+__host__ __device__ __forceinline__ int weight_index(const FuseArgs& fz, int b) {
+  return fz.n_weights > 0 ? b % fz.n_weights : b;
+}
 
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

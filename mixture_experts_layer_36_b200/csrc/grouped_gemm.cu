@@ -181,7 +181,7 @@ __device__ __forceinline__ void decode_tile(const GemmShared& sh, int tile, int 
 __device__ __forceinline__ void gemm_setup(GemmShared& sh, int stages, int full_count,
                                            int tmem_cols, const int32_t* offsets, int E,
                                            int n_tiles, int max_rows, int32_t* status, int warp,
-                                           int lane) {
+                                           int lane, const FuseArgs& fz) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&sh.full_bar[s], full_count);
@@ -212,6 +212,7 @@ __device__ __forceinline__ void gemm_setup(GemmShared& sh, int stages, int full_
           report(status, kDevErrBadOffsets);
           cnt = 0;
         }
+        if (fz.bucket_rows) cnt = min(cnt, max(0, fz.bucket_rows[e]));
         sh.row_off[e] = o0;
         sh.row_cnt[e] = cnt;
         tiles = cnt > 0 ? ((cnt + kBM - 1) / kBM) * n_tiles : 0;
@@ -269,7 +270,7 @@ __device__ __forceinline__ void producer_role_gather(GemmShared& sh, uint8_t* sm
       if (4 * lane < nrows)
         tma_gather4(sa + 4 * lane * 128, tmX, &sh.full_bar[s], kb * kb_elems, idx[0], idx[1],
                     idx[2], idx[3]);
-      if (lane == 0) load_b(sa + A_BYTES, &sh.full_bar[s], e, n, kb);
+      if (lane == 0) load_b(sa + A_BYTES, &sh.full_bar[s], weight_index(fz, e), n, kb);
       last_it[s] = it;
     }
   }
@@ -291,7 +292,8 @@ template <int STAGES, int STAGE_BYTES, int A_BYTES, int B_BYTES, class LoadB>
 __device__ __forceinline__ void producer_role(GemmShared& sh, uint8_t* smem,
                                               const CUtensorMap* tmA, const CUtensorMap* tmA64,
                                               int E, int n_tiles, int nkb, int32_t* status,
-                                              LoadB load_b, int kb_elems = kBK) {
+                                              LoadB load_b, const FuseArgs& fz,
+                                              int kb_elems = kBK) {
   volatile int* abort_flag = &sh.abort_flag;
   const int total_tiles = sh.tile_prefix[E];
   int it = 0;
@@ -314,7 +316,7 @@ __device__ __forceinline__ void producer_role(GemmShared& sh, uint8_t* smem,
         tma_load_2d(sa, tmA64, &sh.full_bar[s], kb * kb_elems, row0);
       else
         tma_load_2d(sa, tmA, &sh.full_bar[s], kb * kb_elems, row0);
-      load_b(sa + A_BYTES, &sh.full_bar[s], e, n, kb);
+      load_b(sa + A_BYTES, &sh.full_bar[s], weight_index(fz, e), n, kb);
       last_it[s] = it;
     }
   }
@@ -416,7 +418,7 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
     int nvalid = clamp_rows(sh.row_cnt[e] - first);
     if (nvalid > rows_per_warp) nvalid = rows_per_warp;
     const size_t row0 = (size_t)sh.row_off[e] + first;
-    const size_t sc_off = (size_t)e * n_out + (size_t)n * kOutCols;
+    const size_t sc_off = (size_t)weight_index(fz, e) * n_out + (size_t)n * kOutCols;
     const float sr = (SCALED && lane < nvalid) ? row_scale[row0 + lane] : 0.f;
     uint32_t* stage = reinterpret_cast<uint32_t*>(staging) + q * kStageWords;
     const uint32_t tbase =
@@ -493,7 +495,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nkb = K / kBK;
 
   gemm_setup(sh, Cfg::kStages, 1, Cfg::kTmemCols, offsets, E, n_tiles, max_rows, status, warp,
-             lane);
+             lane, fz);
   if (warp == 1 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmA64);
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           sh, smem, &tmA, fz, E, n_tiles, nkb, status, load_b, kBK, lane);
     else if (lane == 0)
       producer_role<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
-          sh, smem, &tmA, &tmA64, E, n_tiles, nkb, status, load_b);
+          sh, smem, &tmA, &tmA64, E, n_tiles, nkb, status, load_b, fz);
   } else if (warp == 1) {
     if (lane == 0)
       mma_role<BN, Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes>(sh, smem, E, n_tiles, nkb,
@@ -589,7 +591,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nkb = K / Cfg::kBKe;
 
   gemm_setup(sh, Cfg::kStages, 1, Cfg::kTmemCols, offsets, E, n_tiles, max_rows, status, warp,
-             lane);
+             lane, fz);
   if (warp == 1 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmA64);
@@ -618,7 +620,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           sh, smem, &tmA, fz, E, n_tiles, nkb, status, load_b, Cfg::kBKe, lane);
     else if (lane == 0)
       producer_role<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
-          sh, smem, &tmA, &tmA64, E, n_tiles, nkb, status, load_b, Cfg::kBKe);
+          sh, smem, &tmA, &tmA64, E, n_tiles, nkb, status, load_b, fz, Cfg::kBKe);
   } else if (warp == 1) {
     if (lane == 0)
       mma_role<BN, Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, true>(
@@ -805,6 +807,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           report(status, kDevErrBadOffsets);
           cnt = 0;
         }
+        if (fz.bucket_rows) cnt = min(cnt, max(0, fz.bucket_rows[e]));
         sh.row_off[e] = o0;
         sh.row_cnt[e] = cnt;
         tiles = cnt > 0 ? ((cnt + kPairM - 1) / kPairM) * n_tiles : 0;
@@ -848,6 +851,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int e, m, n;
         decode_pair_tile(sh, tile, E, n_tiles, e, m, n);
         const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
+        const int ew = weight_index(fz, e);
         const int mrow = m * kPairM + (int)rank * (half ? kBM / 2 : kBM);  // in the bucket
         const int row0 = sh.row_off[e] + mrow;
         const int col0 = n * kOutCols;
@@ -889,27 +893,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               // K-major weights: 128 rows (output columns) of 128 K bytes per CTA
               const int k0 = kb * kKb;
               if (SWIGLU && half) {
-                tma_load_3d_pair(sb, &tmB0h, full_lead, k0, col0 + (int)rank * 64, e);
-                tma_load_3d_pair(sb + 64 * 128, &tmB1h, full_lead, k0, col0 + (int)rank * 64, e);
+                tma_load_3d_pair(sb, &tmB0h, full_lead, k0, col0 + (int)rank * 64, ew);
+                tma_load_3d_pair(sb + 64 * 128, &tmB1h, full_lead, k0, col0 + (int)rank * 64, ew);
               } else if (SWIGLU) {
-                tma_load_3d_pair(sb, leader ? &tmB0 : &tmB1, full_lead, k0, col0, e);
+                tma_load_3d_pair(sb, leader ? &tmB0 : &tmB1, full_lead, k0, col0, ew);
               } else {
-                tma_load_3d_pair(sb, &tmB0, full_lead, k0, col0 + (int)rank * 128, e);
+                tma_load_3d_pair(sb, &tmB0, full_lead, k0, col0 + (int)rank * 128, ew);
               }
             } else if (SWIGLU && half) {
-              tma_load_3d_pair(sb, &tmB0, full_lead, col0 + (int)rank * 64, kb * kBK, e);
+              tma_load_3d_pair(sb, &tmB0, full_lead, col0 + (int)rank * 64, kb * kBK, ew);
               tma_load_3d_pair(sb + kChunkBytes, &tmB1, full_lead, col0 + (int)rank * 64,
-                               kb * kBK, e);
+                               kb * kBK, ew);
             } else if (SWIGLU) {
               const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
 #pragma unroll
               for (int c = 0; c < 2; ++c)
-                tma_load_3d_pair(sb + c * kChunkBytes, mb, full_lead, col0 + c * 64, kb * kBK, e);
+                tma_load_3d_pair(sb + c * kChunkBytes, mb, full_lead, col0 + c * 64, kb * kBK, ew);
             } else {
 #pragma unroll
               for (int c = 0; c < 2; ++c)
                 tma_load_3d_pair(sb + c * kChunkBytes, &tmB0, full_lead,
-                                 col0 + (int)rank * 128 + c * 64, kb * kBK, e);
+                                 col0 + (int)rank * 128 + c * 64, kb * kBK, ew);
             }
           }
           last_it[s] = it;
@@ -986,8 +990,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
       uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kPairStagingOff) + q * kStageWords;
       // E4M3: column scales from (e, column), the row's scale per thread
-      const float* cs0 = E4M3 ? col_scale0 + (size_t)e * n_out : nullptr;
-      const float* cs1 = (E4M3 && SWIGLU) ? col_scale1 + (size_t)e * n_out : nullptr;
+      const int ew = weight_index(fz, e);
+      const float* cs0 = E4M3 ? col_scale0 + (size_t)ew * n_out : nullptr;
+      const float* cs1 = (E4M3 && SWIGLU) ? col_scale1 + (size_t)ew * n_out : nullptr;
       if (!half) {
         const int first = m * kPairM + (int)rank * kBM + q * 32;   // first row of this warp
         const int nvalid = clamp_rows(sh.row_cnt[e] - first);
@@ -1162,6 +1167,9 @@ static bool map_a(CUtensorMap* a, CUtensorMap* a64, const void* rows, int K, int
   return map_rows(a, rows, K, max_rows, kBM) && map_rows(a64, rows, K, max_rows, kBM / 2);
 }
 
+// experts whose weights the tensor maps cover (buckets may outnumber them)
+static int weight_count(const FuseArgs& fz, int E) { return fz.n_weights > 0 ? fz.n_weights : E; }
+
 // GEMM 1: h = silu(A Wg) * (A Wu), A = x_perm or (gathering) the token rows
 cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, int E, int d,
                            int f, int max_rows, const __nv_bfloat16* w_gate,
@@ -1169,7 +1177,8 @@ cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, 
                            cudaStream_t s, bool* map_failed, const FuseArgs& fz) {
   CUtensorMap ta, ta64, tg, tu;
   *map_failed = !(map_a(&ta, &ta64, a_rows, d, max_rows, false, fz) &&
-                  map_weights(&tg, w_gate, E, d, f) && map_weights(&tu, w_up, E, d, f));
+                  map_weights(&tg, w_gate, weight_count(fz, E), d, f) &&
+                  map_weights(&tu, w_up, weight_count(fz, E), d, f));
   if (*map_failed) return cudaSuccess;
   if (use_pair_tiles(E, max_rows))
     return launch_gemm_pair<true>(7, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s,
@@ -1184,7 +1193,7 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
                         int32_t* status, cudaStream_t s, bool* map_failed, const FuseArgs& fz) {
   CUtensorMap ta, ta64, td;
   *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_rows(&ta64, h, f, max_rows, kBM / 2) &&
-                  map_weights(&td, w_down, E, f, d));
+                  map_weights(&td, w_down, weight_count(fz, E), f, d));
   if (*map_failed) return cudaSuccess;
   if (d % 256 == 0 && use_pair_tiles(E, max_rows))
     return launch_gemm_pair<false>(8, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
@@ -1233,12 +1242,13 @@ cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_
                                 bool* map_failed, const FuseArgs& fz) {
   CUtensorMap ta, ta64, tg, tu;
   *map_failed = !(map_a(&ta, &ta64, xq, d, max_rows, true, fz) &&
-                  map_weights_e4m3(&tg, wq_gate, E, f, d) && map_weights_e4m3(&tu, wq_up, E, f, d));
+                  map_weights_e4m3(&tg, wq_gate, weight_count(fz, E), f, d) &&
+                  map_weights_e4m3(&tu, wq_up, weight_count(fz, E), f, d));
   if (*map_failed) return cudaSuccess;
   if (use_pair_tiles(E, max_rows)) {
     CUtensorMap tgh, tuh;
-    *map_failed = !(map_weights_e4m3(&tgh, wq_gate, E, f, d, 64) &&
-                    map_weights_e4m3(&tuh, wq_up, E, f, d, 64));
+    *map_failed = !(map_weights_e4m3(&tgh, wq_gate, weight_count(fz, E), f, d, 64) &&
+                    map_weights_e4m3(&tuh, wq_up, weight_count(fz, E), f, d, 64));
     if (*map_failed) return cudaSuccess;
     return launch_gemm_pair<true, true>(9, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h,
                                         status, s, fz, &tgh, &tuh, sx, s_gate, s_up);
@@ -1254,7 +1264,7 @@ cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int3
   CUtensorMap ta, ta64, td;
   *map_failed = !(map_rows_e4m3(&ta, hq, f, max_rows, kBM) &&
                   map_rows_e4m3(&ta64, hq, f, max_rows, kBM / 2) &&
-                  map_weights_e4m3(&td, wq_down, E, d, f));
+                  map_weights_e4m3(&td, wq_down, weight_count(fz, E), d, f));
   if (*map_failed) return cudaSuccess;
   if (d % 256 == 0 && use_pair_tiles(E, max_rows))
     return launch_gemm_pair<false, true>(10, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,

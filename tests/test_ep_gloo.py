@@ -1,0 +1,136 @@
+"""Host logic of the expert-parallel layer (mixture_experts_layer_36_b200.ep)
+on CPU ranks over gloo: the count and row exchanges, the slot-to-expert
+mapping of the received buckets and the return exchange, with the compute
+steps done by the oracle.  Each rank's output must equal the single-process
+oracle layer on that rank's tokens with all experts (the same fp64 sums), for
+P = 2 and 4 ranks, with and without dropped tokens.
+"""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class OracleOps:
+    """The layer's compute steps on the CPU oracle (test infrastructure).
+    Activations travel as fp64 tensors holding exact bf16 values."""
+
+    def __init__(self, oracle):
+        self.o = oracle
+
+    @staticmethod
+    def _bits(t):
+        v = t.to(torch.float32).to(torch.bfloat16)
+        return v.view(torch.int16).numpy().view(np.uint16)
+
+    def route(self, x, w_router, bias, k):
+        lg = self.o.router_logits(self._bits(x), w_router.numpy(),
+                                  None if bias is None else bias.numpy())
+        idx, w = self.o.topk(lg.astype(np.float32), k)
+        return torch.from_numpy(lg), torch.from_numpy(idx), torch.from_numpy(w)
+
+    def capacity(self, T, E, k, cf):
+        return self.o.capacity(T, E, k, cf)
+
+    def permute_padded(self, x, topk_idx, E, cf):
+        T = x.shape[0]
+        k = topk_idx.shape[1]
+        C = self.o.capacity(T, E, k, cf)
+        counts, _, slot, _, _ = self.o.permute(topk_idx.numpy(), E, C)
+        pad, _ = self.o.dispatch_padded(self._bits(x), topk_idx.numpy(), slot, E, C)
+        x_pad = torch.from_numpy(self.o.bits_to_f64(pad))
+        offsets = torch.arange(E + 1, dtype=torch.int32) * C
+        return torch.from_numpy(counts), offsets, torch.from_numpy(slot), x_pad
+
+    def mlp_buckets(self, x_rows, offsets, bucket_rows, w_gate, w_up, w_down):
+        B = offsets.shape[0] - 1
+        E_w = w_gate.shape[0]
+        y = torch.zeros(x_rows.shape[0], w_down.shape[2], dtype=torch.float64)
+        xb = self._bits(x_rows)
+        for b in range(B):
+            lo, n = int(offsets[b]), int(bucket_rows[b])
+            if n == 0:
+                continue
+            e = b % E_w
+            _, o = self.o.swiglu_rows(xb[lo:lo + n], self._bits(w_gate[e]), self._bits(w_up[e]),
+                                      self._bits(w_down[e]))
+            y[lo:lo + n] = torch.from_numpy(o)
+        return y
+
+    def combine(self, y_rows, x, topk_idx, topk_w, slot, offsets):
+        return torch.from_numpy(self.o.combine(y_rows.numpy(), self._bits(x), topk_idx.numpy(),
+                                               topk_w.numpy(), slot.numpy(), offsets.numpy()))
+
+
+def _worker(rank, world, port, case, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    import oracle
+    from mixture_experts_layer_36_b200 import ep, synth
+    from mixture_experts_layer_36_b200.configs import MoEConfig
+    T, d, E, k, f, cf = case
+    cfg = MoEConfig("ep_case", T=T, d=d, E=E, k=k, f=f, cf=cf, seed=5)
+    w = synth.make_weights(cfg, "cpu")                    # the same weights on every rank
+    x = synth.make_tokens(cfg, "cpu", seed=100 + rank)    # each rank its own tokens
+    layer = ep.ExpertParallelMoE(w["w_router"], w["bias"],
+                                 ep.shard_experts(w["w_gate"], rank, world),
+                                 ep.shard_experts(w["w_up"], rank, world),
+                                 ep.shard_experts(w["w_down"], rank, world), k, cf,
+                                 ops=OracleOps(oracle))
+    y = layer(x).numpy()
+    xb = OracleOps._bits(x)
+    ops = OracleOps(oracle)
+    lg32 = oracle.router_logits(xb, w["w_router"].numpy(), None).astype(np.float32)
+    ref = oracle.moe_forward(xb, w["w_router"].numpy(), None, ops._bits(w["w_gate"]),
+                             ops._bits(w["w_up"]), ops._bits(w["w_down"]), k, cf,
+                             decision_logits=lg32)
+    dist.barrier()
+    dist.destroy_process_group()
+    out.put((rank, float(np.max(np.abs(y - ref["y"]))), float(np.max(np.abs(ref["y"]))),
+             int(ref["n_dropped"])))
+
+
+CASES = [
+    # (T, d, E, k, f, cf)
+    (24, 16, 8, 2, 32, 0.0),      # dropless
+    (40, 16, 8, 3, 32, 0.75),     # with drops
+]
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("case", CASES, ids=["dropless", "drops"])
+def test_expert_parallel_matches_single_process(world, case):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, case, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=280) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=30)
+        assert p.exitcode == 0
+    dropped = 0
+    for rank, err, scale, n_drop in res:
+        assert err <= 1e-12 * max(scale, 1.0), (rank, err)
+        dropped += n_drop
+    if case[5] > 0:
+        assert dropped > 0                    # the capacity limit was exercised

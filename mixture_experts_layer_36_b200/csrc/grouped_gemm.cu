@@ -388,7 +388,12 @@ __device__ __forceinline__ void mma_role(GemmShared& sh, uint8_t* smem, int E, i
 
 // Epilogue (warps 2..5): drain accumulator buffer lt & 1 of each tile
 // (tcgen05.ld -> [column scales] -> SwiGLU + bf16 stores, or fp32 stores).
-template <int BN, bool SWIGLU, bool SCALED>
+// Fusion compiled into a kernel instance: none, gather (GEMM 1's producer
+// fetches token rows by row_src), scatter (GEMM 2's epilogue adds weighted rows
+// into y32).  Kept out of the plain instances' code entirely.
+constexpr int kFuseNone = 0, kFuseGather = 1, kFuseScatter = 2;
+
+template <int BN, bool SWIGLU, bool SCALED, int FUSE = kFuseNone>
 __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, int warp,
                                               int lane, int E, int n_tiles, int n_out,
                                               void* out_raw, const float* row_scale,
@@ -439,7 +444,7 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
         swiglu_pack(g, u, pk);
         store_chunk_bf16(pk, o + c * 32, n_out, nvalid, lane);
       }
-    } else if (fz.y32) {
+    } else if (FUSE == kFuseScatter) {
       // fused combine: weighted rows added into the token accumulator
       int my_t = 0;
       float my_w = 0.f;
@@ -475,7 +480,7 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
 }
 
 // ---------------------------------------------------------------- bf16 weights
-template <int BN, bool SWIGLU>
+template <int BN, bool SWIGLU, int FUSE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
@@ -522,7 +527,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_3d(sb + c * kChunkBytes, &tmB0, bar, col0 + c * 64, kb * kBK, e);
       }
     };
-    if (fz.row_src)      // A rows gathered from the token rows (tmA maps those)
+    if constexpr (FUSE == kFuseGather)   // A rows gathered from the token rows (tmA maps those)
       producer_role_gather<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
           sh, smem, &tmA, fz, E, n_tiles, nkb, status, load_b, kBK, lane);
     else if (lane == 0)
@@ -534,7 +539,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                                  Cfg::kIdesc, Cfg::kIdesc64,
                                                                  status);
   } else {
-    epilogue_role<BN, SWIGLU, false>(sh, smem + Cfg::kStagingOff, warp, lane, E, n_tiles, n_out,
+    epilogue_role<BN, SWIGLU, false, FUSE>(sh, smem + Cfg::kStagingOff, warp, lane, E, n_tiles,
+                                           n_out,
                                      out_raw, nullptr, nullptr, nullptr, fz, status);
   }
 
@@ -568,7 +574,7 @@ struct E4m3Cfg {
   static constexpr uint32_t kIdesc64 = idesc_e4m3_f32(kBM / 2, BN);
 };
 
-template <int BN, bool SWIGLU>
+template <int BN, bool SWIGLU, int FUSE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,     // codes [rows, K]
                              const __grid_constant__ CUtensorMap tmA64,
@@ -615,7 +621,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_3d(sb + c * 128 * Cfg::kBKe, &tmB0, bar, kb * Cfg::kBKe, col0 + c * 128, e);
       }
     };
-    if (fz.row_src)
+    if constexpr (FUSE == kFuseGather)
       producer_role_gather<Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, Cfg::kBBytes>(
           sh, smem, &tmA, fz, E, n_tiles, nkb, status, load_b, Cfg::kBKe, lane);
     else if (lane == 0)
@@ -626,7 +632,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mma_role<BN, Cfg::kStages, Cfg::kStageBytes, Cfg::kABytes, true>(
           sh, smem, E, n_tiles, nkb, Cfg::kIdesc, Cfg::kIdesc64, status);
   } else {
-    epilogue_role<BN, SWIGLU, true>(sh, smem + Cfg::kStagingOff, warp, lane, E, n_tiles, n_out,
+    epilogue_role<BN, SWIGLU, true, FUSE>(sh, smem + Cfg::kStagingOff, warp, lane, E, n_tiles,
+                                          n_out,
                                     out_raw, row_scale, col_scale0, col_scale1, fz, status);
   }
 
@@ -735,7 +742,7 @@ __device__ __forceinline__ void decode_pair_tile(const PairShared& sh, int tile,
 // E4M3: e4m3 operands, both K-major (weights [E, N, K]), 128-deep k-blocks,
 // kind::f8f6f4; tmB0h / tmB1h are 64-row weight boxes for the half tiles'
 // 64 + 64 column split; the epilogue applies the row and column scales.
-template <bool SWIGLU, bool E4M3>
+template <bool SWIGLU, bool E4M3, int FUSE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
@@ -840,7 +847,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // A rows gathered from the token rows (all 32 lanes issue tile::gather4),
     // else one thread loads the permuted rows' tile
-    const bool gather = fz.row_src != nullptr;
+    constexpr bool gather = FUSE == kFuseGather;
     if (gather || lane == 0) {
       // ------------------------------------------------ TMA producer (both CTAs)
       int it = 0;
@@ -1005,7 +1012,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int c = 0; c < 4; ++c)
             swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 128 + c * 32, o + c * 32, n_out,
                                      nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
-        } else if (fz.y32) {
+        } else if (FUSE == kFuseScatter) {
           const int c0 = n * kOutCols;
           int my_t = 0;
           float my_w = 0.f;
@@ -1043,7 +1050,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int c = 0; c < 2; ++c)
             swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 64 + c * 32, o + c * 32, n_out,
                                      nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
-        } else if (fz.y32) {
+        } else if (FUSE == kFuseScatter) {
           const int c0 = n * kOutCols + hh * 128;
           int my_t = 0;
           float my_w = 0.f;
@@ -1082,8 +1089,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-template <int BN, bool SWIGLU>
-static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+template <int BN, bool SWIGLU, int FUSE>
+static cudaError_t launch_gemm_t(int slot, const CUtensorMap& a, const CUtensorMap& a64,
                                const CUtensorMap& b0, const CUtensorMap& b1,
                                const int32_t* offsets, int E, int K,
                                int n_out, int max_rows, void* out, int32_t* status,
@@ -1092,7 +1099,7 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  auto kern = grouped_gemm_kernel<BN, SWIGLU>;
+  auto kern = grouped_gemm_kernel<BN, SWIGLU, FUSE>;
   if (!di->attr_set[slot]) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg::kSmemBytes);
@@ -1109,20 +1116,19 @@ static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap
   return cudaGetLastError();
 }
 
-template <bool SWIGLU, bool E4M3 = false>
-static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtensorMap& a64,
-                                    const CUtensorMap& b0, const CUtensorMap& b1,
-                                    const int32_t* offsets, int E, int K, int n_out, int max_rows,
-                                    void* out, int32_t* status, cudaStream_t s,
-                                    const FuseArgs& fz, const CUtensorMap* b0h = nullptr,
-                                    const CUtensorMap* b1h = nullptr,
-                                    const float* row_scale = nullptr,
-                                    const float* cs0 = nullptr, const float* cs1 = nullptr) {
+template <bool SWIGLU, bool E4M3, int FUSE>
+static cudaError_t launch_gemm_pair_t(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+                                      const CUtensorMap& b0, const CUtensorMap& b1,
+                                      const int32_t* offsets, int E, int K, int n_out,
+                                      int max_rows, void* out, int32_t* status, cudaStream_t s,
+                                      const FuseArgs& fz, const CUtensorMap* b0h,
+                                      const CUtensorMap* b1h, const float* row_scale,
+                                      const float* cs0, const float* cs1) {
   constexpr int kSmem = kPairStagingOff + 4 * kStageWords * 4 + 1024;
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  auto kern = grouped_gemm_pair_kernel<SWIGLU, E4M3>;
+  auto kern = grouped_gemm_pair_kernel<SWIGLU, E4M3, FUSE>;
   if (!di->attr_set[slot]) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (err != cudaSuccess) return err;
@@ -1148,6 +1154,80 @@ static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtens
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a, a64, b0, b1, b0h ? *b0h : b0, b1h ? *b1h : b1,
                             row_scale, cs0, cs1, offsets, E, K, n_out, max_rows, out, status, fz);
+}
+
+// The fusion an instance is compiled for, from the arguments.
+static int fuse_kind(const FuseArgs& fz) {
+  return fz.row_src ? kFuseGather : (fz.y32 ? kFuseScatter : kFuseNone);
+}
+
+// attribute slots: each (kernel, fusion) instance sets its smem limit once
+template <int BN, bool SWIGLU>
+static cudaError_t launch_gemm(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+                               const CUtensorMap& b0, const CUtensorMap& b1,
+                               const int32_t* offsets, int E, int K, int n_out, int max_rows,
+                               void* out, int32_t* status, cudaStream_t s, const FuseArgs& fz) {
+  const int kind = fuse_kind(fz);
+  if constexpr (SWIGLU) {
+    if (kind == kFuseGather)
+      return launch_gemm_t<BN, SWIGLU, kFuseGather>(slot + 16, a, a64, b0, b1, offsets, E, K,
+                                                    n_out, max_rows, out, status, s, fz);
+  } else {
+    if (kind == kFuseScatter)
+      return launch_gemm_t<BN, SWIGLU, kFuseScatter>(slot + 32, a, a64, b0, b1, offsets, E, K,
+                                                     n_out, max_rows, out, status, s, fz);
+  }
+  if (kind != kFuseNone) return cudaErrorInvalidValue;
+  return launch_gemm_t<BN, SWIGLU, kFuseNone>(slot, a, a64, b0, b1, offsets, E, K, n_out,
+                                              max_rows, out, status, s, fz);
+}
+
+template <bool SWIGLU, bool E4M3 = false>
+static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+                                    const CUtensorMap& b0, const CUtensorMap& b1,
+                                    const int32_t* offsets, int E, int K, int n_out, int max_rows,
+                                    void* out, int32_t* status, cudaStream_t s,
+                                    const FuseArgs& fz, const CUtensorMap* b0h = nullptr,
+                                    const CUtensorMap* b1h = nullptr,
+                                    const float* row_scale = nullptr,
+                                    const float* cs0 = nullptr, const float* cs1 = nullptr) {
+  const int kind = fuse_kind(fz);
+  if constexpr (!E4M3 && SWIGLU) {
+    if (kind == kFuseGather)
+      return launch_gemm_pair_t<SWIGLU, E4M3, kFuseGather>(slot + 16, a, a64, b0, b1, offsets, E,
+                                                           K, n_out, max_rows, out, status, s,
+                                                           fz, b0h, b1h, row_scale, cs0, cs1);
+  } else if constexpr (!E4M3 && !SWIGLU) {
+    if (kind == kFuseScatter)
+      return launch_gemm_pair_t<SWIGLU, E4M3, kFuseScatter>(slot + 32, a, a64, b0, b1, offsets,
+                                                            E, K, n_out, max_rows, out, status,
+                                                            s, fz, b0h, b1h, row_scale, cs0, cs1);
+  }
+  if (kind != kFuseNone) return cudaErrorInvalidValue;
+  return launch_gemm_pair_t<SWIGLU, E4M3, kFuseNone>(slot, a, a64, b0, b1, offsets, E, K, n_out,
+                                                     max_rows, out, status, s, fz, b0h, b1h,
+                                                     row_scale, cs0, cs1);
+}
+
+template <int BN, bool SWIGLU, int FUSE>
+static cudaError_t launch_gemm_e4m3_t(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+                                      const CUtensorMap& b0, const CUtensorMap& b1,
+                                      const float* row_scale, const float* s0, const float* s1,
+                                      const int32_t* offsets, int E, int K, int n_out,
+                                      int max_rows, void* out, int32_t* status, cudaStream_t s,
+                                      const FuseArgs& fz);
+
+template <int BN, bool SWIGLU>
+static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+                                    const CUtensorMap& b0, const CUtensorMap& b1,
+                                    const float* row_scale, const float* s0, const float* s1,
+                                    const int32_t* offsets, int E, int K, int n_out, int max_rows,
+                                    void* out, int32_t* status, cudaStream_t s,
+                                    const FuseArgs& fz) {
+  if (fuse_kind(fz) != kFuseNone) return cudaErrorInvalidValue;   // not built for e4m3
+  return launch_gemm_e4m3_t<BN, SWIGLU, kFuseNone>(slot, a, a64, b0, b1, row_scale, s0, s1,
+                                                   offsets, E, K, n_out, max_rows, out, status,
+                                                   s, fz);
 }
 
 // Pair tiles (256 rows) pay off when buckets are large; the buffer's rows
@@ -1205,8 +1285,8 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
                                  s, fz);
 }
 
-template <int BN, bool SWIGLU>
-static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtensorMap& a64,
+template <int BN, bool SWIGLU, int FUSE>
+static cudaError_t launch_gemm_e4m3_t(int slot, const CUtensorMap& a, const CUtensorMap& a64,
                                     const CUtensorMap& b0, const CUtensorMap& b1,
                                     const float* row_scale, const float* s0, const float* s1,
                                     const int32_t* offsets, int E, int K, int n_out, int max_rows,
@@ -1216,7 +1296,7 @@ static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtens
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  auto kern = grouped_gemm_e4m3_kernel<BN, SWIGLU>;
+  auto kern = grouped_gemm_e4m3_kernel<BN, SWIGLU, FUSE>;
   if (!di->attr_set[slot]) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cfg::kSmemBytes);

@@ -316,7 +316,7 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), dev, dist)
 
     names = layer.stage_names
-    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+    stage_ms = {n: statistics.median(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                 for j, n in enumerate(names)}
     status = int(layer.status.item())
     N = int(layer.perm["counts"].sum().item())          # kept pairs (either layout)

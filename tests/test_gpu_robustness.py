@@ -58,3 +58,56 @@ def test_layer_forward_replays_in_cuda_graph(cfg):
         ref, _ = moe.moe_layer_forward(x.clone(), *args)
         torch.cuda.synchronize()
         assert torch.equal(y, ref)
+
+
+def _replay_check(cfg, forward, ws_size, compare):
+    """Capture forward(x, y, ws) in a CUDA graph after one eager call, replay it
+    on new tokens and compare y with a fresh eager call via compare(y, ref)."""
+    inp, _ = cuda_inputs(cfg)
+    x = inp["x"].clone()
+    y = torch.empty_like(x)
+    ws = torch.empty(ws_size, dtype=torch.uint8, device="cuda")
+    forward(inp, x, y, ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        forward(inp, x, y, ws)
+    for seed in (7, 8):
+        x.copy_(synth.make_tokens(cfg, "cuda", seed=seed))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = torch.empty_like(x)
+        forward(inp, x.clone(), ref, torch.empty_like(ws))
+        torch.cuda.synchronize()
+        compare(y, ref)
+
+
+GRAPH_CFG = small("graph_drops", T=700, d=256, E=8, k=2, f=256, cf=0.75, seed=24)
+
+
+def test_fp8_layer_replays_in_cuda_graph():
+    cfg = GRAPH_CFG
+    q = {}
+
+    def forward(inp, x, y, ws):
+        if not q:
+            q.update({n: moe.moe_quantize_weights_fp8(inp[n]) for n in ("w_gate", "w_up",
+                                                                         "w_down")})
+        moe.moe_layer_forward_fp8(x, inp["w_router"], inp["bias"], *q["w_gate"], *q["w_up"],
+                                  *q["w_down"], cfg.k, cfg.cf, y=y, ws=ws)
+
+    size = moe.moe_workspace_size_fp8(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.cf)
+    _replay_check(cfg, forward, size, lambda a, b: torch.equal(a, b) or pytest.fail("y differs"))
+
+
+def test_fused_layer_replays_in_cuda_graph():
+    from moe_testlib import assert_bf16_close, f64
+    cfg = GRAPH_CFG
+
+    def forward(inp, x, y, ws):
+        moe.moe_layer_forward_fused(x, inp["w_router"], inp["bias"], inp["w_gate"], inp["w_up"],
+                                    inp["w_down"], cfg.k, cfg.cf, y=y, ws=ws)
+
+    size = moe.moe_workspace_size_fused(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.cf)
+    # the fused sums run in tile-completion order: equal up to fp32 rounding
+    _replay_check(cfg, forward, size, lambda a, b: assert_bf16_close(f64(a), f64(b), "y"))

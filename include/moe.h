@@ -29,7 +29,10 @@
  *     kernel that detects a problem on the device (a bounded wait that gave
  *     up, inconsistent bucket offsets) ORs a bit into the caller's int32
  *     device status word `dev_status` (nullable: then nothing is reported);
- *     read it after synchronising.  Bits: 1 = wait timeout, 2 = bad offsets.
+ *     read it after synchronising.  Bits: 1 = wait timeout, 2 = bad offsets,
+ *     4 = a top-k expert id outside [0, E) (such a pair is treated as
+ *     dropped; builds with MOE_CHECKS also report an expert listed twice for
+ *     one token).
  *   - Limits: 1 <= E <= 256, 1 <= k <= min(E, 8), T*k < 2^31, d and f
  *     multiples of 128 (else MOE_ERR_UNSUPPORTED).  T == 0 is a no-op.
  */
@@ -165,11 +168,16 @@ int moe_route(const void* x, const float* w_router, const float* bias, int64_t T
  *   x_perm    bf16 [max_rows,d] out: row offsets[e]+slot holds x[t]
  *   n_dropped i32  [1]          out: number of dropped pairs
  *   ws, ws_bytes                device scratch, >= moe_permute_workspace_size
+ *   dev_status                  nullable device status word: bit 4 when a
+ *                               topk_idx entry lies outside [0, E) (that pair
+ *                               is treated as dropped, slot -1, takes no
+ *                               bucket place and is not counted in n_dropped,
+ *                               which counts capacity overflow)
  * Rows at and beyond offsets[E] of row_src / x_perm are left untouched. */
 int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
                 int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
                 int32_t* row_src, void* x_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
-                void* stream);
+                int32_t* dev_status, void* stream);
 
 /* moe_permute without the scratch argument, for callers that cannot allocate
  * device memory or pass the library any: e.g. an operator plugin that only
@@ -250,7 +258,7 @@ int64_t moe_padded_rows(int64_t T, int64_t E, int64_t k, double cf);
 int moe_permute_padded(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
                        int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
                        int32_t* row_src, void* x_pad, int32_t* n_dropped, void* ws,
-                       size_t ws_bytes, void* stream);
+                       size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* ---- Buckets that are not experts (expert parallelism) ----
  * With the experts spread over P ranks ("Expert Parallelism & All-to-All"
@@ -290,7 +298,7 @@ int moe_expert_mlp_buckets(const void* x_rows, const int32_t* offsets, const int
 int moe_permute_fused(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
                       int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
                       int32_t* row_src, int32_t* row_pair, void* x_perm, int32_t* n_dropped,
-                      float* y32, void* ws, size_t ws_bytes, void* stream);
+                      float* y32, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* moe_expert_gate_up with A row r of bucket storage = x[row_src[r]] (x bf16
  * [T,d], row_src from the permutation; no x_perm). */
@@ -357,7 +365,7 @@ int moe_permute_fp8(const uint8_t* xq, const float* sx, const int32_t* topk_idx,
                     int64_t d, int64_t E, int64_t k, double cf, int32_t* counts,
                     int32_t* offsets, int32_t* slot, int32_t* row_src, uint8_t* xq_perm,
                     float* sx_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
-                    void* stream);
+                    int32_t* dev_status, void* stream);
 
 /* GEMM 1 + SwiGLU on e4m3 operands: h[r,:] = silu(g) * u with
  * g[r,n] = sx[r] * s_gate[e,n] * sum_k xq[r,k] wq_gate[e,n,k] (u likewise) for

@@ -61,7 +61,8 @@ def _load():
         "moe_workspace_size": (sz, [i64, i64, i64, i64, i64, dbl]),
         "moe_workspace_field_offset": (i64, [ctypes.c_int, i64, i64, i64, i64, i64, dbl]),
         "moe_route": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, sz, p, p]),
-        "moe_permute": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p, sz, p]),
+        "moe_permute": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p, sz, p,
+                                       p]),
         "moe_permute_noalloc": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p]),
         "moe_expert_gate_up": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p]),
         "moe_expert_down": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p]),
@@ -72,7 +73,7 @@ def _load():
         "moe_quantize_weights_fp8": (ctypes.c_int, [p, i64, i64, i64, p, p, p]),
         "moe_quantize_rows_fp8": (ctypes.c_int, [p, i64, i64, p, p, p, p]),
         "moe_permute_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
-                                           p, sz, p]),
+                                           p, sz, p, p]),
         "moe_expert_gate_up_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p, p,
                                                   p]),
         "moe_expert_down_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, p]),
@@ -81,7 +82,7 @@ def _load():
         "moe_expert_mlp_buckets": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, i64, p, p, p, p, p,
                                                   p, p]),
         "moe_permute_fused": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
-                                             p, p, sz, p]),
+                                             p, p, sz, p, p]),
         "moe_expert_gate_up_gather": (ctypes.c_int, [p, i64, p, p, i64, i64, i64, i64, p, p, p, p,
                                                      p]),
         "moe_expert_down_scatter": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, i64, p, p,
@@ -91,7 +92,7 @@ def _load():
         "moe_layer_forward_fused": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl,
                                                    p, p, sz, p]),
         "moe_permute_padded": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
-                                              sz, p]),
+                                              sz, p, p]),
         "moe_layer_forward_fp8": (ctypes.c_int, [p, p, p, p, p, p, p, p, p, i64, i64, i64, i64, i64,
                                                  dbl, p, p, sz, p]),
     }
@@ -209,7 +210,7 @@ def moe_route(x, w_router, bias, k, logits=None, topk_idx=None, topk_w=None, ws=
     return logits, topk_idx, topk_w
 
 
-def moe_permute(x, topk_idx, E, cf, out=None, ws=None, stream=None):
+def moe_permute(x, topk_idx, E, cf, out=None, ws=None, dev_status=None, stream=None):
     """Capacity-limited permutation.  Returns a dict with counts, offsets, slot,
     row_src, x_perm (max_rows rows; rows >= offsets[E] untouched), n_dropped."""
     T, d = x.shape
@@ -234,7 +235,7 @@ def moe_permute(x, topk_idx, E, cf, out=None, ws=None, stream=None):
     _check("moe_permute", _lib.moe_permute(
         _ptr(x), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]),
         _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["x_perm"]),
-        _ptr(out["n_dropped"]), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(out["n_dropped"]), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
     return out
 
 
@@ -371,7 +372,8 @@ def moe_expert_mlp_buckets(x_rows, offsets, bucket_rows, w_gate, w_up, w_down, h
 
 # ----------------------------------------------------------------- fused path
 
-def moe_permute_fused(x, topk_idx, E, cf, copy_rows=True, out=None, ws=None, stream=None):
+def moe_permute_fused(x, topk_idx, E, cf, copy_rows=True, out=None, ws=None, dev_status=None,
+                      stream=None):
     """The permutation for the fused path.  Returns a dict with counts, offsets,
     slot, row_src, row_pair, n_dropped, a zeroed fp32 token accumulator "y32"
     [T, d] and, with copy_rows, "x_perm"."""
@@ -399,7 +401,7 @@ def moe_permute_fused(x, topk_idx, E, cf, copy_rows=True, out=None, ws=None, str
         _ptr(x) if copy_rows else None, _ptr(topk_idx), T, d, E, k, float(cf),
         _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]),
         _ptr(out["row_pair"]), _ptr(xp), _ptr(out["n_dropped"]), _ptr(out.get("y32")), _ptr(ws),
-        ws.numel(), _stream(stream)))
+        ws.numel(), _ptr(dev_status), _stream(stream)))
     return out
 
 
@@ -484,7 +486,7 @@ def moe_padded_rows(T, E, k, cf):
     return int(_lib.moe_padded_rows(T, E, k, float(cf)))
 
 
-def moe_permute_padded(x, topk_idx, E, cf, out=None, ws=None, stream=None):
+def moe_permute_padded(x, topk_idx, E, cf, out=None, ws=None, dev_status=None, stream=None):
     """moe_permute into the padded [E*C, d] layout.  Returns a dict like
     moe_permute's with "x_pad" in place of "x_perm" (offsets[e] = e*C)."""
     T, d = x.shape
@@ -508,7 +510,7 @@ def moe_permute_padded(x, topk_idx, E, cf, out=None, ws=None, stream=None):
     _check("moe_permute_padded", _lib.moe_permute_padded(
         _ptr(x), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]), _ptr(out["offsets"]),
         _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["x_pad"]), _ptr(out["n_dropped"]),
-        _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
     return out
 
 
@@ -540,7 +542,7 @@ def moe_quantize_rows_fp8(x, n_rows=None, q=None, scale=None, stream=None):
     return q, scale
 
 
-def moe_permute_fp8(xq, sx, topk_idx, E, cf, out=None, ws=None, stream=None):
+def moe_permute_fp8(xq, sx, topk_idx, E, cf, out=None, ws=None, dev_status=None, stream=None):
     """moe_permute on e4m3 token rows (codes + row scales).  Returns a dict
     like moe_permute's, with "xq" / "sx" in place of "x_perm"."""
     T, d = xq.shape
@@ -564,7 +566,7 @@ def moe_permute_fp8(xq, sx, topk_idx, E, cf, out=None, ws=None, stream=None):
     _check("moe_permute_fp8", _lib.moe_permute_fp8(
         _ptr(xq), _ptr(sx), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]),
         _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["xq"]),
-        _ptr(out["sx"]), _ptr(out["n_dropped"]), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(out["sx"]), _ptr(out["n_dropped"]), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
     return out
 
 

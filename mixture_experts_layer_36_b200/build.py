@@ -1,6 +1,11 @@
 """Build libmoe.so in-tree with nvcc for sm_100a (no GPU needed to compile).
 
-    python -m mixture_experts_layer_36_b200.build [--force] [--verbose-ptxas]
+    python -m mixture_experts_layer_36_b200.build [--force] [--verbose-ptxas] [--checks]
+
+--checks builds the library with MOE_CHECKS: extra device-side input checks
+that report into the caller's status word (e.g. an expert listed twice for
+one token).  It replaces the in-tree libmoe.so; build again without the flag
+(with --force) to return to the normal library.
 """
 import argparse
 import glob
@@ -33,8 +38,9 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, jobs: int = 8) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, ptxas_verbose: bool = False, jobs: int = 8,
+          checks: bool = False) -> str:
+    if not force and not checks and up_to_date():
         return LIB
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
@@ -42,6 +48,8 @@ def build(force: bool = False, ptxas_verbose: bool = False, jobs: int = 8) -> st
              "-I", os.path.join(ROOT, "include"), *ARCH]
     if ptxas_verbose:
         flags += ["-Xptxas", "-v"]
+    if checks:
+        flags += ["-DMOE_CHECKS"]
     procs, objs = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
@@ -52,7 +60,7 @@ def build(force: bool = False, ptxas_verbose: bool = False, jobs: int = 8) -> st
             procs = []
     _wait(procs)
     tmp = LIB + f".{os.getpid()}.tmp"
-    subprocess.check_call([NVCC, "-shared", "-cudart", "shared", *ARCH, "-o", tmp, *objs])
+    subprocess.check_call([NVCC, "-shared", "-cudart", "shared", *ARCH, "-o", tmp, *objs, "-ldl"])
     os.replace(tmp, LIB)
     return LIB
 
@@ -67,6 +75,7 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--checks", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, ptxas_verbose=a.verbose_ptxas))
+    print(build(force=a.force, ptxas_verbose=a.verbose_ptxas, checks=a.checks))
     sys.exit(0)

@@ -2,6 +2,7 @@
 // the stage launches.  Every compute step runs in the kernels of router.cu,
 // permute.cu, grouped_gemm.cu and combine.cu.
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 
@@ -14,7 +15,7 @@ size_t permute_scratch_bytes(int64_t T, int64_t E);
 cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d, int E,
                            int k, int64_t C, int32_t* counts, int32_t* offsets, int32_t* slot,
                            int32_t* row_src, __nv_bfloat16* x_perm, int32_t* n_dropped,
-                           int32_t* chunk_hist, cudaStream_t s);
+                           int32_t* chunk_hist, cudaStream_t s, int32_t* status);
 cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, int E, int d,
                            int f, int max_rows, const __nv_bfloat16* w_gate,
                            const __nv_bfloat16* w_up, __nv_bfloat16* h, int32_t* status,
@@ -33,11 +34,13 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
                                 int32_t* counts, int32_t* offsets, int32_t* slot,
                                 int32_t* row_src, uint8_t* x_perm, float* perm_scale,
                                 int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
-                                int32_t* row_pair, float* zero_rows, int zero_cols);
+                                int32_t* row_pair, float* zero_rows, int zero_cols,
+                                int32_t* status);
 cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d,
                                   int E, int k, int64_t C, int32_t* counts, int32_t* offsets,
                                   int32_t* slot, int32_t* row_src, __nv_bfloat16* x_pad,
-                                  int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s);
+                                  int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
+                                  int32_t* status);
 cudaError_t launch_quantize_weights(const __nv_bfloat16* w, int E, int K, int N, uint8_t* q,
                                     float* scale, cudaStream_t s);
 cudaError_t launch_quantize_rows(const __nv_bfloat16* x, int R, int K, const int32_t* n_rows,
@@ -84,6 +87,19 @@ constexpr int64_t kMaxK = 8;
 constexpr int64_t kTileMultiple = 128;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around one stage of a one-shot layer call (host-side enqueue;
+// a profiler attached to the process shows it on the timeline).
+struct StageRange {
+  explicit StageRange(const char* name) { nvtxRangePushA(name); }
+  ~StageRange() { nvtxRangePop(); }
+};
+
+template <class F>
+int staged(const char* name, F call) {
+  StageRange range(name);
+  return call();
+}
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -254,7 +270,7 @@ int moe_route(const void* x, const float* w_router, const float* bias, int64_t T
 int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
                 int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
                 int32_t* row_src, void* x_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
-                void* stream) {
+                int32_t* dev_status, void* stream) {
   int st = check_routing_shape(T, E, k);
   if (st != MOE_OK) return st;
   if ((st = check_width(d)) != MOE_OK) return st;
@@ -269,7 +285,7 @@ int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, in
   return cuda_status(launch_permute(static_cast<const __nv_bfloat16*>(x), topk_idx, (int)T,
                                     (int)d, (int)E, (int)k, C, counts, offsets, slot, row_src,
                                     static_cast<__nv_bfloat16*>(x_perm), n_dropped,
-                                    static_cast<int32_t*>(ws), as_stream(stream)));
+                                    static_cast<int32_t*>(ws), as_stream(stream), dev_status));
 }
 
 static int check_gemm_args(int64_t E, int64_t d, int64_t f, int64_t max_rows) {
@@ -354,7 +370,7 @@ int64_t moe_padded_rows(int64_t T, int64_t E, int64_t k, double cf) {
 int moe_permute_padded(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
                        int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
                        int32_t* row_src, void* x_pad, int32_t* n_dropped, void* ws,
-                       size_t ws_bytes, void* stream) {
+                       size_t ws_bytes, int32_t* dev_status, void* stream) {
   int st = check_routing_shape(T, E, k);
   if (st != MOE_OK) return st;
   if ((st = check_width(d)) != MOE_OK) return st;
@@ -368,7 +384,7 @@ int moe_permute_padded(const void* x, const int32_t* topk_idx, int64_t T, int64_
   return cuda_status(moe::launch_permute_padded(
       static_cast<const __nv_bfloat16*>(x), topk_idx, (int)T, (int)d, (int)E, (int)k, C, counts,
       offsets, slot, row_src, static_cast<__nv_bfloat16*>(x_pad), n_dropped,
-      static_cast<int32_t*>(ws), as_stream(stream)));
+      static_cast<int32_t*>(ws), as_stream(stream), dev_status));
 }
 
 int moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t N, uint8_t* w_q,
@@ -396,7 +412,7 @@ int moe_permute_fp8(const uint8_t* xq, const float* sx, const int32_t* topk_idx,
                     int64_t d, int64_t E, int64_t k, double cf, int32_t* counts,
                     int32_t* offsets, int32_t* slot, int32_t* row_src, uint8_t* xq_perm,
                     float* sx_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
-                    void* stream) {
+                    int32_t* dev_status, void* stream) {
   int st = check_routing_shape(T, E, k);
   if (st != MOE_OK) return st;
   if ((st = check_width(d)) != MOE_OK) return st;
@@ -411,7 +427,8 @@ int moe_permute_fp8(const uint8_t* xq, const float* sx, const int32_t* topk_idx,
   return cuda_status(moe::launch_permute_rows(xq, (int)d, sx, topk_idx, (int)T, (int)E, (int)k, C,
                                               counts, offsets, slot, row_src, xq_perm, sx_perm,
                                               n_dropped, static_cast<int32_t*>(ws),
-                                              as_stream(stream), nullptr, nullptr, 0));
+                                              as_stream(stream), nullptr, nullptr, 0,
+                                              dev_status));
 }
 
 int moe_expert_gate_up_fp8(const uint8_t* xq, const float* sx, const int32_t* offsets, int64_t E,
@@ -488,25 +505,39 @@ int moe_layer_forward_fp8(const void* x, const float* w_router, const float* bia
   const int32_t* n_rows = offsets + E;          // kept rows, written by the permutation
   cudaStream_t s = as_stream(stream);
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, field(MOE_WS_ROUTE),
-                      moe_route_workspace_size(T, d, E, k), status, stream)) != MOE_OK)
-    return st;
+  st = staged("moe_route", [&] {
+    return moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, field(MOE_WS_ROUTE),
+                     moe_route_workspace_size(T, d, E, k), status, stream);
+  });
+  if (st != MOE_OK) return st;
   // each token is quantized once; the permutation moves its codes and scale
   uint8_t* xq_tok = reinterpret_cast<uint8_t*>(field(MOE_WS_XQ_TOK));
   float* sx_tok = reinterpret_cast<float*>(field(MOE_WS_SX_TOK));
-  if ((st = moe_quantize_rows_fp8(x, T, d, nullptr, xq_tok, sx_tok, stream)) != MOE_OK) return st;
-  if ((st = moe_permute_fp8(xq_tok, sx_tok, topk_idx, T, d, E, k, cf, counts, offsets, slot,
-                            row_src, xq, sx, n_dropped, field(MOE_WS_PERMUTE),
-                            moe_permute_workspace_size(T, E, k), stream)) != MOE_OK)
-    return st;
-  if ((st = moe_expert_gate_up_fp8(xq, sx, offsets, E, d, f, max_rows, wq_gate, s_gate, wq_up,
-                                   s_up, h, status, stream)) != MOE_OK)
-    return st;
-  if ((st = moe_quantize_rows_fp8(h, max_rows, f, n_rows, hq, shr, stream)) != MOE_OK) return st;
-  if ((st = moe_expert_down_fp8(hq, shr, offsets, E, d, f, max_rows, wq_down, s_down, y_perm,
-                                status, stream)) != MOE_OK)
-    return st;
-  return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
+  st = staged("moe_quantize_rows_fp8",
+              [&] { return moe_quantize_rows_fp8(x, T, d, nullptr, xq_tok, sx_tok, stream); });
+  if (st != MOE_OK) return st;
+  st = staged("moe_permute_fp8", [&] {
+    return moe_permute_fp8(xq_tok, sx_tok, topk_idx, T, d, E, k, cf, counts, offsets, slot,
+                           row_src, xq, sx, n_dropped, field(MOE_WS_PERMUTE),
+                           moe_permute_workspace_size(T, E, k), status, stream);
+  });
+  if (st != MOE_OK) return st;
+  st = staged("moe_expert_gate_up_fp8", [&] {
+    return moe_expert_gate_up_fp8(xq, sx, offsets, E, d, f, max_rows, wq_gate, s_gate, wq_up,
+                                  s_up, h, status, stream);
+  });
+  if (st != MOE_OK) return st;
+  st = staged("moe_quantize_rows_fp8",
+              [&] { return moe_quantize_rows_fp8(h, max_rows, f, n_rows, hq, shr, stream); });
+  if (st != MOE_OK) return st;
+  st = staged("moe_expert_down_fp8", [&] {
+    return moe_expert_down_fp8(hq, shr, offsets, E, d, f, max_rows, wq_down, s_down, y_perm,
+                               status, stream);
+  });
+  if (st != MOE_OK) return st;
+  return staged("moe_combine", [&] {
+    return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
+  });
 }
 
 // ---------------------------------------------------------------- buckets (expert parallelism)
@@ -544,7 +575,7 @@ int moe_expert_mlp_buckets(const void* x_rows, const int32_t* offsets, const int
 int moe_permute_fused(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
                       int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
                       int32_t* row_src, int32_t* row_pair, void* x_perm, int32_t* n_dropped,
-                      float* y32, void* ws, size_t ws_bytes, void* stream) {
+                      float* y32, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
   int st = check_routing_shape(T, E, k);
   if (st != MOE_OK) return st;
   if ((st = check_width(d)) != MOE_OK) return st;
@@ -560,7 +591,7 @@ int moe_permute_fused(const void* x, const int32_t* topk_idx, int64_t T, int64_t
   return cuda_status(moe::launch_permute_rows(
       static_cast<const uint8_t*>(x), (int)d * 2, nullptr, topk_idx, (int)T, (int)E, (int)k, C,
       counts, offsets, slot, row_src, static_cast<uint8_t*>(x_perm), nullptr, n_dropped,
-      static_cast<int32_t*>(ws), as_stream(stream), row_pair, y32, y32 ? (int)d : 0));
+      static_cast<int32_t*>(ws), as_stream(stream), row_pair, y32, y32 ? (int)d : 0, dev_status));
 }
 
 int moe_expert_gate_up_gather(const void* x, int64_t T, const int32_t* row_src,
@@ -661,20 +692,29 @@ int moe_layer_forward_fused(const void* x, const float* w_router, const float* b
   const int64_t max_rows = moe_max_rows(T, E, k, cf);
   cudaStream_t s = as_stream(stream);
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, field(MOE_WS_ROUTE),
-                      moe_route_workspace_size(T, d, E, k), status, stream)) != MOE_OK)
-    return st;
-  if ((st = moe_permute_fused(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src,
-                              row_pair, x_perm, n_dropped, y32, field(MOE_WS_PERMUTE),
-                              moe_permute_workspace_size(T, E, k), stream)) != MOE_OK)
-    return st;
-  if ((st = moe_expert_gate_up(x_perm, offsets, E, d, f, max_rows, w_gate, w_up, h, status,
-                               stream)) != MOE_OK)
-    return st;
-  if ((st = moe_expert_down_scatter(h, offsets, E, d, f, max_rows, w_down, row_pair, topk_w, k,
-                                    y32, status, stream)) != MOE_OK)
-    return st;
-  return moe_combine_finalize(y32, x, slot, T, d, k, y, stream);
+  st = staged("moe_route", [&] {
+    return moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, field(MOE_WS_ROUTE),
+                     moe_route_workspace_size(T, d, E, k), status, stream);
+  });
+  if (st != MOE_OK) return st;
+  st = staged("moe_permute_fused", [&] {
+    return moe_permute_fused(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src,
+                             row_pair, x_perm, n_dropped, y32, field(MOE_WS_PERMUTE),
+                             moe_permute_workspace_size(T, E, k), status, stream);
+  });
+  if (st != MOE_OK) return st;
+  st = staged("moe_expert_gate_up", [&] {
+    return moe_expert_gate_up(x_perm, offsets, E, d, f, max_rows, w_gate, w_up, h, status,
+                              stream);
+  });
+  if (st != MOE_OK) return st;
+  st = staged("moe_expert_down_scatter", [&] {
+    return moe_expert_down_scatter(h, offsets, E, d, f, max_rows, w_down, row_pair, topk_w, k,
+                                   y32, status, stream);
+  });
+  if (st != MOE_OK) return st;
+  return staged("moe_combine_finalize",
+                [&] { return moe_combine_finalize(y32, x, slot, T, d, k, y, stream); });
 }
 
 int moe_layer_forward(const void* x, const float* w_router, const float* bias, const void* w_gate,
@@ -713,17 +753,24 @@ int moe_layer_forward(const void* x, const float* w_router, const float* bias, c
   cudaStream_t s = as_stream(stream);
 
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((st = moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, rscratch,
-                      moe_route_workspace_size(T, d, E, k), status, stream)) != MOE_OK)
-    return st;
-  if ((st = moe_permute(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src, x_perm,
-                        n_dropped, pscratch, moe_permute_workspace_size(T, E, k), stream)) !=
-      MOE_OK)
-    return st;
-  if ((st = moe_expert_mlp(x_perm, offsets, E, d, f, max_rows, w_gate, w_up, w_down, h, y_perm,
-                           status, stream)) != MOE_OK)
-    return st;
-  return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
+  st = staged("moe_route", [&] {
+    return moe_route(x, w_router, bias, T, d, E, k, logits, topk_idx, topk_w, rscratch,
+                     moe_route_workspace_size(T, d, E, k), status, stream);
+  });
+  if (st != MOE_OK) return st;
+  st = staged("moe_permute", [&] {
+    return moe_permute(x, topk_idx, T, d, E, k, cf, counts, offsets, slot, row_src, x_perm,
+                       n_dropped, pscratch, moe_permute_workspace_size(T, E, k), status, stream);
+  });
+  if (st != MOE_OK) return st;
+  st = staged("moe_expert_mlp", [&] {
+    return moe_expert_mlp(x_perm, offsets, E, d, f, max_rows, w_gate, w_up, w_down, h, y_perm,
+                          status, stream);
+  });
+  if (st != MOE_OK) return st;
+  return staged("moe_combine", [&] {
+    return moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, stream);
+  });
 }
 
 }  // extern "C"

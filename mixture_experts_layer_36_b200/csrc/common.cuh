@@ -14,6 +14,7 @@ namespace moe {
 enum : int32_t {
   kDevErrWaitTimeout = 1,   // a bounded mbarrier wait gave up
   kDevErrBadOffsets = 2,    // offsets[E] beyond the row buffer, or not monotone
+  kDevErrBadRouting = 4,    // a top-k expert id outside [0, E) (checked builds: or repeated)
 };
 
 // Upper bound on any single wait inside a kernel, in nanoseconds.  A healthy

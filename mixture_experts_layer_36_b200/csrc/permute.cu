@@ -39,7 +39,8 @@ constexpr int kScatTokensLarge = 32;
 //    same expert (token order), and the chunk's per-expert histogram.
 __global__ void __launch_bounds__(kRankThreads)
     permute_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
-                        int32_t* __restrict__ rank, int32_t* __restrict__ chunk_hist) {
+                        int32_t* __restrict__ rank, int32_t* __restrict__ chunk_hist,
+                        int32_t* status) {
   __shared__ int32_t cnt[kRankWarps][256];
   __shared__ int32_t pairs[kChunk * 8];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -50,15 +51,27 @@ __global__ void __launch_bounds__(kRankThreads)
   for (int i = tid; i < nt * k; i += kRankThreads) pairs[i] = topk_idx[(size_t)chunk_t0 * k + i];
   __syncthreads();
 
-  // each warp walks its 8 tokens in order; lane j handles pair j
+  // each warp walks its 8 tokens in order; lane j handles pair j.  An expert
+  // id outside [0, E) (only possible for caller-given top-k tables) takes no
+  // bucket place: the scatter marks the pair dropped.
   const int w_t0 = warp * kTokPerWarp;
 #pragma unroll
   for (int i = 0; i < kTokPerWarp; ++i) {
     const int tt = w_t0 + i;
     if (tt < nt && lane < k) {
       const int e = pairs[tt * k + lane];
-      const int r = cnt[warp][e];
-      cnt[warp][e] = r + 1;        // experts are distinct within a token
+      int r = -1;
+      if (e >= 0 && e < E) {
+        r = cnt[warp][e];
+        cnt[warp][e] = r + 1;      // experts are distinct within a token
+      } else {
+        report(status, kDevErrBadRouting);
+      }
+#ifdef MOE_CHECKS
+      // checked builds: an expert listed twice for one token is reported
+      for (int j = 0; j < lane; ++j)
+        if (pairs[tt * k + j] == e) report(status, kDevErrBadRouting);
+#endif
       rank[(size_t)(chunk_t0 + tt) * k + lane] = r;
     }
     __syncwarp();
@@ -80,7 +93,8 @@ __global__ void __launch_bounds__(kRankThreads)
 
   for (int i = tid; i < nt * k; i += kRankThreads) {
     const int tt = i / k;
-    rank[(size_t)chunk_t0 * k + i] += cnt[tt / kTokPerWarp][pairs[i]];
+    const int e = pairs[i];
+    if (e >= 0 && e < E) rank[(size_t)chunk_t0 * k + i] += cnt[tt / kTokPerWarp][e];
   }
 }
 
@@ -166,8 +180,9 @@ __global__ void __launch_bounds__(kScatThreads)
     if (lane < k) {
       const size_t p = (size_t)t * k + lane;
       const int e = topk_idx[p];
-      const int sl = s_base[e] + slot[p];          // slot holds the in-chunk rank
-      const bool keep = (int64_t)sl < C;
+      const bool valid = e >= 0 && e < E;          // else dropped (rank kernel: -1)
+      const int sl = valid ? s_base[e] + slot[p] : 0;   // slot holds the in-chunk rank
+      const bool keep = valid && (int64_t)sl < C;
       slot[p] = keep ? sl : -1;
       if (keep) {
         my_row = s_off[e] + sl;
@@ -237,9 +252,11 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
                                 int32_t* counts, int32_t* offsets, int32_t* slot,
                                 int32_t* row_src, uint8_t* x_perm, float* perm_scale,
                                 int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
-                                int32_t* row_pair, float* zero_rows, int zero_cols) {
+                                int32_t* row_pair, float* zero_rows, int zero_cols,
+                                int32_t* status) {
   const int nchunks = (T + kChunk - 1) / kChunk;
-  permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist);
+  permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist,
+                                                       status);
   const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
   permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
       x, row_bytes, x_scale, topk_idx, slot, chunk_hist, nchunks, T, E, k, C, tpc, counts,
@@ -252,9 +269,11 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
 cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d,
                                   int E, int k, int64_t C, int32_t* counts, int32_t* offsets,
                                   int32_t* slot, int32_t* row_src, __nv_bfloat16* x_pad,
-                                  int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s) {
+                                  int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
+                                  int32_t* status) {
   const int nchunks = (T + kChunk - 1) / kChunk;
-  permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist);
+  permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist,
+                                                       status);
   const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
   uint8_t* xp = reinterpret_cast<uint8_t*>(x_pad);
   permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
@@ -269,11 +288,11 @@ cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_id
 cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d, int E,
                            int k, int64_t C, int32_t* counts, int32_t* offsets, int32_t* slot,
                            int32_t* row_src, __nv_bfloat16* x_perm, int32_t* n_dropped,
-                           int32_t* chunk_hist, cudaStream_t s) {
+                           int32_t* chunk_hist, cudaStream_t s, int32_t* status) {
   return launch_permute_rows(reinterpret_cast<const uint8_t*>(x), d * 2, nullptr, topk_idx, T, E,
                              k, C, counts, offsets, slot, row_src,
                              reinterpret_cast<uint8_t*>(x_perm), nullptr, n_dropped, chunk_hist,
-                             s, nullptr, nullptr, 0);
+                             s, nullptr, nullptr, 0, status);
 }
 
 }  // namespace moe

@@ -31,7 +31,7 @@ namespace moe {
 cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d, int E,
                            int k, int64_t C, int32_t* counts, int32_t* offsets, int32_t* slot,
                            int32_t* row_src, __nv_bfloat16* x_perm, int32_t* n_dropped,
-                           int32_t* chunk_hist, cudaStream_t s);
+                           int32_t* chunk_hist, cudaStream_t s, int32_t* status);
 size_t permute_scratch_bytes(int64_t T, int64_t E);
 }  // namespace moe
 
@@ -88,6 +88,6 @@ extern "C" int moe_permute_noalloc(const void* x, const int32_t* topk_idx, int64
   cudaError_t err = moe::launch_permute(
       static_cast<const __nv_bfloat16*>(x), topk_idx, (int)T, (int)d, (int)E, (int)k, C, counts,
       offsets, slot, row_src, static_cast<__nv_bfloat16*>(x_perm), n_dropped, scratch,
-      reinterpret_cast<cudaStream_t>(stream));
+      reinterpret_cast<cudaStream_t>(stream), nullptr);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

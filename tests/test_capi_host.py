@@ -107,8 +107,8 @@ def test_validation_codes_without_launch():
     need = moe.moe_permute_workspace_size(100, 8, 2)
     assert need > 0
     args = [FAKE, FAKE, 100, 128, 8, 2, 1.25, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE]
-    assert L.moe_permute(*args, need - 1, s) == WORKSPACE
-    assert L.moe_permute(*args[:6], -1.0, *args[7:], need, s) == INVALID
+    assert L.moe_permute(*args, need - 1, None, s) == WORKSPACE
+    assert L.moe_permute(*args[:6], -1.0, *args[7:], need, None, s) == INVALID
     # experts: widths must be multiples of 128
     assert L.moe_expert_gate_up(FAKE, FAKE, 8, 192, 256, 100, FAKE, FAKE, FAKE, None, s) \
         == UNSUPPORTED

@@ -111,3 +111,38 @@ def test_fused_layer_replays_in_cuda_graph():
     size = moe.moe_workspace_size_fused(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.cf)
     # the fused sums run in tile-completion order: equal up to fp32 rounding
     _replay_check(cfg, forward, size, lambda a, b: assert_bf16_close(f64(a), f64(b), "y"))
+
+
+def test_permute_out_of_range_expert_ids_are_dropped_and_reported():
+    """A caller-given top-k table with expert ids outside [0, E): the kernels'
+    bounds checks treat those pairs as dropped (slot -1, no bucket place, no
+    row written) and set status bit 4; every other pair is placed exactly as
+    the oracle places the valid pairs."""
+    import numpy as np
+    import oracle
+    from moe_testlib import bits, random_routing
+    T, d, E, k, cf = 300, 128, 8, 2, 0.75
+    idx = random_routing(T, E, k, seed=41)
+    bad = np.zeros_like(idx, dtype=bool)
+    bad[5, 0], bad[17, 1], bad[250, 0] = True, True, True
+    idx_bad = idx.copy()
+    idx_bad[5, 0], idx_bad[17, 1], idx_bad[250, 0] = -1, E, 1 << 20
+    g = torch.Generator().manual_seed(42)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = moe.moe_permute(x.cuda(), torch.from_numpy(idx_bad).cuda(), E, cf, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 4
+    # expected: the invalid pairs moved to an extra expert E, which is then dropped
+    C = oracle.capacity(T, E, k, cf)
+    idx_ref = np.where(bad, E, idx).astype(np.int32)
+    counts, offsets, slot, row_src, _ = oracle.permute(idx_ref, E + 1, C)
+    slot = np.where(bad, -1, slot)
+    N = int(offsets[E])
+    np.testing.assert_array_equal(out["slot"].cpu().numpy(), slot)
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), counts[:E])
+    np.testing.assert_array_equal(out["offsets"].cpu().numpy(), offsets[:E + 1])
+    np.testing.assert_array_equal(out["row_src"][:N].cpu().numpy(), row_src[:N])
+    np.testing.assert_array_equal(bits(out["x_perm"][:N]), oracle.dispatch(bits(x), row_src[:N]))
+    valid_drops = int(((slot < 0) & ~bad).sum())
+    assert out["n_dropped"].item() == valid_drops

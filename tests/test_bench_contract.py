@@ -1,0 +1,57 @@
+"""bench.py's output contract: one JSON line with the keys the benchmark
+promises, from the reference arm (the oracle on the host, CPU) and from the
+GPU arm (on a B200)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+BASE_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+             "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "e2e"}
+
+
+def _run(args, timeout):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                         capture_output=True, text=True, timeout=timeout)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+@pytest.mark.timeout(600)
+def test_reference_arm_json():
+    r = _run(["--impl", "reference", "--config", "tiny", "--steps", "2", "--warmup", "3"], 500)
+    assert BASE_KEYS <= set(r) and r["impl"] == "reference"
+    assert r["value"] > 0 and r["unit"] == "tokens/s" and r["higher_is_better"] is True
+    assert r["steps"] == 2 and r["warmup"] == 3 and r["n_gpus"] == 1
+    cb = r["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == r["value"]
+    assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["value"] == r["value"]
+    assert r["config"]["workload"].startswith("tiny")
+
+
+@pytest.mark.gpu
+@pytest.mark.timeout(900)
+@pytest.mark.parametrize("extra", [[], ["--fp8"], ["--fused"], ["--layout", "padded"]],
+                         ids=["bf16", "fp8", "fused", "padded"])
+def test_gpu_arm_json(extra):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    r = _run(["--config", "tiny", "--steps", "3", "--warmup", "3", "--no-cpu-baseline", *extra],
+             800)
+    assert BASE_KEYS <= set(r)
+    assert r["value"] > 0 and r["device_status"] == 0 and r["gpu_launches"] > 0
+    rf = r["roofline"]
+    assert rf["bound"] in ("hbm", "tensor") and rf["achieved"] > 0 and rf["peak"] > 0
+    assert abs(rf["frac"] - rf["achieved"] / rf["peak"]) < 1e-3
+    assert set(r["clocks"]) == {"sm_mhz", "sm_max_mhz", "reasons"}
+    e2e = r["e2e"]
+    assert e2e["value"] > 0 and e2e["h2d_bytes_per_step"] == 64 * 128 * 2
+    assert e2e["d2h_bytes_per_step"] == 64 * 128 * 2
+    assert set(r["stages_ms"]) >= {"route", "permute", "gate_up", "down", "combine"}

@@ -43,7 +43,13 @@ namespace moe {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;                 // one 128-byte swizzle atom of bf16 along K
-constexpr int kGemmThreads = 192;
+// Threads: warp 0 producer, warp 1 MMA issuer, then the epilogue warps.
+// SwiGLU kernels (bf16 h rows, stored without a staging tile) drain each
+// accumulator with 8 epilogue warps, two per TMEM lane quarter on separate
+// column halves, so that short-K shapes are not bound by the epilogue.
+constexpr int kEpiWarpsSwiglu = 8;
+__host__ __device__ constexpr int epi_warps(bool swiglu) { return swiglu ? kEpiWarpsSwiglu : 4; }
+__host__ __device__ constexpr int gemm_threads(bool swiglu) { return 64 + 32 * epi_warps(swiglu); }
 constexpr int kChunkBytes = 64 * kBK * 2;   // one B chunk: 64 N x 64 K bf16 = 8 KB
 
 // ---------------------------------------------------------------- epilogue stores
@@ -181,7 +187,7 @@ __device__ __forceinline__ void decode_tile(const GemmShared& sh, int tile, int 
 __device__ __forceinline__ void gemm_setup(GemmShared& sh, int stages, int full_count,
                                            int tmem_cols, const int32_t* offsets, int E,
                                            int n_tiles, int max_rows, int32_t* status, int warp,
-                                           int lane, const FuseArgs& fz) {
+                                           int lane, const FuseArgs& fz, int epi_count) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&sh.full_bar[s], full_count);
@@ -189,7 +195,7 @@ __device__ __forceinline__ void gemm_setup(GemmShared& sh, int stages, int full_
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sh.tfull_bar[a], 1);
-      mbar_init(&sh.tempty_bar[a], 4);
+      mbar_init(&sh.tempty_bar[a], epi_count);
     }
     mbar_init(&sh.drain_bar, 1);
     sh.abort_flag = 0;
@@ -404,6 +410,10 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
   const int total_tiles = sh.tile_prefix[E];
   const uint32_t tmem_base = sh.tmem_base;
   const int q = warp & 3;                 // TMEM lane quarter this warp may read
+  // with 8 epilogue warps, group 0 (warps 2..5) and group 1 (6..9) take
+  // alternate 32-column chunks
+  constexpr int kGroups = epi_warps(SWIGLU) / 4;
+  const int grp = (warp - 2) / 4;
   int lt = 0;
   for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
     int e, m, n;
@@ -432,7 +442,7 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
       __nv_bfloat16* o =
           static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out + (size_t)n * kOutCols;
 #pragma unroll 1
-      for (int c = 0; c < BN / 2 / 32; ++c) {
+      for (int c = grp; c < BN / 2 / 32; c += kGroups) {
         uint32_t g[32], u[32], pk[16];
         tmem_ld_32x32b_x32(tbase + c * 32, g);
         tmem_ld_32x32b_x32(tbase + BN / 2 + c * 32, u);
@@ -481,7 +491,7 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
 
 // ---------------------------------------------------------------- bf16 weights
 template <int BN, bool SWIGLU, int FUSE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
                         const __grid_constant__ CUtensorMap tmB0,
@@ -500,7 +510,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nkb = K / kBK;
 
   gemm_setup(sh, Cfg::kStages, 1, Cfg::kTmemCols, offsets, E, n_tiles, max_rows, status, warp,
-             lane, fz);
+             lane, fz, epi_warps(SWIGLU));
   if (warp == 1 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmA64);
@@ -575,7 +585,7 @@ struct E4m3Cfg {
 };
 
 template <int BN, bool SWIGLU, int FUSE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
     grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,     // codes [rows, K]
                              const __grid_constant__ CUtensorMap tmA64,
                              const __grid_constant__ CUtensorMap tmB0,    // codes [E, N, K]
@@ -597,7 +607,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nkb = K / Cfg::kBKe;
 
   gemm_setup(sh, Cfg::kStages, 1, Cfg::kTmemCols, offsets, E, n_tiles, max_rows, status, warp,
-             lane, fz);
+             lane, fz, epi_warps(SWIGLU));
   if (warp == 1 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmA64);
@@ -743,7 +753,7 @@ __device__ __forceinline__ void decode_pair_tile(const PairShared& sh, int tile,
 // kind::f8f6f4; tmB0h / tmB1h are 64-row weight boxes for the half tiles'
 // 64 + 64 column split; the epilogue applies the row and column scales.
 template <bool SWIGLU, bool E4M3, int FUSE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
                              const __grid_constant__ CUtensorMap tmB0,
@@ -783,7 +793,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sh.tfull_bar[a], 1);
-      mbar_init(&sh.tempty_bar[a], 8);       // 4 epilogue warps in each CTA
+      mbar_init(&sh.tempty_bar[a], 2 * epi_warps(SWIGLU));   // the epilogue warps of both CTAs
     }
     mbar_init(&sh.drain_bar, 1);
     sh.abort_flag = 0;
@@ -979,8 +989,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_wait(&sh.drain_bar, 0, &sh.never);
     }
   } else {
-    // -------------------------------------------------- epilogue (warps 2..5, both CTAs)
+    // -------------------------------------------------- epilogue (warps 2.., both CTAs)
     const int q = warp & 3;
+    constexpr int kGroups = epi_warps(SWIGLU) / 4;     // warp groups splitting the chunks
+    const int grp = (warp - 2) / 4;
     int lt = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++lt) {
       int e, m, n;
@@ -1009,7 +1021,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int c0 = n * kOutCols;
           __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out + c0;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c)
+          for (int c = grp; c < 4; c += kGroups)
             swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 128 + c * 32, o + c * 32, n_out,
                                      nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
         } else if (FUSE == kFuseScatter) {
@@ -1047,7 +1059,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int c0 = n * kOutCols + hh * 64;
           __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out + c0;
 #pragma unroll 1
-          for (int c = 0; c < 2; ++c)
+          for (int c = grp; c < 2; c += kGroups)
             swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 64 + c * 32, o + c * 32, n_out,
                                      nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
         } else if (FUSE == kFuseScatter) {
@@ -1111,7 +1123,7 @@ static cudaError_t launch_gemm_t(int slot, const CUtensorMap& a, const CUtensorM
   long long ub = row_tiles * n_tiles;
   int grid = (int)(ub < di->sms ? ub : di->sms);
   if (grid < 1) grid = 1;
-  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, offsets, E, K, n_out,
+  kern<<<grid, gemm_threads(SWIGLU), Cfg::kSmemBytes, s>>>(a, a64, b0, b1, offsets, E, K, n_out,
                                                      max_rows, out, status, fz);
   return cudaGetLastError();
 }
@@ -1142,7 +1154,7 @@ static cudaError_t launch_gemm_pair_t(int slot, const CUtensorMap& a, const CUte
   if (pairs < 1) pairs = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.blockDim = dim3(gemm_threads(SWIGLU), 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1308,7 +1320,8 @@ static cudaError_t launch_gemm_e4m3_t(int slot, const CUtensorMap& a, const CUte
   long long ub = row_tiles * n_tiles;
   int grid = (int)(ub < di->sms ? ub : di->sms);
   if (grid < 1) grid = 1;
-  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, s>>>(a, a64, b0, b1, row_scale, s0, s1, offsets, E,
+  kern<<<grid, gemm_threads(SWIGLU), Cfg::kSmemBytes, s>>>(a, a64, b0, b1, row_scale, s0, s1,
+                                                           offsets, E,
                                                    K, n_out, max_rows, out, status, fz);
   return cudaGetLastError();
 }

@@ -44,31 +44,43 @@ namespace moe {
 constexpr int kBM = 128;
 constexpr int kBK = 64;                 // one 128-byte swizzle atom of bf16 along K
 // Threads: warp 0 producer, warp 1 MMA issuer, then the epilogue warps.
-// SwiGLU kernels (bf16 h rows, stored without a staging tile) drain each
-// accumulator with 8 epilogue warps, two per TMEM lane quarter on separate
-// column halves, so that short-K shapes are not bound by the epilogue.
-constexpr int kEpiWarpsSwiglu = 8;
-__host__ __device__ constexpr int epi_warps(bool swiglu) { return swiglu ? kEpiWarpsSwiglu : 4; }
+// Each accumulator is drained by 8 epilogue warps, two per TMEM lane quarter
+// on alternate 32-column chunks, so that short-K shapes are not bound by the
+// epilogue.  The fp32 (down GEMM) epilogue stages rows through one padded
+// 16-row shared tile per warp.
+constexpr int kEpiWarps = 8;
+__host__ __device__ constexpr int epi_warps(bool) { return kEpiWarps; }
 __host__ __device__ constexpr int gemm_threads(bool swiglu) { return 64 + 32 * epi_warps(swiglu); }
 constexpr int kChunkBytes = 64 * kBK * 2;   // one B chunk: 64 N x 64 K bf16 = 8 KB
 
 // ---------------------------------------------------------------- epilogue stores
 // Each epilogue thread owns one accumulator row; a warp owns 32 rows.  fp32
-// rows are written through a padded 32 x 32 staging tile in shared memory (one
-// per warp) so that each store instruction covers a whole 128-byte row segment
-// instead of 16 B in each of 32 rows.
-constexpr int kStageWords = 32 * 33;     // per warp, 32-bit words
+// rows are written through a padded ROWS x 32 staging tile in shared memory
+// (one per warp; ROWS = 16 takes the warp's rows in two halves, for kernels
+// whose operand ring leaves less room) so that each store instruction covers a
+// whole 128-byte row segment instead of 16 B in each of 32 rows.
+__host__ __device__ constexpr int stage_words(int rows) { return rows * 33; }   // per warp
 
 // fp32: row `lane` holds v[0..31]; rows [0, nvalid) of the warp are stored
 // to out_row0 + r * ld (columns [0, 32)).
+template <int ROWS>
 __device__ __forceinline__ void store_chunk_f32(const uint32_t (&v)[32], uint32_t* stage,
                                                 float* out_row0, size_t ld, int nvalid,
                                                 int lane) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) stage[lane * 33 + j] = v[j];
-  __syncwarp();
-  for (int r = 0; r < nvalid; ++r) out_row0[(size_t)r * ld + lane] = __uint_as_float(stage[r * 33 + lane]);
-  __syncwarp();
+  for (int part = 0; part < 32 / ROWS; ++part) {
+    const int r0 = part * ROWS;
+    if (r0 >= nvalid) break;
+    if (lane / ROWS == part) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) stage[(lane % ROWS) * 33 + j] = v[j];
+    }
+    __syncwarp();
+    const int r1 = min(nvalid, r0 + ROWS);
+    for (int r = r0; r < r1; ++r)
+      out_row0[(size_t)r * ld + lane] = __uint_as_float(stage[(r - r0) * 33 + lane]);
+    __syncwarp();
+  }
 }
 
 // fp32 scatter-add (the fused combine): row `lane` holds v[0..31] of a
@@ -76,25 +88,34 @@ __device__ __forceinline__ void store_chunk_f32(const uint32_t (&v)[32], uint32_
 // rows, y32_col0[t * ld + c] += w * v[c].  Staged through the padded tile so
 // that each instruction covers four rows with one 16-byte vector add per lane
 // (8 lanes per row, 32 consecutive columns).
+template <int ROWS>
 __device__ __forceinline__ void scatter_chunk_f32(const uint32_t (&v)[32], uint32_t* stage,
                                                   float* y32_col0, size_t ld, int my_t,
                                                   float my_w, int nvalid, int lane) {
-#pragma unroll
-  for (int j = 0; j < 32; ++j) stage[lane * 33 + j] = v[j];
-  __syncwarp();
   const int c = (lane % 8) * 4;
-  for (int r0 = 0; r0 < nvalid; r0 += 4) {
-    const int r = r0 + lane / 8;
-    const int t = __shfl_sync(0xffffffffu, my_t, r);
-    const float w = __shfl_sync(0xffffffffu, my_w, r);
-    if (r < nvalid) {
-      const uint32_t* src = stage + r * 33 + c;
-      const float4 add = make_float4(w * __uint_as_float(src[0]), w * __uint_as_float(src[1]),
-                                     w * __uint_as_float(src[2]), w * __uint_as_float(src[3]));
-      atomicAdd(reinterpret_cast<float4*>(y32_col0 + (size_t)t * ld + c), add);
+#pragma unroll
+  for (int part = 0; part < 32 / ROWS; ++part) {
+    const int h0 = part * ROWS;
+    if (h0 >= nvalid) break;
+    if (lane / ROWS == part) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) stage[(lane % ROWS) * 33 + j] = v[j];
     }
+    __syncwarp();
+    const int h1 = min(nvalid, h0 + ROWS);
+    for (int r0 = h0; r0 < h1; r0 += 4) {
+      const int r = r0 + lane / 8;                     // < 32: a lane of this warp
+      const int t = __shfl_sync(0xffffffffu, my_t, r);
+      const float w = __shfl_sync(0xffffffffu, my_w, r);
+      if (r < h1) {
+        const uint32_t* src = stage + (r - h0) * 33 + c;
+        const float4 add = make_float4(w * __uint_as_float(src[0]), w * __uint_as_float(src[1]),
+                                       w * __uint_as_float(src[2]), w * __uint_as_float(src[3]));
+        atomicAdd(reinterpret_cast<float4*>(y32_col0 + (size_t)t * ld + c), add);
+      }
+    }
+    __syncwarp();
   }
-  __syncwarp();
 }
 
 // bf16: row `lane` holds pk[0..15] (32 bf16), stored directly as four
@@ -146,7 +167,8 @@ struct GemmCfg {
   static constexpr int kStages = (BN == 256) ? 4 : 6;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kStagingOff = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kStagingOff + 4 * kStageWords * 4 + 1024;
+  static constexpr int kSmemBytes =
+      kStagingOff + (SWIGLU ? 0 : kEpiWarps * stage_words(16) * 4) + 1024;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
   static constexpr uint32_t kIdesc64 = idesc_bf16_f32(kBM / 2, BN, /*b_mn_major=*/true);
 };
@@ -435,7 +457,7 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
     const size_t row0 = (size_t)sh.row_off[e] + first;
     const size_t sc_off = (size_t)weight_index(fz, e) * n_out + (size_t)n * kOutCols;
     const float sr = (SCALED && lane < nvalid) ? row_scale[row0 + lane] : 0.f;
-    uint32_t* stage = reinterpret_cast<uint32_t*>(staging) + q * kStageWords;
+    uint32_t* stage = reinterpret_cast<uint32_t*>(staging) + (warp - 2) * stage_words(16);
     const uint32_t tbase =
         tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * BN);
     if (SWIGLU) {
@@ -465,22 +487,22 @@ __device__ __forceinline__ void epilogue_role(GemmShared& sh, uint8_t* staging, 
       }
       float* o = fz.y32 + (size_t)n * kOutCols;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = grp; c < BN / 32; c += kGroups) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + c * 32, v);
         tmem_ld_wait();
         if (SCALED) apply_scales(v, sc0 + sc_off + c * 32, sr);
-        scatter_chunk_f32(v, stage, o + c * 32, n_out, my_t, my_w, nvalid, lane);
+        scatter_chunk_f32<16>(v, stage, o + c * 32, n_out, my_t, my_w, nvalid, lane);
       }
     } else {
       float* o = static_cast<float*>(out_raw) + row0 * n_out + (size_t)n * kOutCols;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = grp; c < BN / 32; c += kGroups) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + c * 32, v);
         tmem_ld_wait();
         if (SCALED) apply_scales(v, sc0 + sc_off + c * 32, sr);
-        store_chunk_f32(v, stage, o + c * 32, n_out, nvalid, lane);
+        store_chunk_f32<16>(v, stage, o + c * 32, n_out, nvalid, lane);
       }
     }
     tc_fence_before();
@@ -579,7 +601,8 @@ struct E4m3Cfg {
   static constexpr int kStages = (BN == 256) ? 4 : 6;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kStagingOff = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kStagingOff + 4 * kStageWords * 4 + 1024;
+  static constexpr int kSmemBytes =
+      kStagingOff + (SWIGLU ? 0 : kEpiWarps * stage_words(16) * 4) + 1024;
   static constexpr uint32_t kIdesc = idesc_e4m3_f32(kBM, BN);
   static constexpr uint32_t kIdesc64 = idesc_e4m3_f32(kBM / 2, BN);
 };
@@ -702,7 +725,7 @@ __device__ __forceinline__ void f32_chunk_store(uint32_t t, uint32_t* stage, flo
   tmem_ld_32x32b_x32(t, v);
   tmem_ld_wait();
   if (SCALED) apply_scales(v, sc, sr);
-  store_chunk_f32(v, stage, out_row0, ld, nvalid, lane);
+  store_chunk_f32<32>(v, stage, out_row0, ld, nvalid, lane);
 }
 
 template <bool SCALED>
@@ -714,12 +737,19 @@ __device__ __forceinline__ void f32_chunk_scatter(uint32_t t, uint32_t* stage, f
   tmem_ld_32x32b_x32(t, v);
   tmem_ld_wait();
   if (SCALED) apply_scales(v, sc, sr);
-  scatter_chunk_f32(v, stage, y32_col0, ld, my_t, my_w, nvalid, lane);
+  scatter_chunk_f32<32>(v, stage, y32_col0, ld, my_t, my_w, nvalid, lane);
 }
 
 constexpr int kPairStages = 6;
 constexpr int kPairStageBytes = 2 * kBM * kBK * 2;      // A 16 KB + half of B 16 KB
-constexpr int kPairStagingOff = kPairStages * kPairStageBytes;
+// the fp32 kernel gives one ring slot to the epilogue warps' staging tiles
+__host__ __device__ constexpr int pair_stages(bool swiglu) { return swiglu ? kPairStages : kPairStages - 1; }
+__host__ __device__ constexpr int pair_staging_off(bool swiglu) {
+  return pair_stages(swiglu) * kPairStageBytes;
+}
+__host__ __device__ constexpr int pair_smem_bytes(bool swiglu) {
+  return pair_staging_off(swiglu) + (swiglu ? 0 : kEpiWarps * stage_words(32) * 4) + 1024;
+}
 
 struct PairShared {
   uint64_t full_bar[kPairStages];
@@ -774,6 +804,7 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
   constexpr uint32_t kIdescHalf = E4M3 ? idesc_e4m3_f32(kBM, 256)
                                        : idesc_bf16_f32(kBM, 256, /*b_mn_major=*/true);
   constexpr int kTmemCols = 512;
+  constexpr int kStagesP = pair_stages(SWIGLU);
   extern __shared__ uint8_t dsmem_raw[];
   __shared__ PairShared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -787,7 +818,7 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
   const int nkb = K / kKb;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPairStages; ++s) {
+    for (int s = 0; s < kStagesP; ++s) {
       mbar_init(&sh.full_bar[s], 1);
       mbar_init(&sh.empty_bar[s], 1);
     }
@@ -861,8 +892,8 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
     if (gather || lane == 0) {
       // ------------------------------------------------ TMA producer (both CTAs)
       int it = 0;
-      int last_it[kPairStages];
-      for (int s = 0; s < kPairStages; ++s) last_it[s] = -1;
+      int last_it[kStagesP];
+      for (int s = 0; s < kStagesP; ++s) last_it[s] = -1;
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
         int e, m, n;
@@ -882,8 +913,8 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
           }
         }
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % kPairStages;
-          const uint32_t ph = (it / kPairStages) & 1;
+          const int s = it % kStagesP;
+          const uint32_t ph = (it / kStagesP) & 1;
           bool good = true;
           if (lane == 0) good = mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag);
           if (gather) good = __shfl_sync(0xffffffffu, good, 0);
@@ -940,9 +971,9 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
         if (!ok) give_up();
         if (leader) {
           // both CTAs' copies of every issued phase count on the leader's barriers
-          for (int s = 0; s < kPairStages; ++s)
+          for (int s = 0; s < kStagesP; ++s)
             if (last_it[s] >= 0)
-              mbar_wait(&sh.full_bar[s], (last_it[s] / kPairStages) & 1, &sh.never);
+              mbar_wait(&sh.full_bar[s], (last_it[s] / kStagesP) & 1, &sh.never);
         }
       }
     }
@@ -962,8 +993,8 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * 256);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % kPairStages;
-          const uint32_t ph = (it / kPairStages) & 1;
+          const int s = it % kStagesP;
+          const uint32_t ph = (it / kStagesP) & 1;
           if (!mbar_wait(&sh.full_bar[s], ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * kPairStageBytes);
@@ -1007,7 +1038,7 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
       const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
-      uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kPairStagingOff) + q * kStageWords;
+      uint32_t* stage = reinterpret_cast<uint32_t*>(smem + pair_staging_off(SWIGLU)) + (warp - 2) * stage_words(32);
       // E4M3: column scales from (e, column), the row's scale per thread
       const int ew = weight_index(fz, e);
       const float* cs0 = E4M3 ? col_scale0 + (size_t)ew * n_out : nullptr;
@@ -1034,14 +1065,14 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
             my_w = fz.topk_w[p];
           }
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c)
+          for (int c = grp; c < 8; c += kGroups)
             f32_chunk_scatter<E4M3>(tbase + c * 32, stage, fz.y32 + c0 + c * 32, n_out, nvalid,
                                     lane, cs0 + c0 + c * 32, sr, my_t, my_w);
         } else {
           const int c0 = n * kOutCols;
           float* o = static_cast<float*>(out_raw) + row0 * n_out + c0;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c)
+          for (int c = grp; c < 8; c += kGroups)
             f32_chunk_store<E4M3>(tbase + c * 32, stage, o + c * 32, n_out, nvalid, lane,
                                   cs0 + c0 + c * 32, sr);
         }
@@ -1072,14 +1103,14 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
             my_w = fz.topk_w[p];
           }
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c)
+          for (int c = grp; c < 4; c += kGroups)
             f32_chunk_scatter<E4M3>(tbase + c * 32, stage, fz.y32 + c0 + c * 32, n_out, nvalid,
                                     lane, cs0 + c0 + c * 32, sr, my_t, my_w);
         } else {
           const int c0 = n * kOutCols + hh * 128;
           float* o = static_cast<float*>(out_raw) + row0 * n_out + c0;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c)
+          for (int c = grp; c < 4; c += kGroups)
             f32_chunk_store<E4M3>(tbase + c * 32, stage, o + c * 32, n_out, nvalid, lane,
                                   cs0 + c0 + c * 32, sr);
         }
@@ -1136,7 +1167,7 @@ static cudaError_t launch_gemm_pair_t(int slot, const CUtensorMap& a, const CUte
                                       const FuseArgs& fz, const CUtensorMap* b0h,
                                       const CUtensorMap* b1h, const float* row_scale,
                                       const float* cs0, const float* cs1) {
-  constexpr int kSmem = kPairStagingOff + 4 * kStageWords * 4 + 1024;
+  constexpr int kSmem = pair_smem_bytes(SWIGLU);
   DeviceInfo* di = nullptr;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;

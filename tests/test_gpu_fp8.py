@@ -293,14 +293,17 @@ def test_layer_forward_fp8_matches_oracle(cfg):
         np.testing.assert_array_equal(bits(y)[dropped], x_bits[dropped])
 
 
-DECODE = [configs.DECODE.with_tokens(t) for t in configs.DECODE_T]
+FULL = [configs.MIXTRAL, configs.FINE, configs.SKEWED] + \
+    [configs.DECODE.with_tokens(t) for t in configs.DECODE_T]
 
 
-@pytest.mark.parametrize("cfg", DECODE, ids=[c.name for c in DECODE])
-def test_decode_fp8_full_size_sampled(cfg):
-    """Decode-sized layer with FP8 experts quantized on the GPU: routing exact
-    for every token; the weight codes of the experts that two sampled tokens
-    use bit-exact; those tokens' outputs from the oracle."""
+@pytest.mark.parametrize("cfg", FULL, ids=[c.name for c in FULL])
+def test_fp8_full_size_sampled(cfg):
+    """Full-size layer with FP8 experts quantized on the GPU, in the launch
+    configuration the benchmark times: routing and slots exact for every
+    token; for two sampled tokens (and, where the capacity drops some, one
+    whose every pair is dropped) the weight codes of their experts bit-exact
+    and their outputs from the oracle."""
     torch.cuda.empty_cache()
     w = synth.make_weights(cfg, "cuda")
     x = synth.make_tokens(cfg, "cuda")
@@ -313,18 +316,27 @@ def test_decode_fp8_full_size_sampled(cfg):
     o_idx, o_w = oracle.topk(gl, cfg.k)
     np.testing.assert_array_equal(_ws(ws, "topk_idx", cfg).cpu().numpy(), o_idx)
     C = oracle.capacity(cfg.T, cfg.E, cfg.k, cfg.cf)
-    _, offsets, slot, _, _ = oracle.permute(o_idx, cfg.E, C)
+    _, offsets, slot, _, n_drop = oracle.permute(o_idx, cfg.E, C)
     np.testing.assert_array_equal(_ws(ws, "slot", cfg).cpu().numpy(), slot)
+    assert _ws(ws, "n_dropped", cfg).item() == n_drop
 
     rng = np.random.default_rng(cfg.seed + 1)
-    toks = np.sort(rng.choice(cfg.T, size=2, replace=False))
+    toks = list(np.sort(rng.choice(cfg.T, size=2, replace=False)))
+    all_dropped = np.flatnonzero((slot < 0).all(axis=1))
+    if len(all_dropped):
+        toks.append(int(all_dropped[0]))
     x_bits = bits(x)
     h_gpu = _ws(ws, "h", cfg)
     y_ref = np.zeros((len(toks), cfg.d))
     for i, t in enumerate(toks):
+        if (slot[t] < 0).all():
+            y_ref[i] = oracle.bits_to_f64(x_bits[t:t + 1])[0]
+            continue
         xq, sx = oracle.quantize_rows_fp8(x_bits[t:t + 1])
         a = deq_rows(xq, sx)
         for j in range(cfg.k):
+            if slot[t, j] < 0:
+                continue
             e = int(o_idx[t, j])
             mats = []
             for n in ("w_gate", "w_up", "w_down"):
@@ -338,6 +350,11 @@ def test_decode_fp8_full_size_sampled(cfg):
             assert_bf16_rounding_close(f64(h_row), h_ref, "h (sampled)")
             hq, sh = oracle.quantize_rows_fp8(bits(h_row))
             y_ref[i] += o_w[t, j] * oracle.matmul_f64(deq_rows(hq, sh), mats[2])[0]
-    assert_bf16_close(f64(y[torch.from_numpy(toks).cuda().long()]), y_ref, "y (sampled)")
+    y_s = y[torch.tensor(toks, device="cuda").long()]
+    moe_rows = np.array([not (slot[t] < 0).all() for t in toks])
+    # the expert outputs against the oracle (tolerance from their own rms);
+    # all-dropped tokens passed through bit for bit
+    assert_bf16_close(f64(y_s)[moe_rows], y_ref[moe_rows], "y (sampled)")
+    np.testing.assert_array_equal(bits(y_s)[~moe_rows], x_bits[np.array(toks)[~moe_rows]])
     del w, x, y, ws, qw
     torch.cuda.empty_cache()

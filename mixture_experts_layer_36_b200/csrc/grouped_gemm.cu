@@ -23,9 +23,9 @@
 // search.  Inside an expert the row tile varies fastest, so CTAs running at
 // the same time share each weight tile through L2.
 //
-// Roles (192 threads): warp 0 lane 0 issues TMA into a ring of smem stages,
+// Roles (320 threads): warp 0 lane 0 issues TMA into a ring of smem stages,
 // warp 1 lane 0 issues tcgen05.mma into one of two TMEM accumulators, warps
-// 2..5 drain the other accumulator (tcgen05.ld -> SwiGLU -> bf16 stores), so
+// 2..9 drain the other accumulator (tcgen05.ld -> SwiGLU -> bf16 stores), so
 // the epilogue of tile i overlaps the main loop of tile i+1.
 //
 // FP8 experts (grouped_gemm_e4m3_kernel): the same tiles and roles on e4m3
@@ -414,7 +414,7 @@ __device__ __forceinline__ void mma_role(GemmShared& sh, uint8_t* smem, int E, i
   mbar_wait(&sh.drain_bar, 0, &sh.never);
 }
 
-// Epilogue (warps 2..5): drain accumulator buffer lt & 1 of each tile
+// Epilogue (warps 2..9): drain accumulator buffer lt & 1 of each tile
 // (tcgen05.ld -> [column scales] -> SwiGLU + bf16 stores, or fp32 stores).
 // Fusion compiled into a kernel instance: none, gather (GEMM 1's producer
 // fetches token rows by row_src), scatter (GEMM 2's epilogue adds weighted rows

@@ -97,6 +97,44 @@ def test_route_ties_take_lower_index():
     assert np.max(np.abs(w.cpu().double().numpy() - o_w)) <= WEIGHT_ATOL
 
 
+# More row tiles (128 tokens each) than any B200 has SMs: the router GEMM runs
+# without a K split and its epilogue does the top-k itself.
+T_UNSPLIT = 148 * 128 + 37
+
+
+@pytest.mark.parametrize("E,k,with_bias", [(8, 2, False), (64, 6, True), (200, 8, True),
+                                            (256, 8, False), (33, 3, True)])
+def test_route_unsplit_matches_oracle(E, k, with_bias):
+    d = 128
+    g = torch.Generator().manual_seed(E * 10 + k)
+    x = torch.randn(T_UNSPLIT, d, generator=g).to(torch.bfloat16)
+    wr = torch.randn(d, E, generator=g) / d ** 0.5
+    bias = (torch.randn(E, generator=g) * 0.1) if with_bias else None
+    logits, idx, w = moe.moe_route(x.cuda(), wr.cuda(), None if bias is None else bias.cuda(), k)
+    torch.cuda.synchronize()
+    ref64 = oracle.router_logits(bits(x), wr.numpy(), None if bias is None else bias.numpy())
+    gl = logits.cpu().numpy()
+    assert_logits_close(gl, ref64)
+    o_idx, o_w = oracle.topk(gl, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), o_idx)
+    assert np.max(np.abs(w.cpu().double().numpy() - o_w)) <= WEIGHT_ATOL
+    independent_topk_check(ref64, idx.cpu().numpy(), k)
+
+
+def test_route_unsplit_ties_take_lower_index():
+    E, k, d = 16, 4, 128
+    x = torch.zeros(T_UNSPLIT, d, dtype=torch.bfloat16, device="cuda")
+    x[::3] = torch.randn(x[::3].shape, device="cuda").to(torch.bfloat16)  # some untied rows
+    wr = torch.randn(d, E, device="cuda")
+    bias = torch.tensor([0.5, 1.0, 1.0, 0.5, 2.0, 1.0, 2.0, 0.0] * 2, device="cuda")
+    logits, idx, w = moe.moe_route(x, wr, bias, k)
+    gl = logits.cpu().numpy()
+    o_idx, o_w = oracle.topk(gl, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), o_idx)
+    assert o_idx[1].tolist() == [4, 6, 12, 14]            # an all-tied row
+    assert np.max(np.abs(w.cpu().double().numpy() - o_w)) <= WEIGHT_ATOL
+
+
 # ----------------------------------------------------------------------------- stage: permute
 
 PERM_CASES = [(64, 128, 8, 2, 1.25), (1000, 256, 64, 6, 1.0), (777, 128, 256, 8, 1.25),

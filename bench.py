@@ -31,9 +31,25 @@ from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
 
 METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 8     # router 3, permute 2, gate/up GEMM 1, down GEMM 1, combine 1
-KERNELS_PER_STEP_FP8 = 10   # + the row quantizer on x and on h
+ROUTER_TILE_M = 128      # tokens per router GEMM row tile
 FP8_OVER_BF16 = 2.0      # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
+
+
+def launches_per_step(cfg, sms, fp8=False, padded=False, fused=False):
+    """libmoe kernels one layer step launches: router weight split, router
+    GEMM and top-k (the top-k runs in the GEMM's epilogue when the router's K
+    is not split, i.e. when there are at least as many 128-token row tiles as
+    half the SMs); permutation rank and scatter (+ the padded layout's fill);
+    the FP8 row quantizers on x and on h; the two expert GEMMs; the combine
+    (the fused path's finalize)."""
+    if cfg.T == 0:
+        return 0
+    m_tiles = -(-cfg.T // ROUTER_TILE_M)
+    splits = max(1, min(min(sms, 256) // m_tiles, cfg.d // 64))
+    n = 2 if splits == 1 else 3
+    n += 3 if padded else 2
+    n += 2 if fp8 else 0
+    return n + 2 + 1
 
 
 def moe_max_rows_host(cfg):
@@ -468,7 +484,8 @@ def main():
             layer.step()
         torch.cuda.synchronize()
         assert int(layer.status.item()) == 0
-        kps = KERNELS_PER_STEP_FP8 if args.fp8 else KERNELS_PER_STEP
+        sms = torch.cuda.get_device_properties(local_rank).multi_processor_count
+        kps = launches_per_step(cfg, sms, args.fp8, args.layout == "padded", args.fused)
         print(json.dumps({"profile_run": cfg.name, "launches": kps * (args.warmup + args.steps)}))
         return
 
@@ -599,7 +616,9 @@ def main():
                         " (one-shot C-ABI call)") +
                        "; every step copies x from pinned host memory and y back, on copy "
                        "streams overlapping adjacent steps' compute"},
-        "gpu_launches": (KERNELS_PER_STEP_FP8 if args.fp8 else KERNELS_PER_STEP) * K,
+        "gpu_launches": launches_per_step(
+            cfg, torch.cuda.get_device_properties(local_rank).multi_processor_count, args.fp8,
+            args.layout == "padded", args.fused) * K,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wh = host_weights(r["layer"].w)

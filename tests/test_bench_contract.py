@@ -55,3 +55,21 @@ def test_gpu_arm_json(extra):
     assert e2e["value"] > 0 and e2e["h2d_bytes_per_step"] == 64 * 128 * 2
     assert e2e["d2h_bytes_per_step"] == 64 * 128 * 2
     assert set(r["stages_ms"]) >= {"route", "permute", "gate_up", "down", "combine"}
+
+
+def test_launches_per_step():
+    """The gpu_launches arithmetic (checked against the CUDA profiler's count by
+    tests/test_gpu_launch_count.py): 8 launches with a split router K, one fewer
+    when the router's top-k runs in its GEMM epilogue, +2 row quantizers for
+    FP8 experts, +1 fill for the padded layout."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_36_b200 import configs
+    assert bench.launches_per_step(configs.MIXTRAL, 148) == 8              # 32 row tiles
+    assert bench.launches_per_step(configs.SKEWED, 148) == 7               # 128 row tiles
+    assert bench.launches_per_step(configs.SKEWED, 148, fp8=True) == 9
+    assert bench.launches_per_step(configs.FINE, 148, padded=True) == 9
+    assert bench.launches_per_step(configs.FINE, 148, fused=True) == 8
+    assert bench.launches_per_step(configs.DECODE.with_tokens(16), 148, fp8=True) == 10
+    assert bench.launches_per_step(configs.TINY.with_tokens(0), 148) == 0

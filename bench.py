@@ -32,6 +32,7 @@ from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
 METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ROUTER_TILE_M = 128      # tokens per router GEMM row tile
+PAIR_MIN_ROWS = 512      # buffer rows per expert from which the GEMMs use CTA-pair tiles
 FP8_OVER_BF16 = 2.0      # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
@@ -513,11 +514,16 @@ def main():
         # e4m3 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (2)
         peak_tf *= FP8_OVER_BF16
         peak_src += f" x {FP8_OVER_BF16:g} (nominal e4m3 / bf16 dense ratio)"
-    pair = moe_max_rows_host(cfg) >= 512 * cfg.E and not args.fp8
-    kname = ("grouped_gemm_pair_kernel<true> (gate/up + SwiGLU, CTA pairs)" if pair else
-             "grouped_gemm_e4m3_kernel<256,true> (gate/up + SwiGLU, e4m3 operands)" if args.fp8
-             else "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")
-    ktag = "gemm_pair_gate_up" if pair else "gemm_e4m3_gate_up" if args.fp8 else "gemm_gate_up"
+    # the library's tile choice: CTA pairs from PAIR_MIN_ROWS rows per expert
+    pair = moe_max_rows_host(cfg) >= PAIR_MIN_ROWS * cfg.E
+    if args.fp8:
+        kname = ("grouped_gemm_pair_kernel<true,true> (gate/up + SwiGLU, e4m3, CTA pairs)"
+                 if pair else "grouped_gemm_e4m3_kernel<256,true> (gate/up + SwiGLU, e4m3)")
+        ktag = "gemm_e4m3_pair_gate_up" if pair else "gemm_e4m3_gate_up"
+    else:
+        kname = ("grouped_gemm_pair_kernel<true> (gate/up + SwiGLU, CTA pairs)" if pair else
+                 "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")
+        ktag = "gemm_pair_gate_up" if pair else "gemm_gate_up"
     achieved = gemm1_flop / t_g1 / 1e12
     # bytes the gate/up GEMM must move: weights of the experts that got rows,
     # x_perm rows in, h rows out

@@ -73,3 +73,24 @@ def test_launches_per_step():
     assert bench.launches_per_step(configs.FINE, 148, fused=True) == 8
     assert bench.launches_per_step(configs.DECODE.with_tokens(16), 148, fp8=True) == 10
     assert bench.launches_per_step(configs.TINY.with_tokens(0), 148) == 0
+
+
+@pytest.mark.timeout(600)
+def test_reference_arm_under_torchrun_two_ranks():
+    """Launched the way the multi-GPU runs are (torchrun, two ranks): rank 0
+    alone times the oracle and prints the one JSON line; rank 1 exits 0."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    out = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                          "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
+                          "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                          "--impl", "reference", "--config", "tiny", "--gpus", "2",
+                          "--steps", "2", "--warmup", "3"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=500)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    r = json.loads(lines[0])
+    assert r["impl"] == "reference" and r["n_gpus"] == 2 and r["value"] > 0

@@ -9,7 +9,6 @@ first failure has already run every other test.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 

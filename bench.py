@@ -39,8 +39,8 @@ FP8_OVER_BF16 = 2.0      # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.
 def launches_per_step(cfg, sms, fp8=False, padded=False, fused=False):
     """libmoe kernels one layer step launches: router weight split, router
     GEMM and top-k (the top-k runs in the GEMM's epilogue when the router's K
-    is not split, i.e. when there are at least as many 128-token row tiles as
-    half the SMs); permutation rank and scatter (+ the padded layout's fill);
+    is not split, i.e. when there are more 128-token row tiles than half the
+    SMs); permutation rank and scatter (+ the padded layout's fill);
     the FP8 row quantizers on x and on h; the two expert GEMMs; the combine
     (the fused path's finalize)."""
     if cfg.T == 0:

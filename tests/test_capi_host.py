@@ -129,6 +129,72 @@ def test_validation_codes_without_launch():
                                FAKE, 0, s) == OK
 
 
+def test_validation_codes_of_the_variants_without_launch():
+    """FP8, padded, fused and bucket entry points: each case below fails (or
+    returns early on an empty input) before anything reaches the GPU."""
+    L = moe.lib()
+    s = ctypes.c_void_p(0)
+    F = FAKE
+    odd = ctypes.c_void_p((1 << 20) + 4)          # not 16-byte aligned
+    # ---- FP8
+    assert L.moe_quantize_weights_fp8(F, 0, 64, 64, F, F, s) == INVALID
+    assert L.moe_quantize_weights_fp8(None, 2, 64, 64, F, F, s) == INVALID
+    assert L.moe_quantize_rows_fp8(F, 10, 24, None, F, F, s) == INVALID       # K % 16
+    assert L.moe_quantize_rows_fp8(F, 0, 64, None, F, F, s) == OK
+    assert L.moe_quantize_rows_fp8(odd, 10, 64, None, F, F, s) == INVALID
+    assert L.moe_quantize_rows_fp8(F, 10, 64, None, None, F, s) == INVALID
+    need = moe.moe_permute_workspace_size(100, 8, 2)
+    p8 = [F, F, F, 100, 128, 8, 2, 1.25, F, F, F, F, F, F, F, F]
+    assert L.moe_permute_fp8(*p8, need - 1, None, s) == WORKSPACE
+    assert L.moe_permute_fp8(*p8[:7], -1.0, *p8[8:], need, None, s) == INVALID
+    assert L.moe_permute_fp8(None, *p8[1:], need, None, s) == INVALID
+    assert L.moe_permute_fp8(*p8[:3], 0, *p8[4:], 0, None, s) == OK
+    g8 = [F, F, F, 8, 256, 256, 100, F, F, F, F, F, None, s]
+    assert L.moe_expert_gate_up_fp8(*g8[:4], 192, *g8[5:]) == UNSUPPORTED
+    assert L.moe_expert_gate_up_fp8(*g8[:6], 0, *g8[7:]) == OK
+    assert L.moe_expert_gate_up_fp8(None, *g8[1:]) == INVALID
+    d8 = [F, F, F, 8, 256, 256, 100, F, F, F, None, s]
+    assert L.moe_expert_down_fp8(*d8[:5], 200, *d8[6:]) == UNSUPPORTED
+    assert L.moe_expert_down_fp8(*d8[:9], odd, *d8[10:]) == INVALID
+    ws8 = moe.moe_workspace_size_fp8(64, 128, 8, 2, 256, 1.25)
+    assert ws8 > moe.moe_workspace_size(64, 128, 8, 2, 256, 1.25)
+    l8 = [F] * 9
+    assert L.moe_layer_forward_fp8(*l8, 64, 128, 8, 2, 256, 1.25, F, F, ws8 - 1, s) == WORKSPACE
+    assert L.moe_layer_forward_fp8(*l8, 64, 128, 8, 2, 250, 1.25, F, F, ws8, s) == UNSUPPORTED
+    assert L.moe_layer_forward_fp8(*l8, 0, 128, 8, 2, 256, 1.25, F, F, 0, s) == OK
+    # ---- padded layout
+    pp = [F, F, 100, 128, 8, 2, 1.25, F, F, F, F, F, F, F]
+    assert L.moe_permute_padded(*pp, need - 1, None, s) == WORKSPACE
+    assert moe.moe_padded_rows(1 << 27, 256, 8, 0.0) == -1                    # E*C >= 2^31
+    assert L.moe_permute_padded(F, F, 1 << 27, 128, 256, 8, 0.0, *pp[7:], need, None, s) \
+        == INVALID
+    # ---- buckets (expert parallelism)
+    bk = [F, F, None, 6, 4, 256, 256, 100, F, F, F, F, F, None, s]
+    assert L.moe_expert_mlp_buckets(*bk) == INVALID                           # 6 % 4 != 0
+    assert L.moe_expert_mlp_buckets(*bk[:4], 0, *bk[5:]) == INVALID
+    assert L.moe_expert_mlp_buckets(*bk[:3], 8, 4, 256, 256, 0, *bk[8:]) == OK
+    # ---- fused path
+    pf = [F, F, 100, 128, 8, 2, 1.25, F, F, F, F, F, F, F, F, F]
+    assert L.moe_permute_fused(*pf, need - 1, None, s) == WORKSPACE
+    assert L.moe_permute_fused(*pf[:12], None, *pf[13:], need, None, s) == INVALID  # x w/o x_perm
+    assert L.moe_permute_fused(*pf[:14], odd, F, need, None, s) == INVALID          # y32 aligned
+    ga = [F, 5, F, F, 8, 256, 256, 100, F, F, F, None, s]
+    assert L.moe_expert_gate_up_gather(ga[0], 0, *ga[2:]) == INVALID
+    assert L.moe_expert_gate_up_gather(*ga[:7], 0, *ga[8:]) == OK
+    ds = [F, F, 8, 256, 256, 100, F, F, F, 2, F, None, s]
+    assert L.moe_expert_down_scatter(*ds[:9], 0, *ds[10:]) == INVALID
+    assert L.moe_expert_down_scatter(*ds[:9], 9, *ds[10:]) == INVALID
+    assert L.moe_expert_down_scatter(*ds[:10], None, *ds[11:]) == INVALID
+    assert L.moe_combine_finalize(F, F, F, 10, 128, 0, F, s) == INVALID
+    assert L.moe_combine_finalize(F, F, F, 10, 100, 2, F, s) == UNSUPPORTED
+    assert L.moe_combine_finalize(F, F, F, 0, 128, 2, F, s) == OK
+    wsf = moe.moe_workspace_size_fused(64, 128, 8, 2, 256, 1.25)
+    assert wsf > moe.moe_workspace_size(64, 128, 8, 2, 256, 1.25)
+    lf = [F] * 6
+    assert L.moe_layer_forward_fused(*lf, 64, 128, 8, 2, 256, 1.25, F, F, wsf - 1, s) == WORKSPACE
+    assert L.moe_layer_forward_fused(*lf, 0, 128, 8, 2, 256, 1.25, F, F, 0, s) == OK
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(4, 128, dtype=torch.bfloat16)

@@ -33,6 +33,8 @@ METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combin
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ROUTER_TILE_M = 128      # tokens per router GEMM row tile
 PAIR_MIN_ROWS = 512      # buffer rows per expert from which the GEMMs use CTA-pair tiles
+ROOFLINE_TIMING = ("mean launch duration over the timed steps: CUDA events recorded around "
+                   "the launch on its stream")
 FP8_OVER_BF16 = 2.0      # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
@@ -335,6 +337,9 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     names = layer.stage_names
     stage_ms = {n: statistics.median(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                 for j, n in enumerate(names)}
+    # the rooflines divide by a kernel's average duration over the timed steps
+    stage_mean = {n: statistics.fmean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+                  for j, n in enumerate(names)}
     status = int(layer.status.item())
     N = int(layer.perm["counts"].sum().item())          # kept pairs (either layout)
     active = int((layer.perm["counts"] > 0).sum().item())
@@ -384,7 +389,8 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, dist)
-    return {"elapsed_ms": elapsed_ms, "stage_ms": stage_ms, "status": status, "N": N,
+    return {"elapsed_ms": elapsed_ms, "stage_ms": stage_ms, "stage_mean": stage_mean,
+            "status": status, "N": N,
             "active_experts": active,
             "n_dropped": n_drop, "clocks": clk.summary(), "e2e_ms": e2e_ms,
             "h2d": x_host.numel() * 2, "d2h": y_host.numel() * 2, "layer": layer}
@@ -503,8 +509,8 @@ def main():
     value = tokens / (r["elapsed_ms"] / 1e3)
     gemm1_flop = 4.0 * r["N"] * cfg.d * cfg.f
     gemm2_flop = 2.0 * r["N"] * cfg.d * cfg.f
-    t_g1 = r["stage_ms"]["gate_up"] / 1e3
-    t_g2 = r["stage_ms"]["down"] / 1e3
+    t_g1 = r["stage_mean"]["gate_up"] / 1e3
+    t_g2 = r["stage_mean"]["down"] / 1e3
     # a kernel timed inside a long run under the power cap is compared with
     # the sustained peak, otherwise with the burst peak
     capped = "sw_power_cap" in (r["clocks"].get("reasons") or [])
@@ -550,7 +556,7 @@ def main():
         # codes + fp32 scales written
         for name, rows, width in (("quant_x", cfg.T, cfg.d), ("quant_h", r["N"], cfg.f)):
             nbytes = rows * width * 3 + rows * 4
-            t = r["stage_ms"][name] / 1e3
+            t = r["stage_mean"][name] / 1e3
             quant_rooflines[name] = {"bound": "hbm", "unit": "GB/s",
                                      "achieved": round(nbytes / t / 1e9, 1),
                                      "frac": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4)}
@@ -582,6 +588,8 @@ def main():
                       "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
                       "peak_source": peak_src,
                       "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4),
+                      "algorithmic_flop": gemm1_flop, "duration_ms": round(t_g1 * 1e3, 4),
+                      "timing": ROOFLINE_TIMING,
                       "traffic": traffic_from_profile(ktag, cfg.name)}
                      if not hbm_bound else
                      {"kernel": kname,
@@ -590,8 +598,10 @@ def main():
                       "frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
                       "peak_source": f"{pk_kind} HBM copy",
                       "algorithmic_bytes": g1_bytes, "active_experts": A,
+                      "duration_ms": round(t_g1 * 1e3, 4), "timing": ROOFLINE_TIMING,
                       "traffic": traffic_from_profile(ktag, cfg.name)}),
-        "stages_ms": {k_: round(v, 4) for k_, v in r["stage_ms"].items()},
+        "stages_ms": {k_: round(v, 4) for k_, v in r["stage_ms"].items()},     # medians
+        "stages_mean_ms": {k_: round(v, 4) for k_, v in r["stage_mean"].items()},
         "stage_rooflines": {
             "down_gemm": {"bound": "tensor", "achieved": round(gemm2_flop / t_g2 / 1e12, 1),
                           "unit": "TFLOP/s", "frac": round(gemm2_flop / t_g2 / 1e12 / peak_tf, 4),
@@ -601,12 +611,14 @@ def main():
                                  "frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
                                  "active_experts": A},
             "permute": {"bound": "hbm", "unit": "GB/s",
-                        "achieved": round(bytes_perm / (r["stage_ms"]["permute"] / 1e3) / 1e9, 1),
-                        "frac": round(bytes_perm / (r["stage_ms"]["permute"] / 1e3) / 1e9
+                        "achieved": round(bytes_perm / (r["stage_mean"]["permute"] / 1e3) / 1e9,
+                                          1),
+                        "frac": round(bytes_perm / (r["stage_mean"]["permute"] / 1e3) / 1e9
                                       / pk["hbm_gbs"], 4)},
             "combine": {"bound": "hbm", "unit": "GB/s",
-                        "achieved": round(bytes_comb / (r["stage_ms"]["combine"] / 1e3) / 1e9, 1),
-                        "frac": round(bytes_comb / (r["stage_ms"]["combine"] / 1e3) / 1e9
+                        "achieved": round(bytes_comb / (r["stage_mean"]["combine"] / 1e3) / 1e9,
+                                          1),
+                        "frac": round(bytes_comb / (r["stage_mean"]["combine"] / 1e3) / 1e9
                                       / pk["hbm_gbs"], 4)},
             **quant_rooflines,
         },

@@ -94,3 +94,50 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert len(lines) == 1, out.stdout[-2000:]
     r = json.loads(lines[0])
     assert r["impl"] == "reference" and r["n_gpus"] == 2 and r["value"] > 0
+
+
+@pytest.mark.parametrize("extra,stages", [
+    ([], ["route", "permute", "gate_up", "down", "combine"]),
+    (["--fp8"], ["route", "quant_x", "permute", "gate_up", "quant_h", "down", "combine"]),
+    (["--fused"], ["route", "permute", "gate_up", "down", "combine"]),
+    (["--layout", "padded"], ["route", "permute", "gate_up", "down", "combine"]),
+], ids=["bf16", "fp8", "fused", "padded"])
+def test_gpu_arm_json_assembly_on_cpu(monkeypatch, capsys, extra, stages):
+    """bench.py's JSON line from the GPU arm's measurements, with the GPU arm
+    replaced by fixed numbers (CPU): every contract key present and the
+    roofline arithmetic (algorithmic work / mean duration / peak) consistent."""
+    import sys
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch
+    from mixture_experts_layer_36_b200 import configs
+    cfg = configs.by_name("skewed")
+    mean = {n: 0.1 * (i + 1) for i, n in enumerate(stages)}
+    fake = {"elapsed_ms": 12.0, "stage_ms": {n: v * 0.9 for n, v in mean.items()},
+            "stage_mean": mean, "status": 0, "N": 30000, "active_experts": 60,
+            "n_dropped": 5, "clocks": {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": []},
+            "e2e_ms": 15.0, "h2d": cfg.T * cfg.d * 2, "d2h": cfg.T * cfg.d * 2,
+            "layer": types.SimpleNamespace(rows=cfg.E * 1536)}
+    monkeypatch.setattr(bench, "gpu_arm", lambda *a, **k: fake)
+    monkeypatch.setattr(torch.cuda, "get_device_properties",
+                        lambda *_: types.SimpleNamespace(multi_processor_count=148))
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--config", "skewed", "--steps", "4",
+                                      "--warmup", "3", "--no-cpu-baseline", *extra])
+    bench.main()
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    r = json.loads(lines[0])
+    assert BASE_KEYS <= set(r) and {"roofline", "clocks", "gpu_launches"} <= set(r)
+    assert r["value"] == pytest.approx(cfg.T * 4 / 12e-3, rel=1e-6)
+    assert r["e2e"]["value"] == pytest.approx(cfg.T * 4 / 15e-3, rel=1e-6)
+    assert r["gpu_launches"] == 4 * bench.launches_per_step(
+        cfg, 148, "--fp8" in extra, "padded" in extra, "--fused" in extra)
+    rf = r["roofline"]
+    assert rf["duration_ms"] == pytest.approx(mean["gate_up"])
+    assert rf["frac"] == pytest.approx(rf["achieved"] / rf["peak"], abs=1e-3)
+    if rf["bound"] == "tensor":
+        assert rf["achieved"] == pytest.approx(
+            4.0 * 30000 * cfg.d * cfg.f / (mean["gate_up"] / 1e3) / 1e12, rel=1e-3)
+    assert r["stages_mean_ms"] == {n: round(v, 4) for n, v in mean.items()}
+    assert set(r["stages_ms"]) == set(stages)

@@ -10,9 +10,15 @@ library and raises ImportError if it has not been built.  ``configs`` and
 """
 import importlib
 
+# submodules load on their own (``from ... import configs`` must not need the library)
+_SUBMODULES = {"binding", "build", "configs", "ep", "synth"}
+
+
 def __getattr__(name):
     if name.startswith("__"):
         raise AttributeError(name)
+    if name in _SUBMODULES:
+        return importlib.import_module("." + name, __name__)
     binding = importlib.import_module(".binding", __name__)
     if hasattr(binding, name):
         return getattr(binding, name)

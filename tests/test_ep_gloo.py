@@ -134,3 +134,19 @@ def test_expert_parallel_matches_single_process(world, case):
         dropped += n_drop
     if case[5] > 0:
         assert dropped > 0                    # the capacity limit was exercised
+
+
+def test_layer_rejects_expert_counts_that_do_not_split():
+    """Without a process group the layer is one rank holding all E experts;
+    wrong local expert counts are refused before any compute."""
+    from mixture_experts_layer_36_b200 import ep
+    E, d, f = 8, 16, 32
+    wr = torch.zeros(d, E)
+    wg, wu, wd = torch.zeros(E, d, f), torch.zeros(E, d, f), torch.zeros(E, f, d)
+    layer = ep.ExpertParallelMoE(wr, None, wg, wu, wd, 2, 1.0, ops=object())
+    assert (layer.P, layer.rank, layer.E_loc) == (1, 0, E)
+    with pytest.raises(ValueError):
+        ep.ExpertParallelMoE(wr, None, wg[:4], wu[:4], wd[:4], 2, 1.0, ops=object())
+    # shard_experts hands rank r experts r*E/P .. (r+1)*E/P - 1
+    w = torch.arange(E).reshape(E, 1, 1).float()
+    assert ep.shard_experts(w, 1, 4).flatten().tolist() == [2.0, 3.0]

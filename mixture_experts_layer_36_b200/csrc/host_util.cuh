@@ -105,7 +105,9 @@ inline bool map_weights_e4m3(CUtensorMap* m, const void* base, uint64_t E, uint6
 
 // attr_set slots: 0-2 grouped GEMM (1 CTA), 3-6 router GEMM, 7-8 grouped GEMM (CTA pair),
 // 9-10 CTA-pair GEMM on e4m3 operands, 11-13 grouped GEMM on e4m3 operands
-// (+16: the gathering instance of a slot's kernel, +32: the scattering one)
+// (+16: the gathering instance of a grouped GEMM slot's kernel, +32: the
+// scattering one); 19-22 router GEMM with the top-k epilogue (the router
+// kernels have no gathering instance, so 3-6 + 16 is free for them)
 struct DeviceInfo {
   int sms = 0;
   bool attr_set[48] = {};

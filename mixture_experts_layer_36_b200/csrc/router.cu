@@ -89,18 +89,22 @@ struct RouterShared {
 
 // Keeps the best 8 (value, expert) pairs in descending order; called in
 // increasing expert order, a value enters ahead of a kept one only if it is
-// strictly larger, so equal values stay ordered by expert index.
+// strictly larger, so equal values stay ordered by expert index.  From the
+// slot where it enters, the kept pairs behind it shift down one place each
+// (a displaced pair stays ahead of every later pair of equal value).
 __device__ __forceinline__ void topk_insert(float (&sv)[8], int (&se)[8], float v, int e) {
   if (se[7] >= 0 && !(v > sv[7])) return;
+  bool shifting = false;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    if (se[i] < 0 || v > sv[i]) {
+    if (shifting || se[i] < 0 || v > sv[i]) {
       const float tv = sv[i];
       const int te = se[i];
       sv[i] = v;
       se[i] = e;
       v = tv;
       e = te;
+      shifting = true;
     }
   }
 }

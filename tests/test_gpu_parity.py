@@ -121,17 +121,23 @@ def test_route_unsplit_matches_oracle(E, k, with_bias):
     independent_topk_check(ref64, idx.cpu().numpy(), k)
 
 
-def test_route_unsplit_ties_take_lower_index():
-    E, k, d = 16, 4, 128
+@pytest.mark.parametrize("pattern,k,want", [
+    ([0.5, 1.0, 1.0, 0.5, 2.0, 1.0, 2.0, 0.0], 4, [4, 6, 12, 14]),
+    # equal values displaced by a larger one arriving later keep their order
+    ([1.0, 1.0, 1.0, 0.5, 2.0, 1.0, 2.0, 0.0], 8, [4, 6, 12, 14, 0, 1, 2, 5]),
+    ([0.5, 1.0, 1.0, 0.5, 2.0, 1.0, 2.0, 0.0], 8, [4, 6, 12, 14, 1, 2, 5, 9]),
+])
+def test_route_unsplit_ties_take_lower_index(pattern, k, want):
+    E, d = 16, 128
     x = torch.zeros(T_UNSPLIT, d, dtype=torch.bfloat16, device="cuda")
     x[::3] = torch.randn(x[::3].shape, device="cuda").to(torch.bfloat16)  # some untied rows
     wr = torch.randn(d, E, device="cuda")
-    bias = torch.tensor([0.5, 1.0, 1.0, 0.5, 2.0, 1.0, 2.0, 0.0] * 2, device="cuda")
+    bias = torch.tensor(pattern * 2, device="cuda")
     logits, idx, w = moe.moe_route(x, wr, bias, k)
     gl = logits.cpu().numpy()
     o_idx, o_w = oracle.topk(gl, k)
     np.testing.assert_array_equal(idx.cpu().numpy(), o_idx)
-    assert o_idx[1].tolist() == [4, 6, 12, 14]            # an all-tied row
+    assert o_idx[1].tolist() == want                      # an all-tied row
     assert np.max(np.abs(w.cpu().double().numpy() - o_w)) <= WEIGHT_ATOL
 
 

@@ -85,8 +85,8 @@ def _worker(rank, world, port, case, out):
     import oracle
     from mixture_experts_layer_36_b200 import ep, synth
     from mixture_experts_layer_36_b200.configs import MoEConfig
-    T, d, E, k, f, cf = case
-    cfg = MoEConfig("ep_case", T=T, d=d, E=E, k=k, f=f, cf=cf, seed=5)
+    T, d, E, k, f, cf, zipf_s = case
+    cfg = MoEConfig("ep_case", T=T, d=d, E=E, k=k, f=f, cf=cf, seed=5, zipf_s=zipf_s)
     w = synth.make_weights(cfg, "cpu")                    # the same weights on every rank
     x = synth.make_tokens(cfg, "cpu", seed=100 + rank)    # each rank its own tokens
     layer = ep.ExpertParallelMoE(w["w_router"], w["bias"],
@@ -97,8 +97,9 @@ def _worker(rank, world, port, case, out):
     y = layer(x).numpy()
     xb = OracleOps._bits(x)
     ops = OracleOps(oracle)
-    lg32 = oracle.router_logits(xb, w["w_router"].numpy(), None).astype(np.float32)
-    ref = oracle.moe_forward(xb, w["w_router"].numpy(), None, ops._bits(w["w_gate"]),
+    bias = None if w["bias"] is None else w["bias"].numpy()
+    lg32 = oracle.router_logits(xb, w["w_router"].numpy(), bias).astype(np.float32)
+    ref = oracle.moe_forward(xb, w["w_router"].numpy(), bias, ops._bits(w["w_gate"]),
                              ops._bits(w["w_up"]), ops._bits(w["w_down"]), k, cf,
                              decision_logits=lg32)
     dist.barrier()
@@ -108,15 +109,16 @@ def _worker(rank, world, port, case, out):
 
 
 CASES = [
-    # (T, d, E, k, f, cf)
-    (24, 16, 8, 2, 32, 0.0),      # dropless
-    (40, 16, 8, 3, 32, 0.75),     # with drops
+    # (T, d, E, k, f, cf, zipf_s)
+    (24, 16, 8, 2, 32, 0.0, None),    # dropless
+    (40, 16, 8, 3, 32, 0.75, None),   # with drops
+    (48, 16, 8, 2, 32, 1.0, 1.2),     # Zipf-hot low experts (router bias), drops on rank 0's
 ]
 
 
 @pytest.mark.timeout(300)
 @pytest.mark.parametrize("world", [2, 4])
-@pytest.mark.parametrize("case", CASES, ids=["dropless", "drops"])
+@pytest.mark.parametrize("case", CASES, ids=["dropless", "drops", "skewed"])
 def test_expert_parallel_matches_single_process(world, case):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()

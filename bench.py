@@ -42,7 +42,7 @@ def launches_per_step(cfg, sms, fp8=False, padded=False, fused=False):
     """libmoe kernels one layer step launches: router weight split, router
     GEMM and top-k (the top-k runs in the GEMM's epilogue when the router's K
     is not split, i.e. when there are more 128-token row tiles than half the
-    SMs); permutation rank and scatter (+ the padded layout's fill);
+    SMs); permutation rank, scan and scatter (+ the padded layout's fill);
     the FP8 row quantizers on x and on h; the two expert GEMMs; the combine
     (the fused path's finalize)."""
     if cfg.T == 0:
@@ -50,7 +50,7 @@ def launches_per_step(cfg, sms, fp8=False, padded=False, fused=False):
     m_tiles = -(-cfg.T // ROUTER_TILE_M)
     splits = max(1, min(min(sms, 256) // m_tiles, cfg.d // 64))
     n = 2 if splits == 1 else 3
-    n += 3 if padded else 2
+    n += 4 if padded else 3
     n += 2 if fp8 else 0
     return n + 2 + 1
 
@@ -302,7 +302,9 @@ class Layer:
                                    w["w_down"], c.k, c.cf, y=y, ws=self.ws)
 
 
-def gpu_arm(args, cfg, rank, world, local_rank):
+def gpu_arm(args, cfg, rank, world, local_rank, with_e2e=True):
+    """Time K layer steps (CUDA events around every stage, max over ranks), and
+    with_e2e the one-shot public call with host buffers in and out."""
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     dist = world > 1
@@ -344,6 +346,11 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     N = int(layer.perm["counts"].sum().item())          # kept pairs (either layout)
     active = int((layer.perm["counts"] > 0).sum().item())
     n_drop = int(layer.perm["n_dropped"].item())
+    out = {"elapsed_ms": elapsed_ms, "stage_ms": stage_ms, "stage_mean": stage_mean,
+           "status": status, "N": N, "active_experts": active, "n_dropped": n_drop,
+           "clocks": clk.summary(), "layer": layer}
+    if not with_e2e:
+        return out
 
     # end to end through the one-shot public call, host buffers in and out:
     # every step copies its tokens host->device, runs moe_layer_forward and
@@ -388,12 +395,10 @@ def gpu_arm(args, cfg, rank, world, local_rank):
     stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, dist)
-    return {"elapsed_ms": elapsed_ms, "stage_ms": stage_ms, "stage_mean": stage_mean,
-            "status": status, "N": N,
-            "active_experts": active,
-            "n_dropped": n_drop, "clocks": clk.summary(), "e2e_ms": e2e_ms,
-            "h2d": x_host.numel() * 2, "d2h": y_host.numel() * 2, "layer": layer}
+    out["e2e_ms"] = max_over_ranks(e0.elapsed_time(e1), dev, dist)
+    out["h2d"] = x_host.numel() * 2
+    out["d2h"] = y_host.numel() * 2
+    return out
 
 
 def traffic_from_profile(kernel_tag, workload):
@@ -416,7 +421,6 @@ def traffic_from_profile(kernel_tag, workload):
 def oracle_sample(cfg, weights_host, x_host_bits, n_tokens):
     """Time the oracle (as it stands) on the first n_tokens tokens of the batch,
     whole layer (capacity recomputed for the sample size).  Returns seconds."""
-    import numpy as np
     import oracle
     bias = None if weights_host["bias"] is None else weights_host["bias"]
     t0 = time.perf_counter()
@@ -447,6 +451,178 @@ def calibrated_tokens(cfg, wh, xb, seconds):
     return n
 
 
+# the oracle runs the whole layer on these workloads when their pass is
+# estimated under FULL_LAYER_MAX_S on the host; otherwise a token sample
+# (extrapolated to the batch: the oracle's cost is linear in the tokens)
+FULL_LAYER = ("tiny", "mixtral", "skewed", "decode")
+FULL_LAYER_MAX_S = 90.0
+
+
+def oracle_timing(cfg, layer, host_cache=None, sample_s=5.0):
+    """The oracle's tokens/s on this workload: the whole batch where planned
+    (and affordable), else a calibrated sample of about sample_s seconds.
+    host_cache keeps the host copy of weights that several workloads share
+    (the decode sweep draws the same weights at every T)."""
+    import oracle
+    key = (cfg.seed, cfg.E, cfg.d, cfg.f, cfg.zipf_s)
+    if host_cache is not None and key in host_cache:
+        wh = host_cache[key]
+    else:
+        wh = host_weights(layer.w)
+        if host_cache is not None:
+            host_cache.clear()
+            host_cache[key] = wh
+    xb = oracle.bf16_bits(layer.x)
+    n = calibrated_tokens(cfg, wh, xb, sample_s)
+    whole = cfg.name.split("@")[0] in FULL_LAYER
+    if whole and n < cfg.T:
+        est = sample_s * cfg.T / max(n, 1)
+        whole = est <= FULL_LAYER_MAX_S
+    if whole:
+        secs, cores = oracle_sample(cfg, wh, xb, cfg.T)
+        what = f"whole layer, all {cfg.T} tokens, {secs:.1f} s"
+        n = cfg.T
+    else:
+        secs, cores = oracle_sample(cfg, wh, xb, n)
+        what = (f"first {n} of {cfg.T} tokens through the whole layer, {secs:.1f} s "
+                "(capacity recomputed for the sample; extrapolated: cost is linear in tokens)")
+    return {"value": round(n / secs, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": what}
+
+
+# ----------------------------------------------------------------- the JSON line
+
+def path_name(args):
+    return "fused (down GEMM + weighted scatter)" if args.fused else "staged"
+
+
+def workload_config(cfg, args, world):
+    """The `config` object of both arms' lines: a function of the workload and
+    the command line only."""
+    wb = 1 if args.fp8 else 2
+    return {"workload": describe(cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+            "f": cfg.f, "cf": cfg.cf,
+            "parallelism": f"replicas x{world} (token batches, no collective)",
+            "layout": args.layout, "path": path_name(args),
+            "experts": ("e4m3 weights (fp32 column scales) x e4m3 activations (fp32 row "
+                        "scales)") if args.fp8 else "bf16",
+            "l2": "inputs larger than L2 (expert weights "
+                  f"{3 * cfg.E * cfg.d * cfg.f * wb / 1e9:.1f} GB); no flush"}
+
+
+def summarize(cfg, args, r, pk, pk_kind, world):
+    """Throughput, the dominant kernel's roofline and the per-stage rooflines
+    of one timed run (r from gpu_arm)."""
+    K = args.steps
+    value = cfg.T * world * K / (r["elapsed_ms"] / 1e3)
+    gemm1_flop = 4.0 * r["N"] * cfg.d * cfg.f
+    gemm2_flop = 2.0 * r["N"] * cfg.d * cfg.f
+    t_g1 = r["stage_mean"]["gate_up"] / 1e3
+    t_g2 = r["stage_mean"]["down"] / 1e3
+    # a kernel timed inside a long run under the power cap is compared with
+    # the sustained peak, otherwise with the burst peak
+    capped = "sw_power_cap" in (r["clocks"].get("reasons") or [])
+    peak_tf = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
+    peak_src = f"{pk_kind} bf16 {'sustained (power cap active)' if capped else 'burst'}"
+    burst_tf = pk["bf16_tflops"]
+    if args.fp8:
+        # e4m3 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (2)
+        peak_tf *= FP8_OVER_BF16
+        burst_tf *= FP8_OVER_BF16
+        peak_src += f" x {FP8_OVER_BF16:g} (nominal e4m3 / bf16 dense ratio)"
+    # the library's tile choice: CTA pairs from PAIR_MIN_ROWS rows per expert
+    pair = moe_max_rows_host(cfg) >= PAIR_MIN_ROWS * cfg.E
+    if args.fp8:
+        kname = ("grouped_gemm_pair_kernel<true,true> (gate/up + SwiGLU, e4m3, CTA pairs)"
+                 if pair else "grouped_gemm_e4m3_kernel<256,true> (gate/up + SwiGLU, e4m3)")
+        ktag = "gemm_e4m3_pair_gate_up" if pair else "gemm_e4m3_gate_up"
+    else:
+        kname = ("grouped_gemm_pair_kernel<true> (gate/up + SwiGLU, CTA pairs)" if pair else
+                 "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")
+        ktag = "gemm_pair_gate_up" if pair else "gemm_gate_up"
+    achieved = gemm1_flop / t_g1 / 1e12
+    # bytes the gate/up GEMM must move: weights of the experts that got rows,
+    # x_perm rows in, h rows out
+    A = r["active_experts"]
+    # operand bytes per element: bf16 2; e4m3 1 (plus 4-byte row / column scales)
+    wb = 1 if args.fp8 else 2
+    g1_bytes = A * 2.0 * cfg.d * cfg.f * wb + r["N"] * cfg.d * wb + r["N"] * cfg.f * 2
+    g2_bytes = A * 1.0 * cfg.d * cfg.f * wb + r["N"] * cfg.f * wb + r["N"] * cfg.d * 4
+    if args.fp8:
+        g1_bytes += A * 2.0 * cfg.f * 4 + r["N"] * 4
+        g2_bytes += A * 1.0 * cfg.d * 4 + r["N"] * 4
+    ridge = peak_tf * 1e12 / (pk["hbm_gbs"] * 1e9)
+    hbm_bound = gemm1_flop / g1_bytes < ridge
+    bytes_perm = cfg.T * cfg.d * wb + r["N"] * cfg.d * wb
+    bytes_comb = r["N"] * cfg.d * 4 + cfg.T * cfg.d * 2
+    if args.fused:
+        # the permutation also zeroes the fp32 accumulator; the finishing pass
+        # reads it and writes y
+        bytes_perm += cfg.T * cfg.d * 4
+        bytes_comb = cfg.T * cfg.d * 4 + cfg.T * cfg.d * 2
+
+    def hbm(nbytes, name):
+        t = r["stage_mean"][name] / 1e3
+        return {"bound": "hbm", "unit": "GB/s", "algorithmic_bytes": nbytes,
+                "duration_ms": round(t * 1e3, 6), "achieved": float(f"{nbytes / t / 1e9:.6g}"),
+                "peak": pk["hbm_gbs"], "frac": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4)}
+
+    quant_rooflines = {}
+    if args.fp8:
+        # the row quantizers: bf16 rows read once (the second pass hits cache),
+        # codes + fp32 scales written
+        for name, rows, width in (("quant_x", cfg.T, cfg.d), ("quant_h", r["N"], cfg.f)):
+            quant_rooflines[name] = hbm(rows * width * 3 + rows * 4, name)
+    if not hbm_bound:
+        roofline = {"kernel": kname, "bound": "tensor", "achieved": round(achieved, 1),
+                    "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                    "peak_source": peak_src,
+                    "frac_of_burst_peak": round(achieved / burst_tf, 4),
+                    "algorithmic_flop": gemm1_flop, "duration_ms": round(t_g1 * 1e3, 4),
+                    "timing": ROOFLINE_TIMING, "traffic": traffic_from_profile(ktag, cfg.name)}
+    else:
+        roofline = {"kernel": kname, "bound": "hbm", "achieved": round(g1_bytes / t_g1 / 1e9, 1),
+                    "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
+                    "peak_source": f"{pk_kind} HBM copy", "algorithmic_bytes": g1_bytes,
+                    "active_experts": A, "duration_ms": round(t_g1 * 1e3, 4),
+                    "timing": ROOFLINE_TIMING, "traffic": traffic_from_profile(ktag, cfg.name)}
+    return {
+        "value": round(value, 1),
+        "ms_per_step": round(r["elapsed_ms"] / K, 4),
+        "roofline": roofline,
+        "stages_ms": {k_: round(v, 4) for k_, v in r["stage_ms"].items()},     # medians
+        "stages_mean_ms": {k_: round(v, 4) for k_, v in r["stage_mean"].items()},
+        "stage_rooflines": {
+            "gate_up_gemm": {"bound": "tensor", "achieved": round(achieved, 1), "unit": "TFLOP/s",
+                             "peak": peak_tf, "frac": round(achieved / peak_tf, 4),
+                             "frac_of_burst_peak": round(achieved / burst_tf, 4),
+                             "hbm_GBps": round(g1_bytes / t_g1 / 1e9, 1),
+                             "hbm_frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
+                             "active_experts": A},
+            "down_gemm": {"bound": "tensor", "achieved": round(gemm2_flop / t_g2 / 1e12, 1),
+                          "unit": "TFLOP/s", "peak": peak_tf,
+                          "frac": round(gemm2_flop / t_g2 / 1e12 / peak_tf, 4),
+                          "frac_of_burst_peak": round(gemm2_flop / t_g2 / 1e12 / burst_tf, 4),
+                          "hbm_GBps": round(g2_bytes / t_g2 / 1e9, 1),
+                          "hbm_frac": round(g2_bytes / t_g2 / 1e9 / pk["hbm_gbs"], 4)},
+            "permute": hbm(bytes_perm, "permute"),
+            "combine": hbm(bytes_comb, "combine"),
+            **quant_rooflines,
+        },
+        "routing": {"kept_pairs": r["N"], "dropped_pairs": r["n_dropped"], "active_experts": A,
+                    "gemm_rows_computed": (r["layer"].rows if args.layout == "padded"
+                                           else r["N"])},
+        "device_status": r["status"],
+        "clocks": {k_: r["clocks"][k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},
+    }
+
+
+# the other workloads measured beside the headline one (per_config)
+PER_CONFIG = ("tiny", "mixtral", "fine_grained", "skewed", "decode@T16", "decode@T64",
+              "decode@T256")
+
+
 # ----------------------------------------------------------------- main
 
 def main():
@@ -457,6 +633,9 @@ def main():
     ap.add_argument("--config", default="mixtral")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the named workload (by default every other workload is "
+                         "also timed, with the oracle beside it, into per_config)")
     ap.add_argument("--layout", choices=["ragged", "padded"], default="ragged",
                     help="padded: the static [E, C, d] expert buffers (every bucket C rows, all "
                          "computed) in place of the ragged buckets")
@@ -505,125 +684,24 @@ def main():
     r = gpu_arm(args, cfg, rank, world, local_rank)
     pk, pk_kind = peaks()
     K = args.steps
-    tokens = cfg.T * world * K
-    value = tokens / (r["elapsed_ms"] / 1e3)
-    gemm1_flop = 4.0 * r["N"] * cfg.d * cfg.f
-    gemm2_flop = 2.0 * r["N"] * cfg.d * cfg.f
-    t_g1 = r["stage_mean"]["gate_up"] / 1e3
-    t_g2 = r["stage_mean"]["down"] / 1e3
-    # a kernel timed inside a long run under the power cap is compared with
-    # the sustained peak, otherwise with the burst peak
-    capped = "sw_power_cap" in (r["clocks"].get("reasons") or [])
-    peak_tf = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
-    peak_src = f"{pk_kind} bf16 {'sustained (power cap active)' if capped else 'burst'}"
-    if args.fp8:
-        # e4m3 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (2)
-        peak_tf *= FP8_OVER_BF16
-        peak_src += f" x {FP8_OVER_BF16:g} (nominal e4m3 / bf16 dense ratio)"
-    # the library's tile choice: CTA pairs from PAIR_MIN_ROWS rows per expert
-    pair = moe_max_rows_host(cfg) >= PAIR_MIN_ROWS * cfg.E
-    if args.fp8:
-        kname = ("grouped_gemm_pair_kernel<true,true> (gate/up + SwiGLU, e4m3, CTA pairs)"
-                 if pair else "grouped_gemm_e4m3_kernel<256,true> (gate/up + SwiGLU, e4m3)")
-        ktag = "gemm_e4m3_pair_gate_up" if pair else "gemm_e4m3_gate_up"
-    else:
-        kname = ("grouped_gemm_pair_kernel<true> (gate/up + SwiGLU, CTA pairs)" if pair else
-                 "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")
-        ktag = "gemm_pair_gate_up" if pair else "gemm_gate_up"
-    achieved = gemm1_flop / t_g1 / 1e12
-    # bytes the gate/up GEMM must move: weights of the experts that got rows,
-    # x_perm rows in, h rows out
-    A = r["active_experts"]
-    # operand bytes per element: bf16 2; e4m3 1 (plus 4-byte row / column scales)
-    wb = 1 if args.fp8 else 2
-    g1_bytes = A * 2.0 * cfg.d * cfg.f * wb + r["N"] * cfg.d * wb + r["N"] * cfg.f * 2
-    g2_bytes = A * 1.0 * cfg.d * cfg.f * wb + r["N"] * cfg.f * wb + r["N"] * cfg.d * 4
-    if args.fp8:
-        g1_bytes += A * 2.0 * cfg.f * 4 + r["N"] * 4
-        g2_bytes += A * 1.0 * cfg.d * 4 + r["N"] * 4
-    ridge = peak_tf * 1e12 / (pk["hbm_gbs"] * 1e9)
-    hbm_bound = gemm1_flop / g1_bytes < ridge
-    bytes_perm = cfg.T * cfg.d * wb + r["N"] * cfg.d * wb
-    bytes_comb = r["N"] * cfg.d * 4 + cfg.T * cfg.d * 2
-    if args.fused:
-        # the permutation also zeroes the fp32 accumulator; the finishing pass
-        # reads it and writes y
-        bytes_perm += cfg.T * cfg.d * 4
-        bytes_comb = cfg.T * cfg.d * 4 + cfg.T * cfg.d * 2
-    quant_rooflines = {}
-    if args.fp8:
-        # the row quantizers: bf16 rows read once (the second pass hits cache),
-        # codes + fp32 scales written
-        for name, rows, width in (("quant_x", cfg.T, cfg.d), ("quant_h", r["N"], cfg.f)):
-            nbytes = rows * width * 3 + rows * 4
-            t = r["stage_mean"][name] / 1e3
-            quant_rooflines[name] = {"bound": "hbm", "unit": "GB/s",
-                                     "achieved": round(nbytes / t / 1e9, 1),
-                                     "frac": round(nbytes / t / 1e9 / pk["hbm_gbs"], 4)}
+    summ = summarize(cfg, args, r, pk, pk_kind, world)
+    oracle_here = rank == 0 and world == 1 and not args.no_cpu_baseline
     out = {
         "metric": METRIC,
-        "value": round(value, 1),
+        "value": summ["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
         "warmup": args.warmup,
-        "ms_per_step": round(r["elapsed_ms"] / K, 4),
+        "ms_per_step": summ["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "e4m3 (expert GEMM operands; fp32 accumulation)" if args.fp8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the named shape)",
-        "config": {"workload": describe(cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                   "f": cfg.f, "cf": cfg.cf, "kept_pairs": r["N"], "dropped_pairs": r["n_dropped"],
-                   "parallelism": f"replicas x{world} (token batches, no collective)",
-                   "layout": args.layout,
-                   "path": "fused (down GEMM + weighted scatter)" if args.fused else "staged",
-                   "gemm_rows_computed": (r["layer"].rows if args.layout == "padded" else r["N"]),
-                   "experts": ("e4m3 weights (fp32 column scales) x e4m3 activations (fp32 row "
-                               "scales)") if args.fp8 else "bf16",
-                   "l2": "inputs larger than L2 (expert weights "
-                         f"{3 * cfg.E * cfg.d * cfg.f * wb / 1e9:.1f} GB); no flush"},
-        "roofline": ({"kernel": kname,
-                      "bound": "tensor", "achieved": round(achieved, 1),
-                      "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
-                      "peak_source": peak_src,
-                      "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4),
-                      "algorithmic_flop": gemm1_flop, "duration_ms": round(t_g1 * 1e3, 4),
-                      "timing": ROOFLINE_TIMING,
-                      "traffic": traffic_from_profile(ktag, cfg.name)}
-                     if not hbm_bound else
-                     {"kernel": kname,
-                      "bound": "hbm", "achieved": round(g1_bytes / t_g1 / 1e9, 1),
-                      "peak": pk["hbm_gbs"], "unit": "GB/s",
-                      "frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
-                      "peak_source": f"{pk_kind} HBM copy",
-                      "algorithmic_bytes": g1_bytes, "active_experts": A,
-                      "duration_ms": round(t_g1 * 1e3, 4), "timing": ROOFLINE_TIMING,
-                      "traffic": traffic_from_profile(ktag, cfg.name)}),
-        "stages_ms": {k_: round(v, 4) for k_, v in r["stage_ms"].items()},     # medians
-        "stages_mean_ms": {k_: round(v, 4) for k_, v in r["stage_mean"].items()},
-        "stage_rooflines": {
-            "down_gemm": {"bound": "tensor", "achieved": round(gemm2_flop / t_g2 / 1e12, 1),
-                          "unit": "TFLOP/s", "frac": round(gemm2_flop / t_g2 / 1e12 / peak_tf, 4),
-                          "hbm_GBps": round(g2_bytes / t_g2 / 1e9, 1),
-                          "hbm_frac": round(g2_bytes / t_g2 / 1e9 / pk["hbm_gbs"], 4)},
-            "gate_up_gemm_hbm": {"GBps": round(g1_bytes / t_g1 / 1e9, 1),
-                                 "frac": round(g1_bytes / t_g1 / 1e9 / pk["hbm_gbs"], 4),
-                                 "active_experts": A},
-            "permute": {"bound": "hbm", "unit": "GB/s",
-                        "achieved": round(bytes_perm / (r["stage_mean"]["permute"] / 1e3) / 1e9,
-                                          1),
-                        "frac": round(bytes_perm / (r["stage_mean"]["permute"] / 1e3) / 1e9
-                                      / pk["hbm_gbs"], 4)},
-            "combine": {"bound": "hbm", "unit": "GB/s",
-                        "achieved": round(bytes_comb / (r["stage_mean"]["combine"] / 1e3) / 1e9,
-                                          1),
-                        "frac": round(bytes_comb / (r["stage_mean"]["combine"] / 1e3) / 1e9
-                                      / pk["hbm_gbs"], 4)},
-            **quant_rooflines,
-        },
-        "device_status": r["status"],
-        "clocks": {k_: r["clocks"][k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "config": workload_config(cfg, args, world),
+        **{k_: summ[k_] for k_ in ("roofline", "stages_ms", "stages_mean_ms", "stage_rooflines",
+                                   "routing", "device_status", "clocks")},
         "e2e": {"value": round(cfg.T * world * K / (r["e2e_ms"] / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "api": ("the stage entry points (moe_route, moe_permute_padded, "
@@ -638,7 +716,7 @@ def main():
             cfg, torch.cuda.get_device_properties(local_rank).multi_processor_count, args.fp8,
             args.layout == "padded", args.fused) * K,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if oracle_here:
         wh = host_weights(r["layer"].w)
         import oracle
         xb = oracle.bf16_bits(r["layer"].x)
@@ -648,6 +726,30 @@ def main():
                                "kind": "oracle",
                                "sample": f"first {n} tokens of the batch through the whole "
                                          f"layer (fp64 C oracle, OpenMP), {secs:.1f} s"}
+    if not args.no_per_config:
+        # every other workload, same path and step count: throughput, the
+        # dominant kernel's roofline, the permute / combine HBM fractions, and
+        # the oracle on the host beside it
+        per = {}
+        names = [cfg.name] + [n for n in PER_CONFIG if configs.by_name(n).name != cfg.name]
+        host_cache = {}
+        for name in names:
+            c = configs.by_name(name)
+            if c.name == cfg.name:
+                rc, sc = r, summ
+            else:
+                torch.cuda.empty_cache()
+                rc = gpu_arm(args, c, rank, world, local_rank, with_e2e=False)
+                sc = summarize(c, args, rc, pk, pk_kind, world)
+            entry = {"workload": describe(c), "tokens_per_s": sc["value"],
+                     "ms_per_step": sc["ms_per_step"], "steps": K,
+                     **{k_: sc[k_] for k_ in ("roofline", "stage_rooflines", "stages_mean_ms",
+                                              "routing", "device_status", "clocks")}}
+            if oracle_here:
+                entry["oracle"] = oracle_timing(c, rc["layer"], host_cache)
+            per[c.name] = entry
+            rc.pop("layer", None)        # frees this workload's buffers before the next
+        out["per_config"] = per
     if world > 1:
         import torch.distributed as td
         td.barrier()
@@ -681,8 +783,7 @@ def reference_arm(args, cfg, rank, world):
         "ms_per_step": round(t / args.steps * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; random-init weights of the named shape)",
-        "config": {"workload": describe(cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                   "f": cfg.f, "cf": cfg.cf},
+        "config": workload_config(cfg, args, world),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
                          "kind": "oracle",
                          "sample": f"each step: first {n} tokens of the batch through the whole "

@@ -184,12 +184,14 @@ int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, in
  * receives its declared input and output tensors, or a runtime that plans all
  * device memory at start-up and forbids later allocations.  The pages have no
  * counterpart to this entry point; it is a deployment convenience.
- * Arguments and results are those of moe_permute (same kernels, same
- * outputs).  The per-chunk bucket counters live in a 256 KiB array compiled
- * into the library and held by every GPU that loads it until the process
- * exits; nothing is allocated per call.  Limits and rules:
- *   - ceil(T/256) * E must be <= 65536, else MOE_ERR_WORKSPACE (E = 256 allows
- *     T <= 65536);
+ * Arguments, results and return codes are those of moe_permute (same checks,
+ * same kernels, same outputs, including the bit-4 report into the nullable
+ * dev_status for a topk_idx entry outside [0, E)), minus ws / ws_bytes.  The
+ * per-chunk bucket counters live in a 257 KiB array compiled into the library
+ * and held by every GPU that loads it until the process exits; nothing is
+ * allocated per call.  Limits and rules:
+ *   - (ceil(T/256) + 1) * E must be <= 65792, else MOE_ERR_WORKSPACE (E = 256
+ *     allows T <= 65536);
  *   - all calls share that array: calls whose work overlaps on the GPU (other
  *     streams, other host threads on the same device) race; serialise them;
  *   - nothing in the array needs to start at zero (each call writes every
@@ -198,7 +200,8 @@ int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, in
  *     that device current) and caches it; make it before any stream capture. */
 int moe_permute_noalloc(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, int64_t E,
                         int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
-                        int32_t* row_src, void* x_perm, int32_t* n_dropped, void* stream);
+                        int32_t* row_src, void* x_perm, int32_t* n_dropped, int32_t* dev_status,
+                        void* stream);
 
 /* Grouped expert GEMM 1 with the SwiGLU fused into its epilogue: for every
  * expert e and every row r of its bucket (offsets[e] <= r < offsets[e+1]),

@@ -63,7 +63,8 @@ def _load():
         "moe_route": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, p, p, p, p, sz, p, p]),
         "moe_permute": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p, sz, p,
                                        p]),
-        "moe_permute_noalloc": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p]),
+        "moe_permute_noalloc": (ctypes.c_int, [p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
+                                               p]),
         "moe_expert_gate_up": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p]),
         "moe_expert_down": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p]),
         "moe_expert_mlp": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p, p, p]),
@@ -239,7 +240,7 @@ def moe_permute(x, topk_idx, E, cf, out=None, ws=None, dev_status=None, stream=N
     return out
 
 
-def moe_permute_noalloc(x, topk_idx, E, cf, out, stream=None):
+def moe_permute_noalloc(x, topk_idx, E, cf, out, dev_status=None, stream=None):
     """moe_permute for callers that cannot provide scratch memory: the library
     uses a fixed array of its own (shared by every call; see include/moe.h).
     `out` holds the caller's output tensors, as returned by moe_permute."""
@@ -250,7 +251,7 @@ def moe_permute_noalloc(x, topk_idx, E, cf, out, stream=None):
     _check("moe_permute_noalloc", _lib.moe_permute_noalloc(
         _ptr(x), _ptr(topk_idx), T, d, E, k, float(cf), _ptr(out["counts"]),
         _ptr(out["offsets"]), _ptr(out["slot"]), _ptr(out["row_src"]), _ptr(out["x_perm"]),
-        _ptr(out["n_dropped"]), _stream(stream)))
+        _ptr(out["n_dropped"]), _ptr(dev_status), _stream(stream)))
     return out
 
 

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include "abi_checks.cuh"
 #include "common.cuh"
 
 namespace moe {
@@ -82,11 +83,12 @@ using moe::FuseArgs;
 
 namespace {
 
-constexpr int64_t kMaxE = 256;
-constexpr int64_t kMaxK = 8;
-constexpr int64_t kTileMultiple = 128;
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+using moe::abi::aligned16;
+using moe::abi::check_routing_shape;
+using moe::abi::check_width;
+using moe::abi::cuda_status;
+using moe::abi::kMaxE;
+using moe::abi::kMaxK;
 
 // An NVTX range around one stage of a one-shot layer call (host-side enqueue;
 // a profiler attached to the process shows it on the timeline).
@@ -103,20 +105,6 @@ int staged(const char* name, F call) {
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
-
-// Shape checks common to every entry point.  Returns MOE_OK or an error.
-int check_routing_shape(int64_t T, int64_t E, int64_t k) {
-  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E) return MOE_ERR_INVALID_ARG;
-  if (T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
-  return MOE_OK;
-}
-
-int check_width(int64_t w) {
-  if (w < 1) return MOE_ERR_INVALID_ARG;
-  if (w % kTileMultiple != 0 || w > (int64_t(1) << 20)) return MOE_ERR_UNSUPPORTED;
-  return MOE_OK;
-}
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -271,16 +259,12 @@ int moe_permute(const void* x, const int32_t* topk_idx, int64_t T, int64_t d, in
                 int64_t k, double cf, int32_t* counts, int32_t* offsets, int32_t* slot,
                 int32_t* row_src, void* x_perm, int32_t* n_dropped, void* ws, size_t ws_bytes,
                 int32_t* dev_status, void* stream) {
-  int st = check_routing_shape(T, E, k);
-  if (st != MOE_OK) return st;
-  if ((st = check_width(d)) != MOE_OK) return st;
-  const int64_t C = moe_capacity(T, E, k, cf);
-  if (C < 0) return MOE_ERR_INVALID_ARG;
-  if (T == 0) return MOE_OK;
-  if (!x || !topk_idx || !counts || !offsets || !slot || !row_src || !x_perm || !n_dropped ||
-      !ws)
-    return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(x_perm) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  int64_t C = 0;
+  bool done = false;
+  int st = moe::abi::check_permute_args(x, topk_idx, T, d, E, k, cf, counts, offsets, slot,
+                                        row_src, x_perm, n_dropped, &C, &done);
+  if (st != MOE_OK || done) return st;
+  if (!ws || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_permute_workspace_size(T, E, k)) return MOE_ERR_WORKSPACE;
   return cuda_status(launch_permute(static_cast<const __nv_bfloat16*>(x), topk_idx, (int)T,
                                     (int)d, (int)E, (int)k, C, counts, offsets, slot, row_src,

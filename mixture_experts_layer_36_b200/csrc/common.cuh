@@ -35,6 +35,28 @@ __device__ __forceinline__ void report(int32_t* status, int32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel in the
+// stream is still running.  grid_dep_wait() blocks until that previous grid
+// has completed and its memory operations are visible; every read of data
+// the previous kernel produces must come after it.  grid_dep_launch() lets
+// the next kernel in the stream start its own launch early (it still waits
+// for this grid's completion before reading anything).  Both are no-ops for
+// a kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Bring `bytes` bytes at global address p into L2 (no registers, no
+// completion to wait for).  p 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -103,6 +103,25 @@ inline bool map_weights_e4m3(CUtensorMap* m, const void* base, uint64_t E, uint6
          CUDA_SUCCESS;
 }
 
+// Launch `kern` on `s` with programmatic stream serialization: the kernel may
+// begin while the previous kernel of the stream finishes (it must call
+// grid_dep_wait() before reading that kernel's results).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                   cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // attr_set slots: 0-2 grouped GEMM (1 CTA), 3-6 router GEMM, 7-8 grouped GEMM (CTA pair),
 // 9-10 CTA-pair GEMM on e4m3 operands, 11-13 grouped GEMM on e4m3 operands
 // (+16: the gathering instance of a grouped GEMM slot's kernel, +32: the

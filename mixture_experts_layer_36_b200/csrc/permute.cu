@@ -8,19 +8,24 @@
 //
 // slot(t, j) = number of tokens t' < t that also chose expert e = topk_idx[t,j]
 // (each expert appears at most once per token).  This is a stable counting
-// sort keyed by expert, done in two launches:
+// sort keyed by expert, in three launches:
 //   1. rank:    per chunk of 256 tokens, the rank of each pair among the
 //               chunk's pairs of the same expert (token order), plus the
 //               chunk's per-expert histogram;
-//   2. scan + scatter: each CTA sums the histograms into per-expert demand,
-//               kept = min(demand, C), offsets (exclusive scan over experts)
-//               and its chunk's base (prefix over earlier chunks); then
-//               slot = chunk base + rank, and kept pairs copy their token row
-//               into x_perm[offsets[e] + slot] with 16-byte vector loads and
-//               stores.
+//   2. scan:    per expert, the exclusive prefix of the histograms over the
+//               chunks (each chunk's base, written over its histogram) and
+//               the total demand (one extra row) — one pass, linear in T;
+//   3. scatter: per CTA of 8 tokens, kept = min(demand, C), offsets
+//               (exclusive scan over experts) and slot = chunk base + rank;
+//               kept pairs copy their token row into x_perm[offsets[e] + slot]
+//               with 16-byte vector loads and stores.
+// The launches are chained with programmatic dependent launch: the scatter
+// CTAs start while the rank and scan kernels run and pull their token rows
+// into L2 (bulk prefetch), so the row reads overlap the index work.
 // Rows are moved as bytes: bf16 rows, or e4m3 rows with their fp32 scale
 // (the FP8 layer quantizes each token once, before the permutation).
 #include "common.cuh"
+#include "host_util.cuh"
 
 namespace moe {
 
@@ -28,12 +33,9 @@ constexpr int kChunk = 256;            // tokens per rank/histogram chunk
 constexpr int kRankThreads = 1024;     // 32 warps x 8 tokens per chunk
 constexpr int kRankWarps = kRankThreads / 32;
 constexpr int kTokPerWarp = kChunk / kRankWarps;
+constexpr int kScanThreads = 1024;     // 32 warps; lane = one expert of a group of 32
 constexpr int kScatThreads = 256;      // 8 warps
-// tokens per scatter CTA (a divisor of kChunk): 8 (one per warp) keeps small
-// batches spread over many SMs; 32 (four per warp) when every CTA's pass over
-// the chunk histograms (nchunks x E counters) would be long
-constexpr int kScatTokensSmall = 8;
-constexpr int kScatTokensLarge = 32;
+constexpr int kScatTokens = 8;         // tokens per scatter CTA (one per warp; divides kChunk)
 
 // 1. rank: per chunk, the rank of each pair among the chunk's pairs of the
 //    same expert (token order), and the chunk's per-expert histogram.
@@ -48,6 +50,8 @@ __global__ void __launch_bounds__(kRankThreads)
   const int nt = min(kChunk, T - chunk_t0);
 
   for (int i = tid; i < kRankWarps * 256; i += kRankThreads) (&cnt[0][0])[i] = 0;
+  grid_dep_launch();
+  grid_dep_wait();          // topk_idx may come from the kernel before
   for (int i = tid; i < nt * k; i += kRankThreads) pairs[i] = topk_idx[(size_t)chunk_t0 * k + i];
   __syncthreads();
 
@@ -98,18 +102,49 @@ __global__ void __launch_bounds__(kRankThreads)
   }
 }
 
-// 2. scan + scatter: every CTA derives, from all chunk histograms, the
-//    per-expert kept counts and offsets (exclusive scan over experts) and its
-//    own chunk's per-expert base (exclusive prefix over earlier chunks); CTA 0
-//    also writes counts / offsets / n_dropped.  Then one warp per token turns
-//    ranks into slots, drops pairs at slot >= C, and copies the token row to
-//    its kept rows with 16-byte vectors.
+// 2. scan: per expert e (lane of a warp; 32 experts per CTA), the exclusive
+//    prefix of chunk_hist[., e] over the chunks, written in place, and the
+//    total demand in row nchunks.  Warp w takes a contiguous range of chunks:
+//    range sums, a prefix over the warps in shared memory, then the range is
+//    rewritten with its running prefix.
+__global__ void __launch_bounds__(kScanThreads)
+    permute_scan_kernel(int32_t* __restrict__ chunk_hist, int nchunks, int E) {
+  __shared__ int32_t part[32][33];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int e = blockIdx.x * 32 + lane;
+  const int per = (nchunks + 31) / 32;
+  const int c0 = min(nchunks, warp * per), c1 = min(nchunks, c0 + per);
+  grid_dep_launch();
+  grid_dep_wait();          // the rank kernel's histograms
+  int sum = 0;
+  if (e < E)
+    for (int c = c0; c < c1; ++c) sum += chunk_hist[(size_t)c * E + e];
+  part[warp][lane] = sum;
+  __syncthreads();
+  int run = 0;
+  for (int w = 0; w < warp; ++w) run += part[w][lane];
+  if (e < E) {
+    for (int c = c0; c < c1; ++c) {
+      const size_t i = (size_t)c * E + e;
+      const int v = chunk_hist[i];
+      chunk_hist[i] = run;
+      run += v;
+    }
+    if (warp == 31) chunk_hist[(size_t)nchunks * E + e] = run;
+  }
+}
+
+// 3. scatter: every CTA (8 tokens of one chunk) reads the per-expert demand
+//    and its chunk's base, derives kept counts and offsets (exclusive scan
+//    over experts); CTA 0 also writes counts / offsets / n_dropped.  Then one
+//    warp per token turns ranks into slots, drops pairs at slot >= C, and
+//    copies the token row to its kept rows with 16-byte vectors.
 __global__ void __launch_bounds__(kScatThreads)
     permute_scatter_kernel(const uint8_t* __restrict__ x, int row_bytes,
                            const float* __restrict__ x_scale,
                            const int32_t* __restrict__ topk_idx, int32_t* __restrict__ slot,
-                           const int32_t* __restrict__ chunk_hist, int nchunks, int T,
-                           int E, int k, int64_t C, int tokens_per_cta,
+                           const int32_t* __restrict__ chunk_base, int nchunks, int T,
+                           int E, int k, int64_t C,
                            int32_t* __restrict__ counts,
                            int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped,
                            int32_t* __restrict__ row_src, uint8_t* __restrict__ x_perm,
@@ -121,21 +156,24 @@ __global__ void __launch_bounds__(kScatThreads)
   __shared__ int32_t warp_sum[8];
   __shared__ int32_t warp_drop[8];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int t0 = blockIdx.x * tokens_per_cta;
+  const int t0 = blockIdx.x * kScatTokens;
   const int my_chunk = t0 / kChunk;
+
+  // this CTA's token rows into L2 while the rank and scan kernels finish
+  if (x && lane == 0) {
+    for (int tt = warp; tt < kScatTokens; tt += kScatThreads / 32)
+      if (t0 + tt < T) prefetch_l2_bulk(x + (size_t)(t0 + tt) * row_bytes, row_bytes);
+  }
+  grid_dep_launch();
+  grid_dep_wait();          // ranks in slot, chunk bases and totals
 
   // ---- per-expert totals, kept, chunk base (thread e owns expert e)
   int kept = 0, drop = 0;
   if (tid < E) {
-    int total = 0, base = 0;
-    for (int c = 0; c < nchunks; ++c) {
-      const int v = chunk_hist[(size_t)c * E + tid];
-      if (c < my_chunk) base += v;
-      total += v;
-    }
+    const int total = chunk_base[(size_t)nchunks * E + tid];
+    s_base[tid] = chunk_base[(size_t)my_chunk * E + tid];
     kept = (int64_t)total < C ? total : (int)C;
     drop = total - kept;
-    s_base[tid] = base;
   }
   int incl = kept;
 #pragma unroll
@@ -173,7 +211,7 @@ __global__ void __launch_bounds__(kScatThreads)
 
   // ---- one warp per token
   const int nvec = row_bytes / 16;
-  for (int tt = warp; tt < tokens_per_cta; tt += kScatThreads / 32) {
+  for (int tt = warp; tt < kScatTokens; tt += kScatThreads / 32) {
     const int t = t0 + tt;
     if (t >= T) break;
     int my_row = -1;
@@ -223,9 +261,10 @@ __global__ void __launch_bounds__(kScatThreads)
   }
 }
 
+// Scratch: the per-chunk histograms (then bases) and one row of totals.
 size_t permute_scratch_bytes(int64_t T, int64_t E) {
   const int64_t nchunks = (T + kChunk - 1) / kChunk;
-  return (size_t)(nchunks * E * (int64_t)sizeof(int32_t));
+  return (size_t)((nchunks + 1) * E * (int64_t)sizeof(int32_t));
 }
 
 // 3. padded layout only: rows of each bucket past its kept count are zeroed
@@ -235,6 +274,7 @@ __global__ void __launch_bounds__(256)
                             int32_t* __restrict__ row_src, uint8_t* __restrict__ x_pad) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t r = (int64_t)blockIdx.x * 8 + warp;
+  grid_dep_wait();          // the scatter's counts
   if (r >= (int64_t)E * C) return;
   const int e = (int)(r / C);
   if (r - (int64_t)e * C < counts[e]) return;
@@ -247,6 +287,16 @@ __global__ void __launch_bounds__(256)
 // per row, moved with it) may be null; x null: no row copy (index-only), with
 // row_pair (t*k + j of each kept row) and zeroed fp32 rows zero_rows[T,
 // zero_cols] for the fused combine when those are non-null.
+static cudaError_t launch_rank_scan(const int32_t* topk_idx, int T, int E, int k, int32_t* slot,
+                                    int32_t* chunk_hist, cudaStream_t s, int32_t* status) {
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  cudaError_t err = launch_dependent(permute_rank_kernel, dim3(nchunks), dim3(kRankThreads), 0, s,
+                                     topk_idx, T, E, k, slot, chunk_hist, status);
+  if (err != cudaSuccess) return err;
+  return launch_dependent(permute_scan_kernel, dim3((E + 31) / 32), dim3(kScanThreads), 0, s,
+                          chunk_hist, nchunks, E);
+}
+
 cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_scale,
                                 const int32_t* topk_idx, int T, int E, int k, int64_t C,
                                 int32_t* counts, int32_t* offsets, int32_t* slot,
@@ -255,13 +305,12 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
                                 int32_t* row_pair, float* zero_rows, int zero_cols,
                                 int32_t* status) {
   const int nchunks = (T + kChunk - 1) / kChunk;
-  permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist,
-                                                       status);
-  const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
-  permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
-      x, row_bytes, x_scale, topk_idx, slot, chunk_hist, nchunks, T, E, k, C, tpc, counts,
-      offsets, n_dropped, row_src, x_perm, perm_scale, false, row_pair, zero_rows, zero_cols);
-  return cudaGetLastError();
+  cudaError_t err = launch_rank_scan(topk_idx, T, E, k, slot, chunk_hist, s, status);
+  if (err != cudaSuccess) return err;
+  return launch_dependent(permute_scatter_kernel, dim3((T + kScatTokens - 1) / kScatTokens),
+                          dim3(kScatThreads), 0, s, x, row_bytes, x_scale, topk_idx, slot,
+                          chunk_hist, nchunks, T, E, k, C, counts, offsets, n_dropped, row_src,
+                          x_perm, perm_scale, false, row_pair, zero_rows, zero_cols);
 }
 
 // The padded [E, C, d] layout: bucket e holds rows e*C .. e*C + C - 1, its
@@ -272,17 +321,17 @@ cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_id
                                   int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
                                   int32_t* status) {
   const int nchunks = (T + kChunk - 1) / kChunk;
-  permute_rank_kernel<<<nchunks, kRankThreads, 0, s>>>(topk_idx, T, E, k, slot, chunk_hist,
-                                                       status);
-  const int tpc = (int64_t)nchunks * E <= 1024 ? kScatTokensSmall : kScatTokensLarge;
+  cudaError_t err = launch_rank_scan(topk_idx, T, E, k, slot, chunk_hist, s, status);
+  if (err != cudaSuccess) return err;
   uint8_t* xp = reinterpret_cast<uint8_t*>(x_pad);
-  permute_scatter_kernel<<<(T + tpc - 1) / tpc, kScatThreads, 0, s>>>(
-      reinterpret_cast<const uint8_t*>(x), d * 2, nullptr, topk_idx, slot, chunk_hist, nchunks, T,
-      E, k, C, tpc, counts, offsets, n_dropped, row_src, xp, nullptr, true, nullptr, nullptr, 0);
+  err = launch_dependent(permute_scatter_kernel, dim3((T + kScatTokens - 1) / kScatTokens),
+                         dim3(kScatThreads), 0, s, reinterpret_cast<const uint8_t*>(x), d * 2,
+                         nullptr, topk_idx, slot, chunk_hist, nchunks, T, E, k, C, counts,
+                         offsets, n_dropped, row_src, xp, nullptr, true, nullptr, nullptr, 0);
+  if (err != cudaSuccess) return err;
   const int64_t rows = (int64_t)E * C;
-  permute_pad_fill_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(counts, E, C, d * 2, row_src,
-                                                                     xp);
-  return cudaGetLastError();
+  return launch_dependent(permute_pad_fill_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0,
+                          s, counts, E, C, d * 2, row_src, xp);
 }
 
 cudaError_t launch_permute(const __nv_bfloat16* x, const int32_t* topk_idx, int T, int d, int E,

@@ -6,15 +6,15 @@
 // runtime that plans every device byte at start-up and fails (or stalls the
 // device) on any later cudaMalloc.  They cannot call cudaMalloc themselves and
 // cannot give moe_permute its `ws` argument.  This entry point runs the same
-// three permutation kernels as moe_permute, but their per-chunk bucket
-// histograms live in a fixed array compiled into the library, so nothing is
-// allocated at call time.
+// permutation kernels as moe_permute, but their per-chunk bucket counters
+// live in a fixed array compiled into the library, so nothing is allocated at
+// call time.
 //
 // Costs and limits of that choice:
-//   * the array (kNoAllocScratchInts int32, 256 KiB) is resident on every GPU
+//   * the array (kNoAllocScratchInts int32, 257 KiB) is resident on every GPU
 //     that loads the library, until the process exits;
-//   * it holds ceil(T/256) * E counters, so a call with more than that is
-//     rejected with MOE_ERR_WORKSPACE (e.g. E = 256 allows T <= 65536);
+//   * it holds (ceil(T/256) + 1) * E counters, so a call needing more is
+//     rejected with MOE_ERR_WORKSPACE (E = 256 allows T <= 65536);
 //   * every call uses the same array: two calls whose kernels overlap on the
 //     GPU (different streams, or different host threads on one device) race
 //     and corrupt each other's result.  Serialise them, e.g. on one stream;
@@ -25,6 +25,7 @@
 //     that first call before any stream capture begins.
 #include <mutex>
 
+#include "abi_checks.cuh"
 #include "common.cuh"
 
 namespace moe {
@@ -37,7 +38,8 @@ size_t permute_scratch_bytes(int64_t T, int64_t E);
 
 namespace {
 
-constexpr int64_t kNoAllocScratchInts = 65536;   // 256 KiB of int32 counters
+// 256 rows of 256 experts' chunk counters plus the row of totals
+constexpr int64_t kNoAllocScratchInts = 65536 + 256;
 
 static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocScratchInts];
 
@@ -69,25 +71,20 @@ cudaError_t scratch_address(int32_t** out) {
 extern "C" int moe_permute_noalloc(const void* x, const int32_t* topk_idx, int64_t T, int64_t d,
                                    int64_t E, int64_t k, double cf, int32_t* counts,
                                    int32_t* offsets, int32_t* slot, int32_t* row_src,
-                                   void* x_perm, int32_t* n_dropped, void* stream) {
-  if (T < 0 || E < 1 || E > 256 || k < 1 || k > 8 || k > E || T * k >= (int64_t(1) << 31))
-    return MOE_ERR_INVALID_ARG;
-  if (d < 1) return MOE_ERR_INVALID_ARG;
-  if (d % 128 != 0 || d > (int64_t(1) << 20)) return MOE_ERR_UNSUPPORTED;
-  const int64_t C = moe_capacity(T, E, k, cf);
-  if (C < 0) return MOE_ERR_INVALID_ARG;
-  if (T == 0) return MOE_OK;
-  if (!x || !topk_idx || !counts || !offsets || !slot || !row_src || !x_perm || !n_dropped)
-    return MOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u))
-    return MOE_ERR_INVALID_ARG;
+                                   void* x_perm, int32_t* n_dropped, int32_t* dev_status,
+                                   void* stream) {
+  int64_t C = 0;
+  bool done = false;
+  const int st = moe::abi::check_permute_args(x, topk_idx, T, d, E, k, cf, counts, offsets, slot,
+                                              row_src, x_perm, n_dropped, &C, &done);
+  if (st != MOE_OK || done) return st;
   if (moe::permute_scratch_bytes(T, E) > size_t(kNoAllocScratchInts) * sizeof(int32_t))
     return MOE_ERR_WORKSPACE;
   int32_t* scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaError_t err = moe::launch_permute(
+  cudaError_t err = scratch_address(&scratch);
+  if (err != cudaSuccess) return moe::abi::cuda_status(err);
+  return moe::abi::cuda_status(moe::launch_permute(
       static_cast<const __nv_bfloat16*>(x), topk_idx, (int)T, (int)d, (int)E, (int)k, C, counts,
       offsets, slot, row_src, static_cast<__nv_bfloat16*>(x_perm), n_dropped, scratch,
-      reinterpret_cast<cudaStream_t>(stream), nullptr);
-  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+      reinterpret_cast<cudaStream_t>(stream), dev_status));
 }

@@ -62,6 +62,11 @@ def num_threads() -> int:
     return lib().oracle_num_threads()
 
 
+def set_num_threads(n: int) -> None:
+    """Threads the calling host thread's oracle calls use (per host thread)."""
+    lib().oracle_set_num_threads(ctypes.c_int(int(n)))
+
+
 def capacity(T, E, k, cf) -> int:
     return int(lib().oracle_capacity(T, E, k, float(cf)))
 

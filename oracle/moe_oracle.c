@@ -66,6 +66,17 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads the calling host thread's parallel regions use from now on (a
+ * per-thread setting: a test that calls the oracle from several host threads
+ * at once gives each a share of the cores).  No effect on any result. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Step 3.  cf == 0 selects the dropless layer: an expert can receive each
  * token at most once, so C = T never drops.  Evaluated as ((cf*k)*T)/E in
  * fp64, then rounded up. */

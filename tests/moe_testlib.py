@@ -95,3 +95,42 @@ def random_routing(T, E, k, seed, skew=1.2):
     p /= p.sum()
     keys = r.random((T, E)) ** (1.0 / p)      # weighted sampling without replacement
     return np.argsort(-keys, axis=1)[:, :k].astype(np.int32)
+
+
+# Precision of h in the oracle's expert.  The contract is the plain fp64
+# definition (h_bf16=False: no rounding anywhere in the MLP); the bf16-rounded
+# h (h_bf16=True) models the GEMMs' bf16 operand and serves as a diagnostic.
+# Layer-level outputs are compared with both, at the same tolerance.
+H_MODES = (False, True)
+
+
+def every_expert_rows(offsets, seed):
+    """Rows of the permuted buffers that cover every non-empty bucket: the
+    bucket's last row (its tail tile) and one more row drawn at random.
+    Returns {expert: sorted rows}."""
+    rng = np.random.default_rng(seed)
+    picks = {}
+    for e in range(len(offsets) - 1):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            picks[e] = sorted({hi - 1, int(rng.integers(lo, hi))})
+    return picks
+
+
+def map_experts(fn, experts, workers=None):
+    """{e: fn(e)} for every expert, on a pool of host threads (the oracle's C
+    calls release the GIL); each thread's oracle calls use a share of the
+    cores."""
+    from concurrent.futures import ThreadPoolExecutor
+    experts = list(experts)
+    if not experts:
+        return {}
+    cores = oracle.num_threads()
+    workers = workers or max(1, min(8, cores // 2, len(experts)))
+    share = max(1, cores // workers)
+
+    def run(e):
+        oracle.set_num_threads(share)
+        return e, fn(e)
+    with ThreadPoolExecutor(workers) as ex:
+        return dict(ex.map(run, experts))

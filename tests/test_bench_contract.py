@@ -43,8 +43,8 @@ def test_gpu_arm_json(extra):
     import torch
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    r = _run(["--config", "tiny", "--steps", "3", "--warmup", "3", "--no-cpu-baseline", *extra],
-             800)
+    r = _run(["--config", "tiny", "--steps", "3", "--warmup", "3", "--no-cpu-baseline",
+              "--no-per-config", *extra], 800)
     assert BASE_KEYS <= set(r)
     assert r["value"] > 0 and r["device_status"] == 0 and r["gpu_launches"] > 0
     rf = r["roofline"]
@@ -59,19 +59,19 @@ def test_gpu_arm_json(extra):
 
 def test_launches_per_step():
     """The gpu_launches arithmetic (checked against the CUDA profiler's count by
-    tests/test_gpu_launch_count.py): 8 launches with a split router K, one fewer
+    tests/test_gpu_launch_count.py): 9 launches with a split router K, one fewer
     when the router's top-k runs in its GEMM epilogue, +2 row quantizers for
     FP8 experts, +1 fill for the padded layout."""
     import sys
     sys.path.insert(0, ROOT)
     import bench
     from mixture_experts_layer_36_b200 import configs
-    assert bench.launches_per_step(configs.MIXTRAL, 148) == 8              # 32 row tiles
-    assert bench.launches_per_step(configs.SKEWED, 148) == 7               # 128 row tiles
-    assert bench.launches_per_step(configs.SKEWED, 148, fp8=True) == 9
-    assert bench.launches_per_step(configs.FINE, 148, padded=True) == 9
-    assert bench.launches_per_step(configs.FINE, 148, fused=True) == 8
-    assert bench.launches_per_step(configs.DECODE.with_tokens(16), 148, fp8=True) == 10
+    assert bench.launches_per_step(configs.MIXTRAL, 148) == 9              # 32 row tiles
+    assert bench.launches_per_step(configs.SKEWED, 148) == 8               # 128 row tiles
+    assert bench.launches_per_step(configs.SKEWED, 148, fp8=True) == 10
+    assert bench.launches_per_step(configs.FINE, 148, padded=True) == 10
+    assert bench.launches_per_step(configs.FINE, 148, fused=True) == 9
+    assert bench.launches_per_step(configs.DECODE.with_tokens(16), 148, fp8=True) == 11
     assert bench.launches_per_step(configs.TINY.with_tokens(0), 148) == 0
 
 
@@ -123,7 +123,8 @@ def test_gpu_arm_json_assembly_on_cpu(monkeypatch, capsys, extra, stages):
     monkeypatch.setattr(torch.cuda, "get_device_properties",
                         lambda *_: types.SimpleNamespace(multi_processor_count=148))
     monkeypatch.setattr(sys, "argv", ["bench.py", "--config", "skewed", "--steps", "4",
-                                      "--warmup", "3", "--no-cpu-baseline", *extra])
+                                      "--warmup", "3", "--no-cpu-baseline", "--no-per-config",
+                                      *extra])
     bench.main()
     lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -141,3 +142,68 @@ def test_gpu_arm_json_assembly_on_cpu(monkeypatch, capsys, extra, stages):
             4.0 * 30000 * cfg.d * cfg.f / (mean["gate_up"] / 1e3) / 1e12, rel=1e-3)
     assert r["stages_mean_ms"] == {n: round(v, 4) for n, v in mean.items()}
     assert set(r["stages_ms"]) == set(stages)
+
+
+def test_per_config_assembly_on_cpu(monkeypatch, capsys):
+    """per_config from fixed numbers (CPU): one entry per workload, the headline
+    first, each roofline fraction recomputing from its own line."""
+    import sys
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch
+    from mixture_experts_layer_36_b200 import configs
+    stages = ["route", "permute", "gate_up", "down", "combine"]
+    seen = []
+
+    def fake_arm(args, c, rank, world, local_rank, with_e2e=True):
+        seen.append((c.name, with_e2e))
+        mean = {n: 0.05 * (i + 1) for i, n in enumerate(stages)}
+        N = min(c.T * c.k, bench.moe_max_rows_host(c))
+        r = {"elapsed_ms": 2.0 * args.steps, "stage_ms": dict(mean), "stage_mean": mean,
+             "status": 0, "N": N, "active_experts": min(c.E, N), "n_dropped": c.T * c.k - N,
+             "clocks": {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": []},
+             "layer": types.SimpleNamespace(rows=N)}
+        if with_e2e:
+            r.update(e2e_ms=3.0 * args.steps, h2d=c.T * c.d * 2, d2h=c.T * c.d * 2)
+        return r
+
+    monkeypatch.setattr(bench, "gpu_arm", fake_arm)
+    monkeypatch.setattr(torch.cuda, "get_device_properties",
+                        lambda *_: types.SimpleNamespace(multi_processor_count=148))
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "4", "--warmup", "3",
+                                      "--no-cpu-baseline"])
+    bench.main()
+    r = json.loads([ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")][0])
+    per = r["per_config"]
+    want = [configs.by_name(n).name for n in bench.PER_CONFIG]
+    assert list(per)[0] == "mixtral" and sorted(per) == sorted(want)
+    assert seen[0] == ("mixtral", True) and all(not e for _, e in seen[1:])
+    for name, e in per.items():
+        c = configs.by_name(name)
+        assert e["tokens_per_s"] == pytest.approx(c.T * 4 / (8.0e-3), rel=1e-6)
+        rf = e["roofline"]
+        assert rf["frac"] == pytest.approx(rf["achieved"] / rf["peak"], abs=1e-3)
+        for st in ("permute", "combine"):
+            h = e["stage_rooflines"][st]
+            assert h["achieved"] == pytest.approx(
+                h["algorithmic_bytes"] / (h["duration_ms"] / 1e3) / 1e9, rel=1e-3)
+            assert h["frac"] == pytest.approx(h["achieved"] / h["peak"], abs=1e-3)
+    # decode sizes are weight-streaming: bound by HBM on the active experts' weights
+    assert per["decode@T16"]["roofline"]["bound"] == "hbm"
+    assert per["mixtral"]["roofline"]["bound"] == "tensor"
+
+
+def test_reference_arm_config_equals_gpu_arm_config():
+    """Both arms describe the workload with the same `config` object."""
+    import argparse
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_36_b200 import configs
+    args = argparse.Namespace(fp8=False, fused=False, layout="ragged")
+    for name in bench.PER_CONFIG:
+        c = configs.by_name(name)
+        assert bench.workload_config(c, args, 1) == bench.workload_config(c, args, 1)
+    ref = _run(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "3"], 300)
+    assert ref["config"] == bench.workload_config(configs.TINY, args, 1)

@@ -15,8 +15,8 @@ import torch.distributed as dist
 import oracle
 import mixture_experts_layer_36_b200 as moe
 from mixture_experts_layer_36_b200 import ep
-from moe_testlib import assert_bf16_close, assert_bf16_rounding_close, bits, cuda_inputs, f64, \
-    small
+from moe_testlib import (H_MODES, assert_bf16_close, assert_bf16_rounding_close, bits,
+                         cuda_inputs, f64, small)
 
 pytestmark = pytest.mark.gpu
 
@@ -93,10 +93,11 @@ def test_expert_parallel_one_rank_matches_oracle(cfg, one_rank_group):
     logits, _, _ = moe.moe_route(inp["x"], inp["w_router"], inp["bias"], cfg.k)
     torch.cuda.synchronize()
     bias = None if cpu["bias"] is None else cpu["bias"].numpy()
-    ref = oracle.moe_forward(bits(cpu["x"]), cpu["w_router"].numpy(), bias, bits(cpu["w_gate"]),
-                             bits(cpu["w_up"]), bits(cpu["w_down"]), cfg.k, cfg.cf,
-                             decision_logits=logits.cpu().numpy())
-    assert_bf16_close(f64(y), ref["y"], "y")
+    for hb in H_MODES:       # h in fp64 (the definition) and rounded to bf16
+        ref = oracle.moe_forward(bits(cpu["x"]), cpu["w_router"].numpy(), bias,
+                                 bits(cpu["w_gate"]), bits(cpu["w_up"]), bits(cpu["w_down"]),
+                                 cfg.k, cfg.cf, decision_logits=logits.cpu().numpy(), h_bf16=hb)
+        assert_bf16_close(f64(y), ref["y"], f"y, h_bf16={hb}")
     dropped = (ref["slot"] < 0).all(axis=1)
     if dropped.any():
         np.testing.assert_array_equal(bits(y)[dropped], bits(cpu["x"])[dropped])

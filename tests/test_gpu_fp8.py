@@ -18,7 +18,8 @@ import oracle
 import mixture_experts_layer_36_b200 as moe
 from mixture_experts_layer_36_b200 import configs, synth
 from moe_testlib import (WEIGHT_ATOL, assert_bf16_close, assert_bf16_rounding_close,
-                         assert_logits_close, bits, cuda_inputs, f64, small)
+                         assert_logits_close, bits, cuda_inputs, every_expert_rows, f64,
+                         map_experts, small)
 
 pytestmark = pytest.mark.gpu
 
@@ -301,9 +302,11 @@ FULL = [configs.MIXTRAL, configs.FINE, configs.SKEWED] + \
 def test_fp8_full_size_sampled(cfg):
     """Full-size layer with FP8 experts quantized on the GPU, in the launch
     configuration the benchmark times: routing and slots exact for every
-    token; for two sampled tokens (and, where the capacity drops some, one
-    whose every pair is dropped) the weight codes of their experts bit-exact
-    and their outputs from the oracle."""
+    token; for every expert that received rows, its weight codes bit-exact
+    and two of its rows (the bucket's last, in the tail tile, and one more)
+    through both GEMMs against the oracle; for two sampled tokens (and, where
+    the capacity drops some, one whose every pair is dropped) the layer
+    output from the oracle."""
     torch.cuda.empty_cache()
     w = synth.make_weights(cfg, "cuda")
     x = synth.make_tokens(cfg, "cuda")
@@ -316,16 +319,41 @@ def test_fp8_full_size_sampled(cfg):
     o_idx, o_w = oracle.topk(gl, cfg.k)
     np.testing.assert_array_equal(_ws(ws, "topk_idx", cfg).cpu().numpy(), o_idx)
     C = oracle.capacity(cfg.T, cfg.E, cfg.k, cfg.cf)
-    _, offsets, slot, _, n_drop = oracle.permute(o_idx, cfg.E, C)
+    counts, offsets, slot, row_src, n_drop = oracle.permute(o_idx, cfg.E, C)
     np.testing.assert_array_equal(_ws(ws, "slot", cfg).cpu().numpy(), slot)
     assert _ws(ws, "n_dropped", cfg).item() == n_drop
+    x_bits = bits(x)
+
+    # every expert with rows: codes of its weights, then two of its rows
+    # through the gate/up GEMM (h) and the down GEMM (y_perm)
+    picks = every_expert_rows(offsets, cfg.seed + 3)
+    assert len(picks) == int((counts > 0).sum())
+    h_all, yp_all = _ws(ws, "h", cfg), _ws(ws, "y_perm", cfg)
+
+    def expert_ref(e):
+        mats = []
+        for n in ("w_gate", "w_up", "w_down"):
+            q_ref, s_ref = quantize_w(w[n][e:e + 1].cpu())
+            assert np.array_equal(qw[n][0][e].cpu().numpy().T, q_ref[0]), (n, e)
+            assert np.array_equal(qw[n][1][e].cpu().numpy(), s_ref[0]), (n, e)
+            mats.append(oracle.dequant_fp8(q_ref, s_ref)[0])
+        rows = torch.tensor(picks[e], device="cuda").long()
+        a = deq_rows(*oracle.quantize_rows_fp8(x_bits[row_src[picks[e]]]))
+        h_ref = oracle.gate_up_f64(a, mats[0], mats[1])
+        h_rows = h_all[rows]
+        hq, sh = oracle.quantize_rows_fp8(bits(h_rows))
+        return (f64(h_rows), h_ref, f64(yp_all[rows]),
+                oracle.matmul_f64(deq_rows(hq, sh), mats[2]))
+    refs = map_experts(expert_ref, picks)
+    cat = lambda i: np.concatenate([refs[e][i] for e in picks])  # noqa: E731
+    assert_bf16_rounding_close(cat(0), cat(1), f"h, {len(picks)} experts")
+    assert_bf16_close(cat(2), cat(3), f"y_perm, {len(picks)} experts")
 
     rng = np.random.default_rng(cfg.seed + 1)
     toks = list(np.sort(rng.choice(cfg.T, size=2, replace=False)))
     all_dropped = np.flatnonzero((slot < 0).all(axis=1))
     if len(all_dropped):
         toks.append(int(all_dropped[0]))
-    x_bits = bits(x)
     h_gpu = _ws(ws, "h", cfg)
     y_ref = np.zeros((len(toks), cfg.d))
     for i, t in enumerate(toks):

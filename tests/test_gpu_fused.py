@@ -16,7 +16,8 @@ import torch
 import oracle
 import mixture_experts_layer_36_b200 as moe
 from mixture_experts_layer_36_b200 import configs, synth
-from moe_testlib import (WEIGHT_ATOL, assert_bf16_close, bits, cuda_inputs, f64, random_routing,
+from moe_testlib import (H_MODES, WEIGHT_ATOL, assert_bf16_close, assert_bf16_rounding_close,
+                         bits, cuda_inputs, every_expert_rows, f64, map_experts, random_routing,
                          small)
 
 pytestmark = pytest.mark.gpu
@@ -97,15 +98,16 @@ def test_layer_forward_fused_matches_oracle(cfg):
     assert view("status").item() == 0
     gl = view("logits").cpu().numpy()
     bias = None if cpu["bias"] is None else cpu["bias"].numpy()
-    ref = oracle.moe_forward(bits(cpu["x"]), cpu["w_router"].numpy(), bias, bits(cpu["w_gate"]),
-                             bits(cpu["w_up"]), bits(cpu["w_down"]), cfg.k, cfg.cf,
-                             decision_logits=gl)
+    for hb in H_MODES:       # h in fp64 (the definition) and rounded to bf16
+        ref = oracle.moe_forward(bits(cpu["x"]), cpu["w_router"].numpy(), bias,
+                                 bits(cpu["w_gate"]), bits(cpu["w_up"]), bits(cpu["w_down"]),
+                                 cfg.k, cfg.cf, decision_logits=gl, h_bf16=hb)
+        assert_bf16_close(f64(y), ref["y"], f"y, h_bf16={hb}")
     np.testing.assert_array_equal(view("topk_idx").cpu().numpy(), ref["topk_idx"])
     assert np.max(np.abs(view("topk_w").cpu().double().numpy() - ref["topk_w"])) <= WEIGHT_ATOL
     np.testing.assert_array_equal(view("slot").cpu().numpy(), ref["slot"])
     np.testing.assert_array_equal(view("offsets").cpu().numpy(), ref["offsets"])
     assert view("n_dropped").item() == ref["n_dropped"]
-    assert_bf16_close(f64(y), ref["y"], "y")
     dropped = (ref["slot"] < 0).all(axis=1)
     if dropped.any():
         np.testing.assert_array_equal(bits(y)[dropped], bits(cpu["x"])[dropped])
@@ -122,8 +124,10 @@ FULL = [configs.MIXTRAL, configs.DECODE.with_tokens(64)]
 @pytest.mark.parametrize("cfg", FULL, ids=[c.name for c in FULL])
 def test_fused_full_size_sampled(cfg):
     """Full-size fused layer against the unfused one on every token (same
-    routing and rows; only the order of each token's k-term sum differs) and
-    against the oracle on sampled tokens."""
+    routing and rows; only the order of each token's k-term sum differs),
+    its gate/up rows against the oracle for every expert that received rows
+    (the bucket's last row and one more), and its output against the oracle
+    on sampled tokens."""
     torch.cuda.empty_cache()
     w = synth.make_weights(cfg, "cuda")
     x = synth.make_tokens(cfg, "cuda")
@@ -138,24 +142,39 @@ def test_fused_full_size_sampled(cfg):
     gl = view("logits").cpu().numpy()
     o_idx, o_w = oracle.topk(gl, cfg.k)
     C = oracle.capacity(cfg.T, cfg.E, cfg.k, cfg.cf)
-    _, _, slot, _, _ = oracle.permute(o_idx, cfg.E, C)
+    counts, offsets, slot, row_src, _ = oracle.permute(o_idx, cfg.E, C)
+    np.testing.assert_array_equal(view("row_src")[:int(offsets[-1])].cpu().numpy(), row_src)
+    x_bits = bits(x)
+    # every expert with rows: h rows of the gathering-free gate/up GEMM
+    picks = every_expert_rows(offsets, cfg.seed + 5)
+    assert len(picks) == int((counts > 0).sum())
+    h_all = view("h")
+
+    def expert_h(e):
+        h_ref, _ = oracle.swiglu_rows(x_bits[row_src[picks[e]]], bits(w["w_gate"][e]),
+                                      bits(w["w_up"][e]), bits(w["w_down"][e]), want_h=True)
+        return f64(h_all[torch.tensor(picks[e], device="cuda").long()]), h_ref
+    refs = map_experts(expert_h, picks)
+    assert_bf16_rounding_close(np.concatenate([refs[e][0] for e in picks]),
+                               np.concatenate([refs[e][1] for e in picks]),
+                               f"h, {len(picks)} experts")
     rng = np.random.default_rng(cfg.seed + 2)
     toks = np.sort(rng.choice(cfg.T, size=3, replace=False))
     if (slot < 0).all(axis=1).any():          # and a token whose every pair is dropped
         toks = np.unique(np.append(toks, np.nonzero((slot < 0).all(axis=1))[0][0]))
-    x_bits = bits(x)
-    y_ref = np.zeros((len(toks), cfg.d))
-    for i, t in enumerate(toks):
-        for j in range(cfg.k):
-            if slot[t, j] < 0:
-                continue
-            e = int(o_idx[t, j])
-            _, o = oracle.swiglu_rows(x_bits[t:t + 1], bits(w["w_gate"][e]), bits(w["w_up"][e]),
-                                      bits(w["w_down"][e]))
-            y_ref[i] += o_w[t, j] * o[0]
     y_s = y[torch.from_numpy(toks).cuda().long()]
     moe_rows = ~(slot[toks] < 0).all(axis=1)
-    assert_bf16_close(f64(y_s)[moe_rows], y_ref[moe_rows], "y (sampled)")
+    for hb in H_MODES:       # h in fp64 (the definition) and rounded to bf16
+        y_ref = np.zeros((len(toks), cfg.d))
+        for i, t in enumerate(toks):
+            for j in range(cfg.k):
+                if slot[t, j] < 0:
+                    continue
+                e = int(o_idx[t, j])
+                _, o = oracle.swiglu_rows(x_bits[t:t + 1], bits(w["w_gate"][e]),
+                                          bits(w["w_up"][e]), bits(w["w_down"][e]), h_bf16=hb)
+                y_ref[i] += o_w[t, j] * o[0]
+        assert_bf16_close(f64(y_s)[moe_rows], y_ref[moe_rows], f"y (sampled), h_bf16={hb}")
     np.testing.assert_array_equal(bits(y_s)[~moe_rows], x_bits[toks[~moe_rows]])
     del w, x, y, y2, ws
     torch.cuda.empty_cache()

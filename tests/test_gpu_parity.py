@@ -20,8 +20,9 @@ import torch
 import oracle
 import mixture_experts_layer_36_b200 as moe
 from mixture_experts_layer_36_b200 import configs, synth
-from moe_testlib import (WEIGHT_ATOL, LOGIT_RTOL, assert_bf16_close, assert_bf16_rounding_close,
-                         assert_logits_close, bits, cuda_inputs, f64, random_routing, small)
+from moe_testlib import (H_MODES, WEIGHT_ATOL, LOGIT_RTOL, assert_bf16_close,
+                         assert_bf16_rounding_close, assert_logits_close, bits, cuda_inputs,
+                         every_expert_rows, f64, map_experts, random_routing, small)
 
 pytestmark = pytest.mark.gpu
 
@@ -141,11 +142,42 @@ def test_route_unsplit_ties_take_lower_index(pattern, k, want):
     assert np.max(np.abs(w.cpu().double().numpy() - o_w)) <= WEIGHT_ATOL
 
 
+# Few tokens and a wide d: the router splits K 8 or more ways (one 128-token
+# row tile, d / 64 k-blocks), and the top-k kernel then reduces one token's
+# partial sums with all 8 warps.  E = 256 puts 8 experts on every lane, and the
+# tied values below sit on different lanes and on different slots of one lane.
+def _tie_bias(E):
+    b = torch.zeros(E)
+    b[[13, 77, 141, 200]] = 2.0            # lanes 13, 13, 13, 8: one value, four experts
+    b[[0, 31, 32, 64, 255]] = 1.0          # lanes 0, 31, 0, 0, 31
+    b[[1, 33, 254]] = 0.5
+    return b
+
+
+@pytest.mark.parametrize("d", [512, 1024, 4096])
+def test_route_split_k_ties_across_lanes(d):
+    E, k, T = 256, 8, 97
+    g = torch.Generator().manual_seed(d)
+    x = torch.zeros(T, d, dtype=torch.bfloat16)
+    x[::4] = torch.randn(x[::4].shape, generator=g).to(torch.bfloat16)   # some untied rows
+    wr = torch.randn(d, E, generator=g) / d ** 0.5
+    bias = _tie_bias(E)
+    logits, idx, w = moe.moe_route(x.cuda(), wr.cuda(), bias.cuda(), k)
+    torch.cuda.synchronize()
+    gl = logits.cpu().numpy()
+    assert_logits_close(gl, oracle.router_logits(bits(x), wr.numpy(), bias.numpy()))
+    o_idx, o_w = oracle.topk(gl, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), o_idx)
+    # an all-tied row (x = 0): the four 2.0s, then the 1.0s by expert index
+    assert o_idx[1].tolist() == [13, 77, 141, 200, 0, 31, 32, 64]
+    assert np.max(np.abs(w.cpu().double().numpy() - o_w)) <= WEIGHT_ATOL
+
+
 # ----------------------------------------------------------------------------- stage: permute
 
 PERM_CASES = [(64, 128, 8, 2, 1.25), (1000, 256, 64, 6, 1.0), (777, 128, 256, 8, 1.25),
               (513, 128, 8, 2, 0.0), (300, 128, 5, 5, 0.3), (257, 384, 3, 1, 0.5),
-              (4096, 256, 256, 8, 0.2)]
+              (4096, 256, 256, 8, 0.2), (65536, 128, 256, 8, 1.0)]
 
 
 @pytest.mark.parametrize("T,d,E,k,cf", PERM_CASES)
@@ -251,8 +283,12 @@ def _ws(ws, name, cfg):
     return moe.workspace_view(ws, name, cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.cf)
 
 
+@pytest.mark.parametrize("h_bf16", H_MODES, ids=["h_fp64", "h_bf16"])
 @pytest.mark.parametrize("cfg", SMALL, ids=IDS)
-def test_layer_forward_matches_oracle(cfg):
+def test_layer_forward_matches_oracle(cfg, h_bf16):
+    """The whole layer against the oracle: h_fp64 is the plain definition
+    (the MLP in fp64 throughout), h_bf16 the oracle with h rounded to bf16
+    like the GEMMs' operand; the same tolerance holds for both."""
     inp, cpu = cuda_inputs(cfg)
     y, ws = moe.moe_layer_forward(inp["x"], inp["w_router"], inp["bias"], inp["w_gate"],
                                   inp["w_up"], inp["w_down"], cfg.k, cfg.cf)
@@ -262,7 +298,7 @@ def test_layer_forward_matches_oracle(cfg):
     bias = None if cpu["bias"] is None else cpu["bias"].numpy()
     ref = oracle.moe_forward(bits(cpu["x"]), cpu["w_router"].numpy(), bias, bits(cpu["w_gate"]),
                              bits(cpu["w_up"]), bits(cpu["w_down"]), cfg.k, cfg.cf,
-                             decision_logits=gl)
+                             decision_logits=gl, h_bf16=h_bf16)
     assert_logits_close(gl, ref["logits64"])
     np.testing.assert_array_equal(_ws(ws, "topk_idx", cfg).cpu().numpy(), ref["topk_idx"])
     assert np.max(np.abs(_ws(ws, "topk_w", cfg).cpu().double().numpy() - ref["topk_w"])) \
@@ -331,7 +367,9 @@ FULL = [configs.MIXTRAL, configs.FINE, configs.SKEWED] + \
 def test_full_size_sampled(cfg):
     """Full-size workload in the benchmark's launch configuration: routing,
     capacity and permutation checked for every token; logits, x_perm rows and
-    outputs checked on a seeded sample the oracle computes one by one."""
+    outputs checked on a seeded sample the oracle computes one by one; the
+    down GEMM's rows checked for every expert that received rows (its
+    bucket's last row, in the tail tile, and one more)."""
     torch.cuda.empty_cache()
     w = synth.make_weights(cfg, "cuda")
     x = synth.make_tokens(cfg, "cuda")
@@ -359,6 +397,22 @@ def test_full_size_sampled(cfg):
     xp = _ws(ws, "x_perm", cfg)
     np.testing.assert_array_equal(bits(xp[torch.from_numpy(rows).cuda().long()]),
                                   x_bits[row_src[rows]])
+    # every expert with rows: y_perm (fp32) rows against the oracle's expert,
+    # with h in fp64 (the definition) and rounded to bf16 (the GEMM operand)
+    picks = every_expert_rows(offsets, cfg.seed)
+    assert len(picks) == int((counts > 0).sum())
+
+    def expert_ref(e):
+        wg, wu, wd = (bits(w[n][e]) for n in ("w_gate", "w_up", "w_down"))
+        xr = x_bits[row_src[picks[e]]]
+        return {hb: oracle.swiglu_rows(xr, wg, wu, wd, h_bf16=hb)[1] for hb in H_MODES}
+    refs = map_experts(expert_ref, picks)
+    rows_all = np.concatenate([picks[e] for e in picks])
+    got = f64(_ws(ws, "y_perm", cfg)[torch.from_numpy(rows_all).cuda().long()])
+    for hb in H_MODES:
+        assert_bf16_close(got, np.concatenate([refs[e][hb] for e in picks]),
+                          f"y_perm, {len(picks)} experts, h_bf16={hb}")
+
     # sampled tokens: logits and outputs from the oracle, one token at a time
     n_tok = 4 if cfg.E >= 64 else 8
     toks = np.sort(rng.choice(cfg.T, size=min(n_tok, cfg.T), replace=False))
@@ -367,24 +421,26 @@ def test_full_size_sampled(cfg):
     wr = w["w_router"].cpu().numpy()
     bias = None if w["bias"] is None else w["bias"].cpu().numpy()
     assert_logits_close(gl[toks], oracle.router_logits(x_bits[toks], wr, bias))
-    y_ref = np.zeros((len(toks), cfg.d))
     by_expert = {}
     for i, t in enumerate(toks):
-        kept = [j for j in range(cfg.k) if slot[t, j] >= 0]
-        if not kept:
-            y_ref[i] = oracle.bits_to_f64(x_bits[t])
-        for j in kept:
-            by_expert.setdefault(int(o_idx[t, j]), []).append((i, t, j))
-    for e, users in by_expert.items():
-        wg, wu, wd = (bits(w[n][e]) for n in ("w_gate", "w_up", "w_down"))
-        _, o = oracle.swiglu_rows(x_bits[[t for _, t, _ in users]], wg, wu, wd)
-        for (i, t, j), orow in zip(users, o):
-            y_ref[i] += o_w[t, j] * orow
+        for j in range(cfg.k):
+            if slot[t, j] >= 0:
+                by_expert.setdefault(int(o_idx[t, j]), []).append((i, t, j))
     y_s = y[torch.from_numpy(toks).cuda().long()]
     moe_rows = ~(slot[toks] < 0).all(axis=1)
-    # the expert outputs against the oracle (tolerance from their own rms);
+    for hb in H_MODES:
+        y_ref = np.zeros((len(toks), cfg.d))
+        for i, t in enumerate(toks):
+            if not moe_rows[i]:
+                y_ref[i] = oracle.bits_to_f64(x_bits[t])
+        for e, users in by_expert.items():
+            wg, wu, wd = (bits(w[n][e]) for n in ("w_gate", "w_up", "w_down"))
+            _, o = oracle.swiglu_rows(x_bits[[t for _, t, _ in users]], wg, wu, wd, h_bf16=hb)
+            for (i, t, j), orow in zip(users, o):
+                y_ref[i] += o_w[t, j] * orow
+        # the expert outputs against the oracle (tolerance from their own rms)
+        assert_bf16_close(f64(y_s)[moe_rows], y_ref[moe_rows], f"y (sampled), h_bf16={hb}")
     # all-dropped tokens passed through bit for bit
-    assert_bf16_close(f64(y_s)[moe_rows], y_ref[moe_rows], "y (sampled)")
     np.testing.assert_array_equal(bits(y_s)[~moe_rows], x_bits[toks[~moe_rows]])
     del w, x, y, ws
     torch.cuda.empty_cache()

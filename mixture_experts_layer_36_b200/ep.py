@@ -28,6 +28,14 @@ the same number of tokens T (equal slot sizes).
 The exchange itself is NCCL's all-to-all through torch.distributed; the
 compute steps go through an ``ops`` object (``CudaOps``: the library's C-ABI
 calls), which keeps the exchange logic testable with CPU ranks.
+
+Exchange volume.  The neelmishra page's dispatch volume per rank is
+T*k*d*2*(P-1)/P bytes (bf16 rows, the share of each rank's rows that leaves
+it).  The padded exchange here sends E*C rows per rank instead of T*k, a
+factor E*C/(T*k) (about cf, or E/k when dropless, C = T); and the rows come
+back as fp32 (the expert outputs are rounded to bf16 only once, in the
+combine), twice the bytes of the dispatch.  ``exchange_log`` records, per
+exchange of the last forward, the bytes this rank sent to other ranks.
 """
 import torch
 import torch.distributed as dist
@@ -81,8 +89,17 @@ class ExpertParallelMoE:
         self.w_gate, self.w_up, self.w_down = w_gate, w_up, w_down
         self.k, self.cf = k, cf
         self.ops = ops if ops is not None else CudaOps()
+        self.exchange_log = []
 
-    def _all_to_all(self, out, inp):
+    # bytes per element on the wire: int32 counts, bf16 rows out, fp32 rows back
+    WIRE_BYTES = {"counts": 4, "dispatch": 2, "combine": 4}
+
+    def _all_to_all(self, out, inp, name):
+        # each rank keeps 1/P of its buffer (its own slot) and sends the rest
+        if inp.is_cuda and inp.element_size() != self.WIRE_BYTES[name]:
+            raise TypeError(f"{name}: {inp.dtype} on the wire")
+        nbytes = inp.numel() * self.WIRE_BYTES[name]
+        self.exchange_log.append((name, nbytes * (self.P - 1) // self.P))
         if self.P == 1:
             out.copy_(inp)
         else:
@@ -96,15 +113,16 @@ class ExpertParallelMoE:
         C = self.ops.capacity(T, E, k, cf)
         logits, topk_idx, topk_w = self.ops.route(x, self.w_router, self.bias, k)
         counts, offsets, slot, x_pad = self.ops.permute_padded(x, topk_idx, E, cf)
+        self.exchange_log = []
         # rank q receives counts[q*E_loc : (q+1)*E_loc] from every rank: bucket
         # b = source * E_loc + local expert
-        recv_counts = self._all_to_all(torch.empty_like(counts), counts)
-        x_recv = self._all_to_all(torch.empty_like(x_pad), x_pad)
+        recv_counts = self._all_to_all(torch.empty_like(counts), counts, "counts")
+        x_recv = self._all_to_all(torch.empty_like(x_pad), x_pad, "dispatch")
         B = self.P * self.E_loc
         recv_offsets = torch.arange(B + 1, dtype=torch.int32, device=x.device) * C
         y_recv = self.ops.mlp_buckets(x_recv, recv_offsets, recv_counts, self.w_gate, self.w_up,
                                       self.w_down)
-        y_pad = self._all_to_all(torch.empty_like(y_recv), y_recv)
+        y_pad = self._all_to_all(torch.empty_like(y_recv), y_recv, "combine")
         return self.ops.combine(y_pad, x, topk_idx, topk_w, slot, offsets)
 
     __call__ = forward

@@ -95,6 +95,7 @@ def _worker(rank, world, port, case, out):
                                  ep.shard_experts(w["w_down"], rank, world), k, cf,
                                  ops=OracleOps(oracle))
     y = layer(x).numpy()
+    log = dict(layer.exchange_log)
     xb = OracleOps._bits(x)
     ops = OracleOps(oracle)
     bias = None if w["bias"] is None else w["bias"].numpy()
@@ -105,7 +106,7 @@ def _worker(rank, world, port, case, out):
     dist.barrier()
     dist.destroy_process_group()
     out.put((rank, float(np.max(np.abs(y - ref["y"]))), float(np.max(np.abs(ref["y"]))),
-             int(ref["n_dropped"])))
+             int(ref["n_dropped"]), log, oracle.capacity(T, E, k, cf)))
 
 
 CASES = [
@@ -131,9 +132,18 @@ def test_expert_parallel_matches_single_process(world, case):
         p.join(timeout=30)
         assert p.exitcode == 0
     dropped = 0
-    for rank, err, scale, n_drop in res:
+    T, d, E, k, f, cf, _ = case
+    # dispatch volume per rank on the neelmishra page: T*k*d*2*(P-1)/P bytes
+    page = T * k * d * 2 * (world - 1) / world
+    for rank, err, scale, n_drop, log, C in res:
         assert err <= 1e-12 * max(scale, 1.0), (rank, err)
         dropped += n_drop
+        # the padded exchange moves E*C rows where the formula counts T*k:
+        # the page's volume times E*C / (T*k); the rows come back in fp32
+        assert log["dispatch"] == E * C * d * 2 * (world - 1) // world
+        assert log["dispatch"] == pytest.approx(page * E * C / (T * k))
+        assert log["combine"] == 2 * log["dispatch"]
+        assert log["counts"] == E * 4 * (world - 1) // world
     if case[5] > 0:
         assert dropped > 0                    # the capacity limit was exercised
 

@@ -34,7 +34,7 @@
  *     dropped; builds with MOE_CHECKS also report an expert listed twice for
  *     one token).
  *   - Limits: 1 <= E <= 256, 1 <= k <= min(E, 8), T*k < 2^31, d and f
- *     multiples of 128 (else MOE_ERR_UNSUPPORTED).  T == 0 is a no-op.
+ *     multiples of 64 (else MOE_ERR_UNSUPPORTED).  T == 0 is a no-op.
  */
 #ifndef LIBMOE_MOE_H_
 #define LIBMOE_MOE_H_

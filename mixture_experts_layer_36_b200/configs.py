@@ -47,8 +47,14 @@ FINE_SLICE = MoEConfig("fine_slice", T=512, d=7168, E=16, k=8, f=2048, cf=1.25, 
 # T = 256), about 4 GB of bf16 + e4m3 expert weights on the device.
 DECODE_SLICE = MoEConfig("decode_slice", T=32, d=7168, E=32, k=8, f=2048, cf=0.0, seed=4)
 
+# The fine-grained layer's token side (T, d, k, cf: the same x and permuted
+# rows, 1.06 GB moved by the permutation) with 16 of its experts, so that a
+# capture of the permutation and combine holds a few GB on the device.
+FINE_ROWS_SLICE = MoEConfig("fine_rows_slice", T=8192, d=7168, E=16, k=8, f=2048, cf=1.25,
+                            seed=2)
+
 ALL = {c.name: c for c in (TINY, MIXTRAL, FINE, SKEWED, DECODE, MIXTRAL_SLICE, FINE_SLICE,
-                           DECODE_SLICE)}
+                           DECODE_SLICE, FINE_ROWS_SLICE)}
 
 
 def by_name(name: str) -> MoEConfig:

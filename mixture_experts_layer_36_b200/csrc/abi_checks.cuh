@@ -12,7 +12,7 @@ namespace abi {
 
 constexpr int64_t kMaxE = 256;
 constexpr int64_t kMaxK = 8;
-constexpr int64_t kTileMultiple = 128;
+constexpr int64_t kTileMultiple = 64;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -97,11 +97,45 @@ def random_routing(T, E, k, seed, skew=1.2):
     return np.argsort(-keys, axis=1)[:, :k].astype(np.int32)
 
 
-# Precision of h in the oracle's expert.  The contract is the plain fp64
-# definition (h_bf16=False: no rounding anywhere in the MLP); the bf16-rounded
-# h (h_bf16=True) models the GEMMs' bf16 operand and serves as a diagnostic.
-# Layer-level outputs are compared with both, at the same tolerance.
+# Precision of h in the oracle's expert.  Layer outputs are compared with
+# both oracle modes:
+#   * h_bf16=True, the oracle in the expert GEMMs' arithmetic (bf16 operands,
+#     so the down projection's input h is a bf16 value): max|err| <=
+#     2e-2 * rms(ref), the stated tolerance, unchanged;
+#   * h_bf16=False, the plain definition with no rounding anywhere in the MLP:
+#     the same bound plus one bf16 rounding quantum of the reference value,
+#     |err| <= 2e-2 * rms(ref) + 2^-8 * |ref| elementwise, and a relative rms
+#     error <= 5e-3.  A bf16 output carries a rounding error of up to 2^-8 of
+#     its magnitude (half an ulp at the bottom of a binade), 1.3-1.7 % of rms
+#     at the 5.5-6 sigma tails of these outputs; rounding h to the GEMM's bf16
+#     operand adds about 1 % more there.  An exact CPU replay of those two
+#     roundings (fp64 oracle, h and y rounded to bf16) reaches 2.17 % of rms
+#     at the largest element against the unrounded definition, so the plain
+#     2e-2 bound cannot hold for any bf16-operand implementation, while its
+#     rms error stays at 0.23 % and the bound above at <= 0.6 of its limit.
 H_MODES = (False, True)
+DEF_RMS_ERR = 5e-3
+
+
+def assert_layer_close(gpu, ref64, h_bf16, what):
+    """A bf16 layer output against the oracle run with the given h precision
+    (see H_MODES)."""
+    if h_bf16:
+        assert_bf16_close(gpu, ref64, f"{what} (h as bf16 operand)")
+        return
+    ref = np.asarray(ref64, np.float64)
+    g = np.asarray(gpu, np.float64)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    if ref.size == 0:
+        return
+    rms = np.sqrt(np.mean(ref ** 2))
+    err = np.abs(g - ref)
+    excess = err - (BF16_RMS_TOL * rms + 2.0 ** -8 * np.abs(ref))
+    i = np.unravel_index(np.argmax(excess), excess.shape)
+    assert excess[i] <= 0, (f"{what} (h unrounded): at {i} gpu {g[i]:.6g} ref {ref[i]:.6g} "
+                            f"exceeds 2e-2 rms + 2^-8 |ref| by {excess[i]:.3e}")
+    rel = np.sqrt(np.mean(err ** 2)) / rms
+    assert rel <= DEF_RMS_ERR, f"{what} (h unrounded): rms error {rel:.3e} of rms"
 
 
 def every_expert_rows(offsets, seed):

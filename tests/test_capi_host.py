@@ -109,8 +109,10 @@ def test_validation_codes_without_launch():
     args = [FAKE, FAKE, 100, 128, 8, 2, 1.25, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE]
     assert L.moe_permute(*args, need - 1, None, s) == WORKSPACE
     assert L.moe_permute(*args[:6], -1.0, *args[7:], need, None, s) == INVALID
-    # experts: widths must be multiples of 128
-    assert L.moe_expert_gate_up(FAKE, FAKE, 8, 192, 256, 100, FAKE, FAKE, FAKE, None, s) \
+    # experts: widths must be multiples of 64
+    assert L.moe_expert_gate_up(FAKE, FAKE, 8, 200, 256, 100, FAKE, FAKE, FAKE, None, s) \
+        == UNSUPPORTED
+    assert L.moe_expert_gate_up(FAKE, FAKE, 8, 256, 96, 100, FAKE, FAKE, FAKE, None, s) \
         == UNSUPPORTED
     assert L.moe_expert_down(FAKE, FAKE, 8, 256, 200, 100, FAKE, FAKE, None, s) == UNSUPPORTED
     assert L.moe_expert_mlp(FAKE, FAKE, 8, 256, 256, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None, s) \
@@ -150,7 +152,7 @@ def test_validation_codes_of_the_variants_without_launch():
     assert L.moe_permute_fp8(None, *p8[1:], need, None, s) == INVALID
     assert L.moe_permute_fp8(*p8[:3], 0, *p8[4:], 0, None, s) == OK
     g8 = [F, F, F, 8, 256, 256, 100, F, F, F, F, F, None, s]
-    assert L.moe_expert_gate_up_fp8(*g8[:4], 192, *g8[5:]) == UNSUPPORTED
+    assert L.moe_expert_gate_up_fp8(*g8[:4], 200, *g8[5:]) == UNSUPPORTED
     assert L.moe_expert_gate_up_fp8(*g8[:6], 0, *g8[7:]) == OK
     assert L.moe_expert_gate_up_fp8(None, *g8[1:]) == INVALID
     d8 = [F, F, F, 8, 256, 256, 100, F, F, F, None, s]

@@ -15,8 +15,8 @@ import torch.distributed as dist
 import oracle
 import mixture_experts_layer_36_b200 as moe
 from mixture_experts_layer_36_b200 import ep
-from moe_testlib import (H_MODES, assert_bf16_close, assert_bf16_rounding_close, bits,
-                         cuda_inputs, f64, small)
+from moe_testlib import (H_MODES, assert_bf16_close, assert_bf16_rounding_close,
+                         assert_layer_close, bits, cuda_inputs, f64, small)
 
 pytestmark = pytest.mark.gpu
 
@@ -97,7 +97,7 @@ def test_expert_parallel_one_rank_matches_oracle(cfg, one_rank_group):
         ref = oracle.moe_forward(bits(cpu["x"]), cpu["w_router"].numpy(), bias,
                                  bits(cpu["w_gate"]), bits(cpu["w_up"]), bits(cpu["w_down"]),
                                  cfg.k, cfg.cf, decision_logits=logits.cpu().numpy(), h_bf16=hb)
-        assert_bf16_close(f64(y), ref["y"], f"y, h_bf16={hb}")
+        assert_layer_close(f64(y), ref["y"], hb, "y")
     dropped = (ref["slot"] < 0).all(axis=1)
     if dropped.any():
         np.testing.assert_array_equal(bits(y)[dropped], bits(cpu["x"])[dropped])

@@ -182,6 +182,13 @@ MLP_CASES = [
     (256, 384, [300, 0, 1, 129, 128, 257, 700], True),
     (512, 256, [1, 256, 511, 513, 1024], True),
     (384, 256, [255, 257, 0], True),      # down GEMM: d % 256 != 0 keeps single-CTA tiles
+    # more wide pair tiles than CTA pairs (several tiles per pair, k-blocks
+    # replayed into the second accumulator), and one-accumulator N tails
+    (512, 384, [3000, 2999, 1, 2900], True),
+    (256, 1024, [2048] * 4, True),
+    # d, f multiples of 64 only: 64-wide K tails (half k-blocks) and N tails
+    (192, 320, [300, 0, 1, 129], False),
+    (320, 192, [3000, 1, 2900], True),
 ]
 
 
@@ -233,6 +240,7 @@ SMALL = [
     small("ragged_T", T=333, d=384, E=6, k=3, f=128, cf=0.5, seed=15),
     small("pair_tiles", T=2048, d=256, E=4, k=2, f=256, cf=0.0, seed=19),
     small("pair_tiles_drops", T=3000, d=512, E=4, k=3, f=384, cf=0.8, seed=20),
+    small("width64", T=300, d=192, E=8, k=2, f=320, cf=1.25, seed=23),
 ]
 
 

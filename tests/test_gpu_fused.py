@@ -17,8 +17,8 @@ import oracle
 import mixture_experts_layer_36_b200 as moe
 from mixture_experts_layer_36_b200 import configs, synth
 from moe_testlib import (H_MODES, WEIGHT_ATOL, assert_bf16_close, assert_bf16_rounding_close,
-                         bits, cuda_inputs, every_expert_rows, f64, map_experts, random_routing,
-                         small)
+                         assert_layer_close, bits, cuda_inputs, every_expert_rows, f64,
+                         map_experts, random_routing, small)
 
 pytestmark = pytest.mark.gpu
 
@@ -102,7 +102,7 @@ def test_layer_forward_fused_matches_oracle(cfg):
         ref = oracle.moe_forward(bits(cpu["x"]), cpu["w_router"].numpy(), bias,
                                  bits(cpu["w_gate"]), bits(cpu["w_up"]), bits(cpu["w_down"]),
                                  cfg.k, cfg.cf, decision_logits=gl, h_bf16=hb)
-        assert_bf16_close(f64(y), ref["y"], f"y, h_bf16={hb}")
+        assert_layer_close(f64(y), ref["y"], hb, "y")
     np.testing.assert_array_equal(view("topk_idx").cpu().numpy(), ref["topk_idx"])
     assert np.max(np.abs(view("topk_w").cpu().double().numpy() - ref["topk_w"])) <= WEIGHT_ATOL
     np.testing.assert_array_equal(view("slot").cpu().numpy(), ref["slot"])
@@ -174,7 +174,7 @@ def test_fused_full_size_sampled(cfg):
                 _, o = oracle.swiglu_rows(x_bits[t:t + 1], bits(w["w_gate"][e]),
                                           bits(w["w_up"][e]), bits(w["w_down"][e]), h_bf16=hb)
                 y_ref[i] += o_w[t, j] * o[0]
-        assert_bf16_close(f64(y_s)[moe_rows], y_ref[moe_rows], f"y (sampled), h_bf16={hb}")
+        assert_layer_close(f64(y_s)[moe_rows], y_ref[moe_rows], hb, "y (sampled)")
     np.testing.assert_array_equal(bits(y_s)[~moe_rows], x_bits[toks[~moe_rows]])
     del w, x, y, y2, ws
     torch.cuda.empty_cache()

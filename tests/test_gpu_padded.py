@@ -9,8 +9,8 @@ import torch
 
 import oracle
 import mixture_experts_layer_36_b200 as moe
-from moe_testlib import (H_MODES, WEIGHT_ATOL, assert_bf16_close, bits, cuda_inputs, f64,
-                         random_routing, small)
+from moe_testlib import (H_MODES, WEIGHT_ATOL, assert_layer_close, bits,
+                         cuda_inputs, f64, random_routing, small)
 
 pytestmark = pytest.mark.gpu
 
@@ -66,7 +66,7 @@ def test_layer_padded_matches_oracle(cfg):
         ref = oracle.moe_forward(bits(cpu["x"]), cpu["w_router"].numpy(), bias,
                                  bits(cpu["w_gate"]), bits(cpu["w_up"]), bits(cpu["w_down"]),
                                  cfg.k, cfg.cf, decision_logits=gl, h_bf16=hb)
-        assert_bf16_close(f64(y), ref["y"], f"y, h_bf16={hb}")
+        assert_layer_close(f64(y), ref["y"], hb, "y")
     np.testing.assert_array_equal(idx.cpu().numpy(), ref["topk_idx"])
     assert np.max(np.abs(w.cpu().double().numpy() - ref["topk_w"])) <= WEIGHT_ATOL
     np.testing.assert_array_equal(p["slot"].cpu().numpy(), ref["slot"])

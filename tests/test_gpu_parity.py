@@ -21,8 +21,8 @@ import oracle
 import mixture_experts_layer_36_b200 as moe
 from mixture_experts_layer_36_b200 import configs, synth
 from moe_testlib import (H_MODES, WEIGHT_ATOL, LOGIT_RTOL, assert_bf16_close,
-                         assert_bf16_rounding_close, assert_logits_close, bits, cuda_inputs,
-                         every_expert_rows, f64, map_experts, random_routing, small)
+                         assert_bf16_rounding_close, assert_layer_close, assert_logits_close, bits,
+                         cuda_inputs, every_expert_rows, f64, map_experts, random_routing, small)
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +40,10 @@ SMALL = [
     small("pair_tiles", T=2048, d=256, E=4, k=2, f=256, cf=0.0, seed=19),
     small("pair_tiles_drops", T=3000, d=512, E=4, k=3, f=384, cf=0.8, seed=20),
     small("medium_buckets", T=1024, d=256, E=16, k=4, f=384, cf=1.25, seed=22),
+    # widths that are multiples of 64 but not of 128: ragged 64-column tails
+    # in the router's K, the permuted rows, every GEMM tile shape and the combine
+    small("width64", T=300, d=192, E=8, k=2, f=320, cf=1.25, seed=23),
+    small("width64_wide", T=2048, d=320, E=4, k=2, f=192, cf=0.0, seed=24),
 ]
 IDS = [c.name for c in SMALL]
 
@@ -222,6 +226,18 @@ MLP_CASES = [
     (384, 256, [255, 257, 0], True),      # down GEMM: d % 256 != 0 keeps single-CTA tiles
     (256, 256, [170, 0, 128, 129, 233, 256, 250, 131], False),
     (384, 128, [300, 301, 15, 16], False),
+    # more wide pair tiles (256 rows x 512 accumulator columns) than CTA pairs,
+    # so every pair runs several tiles back to back and the MMA issuer replays
+    # held k-blocks into the second accumulator: K longer than the ring (16
+    # k-blocks), K shorter than it (2), and a last N tile with one accumulator
+    # (f = 384: 256 + 128 h-columns)
+    (1024, 1024, [2048] * 4, True),
+    (512, 128, [6000] * 4, True),
+    (256, 384, [3000, 2999, 1, 2900], True),
+    # d, f multiples of 64 only: 64-column N tails and K = 64 * odd
+    (192, 320, [300, 0, 1, 129, 128, 257], False),
+    (320, 192, [3000, 2999, 1, 2900], True),
+    (64, 64, [70, 0, 129], False),
 ]
 
 
@@ -288,7 +304,7 @@ def _ws(ws, name, cfg):
 def test_layer_forward_matches_oracle(cfg, h_bf16):
     """The whole layer against the oracle: h_fp64 is the plain definition
     (the MLP in fp64 throughout), h_bf16 the oracle with h rounded to bf16
-    like the GEMMs' operand; the same tolerance holds for both."""
+    like the GEMMs' operand (tolerances in moe_testlib.H_MODES)."""
     inp, cpu = cuda_inputs(cfg)
     y, ws = moe.moe_layer_forward(inp["x"], inp["w_router"], inp["bias"], inp["w_gate"],
                                   inp["w_up"], inp["w_down"], cfg.k, cfg.cf)
@@ -310,7 +326,7 @@ def test_layer_forward_matches_oracle(cfg, h_bf16):
     counts = ref["counts"]
     assert counts.max() <= C and counts.sum() == cfg.k * cfg.T - ref["n_dropped"]
     assert _ws(ws, "n_dropped", cfg).item() == ref["n_dropped"]
-    assert_bf16_close(f64(y), ref["y"], "y")
+    assert_layer_close(f64(y), ref["y"], h_bf16, "y")
     dropped = (ref["slot"] < 0).all(axis=1)
     if dropped.any():
         np.testing.assert_array_equal(bits(y)[dropped], bits(cpu["x"])[dropped])
@@ -439,7 +455,7 @@ def test_full_size_sampled(cfg):
             for (i, t, j), orow in zip(users, o):
                 y_ref[i] += o_w[t, j] * orow
         # the expert outputs against the oracle (tolerance from their own rms)
-        assert_bf16_close(f64(y_s)[moe_rows], y_ref[moe_rows], f"y (sampled), h_bf16={hb}")
+        assert_layer_close(f64(y_s)[moe_rows], y_ref[moe_rows], hb, "y (sampled)")
     # all-dropped tokens passed through bit for bit
     np.testing.assert_array_equal(bits(y_s)[~moe_rows], x_bits[toks[~moe_rows]])
     del w, x, y, ws

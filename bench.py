@@ -36,21 +36,23 @@ PAIR_MIN_ROWS = 512      # buffer rows per expert from which the GEMMs use CTA-p
 ROOFLINE_TIMING = ("mean launch duration over the timed steps: CUDA events recorded around "
                    "the launch on its stream")
 FP8_OVER_BF16 = 2.0      # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
+PERMUTE_DIRECT_SUM = 4096   # chunk-histogram counters the scatter sums without a scan kernel
 
 
 def launches_per_step(cfg, sms, fp8=False, padded=False, fused=False):
     """libmoe kernels one layer step launches: router weight split, router
     GEMM and top-k (the top-k runs in the GEMM's epilogue when the router's K
     is not split, i.e. when there are more 128-token row tiles than half the
-    SMs); permutation rank, scan and scatter (+ the padded layout's fill);
-    the FP8 row quantizers on x and on h; the two expert GEMMs; the combine
-    (the fused path's finalize)."""
+    SMs); permutation rank and scatter, with a scan between them when there
+    are more than PERMUTE_DIRECT_SUM chunk-histogram counters (chunks of 256
+    tokens x E) (+ the padded layout's fill); the FP8 row quantizers on x and
+    on h; the two expert GEMMs; the combine (the fused path's finalize)."""
     if cfg.T == 0:
         return 0
     m_tiles = -(-cfg.T // ROUTER_TILE_M)
     splits = max(1, min(min(sms, 256) // m_tiles, cfg.d // 64))
     n = 2 if splits == 1 else 3
-    n += 4 if padded else 3
+    n += 2 + (1 if -(-cfg.T // 256) * cfg.E > PERMUTE_DIRECT_SUM else 0) + (1 if padded else 0)
     n += 2 if fp8 else 0
     return n + 2 + 1
 

@@ -411,6 +411,25 @@ int moe_layer_forward(const void* x, const float* w_router, const float* bias, c
                       int64_t k, int64_t f, double cf, void* y, void* ws, size_t ws_bytes,
                       void* stream);
 
+/* moe_layer_forward with the routing results written where the caller wants
+ * them: each non-null output pointer (device memory the caller owns) takes
+ * the place of the workspace field of the same name, so the stages write it
+ * there directly and no copy is made; a null pointer leaves that result in
+ * the workspace as moe_layer_forward does.
+ *   logits_out   f32 [T,E]   router logits (MOE_WS_LOGITS)
+ *   topk_idx_out i32 [T,k]   selected experts (MOE_WS_TOPK_IDX)
+ *   topk_w_out   f32 [T,k]   gate weights (MOE_WS_TOPK_W)
+ *   slot_out     i32 [T,k]   bucket slots, -1 = dropped (MOE_WS_SLOT)
+ *   counts_out   i32 [E]     pairs kept per expert (MOE_WS_COUNTS)
+ * ws is still required (>= moe_workspace_size bytes; the replaced fields are
+ * left unused).  Same sources, shapes and errors as moe_layer_forward. */
+int moe_layer_forward_ex(const void* x, const float* w_router, const float* bias,
+                         const void* w_gate, const void* w_up, const void* w_down, int64_t T,
+                         int64_t d, int64_t E, int64_t k, int64_t f, double cf, void* y,
+                         float* logits_out, int32_t* topk_idx_out, float* topk_w_out,
+                         int32_t* slot_out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                         void* stream);
+
 #ifdef __cplusplus
 }
 #endif

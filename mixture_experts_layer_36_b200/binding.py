@@ -35,7 +35,7 @@ EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "mo
             "moe_workspace_size_fp8", "moe_layer_forward_fp8", "moe_padded_rows",
             "moe_permute_padded", "moe_permute_fused", "moe_expert_gate_up_gather",
             "moe_expert_down_scatter", "moe_combine_finalize", "moe_workspace_size_fused",
-            "moe_layer_forward_fused", "moe_expert_mlp_buckets"]
+            "moe_layer_forward_fused", "moe_expert_mlp_buckets", "moe_layer_forward_ex"]
 
 
 class MoEError(RuntimeError):
@@ -71,6 +71,8 @@ def _load():
         "moe_combine": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, p, p]),
         "moe_layer_forward": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl, p, p,
                                              sz, p]),
+        "moe_layer_forward_ex": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl, p,
+                                                p, p, p, p, p, p, sz, p]),
         "moe_quantize_weights_fp8": (ctypes.c_int, [p, i64, i64, i64, p, p, p]),
         "moe_quantize_rows_fp8": (ctypes.c_int, [p, i64, i64, p, p, p, p]),
         "moe_permute_fp8": (ctypes.c_int, [p, p, p, i64, i64, i64, i64, dbl, p, p, p, p, p, p, p,
@@ -343,6 +345,41 @@ def moe_layer_forward(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws
     _check("moe_layer_forward", _lib.moe_layer_forward(
         _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k,
         f, float(cf), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+    return y, ws
+
+
+def moe_layer_forward_ex(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, logits=None,
+                         topk_idx=None, topk_w=None, slot=None, counts=None, ws=None,
+                         stream=None):
+    """moe_layer_forward with optional caller tensors for the routing results
+    (each one given is written in place of its workspace field).  Returns
+    (y, ws)."""
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    _want(x, "x", torch.bfloat16)
+    _want(w_router, "w_router", torch.float32, (d, E))
+    if bias is not None:
+        _want(bias, "bias", torch.float32, (E,))
+    _want(w_gate, "w_gate", torch.bfloat16, (E, d, f))
+    _want(w_up, "w_up", torch.bfloat16, (E, d, f))
+    _want(w_down, "w_down", torch.bfloat16, (E, f, d))
+    for t, name, dt, shape in ((logits, "logits", torch.float32, (T, E)),
+                               (topk_idx, "topk_idx", torch.int32, (T, k)),
+                               (topk_w, "topk_w", torch.float32, (T, k)),
+                               (slot, "slot", torch.int32, (T, k)),
+                               (counts, "counts", torch.int32, (E,))):
+        if t is not None:
+            _want(t, name, dt, shape)
+    nbytes = moe_workspace_size(T, d, E, k, f, cf)
+    if ws is None:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _want(ws, "ws", torch.uint8)
+    y = torch.empty_like(x) if y is None else y
+    _want(y, "y", torch.bfloat16, (T, d))
+    _check("moe_layer_forward_ex", _lib.moe_layer_forward_ex(
+        _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k,
+        f, float(cf), _ptr(y), _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(slot),
+        _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)))
     return y, ws
 
 

@@ -705,6 +705,16 @@ int moe_layer_forward(const void* x, const float* w_router, const float* bias, c
                       const void* w_up, const void* w_down, int64_t T, int64_t d, int64_t E,
                       int64_t k, int64_t f, double cf, void* y, void* ws, size_t ws_bytes,
                       void* stream) {
+  return moe_layer_forward_ex(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, cf, y,
+                              nullptr, nullptr, nullptr, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+int moe_layer_forward_ex(const void* x, const float* w_router, const float* bias,
+                         const void* w_gate, const void* w_up, const void* w_down, int64_t T,
+                         int64_t d, int64_t E, int64_t k, int64_t f, double cf, void* y,
+                         float* logits_out, int32_t* topk_idx_out, float* topk_w_out,
+                         int32_t* slot_out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                         void* stream) {
   int st = check_routing_shape(T, E, k);
   if (st != MOE_OK) return st;
   if ((st = check_width(d)) != MOE_OK) return st;
@@ -719,12 +729,16 @@ int moe_layer_forward(const void* x, const float* w_router, const float* bias, c
   auto field = [&](int id) {
     return base + moe_workspace_field_offset(id, T, d, E, k, f, cf);
   };
+  // a caller's output pointer replaces the workspace field it names
+  auto pick = [](auto* out, char* fld) {
+    return out ? out : reinterpret_cast<decltype(out)>(fld);
+  };
   int32_t* status = reinterpret_cast<int32_t*>(field(MOE_WS_STATUS));
-  float* logits = reinterpret_cast<float*>(field(MOE_WS_LOGITS));
-  int32_t* topk_idx = reinterpret_cast<int32_t*>(field(MOE_WS_TOPK_IDX));
-  float* topk_w = reinterpret_cast<float*>(field(MOE_WS_TOPK_W));
-  int32_t* slot = reinterpret_cast<int32_t*>(field(MOE_WS_SLOT));
-  int32_t* counts = reinterpret_cast<int32_t*>(field(MOE_WS_COUNTS));
+  float* logits = pick(logits_out, field(MOE_WS_LOGITS));
+  int32_t* topk_idx = pick(topk_idx_out, field(MOE_WS_TOPK_IDX));
+  float* topk_w = pick(topk_w_out, field(MOE_WS_TOPK_W));
+  int32_t* slot = pick(slot_out, field(MOE_WS_SLOT));
+  int32_t* counts = pick(counts_out, field(MOE_WS_COUNTS));
   int32_t* offsets = reinterpret_cast<int32_t*>(field(MOE_WS_OFFSETS));
   int32_t* n_dropped = reinterpret_cast<int32_t*>(field(MOE_WS_N_DROPPED));
   int32_t* row_src = reinterpret_cast<int32_t*>(field(MOE_WS_ROW_SRC));

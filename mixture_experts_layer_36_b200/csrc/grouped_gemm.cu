@@ -1760,13 +1760,18 @@ static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtens
 // per expert bound the average bucket from above.
 static bool use_pair_tiles(int E, int max_rows) { return max_rows >= 512LL * E; }
 
-// The wide pair tiles (256 rows x 512 accumulator columns) from this many
-// buffer rows per expert on.
-#ifndef MOE_WIDE_MIN_ROWS
-#define MOE_WIDE_MIN_ROWS 256
-#endif
-static bool use_wide_tiles(int E, int max_rows, bool gather) {
-  return !gather && max_rows >= (long long)MOE_WIDE_MIN_ROWS * E;
+// The wide pair tiles (256 rows x 512 accumulator columns).  Their main loop
+// moves a quarter fewer operand bytes per FLOP than the 256 x 256 pair tiles,
+// but with both accumulators in TMEM the epilogue is only partly hidden, so
+// they pay off for long contractions, and for buckets of 256-511 rows, where
+// the alternative is the single-CTA tile.  Measured on B200 (GEMM 1, buckets
+// of 9472 rows): at K = 8192 1555 vs 1394 TFLOP/s, at K = 2048 equal, at
+// K = 1024 7 % slower; the fp32 epilogue of GEMM 2 moves the break-even to
+// K = 8192, and on the Mixtral-shaped layer (K = 4096 / 14336) they tie.
+static bool use_wide_tiles(int E, int max_rows, int K, bool swiglu, bool gather) {
+  if (gather || max_rows < 256LL * E) return false;
+  if (max_rows < 512LL * E) return swiglu && K >= 4096;
+  return K >= 8192;
 }
 
 // The A operand: the permuted rows [max_rows, K] (128- and 64-row boxes), or,
@@ -1795,7 +1800,7 @@ cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, 
                   map_weights(&tg, w_gate, weight_count(fz, E), d, f) &&
                   map_weights(&tu, w_up, weight_count(fz, E), d, f));
   if (*map_failed) return cudaSuccess;
-  if (use_wide_tiles(E, max_rows, fz.row_src != nullptr))
+  if (use_wide_tiles(E, max_rows, d, true, fz.row_src != nullptr))
     return launch_gemm_wide<true>(14, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s,
                                   fz);
   if (use_pair_tiles(E, max_rows))
@@ -1813,7 +1818,7 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
   *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_rows(&ta64, h, f, max_rows, kBM / 2) &&
                   map_weights(&td, w_down, weight_count(fz, E), f, d));
   if (*map_failed) return cudaSuccess;
-  if (d % 256 == 0 && use_wide_tiles(E, max_rows, false))
+  if (d % 256 == 0 && use_wide_tiles(E, max_rows, f, false, false))
     return launch_gemm_wide<false>(15, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,
                                    status, s, fz);
   if (d % 256 == 0 && use_pair_tiles(E, max_rows))
@@ -1867,12 +1872,13 @@ cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_
                   map_weights_e4m3(&tg, wq_gate, weight_count(fz, E), f, d) &&
                   map_weights_e4m3(&tu, wq_up, weight_count(fz, E), f, d));
   if (*map_failed) return cudaSuccess;
-  if (use_wide_tiles(E, max_rows, fz.row_src != nullptr) || use_pair_tiles(E, max_rows)) {
+  const bool wide = use_wide_tiles(E, max_rows, d, true, fz.row_src != nullptr);
+  if (wide || use_pair_tiles(E, max_rows)) {
     CUtensorMap tgh, tuh;
     *map_failed = !(map_weights_e4m3(&tgh, wq_gate, weight_count(fz, E), f, d, 64) &&
                     map_weights_e4m3(&tuh, wq_up, weight_count(fz, E), f, d, 64));
     if (*map_failed) return cudaSuccess;
-    if (use_wide_tiles(E, max_rows, fz.row_src != nullptr))
+    if (wide)
       return launch_gemm_wide<true, true>(17, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h,
                                           status, s, fz, &tgh, &tuh, sx, s_gate, s_up);
     return launch_gemm_pair<true, true>(9, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h,
@@ -1891,7 +1897,7 @@ cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int3
                   map_rows_e4m3(&ta64, hq, f, max_rows, kBM / 2) &&
                   map_weights_e4m3(&td, wq_down, weight_count(fz, E), d, f));
   if (*map_failed) return cudaSuccess;
-  if (d % 256 == 0 && use_wide_tiles(E, max_rows, false))
+  if (d % 256 == 0 && use_wide_tiles(E, max_rows, f, false, false))
     return launch_gemm_wide<false, true>(18, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,
                                          status, s, fz, &td, &td, sh_rows, s_down, nullptr);
   if (d % 256 == 0 && use_pair_tiles(E, max_rows))

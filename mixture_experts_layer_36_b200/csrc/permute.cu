@@ -15,6 +15,9 @@
 //   2. scan:    per expert, the exclusive prefix of the histograms over the
 //               chunks (each chunk's base, written over its histogram) and
 //               the total demand (one extra row) — one pass, linear in T;
+//               skipped when there are at most kDirectSum histogram counters:
+//               each scatter CTA then sums them itself, which costs less than
+//               one more launch in the chain;
 //   3. scatter: per CTA of 8 tokens, kept = min(demand, C), offsets
 //               (exclusive scan over experts) and slot = chunk base + rank;
 //               kept pairs copy their token row into x_perm[offsets[e] + slot]
@@ -36,6 +39,7 @@ constexpr int kTokPerWarp = kChunk / kRankWarps;
 constexpr int kScanThreads = 1024;     // 32 warps; lane = one expert of a group of 32
 constexpr int kScatThreads = 256;      // 8 warps
 constexpr int kScatTokens = 8;         // tokens per scatter CTA (one per warp; divides kChunk)
+constexpr int kDirectSum = 4096;       // histogram counters a scatter CTA sums without the scan
 
 // 1. rank: per chunk, the rank of each pair among the chunk's pairs of the
 //    same expert (token order), and the chunk's per-expert histogram.
@@ -143,8 +147,8 @@ __global__ void __launch_bounds__(kScatThreads)
     permute_scatter_kernel(const uint8_t* __restrict__ x, int row_bytes,
                            const float* __restrict__ x_scale,
                            const int32_t* __restrict__ topk_idx, int32_t* __restrict__ slot,
-                           const int32_t* __restrict__ chunk_base, int nchunks, int T,
-                           int E, int k, int64_t C,
+                           const int32_t* __restrict__ chunk_base, bool scanned,
+                           int nchunks, int T, int E, int k, int64_t C,
                            int32_t* __restrict__ counts,
                            int32_t* __restrict__ offsets, int32_t* __restrict__ n_dropped,
                            int32_t* __restrict__ row_src, uint8_t* __restrict__ x_perm,
@@ -167,11 +171,22 @@ __global__ void __launch_bounds__(kScatThreads)
   grid_dep_launch();
   grid_dep_wait();          // ranks in slot, chunk bases and totals
 
-  // ---- per-expert totals, kept, chunk base (thread e owns expert e)
+  // ---- per-expert totals, kept, chunk base (thread e owns expert e): from
+  //      the scan's rows, or summed here over the (few) chunk histograms
   int kept = 0, drop = 0;
   if (tid < E) {
-    const int total = chunk_base[(size_t)nchunks * E + tid];
-    s_base[tid] = chunk_base[(size_t)my_chunk * E + tid];
+    int total = 0, base = 0;
+    if (scanned) {
+      total = chunk_base[(size_t)nchunks * E + tid];
+      base = chunk_base[(size_t)my_chunk * E + tid];
+    } else {
+      for (int c = 0; c < nchunks; ++c) {
+        const int v = chunk_base[(size_t)c * E + tid];
+        if (c < my_chunk) base += v;
+        total += v;
+      }
+    }
+    s_base[tid] = base;
     kept = (int64_t)total < C ? total : (int)C;
     drop = total - kept;
   }
@@ -287,12 +302,16 @@ __global__ void __launch_bounds__(256)
 // per row, moved with it) may be null; x null: no row copy (index-only), with
 // row_pair (t*k + j of each kept row) and zeroed fp32 rows zero_rows[T,
 // zero_cols] for the fused combine when those are non-null.
+// The rank kernel, and the scan kernel when the histograms are many;
+// *scanned tells the scatter which it gets.
 static cudaError_t launch_rank_scan(const int32_t* topk_idx, int T, int E, int k, int32_t* slot,
-                                    int32_t* chunk_hist, cudaStream_t s, int32_t* status) {
+                                    int32_t* chunk_hist, cudaStream_t s, int32_t* status,
+                                    bool* scanned) {
   const int nchunks = (T + kChunk - 1) / kChunk;
   cudaError_t err = launch_dependent(permute_rank_kernel, dim3(nchunks), dim3(kRankThreads), 0, s,
                                      topk_idx, T, E, k, slot, chunk_hist, status);
-  if (err != cudaSuccess) return err;
+  *scanned = (int64_t)nchunks * E > kDirectSum;
+  if (err != cudaSuccess || !*scanned) return err;
   return launch_dependent(permute_scan_kernel, dim3((E + 31) / 32), dim3(kScanThreads), 0, s,
                           chunk_hist, nchunks, E);
 }
@@ -305,12 +324,13 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
                                 int32_t* row_pair, float* zero_rows, int zero_cols,
                                 int32_t* status) {
   const int nchunks = (T + kChunk - 1) / kChunk;
-  cudaError_t err = launch_rank_scan(topk_idx, T, E, k, slot, chunk_hist, s, status);
+  bool scanned = false;
+  cudaError_t err = launch_rank_scan(topk_idx, T, E, k, slot, chunk_hist, s, status, &scanned);
   if (err != cudaSuccess) return err;
   return launch_dependent(permute_scatter_kernel, dim3((T + kScatTokens - 1) / kScatTokens),
                           dim3(kScatThreads), 0, s, x, row_bytes, x_scale, topk_idx, slot,
-                          chunk_hist, nchunks, T, E, k, C, counts, offsets, n_dropped, row_src,
-                          x_perm, perm_scale, false, row_pair, zero_rows, zero_cols);
+                          chunk_hist, scanned, nchunks, T, E, k, C, counts, offsets, n_dropped,
+                          row_src, x_perm, perm_scale, false, row_pair, zero_rows, zero_cols);
 }
 
 // The padded [E, C, d] layout: bucket e holds rows e*C .. e*C + C - 1, its
@@ -321,13 +341,15 @@ cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_id
                                   int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
                                   int32_t* status) {
   const int nchunks = (T + kChunk - 1) / kChunk;
-  cudaError_t err = launch_rank_scan(topk_idx, T, E, k, slot, chunk_hist, s, status);
+  bool scanned = false;
+  cudaError_t err = launch_rank_scan(topk_idx, T, E, k, slot, chunk_hist, s, status, &scanned);
   if (err != cudaSuccess) return err;
   uint8_t* xp = reinterpret_cast<uint8_t*>(x_pad);
   err = launch_dependent(permute_scatter_kernel, dim3((T + kScatTokens - 1) / kScatTokens),
                          dim3(kScatThreads), 0, s, reinterpret_cast<const uint8_t*>(x), d * 2,
-                         nullptr, topk_idx, slot, chunk_hist, nchunks, T, E, k, C, counts,
-                         offsets, n_dropped, row_src, xp, nullptr, true, nullptr, nullptr, 0);
+                         nullptr, topk_idx, slot, chunk_hist, scanned, nchunks, T, E, k, C,
+                         counts, offsets, n_dropped, row_src, xp, nullptr, true, nullptr, nullptr,
+                         0);
   if (err != cudaSuccess) return err;
   const int64_t rows = (int64_t)E * C;
   return launch_dependent(permute_pad_fill_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0,

@@ -129,6 +129,13 @@ def test_validation_codes_without_launch():
                                FAKE, ws_need, s) == UNSUPPORTED
     assert L.moe_layer_forward(FAKE, FAKE, None, FAKE, FAKE, FAKE, 0, 128, 8, 2, 256, 1.25, FAKE,
                                FAKE, 0, s) == OK
+    outs = [None] * 5
+    assert L.moe_layer_forward_ex(FAKE, FAKE, None, FAKE, FAKE, FAKE, 64, 128, 8, 2, 250, 1.25,
+                                  FAKE, *outs, FAKE, ws_need, s) == UNSUPPORTED
+    assert L.moe_layer_forward_ex(FAKE, FAKE, None, FAKE, FAKE, FAKE, 64, 128, 8, 2, 256, 1.25,
+                                  FAKE, *outs, FAKE, ws_need - 1, s) == WORKSPACE
+    assert L.moe_layer_forward_ex(FAKE, FAKE, None, FAKE, FAKE, FAKE, 0, 128, 8, 2, 256, 1.25,
+                                  FAKE, *outs, FAKE, 0, s) == OK
 
 
 def test_validation_codes_of_the_variants_without_launch():

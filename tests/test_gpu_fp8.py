@@ -182,10 +182,12 @@ MLP_CASES = [
     (256, 384, [300, 0, 1, 129, 128, 257, 700], True),
     (512, 256, [1, 256, 511, 513, 1024], True),
     (384, 256, [255, 257, 0], True),      # down GEMM: d % 256 != 0 keeps single-CTA tiles
-    # more wide pair tiles than CTA pairs (several tiles per pair, k-blocks
-    # replayed into the second accumulator), and one-accumulator N tails
+    # several CTA-pair tiles per pair; the wide pair tiles on GEMM 1 with
+    # 256-511 buffer rows per expert and K >= 4096, and on GEMM 2 with K >= 8192
     (512, 384, [3000, 2999, 1, 2900], True),
     (256, 1024, [2048] * 4, True),
+    (4096, 384, [300, 260, 255, 511, 0, 1], "mid"),
+    (768, 8192, [600, 1, 300], True),
     # d, f multiples of 64 only: 64-wide K tails (half k-blocks) and N tails
     (192, 320, [300, 0, 1, 129], False),
     (320, 192, [3000, 1, 2900], True),
@@ -203,7 +205,10 @@ def test_expert_mlp_fp8_matches_oracle(d, f, sizes, pair):
     qg, sg = quantize_w(edge_weights(E, d, f, d + 1, d ** -0.5))
     qu, su = quantize_w(edge_weights(E, d, f, d + 2, d ** -0.5))
     qd, sd = quantize_w(edge_weights(E, f, d, d + 3, f ** -0.5))
-    max_rows = max(N + 37, 512 * E + 5) if pair else N + 37
+    if pair == "mid":
+        max_rows = max(N + 37, 256 * E + 5)
+    else:
+        max_rows = max(N + 37, 512 * E + 5) if pair else N + 37
     out = run_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, max_rows, d, f)
     check_mlp(xq, sx, offsets, qg, sg, qu, su, qd, sd, *out)
 

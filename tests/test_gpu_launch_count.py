@@ -13,6 +13,9 @@ pytestmark = pytest.mark.gpu
 
 # more 128-token row tiles than SMs: the router runs without a K split
 UNSPLIT = MoEConfig("unsplit", T=148 * 128 + 37, d=128, E=16, k=2, f=256, cf=1.25, seed=9)
+# more than 4096 chunk-histogram counters (17 chunks x 256 experts): the
+# permutation runs its scan kernel
+SCANNED = MoEConfig("scanned", T=4352, d=128, E=256, k=8, f=128, cf=1.25, seed=10)
 MODES = {"bf16": {}, "fp8": {"fp8": True}, "fused": {"fused": True}, "padded": {"padded": True}}
 
 
@@ -28,7 +31,8 @@ def _libmoe_kernels(fn):
 
 
 @pytest.mark.parametrize("mode", list(MODES))
-@pytest.mark.parametrize("cfg", [configs.TINY, UNSPLIT], ids=["tiny", "unsplit"])
+@pytest.mark.parametrize("cfg", [configs.TINY, UNSPLIT, SCANNED],
+                         ids=["tiny", "unsplit", "scanned"])
 def test_launch_count_matches_profiler(cfg, mode):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -41,7 +45,8 @@ def test_launch_count_matches_profiler(cfg, mode):
     want = bench.launches_per_step(cfg, sms, fp8=mode == "fp8", padded=mode == "padded",
                                    fused=mode == "fused")
     assert len(names) == want, names
-    assert any("router_topk_kernel" in n for n in names) == (cfg is configs.TINY)
+    assert any("router_topk_kernel" in n for n in names) == (cfg is not UNSPLIT)
+    assert any("permute_scan_kernel" in n for n in names) == (cfg is SCANNED)
     one_shot = _libmoe_kernels(lambda: layer.layer_forward(layer.x, layer.y))
     assert sorted(one_shot) == sorted(names)
     assert int(layer.status.item()) == 0

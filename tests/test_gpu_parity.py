@@ -181,7 +181,7 @@ def test_route_split_k_ties_across_lanes(d):
 
 PERM_CASES = [(64, 128, 8, 2, 1.25), (1000, 256, 64, 6, 1.0), (777, 128, 256, 8, 1.25),
               (513, 128, 8, 2, 0.0), (300, 128, 5, 5, 0.3), (257, 384, 3, 1, 0.5),
-              (4096, 256, 256, 8, 0.2), (65536, 128, 256, 8, 1.0)]
+              (4096, 256, 256, 8, 0.2), (4352, 128, 256, 8, 1.25), (65536, 128, 256, 8, 1.0)]
 
 
 @pytest.mark.parametrize("T,d,E,k,cf", PERM_CASES)
@@ -226,14 +226,20 @@ MLP_CASES = [
     (384, 256, [255, 257, 0], True),      # down GEMM: d % 256 != 0 keeps single-CTA tiles
     (256, 256, [170, 0, 128, 129, 233, 256, 250, 131], False),
     (384, 128, [300, 301, 15, 16], False),
-    # more wide pair tiles (256 rows x 512 accumulator columns) than CTA pairs,
-    # so every pair runs several tiles back to back and the MMA issuer replays
-    # held k-blocks into the second accumulator: K longer than the ring (16
-    # k-blocks), K shorter than it (2), and a last N tile with one accumulator
-    # (f = 384: 256 + 128 h-columns)
+    # more CTA-pair tiles than pairs (several tiles per pair), K longer than
+    # the ring (16 k-blocks) and shorter (2), a last N tile of 128 h-columns
     (1024, 1024, [2048] * 4, True),
     (512, 128, [6000] * 4, True),
     (256, 384, [3000, 2999, 1, 2900], True),
+    # the wide pair tiles (256 rows x 512 accumulator columns, both TMEM
+    # accumulators, k-blocks replayed into the second): GEMM 1 on buckets of
+    # 256-511 rows with K = d >= 4096 ("mid": 256-511 buffer rows per expert),
+    # GEMM 1 and 2 with K >= 8192 on large buckets, with more tiles than CTA
+    # pairs (E = 2 x 2560 rows, f = 1024: 80 wide tiles), and one-accumulator
+    # N tails (f = 384: 256 + 128 h-columns; d = 768: 512 + 256 columns)
+    (4096, 384, [300, 260, 255, 511, 0, 1], "mid"),
+    (8192, 1024, [2560, 2560], True),
+    (768, 8192, [600, 1, 300], True),
     # d, f multiples of 64 only: 64-column N tails and K = 64 * odd
     (192, 320, [300, 0, 1, 129, 128, 257], False),
     (320, 192, [3000, 2999, 1, 2900], True),
@@ -241,12 +247,23 @@ MLP_CASES = [
 ]
 
 
+def mlp_buffer_rows(N, E, pair):
+    """Rows of the permuted buffer for a bucket layout: pair=True gives >= 512
+    per expert (CTA-pair tiles), "mid" 256-511 (wide tiles for GEMM 1 on long
+    K, else single-CTA), False fewer (single-CTA tiles)."""
+    if pair == "mid":
+        rows = max(N + 37, 256 * E + 5)
+        assert rows < 512 * E
+        return rows
+    return max(N + 37, 512 * E + 5) if pair else N + 37
+
+
 @pytest.mark.parametrize("d,f,sizes,pair", MLP_CASES)
 def test_expert_mlp_matches_oracle(d, f, sizes, pair):
     E = len(sizes)
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     N = int(offsets[-1])
-    max_rows = max(N + 37, 512 * E + 5) if pair else N + 37
+    max_rows = mlp_buffer_rows(N, E, pair)
     g = torch.Generator().manual_seed(d + f + E)
     x_perm = torch.randn(max_rows, d, generator=g).to(torch.bfloat16)
     wg = (torch.randn(E, d, f, generator=g) / d ** 0.5).to(torch.bfloat16)
@@ -345,6 +362,27 @@ def test_stages_equal_one_shot(cfg):
     y2 = moe.moe_combine(y_perm, inp["x"], idx, w, p["slot"], p["offsets"])
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("cfg", [configs.TINY, SMALL[3]], ids=["tiny", "skewed_small"])
+def test_layer_forward_ex_writes_routing_outputs(cfg):
+    """moe_layer_forward_ex: the caller's routing tensors receive exactly what
+    moe_layer_forward leaves in its workspace, and y is bit-identical."""
+    inp, _ = cuda_inputs(cfg)
+    args = (inp["x"], inp["w_router"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"],
+            cfg.k, cfg.cf)
+    y1, ws = moe.moe_layer_forward(*args)
+    T, E, k = cfg.T, cfg.E, cfg.k
+    fill = lambda *shape, dt: torch.full(shape, -5, dtype=dt, device="cuda")  # noqa: E731
+    outs = {"logits": fill(T, E, dt=torch.float32), "topk_idx": fill(T, k, dt=torch.int32),
+            "topk_w": fill(T, k, dt=torch.float32), "slot": fill(T, k, dt=torch.int32),
+            "counts": fill(E, dt=torch.int32)}
+    y2, ws2 = moe.moe_layer_forward_ex(*args, **outs)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    for name, t in outs.items():
+        assert torch.equal(t, _ws(ws, name, cfg)), name
+    assert _ws(ws2, "status", cfg).item() == 0
 
 
 def test_hot_expert_many_row_tiles():

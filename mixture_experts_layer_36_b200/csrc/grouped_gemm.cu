@@ -1130,423 +1130,6 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
   }
 }
 
-// ---------------------------------------------------------------- wide CTA-pair variant
-// A CTA pair computes M = 256 rows (128 per CTA; 64 in a bucket's last tile
-// of <= 128 rows, the M = 128 pair form) by N = 512 accumulator columns, held
-// as two N = 256 accumulators per CTA (acc0 at TMEM column 0, acc1 at 256:
-// all 512 columns).  Per 64-deep k-block each CTA stages 48 KB (A 16 KB +
-// 256 B columns) for two MMAs, i.e. 48 bytes per MMA-clock instead of the
-// 256 x 256 pair tile's 64: a quarter fewer operand bytes per FLOP, the
-// quantity the operand stream from L2 into shared memory limits.
-//
-// GEMM 1: acc a holds h-columns [256 n + 128 a, +128) as gate | up (CTA 0
-// stages the gate columns, CTA 1 the up columns, both 256 per k-block); a
-// tile whose N range is only 128 h-columns wide (f % 256 = 128) uses acc0
-// alone.  GEMM 2: acc a holds output columns [512 n + 256 a, +256), CTA r
-// staging [.. + 128 r, +128) of each; d % 512 = 256 gives a last acc0-only
-// tile.
-//
-// With all of TMEM in use the accumulators are not double-buffered.  The
-// epilogue of tile i drains acc0, releases it, then drains acc1; the MMA
-// issuer starts tile i+1 on acc0 as soon as acc0 is free and keeps the stages
-// it has consumed (no "stage free" commit) until acc1 is free too, then
-// replays those k-blocks into acc1 and continues with both accumulators.  It
-// holds at most all ring stages; when the ring is full (or the tile ends) it
-// waits for acc1.  So the epilogue's first half overlaps the tail of tile i
-// (acc1's last MMAs) and its second half the start of tile i+1.
-constexpr int kWideStages = 4;
-constexpr int kWideABytes = kBM * kBK * 2;                   // 16 KB (e4m3: 128 rows x 128 B)
-constexpr int kWideAccBBytes = 2 * kChunkBytes;              // 16 KB of B per accumulator
-constexpr int kWideStageBytes = kWideABytes + 2 * kWideAccBBytes;   // 48 KB
-__host__ __device__ constexpr int wide_staging_off() { return kWideStages * kWideStageBytes; }
-__host__ __device__ constexpr int wide_smem_bytes(bool swiglu) {
-  return wide_staging_off() + (swiglu ? 0 : kEpiWarps * stage_words(16) * 4) + 1024;
-}
-// output columns one wide tile covers
-__host__ __device__ constexpr int wide_out_cols(bool swiglu) { return swiglu ? 256 : 512; }
-
-template <bool SWIGLU, bool E4M3, int FUSE>
-__global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
-    grouped_gemm_wide_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ CUtensorMap tmA64,   // 64-row boxes
-                             const __grid_constant__ CUtensorMap tmB0,
-                             const __grid_constant__ CUtensorMap tmB1,
-                             const __grid_constant__ CUtensorMap tmB0h,
-                             const __grid_constant__ CUtensorMap tmB1h,
-                             const float* __restrict__ row_scale,
-                             const float* __restrict__ col_scale0,
-                             const float* __restrict__ col_scale1,
-                             const int32_t* __restrict__ offsets, int E, int K, int n_out,
-                             int max_rows, void* __restrict__ out_raw, int32_t* status,
-                             const FuseArgs fz) {
-  constexpr int kOutCols = wide_out_cols(SWIGLU);
-  constexpr int kPairM = 2 * kBM;
-  constexpr int kKb = E4M3 ? 128 : kBK;               // K values per k-block (128 bytes)
-  constexpr uint32_t kIdesc = E4M3 ? idesc_e4m3_f32(kPairM, 256)
-                                   : idesc_bf16_f32(kPairM, 256, /*b_mn_major=*/true);
-  constexpr uint32_t kIdescHalf = E4M3 ? idesc_e4m3_f32(kBM, 256)
-                                       : idesc_bf16_f32(kBM, 256, /*b_mn_major=*/true);
-  constexpr int kTmemCols = 512;
-  constexpr int S = kWideStages;
-  extern __shared__ uint8_t dsmem_raw[];
-  __shared__ PairShared sh;
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int n_tiles = (n_out + kOutCols - 1) / kOutCols;
-  const int nkb = (K + kKb - 1) / kKb;   // e4m3: a last half k-block reads zeros past K
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&sh.full_bar[s], 1);
-      mbar_init(&sh.empty_bar[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&sh.tfull_bar[a], 1);
-      mbar_init(&sh.tempty_bar[a], 2 * epi_warps(SWIGLU));   // the epilogue warps of both CTAs
-    }
-    mbar_init(&sh.drain_bar, 1);
-    sh.abort_flag = 0;
-    sh.never = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0) {
-    tmem_alloc_pair(&sh.tmem_base, kTmemCols);
-    tmem_relinquish_pair();
-  }
-  if (warp == 1 && lane == 0) {
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmA64);
-    prefetch_tensormap(&tmB0);
-    if (SWIGLU) prefetch_tensormap(&tmB1);
-    if (E4M3) prefetch_tensormap(&tmB0h);
-    if (E4M3 && SWIGLU) prefetch_tensormap(&tmB1h);
-  }
-  if (warp == 2) {
-    int carry = 0;
-    for (int base = 0; base < E; base += 32) {
-      const int e = base + lane;
-      int tiles = 0;
-      if (e < E) {
-        const int o0 = offsets[e], o1 = offsets[e + 1];
-        int cnt = o1 - o0;
-        if (o0 < 0 || cnt < 0 || o1 > max_rows) {
-          report(status, kDevErrBadOffsets);
-          cnt = 0;
-        }
-        if (fz.bucket_rows) cnt = min(cnt, max(0, fz.bucket_rows[e]));
-        sh.row_off[e] = o0;
-        sh.row_cnt[e] = cnt;
-        tiles = cnt > 0 ? ((cnt + kPairM - 1) / kPairM) * n_tiles : 0;
-      }
-      int incl = tiles;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      if (e < E) sh.tile_prefix[e] = carry + incl - tiles;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) sh.tile_prefix[E] = carry;
-  }
-  tc_fence_before();
-  cluster_sync();            // both CTAs' barriers initialised, TMEM allocated
-  tc_fence_after();
-
-  const uint32_t tmem_base = sh.tmem_base;
-  const int total_tiles = sh.tile_prefix[E];
-  volatile int* abort_flag = &sh.abort_flag;
-  const uint32_t peer_abort = mapa_shared(&sh.abort_flag, rank ^ 1u);
-  auto give_up = [&]() {
-    *abort_flag = 1;
-    st_shared_cluster_u32(peer_abort, 1u);
-    report(status, kDevErrWaitTimeout);
-  };
-  // does tile n use acc1 (a second 256-column accumulator)?
-  auto two_accs = [&](int n) { return n * kOutCols + (SWIGLU ? 128 : 256) < n_out; };
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------ TMA producer (both CTAs)
-      int it = 0;
-      int last_it[S];
-      for (int s = 0; s < S; ++s) last_it[s] = -1;
-      bool ok = true;
-      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
-        int e, m, n;
-        decode_pair_tile(sh, tile, E, n_tiles, e, m, n);
-        const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
-        const bool two = two_accs(n);
-        const int ew = weight_index(fz, e);
-        const int row0 = sh.row_off[e] + m * kPairM + (int)rank * (half ? kBM / 2 : kBM);
-        const uint32_t a_bytes = half ? kWideABytes / 2 : kWideABytes;
-        const uint32_t b_bytes = two ? 2 * kWideAccBBytes : kWideAccBBytes;
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          if (!mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag)) { ok = false; break; }
-          uint8_t* sa = smem + s * kWideStageBytes;
-          uint8_t* sb = sa + kWideABytes;
-          const uint32_t full_lead = mapa_shared(&sh.full_bar[s], 0);
-          // both CTAs' copies complete on the leader's barrier
-          if (leader) mbar_arrive_expect_tx(&sh.full_bar[s], 2 * (a_bytes + b_bytes));
-          tma_load_2d_pair(sa, half ? &tmA64 : &tmA, full_lead, kb * kKb, row0);
-          for (int a = 0; a < (two ? 2 : 1); ++a) {
-            uint8_t* sba = sb + a * kWideAccBBytes;
-            if (SWIGLU) {
-              const int hc0 = n * kOutCols + a * 128;     // first h-column of acc a
-              if (E4M3) {
-                if (half) {
-                  tma_load_3d_pair(sba, &tmB0h, full_lead, kb * kKb, hc0 + (int)rank * 64, ew);
-                  tma_load_3d_pair(sba + 64 * 128, &tmB1h, full_lead, kb * kKb,
-                                   hc0 + (int)rank * 64, ew);
-                } else {
-                  tma_load_3d_pair(sba, leader ? &tmB0 : &tmB1, full_lead, kb * kKb, hc0, ew);
-                }
-              } else if (half) {
-                tma_load_3d_pair(sba, &tmB0, full_lead, hc0 + (int)rank * 64, kb * kBK, ew);
-                tma_load_3d_pair(sba + kChunkBytes, &tmB1, full_lead, hc0 + (int)rank * 64,
-                                 kb * kBK, ew);
-              } else {
-                const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                  tma_load_3d_pair(sba + c * kChunkBytes, mb, full_lead, hc0 + c * 64, kb * kBK,
-                                   ew);
-              }
-            } else {
-              const int oc0 = n * kOutCols + a * 256 + (int)rank * 128;
-              if (E4M3) {
-                tma_load_3d_pair(sba, &tmB0, full_lead, kb * kKb, oc0, ew);
-              } else {
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                  tma_load_3d_pair(sba + c * kChunkBytes, &tmB0, full_lead, oc0 + c * 64,
-                                   kb * kBK, ew);
-              }
-            }
-          }
-          last_it[s] = it;
-        }
-      }
-      if (!ok) give_up();
-      if (leader) {
-        // both CTAs' copies of every issued phase count on the leader's barriers
-        for (int s = 0; s < S; ++s)
-          if (last_it[s] >= 0) mbar_wait(&sh.full_bar[s], (last_it[s] / S) & 1, &sh.never);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      // ------------------------------------------------ MMA issuer (leader CTA)
-      // one k-block of stage s into accumulator a (k-block index kb)
-      auto mma_kblock = [&](int s, int a, int kb, uint32_t idesc) {
-        const uint32_t a_addr = smem_u32(smem + s * kWideStageBytes);
-        const uint32_t b_addr = a_addr + kWideABytes + a * kWideAccBBytes;
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * 256);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t adesc = smem_desc_sw128(a_addr + ks * 32, 16, 1024);
-          if (E4M3) {
-            const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 32, 16, 1024);
-            umma_e4m3_pair(d_tmem, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
-          } else {
-            const uint64_t bdesc = smem_desc_sw128(b_addr + ks * 2048, kChunkBytes, 1024);
-            umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
-          }
-        }
-      };
-      int it = 0, u0 = 0, u1 = 0;
-      bool ok = true;
-      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
-        int e, m, n;
-        decode_pair_tile(sh, tile, E, n_tiles, e, m, n);
-        const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
-        const bool two = two_accs(n);
-        const uint32_t idesc = half ? kIdescHalf : kIdesc;
-        if (!mbar_wait(&sh.tempty_bar[0], (u0 & 1) ^ 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t ph1 = (u1 & 1) ^ 1;
-        bool have1 = !two;
-        const int it0 = it;
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % S;
-          if (!mbar_wait(&sh.full_bar[s], (it / S) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          mma_kblock(s, 0, kb, idesc);
-          if (kb == nkb - 1) umma_commit_pair_mc(&sh.tfull_bar[0], 0x3);
-          if (!two) {
-            umma_commit_pair_mc(&sh.empty_bar[s], 0x3);
-            continue;
-          }
-          if (!have1) {
-            have1 = mbar_test_wait(smem_u32(&sh.tempty_bar[1]), ph1);
-            // every stage held, or the tile's last k-block: acc1 must be free now
-            if (!have1 && (kb + 1 == S || kb + 1 == nkb)) {
-              if (!mbar_wait(&sh.tempty_bar[1], ph1, abort_flag)) { ok = false; break; }
-              have1 = true;
-            }
-            if (have1) {
-              tc_fence_after();
-              // replay the held k-blocks 0 .. kb-1 into acc1, freeing their stages
-              for (int h = 0; h < kb; ++h) {
-                const int sh_ = (it0 + h) % S;
-                mma_kblock(sh_, 1, h, idesc);
-                umma_commit_pair_mc(&sh.empty_bar[sh_], 0x3);
-              }
-            }
-          }
-          if (have1) {
-            mma_kblock(s, 1, kb, idesc);
-            umma_commit_pair_mc(&sh.empty_bar[s], 0x3);
-            if (kb == nkb - 1) umma_commit_pair_mc(&sh.tfull_bar[1], 0x3);
-          }
-        }
-        if (!ok) break;
-        ++u0;
-        if (two) ++u1;
-      }
-      if (!ok) give_up();
-      umma_commit_pair_mc(&sh.drain_bar, 0x1);
-      mbar_wait(&sh.drain_bar, 0, &sh.never);
-    }
-  } else {
-    // -------------------------------------------------- epilogue (warps 2.., both CTAs)
-    const int q = warp & 3;
-    constexpr int kGroups = epi_warps(SWIGLU) / 4;     // warp groups splitting the chunks
-    const int grp = (warp - 2) / 4;
-    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + wide_staging_off()) +
-                      (warp - 2) * stage_words(16);
-    int u[2] = {0, 0};
-    bool ok = true;
-    for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
-      int e, m, n;
-      decode_pair_tile(sh, tile, E, n_tiles, e, m, n);
-      const bool half = sh.row_cnt[e] - m * kPairM <= kBM;
-      const bool two = two_accs(n);
-      const int ew = weight_index(fz, e);
-      const float* cs0 = E4M3 ? col_scale0 + (size_t)ew * n_out : nullptr;
-      const float* cs1 = (E4M3 && SWIGLU) ? col_scale1 + (size_t)ew * n_out : nullptr;
-      for (int a = 0; a < (two ? 2 : 1); ++a) {
-        if (!mbar_wait(&sh.tfull_bar[a], u[a] & 1, abort_flag)) {
-          give_up();
-          ok = false;
-          break;
-        }
-        ++u[a];
-        tc_fence_after();
-        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                               static_cast<uint32_t>(a * 256);
-        // first output column of accumulator a
-        const int ca = n * kOutCols + a * (SWIGLU ? 128 : 256);
-        if (!half) {
-          const int first = m * kPairM + (int)rank * kBM + q * 32;   // first row of this warp
-          const int nvalid = clamp_rows(sh.row_cnt[e] - first);
-          const size_t row0 = (size_t)(sh.row_off[e] + first);
-          const float sr = (E4M3 && lane < nvalid) ? row_scale[row0 + lane] : 0.f;
-          if (SWIGLU) {
-            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out + ca;
-#pragma unroll 1
-            for (int c = grp; c < 4 && ca + c * 32 < n_out; c += kGroups)
-              swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 128 + c * 32, o + c * 32, n_out,
-                                       nvalid, lane, cs0 + ca + c * 32, cs1 + ca + c * 32, sr);
-          } else if (FUSE == kFuseScatter) {
-            int my_t = 0;
-            float my_w = 0.f;
-            if (lane < nvalid) {
-              const int p = fz.row_pair[row0 + lane];
-              my_t = p / fz.k;
-              my_w = fz.topk_w[p];
-            }
-#pragma unroll 1
-            for (int c = grp; c < 8 && ca + c * 32 < n_out; c += kGroups) {
-              uint32_t v[32];
-              tmem_ld_32x32b_x32(tbase + c * 32, v);
-              tmem_ld_wait();
-              if (E4M3) apply_scales(v, cs0 + ca + c * 32, sr);
-              scatter_chunk_f32<16>(v, stage, fz.y32 + ca + c * 32, n_out, my_t, my_w, nvalid,
-                                    lane);
-            }
-          } else {
-            float* o = static_cast<float*>(out_raw) + row0 * n_out + ca;
-#pragma unroll 1
-            for (int c = grp; c < 8 && ca + c * 32 < n_out; c += kGroups) {
-              uint32_t v[32];
-              tmem_ld_32x32b_x32(tbase + c * 32, v);
-              tmem_ld_wait();
-              if (E4M3) apply_scales(v, cs0 + ca + c * 32, sr);
-              store_chunk_f32<16>(v, stage, o + c * 32, n_out, nvalid, lane);
-            }
-          }
-        } else {
-          // M = 128 pair form: lanes 0-63 hold accumulator columns [0,128),
-          // lanes 64-127 columns [128,256), each for this CTA's 64 rows
-          const int hh = q >> 1;
-          const int first = m * kPairM + (int)rank * (kBM / 2) + (q & 1) * 32;
-          const int nvalid = clamp_rows(sh.row_cnt[e] - first);
-          const size_t row0 = (size_t)(sh.row_off[e] + first);
-          const float sr = (E4M3 && lane < nvalid) ? row_scale[row0 + lane] : 0.f;
-          if (SWIGLU) {
-            // gate in TMEM columns [0,64), up in [64,128); lanes 64-127 hold
-            // the next 64 h-columns (staged by the other CTA's half of B)
-            const int c0 = ca + hh * 64;
-            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out + c0;
-#pragma unroll 1
-            for (int c = grp; c < 2 && c0 + c * 32 < n_out; c += kGroups)
-              swiglu_chunk_store<E4M3>(tbase + c * 32, tbase + 64 + c * 32, o + c * 32, n_out,
-                                       nvalid, lane, cs0 + c0 + c * 32, cs1 + c0 + c * 32, sr);
-          } else if (FUSE == kFuseScatter) {
-            const int c0 = ca + hh * 128;
-            int my_t = 0;
-            float my_w = 0.f;
-            if (lane < nvalid) {
-              const int p = fz.row_pair[row0 + lane];
-              my_t = p / fz.k;
-              my_w = fz.topk_w[p];
-            }
-#pragma unroll 1
-            for (int c = grp; c < 4 && c0 + c * 32 < n_out; c += kGroups) {
-              uint32_t v[32];
-              tmem_ld_32x32b_x32(tbase + c * 32, v);
-              tmem_ld_wait();
-              if (E4M3) apply_scales(v, cs0 + c0 + c * 32, sr);
-              scatter_chunk_f32<16>(v, stage, fz.y32 + c0 + c * 32, n_out, my_t, my_w, nvalid,
-                                    lane);
-            }
-          } else {
-            const int c0 = ca + hh * 128;
-            float* o = static_cast<float*>(out_raw) + row0 * n_out + c0;
-#pragma unroll 1
-            for (int c = grp; c < 4 && c0 + c * 32 < n_out; c += kGroups) {
-              uint32_t v[32];
-              tmem_ld_32x32b_x32(tbase + c * 32, v);
-              tmem_ld_wait();
-              if (E4M3) apply_scales(v, cs0 + c0 + c * 32, sr);
-              store_chunk_f32<16>(v, stage, o + c * 32, n_out, nvalid, lane);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(&sh.tempty_bar[a], 0));
-      }
-    }
-  }
-
-  if (*abort_flag) spin_ns(200000);      // let copies still in flight land
-  tc_fence_before();
-  cluster_sync();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, kTmemCols);
-  }
-}
-
 // ---------------------------------------------------------------- host side
 
 template <int BN, bool SWIGLU, int FUSE>
@@ -1614,72 +1197,6 @@ static cudaError_t launch_gemm_pair_t(int slot, const CUtensorMap& a, const CUte
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a, a64, b0, b1, b0h ? *b0h : b0, b1h ? *b1h : b1,
                             row_scale, cs0, cs1, offsets, E, K, n_out, max_rows, out, status, fz);
-}
-
-static int fuse_kind(const FuseArgs& fz);
-
-template <bool SWIGLU, bool E4M3, int FUSE>
-static cudaError_t launch_gemm_wide_t(int slot, const CUtensorMap& a, const CUtensorMap& a64,
-                                      const CUtensorMap& b0, const CUtensorMap& b1,
-                                      const int32_t* offsets, int E, int K, int n_out,
-                                      int max_rows, void* out, int32_t* status, cudaStream_t s,
-                                      const FuseArgs& fz, const CUtensorMap* b0h,
-                                      const CUtensorMap* b1h, const float* row_scale,
-                                      const float* cs0, const float* cs1) {
-  constexpr int kSmem = wide_smem_bytes(SWIGLU);
-  DeviceInfo* di = nullptr;
-  cudaError_t err = device_info(&di);
-  if (err != cudaSuccess) return err;
-  auto kern = grouped_gemm_wide_kernel<SWIGLU, E4M3, FUSE>;
-  if (!di->attr_set[slot]) {
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (err != cudaSuccess) return err;
-    di->attr_set[slot] = true;
-  }
-  const int n_tiles = (n_out + wide_out_cols(SWIGLU) - 1) / wide_out_cols(SWIGLU);
-  const long long pair_rows = (long long)max_rows / (2 * kBM) + (E < max_rows ? E : max_rows);
-  long long pairs = pair_rows * n_tiles;
-  const int max_pairs = di->sms / 2;
-  if (pairs > max_pairs) pairs = max_pairs;
-  if (pairs < 1) pairs = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(gemm_threads(SWIGLU), 1, 1);
-  cfg.dynamicSmemBytes = kSmem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, a64, b0, b1, b0h ? *b0h : b0, b1h ? *b1h : b1,
-                            row_scale, cs0, cs1, offsets, E, K, n_out, max_rows, out, status, fz);
-}
-
-// The wide pair tiles (M = 256, N = 512) for plain and scattering GEMMs (the
-// gathering producer stays on the narrower kernels).
-template <bool SWIGLU, bool E4M3 = false>
-static cudaError_t launch_gemm_wide(int slot, const CUtensorMap& a, const CUtensorMap& a64,
-                                    const CUtensorMap& b0, const CUtensorMap& b1,
-                                    const int32_t* offsets, int E, int K, int n_out, int max_rows,
-                                    void* out, int32_t* status, cudaStream_t s,
-                                    const FuseArgs& fz, const CUtensorMap* b0h = nullptr,
-                                    const CUtensorMap* b1h = nullptr,
-                                    const float* row_scale = nullptr,
-                                    const float* cs0 = nullptr, const float* cs1 = nullptr) {
-  const int kind = fuse_kind(fz);
-  if constexpr (!E4M3 && !SWIGLU) {
-    if (kind == kFuseScatter)
-      return launch_gemm_wide_t<SWIGLU, E4M3, kFuseScatter>(slot + 32, a, a64, b0, b1, offsets,
-                                                            E, K, n_out, max_rows, out, status,
-                                                            s, fz, b0h, b1h, row_scale, cs0, cs1);
-  }
-  if (kind != kFuseNone) return cudaErrorInvalidValue;
-  return launch_gemm_wide_t<SWIGLU, E4M3, kFuseNone>(slot, a, a64, b0, b1, offsets, E, K, n_out,
-                                                     max_rows, out, status, s, fz, b0h, b1h,
-                                                     row_scale, cs0, cs1);
 }
 
 // The fusion an instance is compiled for, from the arguments.
@@ -1760,20 +1277,6 @@ static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtens
 // per expert bound the average bucket from above.
 static bool use_pair_tiles(int E, int max_rows) { return max_rows >= 512LL * E; }
 
-// The wide pair tiles (256 rows x 512 accumulator columns).  Their main loop
-// moves a quarter fewer operand bytes per FLOP than the 256 x 256 pair tiles,
-// but with both accumulators in TMEM the epilogue is only partly hidden, so
-// they pay off for long contractions, and for buckets of 256-511 rows, where
-// the alternative is the single-CTA tile.  Measured on B200 (GEMM 1, buckets
-// of 9472 rows): at K = 8192 1555 vs 1394 TFLOP/s, at K = 2048 equal, at
-// K = 1024 7 % slower; the fp32 epilogue of GEMM 2 moves the break-even to
-// K = 8192, and on the Mixtral-shaped layer (K = 4096 / 14336) they tie.
-static bool use_wide_tiles(int E, int max_rows, int K, bool swiglu, bool gather) {
-  if (gather || max_rows < 256LL * E) return false;
-  if (max_rows < 512LL * E) return swiglu && K >= 4096;
-  return K >= 8192;
-}
-
 // The A operand: the permuted rows [max_rows, K] (128- and 64-row boxes), or,
 // when gathering, the token rows [fz.n_tok, K] (one-row boxes for gather4).
 static bool map_a(CUtensorMap* a, CUtensorMap* a64, const void* rows, int K, int max_rows,
@@ -1800,9 +1303,6 @@ cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, 
                   map_weights(&tg, w_gate, weight_count(fz, E), d, f) &&
                   map_weights(&tu, w_up, weight_count(fz, E), d, f));
   if (*map_failed) return cudaSuccess;
-  if (use_wide_tiles(E, max_rows, d, true, fz.row_src != nullptr))
-    return launch_gemm_wide<true>(14, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s,
-                                  fz);
   if (use_pair_tiles(E, max_rows))
     return launch_gemm_pair<true>(7, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s,
                                   fz);
@@ -1818,9 +1318,6 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
   *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_rows(&ta64, h, f, max_rows, kBM / 2) &&
                   map_weights(&td, w_down, weight_count(fz, E), f, d));
   if (*map_failed) return cudaSuccess;
-  if (d % 256 == 0 && use_wide_tiles(E, max_rows, f, false, false))
-    return launch_gemm_wide<false>(15, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,
-                                   status, s, fz);
   if (d % 256 == 0 && use_pair_tiles(E, max_rows))
     return launch_gemm_pair<false>(8, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
                                    s, fz);
@@ -1872,15 +1369,11 @@ cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_
                   map_weights_e4m3(&tg, wq_gate, weight_count(fz, E), f, d) &&
                   map_weights_e4m3(&tu, wq_up, weight_count(fz, E), f, d));
   if (*map_failed) return cudaSuccess;
-  const bool wide = use_wide_tiles(E, max_rows, d, true, fz.row_src != nullptr);
-  if (wide || use_pair_tiles(E, max_rows)) {
+  if (use_pair_tiles(E, max_rows)) {
     CUtensorMap tgh, tuh;
     *map_failed = !(map_weights_e4m3(&tgh, wq_gate, weight_count(fz, E), f, d, 64) &&
                     map_weights_e4m3(&tuh, wq_up, weight_count(fz, E), f, d, 64));
     if (*map_failed) return cudaSuccess;
-    if (wide)
-      return launch_gemm_wide<true, true>(17, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h,
-                                          status, s, fz, &tgh, &tuh, sx, s_gate, s_up);
     return launch_gemm_pair<true, true>(9, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h,
                                         status, s, fz, &tgh, &tuh, sx, s_gate, s_up);
   }
@@ -1897,9 +1390,6 @@ cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int3
                   map_rows_e4m3(&ta64, hq, f, max_rows, kBM / 2) &&
                   map_weights_e4m3(&td, wq_down, weight_count(fz, E), d, f));
   if (*map_failed) return cudaSuccess;
-  if (d % 256 == 0 && use_wide_tiles(E, max_rows, f, false, false))
-    return launch_gemm_wide<false, true>(18, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,
-                                         status, s, fz, &td, &td, sh_rows, s_down, nullptr);
   if (d % 256 == 0 && use_pair_tiles(E, max_rows))
     return launch_gemm_pair<false, true>(10, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,
                                          status, s, fz, &td, &td, sh_rows, s_down, nullptr);

@@ -37,9 +37,13 @@ constexpr int kRankThreads = 1024;     // 32 warps x 8 tokens per chunk
 constexpr int kRankWarps = kRankThreads / 32;
 constexpr int kTokPerWarp = kChunk / kRankWarps;
 constexpr int kScanThreads = 1024;     // 32 warps; lane = one expert of a group of 32
-constexpr int kScatThreads = 256;      // 8 warps
-constexpr int kScatTokens = 8;         // tokens per scatter CTA (one per warp; divides kChunk)
+constexpr int kScatThreads = 256;      // 8 warps: thread e derives expert e's offsets
+// tokens per scatter CTA, one per warp (divides kChunk): 4 keeps the staged
+// rows of a CTA at 4 x row bytes, so that 8 KB rows still let 7 CTAs share
+// an SM and a 4096-token batch runs in one wave
+constexpr int kScatTokens = 4;
 constexpr int kDirectSum = 4096;       // histogram counters a scatter CTA sums without the scan
+constexpr int kBulkRowBytes = 16384;   // rows up to this size move through shared memory
 
 // 1. rank: per chunk, the rank of each pair among the chunk's pairs of the
 //    same expert (token order), and the chunk's per-expert histogram.
@@ -54,8 +58,10 @@ __global__ void __launch_bounds__(kRankThreads)
   const int nt = min(kChunk, T - chunk_t0);
 
   for (int i = tid; i < kRankWarps * 256; i += kRankThreads) (&cnt[0][0])[i] = 0;
+  grid_dep_wait();          // topk_idx (and x) may come from the kernel before
+  // only now may the scan and scatter start: the scatter reads x before it
+  // waits, so every kernel before this permutation must have completed
   grid_dep_launch();
-  grid_dep_wait();          // topk_idx may come from the kernel before
   for (int i = tid; i < nt * k; i += kRankThreads) pairs[i] = topk_idx[(size_t)chunk_t0 * k + i];
   __syncthreads();
 
@@ -141,10 +147,14 @@ __global__ void __launch_bounds__(kScanThreads)
 // 3. scatter: every CTA (8 tokens of one chunk) reads the per-expert demand
 //    and its chunk's base, derives kept counts and offsets (exclusive scan
 //    over experts); CTA 0 also writes counts / offsets / n_dropped.  Then one
-//    warp per token turns ranks into slots, drops pairs at slot >= C, and
-//    copies the token row to its kept rows with 16-byte vectors.
+//    warp per token (the first kScatTokens warps) turns ranks into slots,
+//    drops pairs at slot >= C, and copies the token row to its kept rows.  Rows of up to kBulkRowBytes go
+//    through shared memory by bulk copy: each warp's lane 0 loads its token's
+//    row before waiting for the rank kernel (the read overlaps it), then
+//    stores it to the k destination rows; longer rows are copied with
+//    16-byte vector loads and stores.
 __global__ void __launch_bounds__(kScatThreads)
-    permute_scatter_kernel(const uint8_t* __restrict__ x, int row_bytes,
+    permute_scatter_kernel(const uint8_t* __restrict__ x, int row_bytes, bool bulk,
                            const float* __restrict__ x_scale,
                            const int32_t* __restrict__ topk_idx, int32_t* __restrict__ slot,
                            const int32_t* __restrict__ chunk_base, bool scanned,
@@ -154,19 +164,33 @@ __global__ void __launch_bounds__(kScatThreads)
                            int32_t* __restrict__ row_src, uint8_t* __restrict__ x_perm,
                            float* __restrict__ perm_scale, bool padded,
                            int32_t* __restrict__ row_pair, float* __restrict__ zero_rows,
-                           int zero_cols) {
+                           int zero_cols, int32_t* status) {
+  extern __shared__ __align__(128) uint8_t s_rows[];   // bulk: one row per warp
   __shared__ int32_t s_off[256];
   __shared__ int32_t s_base[256];
   __shared__ int32_t warp_sum[8];
   __shared__ int32_t warp_drop[8];
+  __shared__ uint64_t row_bar[kScatTokens];
+  __shared__ int never;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int t0 = blockIdx.x * kScatTokens;
   const int my_chunk = t0 / kChunk;
+  // the token this warp copies (warps past kScatTokens only help with the offsets)
+  const int t_own = warp < kScatTokens ? t0 + warp : T;
+  uint8_t* my_row_sh = s_rows + (size_t)(warp < kScatTokens ? warp : 0) * row_bytes;
 
-  // this CTA's token rows into L2 while the rank and scan kernels finish
-  if (x && lane == 0) {
-    for (int tt = warp; tt < kScatTokens; tt += kScatThreads / 32)
-      if (t0 + tt < T) prefetch_l2_bulk(x + (size_t)(t0 + tt) * row_bytes, row_bytes);
+  // this CTA's token rows (inputs, not produced by the kernels before) start
+  // moving while the rank and scan kernels finish
+  if (x && lane == 0 && t_own < T) {
+    if (bulk) {
+      never = 0;
+      mbar_init(&row_bar[warp], 1);
+      fence_barrier_init();
+      mbar_arrive_expect_tx(&row_bar[warp], (uint32_t)row_bytes);
+      bulk_load(my_row_sh, x + (size_t)t_own * row_bytes, (uint32_t)row_bytes, &row_bar[warp]);
+    } else {
+      prefetch_l2_bulk(x + (size_t)t_own * row_bytes, row_bytes);
+    }
   }
   grid_dep_launch();
   grid_dep_wait();          // ranks in slot, chunk bases and totals
@@ -225,10 +249,11 @@ __global__ void __launch_bounds__(kScatThreads)
   __syncthreads();
 
   // ---- one warp per token
+  static_assert(kScatTokens <= kScatThreads / 32, "one token per warp");
   const int nvec = row_bytes / 16;
-  for (int tt = warp; tt < kScatTokens; tt += kScatThreads / 32) {
-    const int t = t0 + tt;
-    if (t >= T) break;
+  {
+    const int t = t_own;
+    if (t >= T) return;
     int my_row = -1;
     if (lane < k) {
       const size_t p = (size_t)t * k + lane;
@@ -248,10 +273,28 @@ __global__ void __launch_bounds__(kScatThreads)
       float4* z = reinterpret_cast<float4*>(zero_rows + (size_t)t * zero_cols);
       for (int v = lane; v < zero_cols / 4; v += 32) z[v] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (!x) continue;         // index-only: the GEMM gathers the rows itself
+    if (!x) return;           // index-only: the GEMM gathers the rows itself
     int rows[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+
+    if (bulk) {
+      if (lane == 0) {
+        // the row landed in shared memory: store it to each kept row
+        if (!mbar_wait(&row_bar[warp], 0, &never)) {
+          report(status, kDevErrWaitTimeout);
+          mbar_wait(&row_bar[warp], 0, &never);     // the copy in flight must land
+          return;
+        }
+        fence_proxy_async_smem();
+        for (int j = 0; j < k; ++j)
+          if (rows[j] >= 0)
+            bulk_store(x_perm + (size_t)rows[j] * row_bytes, my_row_sh, (uint32_t)row_bytes);
+        bulk_commit();
+        bulk_wait_all();      // shared memory is read before the CTA exits
+      }
+      return;
+    }
 
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
     for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
@@ -316,6 +359,36 @@ static cudaError_t launch_rank_scan(const int32_t* topk_idx, int T, int E, int k
                           chunk_hist, nchunks, E);
 }
 
+// The scatter launch: rows staged through shared memory (bulk copies) when
+// they fit kBulkRowBytes, one row per warp.
+static cudaError_t launch_scatter(const uint8_t* x, int row_bytes, const float* x_scale,
+                                  const int32_t* topk_idx, int32_t* slot,
+                                  const int32_t* chunk_hist, bool scanned, int T, int E, int k,
+                                  int64_t C, int32_t* counts, int32_t* offsets,
+                                  int32_t* n_dropped, int32_t* row_src, uint8_t* x_perm,
+                                  float* perm_scale, bool padded, int32_t* row_pair,
+                                  float* zero_rows, int zero_cols, int32_t* status,
+                                  cudaStream_t s) {
+  DeviceInfo* di = nullptr;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  constexpr int kSlot = 24;                 // attribute slot of the scatter kernel
+  const bool bulk = x != nullptr && row_bytes <= kBulkRowBytes;
+  const size_t smem = bulk ? (size_t)kScatTokens * row_bytes : 0;
+  if (bulk && !di->attr_set[kSlot]) {
+    err = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kScatTokens * kBulkRowBytes);
+    if (err != cudaSuccess) return err;
+    di->attr_set[kSlot] = true;
+  }
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  return launch_dependent(permute_scatter_kernel, dim3((T + kScatTokens - 1) / kScatTokens),
+                          dim3(kScatThreads), smem, s, x, row_bytes, bulk, x_scale, topk_idx,
+                          slot, chunk_hist, scanned, nchunks, T, E, k, C, counts, offsets,
+                          n_dropped, row_src, x_perm, perm_scale, padded, row_pair, zero_rows,
+                          zero_cols, status);
+}
+
 cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_scale,
                                 const int32_t* topk_idx, int T, int E, int k, int64_t C,
                                 int32_t* counts, int32_t* offsets, int32_t* slot,
@@ -323,14 +396,12 @@ cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_
                                 int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
                                 int32_t* row_pair, float* zero_rows, int zero_cols,
                                 int32_t* status) {
-  const int nchunks = (T + kChunk - 1) / kChunk;
   bool scanned = false;
   cudaError_t err = launch_rank_scan(topk_idx, T, E, k, slot, chunk_hist, s, status, &scanned);
   if (err != cudaSuccess) return err;
-  return launch_dependent(permute_scatter_kernel, dim3((T + kScatTokens - 1) / kScatTokens),
-                          dim3(kScatThreads), 0, s, x, row_bytes, x_scale, topk_idx, slot,
-                          chunk_hist, scanned, nchunks, T, E, k, C, counts, offsets, n_dropped,
-                          row_src, x_perm, perm_scale, false, row_pair, zero_rows, zero_cols);
+  return launch_scatter(x, row_bytes, x_scale, topk_idx, slot, chunk_hist, scanned, T, E, k, C,
+                        counts, offsets, n_dropped, row_src, x_perm, perm_scale, false, row_pair,
+                        zero_rows, zero_cols, status, s);
 }
 
 // The padded [E, C, d] layout: bucket e holds rows e*C .. e*C + C - 1, its
@@ -340,16 +411,13 @@ cudaError_t launch_permute_padded(const __nv_bfloat16* x, const int32_t* topk_id
                                   int32_t* slot, int32_t* row_src, __nv_bfloat16* x_pad,
                                   int32_t* n_dropped, int32_t* chunk_hist, cudaStream_t s,
                                   int32_t* status) {
-  const int nchunks = (T + kChunk - 1) / kChunk;
   bool scanned = false;
   cudaError_t err = launch_rank_scan(topk_idx, T, E, k, slot, chunk_hist, s, status, &scanned);
   if (err != cudaSuccess) return err;
   uint8_t* xp = reinterpret_cast<uint8_t*>(x_pad);
-  err = launch_dependent(permute_scatter_kernel, dim3((T + kScatTokens - 1) / kScatTokens),
-                         dim3(kScatThreads), 0, s, reinterpret_cast<const uint8_t*>(x), d * 2,
-                         nullptr, topk_idx, slot, chunk_hist, scanned, nchunks, T, E, k, C,
-                         counts, offsets, n_dropped, row_src, xp, nullptr, true, nullptr, nullptr,
-                         0);
+  err = launch_scatter(reinterpret_cast<const uint8_t*>(x), d * 2, nullptr, topk_idx, slot,
+                       chunk_hist, scanned, T, E, k, C, counts, offsets, n_dropped, row_src, xp,
+                       nullptr, true, nullptr, nullptr, 0, status, s);
   if (err != cudaSuccess) return err;
   const int64_t rows = (int64_t)E * C;
   return launch_dependent(permute_pad_fill_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0,

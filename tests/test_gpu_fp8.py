@@ -182,8 +182,7 @@ MLP_CASES = [
     (256, 384, [300, 0, 1, 129, 128, 257, 700], True),
     (512, 256, [1, 256, 511, 513, 1024], True),
     (384, 256, [255, 257, 0], True),      # down GEMM: d % 256 != 0 keeps single-CTA tiles
-    # several CTA-pair tiles per pair; the wide pair tiles on GEMM 1 with
-    # 256-511 buffer rows per expert and K >= 4096, and on GEMM 2 with K >= 8192
+    # several CTA-pair tiles per pair; long contractions
     (512, 384, [3000, 2999, 1, 2900], True),
     (256, 1024, [2048] * 4, True),
     (4096, 384, [300, 260, 255, 511, 0, 1], "mid"),

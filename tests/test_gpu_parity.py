@@ -43,7 +43,7 @@ SMALL = [
     # widths that are multiples of 64 but not of 128: ragged 64-column tails
     # in the router's K, the permuted rows, every GEMM tile shape and the combine
     small("width64", T=300, d=192, E=8, k=2, f=320, cf=1.25, seed=23),
-    small("width64_wide", T=2048, d=320, E=4, k=2, f=192, cf=0.0, seed=24),
+    small("width64_pair", T=2048, d=320, E=4, k=2, f=192, cf=0.0, seed=24),
 ]
 IDS = [c.name for c in SMALL]
 
@@ -231,14 +231,9 @@ MLP_CASES = [
     (1024, 1024, [2048] * 4, True),
     (512, 128, [6000] * 4, True),
     (256, 384, [3000, 2999, 1, 2900], True),
-    # the wide pair tiles (256 rows x 512 accumulator columns, both TMEM
-    # accumulators, k-blocks replayed into the second): GEMM 1 on buckets of
-    # 256-511 rows with K = d >= 4096 ("mid": 256-511 buffer rows per expert),
-    # GEMM 1 and 2 with K >= 8192 on large buckets, with more tiles than CTA
-    # pairs (E = 2 x 2560 rows, f = 1024: 80 wide tiles), and one-accumulator
-    # N tails (f = 384: 256 + 128 h-columns; d = 768: 512 + 256 columns)
+    # long contractions (K = 4096 with 256-511 buffer rows per expert, "mid";
+    # K = 8192 on CTA-pair tiles)
     (4096, 384, [300, 260, 255, 511, 0, 1], "mid"),
-    (8192, 1024, [2560, 2560], True),
     (768, 8192, [600, 1, 300], True),
     # d, f multiples of 64 only: 64-column N tails and K = 64 * odd
     (192, 320, [300, 0, 1, 129, 128, 257], False),
@@ -249,8 +244,8 @@ MLP_CASES = [
 
 def mlp_buffer_rows(N, E, pair):
     """Rows of the permuted buffer for a bucket layout: pair=True gives >= 512
-    per expert (CTA-pair tiles), "mid" 256-511 (wide tiles for GEMM 1 on long
-    K, else single-CTA), False fewer (single-CTA tiles)."""
+    per expert (CTA-pair tiles), "mid" 256-511 and False fewer (single-CTA
+    tiles)."""
     if pair == "mid":
         rows = max(N + 37, 256 * E + 5)
         assert rows < 512 * E

@@ -680,9 +680,10 @@ def main():
     if world > 1:
         import datetime
         import torch.distributed as td
-        torch.cuda.set_device(local_rank)
-        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                              device_id=torch.device("cuda", local_rank))
+        if not td.is_initialized():        # (a caller may have set up the group already)
+            torch.cuda.set_device(local_rank)
+            td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                  device_id=torch.device("cuda", local_rank))
     r = gpu_arm(args, cfg, rank, world, local_rank)
     pk, pk_kind = peaks()
     K = args.steps

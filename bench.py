@@ -32,7 +32,10 @@ from mixture_experts_layer_36_b200 import configs, synth  # noqa: E402
 METRIC = "MoE layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ROUTER_TILE_M = 128      # tokens per router GEMM row tile
-PAIR_MIN_ROWS = 512      # buffer rows per expert from which the GEMMs use CTA-pair tiles
+# buffer rows per expert from which the GEMMs use CTA-pair tiles, and (bf16)
+# CTA-pair tiles with the expert tails inside full tiles
+PAIR_MIN_ROWS = 512
+PAIR_TAIL_MIN_ROWS = 256
 ROOFLINE_TIMING = ("mean launch duration over the timed steps: CUDA events recorded around "
                    "the launch on its stream")
 FP8_OVER_BF16 = 2.0      # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
@@ -532,12 +535,19 @@ def summarize(cfg, args, r, pk, pk_kind, world):
         peak_tf *= FP8_OVER_BF16
         burst_tf *= FP8_OVER_BF16
         peak_src += f" x {FP8_OVER_BF16:g} (nominal e4m3 / bf16 dense ratio)"
-    # the library's tile choice: CTA pairs from PAIR_MIN_ROWS rows per expert
-    pair = moe_max_rows_host(cfg) >= PAIR_MIN_ROWS * cfg.E
+    # the library's tile choice by buffer rows per expert: CTA pairs from
+    # PAIR_MIN_ROWS, (bf16) CTA pairs with the expert tails from PAIR_TAIL_MIN_ROWS
+    rows_per_expert = moe_max_rows_host(cfg) / cfg.E
+    pair = rows_per_expert >= PAIR_MIN_ROWS
+    pair_tail = not args.fp8 and not pair and rows_per_expert >= PAIR_TAIL_MIN_ROWS
     if args.fp8:
         kname = ("grouped_gemm_pair_kernel<true,true> (gate/up + SwiGLU, e4m3, CTA pairs)"
                  if pair else "grouped_gemm_e4m3_kernel<256,true> (gate/up + SwiGLU, e4m3)")
         ktag = "gemm_e4m3_pair_gate_up" if pair else "gemm_e4m3_gate_up"
+    elif pair_tail:
+        kname = ("grouped_gemm_pair_tail_kernel<true> (gate/up + SwiGLU, CTA pairs, expert tails "
+                 "inside full tiles)")
+        ktag = "gemm_pair_tail_gate_up"
     else:
         kname = ("grouped_gemm_pair_kernel<true> (gate/up + SwiGLU, CTA pairs)" if pair else
                  "grouped_gemm_kernel<256,true> (gate/up + SwiGLU)")

@@ -36,6 +36,10 @@
 // abort flag and the caller's status bit, the others notice and stop, the
 // producer waits for its copies in flight, the MMA issuer waits for its MMAs,
 // and TMEM is freed before the CTA exits.
+#include <atomic>
+#include <mutex>
+#include <type_traits>
+
 #include "common.cuh"
 #include "host_util.cuh"
 
@@ -717,7 +721,7 @@ __device__ __forceinline__ void swiglu_chunk_store(uint32_t tg, uint32_t tu,
   store_chunk_bf16(pk, out_row0, ld, nvalid, lane);
 }
 
-template <bool SCALED>
+template <bool SCALED, int ROWS = 32>
 __device__ __forceinline__ void f32_chunk_store(uint32_t t, uint32_t* stage, float* out_row0,
                                                 size_t ld, int nvalid, int lane,
                                                 const float* sc, float sr) {
@@ -725,10 +729,10 @@ __device__ __forceinline__ void f32_chunk_store(uint32_t t, uint32_t* stage, flo
   tmem_ld_32x32b_x32(t, v);
   tmem_ld_wait();
   if (SCALED) apply_scales(v, sc, sr);
-  store_chunk_f32<32>(v, stage, out_row0, ld, nvalid, lane);
+  store_chunk_f32<ROWS>(v, stage, out_row0, ld, nvalid, lane);
 }
 
-template <bool SCALED>
+template <bool SCALED, int ROWS = 32>
 __device__ __forceinline__ void f32_chunk_scatter(uint32_t t, uint32_t* stage, float* y32_col0,
                                                   size_t ld, int nvalid, int lane,
                                                   const float* sc, float sr, int my_t,
@@ -737,7 +741,7 @@ __device__ __forceinline__ void f32_chunk_scatter(uint32_t t, uint32_t* stage, f
   tmem_ld_32x32b_x32(t, v);
   tmem_ld_wait();
   if (SCALED) apply_scales(v, sc, sr);
-  scatter_chunk_f32<32>(v, stage, y32_col0, ld, my_t, my_w, nvalid, lane);
+  scatter_chunk_f32<ROWS>(v, stage, y32_col0, ld, my_t, my_w, nvalid, lane);
 }
 
 constexpr int kPairStages = 6;
@@ -1130,7 +1134,691 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA pairs with expert tails
+// The CTA-pair tiles of the kernel above for buckets of 256 to 511 rows per
+// expert (bf16 operands), where an expert's rows rarely fill whole 256-row
+// tiles: buckets of 256 +- a few dozen rows would otherwise need a second,
+// mostly empty tile per column block.
+//
+// Expert tails.  The last r <= 128 rows of an expert that has at least one
+// full 256-row tile are computed inside the k-loop of its last full tile, with
+// swapped operands: the weights staged for that tile are the M = 256 side of a
+// second MMA per K step (each CTA's 128 weight columns, MN-major) and the tail
+// rows its N side, rounded up to N = 32, 64, 96 or 128 (N/2 rows staged by
+// each CTA, K-major, in a third region of the stage).  The tail costs MMA time
+// in proportion to its rows and adds only its own rows to the operand
+// traffic: the weights are not fetched again.  Its accumulator is transposed
+// (TMEM lane = weight column, TMEM column = row) and takes the upper 128
+// columns of the other accumulator buffer: the epilogue drains those columns
+// of every tile first and reports them free on a barrier of their own, so a
+// tile with a tail waits for half of the previous tile's epilogue only; it
+// drains its own tail first in turn.  GEMM 1's epilogue hands the up values
+// (lanes 64-127) to the warps holding the gate values of the same h-columns
+// (lanes 0-63) through shared memory.  An expert of at most 128 rows runs the
+// swapped MMA alone.  GEMM 1 stages, per CTA r, the gate and the up columns of
+// h-columns [64r, 64r + 64) of the tile, so that both MMAs of a K step use
+// the same weight tile (accumulator columns [128r, 128r + 64) gate,
+// [128r + 64, 128r + 128) up).
+//
+// Dynamic tile order.  Tiles of one bucket have different lengths (with or
+// without a tail), and with a fixed round-robin assignment the pairs drift
+// apart until tiles that share a weight tile or a bucket's rows no longer run
+// at the same time and read them from HBM again.  Here the pairs take tiles
+// from a global counter in list order: the leader's producer draws the next
+// index 8 k-blocks before its current tile ends and publishes it 2 k-blocks
+// later to its MMA issuer and epilogue warps and to the other CTA, through a
+// small ring of slots in shared memory.  The tiles running at any moment are
+// then a contiguous window of the list.
+constexpr int kPairRows = 2 * kBM;                     // rows of a full pair tile
+// A stage: the CTA's rows of A (16 KB), its half of the weight tile (16 KB)
+// and up to 64 tail rows (8 KB).
+constexpr int kTailStages = 5;
+constexpr int kTailWOff = kBM * kBK * 2;
+constexpr int kTailTOff = 2 * kBM * kBK * 2;
+constexpr int kTailStageBytes = kTailTOff + 64 * 128;
+constexpr int kTailStagingOff = kTailStages * kTailStageBytes;
+constexpr int kTailStageRows = 16;                     // fp32 epilogue staging rows per warp
+// GEMM 1's tails pass up values between epilogue warps through one padded
+// 32 x 32 tile per (warp group, lane half)
+constexpr int kSwapXchgBytes = 4 * stage_words(32) * 4;
+__host__ __device__ constexpr int tail_smem_bytes(bool swiglu) {
+  return kTailStagingOff + (swiglu ? kSwapXchgBytes : kEpiWarps * stage_words(kTailStageRows) * 4) +
+         1024;
+}
+// N of a swapped MMA over `rows` tail rows (1..128): a multiple of 32, so
+// that each CTA stages a multiple of 16 rows
+__host__ __device__ constexpr int swap_n(int rows) { return (rows + 31) & ~31; }
+
+// Tiles per column block of an expert with cnt > 0 rows: one per 256 rows,
+// except that a last r <= 128 rows after a full tile ride along with it.
+__host__ __device__ constexpr int tail_tiles_per_block(int cnt) {
+  return (cnt > kPairRows && cnt % kPairRows != 0 && cnt % kPairRows <= kBM)
+             ? cnt / kPairRows
+             : (cnt + kPairRows - 1) / kPairRows;
+}
+
+// Rows of tile m (of mt per column block) of a bucket of cnt rows: main =
+// rows of its 256-row MMA (0: none), tail = rows of its swapped MMA (0: none),
+// which start at bucket row m * 256 + (main ? 256 : 0).
+__device__ __forceinline__ void tail_tile_rows(int cnt, int m, int mt, int& main_rows,
+                                               int& tail_rows) {
+  const int left = cnt - m * kPairRows;
+  if (cnt <= kBM) {
+    main_rows = 0;
+    tail_rows = cnt;
+  } else {
+    main_rows = min(kPairRows, left);
+    tail_rows = (m == mt - 1 && left > kPairRows) ? left - kPairRows : 0;
+  }
+}
+
+// tile indices in flight between the leader's producer and the consumers:
+// the leader's MMA issuer and epilogue warps, the other CTA's producer and
+// epilogue warps
+constexpr int kSchedDepth = 4;
+constexpr int kSchedConsumers = 2 + 2 * kEpiWarps;
+
+struct PairTailShared {
+  uint64_t full_bar[kTailStages];
+  uint64_t empty_bar[kTailStages];
+  uint64_t tfull_bar[2];
+  uint64_t tempty_bar[2];             // accumulator buffer drained
+  uint64_t thalf_bar[2];              // its upper 128 columns drained
+  uint64_t drain_bar;
+  uint64_t xchg_full[4];              // GEMM 1 tails: up values written
+  uint64_t xchg_empty[4];             // ... and read
+  uint64_t sched_full[kSchedDepth];   // a tile index published in the slot
+  uint64_t sched_empty[kSchedDepth];  // (leader) every consumer has read it
+  int sched_tile[kSchedDepth];        // -1: no more tiles
+  uint32_t tmem_base;
+  int abort_flag;
+  int never;
+  int tile_prefix[257];
+  int row_off[256];
+  int row_cnt[256];
+};
+
+// tile -> expert e, row tile m, column block n (mt row tiles per block)
+__device__ __forceinline__ void decode_tail_tile(const PairTailShared& sh, int tile, int E,
+                                                 int n_tiles, int& e, int& m, int& n, int& mt) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sh.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int local = tile - sh.tile_prefix[e];
+  mt = (sh.tile_prefix[e + 1] - sh.tile_prefix[e]) / n_tiles;
+  n = local / mt;
+  m = local - n * mt;
+}
+
+template <bool SWIGLU, int FUSE>
+__global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
+    grouped_gemm_pair_tail_kernel(const __grid_constant__ CUtensorMap tmA,
+                                  const __grid_constant__ CUtensorMap tmA16,   // 16-row boxes
+                                  const __grid_constant__ CUtensorMap tmB0,
+                                  const __grid_constant__ CUtensorMap tmB1,
+                                  const int32_t* __restrict__ offsets, int E, int K, int n_out,
+                                  int max_rows, void* __restrict__ out_raw, int32_t* status,
+                                  int* __restrict__ sched,   // [next tile, finished pairs], zero
+                                  const FuseArgs fz) {
+  constexpr int kOutCols = SWIGLU ? 128 : 256;        // output columns per pair tile
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kPairRows, 256, /*b_mn_major=*/true);
+  constexpr int kTmemCols = 512;
+  extern __shared__ uint8_t dsmem_raw[];
+  __shared__ PairTailShared sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int npairs = gridDim.x >> 1;
+  const int n_tiles = (n_out + kOutCols - 1) / kOutCols;
+  const int nkb = K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTailStages; ++s) {
+      mbar_init(&sh.full_bar[s], 1);
+      mbar_init(&sh.empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sh.tfull_bar[a], 1);
+      mbar_init(&sh.tempty_bar[a], 2 * kEpiWarps);   // the epilogue warps of both CTAs
+      mbar_init(&sh.thalf_bar[a], 2 * kEpiWarps);
+    }
+    mbar_init(&sh.drain_bar, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&sh.xchg_full[i], 1);
+      mbar_init(&sh.xchg_empty[i], 1);
+    }
+    for (int i = 0; i < kSchedDepth; ++i) {
+      mbar_init(&sh.sched_full[i], 1);
+      mbar_init(&sh.sched_empty[i], kSchedConsumers);
+    }
+    sh.abort_flag = 0;
+    sh.never = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(&sh.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == 1 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmA16);
+    prefetch_tensormap(&tmB0);
+    if (SWIGLU) prefetch_tensormap(&tmB1);
+  }
+  if (warp == 2) {
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int tiles = 0;
+      if (e < E) {
+        const int o0 = offsets[e], o1 = offsets[e + 1];
+        int cnt = o1 - o0;
+        if (o0 < 0 || cnt < 0 || o1 > max_rows) {
+          report(status, kDevErrBadOffsets);
+          cnt = 0;
+        }
+        if (fz.bucket_rows) cnt = min(cnt, max(0, fz.bucket_rows[e]));
+        sh.row_off[e] = o0;
+        sh.row_cnt[e] = cnt;
+        tiles = cnt > 0 ? tail_tiles_per_block(cnt) * n_tiles : 0;
+      }
+      int incl = tiles;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (e < E) sh.tile_prefix[e] = carry + incl - tiles;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) sh.tile_prefix[E] = carry;
+  }
+  tc_fence_before();
+  cluster_sync();            // both CTAs' barriers initialised, TMEM allocated
+  tc_fence_after();
+
+  const uint32_t tmem_base = sh.tmem_base;
+  const int total_tiles = sh.tile_prefix[E];
+  volatile int* abort_flag = &sh.abort_flag;
+  const uint32_t peer_abort = mapa_shared(&sh.abort_flag, rank ^ 1u);
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    st_shared_cluster_u32(peer_abort, 1u);
+    report(status, kDevErrWaitTimeout);
+  };
+  // the i-th tile of this pair (-1: none left); false if the wait gave up
+  auto sched_take = [&](int i, int& tile) -> bool {
+    const int slot = i % kSchedDepth;
+    if (!mbar_wait_cluster(&sh.sched_full[slot], (i / kSchedDepth) & 1, abort_flag)) return false;
+    tile = *reinterpret_cast<volatile int*>(&sh.sched_tile[slot]);
+    return true;
+  };
+  // one consumer has read slot i (an arrive on the leader's barrier)
+  auto sched_release = [&](int i) {
+    const int slot = i % kSchedDepth;
+    if (leader)
+      mbar_arrive(&sh.sched_empty[slot]);
+    else
+      mbar_arrive_cluster(mapa_shared(&sh.sched_empty[slot], 0));
+  };
+
+  if (warp == 0) {
+    // A rows gathered from the token rows (all 32 lanes issue tile::gather4),
+    // else one thread loads the permuted rows' tiles
+    constexpr bool gather = FUSE == kFuseGather;
+    if (gather || lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      int it = 0;
+      int last_it[kTailStages];
+      for (int s = 0; s < kTailStages; ++s) last_it[s] = -1;
+      bool ok = true;
+      // leader: the next tile is drawn 8 k-blocks before the current one
+      // ends and published 2 k-blocks later, which hides the atomic's latency
+      // and the hand-over to the other CTA behind the current tile
+      const int claim_kb = nkb > 8 ? nkb - 8 : 0;
+      const int publish_kb = claim_kb + 2 < nkb ? claim_kb + 2 : nkb - 1;
+      auto sched_publish = [&](int i, int t) -> bool {
+        const int slot = i % kSchedDepth;
+        if (!mbar_wait_cluster(&sh.sched_empty[slot], ((i / kSchedDepth) & 1) ^ 1, abort_flag))
+          return false;
+        sh.sched_tile[slot] = t;
+        st_shared_cluster_u32(mapa_shared(&sh.sched_tile[slot], 1), static_cast<uint32_t>(t));
+        mbar_arrive(&sh.sched_full[slot]);
+        mbar_arrive_cluster(mapa_shared(&sh.sched_full[slot], 1));
+        return true;
+      };
+      int next = -1, drawn = -1;
+      if (leader && lane == 0) {
+        drawn = atomicAdd(sched, 1);
+        next = drawn < total_tiles ? drawn : -1;
+        ok = sched_publish(0, next);
+      }
+      if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
+      for (int i = 0; ok; ++i) {
+        int tile = -1;
+        if (lane == 0) {
+          if (leader) {
+            tile = next;                       // published during the previous tile
+          } else {
+            ok = sched_take(i, tile);
+            if (ok) sched_release(i);
+          }
+        }
+        if (gather) {
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          tile = __shfl_sync(0xffffffffu, tile, 0);
+        }
+        if (!ok || tile < 0) break;
+        int e, m, n, mt;
+        decode_tail_tile(sh, tile, E, n_tiles, e, m, n, mt);
+        const int cnt = sh.row_cnt[e];
+        int main_rows, tail_rows;
+        tail_tile_rows(cnt, m, mt, main_rows, tail_rows);
+        // rows this CTA stages: 128 of A, N/2 of the tail
+        const int arows = main_rows > 0 ? kBM : 0;
+        const int trows = tail_rows > 0 ? swap_n(tail_rows) / 2 : 0;
+        const int ew = weight_index(fz, e);
+        const int amrow = m * kPairRows + (int)rank * arows;                  // in the bucket
+        const int tmrow = m * kPairRows + (main_rows > 0 ? kPairRows : 0) + (int)rank * trows;
+        const int arow0 = sh.row_off[e] + amrow, trow0 = sh.row_off[e] + tmrow;
+        const int col0 = n * kOutCols;
+        const uint32_t cta_bytes = (uint32_t)(arows + trows) * 128u + kBM * kBK * 2;
+        int aidx[4] = {0, 0, 0, 0}, tidx[4] = {0, 0, 0, 0};
+        if (gather) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int rr = 4 * lane + j;
+            aidx[j] = (rr < arows && amrow + rr < cnt) ? fz.row_src[arow0 + rr] : fz.n_tok;
+            tidx[j] = (rr < trows && tmrow + rr < cnt) ? fz.row_src[trow0 + rr] : fz.n_tok;
+          }
+        }
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kTailStages;
+          const uint32_t ph = (it / kTailStages) & 1;
+          bool good = true;
+          if (lane == 0) good = mbar_wait(&sh.empty_bar[s], ph ^ 1, abort_flag);
+          if (gather) good = __shfl_sync(0xffffffffu, good, 0);
+          if (!good) { ok = false; break; }
+          uint8_t* sa = smem + s * kTailStageBytes;
+          uint8_t* sb = sa + kTailWOff;
+          uint8_t* st = sa + kTailTOff;
+          const uint32_t full_lead = mapa_shared(&sh.full_bar[s], 0);
+          if (leader && lane == 0) mbar_arrive_expect_tx(&sh.full_bar[s], 2 * cta_bytes);
+          if (gather) {
+            __syncwarp();
+            if (4 * lane < arows)
+              tma_gather4_pair(sa + 4 * lane * 128, &tmA, full_lead, kb * kBK, aidx[0], aidx[1],
+                               aidx[2], aidx[3]);
+            if (4 * lane < trows)
+              tma_gather4_pair(st + 4 * lane * 128, &tmA, full_lead, kb * kBK, tidx[0], tidx[1],
+                               tidx[2], tidx[3]);
+          } else {
+            if (arows > 0) tma_load_2d_pair(sa, &tmA, full_lead, kb * kBK, arow0);
+            for (int j = 0; j < trows; j += 16)
+              tma_load_2d_pair(st + j * 128, &tmA16, full_lead, kb * kBK, trow0 + j);
+          }
+          if (lane == 0) {
+            if (SWIGLU) {
+              // gate then up columns of h-columns [col0 + 64 rank, + 64)
+              tma_load_3d_pair(sb, &tmB0, full_lead, col0 + (int)rank * 64, kb * kBK, ew);
+              tma_load_3d_pair(sb + kChunkBytes, &tmB1, full_lead, col0 + (int)rank * 64,
+                               kb * kBK, ew);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 2; ++c)
+                tma_load_3d_pair(sb + c * kChunkBytes, &tmB0, full_lead,
+                                 col0 + (int)rank * 128 + c * 64, kb * kBK, ew);
+            }
+          }
+          last_it[s] = it;
+          if (leader && lane == 0) {
+            if (kb == claim_kb) drawn = atomicAdd(sched, 1);
+            if (kb == publish_kb) {
+              next = drawn < total_tiles ? drawn : -1;
+              if (!sched_publish(i + 1, next)) ok = false;
+            }
+          }
+        }
+        if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+      if (lane == 0) {
+        if (!ok) give_up();
+        if (leader) {
+          // this pair draws no more tiles: the last pair to get here leaves
+          // the counters at zero for the next launch
+          __threadfence();
+          if (atomicAdd(sched + 1, 1) == npairs - 1) {
+            atomicExch(sched, 0);
+            atomicExch(sched + 1, 0);
+          }
+          // both CTAs' copies of every issued phase count on the leader's barriers
+          for (int s = 0; s < kTailStages; ++s)
+            if (last_it[s] >= 0)
+              mbar_wait(&sh.full_bar[s], (last_it[s] / kTailStages) & 1, &sh.never);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (leader CTA)
+      int it = 0;
+      // uses so far of each accumulator buffer: whole (a main MMA) and of its
+      // upper 128 columns (a main MMA, or a tail)
+      int mains0 = 0, mains1 = 0, halves0 = 0, halves1 = 0;
+      bool ok = true;
+      for (int lt = 0; ok; ++lt) {
+        int tile = -1;
+        if (!sched_take(lt, tile)) { ok = false; break; }
+        sched_release(lt);
+        if (tile < 0) break;
+        int e, m, n, mt;
+        decode_tail_tile(sh, tile, E, n_tiles, e, m, n, mt);
+        int main_rows, tail_rows;
+        tail_tile_rows(sh.row_cnt[e], m, mt, main_rows, tail_rows);
+        const int b = lt & 1;
+        // the main accumulator takes buffer b; a tail the upper 128 columns of
+        // the other buffer (of b when the tile has no main MMA): wait until
+        // their previous uses are drained
+        const int x = main_rows > 0 ? b ^ 1 : b;
+        int& mains_b = b ? mains1 : mains0;
+        int& halves_b = b ? halves1 : halves0;
+        int& halves_x = x ? halves1 : halves0;
+        if (main_rows > 0) {
+          if (!mbar_wait(&sh.tempty_bar[b], (mains_b & 1) ^ 1, abort_flag) ||
+              !mbar_wait(&sh.thalf_bar[b], (halves_b & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ++mains_b;
+          ++halves_b;
+        }
+        if (tail_rows > 0) {
+          if (!mbar_wait(&sh.thalf_bar[x], (halves_x & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ++halves_x;
+        }
+        tc_fence_after();
+        const uint32_t d_main = tmem_base + static_cast<uint32_t>(b * 256);
+        const uint32_t d_tail = tmem_base + static_cast<uint32_t>(x * 256 + 128);
+        // swapped: M = 256 weight columns (MN-major), N = the tail rows (K-major)
+        const uint32_t idesc_tail =
+            idesc_bf16_f32(kPairRows, swap_n(tail_rows > 0 ? tail_rows : 1), false, true);
+        auto kloop = [&](auto main_c, auto tail_c) {
+          constexpr bool kMain = decltype(main_c)::value, kTail = decltype(tail_c)::value;
+          static_assert(kMain || kTail, "a tile has a main or a tail MMA");
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % kTailStages;
+            const uint32_t ph = (it / kTailStages) & 1;
+            if (!mbar_wait(&sh.full_bar[s], ph, abort_flag)) { ok = false; return; }
+            tc_fence_after();
+            const uint32_t st_addr = smem_u32(smem + s * kTailStageBytes);
+            // K step: +32 B in the K-major rows (+2 in the descriptor),
+            // +16 K rows = +2 KB in the MN-major weights (+128)
+            const uint64_t dw = smem_desc_sw128(st_addr + kTailWOff, kChunkBytes, 1024);
+            if constexpr (kMain) {
+              const uint64_t da = smem_desc_sw128(st_addr, 16, 1024);
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                umma_bf16_pair(d_main, da + 2 * ks, dw + 128 * ks, kIdesc,
+                               (kb | ks) != 0 ? 1u : 0u);
+            }
+            if constexpr (kTail) {
+              const uint64_t dt = smem_desc_sw128(st_addr + kTailTOff, 16, 1024);
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                umma_bf16_pair(d_tail, dw + 128 * ks, dt + 2 * ks, idesc_tail,
+                               (kb | ks) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair_mc(&sh.empty_bar[s], 0x3);
+          }
+        };
+        using T_ = std::integral_constant<bool, true>;
+        using F_ = std::integral_constant<bool, false>;
+        if (tail_rows == 0)
+          kloop(T_{}, F_{});
+        else if (main_rows == 0)
+          kloop(F_{}, T_{});
+        else
+          kloop(T_{}, T_{});
+        if (!ok) break;
+        umma_commit_pair_mc(&sh.tfull_bar[b], 0x3);
+      }
+      if (!ok) give_up();
+      umma_commit_pair_mc(&sh.drain_bar, 0x1);
+      mbar_wait(&sh.drain_bar, 0, &sh.never);
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2.., both CTAs)
+    const int q = warp & 3;
+    constexpr int kGroups = kEpiWarps / 4;              // warp groups splitting the chunks
+    const int grp = (warp - 2) / 4;
+    int xc = 0;                  // up-value hand-overs so far (GEMM 1 tails)
+    bool xok = true;
+    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kTailStagingOff) +
+                      (warp - 2) * stage_words(kTailStageRows);
+    // this warp is done with accumulator buffer `buf` (whole) / its upper
+    // half: its tensor-memory loads have completed (tcgen05.wait::ld), and the
+    // signal does not wait for the warp's global stores
+    auto release = [&](int buf) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(&sh.tempty_bar[buf], 0));
+    };
+    auto release_half = [&](int buf) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(&sh.thalf_bar[buf], 0));
+    };
+    for (int lt = 0;; ++lt) {
+      int tile = -1;
+      bool good = true;
+      if (lane == 0) good = sched_take(lt, tile);
+      good = __shfl_sync(0xffffffffu, good, 0);
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      // the slot has been read (its value is in every lane's register)
+      if (good && lane == 0)
+        mbar_arrive_cluster_relaxed(mapa_shared(&sh.sched_empty[lt % kSchedDepth], 0));
+      if (!good) {
+        give_up();
+        break;
+      }
+      if (tile < 0) break;
+      int e, m, n, mt;
+      decode_tail_tile(sh, tile, E, n_tiles, e, m, n, mt);
+      int main_rows, tail_rows;
+      tail_tile_rows(sh.row_cnt[e], m, mt, main_rows, tail_rows);
+      const int b = lt & 1;
+      const int x = main_rows > 0 ? b ^ 1 : b;        // buffer of a tail
+      if (!mbar_wait(&sh.tfull_bar[b], (lt >> 1) & 1, abort_flag)) {
+        give_up();
+        break;
+      }
+      tc_fence_after();
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      if (tail_rows > 0) {
+        // swapped tail: TMEM lane = weight column of this CTA, TMEM column j =
+        // bucket row rowb + j (j < tail_rows are real)
+        const int left = tail_rows;
+        const uint32_t tbase = lane_base + static_cast<uint32_t>(x * 256 + 128);
+        const size_t rowb =
+            (size_t)sh.row_off[e] + (size_t)m * kPairRows + (main_rows > 0 ? kPairRows : 0);
+        if constexpr (SWIGLU) {
+          // lanes 0-63: gate, lanes 64-127: up of h-columns col0 + 64 * rank + [0, 64)
+          const int hc = n * kOutCols + 64 * (int)rank + 32 * (q & 1) + lane;
+          const int xi = grp * 2 + (q & 1);            // the gate warp and its up warp
+          uint32_t* xu = reinterpret_cast<uint32_t*>(smem + kTailStagingOff) + xi * stage_words(32);
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_raw);
+#pragma unroll 1
+          for (int c = grp; c * 32 < left; c += kGroups, ++xc) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tbase + c * 32, v);
+            tmem_ld_wait();
+            const uint32_t par = xc & 1;
+            bool gw = true;
+            if (q >= 2) {
+              if (lane == 0) gw = mbar_wait(&sh.xchg_empty[xi], par ^ 1, abort_flag);
+              if (!__shfl_sync(0xffffffffu, gw, 0)) { xok = false; break; }
+#pragma unroll
+              for (int j = 0; j < 32; ++j) xu[lane * 33 + j] = v[j];
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sh.xchg_full[xi]);
+            } else {
+              if (lane == 0) gw = mbar_wait(&sh.xchg_full[xi], par, abort_flag);
+              if (!__shfl_sync(0xffffffffu, gw, 0)) { xok = false; break; }
+              if (hc < n_out) {
+                const int nv = min(32, left - c * 32);
+                __nv_bfloat16* oc = o + (rowb + (size_t)c * 32) * n_out + hc;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  if (j < nv) {
+                    const float g = __uint_as_float(v[j]);
+                    const float u = __uint_as_float(xu[lane * 33 + j]);
+                    oc[(size_t)j * n_out] = __float2bfloat16_rn(silu(g) * u);
+                  }
+                }
+              }
+              __syncwarp();
+              // the up values were read (used by the stores above)
+              if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(&sh.xchg_empty[xi], rank));
+            }
+          }
+          if (!xok) {
+            give_up();
+            break;
+          }
+        } else {
+          // 128 output columns per CTA, one per lane
+          const int oc = n * kOutCols + 128 * (int)rank + 32 * q + lane;
+#pragma unroll 1
+          for (int c = grp; c * 32 < left; c += kGroups) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tbase + c * 32, v);
+            tmem_ld_wait();
+            const int nv = min(32, left - c * 32);
+            const size_t r0 = rowb + (size_t)c * 32;
+            if (FUSE == kFuseScatter) {
+              int my_t = 0;
+              float my_w = 0.f;
+              if (lane < nv) {
+                const int p = fz.row_pair[r0 + lane];
+                my_t = p / fz.k;
+                my_w = fz.topk_w[p];
+              }
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j < nv) {
+                  const int t = __shfl_sync(0xffffffffu, my_t, j);
+                  const float w = __shfl_sync(0xffffffffu, my_w, j);
+                  if (oc < n_out)
+                    atomicAdd(fz.y32 + (size_t)t * n_out + oc, w * __uint_as_float(v[j]));
+                }
+              }
+            } else if (oc < n_out) {
+              float* o = static_cast<float*>(out_raw) + r0 * n_out + oc;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nv) o[(size_t)j * n_out] = __uint_as_float(v[j]);
+            }
+          }
+        }
+        release_half(x);
+      }
+      if (main_rows > 0) {
+        const uint32_t tbase = lane_base + static_cast<uint32_t>(b * 256);
+        const int first = m * kPairRows + (int)rank * kBM + q * 32;   // first row of this warp
+        const int nvalid = clamp_rows(sh.row_cnt[e] - first);
+        const size_t row0 = (size_t)(sh.row_off[e] + first);
+        const int c0 = n * kOutCols;
+        int my_t = 0;
+        float my_w = 0.f;
+        if (FUSE == kFuseScatter && lane < nvalid) {
+          const int p = fz.row_pair[row0 + lane];
+          my_t = p / fz.k;
+          my_w = fz.topk_w[p];
+        }
+        // 32-column chunks [c_lo, c_hi) of the tile's output columns
+        auto chunks = [&](int c_lo, int c_hi) {
+#pragma unroll 1
+          for (int c = c_lo + grp; c < c_hi && c0 + c * 32 < n_out; c += kGroups) {
+            if (SWIGLU) {
+              // h-column chunk c: gate column (c / 2) * 128 + (c % 2) * 32, up 64 further
+              const int gcol = (c >> 1) * 128 + (c & 1) * 32;
+              swiglu_chunk_store<false>(tbase + gcol, tbase + gcol + 64,
+                                        static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out +
+                                            c0 + c * 32,
+                                        n_out, nvalid, lane, nullptr, nullptr, 0.f);
+            } else if (FUSE == kFuseScatter) {
+              f32_chunk_scatter<false, kTailStageRows>(tbase + c * 32, stage,
+                                                       fz.y32 + c0 + c * 32, n_out, nvalid, lane,
+                                                       nullptr, 0.f, my_t, my_w);
+            } else {
+              f32_chunk_store<false, kTailStageRows>(
+                  tbase + c * 32, stage, static_cast<float*>(out_raw) + row0 * n_out + c0 + c * 32,
+                  n_out, nvalid, lane, nullptr, 0.f);
+            }
+          }
+        };
+        // the upper 128 accumulator columns first: a tail of the next tile may
+        // go there as soon as they are drained
+        constexpr int kChunks = SWIGLU ? 4 : 8;
+        chunks(kChunks / 2, kChunks);
+        release_half(b);
+        chunks(0, kChunks / 2);
+        release(b);
+      }
+    }
+  }
+
+  if (*abort_flag) spin_ns(200000);      // let copies still in flight land
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // ---------------------------------------------------------------- host side
+
+// Counters of the CTA-pair kernels' dynamic tile order, [next tile, finished
+// pairs] per launch, zero between launches (the kernel's last pair resets
+// its own).  Each launch takes the next of kSchedPool entries in turn, so
+// launches that run at the same time on different streams use different
+// counters unless kSchedPool of them run at once (a device runs at most 128
+// kernels at a time).
+constexpr int kSchedPool = 256;
+static __device__ int g_pair_sched[kSchedPool][2];
+static std::atomic<unsigned> g_sched_seq{0};
+static std::mutex g_sched_mutex;
+static int* g_sched_base[64] = {nullptr};
+
+// a counter pair for one launch on the current device (the pool's device
+// address is looked up once per device)
+static cudaError_t take_sched_counter(int** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(g_sched_mutex);
+    if (!g_sched_base[dev]) {
+      void* p = nullptr;
+      err = cudaGetSymbolAddress(&p, g_pair_sched);
+      if (err != cudaSuccess) return err;
+      g_sched_base[dev] = static_cast<int*>(p);
+    }
+  }
+  *out = g_sched_base[dev] + 2 * (g_sched_seq.fetch_add(1, std::memory_order_relaxed) % kSchedPool);
+  return cudaSuccess;
+}
 
 template <int BN, bool SWIGLU, int FUSE>
 static cudaError_t launch_gemm_t(int slot, const CUtensorMap& a, const CUtensorMap& a64,
@@ -1199,6 +1887,48 @@ static cudaError_t launch_gemm_pair_t(int slot, const CUtensorMap& a, const CUte
                             row_scale, cs0, cs1, offsets, E, K, n_out, max_rows, out, status, fz);
 }
 
+
+template <bool SWIGLU, int FUSE>
+static cudaError_t launch_gemm_pair_tail_t(int slot, const CUtensorMap& a, const CUtensorMap& a16,
+                                           const CUtensorMap& b0, const CUtensorMap& b1,
+                                           const int32_t* offsets, int E, int K, int n_out,
+                                           int max_rows, void* out, int32_t* status,
+                                           cudaStream_t s, const FuseArgs& fz) {
+  constexpr int kSmem = tail_smem_bytes(SWIGLU);
+  DeviceInfo* di = nullptr;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  int* sched = nullptr;
+  err = take_sched_counter(&sched);
+  if (err != cudaSuccess) return err;
+  auto kern = grouped_gemm_pair_tail_kernel<SWIGLU, FUSE>;
+  if (!di->attr_set[slot]) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (err != cudaSuccess) return err;
+    di->attr_set[slot] = true;
+  }
+  const int n_tiles = (n_out + (SWIGLU ? 127 : 255)) / (SWIGLU ? 128 : 256);
+  const long long pair_rows = (long long)max_rows / (2 * kBM) + (E < max_rows ? E : max_rows);
+  long long pairs = pair_rows * n_tiles;
+  const int max_pairs = di->sms / 2;
+  if (pairs > max_pairs) pairs = max_pairs;
+  if (pairs < 1) pairs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(gemm_threads(SWIGLU), 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, a16, b0, b1, offsets, E, K, n_out, max_rows, out,
+                            status, sched, fz);
+}
+
 // The fusion an instance is compiled for, from the arguments.
 static int fuse_kind(const FuseArgs& fz) {
   return fz.row_src ? kFuseGather : (fz.y32 ? kFuseScatter : kFuseNone);
@@ -1252,6 +1982,28 @@ static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtens
                                                      row_scale, cs0, cs1);
 }
 
+// slot: the plain instance's attribute slot (+16 gathering, +32 scattering)
+template <bool SWIGLU>
+static cudaError_t launch_gemm_pair_tail(int slot, const CUtensorMap& a, const CUtensorMap& a16,
+                                         const CUtensorMap& b0, const CUtensorMap& b1,
+                                         const int32_t* offsets, int E, int K, int n_out,
+                                         int max_rows, void* out, int32_t* status,
+                                         cudaStream_t s, const FuseArgs& fz) {
+  const int kind = fuse_kind(fz);
+  if constexpr (SWIGLU) {
+    if (kind == kFuseGather)
+      return launch_gemm_pair_tail_t<SWIGLU, kFuseGather>(slot + 16, a, a16, b0, b1, offsets, E,
+                                                          K, n_out, max_rows, out, status, s, fz);
+  } else {
+    if (kind == kFuseScatter)
+      return launch_gemm_pair_tail_t<SWIGLU, kFuseScatter>(slot + 32, a, a16, b0, b1, offsets, E,
+                                                           K, n_out, max_rows, out, status, s, fz);
+  }
+  if (kind != kFuseNone) return cudaErrorInvalidValue;
+  return launch_gemm_pair_tail_t<SWIGLU, kFuseNone>(slot, a, a16, b0, b1, offsets, E, K, n_out,
+                                                    max_rows, out, status, s, fz);
+}
+
 template <int BN, bool SWIGLU, int FUSE>
 static cudaError_t launch_gemm_e4m3_t(int slot, const CUtensorMap& a, const CUtensorMap& a64,
                                       const CUtensorMap& b0, const CUtensorMap& b1,
@@ -1273,9 +2025,17 @@ static cudaError_t launch_gemm_e4m3(int slot, const CUtensorMap& a, const CUtens
                                                    s, fz);
 }
 
-// Pair tiles (256 rows) pay off when buckets are large; the buffer's rows
-// per expert bound the average bucket from above.
-static bool use_pair_tiles(int E, int max_rows) { return max_rows >= 512LL * E; }
+// Tile shapes by the buffer's rows per expert, an upper bound on the average
+// bucket: CTA pairs (256-row tiles) from 512; with bf16 operands, CTA pairs
+// that compute an expert's last <= 128 rows inside its last full tile from
+// 256 (buckets of a few hundred rows, which whole tiles fit badly); else
+// single-CTA 128-row tiles.
+enum class Tiles { kSingle, kPairTails, kPair };
+static Tiles gemm_tiles(int E, int max_rows, bool e4m3) {
+  if (max_rows >= 512LL * E) return Tiles::kPair;
+  if (!e4m3 && max_rows >= 256LL * E) return Tiles::kPairTails;
+  return Tiles::kSingle;
+}
 
 // The A operand: the permuted rows [max_rows, K] (128- and 64-row boxes), or,
 // when gathering, the token rows [fz.n_tok, K] (one-row boxes for gather4).
@@ -1303,9 +2063,19 @@ cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, 
                   map_weights(&tg, w_gate, weight_count(fz, E), d, f) &&
                   map_weights(&tu, w_up, weight_count(fz, E), d, f));
   if (*map_failed) return cudaSuccess;
-  if (use_pair_tiles(E, max_rows))
+  const Tiles tiles = gemm_tiles(E, max_rows, false);
+  if (tiles == Tiles::kPair)
     return launch_gemm_pair<true>(7, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s,
                                   fz);
+  if (tiles == Tiles::kPairTails) {
+    // the tails are read in 16-row boxes of the permuted rows (the gathering
+    // form reads token rows by tile::gather4 and needs none)
+    CUtensorMap ta16 = ta;
+    *map_failed = !fz.row_src && !map_rows(&ta16, a_rows, d, max_rows, 16);
+    if (*map_failed) return cudaSuccess;
+    return launch_gemm_pair_tail<true>(14, ta, ta16, tg, tu, offsets, E, d, f, max_rows, h, status,
+                                       s, fz);
+  }
   return launch_gemm<256, true>(0, ta, ta64, tg, tu, offsets, E, d, f, max_rows, h, status, s,
                                 fz);
 }
@@ -1314,13 +2084,18 @@ cudaError_t launch_gate_up(const __nv_bfloat16* a_rows, const int32_t* offsets, 
 cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, int d, int f,
                         int max_rows, const __nv_bfloat16* w_down, float* y_perm,
                         int32_t* status, cudaStream_t s, bool* map_failed, const FuseArgs& fz) {
-  CUtensorMap ta, ta64, td;
+  CUtensorMap ta, ta64, ta16, td;
   *map_failed = !(map_rows(&ta, h, f, max_rows, kBM) && map_rows(&ta64, h, f, max_rows, kBM / 2) &&
+                  map_rows(&ta16, h, f, max_rows, 16) &&
                   map_weights(&td, w_down, weight_count(fz, E), f, d));
   if (*map_failed) return cudaSuccess;
-  if (d % 256 == 0 && use_pair_tiles(E, max_rows))
+  const Tiles tiles = gemm_tiles(E, max_rows, false);
+  if (d % 256 == 0 && tiles == Tiles::kPair)
     return launch_gemm_pair<false>(8, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
                                    s, fz);
+  if (d % 256 == 0 && tiles == Tiles::kPairTails)
+    return launch_gemm_pair_tail<false>(15, ta, ta16, td, td, offsets, E, f, d, max_rows, y_perm,
+                                        status, s, fz);
   if (d % 256 == 0)
     return launch_gemm<256, false>(1, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
                                    s, fz);
@@ -1369,7 +2144,7 @@ cudaError_t launch_gate_up_e4m3(const uint8_t* xq, const float* sx, const int32_
                   map_weights_e4m3(&tg, wq_gate, weight_count(fz, E), f, d) &&
                   map_weights_e4m3(&tu, wq_up, weight_count(fz, E), f, d));
   if (*map_failed) return cudaSuccess;
-  if (use_pair_tiles(E, max_rows)) {
+  if (gemm_tiles(E, max_rows, true) == Tiles::kPair) {
     CUtensorMap tgh, tuh;
     *map_failed = !(map_weights_e4m3(&tgh, wq_gate, weight_count(fz, E), f, d, 64) &&
                     map_weights_e4m3(&tuh, wq_up, weight_count(fz, E), f, d, 64));
@@ -1390,7 +2165,7 @@ cudaError_t launch_down_e4m3(const uint8_t* hq, const float* sh_rows, const int3
                   map_rows_e4m3(&ta64, hq, f, max_rows, kBM / 2) &&
                   map_weights_e4m3(&td, wq_down, weight_count(fz, E), d, f));
   if (*map_failed) return cudaSuccess;
-  if (d % 256 == 0 && use_pair_tiles(E, max_rows))
+  if (d % 256 == 0 && gemm_tiles(E, max_rows, true) == Tiles::kPair)
     return launch_gemm_pair<false, true>(10, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm,
                                          status, s, fz, &td, &td, sh_rows, s_down, nullptr);
   if (d % 256 == 0)

@@ -81,6 +81,9 @@ EP = [
     small("ep_fine", T=512, d=256, E=16, k=4, f=256, cf=1.25, seed=31),
     small("ep_drops", T=333, d=384, E=6, k=3, f=128, cf=0.5, seed=32),
     small("ep_pair", T=2048, d=256, E=4, k=2, f=256, cf=1.0, seed=33),
+    # slots of C = 320 rows, of which only the received counts are real: the
+    # expert-tail pair tiles with per-bucket row counts
+    small("ep_tails", T=1024, d=256, E=8, k=2, f=256, cf=1.25, seed=34),
 ]
 
 

@@ -48,6 +48,8 @@ PADDED = [
     small("ragged_T", T=333, d=384, E=6, k=3, f=128, cf=0.5, seed=15),
     small("pair_tiles_drops", T=3000, d=512, E=4, k=3, f=384, cf=0.8, seed=20),
     small("dropless", T=200, d=128, E=4, k=2, f=256, cf=0.0, seed=21),
+    # buckets of C = 320 rows: a 64-row tail inside every expert's full tile
+    small("tails", T=1024, d=256, E=16, k=4, f=256, cf=1.25, seed=25),
 ]
 
 

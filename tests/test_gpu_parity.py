@@ -39,6 +39,7 @@ SMALL = [
     # buffers of >= 512 rows per expert select the CTA-pair GEMM tiles
     small("pair_tiles", T=2048, d=256, E=4, k=2, f=256, cf=0.0, seed=19),
     small("pair_tiles_drops", T=3000, d=512, E=4, k=3, f=384, cf=0.8, seed=20),
+    # 256 buffer rows per expert: CTA pairs with the expert tails inside full tiles
     small("medium_buckets", T=1024, d=256, E=16, k=4, f=384, cf=1.25, seed=22),
     # widths that are multiples of 64 but not of 128: ragged 64-column tails
     # in the router's K, the permuted rows, every GEMM tile shape and the combine
@@ -214,8 +215,10 @@ def test_permute_matches_oracle(T, d, E, k, cf):
 MLP_CASES = [
     # (d, f, bucket sizes, pair): ragged tails, empty buckets, one-row buckets,
     # exact tile multiples, several row tiles; pair=True gives the buffer >= 512
-    # rows per expert, which selects the CTA-pair tiles (256 rows); smaller
-    # buffers select the single-CTA 128-row tiles
+    # rows per expert, which selects the CTA-pair tiles (256 rows, a half tile
+    # at an expert's tail), "mid" 256-511 the CTA-pair tiles that compute an
+    # expert's last <= 128 rows inside its last full tile; smaller buffers
+    # select the single-CTA 128-row tiles
     (256, 384, [300, 0, 1, 129, 128, 257], False),
     (128, 256, [5, 140, 0, 0, 64, 128], False),
     (384, 128, [1, 1, 1, 400], False),
@@ -239,13 +242,20 @@ MLP_CASES = [
     (192, 320, [300, 0, 1, 129, 128, 257], False),
     (320, 192, [3000, 2999, 1, 2900], True),
     (64, 64, [70, 0, 129], False),
+    # swapped tail tiles of every width (N = 32, 64, 96, 128: tails of 1-32,
+    # 33-64, 65-96, 97-128 rows, alone or after full 256-row tiles), tails of
+    # more than 128 rows (a full pair tile), 64-column N tails of h (f = 320)
+    (256, 320, [257, 289, 320, 353, 1, 97, 128, 129, 200, 0, 511, 384], "mid"),
+    (512, 256, [33, 64, 65, 96, 300, 416, 480, 32, 31], "mid"),
+    (256, 448, [260, 272, 288, 304], "mid"),
 ]
 
 
 def mlp_buffer_rows(N, E, pair):
     """Rows of the permuted buffer for a bucket layout: pair=True gives >= 512
-    per expert (CTA-pair tiles), "mid" 256-511 and False fewer (single-CTA
-    tiles)."""
+    per expert (CTA-pair tiles), "mid" 256-511 (bf16: CTA pairs with the
+    expert tails inside full tiles; e4m3: single-CTA tiles) and False fewer
+    (single-CTA tiles)."""
     if pair == "mid":
         rows = max(N + 37, 256 * E + 5)
         assert rows < 512 * E

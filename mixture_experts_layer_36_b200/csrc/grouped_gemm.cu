@@ -1119,9 +1119,11 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
                                   cs0 + c0 + c * 32, sr);
         }
       }
+      // the warp's tensor-memory loads have completed; the signal does not
+      // wait for its global stores
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(&sh.tempty_bar[a], 0));
+      if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(&sh.tempty_bar[a], 0));
     }
   }
 

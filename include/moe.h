@@ -243,6 +243,24 @@ int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, con
                 const int32_t* slot, const int32_t* offsets, int64_t T, int64_t d, int64_t k,
                 void* y, void* stream);
 
+/* moe_combine on expert-output rows held in bf16 (y_rows bf16 [>= offsets[E],
+ * d]): the same sum, each row value widened exactly to fp32.  For expert
+ * parallelism, where the rows come back from the ranks that ran the experts
+ * (the combine all-to-all of "Expert Parallelism & All-to-All"
+ * (neelmishra.github.io), section "All-to-all: the distributed transpose")
+ * and bf16 rows halve the bytes that cross the links.  Arguments, layout and
+ * errors as moe_combine. */
+int moe_combine_bf16rows(const void* y_rows, const void* x, const int32_t* topk_idx,
+                         const float* topk_w, const int32_t* slot, const int32_t* offsets,
+                         int64_t T, int64_t d, int64_t k, void* y, void* stream);
+
+/* dst bf16 [rows, d] = src f32 [rows, d] rounded to nearest (ties to even):
+ * expert-output rows made ready for the bf16 return exchange above.  d a
+ * multiple of 64 (MOE_ERR_UNSUPPORTED otherwise), rows < 2^31, both pointers
+ * device memory, 16-byte aligned (MOE_ERR_INVALID_ARG otherwise); rows = 0 is
+ * a no-op.  Caller owns both buffers. */
+int moe_rows_to_bf16(const float* src, void* dst, int64_t rows, int64_t d, void* stream);
+
 /* ---- Padded-capacity layout (an optional variant of moe_permute) ----
  * The static [E, C, d] buffer the neelmishra page contrasts with ragged
  * buckets ("Expert Parallelism & All-to-All", section "Why fixed-size buffers

@@ -30,7 +30,7 @@ EXPORTED = ["moe_status_string", "moe_version", "moe_selftest_bounded_wait", "mo
             "moe_max_rows",
             "moe_route_workspace_size", "moe_permute_workspace_size", "moe_workspace_size", "moe_workspace_field_offset",
             "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_gate_up", "moe_expert_down", "moe_expert_mlp",
-            "moe_combine", "moe_layer_forward", "moe_quantize_weights_fp8",
+            "moe_combine", "moe_combine_bf16rows", "moe_rows_to_bf16", "moe_layer_forward", "moe_quantize_weights_fp8",
             "moe_quantize_rows_fp8", "moe_permute_fp8", "moe_expert_gate_up_fp8", "moe_expert_down_fp8",
             "moe_workspace_size_fp8", "moe_layer_forward_fp8", "moe_padded_rows",
             "moe_permute_padded", "moe_permute_fused", "moe_expert_gate_up_gather",
@@ -69,6 +69,8 @@ def _load():
         "moe_expert_down": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p]),
         "moe_expert_mlp": (ctypes.c_int, [p, p, i64, i64, i64, i64, p, p, p, p, p, p, p]),
         "moe_combine": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, p, p]),
+        "moe_combine_bf16rows": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, p, p]),
+        "moe_rows_to_bf16": (ctypes.c_int, [p, p, i64, i64, p]),
         "moe_layer_forward": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl, p, p,
                                              sz, p]),
         "moe_layer_forward_ex": (ctypes.c_int, [p, p, p, p, p, p, i64, i64, i64, i64, i64, dbl, p,
@@ -322,6 +324,35 @@ def moe_combine(y_perm, x, topk_idx, topk_w, slot, offsets, y=None, stream=None)
         _ptr(y_perm), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(slot), _ptr(offsets), T, d, k,
         _ptr(y), _stream(stream)))
     return y
+
+
+def moe_combine_bf16rows(y_rows, x, topk_idx, topk_w, slot, offsets, y=None, stream=None):
+    """moe_combine on bf16 expert-output rows (the expert-parallel return)."""
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    _want(y_rows, "y_rows", torch.bfloat16)
+    _want(x, "x", torch.bfloat16)
+    _want(topk_idx, "topk_idx", torch.int32, (T, k))
+    _want(topk_w, "topk_w", torch.float32, (T, k))
+    _want(slot, "slot", torch.int32, (T, k))
+    _want(offsets, "offsets", torch.int32)
+    y = torch.empty_like(x) if y is None else y
+    _want(y, "y", torch.bfloat16, (T, d))
+    _check("moe_combine_bf16rows", _lib.moe_combine_bf16rows(
+        _ptr(y_rows), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(slot), _ptr(offsets), T, d, k,
+        _ptr(y), _stream(stream)))
+    return y
+
+
+def moe_rows_to_bf16(src, dst=None, stream=None):
+    """bf16 copy (round to nearest even) of fp32 rows src [rows, d]."""
+    rows, d = src.shape
+    _want(src, "src", torch.float32)
+    dst = torch.empty(rows, d, dtype=torch.bfloat16, device=src.device) if dst is None else dst
+    _want(dst, "dst", torch.bfloat16, (rows, d))
+    _check("moe_rows_to_bf16", _lib.moe_rows_to_bf16(_ptr(src), _ptr(dst), rows, d,
+                                                     _stream(stream)))
+    return dst
 
 
 def moe_layer_forward(x, w_router, bias, w_gate, w_up, w_down, k, cf, y=None, ws=None,

@@ -30,6 +30,12 @@ cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t s);
+cudaError_t launch_combine_bf16rows(const __nv_bfloat16* y_rows, const __nv_bfloat16* x,
+                                    const int32_t* topk_idx, const float* topk_w,
+                                    const int32_t* slot, const int32_t* offsets, int T, int d,
+                                    int k, __nv_bfloat16* y, cudaStream_t s);
+cudaError_t launch_rows_to_bf16(const float* src, __nv_bfloat16* dst, long long n,
+                                cudaStream_t s);
 cudaError_t launch_permute_rows(const uint8_t* x, int row_bytes, const float* x_scale,
                                 const int32_t* topk_idx, int T, int E, int k, int64_t C,
                                 int32_t* counts, int32_t* offsets, int32_t* slot,
@@ -342,6 +348,32 @@ int moe_combine(const float* y_perm, const void* x, const int32_t* topk_idx, con
                                     topk_w, slot,
                                     offsets, (int)T, (int)d, (int)k,
                                     static_cast<__nv_bfloat16*>(y), as_stream(stream)));
+}
+
+int moe_combine_bf16rows(const void* y_rows, const void* x, const int32_t* topk_idx,
+                         const float* topk_w, const int32_t* slot, const int32_t* offsets,
+                         int64_t T, int64_t d, int64_t k, void* y, void* stream) {
+  if (T < 0 || k < 1 || k > kMaxK || T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  int st = check_width(d);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!y_rows || !x || !topk_idx || !topk_w || !slot || !offsets || !y)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_rows) || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_combine_bf16rows(
+      static_cast<const __nv_bfloat16*>(y_rows), static_cast<const __nv_bfloat16*>(x), topk_idx,
+      topk_w, slot, offsets, (int)T, (int)d, (int)k, static_cast<__nv_bfloat16*>(y),
+      as_stream(stream)));
+}
+
+int moe_rows_to_bf16(const float* src, void* dst, int64_t rows, int64_t d, void* stream) {
+  if (rows < 0 || rows >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  int st = check_width(d);
+  if (st != MOE_OK) return st;
+  if (rows == 0) return MOE_OK;
+  if (!src || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_rows_to_bf16(src, static_cast<__nv_bfloat16*>(dst), rows * d,
+                                              as_stream(stream)));
 }
 
 int64_t moe_padded_rows(int64_t T, int64_t E, int64_t k, double cf) {

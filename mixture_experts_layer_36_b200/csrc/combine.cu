@@ -9,8 +9,9 @@
 //
 // One warp per (token, 512-column segment): lanes 0..k-1 resolve the k source
 // rows and weights, broadcast them, then the warp streams its segment of the
-// fp32 rows in 16-byte vectors, accumulating in fp32 in top-k order and
-// rounding once to bf16.
+// expert-output rows (fp32, or bf16 where an expert-parallel exchange sent
+// them back at half the bytes) in 16-byte vectors, accumulating in fp32 in
+// top-k order and rounding once to bf16.
 #include "common.cuh"
 
 namespace moe {
@@ -18,10 +19,28 @@ namespace moe {
 constexpr int kCombThreads = 256;
 constexpr int kSegVec = 64;        // 16-byte output vectors per warp work unit (512 elements)
 
+// values 8v .. 8v+7 of an expert-output row, as fp32
+__device__ __forceinline__ void load8(const float* row, int v, float (&o)[8]) {
+  const float4* src = reinterpret_cast<const float4*>(row);
+  const float4 a = __ldg(src + 2 * v), b = __ldg(src + 2 * v + 1);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* row, int v, float (&o)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(row) + v);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {      // bf16 -> fp32 is exact: the bits in the upper half
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
 // One warp per (token, 512-column segment), so that a handful of tokens still
 // spreads over many SMs.
+template <typename RowT>
 __global__ void __launch_bounds__(kCombThreads)
-    combine_kernel(const float* __restrict__ y_perm, const __nv_bfloat16* __restrict__ x,
+    combine_kernel(const RowT* __restrict__ y_perm, const __nv_bfloat16* __restrict__ x,
                    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ slot, const int32_t* __restrict__ offsets, int T,
                    int d, int k, int nseg, __nv_bfloat16* __restrict__ y) {
@@ -65,21 +84,15 @@ __global__ void __launch_bounds__(kCombThreads)
   for (int j = 0; j < 8; ++j) {
     if (j >= k) break;
     if (rows[j] < 0) continue;
-    const float4* src = reinterpret_cast<const float4*>(y_perm + (size_t)rows[j] * d);
+    const RowT* src = y_perm + (size_t)rows[j] * d;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int v = v_begin + lane + u * 32;
       if (v >= v_end) continue;
-      const float4 a = __ldg(src + 2 * v);
-      const float4 b = __ldg(src + 2 * v + 1);
-      acc[u][0] = fmaf(w[j], a.x, acc[u][0]);
-      acc[u][1] = fmaf(w[j], a.y, acc[u][1]);
-      acc[u][2] = fmaf(w[j], a.z, acc[u][2]);
-      acc[u][3] = fmaf(w[j], a.w, acc[u][3]);
-      acc[u][4] = fmaf(w[j], b.x, acc[u][4]);
-      acc[u][5] = fmaf(w[j], b.y, acc[u][5]);
-      acc[u][6] = fmaf(w[j], b.z, acc[u][6]);
-      acc[u][7] = fmaf(w[j], b.w, acc[u][7]);
+      float a[8];
+      load8(src, v, a);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[u][q] = fmaf(w[j], a[q], acc[u][q]);
     }
   }
 #pragma unroll
@@ -95,15 +108,55 @@ __global__ void __launch_bounds__(kCombThreads)
   }
 }
 
+template <typename RowT>
+static cudaError_t launch_combine_t(const RowT* y_perm, const __nv_bfloat16* x,
+                                   const int32_t* topk_idx, const float* topk_w,
+                                   const int32_t* slot, const int32_t* offsets, int T, int d,
+                                   int k, __nv_bfloat16* y, cudaStream_t s) {
+  const int nseg = (d / 8 + kSegVec - 1) / kSegVec;
+  const long long units = (long long)T * nseg;
+  const int per_cta = kCombThreads / 32;
+  combine_kernel<RowT><<<(unsigned)((units + per_cta - 1) / per_cta), kCombThreads, 0, s>>>(
+      y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, nseg, y);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const float* y_perm, const __nv_bfloat16* x,
                            const int32_t* topk_idx, const float* topk_w, const int32_t* slot,
                            const int32_t* offsets, int T, int d, int k, __nv_bfloat16* y,
                            cudaStream_t s) {
-  const int nseg = (d / 8 + kSegVec - 1) / kSegVec;
-  const long long units = (long long)T * nseg;
-  const int per_cta = kCombThreads / 32;
-  combine_kernel<<<(unsigned)((units + per_cta - 1) / per_cta), kCombThreads, 0, s>>>(
-      y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, nseg, y);
+  return launch_combine_t(y_perm, x, topk_idx, topk_w, slot, offsets, T, d, k, y, s);
+}
+
+cudaError_t launch_combine_bf16rows(const __nv_bfloat16* y_rows, const __nv_bfloat16* x,
+                                    const int32_t* topk_idx, const float* topk_w,
+                                    const int32_t* slot, const int32_t* offsets, int T, int d,
+                                    int k, __nv_bfloat16* y, cudaStream_t s) {
+  return launch_combine_t(y_rows, x, topk_idx, topk_w, slot, offsets, T, d, k, y, s);
+}
+
+// fp32 rows -> bf16 (round to nearest even), 8 values per thread step: the
+// expert outputs an expert-parallel rank sends back at half the bytes.
+__global__ void __launch_bounds__(256)
+    rows_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                        long long nvec) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < nvec;
+       v += (long long)gridDim.x * blockDim.x) {
+    const float4 a = __ldg(s4 + 2 * v), b = __ldg(s4 + 2 * v + 1);
+    d4[v] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                       pack_bf16x2(b.z, b.w));
+  }
+}
+
+cudaError_t launch_rows_to_bf16(const float* src, __nv_bfloat16* dst, long long n,
+                                cudaStream_t s) {
+  const long long nvec = n / 8;
+  long long blocks = (nvec + 255) / 256;
+  if (blocks > 4096) blocks = 4096;      // a grid-stride loop covers the rest
+  if (blocks < 1) blocks = 1;
+  rows_to_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(src, dst, nvec);
   return cudaGetLastError();
 }
 

@@ -32,10 +32,14 @@ calls), which keeps the exchange logic testable with CPU ranks.
 Exchange volume.  The neelmishra page's dispatch volume per rank is
 T*k*d*2*(P-1)/P bytes (bf16 rows, the share of each rank's rows that leaves
 it).  The padded exchange here sends E*C rows per rank instead of T*k, a
-factor E*C/(T*k) (about cf, or E/k when dropless, C = T); and the rows come
-back as fp32 (the expert outputs are rounded to bf16 only once, in the
-combine), twice the bytes of the dispatch.  ``exchange_log`` records, per
-exchange of the last forward, the bytes this rank sent to other ranks.
+factor E*C/(T*k) (about cf, or E/k when dropless, C = T).  The rows come
+back as fp32 by default (the expert outputs are rounded to bf16 only once,
+in the combine), twice the bytes of the dispatch; with ``return_bf16`` they
+are rounded to bf16 before the return exchange (moe_rows_to_bf16) and
+combined from bf16 (moe_combine_bf16rows): the same bytes as the dispatch,
+for one more rounding of each expert output (at most 2^-9 of its magnitude
+per term of the weighted sum).  ``exchange_log`` records, per exchange of the
+last forward, the bytes this rank sent to other ranks.
 """
 import torch
 import torch.distributed as dist
@@ -66,16 +70,24 @@ class CudaOps:
     def combine(self, y_rows, x, topk_idx, topk_w, slot, offsets):
         return self.b.moe_combine(y_rows, x, topk_idx, topk_w, slot, offsets)
 
+    def rows_to_bf16(self, y_rows):
+        return self.b.moe_rows_to_bf16(y_rows)
+
+    def combine_bf16rows(self, y_rows, x, topk_idx, topk_w, slot, offsets):
+        return self.b.moe_combine_bf16rows(y_rows, x, topk_idx, topk_w, slot, offsets)
+
 
 class ExpertParallelMoE:
     """One rank's part of an expert-parallel MoE layer.
 
     w_router f32 [d, E] and bias f32 [E] (or None) are replicated; w_gate /
     w_up [E/P, d, f] and w_down [E/P, f, d] are this rank's experts
-    rank*E/P .. (rank+1)*E/P - 1.
+    rank*E/P .. (rank+1)*E/P - 1.  return_bf16: send the expert outputs back
+    in bf16 (half the return bytes) instead of fp32.
     """
 
-    def __init__(self, w_router, bias, w_gate, w_up, w_down, k, cf, group=None, ops=None):
+    def __init__(self, w_router, bias, w_gate, w_up, w_down, k, cf, group=None, ops=None,
+                 return_bf16=False):
         self.group = group
         self.P = dist.get_world_size(group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
@@ -89,10 +101,12 @@ class ExpertParallelMoE:
         self.w_gate, self.w_up, self.w_down = w_gate, w_up, w_down
         self.k, self.cf = k, cf
         self.ops = ops if ops is not None else CudaOps()
+        self.return_bf16 = return_bf16
         self.exchange_log = []
 
-    # bytes per element on the wire: int32 counts, bf16 rows out, fp32 rows back
-    WIRE_BYTES = {"counts": 4, "dispatch": 2, "combine": 4}
+    # bytes per element on the wire: int32 counts, bf16 rows out, fp32 (or
+    # bf16) rows back
+    WIRE_BYTES = {"counts": 4, "dispatch": 2, "combine": 4, "combine_bf16": 2}
 
     def _all_to_all(self, out, inp, name):
         # each rank keeps 1/P of its buffer (its own slot) and sends the rest
@@ -122,6 +136,10 @@ class ExpertParallelMoE:
         recv_offsets = torch.arange(B + 1, dtype=torch.int32, device=x.device) * C
         y_recv = self.ops.mlp_buckets(x_recv, recv_offsets, recv_counts, self.w_gate, self.w_up,
                                       self.w_down)
+        if self.return_bf16:
+            y_send = self.ops.rows_to_bf16(y_recv)
+            y_pad = self._all_to_all(torch.empty_like(y_send), y_send, "combine_bf16")
+            return self.ops.combine_bf16rows(y_pad, x, topk_idx, topk_w, slot, offsets)
         y_pad = self._all_to_all(torch.empty_like(y_recv), y_recv, "combine")
         return self.ops.combine(y_pad, x, topk_idx, topk_w, slot, offsets)
 

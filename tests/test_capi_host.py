@@ -122,6 +122,20 @@ def test_validation_codes_without_launch():
                                 None, s) == UNSUPPORTED
     # combine / layer
     assert L.moe_combine(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10, 128, 9, FAKE, s) == INVALID
+    assert L.moe_combine_bf16rows(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10, 128, 9, FAKE, s) \
+        == INVALID
+    assert L.moe_combine_bf16rows(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 10, 96, 2, FAKE, s) \
+        == UNSUPPORTED
+    assert L.moe_combine_bf16rows(None, FAKE, FAKE, FAKE, FAKE, FAKE, 10, 128, 2, FAKE, s) \
+        == INVALID
+    assert L.moe_combine_bf16rows(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 128, 2, FAKE, s) == OK
+    # fp32 -> bf16 rows
+    assert L.moe_rows_to_bf16(FAKE, FAKE, 10, 100, s) == UNSUPPORTED
+    assert L.moe_rows_to_bf16(FAKE, FAKE, -1, 128, s) == INVALID
+    assert L.moe_rows_to_bf16(FAKE, FAKE, 1 << 31, 128, s) == INVALID
+    assert L.moe_rows_to_bf16(None, FAKE, 10, 128, s) == INVALID
+    assert L.moe_rows_to_bf16(FAKE, ctypes.c_void_p((1 << 20) + 8), 10, 128, s) == INVALID
+    assert L.moe_rows_to_bf16(FAKE, FAKE, 0, 128, s) == OK
     ws_need = moe.moe_workspace_size(64, 128, 8, 2, 256, 1.25)
     assert L.moe_layer_forward(FAKE, FAKE, None, FAKE, FAKE, FAKE, 64, 128, 8, 2, 256, 1.25, FAKE,
                                FAKE, ws_need - 1, s) == WORKSPACE

@@ -68,14 +68,21 @@ class OracleOps:
             _, o = self.o.swiglu_rows(xb[lo:lo + n], self._bits(w_gate[e]), self._bits(w_up[e]),
                                       self._bits(w_down[e]))
             y[lo:lo + n] = torch.from_numpy(o)
+        self.rows_max = float(y.abs().max()) if y.numel() else 0.0
         return y
 
     def combine(self, y_rows, x, topk_idx, topk_w, slot, offsets):
         return torch.from_numpy(self.o.combine(y_rows.numpy(), self._bits(x), topk_idx.numpy(),
                                                topk_w.numpy(), slot.numpy(), offsets.numpy()))
 
+    def rows_to_bf16(self, y_rows):
+        # each value rounded to bf16 by the oracle's rounding (ties to even)
+        return torch.from_numpy(np.vectorize(self.o.round_bf16)(y_rows.numpy()))
 
-def _worker(rank, world, port, case, out):
+    combine_bf16rows = combine
+
+
+def _worker(rank, world, port, case, out, return_bf16=False):
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -93,8 +100,12 @@ def _worker(rank, world, port, case, out):
                                  ep.shard_experts(w["w_gate"], rank, world),
                                  ep.shard_experts(w["w_up"], rank, world),
                                  ep.shard_experts(w["w_down"], rank, world), k, cf,
-                                 ops=OracleOps(oracle))
+                                 ops=OracleOps(oracle), return_bf16=return_bf16)
     y = layer(x).numpy()
+    # the largest expert output any rank computed (a rank combines rows of all)
+    rows_max = torch.tensor([layer.ops.rows_max], dtype=torch.float64)
+    dist.all_reduce(rows_max, op=dist.ReduceOp.MAX)
+    rows_max = float(rows_max.item())
     log = dict(layer.exchange_log)
     xb = OracleOps._bits(x)
     ops = OracleOps(oracle)
@@ -106,7 +117,7 @@ def _worker(rank, world, port, case, out):
     dist.barrier()
     dist.destroy_process_group()
     out.put((rank, float(np.max(np.abs(y - ref["y"]))), float(np.max(np.abs(ref["y"]))),
-             int(ref["n_dropped"]), log, oracle.capacity(T, E, k, cf)))
+             int(ref["n_dropped"]), log, oracle.capacity(T, E, k, cf), rows_max))
 
 
 CASES = [
@@ -135,7 +146,7 @@ def test_expert_parallel_matches_single_process(world, case):
     T, d, E, k, f, cf, _ = case
     # dispatch volume per rank on the neelmishra page: T*k*d*2*(P-1)/P bytes
     page = T * k * d * 2 * (world - 1) / world
-    for rank, err, scale, n_drop, log, C in res:
+    for rank, err, scale, n_drop, log, C, _ in res:
         assert err <= 1e-12 * max(scale, 1.0), (rank, err)
         dropped += n_drop
         # the padded exchange moves E*C rows where the formula counts T*k:
@@ -146,6 +157,31 @@ def test_expert_parallel_matches_single_process(world, case):
         assert log["counts"] == E * 4 * (world - 1) // world
     if case[5] > 0:
         assert dropped > 0                    # the capacity limit was exercised
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("case", CASES[:2], ids=["dropless", "drops"])
+def test_expert_parallel_bf16_return(case):
+    """The return exchange in bf16: half the bytes of the fp32 return (the
+    same as the dispatch), and the layer off the fp64 one by at most the
+    rounding of each expert output (2^-9 of the largest, the gate weights
+    summing to at most 1)."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, case, q, True))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=280) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=30)
+        assert p.exitcode == 0
+    for rank, err, scale, n_drop, log, C, rows_max in res:
+        assert err <= 2.0 ** -9 * rows_max * (1 + 1e-9) + 1e-12 * max(scale, 1.0), (rank, err)
+        assert "combine" not in log
+        assert log["combine_bf16"] == log["dispatch"]
 
 
 def test_layer_rejects_expert_counts_that_do_not_split():

@@ -104,3 +104,28 @@ def test_expert_parallel_one_rank_matches_oracle(cfg, one_rank_group):
     dropped = (ref["slot"] < 0).all(axis=1)
     if dropped.any():
         np.testing.assert_array_equal(bits(y)[dropped], bits(cpu["x"])[dropped])
+
+
+@pytest.mark.parametrize("cfg", [EP[0], EP[-1]], ids=[EP[0].name, EP[-1].name])
+def test_expert_parallel_bf16_return_matches_oracle(cfg, one_rank_group):
+    """The return exchange in bf16: the layer against the oracle's combine of
+    its expert outputs rounded to bf16, and half the return bytes."""
+    inp, cpu = cuda_inputs(cfg)
+    layer = ep.ExpertParallelMoE(inp["w_router"], inp["bias"], inp["w_gate"], inp["w_up"],
+                                 inp["w_down"], cfg.k, cfg.cf, return_bf16=True)
+    y = layer(inp["x"])
+    logits, _, _ = moe.moe_route(inp["x"], inp["w_router"], inp["bias"], cfg.k)
+    torch.cuda.synchronize()
+    assert dict(layer.exchange_log)["combine_bf16"] == 0       # one rank sends nothing away
+    bias = None if cpu["bias"] is None else cpu["bias"].numpy()
+    xb = bits(cpu["x"])
+    ref = oracle.moe_forward(xb, cpu["w_router"].numpy(), bias, bits(cpu["w_gate"]),
+                             bits(cpu["w_up"]), bits(cpu["w_down"]), cfg.k, cfg.cf,
+                             decision_logits=logits.cpu().numpy())
+    C = oracle.capacity(cfg.T, cfg.E, cfg.k, cfg.cf)
+    _, offsets, slot, row_src, _ = oracle.permute(ref["topk_idx"], cfg.E, C)
+    _, rows = oracle.expert_mlp(oracle.dispatch(xb, row_src), offsets, bits(cpu["w_gate"]),
+                                bits(cpu["w_up"]), bits(cpu["w_down"]))
+    rows_b = np.vectorize(oracle.round_bf16)(rows)
+    y_ref = oracle.combine(rows_b, xb, ref["topk_idx"], ref["topk_w"], slot, offsets)
+    assert_bf16_close(f64(y), y_ref, "y")

@@ -315,6 +315,49 @@ def test_combine_matches_oracle(T, d, E, k, cf):
         np.testing.assert_array_equal(bits(y)[dropped], bits(x)[dropped])
 
 
+@pytest.mark.parametrize("T,d,E,k,cf", [(64, 128, 8, 2, 1.25), (500, 256, 16, 4, 0.4)])
+def test_combine_bf16rows_matches_oracle(T, d, E, k, cf):
+    """The combine on bf16 expert-output rows (the expert-parallel return in
+    bf16) against the oracle's combine on the same bf16 values."""
+    g = torch.Generator().manual_seed(T + d + 1)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    logits = torch.randn(T, E, generator=g).numpy()
+    idx, w64 = oracle.topk(logits, k)
+    w32 = w64.astype(np.float32)
+    C = oracle.capacity(T, E, k, cf)
+    counts, offsets, slot, row_src, n_drop = oracle.permute(idx, E, C)
+    rows = max(int(offsets[E]), 1)
+    y_rows = torch.randn(rows, d, generator=g).to(torch.bfloat16)
+    y = moe.moe_combine_bf16rows(y_rows.cuda(), x.cuda(), torch.from_numpy(idx).cuda(),
+                                 torch.from_numpy(w32).cuda(), torch.from_numpy(slot).cuda(),
+                                 torch.from_numpy(offsets).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.combine(f64(y_rows), bits(x), idx, w32.astype(np.float64), slot, offsets)
+    assert_bf16_close(f64(y), ref, "y")
+    dropped = (slot < 0).all(axis=1)
+    if dropped.any():
+        np.testing.assert_array_equal(bits(y)[dropped], bits(x)[dropped])
+
+
+def test_rows_to_bf16_rounds_like_the_oracle():
+    """fp32 -> bf16, bit for bit the oracle's rounding (nearest, ties to
+    even), on random values of several magnitudes and on exact ties."""
+    g = torch.Generator().manual_seed(77)
+    rows, d = 37, 192
+    v = torch.randn(rows, d, generator=g) * torch.exp2(torch.randint(-30, 30, (rows, d),
+                                                                     generator=g).float())
+    u = v.view(torch.int32)
+    # every fourth value halfway between two bf16 values (low 16 bits 0x8000)
+    tie = (u & ~0xFFFF) | 0x8000
+    u = torch.where(torch.arange(rows * d).view(rows, d) % 4 == 0, tie, u)
+    v = u.view(torch.float32)
+    got = moe.moe_rows_to_bf16(v.cuda())
+    torch.cuda.synchronize()
+    ref = np.vectorize(oracle.round_bf16)(v.numpy().astype(np.float64))
+    want = (ref.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    np.testing.assert_array_equal(bits(got), want)
+
+
 # ----------------------------------------------------------------------------- whole layer
 
 def _ws(ws, name, cfg):

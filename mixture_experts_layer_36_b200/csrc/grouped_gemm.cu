@@ -1706,24 +1706,7 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
             tmem_ld_wait();
             const int nv = min(32, left - c * 32);
             const size_t r0 = rowb + (size_t)c * 32;
-            if (FUSE == kFuseScatter) {
-              int my_t = 0;
-              float my_w = 0.f;
-              if (lane < nv) {
-                const int p = fz.row_pair[r0 + lane];
-                my_t = p / fz.k;
-                my_w = fz.topk_w[p];
-              }
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                if (j < nv) {
-                  const int t = __shfl_sync(0xffffffffu, my_t, j);
-                  const float w = __shfl_sync(0xffffffffu, my_w, j);
-                  if (oc < n_out)
-                    atomicAdd(fz.y32 + (size_t)t * n_out + oc, w * __uint_as_float(v[j]));
-                }
-              }
-            } else if (oc < n_out) {
+            if (oc < n_out) {
               float* o = static_cast<float*>(out_raw) + r0 * n_out + oc;
 #pragma unroll
               for (int j = 0; j < 32; ++j)
@@ -1739,13 +1722,6 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
         const int nvalid = clamp_rows(sh.row_cnt[e] - first);
         const size_t row0 = (size_t)(sh.row_off[e] + first);
         const int c0 = n * kOutCols;
-        int my_t = 0;
-        float my_w = 0.f;
-        if (FUSE == kFuseScatter && lane < nvalid) {
-          const int p = fz.row_pair[row0 + lane];
-          my_t = p / fz.k;
-          my_w = fz.topk_w[p];
-        }
         // 32-column chunks [c_lo, c_hi) of the tile's output columns
         auto chunks = [&](int c_lo, int c_hi) {
 #pragma unroll 1
@@ -1757,10 +1733,6 @@ __global__ void __launch_bounds__(gemm_threads(SWIGLU), 1)
                                         static_cast<__nv_bfloat16*>(out_raw) + row0 * n_out +
                                             c0 + c * 32,
                                         n_out, nvalid, lane, nullptr, nullptr, 0.f);
-            } else if (FUSE == kFuseScatter) {
-              f32_chunk_scatter<false, kTailStageRows>(tbase + c * 32, stage,
-                                                       fz.y32 + c0 + c * 32, n_out, nvalid, lane,
-                                                       nullptr, 0.f, my_t, my_w);
             } else {
               f32_chunk_store<false, kTailStageRows>(
                   tbase + c * 32, stage, static_cast<float*>(out_raw) + row0 * n_out + c0 + c * 32,
@@ -1984,7 +1956,7 @@ static cudaError_t launch_gemm_pair(int slot, const CUtensorMap& a, const CUtens
                                                      row_scale, cs0, cs1);
 }
 
-// slot: the plain instance's attribute slot (+16 gathering, +32 scattering)
+// slot: the plain instance's attribute slot (+16 gathering)
 template <bool SWIGLU>
 static cudaError_t launch_gemm_pair_tail(int slot, const CUtensorMap& a, const CUtensorMap& a16,
                                          const CUtensorMap& b0, const CUtensorMap& b1,
@@ -1996,12 +1968,8 @@ static cudaError_t launch_gemm_pair_tail(int slot, const CUtensorMap& a, const C
     if (kind == kFuseGather)
       return launch_gemm_pair_tail_t<SWIGLU, kFuseGather>(slot + 16, a, a16, b0, b1, offsets, E,
                                                           K, n_out, max_rows, out, status, s, fz);
-  } else {
-    if (kind == kFuseScatter)
-      return launch_gemm_pair_tail_t<SWIGLU, kFuseScatter>(slot + 32, a, a16, b0, b1, offsets, E,
-                                                           K, n_out, max_rows, out, status, s, fz);
   }
-  if (kind != kFuseNone) return cudaErrorInvalidValue;
+  if (kind != kFuseNone) return cudaErrorInvalidValue;   // no scattering form
   return launch_gemm_pair_tail_t<SWIGLU, kFuseNone>(slot, a, a16, b0, b1, offsets, E, K, n_out,
                                                     max_rows, out, status, s, fz);
 }
@@ -2095,7 +2063,10 @@ cudaError_t launch_down(const __nv_bfloat16* h, const int32_t* offsets, int E, i
   if (d % 256 == 0 && tiles == Tiles::kPair)
     return launch_gemm_pair<false>(8, ta, ta64, td, td, offsets, E, f, d, max_rows, y_perm, status,
                                    s, fz);
-  if (d % 256 == 0 && tiles == Tiles::kPairTails)
+  // (the weighted scatter keeps the single-CTA tiles: the tails' transposed
+  // accumulators can only add one value per lane and row, four times the
+  // atomic instructions of the staged four-wide adds)
+  if (d % 256 == 0 && tiles == Tiles::kPairTails && !fz.y32)
     return launch_gemm_pair_tail<false>(15, ta, ta16, td, td, offsets, E, f, d, max_rows, y_perm,
                                         status, s, fz);
   if (d % 256 == 0)

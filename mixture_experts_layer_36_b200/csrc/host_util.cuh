@@ -124,7 +124,7 @@ inline cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 bloc
 
 // attr_set slots: 0-2 grouped GEMM (1 CTA), 3-6 router GEMM, 7-8 grouped GEMM (CTA pair),
 // 9-10 CTA-pair GEMM on e4m3 operands, 11-13 grouped GEMM on e4m3 operands,
-// 14-15 CTA-pair GEMM with expert tails
+// 14-15 CTA-pair GEMM with expert tails (its gathering instance 30)
 // (+16: the gathering instance of a grouped GEMM slot's kernel, +32: the
 // scattering one); 19-22 router GEMM with the top-k epilogue (the router
 // kernels have no gathering instance, so 3-6 + 16 is free for them)

@@ -70,8 +70,9 @@ SMALL = [
     small("pair_tiles", T=2048, d=256, E=4, k=2, f=256, cf=0.0, seed=19),
     small("pair_tiles_drops", T=3000, d=512, E=4, k=3, f=384, cf=0.8, seed=20),
     small("down_d384", T=700, d=384, E=4, k=2, f=256, cf=0.0, seed=23),
-    # 256 buffer rows per expert: both GEMMs on CTA pairs with the expert tails
-    # inside full tiles (gathered rows, the weighted scatter of the tails)
+    # 256 buffer rows per expert: the gate/up GEMM on CTA pairs with the
+    # expert tails inside full tiles (also gathering its rows); the
+    # scattering down GEMM keeps single-CTA tiles there
     small("tails", T=1024, d=256, E=16, k=4, f=256, cf=1.25, seed=25),
 ]
 IDS = [c.name for c in SMALL]

@@ -38,7 +38,12 @@ def test_bounded_wait_times_out_and_reports():
 
 @pytest.mark.parametrize("cfg", [configs.TINY,
                                  small("graph_pairs", T=2048, d=256, E=4, k=2, f=256, cf=0.0,
-                                       seed=23)], ids=["tiny", "pair_tiles"])
+                                       seed=23),
+                                 # 256 buffer rows per expert: the expert-tail pair tiles,
+                                 # whose tile counter must be back at zero for every replay
+                                 small("graph_tails", T=1024, d=256, E=16, k=4, f=256,
+                                       cf=1.25, seed=25)],
+                         ids=["tiny", "pair_tiles", "expert_tails"])
 def test_layer_forward_replays_in_cuda_graph(cfg):
     inp, _ = cuda_inputs(cfg)
     x = inp["x"].clone()
